@@ -1,0 +1,390 @@
+"""Benchmark of the MoE layer forward (one JSON line on stdout, rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one moe_forward (route -> dispatch -> expert GEMMs -> combine, plus
+the Switch loss) over one batch of synthetic tokens of the named workload
+(default: the Mixtral-shaped layer, N=4096 tokens, d_model=4096, E=8, k=2,
+SwiGLU d_ff=14336, bf16).  Under torchrun every rank runs its own batch on
+its own GPU (data-parallel tokens, no collective on the data path: weak
+scaling); the timed region is bracketed by a barrier and a device
+synchronisation, timed with CUDA events and reduced with MAX over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (single thread) on a bounded
+sample of the same workload instead; only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/sec (bf16, 1 B200); expert-GEMM TFLOPS as % of bf16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+# tokens of the workload the CPU oracle handles per reference step (about 1-3 s each)
+REF_TOKENS_PER_STEP = {"tiny_fp32": 64, "gpt2_moe": 32, "mixtral": 1, "deepseek_v3": 1, "qwen3_skew": 8}
+KERNELS_PER_STEP = 7  # router, scan, scatter, gather, GEMM1, GEMM2, combine
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="mixtral")
+    p.add_argument("--impl", default="native", choices=["native", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), int(
+        os.environ.get("WORLD_SIZE", "1"))
+
+
+def weights_bytes(wl) -> int:
+    es = 4 if wl.dtype == "f32" else 2
+    return wl.E * wl.mats * wl.d_model * wl.d_ff * es
+
+
+def traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        table = json.load(f)
+    ent = table.get(f"{kernel}:{workload}")
+    if not ent:
+        return None
+    src = os.path.join(ROOT, ent["source"])
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return ent["bytes_per_launch"] if h == ent["source_sha256_16"] else None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+class OracleSample:
+    """The fp64 oracle (single thread) on a bounded sample of the workload's tokens.
+
+    Expert weights are drawn on the host on demand (same recipe as the GPU
+    run) and kept in a small LRU cache; only the oracle's own calls --
+    routing, the per-token expert FFNs and the weighted sum -- are timed.
+    """
+
+    def __init__(self, wl, cache_bytes: int = 6 << 30):
+        import numpy as np
+        import oracle as O
+        import workloads as W
+        self.np, self.O, self.W, self.wl = np, O, W, wl
+        self.x = W.make_x(wl)
+        r = W.make_router(wl)
+        self.Wg = r["W_g"].float().numpy().astype(np.float64)
+        self.b = None if r["b_e"] is None else r["b_e"].numpy().astype(np.float64)
+        self.L = O.lib()
+        self.cache = {}
+        self.cache_bytes = cache_bytes
+
+    def _expert(self, e):
+        if e in self.cache:
+            self.cache[e] = self.cache.pop(e)  # most recent last
+            return self.cache[e]
+        ex = self.W.make_expert(self.wl, e, "cpu")
+        arrs = {k: (None if v is None else v.float().numpy().astype(self.np.float64)) for k, v in ex.items()}
+        size = sum(a.nbytes for a in arrs.values() if a is not None)
+        while self.cache and sum(sum(a.nbytes for a in v.values() if a is not None)
+                                 for v in self.cache.values()) + size > self.cache_bytes:
+            self.cache.pop(next(iter(self.cache)))
+        self.cache[e] = arrs
+        return arrs
+
+    def run(self, tokens):
+        """Oracle forward of the given token indices; returns seconds spent in the oracle."""
+        np, O, wl = self.np, self.O, self.wl
+        x = self.x[tokens].float().numpy().astype(np.float64)
+        t0 = time.perf_counter()
+        rt = O.route(x, self.Wg, wl.k, wl.router, wl.norm_topk, wl.routed_scaling, b_sel=self.b, L=self.L)
+        spent = time.perf_counter() - t0
+        for s in range(len(tokens)):
+            y = np.zeros(wl.d_model)
+            for j in range(wl.k):
+                ew = self._expert(int(rt["ids"][s, j]))
+                t0 = time.perf_counter()
+                o = O.expert_ffn(x[s], ew["W1"], ew["W2"], wl.act, ew["b1"], ew["W3"], ew["b2"], L=self.L)
+                y += rt["w"][s, j] * o
+                spent += time.perf_counter() - t0
+        return spent
+
+
+def cpu_baseline(wl, tokens: int):
+    """Oracle tokens/s on the first `tokens` tokens of the workload (one host core)."""
+    t = OracleSample(wl).run(list(range(tokens)))
+    return tokens / t, t
+
+
+def run_reference(args, wl):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    per = min(REF_TOKENS_PER_STEP.get(wl.name, 4), wl.N)
+    sampler = OracleSample(wl)
+    nxt = 0
+
+    def take():
+        nonlocal nxt
+        toks = [(nxt + i) % wl.N for i in range(per)]
+        nxt += per
+        return toks
+
+    for _ in range(args.warmup):
+        sampler.run(take())
+    total_t = 0.0
+    for _ in range(args.steps):
+        total_t += sampler.run(take())
+    value = per * args.steps / total_t
+    sample = (f"first {per} tokens of the {wl.name} workload per step (routing + per-token expert FFNs, "
+              f"fp64, single thread); value = tokens/s over {args.steps} steps")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": describe(wl),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def describe(wl):
+    import workloads as W
+    d = W.describe(wl)
+    d["parallelism"] = "data-parallel tokens, one batch per GPU"
+    return d
+
+
+def run_native(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    import mixture_experts_layer_53_b200 as M
+    import workloads as W
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    M.library()
+    cfg = M.make_config(wl.N, wl.d_model, wl.d_ff, wl.E, wl.k, wl.router, wl.norm_topk, wl.routed_scaling,
+                        wl.act, wl.dtype)
+    inp = W.make_inputs(wl.scaled(seed=wl.seed + 100 * rank) if rank else wl, dev)
+    ws = M.workspace(cfg, dev)
+    out = M.forward_outputs(cfg, dev)
+    b_e = inp["b_e"]
+    stream = torch.cuda.current_stream()
+    big_inputs = weights_bytes(wl) > 2 * L2_BYTES
+    flush = None if big_inputs else torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(events=None):
+        M.moe_forward(cfg, inp["x"], inp["W_g"], inp["W1"], inp["W2"], W3=inp["W3"], b1=inp["b1"], b2=inp["b2"],
+                      b_e=b_e, gamma=wl.gamma, ws=ws, out=out, stage_events=events)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert int(out["status"][0]) == 0, f"device status {int(out['status'][0])}"
+
+    stage_ev = [M.StageEvents() for _ in range(args.steps)]
+    start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    with ClockSampler(local_rank) as clocks:
+        t_all0 = torch.cuda.Event(enable_timing=True)
+        t_all1 = torch.cuda.Event(enable_timing=True)
+        t_all0.record(stream)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.fill_(i & 0xFF)
+            start[i].record(stream)
+            step(stage_ev[i])
+            end[i].record(stream)
+        t_all1.record(stream)
+        barrier()
+    if flush is None:
+        local_ms = t_all0.elapsed_time(t_all1)
+    else:
+        local_ms = sum(start[i].elapsed_time(end[i]) for i in range(args.steps))
+    stages = {k: 0.0 for k in M.STAGE_NAMES}
+    for ev in stage_ev:
+        for k, v in ev.elapsed_ms().items():
+            stages[k] += v / args.steps
+    t = torch.tensor([local_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+
+    # end to end through the public call with host buffers: H2D of x, the
+    # forward, D2H of y and of the loss, every step
+    x_host = inp["x"].cpu().pin_memory()
+    y_host = torch.empty_like(out["y"], device="cpu").pin_memory()
+    aux_host = torch.empty(1, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        M.moe_forward(cfg, x_dev, inp["W_g"], inp["W1"], inp["W2"], W3=inp["W3"], b1=inp["b1"], b2=inp["b2"],
+                      b_e=b_e, gamma=wl.gamma, ws=ws, out=out)
+        y_host.copy_(out["y"], non_blocking=True)
+        aux_host.copy_(out["aux"], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        if flush is not None:
+            flush.fill_(i & 0xFF)
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        tokens = wl.N * args.steps * world
+        value = tokens / (total_ms / 1000.0)
+        gemm1_flops = 2 * (2 if wl.act == "swiglu" else 1) * wl.d_model * wl.d_ff * wl.N * wl.k
+        gemm1_s = stages["gemm1"] / 1000.0
+        ffn_s = (stages["gemm1"] + stages["gemm2"]) / 1000.0
+        bf16_peak = peaks["bf16_tflops"]
+        achieved = gemm1_flops / gemm1_s / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": dict(describe(wl), l2=("inputs larger than L2 (expert weights %.2f GB)" % (weights_bytes(wl) / 1e9))
+                           if big_inputs else "L2 flushed between steps (256 MiB write), per-step events"),
+            "roofline": {"kernel": "ffn_gemm_kernel<SwiGLU> (GEMM1)" if wl.act == "swiglu" else "ffn_gemm_kernel<GELU> (GEMM1)",
+                         "bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
+                         "frac": achieved / bf16_peak, "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "traffic": traffic_for("gemm1", wl.name), "flops_per_launch": gemm1_flops},
+            "expert_ffn": {"tflops": wl.expert_flops / ffn_s / 1e12,
+                           "frac_of_measured_peak": wl.expert_flops / ffn_s / 1e12 / bf16_peak,
+                           "frac_of_datasheet_2250": wl.expert_flops / ffn_s / 1e12 / 2250.0},
+            "stages_ms": stages,
+            "e2e": {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s",
+                    "h2d_bytes_per_step": inp["x"].numel() * inp["x"].element_size(),
+                    "d2h_bytes_per_step": out["y"].numel() * out["y"].element_size() + 4},
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "clocks": clocks.summary(),
+        }
+        if not args.no_cpu_baseline and world == 1:
+            per = min(REF_TOKENS_PER_STEP.get(wl.name, 4) * 16, wl.N)
+            v, dt = cpu_baseline(wl, per)
+            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                    "sample": f"first {per} tokens of the workload, routing + per-token expert "
+                                              f"FFNs in fp64 on one host core ({dt:.1f} s)"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    import workloads as W
+    wl = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_native(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,219 @@
+/*
+ * moe.h -- C ABI of libmoe.so, the forward pass of a dropless
+ * Mixture-of-Experts layer on one NVIDIA B200 (sm_100a).
+ *
+ * Symbols follow the course module "Mixture of Experts: routing, sorted
+ * dispatch, Switch aux loss, aux-free bias" (sec. 2 symbol table): N tokens,
+ * E experts, k experts per token, d_model, d_ff, router W_g, selection bias
+ * b_e.  Its sec. 4 interface (topk_ids, dispatch, combine,
+ * load_balance_loss, MoE.route / forward / update_bias) maps onto the entry
+ * points below.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.  Every tensor pointer is DEVICE memory owned by the caller.  The
+ *   library allocates nothing, frees nothing and never synchronises the
+ *   host; all work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *   default stream).  Scratch comes from the caller's workspace `ws` of
+ *   `ws_bytes` bytes, at least moe_workspace_size(cfg) and 256-byte aligned.
+ * Layouts.  Row-major, contiguous:
+ *   x         [N, d_model]            dtype
+ *   W_g       [E, d_model]            dtype      (z_n = W_g x_n)
+ *   W1, W3    [E, d_ff, d_model]      dtype      (row f of W1[e]: hidden unit f)
+ *   W2        [E, d_model, d_ff]      dtype      (row c of W2[e]: output c)
+ *   b1        [E, d_ff], b2 [E, d_model]  dtype  (optional)
+ *   b_e       [E]                     float32
+ *   topk_ids  [N, k] int32, topk_w [N, k] float32, probs [N, E] float32
+ *   x_sorted, y_sorted [N*k, d_model] dtype
+ *   perm, inv_perm [N*k] int32; offsets [E+1] int32; counts [E] int32
+ *   Weights are stored output-feature-major (the nn.Linear convention), so
+ *   both GEMM operands are contiguous along the reduction dimension.
+ * dtype.  MOE_F32 (all fp32) or MOE_BF16 (x, weights, biases, outputs bf16;
+ *   router, softmax, gates and every accumulation in fp32).
+ * Errors.  Arguments are validated before anything is enqueued; a bad
+ *   argument returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED /
+ *   MOE_ERR_WORKSPACE and launches nothing.  A CUDA launch error returns
+ *   MOE_ERR_CUDA (moe_last_error() gives the CUDA message).  Errors found on
+ *   the device (an expert id outside [0, E), a device wait that ran out) are
+ *   written to the caller's optional `dev_status` int32 word: the first
+ *   error code is kept (the word must be 0 before the call; moe_forward
+ *   clears it itself).  The library never traps.
+ * Limits.  1 <= k <= min(E, 16); E <= 256; d_model and d_ff multiples of 8;
+ *   N*k < 2^31; every pointer 16-byte aligned.
+ * Threading.  No global mutable state besides a per-device attribute cache;
+ *   calls on different streams may run concurrently with separate
+ *   workspaces.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,
+    MOE_ERR_UNSUPPORTED = 2,
+    MOE_ERR_CUDA = 3,
+    MOE_ERR_WORKSPACE = 4,
+    MOE_ERR_TIMEOUT = 5,
+    MOE_ERR_BAD_EXPERT_ID = 6
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Router table of the course module (sec. 2.1). */
+typedef enum {
+    MOE_ROUTER_SOFTMAX_TOPK = 0, /* top k of p = softmax(z); w = p, renormalised if norm_topk */
+    MOE_ROUTER_TOPK_SOFTMAX = 1, /* top k of z; w = softmax over the chosen logits */
+    MOE_ROUTER_SIGMOID = 2       /* top k of sigmoid(z) + b_e; w = sigmoid(z), renormalised if norm_topk */
+} moe_router;
+
+typedef enum {
+    MOE_ACT_GELU = 0,  /* h = gelu_erf(W1 x + b1); y = W2 h + b2     ("nano-moe" MLP) */
+    MOE_ACT_SWIGLU = 1 /* h = silu(W1 x) * (W3 x); y = W2 h (+ b2)   (gated MLP, act="silu") */
+} moe_act;
+
+typedef struct {
+    int64_t N;            /* tokens (every leading axis flattened) */
+    int32_t d_model;
+    int32_t d_ff;         /* hidden width of one expert */
+    int32_t E;            /* routed experts */
+    int32_t k;            /* experts per token */
+    int32_t router;       /* moe_router */
+    int32_t norm_topk;    /* 1: renormalise the chosen weights to sum to 1 */
+    float routed_scaling; /* every weight is multiplied by it (1.0 = off) */
+    int32_t act;          /* moe_act */
+    int32_t dtype;        /* moe_dtype */
+} moe_config;
+
+/* Stage boundaries recorded by moe_forward when stage_events is given. */
+#define MOE_STAGE_ROUTE 0    /* router GEMM + scores + top-k + gates */
+#define MOE_STAGE_DISPATCH 1 /* counts/offsets/loss/bias rule, scatter, row gather */
+#define MOE_STAGE_GEMM1 2    /* x_sorted -> h (first expert GEMM + activation) */
+#define MOE_STAGE_GEMM2 3    /* h -> y_sorted (second expert GEMM + bias) */
+#define MOE_STAGE_COMBINE 4  /* weighted sum back in token order */
+#define MOE_NUM_STAGES 5
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char *moe_status_string(moe_status s);
+
+/* Last CUDA error message seen by a failing call on this host thread. */
+MOE_API const char *moe_last_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+MOE_API int32_t moe_version(void);
+
+/*
+ * Bytes of workspace that every entry point below accepts for `cfg` (the
+ * largest need, that of moe_forward): per-chunk histograms and partial
+ * probability sums, offsets, the GEMM tile table, perm / inv_perm, x_sorted,
+ * the hidden activations h [N*k, d_ff] and y_sorted.  Returns 0 for an
+ * invalid cfg.
+ */
+MOE_API size_t moe_workspace_size(const moe_config *cfg);
+
+/*
+ * Router: course module sec. 2 (z_n = W_g x_n, p_n = softmax(z_n)) and the
+ * sec. 2.1 router table, "ties go to the lowest id"; the sec. 4 topk_ids and
+ * MoE.route.  For each token writes the k chosen expert ids, largest
+ * selection score first (ties: lowest id), and their weights (times
+ * routed_scaling).  b_e (sigmoid router only, may be NULL) enters the
+ * selection score only, never the weights (sec. 2.5).  probs [N, E] (may be
+ * NULL) receives softmax(z_n) for every router.  Needs no workspace.
+ */
+MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const void *W_g,
+                     const float *b_e, int32_t *topk_ids, float *topk_w,
+                     float *probs, moe_stream_t stream);
+
+/*
+ * Sorted dispatch: course module sec. 2.2 and the sec. 4 dispatch.
+ * Assignments a = n*k + j are stably sorted by expert id: perm[i] is the
+ * assignment at sorted position i, inv_perm[perm[i]] = i,
+ * x_sorted[i] = x[perm[i] / k], counts[e] = assignments to e,
+ * offsets[e] = start of expert e's slice (offsets[0] = 0, offsets[E] = N*k).
+ * perm, x and x_sorted may be NULL (then that output is skipped).  An
+ * expert id outside [0, E) sets MOE_ERR_BAD_EXPERT_ID in dev_status; the
+ * outputs are then unspecified.
+ */
+MOE_API moe_status moe_dispatch(const moe_config *cfg, const void *x,
+                        const int32_t *topk_ids, void *x_sorted, int32_t *perm,
+                        int32_t *inv_perm, int32_t *offsets, int32_t *counts,
+                        int32_t *dev_status, void *ws, size_t ws_bytes,
+                        moe_stream_t stream);
+
+/*
+ * Expert FFNs over the ragged slices: course module sec. 2.2 ("each expert
+ * runs once on its slice"), experts as in moe_act.  Rows
+ * offsets[e] .. offsets[e+1]-1 of x_sorted go through expert e and land in
+ * the same rows of y_sorted.  b1 (GELU only), W3 (SwiGLU only) and b2 may be
+ * NULL where the activation does not use them.  offsets is read on the
+ * device (no host synchronisation).
+ */
+MOE_API moe_status moe_expert_ffn(const moe_config *cfg, const void *x_sorted,
+                          const int32_t *offsets, const void *W1,
+                          const void *b1, const void *W3, const void *W2,
+                          const void *b2, void *y_sorted, int32_t *dev_status,
+                          void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Combine: course module sec. 2.2 and the sec. 4 combine:
+ * y_n = sum_{j<k} topk_w[n, j] * y_sorted[inv_perm[n*k + j]], summed in slot
+ * order with fp32 accumulation.  Needs no workspace.
+ */
+MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_sorted,
+                       const float *topk_w, const int32_t *inv_perm, void *y,
+                       moe_stream_t stream);
+
+/*
+ * Switch load-balance loss: course module sec. 2.3 and the sec. 4
+ * load_balance_loss:  L = E * sum_e f_e P_e with f_e = (assignments to e)/N
+ * and P_e = mean_n probs[n, e]; written as float to the device scalar
+ * aux_out (reduced in fp64).  counts_out [E] (may be NULL) receives the
+ * assignment counts.  If gamma > 0 and b_e_inout is given, also applies one
+ * step of the sec. 2.5 sign rule b_e += gamma * sign(N*k/E - count_e)
+ * (MoE.update_bias).
+ */
+MOE_API moe_status moe_aux_loss(const moe_config *cfg, const float *probs,
+                        const int32_t *topk_ids, float *aux_out,
+                        int32_t *counts_out, float gamma, float *b_e_inout,
+                        int32_t *dev_status, void *ws, size_t ws_bytes,
+                        moe_stream_t stream);
+
+/*
+ * The whole layer forward (course module sec. 4 MoE.forward, no shared
+ * expert): route -> dispatch -> expert FFNs -> combine, plus the Switch loss
+ * (aux_out, may be NULL) and the assignment counts (counts, may be NULL; the
+ * sec. 4 expert_load).  If gamma > 0 and b_e_inout is given (sigmoid
+ * router), b_e is used for this forward's selection and then moved by one
+ * sign-rule step (sec. 2.5), after the selection.  topk_ids / topk_w (may be
+ * NULL) receive the routing.  dev_status (may be NULL) is cleared at the
+ * start.  stage_events (may be NULL) is an array of MOE_NUM_STAGES + 1
+ * cudaEvent_t handles recorded on `stream` at the stage boundaries
+ * (MOE_STAGE_*), for timing.  Enqueues only: no host synchronisation.
+ */
+MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const void *W_g,
+                       float *b_e_inout, float gamma, const void *W1,
+                       const void *b1, const void *W3, const void *W2,
+                       const void *b2, void *y, int32_t *topk_ids,
+                       float *topk_w, int32_t *counts, float *aux_out,
+                       int32_t *dev_status, void *ws, size_t ws_bytes,
+                       void *const *stage_events, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

@@ -1,0 +1,267 @@
+"""Dropless Mixture-of-Experts layer forward on one B200 -- Python binding.
+
+A thin ctypes layer over ``libmoe.so`` (built from ``csrc/`` for sm_100a):
+it marshals torch tensors to device pointers, allocates outputs with torch
+and passes the current CUDA stream.  Every step of the layer runs in the
+library's CUDA kernels; there is no other implementation behind these
+functions.  If the library is missing, every call raises.
+
+The functions carry the names of the C entry points in ``include/moe.h``:
+``moe_route``, ``moe_dispatch``, ``moe_expert_ffn``, ``moe_combine``,
+``moe_aux_loss``, ``moe_forward`` and ``moe_workspace_size``.  Symbols follow
+the course module "Mixture of Experts: routing, sorted dispatch, Switch aux
+loss, aux-free bias" (sec. 2): N, E, k, d_model, d_ff, W_g, b_e.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional, Sequence
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe.so")
+
+ROUTERS = {"softmax_topk": 0, "topk_softmax": 1, "sigmoid": 2}
+ACTS = {"gelu": 0, "swiglu": 1}
+DTYPES = {"f32": 0, "bf16": 1}
+TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_CUDA",
+          4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_BAD_EXPERT_ID"}
+NUM_STAGES = 5
+STAGE_NAMES = ("route", "dispatch", "gemm1", "gemm2", "combine")
+EXPORTS = ("moe_status_string", "moe_last_error", "moe_version", "moe_workspace_size", "moe_route",
+           "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_aux_loss", "moe_forward")
+
+
+class MoeConfig(ctypes.Structure):
+    """Mirror of ``moe_config`` in include/moe.h."""
+    _fields_ = [("N", ctypes.c_int64), ("d_model", ctypes.c_int32), ("d_ff", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("router", ctypes.c_int32),
+                ("norm_topk", ctypes.c_int32), ("routed_scaling", ctypes.c_float),
+                ("act", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == 0 else torch.bfloat16
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        msg = f"{where}: {STATUS.get(status, status)}"
+        if detail:
+            msg += f" ({detail})"
+        super().__init__(msg)
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libmoe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"{p} is missing: build it with `python -m mixture_experts_layer_53_b200.build`")
+    lib = ctypes.CDLL(p)
+    vp, cfgp, i32p, f32p = ctypes.c_void_p, ctypes.POINTER(MoeConfig), ctypes.c_void_p, ctypes.c_void_p
+    st, sz = ctypes.c_int, ctypes.c_size_t
+    lib.moe_status_string.argtypes = [st]
+    lib.moe_status_string.restype = ctypes.c_char_p
+    lib.moe_last_error.argtypes = []
+    lib.moe_last_error.restype = ctypes.c_char_p
+    lib.moe_version.argtypes = []
+    lib.moe_version.restype = ctypes.c_int32
+    lib.moe_workspace_size.argtypes = [cfgp]
+    lib.moe_workspace_size.restype = sz
+    lib.moe_route.argtypes = [cfgp, vp, vp, f32p, i32p, f32p, f32p, vp]
+    lib.moe_route.restype = st
+    lib.moe_dispatch.argtypes = [cfgp, vp, i32p, vp, i32p, i32p, i32p, i32p, i32p, vp, sz, vp]
+    lib.moe_dispatch.restype = st
+    lib.moe_expert_ffn.argtypes = [cfgp, vp, i32p, vp, vp, vp, vp, vp, vp, i32p, vp, sz, vp]
+    lib.moe_expert_ffn.restype = st
+    lib.moe_combine.argtypes = [cfgp, vp, f32p, i32p, vp, vp]
+    lib.moe_combine.restype = st
+    lib.moe_aux_loss.argtypes = [cfgp, f32p, i32p, f32p, i32p, ctypes.c_float, f32p, i32p, vp, sz, vp]
+    lib.moe_aux_loss.restype = st
+    lib.moe_forward.argtypes = [cfgp, vp, vp, f32p, ctypes.c_float, vp, vp, vp, vp, vp, vp, i32p, f32p, i32p,
+                                f32p, i32p, vp, sz, ctypes.c_void_p, vp]
+    lib.moe_forward.restype = st
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def make_config(N: int, d_model: int, d_ff: int, E: int, k: int, router: str = "softmax_topk",
+                norm_topk: bool = True, routed_scaling: float = 1.0, act: str = "gelu",
+                dtype: str = "bf16") -> MoeConfig:
+    return MoeConfig(int(N), int(d_model), int(d_ff), int(E), int(k), ROUTERS[router], int(bool(norm_topk)),
+                     float(routed_scaling), ACTS[act], DTYPES[dtype])
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor arguments must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != 0:
+        detail = library().moe_last_error().decode() if rc == 3 else ""
+        raise MoeError(rc, where, detail)
+
+
+def moe_workspace_size(cfg: MoeConfig) -> int:
+    return int(library().moe_workspace_size(ctypes.byref(cfg)))
+
+
+def workspace(cfg: MoeConfig, device=None) -> torch.Tensor:
+    """A device workspace large enough for every entry point (256-byte aligned)."""
+    n = moe_workspace_size(cfg)
+    if n == 0:
+        raise MoeError(1, "moe_workspace_size")
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=device or "cuda")
+    off = (-ws.data_ptr()) % 256
+    return ws[off:off + n]
+
+
+def moe_route(cfg: MoeConfig, x: torch.Tensor, W_g: torch.Tensor, b_e: Optional[torch.Tensor] = None,
+              want_probs: bool = False, stream=None):
+    """Returns (topk_ids [N,k] int32, topk_w [N,k] f32, probs [N,E] f32 or None)."""
+    dev = x.device
+    ids = torch.empty((cfg.N, cfg.k), dtype=torch.int32, device=dev)
+    w = torch.empty((cfg.N, cfg.k), dtype=torch.float32, device=dev)
+    probs = torch.empty((cfg.N, cfg.E), dtype=torch.float32, device=dev) if want_probs else None
+    rc = library().moe_route(ctypes.byref(cfg), _ptr(x), _ptr(W_g), _ptr(b_e), _ptr(ids), _ptr(w), _ptr(probs),
+                             _stream(stream))
+    _check(rc, "moe_route")
+    return ids, w, probs
+
+
+def moe_dispatch(cfg: MoeConfig, topk_ids: torch.Tensor, x: Optional[torch.Tensor] = None,
+                 ws: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
+    """Sorted dispatch: x_sorted (if x given), perm, inv_perm, offsets, counts, status."""
+    dev = topk_ids.device
+    A = cfg.N * cfg.k
+    ws = ws if ws is not None else workspace(cfg, dev)
+    out = {
+        "x_sorted": torch.empty((A, cfg.d_model), dtype=cfg.torch_dtype, device=dev) if x is not None else None,
+        "perm": torch.empty(A, dtype=torch.int32, device=dev),
+        "inv_perm": torch.empty(A, dtype=torch.int32, device=dev),
+        "offsets": torch.empty(cfg.E + 1, dtype=torch.int32, device=dev),
+        "counts": torch.empty(cfg.E, dtype=torch.int32, device=dev),
+        "status": torch.zeros(1, dtype=torch.int32, device=dev),
+    }
+    rc = library().moe_dispatch(ctypes.byref(cfg), _ptr(x), _ptr(topk_ids), _ptr(out["x_sorted"]), _ptr(out["perm"]),
+                                _ptr(out["inv_perm"]), _ptr(out["offsets"]), _ptr(out["counts"]),
+                                _ptr(out["status"]), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "moe_dispatch")
+    return out
+
+
+def moe_expert_ffn(cfg: MoeConfig, x_sorted: torch.Tensor, offsets: torch.Tensor, W1: torch.Tensor,
+                   W2: torch.Tensor, b1: Optional[torch.Tensor] = None, W3: Optional[torch.Tensor] = None,
+                   b2: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                   status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    dev = x_sorted.device
+    ws = ws if ws is not None else workspace(cfg, dev)
+    y_sorted = torch.empty((cfg.N * cfg.k, cfg.d_model), dtype=cfg.torch_dtype, device=dev)
+    rc = library().moe_expert_ffn(ctypes.byref(cfg), _ptr(x_sorted), _ptr(offsets), _ptr(W1), _ptr(b1), _ptr(W3),
+                                  _ptr(W2), _ptr(b2), _ptr(y_sorted), _ptr(status), _ptr(ws), ws.numel(),
+                                  _stream(stream))
+    _check(rc, "moe_expert_ffn")
+    return y_sorted
+
+
+def moe_combine(cfg: MoeConfig, y_sorted: torch.Tensor, topk_w: torch.Tensor, inv_perm: torch.Tensor,
+                stream=None) -> torch.Tensor:
+    y = torch.empty((cfg.N, cfg.d_model), dtype=cfg.torch_dtype, device=y_sorted.device)
+    rc = library().moe_combine(ctypes.byref(cfg), _ptr(y_sorted), _ptr(topk_w), _ptr(inv_perm), _ptr(y),
+                               _stream(stream))
+    _check(rc, "moe_combine")
+    return y
+
+
+def moe_aux_loss(cfg: MoeConfig, probs: torch.Tensor, topk_ids: torch.Tensor, gamma: float = 0.0,
+                 b_e: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """Returns (aux [1] f32, counts [E] int32, status [1] int32); updates b_e in place if gamma > 0."""
+    dev = probs.device
+    ws = ws if ws is not None else workspace(cfg, dev)
+    aux = torch.empty(1, dtype=torch.float32, device=dev)
+    counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    rc = library().moe_aux_loss(ctypes.byref(cfg), _ptr(probs), _ptr(topk_ids), _ptr(aux), _ptr(counts),
+                                float(gamma), _ptr(b_e), _ptr(status), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "moe_aux_loss")
+    return aux, counts, status
+
+
+class StageEvents:
+    """MOE_NUM_STAGES + 1 CUDA events that moe_forward records at stage boundaries."""
+
+    def __init__(self):
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(NUM_STAGES + 1)]
+        for e in self.events:           # materialise the CUDA event handles
+            e.record()
+        self._arr = (ctypes.c_void_p * (NUM_STAGES + 1))(*[e.cuda_event for e in self.events])
+
+    @property
+    def pointer(self):
+        return ctypes.cast(self._arr, ctypes.c_void_p)
+
+    def elapsed_ms(self) -> Dict[str, float]:
+        """Per-stage milliseconds of the last recorded forward (synchronises)."""
+        self.events[-1].synchronize()
+        return {STAGE_NAMES[i]: self.events[i].elapsed_time(self.events[i + 1]) for i in range(NUM_STAGES)}
+
+
+def moe_forward(cfg: MoeConfig, x: torch.Tensor, W_g: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor,
+                W3: Optional[torch.Tensor] = None, b1: Optional[torch.Tensor] = None,
+                b2: Optional[torch.Tensor] = None, b_e: Optional[torch.Tensor] = None, gamma: float = 0.0,
+                ws: Optional[torch.Tensor] = None, out: Optional[Dict[str, torch.Tensor]] = None,
+                stage_events: Optional[StageEvents] = None, stream=None) -> Dict[str, torch.Tensor]:
+    """The whole layer: y, topk_ids, topk_w, counts, aux (Switch loss), status.
+
+    b_e (sigmoid router) selects only; with gamma > 0 it is moved in place by one
+    sign-rule step after the selection.  ``out`` may hold preallocated outputs.
+    """
+    dev = x.device
+    ws = ws if ws is not None else workspace(cfg, dev)
+    if out is None:
+        out = forward_outputs(cfg, dev)
+    rc = library().moe_forward(ctypes.byref(cfg), _ptr(x), _ptr(W_g), _ptr(b_e), float(gamma), _ptr(W1), _ptr(b1),
+                               _ptr(W3), _ptr(W2), _ptr(b2), _ptr(out["y"]), _ptr(out["topk_ids"]),
+                               _ptr(out["topk_w"]), _ptr(out["counts"]), _ptr(out["aux"]), _ptr(out["status"]),
+                               _ptr(ws), ws.numel(), stage_events.pointer if stage_events else None,
+                               _stream(stream))
+    _check(rc, "moe_forward")
+    return out
+
+
+def forward_outputs(cfg: MoeConfig, device) -> Dict[str, torch.Tensor]:
+    return {
+        "y": torch.empty((cfg.N, cfg.d_model), dtype=cfg.torch_dtype, device=device),
+        "topk_ids": torch.empty((cfg.N, cfg.k), dtype=torch.int32, device=device),
+        "topk_w": torch.empty((cfg.N, cfg.k), dtype=torch.float32, device=device),
+        "counts": torch.empty(cfg.E, dtype=torch.int32, device=device),
+        "aux": torch.empty(1, dtype=torch.float32, device=device),
+        "status": torch.zeros(1, dtype=torch.int32, device=device),
+    }
+
+
+__all__ = ["MoeConfig", "MoeError", "make_config", "library", "workspace", "moe_workspace_size", "moe_route",
+           "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_aux_loss", "moe_forward", "forward_outputs",
+           "StageEvents", "EXPORTS", "LIB_PATH"]

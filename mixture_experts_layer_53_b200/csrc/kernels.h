@@ -1,0 +1,107 @@
+// kernels.h -- host-side launchers of the MoE kernels (internal to libmoe).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// dtype / router / activation codes are those of moe.h.
+enum { kF32 = 0, kBF16 = 1 };
+enum { kSoftmaxTopk = 0, kTopkSoftmax = 1, kSigmoid = 2 };
+enum { kGelu = 0, kSwiglu = 1 };
+
+inline int64_t num_chunks(int64_t N) { return (N + 31) / 32; }
+
+struct RouterArgs {
+    const void *x;       // [N, d]
+    const void *Wg;      // [E, d]
+    const float *b_sel;  // [E] or null (sigmoid router only)
+    int32_t *ids;        // [N, k]
+    float *w;            // [N, k]
+    float *probs;        // [N, E] or null
+    int32_t *hist;       // [chunks, E] or null
+    float *psum;         // [chunks, E] or null
+    int64_t N;
+    int d, E, k, router, norm_topk;
+    float scaling;
+};
+cudaError_t launch_router(int dtype, const RouterArgs &a, cudaStream_t s);
+
+// Per-chunk histograms of expert ids (with range check) and, optionally,
+// per-chunk sums of probs.
+struct HistArgs {
+    const int32_t *ids;  // [N, k] or null (then hist is not written)
+    const float *probs;  // [N, E] or null
+    int32_t *hist;       // [chunks, E]
+    float *psum;         // [chunks, E] or null
+    int32_t *status;
+    int64_t N;
+    int E, k;
+};
+cudaError_t launch_hist(const HistArgs &a, cudaStream_t s);
+
+// One CTA: counts, offsets, per-chunk bases (in place over hist), the GEMM
+// tile table, the Switch loss and the sign-rule bias step.
+struct ScanArgs {
+    int32_t *hist;        // in: [chunks, E] counts; out: per-chunk slice bases
+    const float *psum;    // [chunks, E] or null (no loss then)
+    int64_t chunks, N;
+    int E, k;
+    int32_t *counts;      // [E] or null
+    int32_t *offsets;     // [E+1]
+    int32_t *mt_prefix;   // [E+1] or null
+    float *aux_out;       // scalar or null
+    float gamma;
+    float *b_e;           // [E] or null
+};
+cudaError_t launch_scan(const ScanArgs &a, cudaStream_t s);
+
+struct ScatterArgs {
+    const int32_t *ids;
+    const int32_t *chunk_base;  // [chunks, E]
+    int32_t *perm;              // [N k] or null
+    int32_t *inv_perm;          // [N k]
+    int64_t N;
+    int E, k;
+};
+cudaError_t launch_scatter(const ScatterArgs &a, cudaStream_t s);
+
+struct GatherArgs {
+    const void *x;
+    const int32_t *inv_perm;
+    void *x_sorted;
+    int64_t N;
+    int d, k;
+};
+cudaError_t launch_gather(int dtype, const GatherArgs &a, int num_sms, cudaStream_t s);
+
+struct CombineArgs {
+    const void *y_sorted;
+    const float *w;
+    const int32_t *inv_perm;
+    void *y;
+    int64_t N;
+    int d, k;
+};
+cudaError_t launch_combine(int dtype, const CombineArgs &a, int num_sms, cudaStream_t s);
+
+// mt_prefix[e+1] = mt_prefix[e] + ceil((offsets[e+1] - offsets[e]) / 128).
+cudaError_t launch_tile_table(const int32_t *offsets, int32_t *mt_prefix, int E, cudaStream_t s);
+
+struct FfnArgs {
+    const void *x_sorted;      // [rows, d]
+    const int32_t *offsets;    // [E+1]
+    const int32_t *mt_prefix;  // [E+1]
+    const void *W1, *b1, *W3, *W2, *b2;
+    void *h;                   // [rows, F] scratch
+    void *y_sorted;            // [rows, d]
+    int32_t *status;
+    int64_t rows;              // N k
+    int d, F, E, act;
+};
+// Both expert GEMMs; `mid` (may be null) is recorded between them.
+cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid, cudaStream_t s);
+cudaError_t launch_ffn_f32_simt(const FfnArgs &a, int num_sms, cudaEvent_t mid, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,386 @@
+// moe_api.cu -- the extern "C" entry points of libmoe.so (declared in
+// include/moe.h): argument validation, workspace carving and the launch
+// sequence of each operation.  No allocation, no host synchronisation.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+#include <string>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+using namespace moe;
+
+thread_local std::string g_last_error;
+
+moe_status cuda_fail(cudaError_t err)
+{
+    g_last_error = cudaGetErrorString(err);
+    return MOE_ERR_CUDA;
+}
+
+int num_sms()
+{
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+size_t elem_size(const moe_config *c) { return c->dtype == MOE_F32 ? 4 : 2; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status validate(const moe_config *c)
+{
+    if (!c) return MOE_ERR_INVALID_ARG;
+    if (c->N < 0 || c->d_model <= 0 || c->d_ff <= 0 || c->E <= 0 || c->k <= 0) return MOE_ERR_INVALID_ARG;
+    if (c->k > c->E) return MOE_ERR_INVALID_ARG;
+    if (c->router < MOE_ROUTER_SOFTMAX_TOPK || c->router > MOE_ROUTER_SIGMOID) return MOE_ERR_INVALID_ARG;
+    if (c->act < MOE_ACT_GELU || c->act > MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
+    if (c->dtype < MOE_F32 || c->dtype > MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (c->norm_topk != 0 && c->norm_topk != 1) return MOE_ERR_INVALID_ARG;
+    if (!std::isfinite(c->routed_scaling)) return MOE_ERR_INVALID_ARG;
+    if (c->E > kMaxE || c->k > kMaxK) return MOE_ERR_UNSUPPORTED;
+    if (c->d_model % 8 != 0 || c->d_ff % 8 != 0) return MOE_ERR_UNSUPPORTED;
+    if (c->N * static_cast<int64_t>(c->k) >= (static_cast<int64_t>(1) << 31)) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+struct Layout {
+    size_t hist, psum, offsets, mt, counts, ids, w, perm, inv, xs, h, ys, total;
+};
+
+size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+Layout layout(const moe_config *c)
+{
+    Layout L{};
+    size_t o = 0;
+    auto take = [&o](size_t bytes) {
+        const size_t at = o;
+        o += align256(bytes > 0 ? bytes : 1);
+        return at;
+    };
+    const size_t C = static_cast<size_t>(num_chunks(c->N));
+    const size_t E = static_cast<size_t>(c->E);
+    const size_t A = static_cast<size_t>(c->N) * static_cast<size_t>(c->k);
+    const size_t es = elem_size(c);
+    L.hist = take(C * E * 4);
+    L.psum = take(C * E * 4);
+    L.offsets = take((E + 1) * 4);
+    L.mt = take((E + 1) * 4);
+    L.counts = take(E * 4);
+    L.ids = take(A * 4);
+    L.w = take(A * 4);
+    L.perm = take(A * 4);
+    L.inv = take(A * 4);
+    L.xs = take(A * c->d_model * es);
+    L.h = take(A * c->d_ff * es);
+    L.ys = take(A * c->d_model * es);
+    L.total = o;
+    return L;
+}
+
+template <typename T> T *at(void *ws, size_t off) { return reinterpret_cast<T *>(static_cast<char *>(ws) + off); }
+
+moe_status check_ws(const moe_config *c, const void *ws, size_t ws_bytes)
+{
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < layout(c).total) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+RouterArgs router_args(const moe_config *c, const void *x, const void *W_g, const float *b_e, int32_t *ids,
+                       float *w, float *probs, int32_t *hist, float *psum)
+{
+    RouterArgs r{};
+    r.x = x;
+    r.Wg = W_g;
+    r.b_sel = c->router == MOE_ROUTER_SIGMOID ? b_e : nullptr;
+    r.ids = ids;
+    r.w = w;
+    r.probs = probs;
+    r.hist = hist;
+    r.psum = psum;
+    r.N = c->N;
+    r.d = c->d_model;
+    r.E = c->E;
+    r.k = c->k;
+    r.router = c->router;
+    r.norm_topk = c->norm_topk;
+    r.scaling = c->routed_scaling;
+    return r;
+}
+
+FfnArgs ffn_args(const moe_config *c, const void *x_sorted, const int32_t *offsets, const int32_t *mt,
+                 const void *W1, const void *b1, const void *W3, const void *W2, const void *b2, void *h,
+                 void *y_sorted, int32_t *status)
+{
+    FfnArgs f{};
+    f.x_sorted = x_sorted;
+    f.offsets = offsets;
+    f.mt_prefix = mt;
+    f.W1 = W1;
+    f.b1 = c->act == MOE_ACT_GELU ? b1 : nullptr;
+    f.W3 = W3;
+    f.W2 = W2;
+    f.b2 = b2;
+    f.h = h;
+    f.y_sorted = y_sorted;
+    f.status = status;
+    f.rows = c->N * c->k;
+    f.d = c->d_model;
+    f.F = c->d_ff;
+    f.E = c->E;
+    f.act = c->act;
+    return f;
+}
+
+moe_status check_ffn_ptrs(const moe_config *c, const void *W1, const void *b1, const void *W3, const void *W2,
+                          const void *b2)
+{
+    if (!W1 || !W2) return MOE_ERR_INVALID_ARG;
+    if (c->act == MOE_ACT_SWIGLU && !W3) return MOE_ERR_INVALID_ARG;
+    if (c->act == MOE_ACT_SWIGLU && b1) return MOE_ERR_INVALID_ARG;  // SwiGLU experts carry no hidden bias
+    if (!aligned16(W1) || !aligned16(W2) || (W3 && !aligned16(W3)) || (b1 && !aligned16(b1)) ||
+        (b2 && !aligned16(b2)))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+cudaError_t launch_ffn(const moe_config *c, const FfnArgs &f, cudaEvent_t mid, cudaStream_t s)
+{
+    return c->dtype == MOE_BF16 ? launch_ffn_bf16_sm100(f, num_sms(), mid, s)
+                                : launch_ffn_f32_simt(f, num_sms(), mid, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_status_string(moe_status s)
+{
+    switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_BAD_EXPERT_ID: return "expert id out of range";
+    }
+    return "unknown status";
+}
+
+const char *moe_last_error(void) { return g_last_error.c_str(); }
+
+int32_t moe_version(void) { return 100; }
+
+size_t moe_workspace_size(const moe_config *cfg)
+{
+    if (validate(cfg) != MOE_OK) return 0;
+    return layout(cfg).total;
+}
+
+moe_status moe_route(const moe_config *cfg, const void *x, const void *W_g, const float *b_e, int32_t *topk_ids,
+                     float *topk_w, float *probs, moe_stream_t stream)
+{
+    moe_status st = validate(cfg);
+    if (st != MOE_OK) return st;
+    const bool empty = cfg->N == 0;  // token-sized buffers may then be NULL
+    if (!W_g || (!empty && (!x || !topk_ids || !topk_w))) return MOE_ERR_INVALID_ARG;
+    if (b_e && cfg->router != MOE_ROUTER_SIGMOID) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W_g)) return MOE_ERR_INVALID_ARG;
+    if (cfg->N == 0) return MOE_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const RouterArgs r = router_args(cfg, x, W_g, b_e, topk_ids, topk_w, probs, nullptr, nullptr);
+    cudaError_t err = launch_router(cfg->dtype, r, s);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err);
+}
+
+moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *topk_ids, void *x_sorted,
+                        int32_t *perm, int32_t *inv_perm, int32_t *offsets, int32_t *counts, int32_t *dev_status,
+                        void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status st = validate(cfg);
+    if (st != MOE_OK) return st;
+    const bool empty = cfg->N == 0;
+    if (!offsets || !counts || (!empty && (!topk_ids || !inv_perm))) return MOE_ERR_INVALID_ARG;
+    if ((x == nullptr) != (x_sorted == nullptr)) return MOE_ERR_INVALID_ARG;
+    if ((x && !aligned16(x)) || (x_sorted && !aligned16(x_sorted))) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Layout L = layout(cfg);
+    int32_t *hist = at<int32_t>(ws, L.hist);
+    cudaError_t err;
+    HistArgs h{topk_ids, nullptr, hist, nullptr, dev_status, cfg->N, cfg->E, cfg->k};
+    if ((err = launch_hist(h, s)) != cudaSuccess) return cuda_fail(err);
+    ScanArgs sc{};
+    sc.hist = hist;
+    sc.chunks = num_chunks(cfg->N);
+    sc.N = cfg->N;
+    sc.E = cfg->E;
+    sc.k = cfg->k;
+    sc.counts = counts;
+    sc.offsets = offsets;
+    if ((err = launch_scan(sc, s)) != cudaSuccess) return cuda_fail(err);
+    ScatterArgs sa{topk_ids, hist, perm, inv_perm, cfg->N, cfg->E, cfg->k};
+    if ((err = launch_scatter(sa, s)) != cudaSuccess) return cuda_fail(err);
+    if (x) {
+        GatherArgs ga{x, inv_perm, x_sorted, cfg->N, cfg->d_model, cfg->k};
+        if ((err = launch_gather(cfg->dtype, ga, num_sms(), s)) != cudaSuccess) return cuda_fail(err);
+    }
+    return MOE_OK;
+}
+
+moe_status moe_expert_ffn(const moe_config *cfg, const void *x_sorted, const int32_t *offsets, const void *W1,
+                          const void *b1, const void *W3, const void *W2, const void *b2, void *y_sorted,
+                          int32_t *dev_status, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status st = validate(cfg);
+    if (st != MOE_OK) return st;
+    const bool empty = cfg->N == 0;
+    if (!offsets || (!empty && (!x_sorted || !y_sorted))) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_sorted) || !aligned16(y_sorted)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ffn_ptrs(cfg, W1, b1, W3, W2, b2)) != MOE_OK) return st;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Layout L = layout(cfg);
+    int32_t *mt = at<int32_t>(ws, L.mt);
+    cudaError_t err;
+    if ((err = launch_tile_table(offsets, mt, cfg->E, s)) != cudaSuccess) return cuda_fail(err);
+    const FfnArgs f = ffn_args(cfg, x_sorted, offsets, mt, W1, b1, W3, W2, b2, at<void>(ws, L.h), y_sorted,
+                               dev_status);
+    if ((err = launch_ffn(cfg, f, nullptr, s)) != cudaSuccess) return cuda_fail(err);
+    return MOE_OK;
+}
+
+moe_status moe_combine(const moe_config *cfg, const void *y_sorted, const float *topk_w, const int32_t *inv_perm,
+                       void *y, moe_stream_t stream)
+{
+    moe_status st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (cfg->N > 0 && (!y_sorted || !topk_w || !inv_perm || !y)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y_sorted) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    CombineArgs ca{y_sorted, topk_w, inv_perm, y, cfg->N, cfg->d_model, cfg->k};
+    cudaError_t err = launch_combine(cfg->dtype, ca, num_sms(), s);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err);
+}
+
+moe_status moe_aux_loss(const moe_config *cfg, const float *probs, const int32_t *topk_ids, float *aux_out,
+                        int32_t *counts_out, float gamma, float *b_e_inout, int32_t *dev_status, void *ws,
+                        size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (!aux_out || (cfg->N > 0 && (!probs || !topk_ids))) return MOE_ERR_INVALID_ARG;
+    if (!(gamma >= 0.f) || !std::isfinite(gamma)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Layout L = layout(cfg);
+    int32_t *hist = at<int32_t>(ws, L.hist);
+    float *psum = at<float>(ws, L.psum);
+    cudaError_t err;
+    HistArgs h{topk_ids, probs, hist, psum, dev_status, cfg->N, cfg->E, cfg->k};
+    if ((err = launch_hist(h, s)) != cudaSuccess) return cuda_fail(err);
+    ScanArgs sc{};
+    sc.hist = hist;
+    sc.psum = psum;
+    sc.chunks = num_chunks(cfg->N);
+    sc.N = cfg->N;
+    sc.E = cfg->E;
+    sc.k = cfg->k;
+    sc.counts = counts_out;
+    sc.offsets = at<int32_t>(ws, L.offsets);
+    sc.aux_out = aux_out;
+    sc.gamma = gamma;
+    sc.b_e = b_e_inout;
+    if ((err = launch_scan(sc, s)) != cudaSuccess) return cuda_fail(err);
+    return MOE_OK;
+}
+
+moe_status moe_forward(const moe_config *cfg, const void *x, const void *W_g, float *b_e_inout, float gamma,
+                       const void *W1, const void *b1, const void *W3, const void *W2, const void *b2, void *y,
+                       int32_t *topk_ids, float *topk_w, int32_t *counts, float *aux_out, int32_t *dev_status,
+                       void *ws, size_t ws_bytes, void *const *stage_events, moe_stream_t stream)
+{
+    moe_status st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (!W_g || (cfg->N > 0 && (!x || !y))) return MOE_ERR_INVALID_ARG;  // N = 0: x, y may be NULL
+    if (!aligned16(x) || !aligned16(W_g) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+    if (b_e_inout && cfg->router != MOE_ROUTER_SIGMOID) return MOE_ERR_INVALID_ARG;
+    if (!(gamma >= 0.f) || !std::isfinite(gamma)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ffn_ptrs(cfg, W1, b1, W3, W2, b2)) != MOE_OK) return st;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Layout L = layout(cfg);
+    cudaEvent_t ev[MOE_NUM_STAGES + 1] = {};
+    if (stage_events)
+        for (int i = 0; i <= MOE_NUM_STAGES; ++i) ev[i] = static_cast<cudaEvent_t>(stage_events[i]);
+    auto mark = [&](int i) { return ev[i] ? cudaEventRecord(ev[i], s) : cudaSuccess; };
+
+    int32_t *hist = at<int32_t>(ws, L.hist);
+    float *psum = at<float>(ws, L.psum);
+    int32_t *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *mt = at<int32_t>(ws, L.mt);
+    int32_t *ids = topk_ids ? topk_ids : at<int32_t>(ws, L.ids);
+    float *w = topk_w ? topk_w : at<float>(ws, L.w);
+    int32_t *inv = at<int32_t>(ws, L.inv);
+    void *xs = at<void>(ws, L.xs);
+    void *ys = at<void>(ws, L.ys);
+
+    cudaError_t err;
+    if ((err = mark(0)) != cudaSuccess) return cuda_fail(err);
+    if (dev_status && (err = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s)) != cudaSuccess)
+        return cuda_fail(err);
+    // route: logits, scores, top-k, gates, per-chunk histograms and P sums
+    const RouterArgs r = router_args(cfg, x, W_g, b_e_inout, ids, w, nullptr, hist, psum);
+    if (cfg->N > 0 && (err = launch_router(cfg->dtype, r, s)) != cudaSuccess) return cuda_fail(err);
+    if ((err = mark(1)) != cudaSuccess) return cuda_fail(err);
+    // dispatch: counts, offsets, tile table, Switch loss, bias step; scatter; gather
+    ScanArgs sc{};
+    sc.hist = hist;
+    sc.psum = psum;
+    sc.chunks = num_chunks(cfg->N);
+    sc.N = cfg->N;
+    sc.E = cfg->E;
+    sc.k = cfg->k;
+    sc.counts = counts;
+    sc.offsets = offsets;
+    sc.mt_prefix = mt;
+    sc.aux_out = aux_out;
+    sc.gamma = gamma;
+    sc.b_e = b_e_inout;
+    if ((err = launch_scan(sc, s)) != cudaSuccess) return cuda_fail(err);
+    ScatterArgs sa{ids, hist, nullptr, inv, cfg->N, cfg->E, cfg->k};
+    if ((err = launch_scatter(sa, s)) != cudaSuccess) return cuda_fail(err);
+    GatherArgs ga{x, inv, xs, cfg->N, cfg->d_model, cfg->k};
+    if ((err = launch_gather(cfg->dtype, ga, num_sms(), s)) != cudaSuccess) return cuda_fail(err);
+    if ((err = mark(2)) != cudaSuccess) return cuda_fail(err);
+    // expert FFNs over the ragged slices
+    const FfnArgs f = ffn_args(cfg, xs, offsets, mt, W1, b1, W3, W2, b2, at<void>(ws, L.h), ys, dev_status);
+    if ((err = launch_ffn(cfg, f, ev[3], s)) != cudaSuccess) return cuda_fail(err);
+    if ((err = mark(4)) != cudaSuccess) return cuda_fail(err);
+    // combine back in token order
+    CombineArgs ca{ys, w, inv, y, cfg->N, cfg->d_model, cfg->k};
+    if ((err = launch_combine(cfg->dtype, ca, num_sms(), s)) != cudaSuccess) return cuda_fail(err);
+    if ((err = mark(5)) != cudaSuccess) return cuda_fail(err);
+    return MOE_OK;
+}
+
+}  // extern "C"

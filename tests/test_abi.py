@@ -1,0 +1,160 @@
+"""The C ABI of libmoe.so on the CPU: exports, struct layout, validation.
+
+No compute call is made here: every call below fails argument validation,
+which returns before anything touches CUDA.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import mixture_experts_layer_53_b200 as M
+from mixture_experts_layer_53_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+BAD = ctypes.c_void_p(0x1001)  # never dereferenced: every call here fails validation first
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return M.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(M.EXPORTS), names
+    out = subprocess.check_output(["nm", "-D", "--defined-only", M.LIB_PATH], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in names:
+        assert name in exported, f"{name} declared in moe.h but not exported"
+        assert hasattr(lib, name)
+    assert all(e.startswith("moe_") for e in exported), sorted(e for e in exported if not e.startswith("moe_"))
+
+
+def test_config_layout_matches_header(tmp_path):
+    src = tmp_path / "probe.c"
+    src.write_text("""
+#include <stddef.h>
+#include <stdio.h>
+#include "moe.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(moe_config),
+         offsetof(moe_config, N), offsetof(moe_config, d_model), offsetof(moe_config, d_ff),
+         offsetof(moe_config, E), offsetof(moe_config, k), offsetof(moe_config, router),
+         offsetof(moe_config, norm_topk), offsetof(moe_config, routed_scaling),
+         offsetof(moe_config, act), offsetof(moe_config, dtype));
+  return 0;
+}
+""")
+    exe = tmp_path / "probe"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)])
+    got = [int(v) for v in subprocess.check_output([str(exe)], text=True).split()]
+    C = M.MoeConfig
+    want = [ctypes.sizeof(C)] + [getattr(C, f).offset for f, _ in C._fields_]
+    assert got == want
+
+
+def test_status_strings_and_version(lib):
+    for code in range(7):
+        assert lib.moe_status_string(code)
+    assert lib.moe_version() >= 100
+
+
+def cfg(**kw):
+    base = dict(N=64, d_model=64, d_ff=128, E=4, k=2, router="softmax_topk", act="gelu", dtype="f32")
+    base.update(kw)
+    return M.make_config(**base)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(k=5), 1), (dict(k=0), 1), (dict(E=0), 1), (dict(N=-1), 1), (dict(d_model=0), 1),
+    (dict(E=257, k=2), 2), (dict(E=32, k=17), 2), (dict(d_model=60), 2), (dict(d_ff=100), 2),
+    (dict(N=2 ** 31, k=2), 2),
+])
+def test_invalid_configs(lib, bad, code):
+    c = cfg(**bad)
+    assert lib.moe_workspace_size(ctypes.byref(c)) == 0
+    rc = lib.moe_route(ctypes.byref(c), BAD, BAD, None, BAD, BAD, None, None)
+    assert rc == code
+
+
+def test_invalid_enums(lib):
+    for field, value in (("router", 3), ("act", 2), ("dtype", 5), ("norm_topk", 2)):
+        c = cfg()
+        setattr(c, field, value)
+        assert lib.moe_workspace_size(ctypes.byref(c)) == 0
+        assert lib.moe_combine(ctypes.byref(c), BAD, BAD, BAD, BAD, None) == 1
+    c = cfg()
+    c.routed_scaling = float("nan")
+    assert lib.moe_workspace_size(ctypes.byref(c)) == 0
+
+
+def test_null_and_misaligned_pointers(lib):
+    c = cfg()
+    assert lib.moe_route(ctypes.byref(c), None, BAD, None, BAD, BAD, None, None) == 1
+    assert lib.moe_route(ctypes.byref(c), ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2008), None,
+                         ctypes.c_void_p(0x3000), ctypes.c_void_p(0x4000), None, None) == 1
+    assert lib.moe_combine(ctypes.byref(c), None, BAD, BAD, BAD, None) == 1
+    assert lib.moe_route(None, BAD, BAD, None, BAD, BAD, None, None) == 1
+
+
+def test_bias_only_for_sigmoid_router(lib):
+    c = cfg()
+    a = ctypes.c_void_p(0x10000)
+    assert lib.moe_route(ctypes.byref(c), a, a, a, a, a, None, None) == 1
+    rc = lib.moe_forward(ctypes.byref(c), a, a, a, ctypes.c_float(0.0), a, a, None, a, a, a, None, None, None,
+                         None, None, a, ctypes.c_size_t(1 << 40), None, None)
+    assert rc == 1
+
+
+def test_swiglu_rejects_hidden_bias_and_needs_W3(lib):
+    c = cfg(act="swiglu")
+    a = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x100000)
+    # b1 given with SwiGLU
+    assert lib.moe_expert_ffn(ctypes.byref(c), a, a, a, a, a, a, None, a, None, ws, ctypes.c_size_t(1 << 40),
+                              None) == 1
+    # W3 missing
+    assert lib.moe_expert_ffn(ctypes.byref(c), a, a, a, None, None, a, None, a, None, ws,
+                              ctypes.c_size_t(1 << 40), None) == 1
+
+
+def test_workspace_checks(lib):
+    c = cfg()
+    need = lib.moe_workspace_size(ctypes.byref(c))
+    assert need > 0
+    a = ctypes.c_void_p(0x10000)
+    ws_misaligned = ctypes.c_void_p(0x100010)
+    ws = ctypes.c_void_p(0x100000)
+    assert lib.moe_dispatch(ctypes.byref(c), None, a, None, None, a, a, a, None, None, ctypes.c_size_t(need),
+                            None) == 4
+    assert lib.moe_dispatch(ctypes.byref(c), None, a, None, None, a, a, a, None, ws_misaligned,
+                            ctypes.c_size_t(need), None) == 4
+    assert lib.moe_dispatch(ctypes.byref(c), None, a, None, None, a, a, a, None, ws, ctypes.c_size_t(need - 1),
+                            None) == 4
+    # gamma must be finite and >= 0
+    assert lib.moe_aux_loss(ctypes.byref(c), a, a, a, None, ctypes.c_float(-1.0), None, None, ws,
+                            ctypes.c_size_t(need), None) == 1
+
+
+def test_workspace_grows_with_tokens(lib):
+    sizes = [lib.moe_workspace_size(ctypes.byref(cfg(N=n, dtype="bf16"))) for n in (0, 1, 64, 1000)]
+    assert sizes[0] > 0 and sizes == sorted(sizes) and sizes[3] > sizes[2]
+    # x_sorted + h + y_sorted dominate: N k (2 d + F) elements
+    c = cfg(N=4096, d_model=4096, d_ff=14336, E=8, k=2, act="swiglu", dtype="bf16")
+    n = lib.moe_workspace_size(ctypes.byref(c))
+    assert n >= 4096 * 2 * (2 * 4096 + 14336) * 2
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    with pytest.raises(RuntimeError, match="missing"):
+        M.library(str(tmp_path / "libmoe.so"))

@@ -1,0 +1,227 @@
+"""CUDA layer vs the fp64 oracle, through the C ABI, on a B200 (marked gpu).
+
+Small cases (all tokens compared) span several 128-row GEMM tiles with
+ragged expert slices, reduction dims that are not multiples of the 64-wide
+k-block and hidden widths that are not multiples of the N tile.  The five
+full-size workloads run in the launch configuration the benchmark times;
+there the routing, dispatch and loss are compared on every token and y on
+sampled tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_layer_53_b200 as M
+import oracle as O
+import workloads as W
+from parity import (MARGIN, TOL_Y, check_forward, config_of, gpu_forward, np64, oracle_routing,
+                    sample_tokens)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+SMALL = {
+    "tiny_fp32": W.WORKLOADS["tiny_fp32"],
+    "tiny_fp32_ragged": W.WORKLOADS["tiny_fp32"].scaled(N=333, d_model=72, d_ff=136, E=5, k=3),
+    "gpt2_small": W.WORKLOADS["gpt2_moe"].scaled(N=300, d_model=256, d_ff=512),
+    "gpt2_odd": W.WORKLOADS["gpt2_moe"].scaled(N=257, d_model=200, d_ff=328, E=5),
+    "mixtral_small": W.WORKLOADS["mixtral"].scaled(N=200, d_model=512, d_ff=768),
+    "mixtral_odd": W.WORKLOADS["mixtral"].scaled(N=161, d_model=136, d_ff=200, E=3),
+    "deepseek_small": W.WORKLOADS["deepseek_v3"].scaled(N=256, d_model=384, d_ff=256, E=64),
+    "qwen3_small": W.WORKLOADS["qwen3_skew"].scaled(N=512, d_model=256, d_ff=128),
+    "topk_softmax_small": W.WORKLOADS["gpt2_moe"].scaled(N=130, d_model=128, d_ff=256, E=7, k=3,
+                                                         router="topk_softmax"),
+    "sigmoid_no_norm_scaled": W.WORKLOADS["deepseek_v3"].scaled(N=96, d_model=128, d_ff=128, E=16, k=4,
+                                                               norm_topk=False, routed_scaling=2.5),
+}
+
+FULL_SAMPLES = {"tiny_fp32": None, "gpt2_moe": 24, "mixtral": 8, "deepseek_v3": 4, "qwen3_skew": 12}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from mixture_experts_layer_53_b200 import build
+    build.build()
+    M.library()
+    assert torch.cuda.is_available()
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_forward_small(name):
+    wl = SMALL[name]
+    inp = W.make_inputs(wl, DEV)
+    gpu = gpu_forward(wl, inp)
+    rep = check_forward(wl, inp, gpu)
+    print(name, rep.as_dict())
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "gpt2_moe", "mixtral", "deepseek_v3", "qwen3_skew"])
+def test_forward_full_size(name):
+    wl = W.WORKLOADS[name]
+    inp = W.make_inputs(wl, DEV)
+    gpu = gpu_forward(wl, inp)
+    n = FULL_SAMPLES[name]
+    tokens = None if n is None else sample_tokens(wl.N, n, seed=wl.seed)
+    rep = check_forward(wl, inp, gpu, y_tokens=tokens)
+    print(name, rep.as_dict())
+    del inp
+    torch.cuda.empty_cache()
+
+
+def test_forward_is_deterministic():
+    wl = SMALL["qwen3_small"]
+    inp = W.make_inputs(wl, DEV)
+    a = gpu_forward(wl, inp)
+    b = gpu_forward(wl, inp)
+    for key in ("y", "topk_ids", "topk_w", "counts", "aux"):
+        assert np.array_equal(a[key], b[key]), key
+
+
+@pytest.mark.parametrize("name", ["gpt2_small", "deepseek_small", "tiny_fp32"])
+def test_route_entry_point(name):
+    wl = SMALL[name]
+    inp = W.make_inputs(wl, DEV)
+    cfg = config_of(wl)
+    ids, w, probs = M.moe_route(cfg, inp["x"], inp["W_g"], b_e=inp["b_e"], want_probs=True)
+    torch.cuda.synchronize()
+    r = oracle_routing(wl, inp)
+    near = r["margin"] < MARGIN
+    ids = ids.cpu().numpy()
+    assert np.all(ids[~near] == r["ids"][~near])
+    assert np.max(np.abs(probs.cpu().numpy() - r["probs"])) <= 1e-6
+    ok = ~near
+    assert np.max(np.abs(w.cpu().numpy()[ok] - r["w"][ok])) <= 2e-5
+
+
+@pytest.mark.parametrize("E,k,N", [(4, 2, 64), (128, 8, 777), (6, 2, 1), (1, 1, 40), (8, 8, 50), (256, 16, 99)])
+def test_dispatch_entry_point(E, k, N):
+    rng = np.random.default_rng(E * 1000 + k)
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(N)]).astype(np.int32)
+    cfg = M.make_config(N, 64, 64, E, k, dtype="bf16")
+    x = torch.randn((N, 64), device=DEV).to(torch.bfloat16)
+    out = M.moe_dispatch(cfg, torch.from_numpy(ids).to(DEV), x=x)
+    torch.cuda.synchronize()
+    want = O.dispatch(ids, E)
+    for key in ("perm", "inv_perm", "offsets", "counts"):
+        assert np.array_equal(out[key].cpu().numpy(), want[key]), key
+    assert torch.equal(out["x_sorted"], x[torch.from_numpy(want["perm"] // k).long().to(DEV)])
+    assert int(out["status"][0]) == 0
+
+
+def test_dispatch_reports_bad_expert_id():
+    N, E, k = 50, 8, 2
+    ids = np.tile(np.array([[0, 1]], np.int32), (N, 1))
+    ids[7, 1] = 8
+    ids[20, 0] = -1
+    cfg = M.make_config(N, 64, 64, E, k, dtype="bf16")
+    x = torch.randn((N, 64), device=DEV).to(torch.bfloat16)
+    out = M.moe_dispatch(cfg, torch.from_numpy(ids).to(DEV), x=x)
+    torch.cuda.synchronize()
+    assert int(out["status"][0]) == 6
+
+
+@pytest.mark.parametrize("dtype,act", [("bf16", "swiglu"), ("bf16", "gelu"), ("f32", "gelu"), ("f32", "swiglu")])
+def test_expert_ffn_entry_point(dtype, act):
+    """Random ragged slices with idle experts; every row checked."""
+    rng = np.random.default_rng(3)
+    E, d, F = 9, 200, 264
+    counts = np.array([0, 130, 1, 0, 257, 5, 128, 0, 40], np.int32)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    rows = int(offsets[-1])
+    wl = W.Workload("ffn", N=rows, d_model=d, d_ff=F, E=E, k=1, act=act, router="softmax_topk",
+                    dtype=dtype, biases=(act == "gelu"), seed=77)
+    ex = W.make_experts(wl, DEV)
+    xs = torch.randn((rows, d), device=DEV).to(wl.torch_dtype)
+    cfg = M.make_config(rows, d, F, E, 1, act=act, dtype=dtype)
+    ys = M.moe_expert_ffn(cfg, xs, torch.from_numpy(offsets).to(DEV), ex["W1"], ex["W2"], b1=ex["b1"],
+                          W3=ex["W3"], b2=ex["b2"])
+    torch.cuda.synchronize()
+    ys = np64(ys)
+    x64 = np64(xs)
+    worst = 0.0
+    for e in range(E):
+        for i in range(offsets[e], offsets[e + 1]):
+            ref = O.expert_ffn(x64[i], np64(ex["W1"][e]), np64(ex["W2"][e]), act,
+                               None if ex["b1"] is None else np64(ex["b1"][e]),
+                               None if ex["W3"] is None else np64(ex["W3"][e]),
+                               None if ex["b2"] is None else np64(ex["b2"][e]))
+            worst = max(worst, float(np.max(np.abs(ys[i] - ref)) / max(np.max(np.abs(ref)), 1e-30)))
+    assert worst <= TOL_Y[dtype], worst
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_combine_entry_point(dtype):
+    rng = np.random.default_rng(5)
+    N, k, d = 300, 3, 136
+    inv = rng.permutation(N * k).astype(np.int32)
+    w = rng.uniform(0, 1, (N, k)).astype(np.float32)
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    ys = torch.randn((N * k, d), device=DEV).to(td)
+    cfg = M.make_config(N, d, 64, 8, k, dtype=dtype)
+    y = M.moe_combine(cfg, ys, torch.from_numpy(w).to(DEV), torch.from_numpy(inv).to(DEV))
+    torch.cuda.synchronize()
+    ref = O.combine(np64(ys), w, inv)
+    err = np.max(np.max(np.abs(np64(y) - ref), axis=1) / np.max(np.abs(ref), axis=1))
+    assert err <= TOL_Y[dtype], err
+
+
+def test_aux_loss_entry_point_and_bias_rule():
+    rng = np.random.default_rng(8)
+    N, E, k = 500, 16, 4
+    z = rng.standard_normal((N, E))
+    p = np.exp(z - z.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    ids = np.argsort(-z, axis=1, kind="stable")[:, :k].astype(np.int32)
+    cfg = M.make_config(N, 64, 64, E, k, router="sigmoid", dtype="bf16")
+    b = torch.from_numpy(rng.uniform(-0.1, 0.1, E).astype(np.float32)).to(DEV)
+    b0 = b.cpu().numpy().copy()
+    aux, counts, status = M.moe_aux_loss(cfg, torch.from_numpy(p.astype(np.float32)).to(DEV),
+                                         torch.from_numpy(ids).to(DEV), gamma=1e-3, b_e=b)
+    torch.cuda.synchronize()
+    want, want_counts = O.aux_loss(p.astype(np.float32), ids)
+    assert abs(float(aux[0]) - want) <= 1e-5
+    assert np.array_equal(counts.cpu().numpy(), want_counts)
+    assert np.max(np.abs(b.cpu().numpy() - O.bias_update(b0, want_counts, N, k, 1e-3))) <= 1e-7
+    assert int(status[0]) == 0
+
+
+def test_balanced_router_gives_loss_k():
+    """Circulant router: every expert in exactly k top-k sets, so L = k."""
+    E, k = 8, 2
+    v = np.array([1.5, -0.5, 0.75, 0.0, -1.25, 0.5, 1.0, -0.25], np.float32)
+    Wg = np.array([[v[(e - n) % E] for n in range(E)] for e in range(E)], np.float32)
+    wl = W.Workload("bal", N=E, d_model=E, d_ff=64, E=E, k=k, act="gelu", router="softmax_topk", dtype="f32",
+                    biases=True, seed=5)
+    inp = W.make_inputs(wl.scaled(d_model=8), DEV)
+    inp["x"] = torch.eye(E, device=DEV)
+    inp["W_g"] = torch.from_numpy(Wg).to(DEV)
+    gpu = gpu_forward(wl, inp)
+    assert np.array_equal(gpu["counts"], np.full(E, k))
+    assert abs(float(gpu["aux"][0]) - k) <= 1e-5
+
+
+@pytest.mark.parametrize("N,E,k", [(1, 8, 2), (0, 8, 2), (37, 1, 1), (45, 4, 4), (129, 16, 1)])
+def test_edge_shapes(N, E, k):
+    wl = W.Workload("edge", N=N, d_model=64, d_ff=128, E=E, k=k, act="swiglu", router="softmax_topk",
+                    dtype="bf16", seed=11 + N)
+    inp = W.make_inputs(wl, DEV)
+    gpu = gpu_forward(wl, inp)
+    if N == 0:
+        assert gpu["counts"].sum() == 0 and float(gpu["aux"][0]) == 0.0
+        return
+    check_forward(wl, inp, gpu)
+
+
+def test_collapsed_routing_single_expert_gets_everything():
+    wl = W.Workload("collapse", N=300, d_model=64, d_ff=128, E=8, k=2, act="swiglu", router="softmax_topk",
+                    dtype="bf16", seed=21)
+    inp = W.make_inputs(wl, DEV)
+    Wg = torch.zeros((8, 64), device=DEV)
+    Wg[3, :] = 1.0
+    Wg[6, :] = 0.5
+    inp["x"] = inp["x"].abs()
+    inp["W_g"] = Wg.to(torch.bfloat16)
+    gpu = gpu_forward(wl, inp)
+    assert gpu["counts"][3] == 300 and gpu["counts"][6] == 300
+    check_forward(wl, inp, gpu)
