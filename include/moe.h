@@ -154,6 +154,37 @@ MOE_API moe_status moe_dispatch(const moe_config *cfg, const void *x,
                         int32_t *dev_status, void *ws, size_t ws_bytes,
                         moe_stream_t stream);
 
+/* Largest ceil(N / 32) * E that moe_dispatch_noalloc accepts (int32 slots of
+ * its built-in scratch, 2 MiB): e.g. N <= 65536 tokens with E = 256. */
+#define MOE_NOALLOC_DISPATCH_MAX_SLOTS (1 << 19)
+
+/*
+ * moe_dispatch without a workspace.  The pages have no counterpart of this
+ * entry point; it exists for callers that cannot hand the library any scratch
+ * memory: code that runs under a device-memory budget fixed before it starts
+ * (a serving process that plans every buffer up front, or a plugin called by
+ * a framework that owns the allocator) may not call cudaMalloc at all -- it
+ * would break the owner's accounting and can stall the whole device -- and
+ * has no spare buffer of moe_workspace_size bytes to pass in.
+ *
+ * Same arguments, outputs and errors as moe_dispatch, minus ws / ws_bytes.
+ * The per-chunk scratch lives in a device array inside libmoe.so
+ * (MOE_NOALLOC_DISPATCH_MAX_SLOTS int32, held by every GPU that loads the
+ * library until the process exits); a larger problem returns
+ * MOE_ERR_WORKSPACE and enqueues nothing.  Nothing is allocated, here or
+ * later.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it: make that
+ * first call before any stream capture.  Every call uses the same array, so
+ * calls whose work overlaps on the GPU (e.g. on two streams) race: order them.
+ * Each call overwrites all the scratch it later reads, so earlier contents
+ * never matter.
+ */
+MOE_API moe_status moe_dispatch_noalloc(const moe_config *cfg, const void *x,
+                                const int32_t *topk_ids, void *x_sorted,
+                                int32_t *perm, int32_t *inv_perm,
+                                int32_t *offsets, int32_t *counts,
+                                int32_t *dev_status, moe_stream_t stream);
+
 /*
  * Expert FFNs over the ragged slices: course module sec. 2.2 ("each expert
  * runs once on its slice"), experts as in moe_act.  Rows

@@ -32,7 +32,10 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
 NUM_STAGES = 5
 STAGE_NAMES = ("route", "dispatch", "gemm1", "gemm2", "combine")
 EXPORTS = ("moe_status_string", "moe_last_error", "moe_version", "moe_workspace_size", "moe_route",
-           "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_aux_loss", "moe_forward")
+           "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_combine", "moe_aux_loss",
+           "moe_forward")
+# ceil(N / 32) * E limit of moe_dispatch_noalloc (MOE_NOALLOC_DISPATCH_MAX_SLOTS)
+NOALLOC_DISPATCH_MAX_SLOTS = 1 << 19
 
 
 class MoeConfig(ctypes.Structure):
@@ -82,6 +85,8 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_route.restype = st
     lib.moe_dispatch.argtypes = [cfgp, vp, i32p, vp, i32p, i32p, i32p, i32p, i32p, vp, sz, vp]
     lib.moe_dispatch.restype = st
+    lib.moe_dispatch_noalloc.argtypes = [cfgp, vp, i32p, vp, i32p, i32p, i32p, i32p, i32p, vp]
+    lib.moe_dispatch_noalloc.restype = st
     lib.moe_expert_ffn.argtypes = [cfgp, vp, i32p, vp, vp, vp, vp, vp, vp, i32p, vp, sz, vp]
     lib.moe_expert_ffn.restype = st
     lib.moe_combine.argtypes = [cfgp, vp, f32p, i32p, vp, vp]
@@ -169,6 +174,32 @@ def moe_dispatch(cfg: MoeConfig, topk_ids: torch.Tensor, x: Optional[torch.Tenso
                                 _ptr(out["inv_perm"]), _ptr(out["offsets"]), _ptr(out["counts"]),
                                 _ptr(out["status"]), _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "moe_dispatch")
+    return out
+
+
+def moe_dispatch_noalloc(cfg: MoeConfig, topk_ids: torch.Tensor, x: Optional[torch.Tensor] = None,
+                         stream=None) -> Dict[str, torch.Tensor]:
+    """moe_dispatch for callers that cannot give the library a workspace.
+
+    The scratch is a fixed array inside libmoe.so (ceil(N/32) * E must not
+    exceed NOALLOC_DISPATCH_MAX_SLOTS); the library allocates nothing.  This
+    wrapper still creates the output tensors with torch; a caller without an
+    allocator passes its own buffers to the C entry point instead.
+    """
+    dev = topk_ids.device
+    A = cfg.N * cfg.k
+    out = {
+        "x_sorted": torch.empty((A, cfg.d_model), dtype=cfg.torch_dtype, device=dev) if x is not None else None,
+        "perm": torch.empty(A, dtype=torch.int32, device=dev),
+        "inv_perm": torch.empty(A, dtype=torch.int32, device=dev),
+        "offsets": torch.empty(cfg.E + 1, dtype=torch.int32, device=dev),
+        "counts": torch.empty(cfg.E, dtype=torch.int32, device=dev),
+        "status": torch.zeros(1, dtype=torch.int32, device=dev),
+    }
+    rc = library().moe_dispatch_noalloc(ctypes.byref(cfg), _ptr(x), _ptr(topk_ids), _ptr(out["x_sorted"]),
+                                        _ptr(out["perm"]), _ptr(out["inv_perm"]), _ptr(out["offsets"]),
+                                        _ptr(out["counts"]), _ptr(out["status"]), _stream(stream))
+    _check(rc, "moe_dispatch_noalloc")
     return out
 
 
