@@ -34,16 +34,19 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_BYTES = 126 * 1024 * 1024
 # tokens of the workload the CPU oracle handles per reference step (about 1-3 s each)
 REF_TOKENS_PER_STEP = {"tiny_fp32": 64, "gpt2_moe": 32, "mixtral": 1, "deepseek_v3": 1, "qwen3_skew": 8}
-KERNELS_PER_STEP = 7  # router, scan, scatter, gather, GEMM1, GEMM2, combine
+# libmoe kernels per forward: router logits + selection (bf16; one fused router
+# kernel for fp32), scan, scatter, gather, GEMM1, GEMM2, combine
+KERNELS_PER_STEP = {"bf16": 8, "f32": 7}
 
 
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--workload", default="mixtral")
     p.add_argument("--impl", default="native", choices=["native", "reference"])
+    p.add_argument("--tokens", type=int, default=0, help="override N (small profiling cases)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
 
@@ -60,6 +63,17 @@ def load_peaks():
 def dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), int(
         os.environ.get("WORLD_SIZE", "1"))
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest per-rank value (the job's time is its slowest rank's)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def weights_bytes(wl) -> int:
@@ -85,21 +99,24 @@ def traffic_for(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled every 50 ms, kept for the timed region."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, interval_ms: int = 50):
         self.gpu = gpu_index
+        self.interval_ms = interval_ms
         self.proc = None
         self.lines = []
+        self.window = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
-                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms",
+                 str(self.interval_ms), "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except OSError:
@@ -108,7 +125,11 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def mark(self, t0: float, t1: float):
+        """The timed region in time.monotonic() seconds; samples outside it are ignored."""
+        self.window = (t0, t1)
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -121,7 +142,12 @@ class ClockSampler:
     def summary(self):
         sm, smax, reasons = [], None, set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in self.lines:
+        lines = self.lines
+        if self.window is not None:
+            t0, t1 = self.window
+            inside = [(t, l) for t, l in lines if t0 <= t <= t1 + self.interval_ms / 1000.0]
+            lines = inside if inside else lines
+        for _, line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -270,16 +296,16 @@ def run_native(args, wl):
             dist.barrier()
         torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    assert int(out["status"][0]) == 0, f"device status {int(out['status'][0])}"
-
     stage_ev = [M.StageEvents() for _ in range(args.steps)]
     start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    barrier()
     with ClockSampler(local_rank) as clocks:
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        assert int(out["status"][0]) == 0, f"device status {int(out['status'][0])}"
+        barrier()
+        w0 = time.monotonic()
         t_all0 = torch.cuda.Event(enable_timing=True)
         t_all1 = torch.cuda.Event(enable_timing=True)
         t_all0.record(stream)
@@ -291,6 +317,7 @@ def run_native(args, wl):
             end[i].record(stream)
         t_all1.record(stream)
         barrier()
+        clocks.mark(w0, time.monotonic())
     if flush is None:
         local_ms = t_all0.elapsed_time(t_all1)
     else:
@@ -299,10 +326,7 @@ def run_native(args, wl):
     for ev in stage_ev:
         for k, v in ev.elapsed_ms().items():
             stages[k] += v / args.steps
-    t = torch.tensor([local_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(local_ms, world, dev)
 
     # end to end through the public call with host buffers: H2D of x, the
     # forward, D2H of y and of the loss, every step
@@ -330,10 +354,7 @@ def run_native(args, wl):
         e2e_step()
     e1.record(stream)
     barrier()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
 
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -361,7 +382,7 @@ def run_native(args, wl):
             "e2e": {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s",
                     "h2d_bytes_per_step": inp["x"].numel() * inp["x"].element_size(),
                     "d2h_bytes_per_step": out["y"].numel() * out["y"].element_size() + 4},
-            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "gpu_launches": KERNELS_PER_STEP[wl.dtype] * args.steps,
             "clocks": clocks.summary(),
         }
         if not args.no_cpu_baseline and world == 1:
@@ -380,6 +401,8 @@ def main():
     args = parse_args()
     import workloads as W
     wl = W.WORKLOADS[args.workload]
+    if args.tokens:
+        wl = wl.scaled(N=args.tokens)
     if args.impl == "reference":
         run_reference(args, wl)
     else:

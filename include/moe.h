@@ -132,11 +132,14 @@ MOE_API size_t moe_workspace_size(const moe_config *cfg);
  * selection score first (ties: lowest id), and their weights (times
  * routed_scaling).  b_e (sigmoid router only, may be NULL) enters the
  * selection score only, never the weights (sec. 2.5).  probs [N, E] (may be
- * NULL) receives softmax(z_n) for every router.  Needs no workspace.
+ * NULL) receives softmax(z_n) for every router.  The workspace holds the
+ * bf16 path's fp32 logits between its two kernels (tensor-core logits, then
+ * one warp per token for scores, top-k and gates).
  */
 MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const void *W_g,
                      const float *b_e, int32_t *topk_ids, float *topk_w,
-                     float *probs, moe_stream_t stream);
+                     float *probs, void *ws, size_t ws_bytes,
+                     moe_stream_t stream);
 
 /*
  * Sorted dispatch: course module sec. 2.2 and the sec. 4 dispatch.

@@ -81,7 +81,7 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_version.restype = ctypes.c_int32
     lib.moe_workspace_size.argtypes = [cfgp]
     lib.moe_workspace_size.restype = sz
-    lib.moe_route.argtypes = [cfgp, vp, vp, f32p, i32p, f32p, f32p, vp]
+    lib.moe_route.argtypes = [cfgp, vp, vp, f32p, i32p, f32p, f32p, vp, sz, vp]
     lib.moe_route.restype = st
     lib.moe_dispatch.argtypes = [cfgp, vp, i32p, vp, i32p, i32p, i32p, i32p, i32p, vp, sz, vp]
     lib.moe_dispatch.restype = st
@@ -144,14 +144,15 @@ def workspace(cfg: MoeConfig, device=None) -> torch.Tensor:
 
 
 def moe_route(cfg: MoeConfig, x: torch.Tensor, W_g: torch.Tensor, b_e: Optional[torch.Tensor] = None,
-              want_probs: bool = False, stream=None):
+              want_probs: bool = False, ws: Optional[torch.Tensor] = None, stream=None):
     """Returns (topk_ids [N,k] int32, topk_w [N,k] f32, probs [N,E] f32 or None)."""
     dev = x.device
+    ws = ws if ws is not None else workspace(cfg, dev)
     ids = torch.empty((cfg.N, cfg.k), dtype=torch.int32, device=dev)
     w = torch.empty((cfg.N, cfg.k), dtype=torch.float32, device=dev)
     probs = torch.empty((cfg.N, cfg.E), dtype=torch.float32, device=dev) if want_probs else None
     rc = library().moe_route(ctypes.byref(cfg), _ptr(x), _ptr(W_g), _ptr(b_e), _ptr(ids), _ptr(w), _ptr(probs),
-                             _stream(stream))
+                             _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "moe_route")
     return ids, w, probs
 

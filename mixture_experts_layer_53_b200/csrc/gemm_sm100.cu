@@ -336,9 +336,11 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
+}  // namespace
+
 // bf16 matrix [outer, inner] (inner contiguous), box [box_outer, 64],
 // 128-byte swizzle, zero fill outside the matrix.
-bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_outer)
+bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_outer)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -350,6 +352,8 @@ bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <int EPI>
 cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b3, const GemmArgs &g,
@@ -374,10 +378,10 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid
     const uint64_t rows = static_cast<uint64_t>(a.rows);
     const uint64_t E = static_cast<uint64_t>(a.E);
     CUtensorMap tA, tB, tB3, tH, tW2;
-    if (!make_tmap(&tA, a.x_sorted, a.d, rows, BM) ||
-        !make_tmap(&tB, a.W1, a.d, E * a.F, swiglu ? 128 : 256) ||
-        !make_tmap(&tB3, swiglu ? a.W3 : a.W1, a.d, E * a.F, swiglu ? 128 : 256) ||
-        !make_tmap(&tH, a.h, a.F, rows, BM) || !make_tmap(&tW2, a.W2, a.F, E * a.d, 256))
+    if (!make_tmap_bf16(&tA, a.x_sorted, a.d, rows, BM) ||
+        !make_tmap_bf16(&tB, a.W1, a.d, E * a.F, swiglu ? 128 : 256) ||
+        !make_tmap_bf16(&tB3, swiglu ? a.W3 : a.W1, a.d, E * a.F, swiglu ? 128 : 256) ||
+        !make_tmap_bf16(&tH, a.h, a.F, rows, BM) || !make_tmap_bf16(&tW2, a.W2, a.F, E * a.d, 256))
         return cudaErrorInvalidValue;
 
     GemmArgs g1{};

@@ -26,7 +26,28 @@ struct RouterArgs {
     int d, E, k, router, norm_topk;
     float scaling;
 };
+// CUDA-core router (fp32 path).
 cudaError_t launch_router(int dtype, const RouterArgs &a, cudaStream_t s);
+// tcgen05 router logits (bf16 path): logits [N, logits_ld(E)] fp32;
+// `status` receives device wait timeouts.
+int logits_ld(int E);
+cudaError_t launch_router_logits_sm100(const void *x, const void *W_g, float *logits, int64_t N, int d, int E,
+                                       int32_t *status, cudaStream_t s);
+
+// Scores, top-k, gates and per-chunk statistics from fp32 logits.
+struct SelectKernelArgs {
+    const float *logits;  // [N, ld]
+    const float *b_sel;   // [E] or null (sigmoid router only)
+    int32_t *ids;
+    float *w;
+    float *probs;         // [N, E] or null
+    int32_t *hist;        // [chunks, E] or null
+    float *psum;          // [chunks, E] or null
+    int64_t N;
+    int ld, E, k, router, norm_topk;
+    float scaling;
+};
+cudaError_t launch_select(const SelectKernelArgs &a, cudaStream_t s);
 
 // Per-chunk histograms of expert ids (with range check) and, optionally,
 // per-chunk sums of probs.
@@ -100,6 +121,16 @@ struct FfnArgs {
     int64_t rows;              // N k
     int d, F, E, act;
 };
+}  // namespace moe
+
+#include <cuda.h>
+
+namespace moe {
+
+// TMA descriptor of a bf16 matrix [outer, inner] (inner contiguous) with a
+// box of [box_outer, 64] elements, 128-byte swizzle, zero fill outside.
+bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_outer);
+
 // Both expert GEMMs; `mid` (may be null) is recorded between them.
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid, cudaStream_t s);
 cudaError_t launch_ffn_f32_simt(const FfnArgs &a, int num_sms, cudaEvent_t mid, cudaStream_t s);

@@ -60,7 +60,7 @@ moe_status validate(const moe_config *c)
 }
 
 struct Layout {
-    size_t hist, psum, offsets, mt, counts, ids, w, perm, inv, xs, h, ys, total;
+    size_t hist, psum, logits, offsets, mt, counts, ids, w, perm, inv, xs, h, ys, total;
 };
 
 size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
@@ -79,6 +79,7 @@ Layout layout(const moe_config *c)
     const size_t A = static_cast<size_t>(c->N) * static_cast<size_t>(c->k);
     const size_t es = elem_size(c);
     L.hist = take(C * E * 4);
+    L.logits = take(static_cast<size_t>(c->N) * static_cast<size_t>(logits_ld(c->E)) * 4);
     L.psum = take(C * E * 4);
     L.offsets = take((E + 1) * 4);
     L.mt = take((E + 1) * 4);
@@ -161,6 +162,18 @@ moe_status check_ffn_ptrs(const moe_config *c, const void *W1, const void *b1, c
     return MOE_OK;
 }
 
+// bf16 routes on the tensor cores; fp32 keeps the CUDA-core router (tf32
+// products would not meet the fp32 tolerance).
+cudaError_t launch_route(const moe_config *c, const RouterArgs &r, int32_t *status, float *logits, cudaStream_t s)
+{
+    if (c->dtype != MOE_BF16) return launch_router(c->dtype, r, s);
+    cudaError_t err = launch_router_logits_sm100(r.x, r.Wg, logits, r.N, r.d, r.E, status, s);
+    if (err != cudaSuccess) return err;
+    SelectKernelArgs sk{logits, r.b_sel, r.ids, r.w, r.probs, r.hist, r.psum, r.N, logits_ld(r.E), r.E, r.k,
+                        r.router, r.norm_topk, r.scaling};
+    return launch_select(sk, s);
+}
+
 cudaError_t launch_ffn(const moe_config *c, const FfnArgs &f, cudaEvent_t mid, cudaStream_t s)
 {
     return c->dtype == MOE_BF16 ? launch_ffn_bf16_sm100(f, num_sms(), mid, s)
@@ -196,7 +209,7 @@ size_t moe_workspace_size(const moe_config *cfg)
 }
 
 moe_status moe_route(const moe_config *cfg, const void *x, const void *W_g, const float *b_e, int32_t *topk_ids,
-                     float *topk_w, float *probs, moe_stream_t stream)
+                     float *topk_w, float *probs, void *ws, size_t ws_bytes, moe_stream_t stream)
 {
     moe_status st = validate(cfg);
     if (st != MOE_OK) return st;
@@ -204,10 +217,11 @@ moe_status moe_route(const moe_config *cfg, const void *x, const void *W_g, cons
     if (!W_g || (!empty && (!x || !topk_ids || !topk_w))) return MOE_ERR_INVALID_ARG;
     if (b_e && cfg->router != MOE_ROUTER_SIGMOID) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(W_g)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
     if (cfg->N == 0) return MOE_OK;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const RouterArgs r = router_args(cfg, x, W_g, b_e, topk_ids, topk_w, probs, nullptr, nullptr);
-    cudaError_t err = launch_router(cfg->dtype, r, s);
+    cudaError_t err = launch_route(cfg, r, nullptr, at<float>(ws, layout(cfg).logits), s);
     return err == cudaSuccess ? MOE_OK : cuda_fail(err);
 }
 
@@ -350,7 +364,7 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const void *W_g, fl
         return cuda_fail(err);
     // route: logits, scores, top-k, gates, per-chunk histograms and P sums
     const RouterArgs r = router_args(cfg, x, W_g, b_e_inout, ids, w, nullptr, hist, psum);
-    if (cfg->N > 0 && (err = launch_router(cfg->dtype, r, s)) != cudaSuccess) return cuda_fail(err);
+    if (cfg->N > 0 && (err = launch_route(cfg, r, dev_status, at<float>(ws, L.logits), s)) != cudaSuccess) return cuda_fail(err);
     if ((err = mark(1)) != cudaSuccess) return cuda_fail(err);
     // dispatch: counts, offsets, tile table, Switch loss, bias step; scatter; gather
     ScanArgs sc{};

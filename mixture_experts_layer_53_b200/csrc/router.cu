@@ -20,6 +20,7 @@
 #include "common.cuh"
 #include "host_util.h"
 #include "kernels.h"
+#include "router_select.cuh"
 
 namespace moe {
 namespace {
@@ -47,12 +48,6 @@ template <> struct Load4<__nv_bfloat16> {
         f[3] = __uint_as_float(v.y & 0xFFFF0000u);
     }
 };
-
-// (value desc, id asc): does candidate (v, e) rank ahead of (bv, be)?
-__device__ __forceinline__ bool ahead(float v, int e, float bv, int be)
-{
-    return v > bv || (v == bv && e < be);
-}
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a)
@@ -114,97 +109,22 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a)
     }
 
     // ---- scores, top-k and gates, one token at a time per warp
+    SelectArgs sa{a.b_sel, a.ids, a.w, a.probs, E, k, a.router, a.norm_topk, a.scaling};
 #pragma unroll 1
     for (int i = 0; i < 4; ++i) {
         const int t = warp + 8 * i;
         if (t >= ntok) break;  // warp-uniform
-        const int64_t n = tok0 + t;
-
-        float zmax = -FLT_MAX;
+        float z[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (j < EJ && lane + 32 * j < E) zmax = fmaxf(zmax, acc[i][j]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
-
-        float ex[8], sel[8], graw[8];
-        float esum = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = lane + 32 * j;
-            ex[j] = 0.f; sel[j] = -FLT_MAX; graw[j] = 0.f;
-            if (j < EJ && e < E) {
-                ex[j] = expf(acc[i][j] - zmax);
-                esum += ex[j];
-                if (a.router == kSigmoid) {
-                    const float sg = 1.0f / (1.0f + expf(-acc[i][j]));
-                    sel[j] = sg + (a.b_sel ? a.b_sel[e] : 0.f);
-                    graw[j] = sg;
-                } else {
-                    sel[j] = acc[i][j];
-                    graw[j] = ex[j];
-                }
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) esum += __shfl_xor_sync(0xffffffffu, esum, o);
-        const float inv_esum = 1.0f / esum;
-
-        uint32_t taken = 0;
-        int idsel[kMaxK];
-        float gsel[kMaxK];
-#pragma unroll
-        for (int r = 0; r < kMaxK; ++r) {
-            idsel[r] = 0;
-            gsel[r] = 0.f;
-            if (r < k) {
-                float bv = -FLT_MAX, bg = 0.f;
-                int be = INT_MAX;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int e = lane + 32 * j;
-                    if (j < EJ && e < E && !((taken >> j) & 1u) && ahead(sel[j], e, bv, be)) {
-                        bv = sel[j]; be = e; bg = graw[j];
-                    }
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                    const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                    const float og = __shfl_xor_sync(0xffffffffu, bg, o);
-                    if (ahead(ov, oe, bv, be)) { bv = ov; be = oe; bg = og; }
-                }
-                if ((be & 31) == lane) taken |= 1u << (be >> 5);
-                idsel[r] = be;
-                gsel[r] = bg;
-            }
-        }
-
-        float gs = 0.f;
+        for (int j = 0; j < 8; ++j) z[j] = acc[i][j];
+        int sel_ids[kMaxK];
+        select_token(z, sa, tok0 + t, true, sel_ids);
 #pragma unroll
         for (int r = 0; r < kMaxK; ++r)
-            if (r < k) gs += gsel[r];
+            if (r < k && lane == r) ids_s[t * k + r] = sel_ids[r];
 #pragma unroll
-        for (int r = 0; r < kMaxK; ++r) {
-            if (r < k && lane == r) {
-                float wr;
-                if (a.router == kSoftmaxTopk) wr = a.norm_topk ? gsel[r] / gs : gsel[r] * inv_esum;
-                else if (a.router == kTopkSoftmax) wr = gsel[r] / gs;
-                else wr = a.norm_topk ? gsel[r] / gs : gsel[r];
-                a.ids[n * k + r] = idsel[r];
-                a.w[n * k + r] = wr * a.scaling;
-                ids_s[t * k + r] = idsel[r];
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = lane + 32 * j;
-            if (j < EJ && e < E) {
-                const float p = ex[j] * inv_esum;
-                zt[t * ZS + e] = p;
-                if (a.probs) a.probs[n * E + e] = p;
-            }
-        }
+        for (int j = 0; j < 8; ++j)
+            if (j < EJ && lane + 32 * j < E) zt[t * ZS + lane + 32 * j] = z[j];
     }
     __syncthreads();
 
@@ -221,6 +141,57 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a)
                 for (int q = 0; q < ntok * k; ++q) c += (ids_s[q] == e);
                 a.hist[static_cast<int64_t>(blockIdx.x) * E + e] = c;
             }
+        }
+    }
+}
+
+// Scores, top-k and gates from precomputed fp32 logits (the tcgen05 router
+// of the bf16 path writes them).  One CTA per 32-token dispatch chunk, one
+// warp per token (16 warps, 2 tokens each): thousands of independent warps
+// hide the shuffle latency of the selection, which is a serial chain per
+// token.  Also writes the chunk's expert histogram and sum of p.
+constexpr int kSelWarps = 16;
+
+__global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs a)
+{
+    extern __shared__ float smem[];
+    const int E = a.E, k = a.k;
+    const int ZS = E + 1;
+    const int EJ = (E + 31) >> 5;
+    float *pt = smem;                                     // [32][E+1] p
+    int *ids_s = reinterpret_cast<int *>(pt + kRT * ZS);  // [32][k]
+    const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kRT;
+    const int ntok = static_cast<int>(min64(kRT, a.N - tok0));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    SelectArgs sa{a.b_sel, a.ids, a.w, a.probs, E, k, a.router, a.norm_topk, a.scaling};
+    for (int t = warp; t < ntok; t += kSelWarps) {
+        const int64_t n = tok0 + t;
+        float z[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane + 32 * j;
+            z[j] = (j < EJ && e < E) ? a.logits[n * a.ld + e] : 0.f;
+        }
+        int sel_ids[kMaxK];
+        select_token(z, sa, n, true, sel_ids);
+#pragma unroll
+        for (int r = 0; r < kMaxK; ++r)
+            if (r < k && lane == r) ids_s[t * k + r] = sel_ids[r];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < EJ && lane + 32 * j < E) pt[t * ZS + lane + 32 * j] = z[j];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kSelWarps * 32) {
+        if (a.psum) {
+            float s = 0.f;
+            for (int t = 0; t < ntok; ++t) s += pt[t * ZS + e];
+            a.psum[static_cast<int64_t>(blockIdx.x) * E + e] = s;
+        }
+        if (a.hist) {
+            int c = 0;
+            for (int q = 0; q < ntok * k; ++q) c += (ids_s[q] == e);
+            a.hist[static_cast<int64_t>(blockIdx.x) * E + e] = c;
         }
     }
 }
@@ -244,6 +215,15 @@ template <typename T> cudaError_t launch_router_t(const RouterArgs &a, cudaStrea
 }
 
 }  // namespace
+
+cudaError_t launch_select(const SelectKernelArgs &a, cudaStream_t s)
+{
+    const int64_t grid = num_chunks(a.N);
+    if (grid == 0) return cudaSuccess;
+    const size_t smem = sizeof(float) * kRT * (a.E + 1) + sizeof(int) * kRT * a.k;
+    select_kernel<<<static_cast<unsigned>(grid), kSelWarps * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_router(int dtype, const RouterArgs &a, cudaStream_t s)
 {

@@ -1,0 +1,138 @@
+// router_select.cuh -- scores, top-k and gates of one token, computed by one
+// warp with the token's E logits spread over the lanes (lane l holds experts
+// l, l+32, ...).  Shared by the CUDA-core router and the tcgen05 router.
+//
+// Course module "Mixture of Experts: routing, sorted dispatch, Switch aux
+// loss, aux-free bias": sec. 2 symbol table (p_n = softmax(z_n)), sec. 2.1
+// router table (softmax_topk / topk_softmax / sigmoid, ties to the lowest id,
+// routed_scaling), sec. 2.5 (b_e enters the selection score only).
+// Selection for the softmax routers compares logits: softmax is increasing,
+// so the chosen set and slot order are those of p, without exp rounding.
+#pragma once
+
+#include <float.h>
+#include <limits.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+struct SelectArgs {
+    const float *b_sel;  // [E] or null
+    int32_t *ids;        // [N, k]
+    float *w;            // [N, k]
+    float *probs;        // [N, E] or null
+    int E, k, router, norm_topk;
+    float scaling;
+};
+
+// (value desc, id asc): does (v, e) rank ahead of (bv, be)?
+__device__ __forceinline__ bool rank_ahead(float v, int e, float bv, int be)
+{
+    return v > bv || (v == bv && e < be);
+}
+
+// z[j] = logit of expert lane + 32 j (j < ceil(E/32) <= 8).  Writes the
+// token's ids / weights / probs rows (if `write`), returns p in z[] and the
+// chosen ids in sel_ids[0..k) (valid in every lane).
+__device__ __forceinline__ void select_token(float (&z)[8], const SelectArgs &a, int64_t n, bool write,
+                                             int (&sel_ids)[kMaxK])
+{
+    const int lane = threadIdx.x & 31;
+    const int E = a.E, k = a.k;
+    const int EJ = (E + 31) >> 5;
+    float zmax = -FLT_MAX;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (j < EJ && lane + 32 * j < E) zmax = fmaxf(zmax, z[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
+
+    float ex[8], sel[8], graw[8];
+    float esum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int e = lane + 32 * j;
+        ex[j] = 0.f;
+        sel[j] = -FLT_MAX;
+        graw[j] = 0.f;
+        if (j < EJ && e < E) {
+            ex[j] = expf(z[j] - zmax);
+            esum += ex[j];
+            if (a.router == kSigmoid) {
+                const float sg = 1.0f / (1.0f + expf(-z[j]));
+                sel[j] = sg + (a.b_sel ? a.b_sel[e] : 0.f);
+                graw[j] = sg;
+            } else {
+                sel[j] = z[j];
+                graw[j] = ex[j];
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) esum += __shfl_xor_sync(0xffffffffu, esum, o);
+    const float inv_esum = 1.0f / esum;
+
+    // k rounds of a warp argmax under the (score desc, id asc) order
+    uint32_t taken = 0;
+    float gsel[kMaxK];
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) {
+        sel_ids[r] = 0;
+        gsel[r] = 0.f;
+        if (r < k) {
+            float bv = -FLT_MAX, bg = 0.f;
+            int be = INT_MAX;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int e = lane + 32 * j;
+                if (j < EJ && e < E && !((taken >> j) & 1u) && rank_ahead(sel[j], e, bv, be)) {
+                    bv = sel[j];
+                    be = e;
+                    bg = graw[j];
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                const float og = __shfl_xor_sync(0xffffffffu, bg, o);
+                if (rank_ahead(ov, oe, bv, be)) {
+                    bv = ov;
+                    be = oe;
+                    bg = og;
+                }
+            }
+            if ((be & 31) == lane) taken |= 1u << (be >> 5);
+            sel_ids[r] = be;
+            gsel[r] = bg;
+        }
+    }
+
+    float gs = 0.f;
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r)
+        if (r < k) gs += gsel[r];
+    if (write) {
+#pragma unroll
+        for (int r = 0; r < kMaxK; ++r) {
+            if (r < k && lane == r) {
+                float wr;
+                if (a.router == kSoftmaxTopk) wr = a.norm_topk ? gsel[r] / gs : gsel[r] * inv_esum;
+                else if (a.router == kTopkSoftmax) wr = gsel[r] / gs;
+                else wr = a.norm_topk ? gsel[r] / gs : gsel[r];
+                a.ids[n * k + r] = sel_ids[r];
+                a.w[n * k + r] = wr * a.scaling;
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int e = lane + 32 * j;
+        z[j] = (j < EJ && e < E) ? ex[j] * inv_esum : 0.f;
+        if (write && a.probs && j < EJ && e < E) a.probs[n * E + e] = z[j];
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,235 @@
+// router_sm100.cu -- router logits z = x W_g^T on the Blackwell tensor cores
+// (bf16 inputs, fp32 accumulation), for the bf16 path.
+//
+// Course module "Mixture of Experts: routing, sorted dispatch, Switch aux
+// loss, aux-free bias", sec. 2 symbol table: z_n = W_g x_n.  The scores,
+// top-k and gates follow in select_kernel (router.cu), which spreads the
+// tokens over every SM, one warp per token.
+//
+// The product is [N, d] x [d, E] with small E, so the kernel is bound by
+// reading x.  One CTA takes a tile of 128 tokens:
+//   warp 0      TMA: x tile (128 x 64) and W_g tile (E_pad x 64) per k-block
+//               into a shared-memory ring (up to 8 stages)
+//   warp 1      allocates TMEM, one lane issues tcgen05.mma M=128, N=E_pad
+//               (E rounded up to 16; the W_g rows past E are TMA zero fill)
+//   warps 2-5   one thread per token row: tcgen05.ld, fp32 stores of the row
+// k-blocks are spread round-robin over several TMEM accumulators, which the
+// epilogue then adds in fp32 round-to-nearest: the tensor core's own running
+// sums are only num_kb / nacc steps deep, which keeps the logits close enough
+// to an fp32 dot product for the 1e-5 tolerance of the Switch loss.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "host_util.h"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int MAX_STAGES = 8;
+constexpr int THREADS = 192;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int SMEM_TILE_BUDGET = 196608;
+
+struct Ctl {
+    uint64_t full[MAX_STAGES];
+    uint64_t empty[MAX_STAGES];
+    uint64_t tfull;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct LArgs {
+    float *logits;  // [N, ld]
+    int32_t *status;
+    int64_t N;
+    int d, E, E_pad, ld, stages;
+    int nacc;            // TMEM accumulators, k-block kb -> kb % nacc
+    uint32_t acc_cols;   // TMEM columns per accumulator (power of 2 >= E_pad)
+    uint32_t tmem_cols;  // nacc * acc_cols
+};
+
+__global__ void __launch_bounds__(THREADS, 1)
+    router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                         const LArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                 ~static_cast<uintptr_t>(1023));
+    const int stage_bytes = A_BYTES + a.E_pad * BK * 2;
+    Ctl *ctl = reinterpret_cast<Ctl *>(tiles + a.stages * stage_bytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int *abort_flag = &ctl->abort;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < a.stages; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        mbar_init(&ctl->tfull, 1);
+        mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    if (threadIdx.x == 32) {
+        prefetch_tmap(&tmX);
+        prefetch_tmap(&tmW);
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_base, a.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem_base = ctl->tmem_base;
+    const int num_kb = (a.d + BK - 1) / BK;
+    const int row0 = blockIdx.x * BM;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------- TMA producer
+            int stage = 0;
+            uint32_t phase = 0, armed = 0, armed_parity = 0;
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort_flag, a.status)) break;
+                uint8_t *sA = tiles + stage * stage_bytes;
+                mbar_arrive_expect_tx(&ctl->full[stage], static_cast<uint32_t>(stage_bytes));
+                armed |= 1u << stage;
+                armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                tma_load_2d(sA, &tmX, &ctl->full[stage], kb * BK, row0);
+                tma_load_2d(sA + A_BYTES, &tmW, &ctl->full[stage], kb * BK, 0);
+                if (++stage == a.stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (*abort_flag) {
+                for (int s = 0; s < a.stages; ++s)
+                    if ((armed >> s) & 1u)
+                        mbar_wait(&ctl->full[s], (armed_parity >> s) & 1u, abort_flag, a.status, false);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------------ MMA issuer
+            const uint32_t idesc = idesc_bf16_f32(BM, a.E_pad);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true, issued = false;
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!mbar_wait(&ctl->full[stage], phase, abort_flag, a.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(tiles + stage * stage_bytes);
+                const uint32_t b_addr = a_addr + A_BYTES;
+                // k-block kb accumulates into accumulator kb % nacc; the first
+                // k-block of each accumulator overwrites it
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(kb % a.nacc) * a.acc_cols;
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    umma_bf16(d_tmem, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32), idesc,
+                              (kb >= a.nacc || kk != 0) ? 1u : 0u);
+                issued = true;
+                umma_commit(&ctl->empty[stage]);
+                if (++stage == a.stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (ok && issued) umma_commit(&ctl->tfull);
+            if (*abort_flag && issued) {
+                umma_commit(&ctl->drain);
+                mbar_wait(&ctl->drain, 0, abort_flag, a.status, false);
+            }
+        }
+    } else {
+        // -------------------------------------------------------- epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int64_t n = static_cast<int64_t>(row0) + q * 32 + lane;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&ctl->tfull, 0, abort_flag, a.status));
+        if (ok && num_kb > 0) {
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+            const int used = min(a.nacc, num_kb);
+            float *zrow = a.logits + n * a.ld;
+            for (int c0 = 0; c0 < a.E_pad; c0 += 32) {
+                uint32_t r[32], t[32];
+                tmem_ld32(taddr + c0, r);
+                tmem_ld_wait();
+                for (int s = 1; s < used; ++s) {
+                    tmem_ld32(taddr + static_cast<uint32_t>(s) * a.acc_cols + c0, t);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        r[u] = __float_as_uint(__uint_as_float(r[u]) + __uint_as_float(t[u]));
+                }
+                if (n < a.N) {
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        const int c = c0 + 4 * v;
+                        if (c < a.ld)  // ld is a multiple of 4
+                            st16(zrow + c, make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]));
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, a.tmem_cols);
+    }
+}
+
+}  // namespace
+
+int logits_ld(int E) { return (E + 3) / 4 * 4; }
+
+cudaError_t launch_router_logits_sm100(const void *x, const void *W_g, float *logits, int64_t N, int d, int E,
+                                       int32_t *status, cudaStream_t s)
+{
+    if (N == 0) return cudaSuccess;
+    LArgs a{};
+    a.logits = logits;
+    a.status = status;
+    a.N = N;
+    a.d = d;
+    a.E = E;
+    a.E_pad = ((E + 15) / 16) * 16;
+    a.ld = logits_ld(E);
+    uint32_t cols = 32;
+    while (cols < static_cast<uint32_t>(a.E_pad)) cols <<= 1;
+    a.acc_cols = cols;
+    a.nacc = static_cast<int>(512 / cols);
+    if (a.nacc > 8) a.nacc = 8;
+    a.tmem_cols = cols * static_cast<uint32_t>(a.nacc);
+    const int stage_bytes = A_BYTES + a.E_pad * BK * 2;
+    a.stages = SMEM_TILE_BUDGET / stage_bytes;
+    if (a.stages > MAX_STAGES) a.stages = MAX_STAGES;
+
+    CUtensorMap tX, tW;
+    if (!make_tmap_bf16(&tX, x, d, static_cast<uint64_t>(N), BM) ||
+        !make_tmap_bf16(&tW, W_g, d, static_cast<uint64_t>(E), static_cast<uint32_t>(a.E_pad)))
+        return cudaErrorInvalidValue;
+    const size_t smem = 1024 + static_cast<size_t>(a.stages) * stage_bytes + sizeof(Ctl);
+    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&router_logits_kernel),
+                                       1024 + SMEM_TILE_BUDGET + static_cast<int>(sizeof(Ctl)));
+    if (err != cudaSuccess) return err;
+    const int64_t grid = (N + BM - 1) / BM;
+    router_logits_kernel<<<static_cast<unsigned>(grid), THREADS, smem, s>>>(tX, tW, a);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

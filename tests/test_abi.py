@@ -83,7 +83,7 @@ def cfg(**kw):
 def test_invalid_configs(lib, bad, code):
     c = cfg(**bad)
     assert lib.moe_workspace_size(ctypes.byref(c)) == 0
-    rc = lib.moe_route(ctypes.byref(c), BAD, BAD, None, BAD, BAD, None, None)
+    rc = lib.moe_route(ctypes.byref(c), BAD, BAD, None, BAD, BAD, None, None, 0, None)
     assert rc == code
 
 
@@ -100,17 +100,17 @@ def test_invalid_enums(lib):
 
 def test_null_and_misaligned_pointers(lib):
     c = cfg()
-    assert lib.moe_route(ctypes.byref(c), None, BAD, None, BAD, BAD, None, None) == 1
+    assert lib.moe_route(ctypes.byref(c), None, BAD, None, BAD, BAD, None, None, 0, None) == 1
     assert lib.moe_route(ctypes.byref(c), ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2008), None,
-                         ctypes.c_void_p(0x3000), ctypes.c_void_p(0x4000), None, None) == 1
+                         ctypes.c_void_p(0x3000), ctypes.c_void_p(0x4000), None, None, 0, None) == 1
     assert lib.moe_combine(ctypes.byref(c), None, BAD, BAD, BAD, None) == 1
-    assert lib.moe_route(None, BAD, BAD, None, BAD, BAD, None, None) == 1
+    assert lib.moe_route(None, BAD, BAD, None, BAD, BAD, None, None, 0, None) == 1
 
 
 def test_bias_only_for_sigmoid_router(lib):
     c = cfg()
     a = ctypes.c_void_p(0x10000)
-    assert lib.moe_route(ctypes.byref(c), a, a, a, a, a, None, None) == 1
+    assert lib.moe_route(ctypes.byref(c), a, a, a, a, a, None, None, 0, None) == 1
     rc = lib.moe_forward(ctypes.byref(c), a, a, a, ctypes.c_float(0.0), a, a, None, a, a, a, None, None, None,
                          None, None, a, ctypes.c_size_t(1 << 40), None, None)
     assert rc == 1
