@@ -13,8 +13,6 @@ enum : int32_t { kDevOk = 0, kDevTimeout = 5, kDevBadExpertId = 6 };
 // Tokens handled by one router CTA; also the dispatch chunk (chunk c holds
 // tokens [c*kChunkTokens, (c+1)*kChunkTokens) and their assignments).
 constexpr int kChunkTokens = 32;
-// Rows of one expert-GEMM M-tile; the tile table counts ceil(rows / kTileM).
-constexpr int kTileM = 128;
 constexpr int kMaxE = 256;
 constexpr int kMaxK = 16;
 

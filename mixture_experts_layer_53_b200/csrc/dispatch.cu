@@ -54,92 +54,103 @@ __global__ void __launch_bounds__(256) hist_kernel(HistArgs a)
 
 // ------------------------------------------------------------------- scan
 
-constexpr int kScanThreads = 1024;
+constexpr int kScanThreads = 256;
 
-__global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a)
+// Exclusive prefix of v over the block (kScanThreads threads, fixed order).
+__device__ __forceinline__ int block_exclusive_scan(int v, int *total)
 {
-    __shared__ int part[kScanThreads];       // [seg][e]
-    __shared__ int segbase[kScanThreads];    // [seg][e]
-    __shared__ double ppart[kScanThreads];   // [seg][e]
-    __shared__ int off_s[kMaxE + 1];
+    __shared__ int warp_sums[kScanThreads / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int base = 0, tot = 0;
+    for (int w = 0; w < kScanThreads / 32; ++w) {
+        if (w < warp) base += warp_sums[w];
+        tot += warp_sums[w];
+    }
+    __syncthreads();
+    *total = tot;
+    return base + incl - v;
+}
+
+// One CTA per expert e: the chunk bases inside e's slice (prefix over chunks
+// of hist[c][e], in place), count_e (into offsets[e+1]) and, if psum is given,
+// P_e * N = sum over chunks of psum[c][e] in fp64 (fixed tree order).
+__global__ void __launch_bounds__(kScanThreads) scan_cols_kernel(ScanArgs a)
+{
+    const int e = blockIdx.x, E = a.E;
+    const int64_t C = a.chunks;
+    const int64_t per = (C + kScanThreads - 1) / kScanThreads;
+    const int64_t c0 = min64(C, threadIdx.x * per), c1 = min64(C, c0 + per);
+    int s = 0;
+    double p = 0.0;
+    for (int64_t c = c0; c < c1; ++c) {
+        s += a.hist[c * E + e];
+        if (a.psum) p += static_cast<double>(a.psum[c * E + e]);
+    }
+    int total;
+    int run = block_exclusive_scan(s, &total);
+    for (int64_t c = c0; c < c1; ++c) {
+        const int v = a.hist[c * E + e];
+        a.hist[c * E + e] = run;
+        run += v;
+    }
+    if (a.psum && a.pe) {
+        __shared__ double wsum[kScanThreads / 32];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+        if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = p;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double P = 0.0;
+            for (int w = 0; w < kScanThreads / 32; ++w) P += wsum[w];
+            a.pe[e] = P;
+        }
+    }
+    if (threadIdx.x == 0) a.offsets[e + 1] = total;
+}
+
+// One CTA (E <= 256 threads' worth): offsets = exclusive prefix of counts,
+// the GEMM tile table, the Switch loss L = E sum_e (count_e/N)(P_e/N) in fp64
+// (course module sec. 2.3) and the sign-rule step b_e += gamma *
+// sign(N k - E count_e) (sec. 2.5).
+__global__ void __launch_bounds__(kScanThreads) scan_finalize_kernel(ScanArgs a)
+{
     __shared__ int cnt_s[kMaxE];
-    __shared__ double P_s[kMaxE];
-
-    const int E = a.E;
-    const int nseg = kScanThreads / E;  // >= 4 because E <= 256
-    const int64_t seglen = (a.chunks + nseg - 1) / nseg;
-    const int tid = threadIdx.x;
-    const int e = tid % E, s = tid / E;
-    const bool active = s < nseg;
-    const int64_t c_begin = active ? min64(a.chunks, s * seglen) : 0;
-    const int64_t c_end = active ? min64(a.chunks, (s + 1) * seglen) : 0;
-
-    if (active) {
-        int sum = 0;
-        double psum = 0.0;
-        for (int64_t c = c_begin; c < c_end; ++c) {
-            sum += a.hist[c * E + e];
-            if (a.psum) psum += static_cast<double>(a.psum[c * E + e]);
-        }
-        part[s * E + e] = sum;
-        ppart[s * E + e] = psum;
-    }
-    __syncthreads();
-    if (tid < E) {
-        int run = 0;
-        double P = 0.0;
-        for (int q = 0; q < nseg; ++q) {
-            segbase[q * E + tid] = run;
-            run += part[q * E + tid];
-            P += ppart[q * E + tid];
-        }
-        cnt_s[tid] = run;
-        P_s[tid] = P;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        int run = 0;
-        for (int q = 0; q < E; ++q) {
-            off_s[q] = run;
-            run += cnt_s[q];
-        }
-        off_s[E] = run;
-        if (a.mt_prefix) {
-            int mt = 0;
-            a.mt_prefix[0] = 0;
-            for (int q = 0; q < E; ++q) {
-                mt += (cnt_s[q] + kTileM - 1) / kTileM;
-                a.mt_prefix[q + 1] = mt;
-            }
-        }
-        if (a.aux_out && a.psum && a.N == 0) {
-            *a.aux_out = 0.0f;  // no tokens: every sum is empty
-        } else if (a.aux_out && a.psum) {
-            // L = E * sum_e (count_e / N) * (P_e / N), in fp64 (sec. 2.3)
-            const double Nd = static_cast<double>(a.N);
-            double L = 0.0;
-            for (int q = 0; q < E; ++q)
-                L += (static_cast<double>(cnt_s[q]) / Nd) * (P_s[q] / Nd);
-            *a.aux_out = static_cast<float>(L * static_cast<double>(E));
-        }
-    }
-    __syncthreads();
-    for (int q = tid; q <= E; q += kScanThreads) a.offsets[q] = off_s[q];
-    if (tid < E) {
-        if (a.counts) a.counts[tid] = cnt_s[tid];
+    const int E = a.E, t = threadIdx.x;
+    const int cnt = t < E ? a.offsets[t + 1] : 0;
+    if (t < E) cnt_s[t] = cnt;
+    int total, mt_total;
+    const int off = block_exclusive_scan(cnt, &total);
+    const int mt = (t < E && a.mt_prefix) ? (cnt + a.tile_m - 1) / a.tile_m : 0;
+    const int mt_off = block_exclusive_scan(mt, &mt_total);
+    if (t < E) {
+        a.offsets[t] = off;
+        if (a.counts) a.counts[t] = cnt;
+        if (a.mt_prefix) a.mt_prefix[t] = mt_off;
         if (a.b_e && a.gamma > 0.f) {
-            // b_e += gamma * sign(mean load - load_e), mean load = N k / E (sec. 2.5)
-            const long long diff = static_cast<long long>(a.N) * a.k - static_cast<long long>(E) * cnt_s[tid];
-            const float sg = static_cast<float>((diff > 0) - (diff < 0));
-            a.b_e[tid] += a.gamma * sg;
+            const long long diff = static_cast<long long>(a.N) * a.k - static_cast<long long>(E) * cnt;
+            a.b_e[t] += a.gamma * static_cast<float>((diff > 0) - (diff < 0));
         }
     }
-    if (active) {
-        int run = off_s[e] + segbase[s * E + e];
-        for (int64_t c = c_begin; c < c_end; ++c) {
-            const int v = a.hist[c * E + e];
-            a.hist[c * E + e] = run;
-            run += v;
+    if (t == 0) {
+        a.offsets[E] = total;
+        if (a.mt_prefix) a.mt_prefix[E] = mt_total;
+        if (a.aux_out && a.psum && a.pe) {
+            if (a.N == 0) {
+                *a.aux_out = 0.0f;  // no tokens: every sum is empty
+            } else {
+                const double Nd = static_cast<double>(a.N);
+                double L = 0.0;
+                for (int q = 0; q < E; ++q) L += (static_cast<double>(cnt_s[q]) / Nd) * (a.pe[q] / Nd);
+                *a.aux_out = static_cast<float>(L * static_cast<double>(E));
+            }
         }
     }
 }
@@ -160,7 +171,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a)
         if (e < 0 || e >= a.E) continue;  // reported by the histogram pass
         int rank = 0;
         for (int r = 0; r < q; ++r) rank += (ids_s[r] == e);
-        const int pos = a.chunk_base[c * a.E + e] + rank;
+        const int pos = a.offsets[e] + a.chunk_base[c * a.E + e] + rank;
         if (a.perm) a.perm[pos] = static_cast<int32_t>(a0 + q);
         a.inv_perm[a0 + q] = pos;
     }
@@ -240,13 +251,13 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
 
 // ------------------------------------------------------------- tile table
 
-__global__ void tile_table_kernel(const int32_t *offsets, int32_t *mt_prefix, int E)
+__global__ void tile_table_kernel(const int32_t *offsets, int32_t *mt_prefix, int E, int tile_m)
 {
     if (threadIdx.x == 0 && blockIdx.x == 0) {
         int mt = 0;
         mt_prefix[0] = 0;
         for (int e = 0; e < E; ++e) {
-            mt += (offsets[e + 1] - offsets[e] + kTileM - 1) / kTileM;
+            mt += (offsets[e + 1] - offsets[e] + tile_m - 1) / tile_m;
             mt_prefix[e + 1] = mt;
         }
     }
@@ -271,7 +282,11 @@ cudaError_t launch_hist(const HistArgs &a, cudaStream_t s)
 
 cudaError_t launch_scan(const ScanArgs &a, cudaStream_t s)
 {
-    scan_kernel<<<1, kScanThreads, 0, s>>>(a);
+    if (a.E > kScanThreads) return cudaErrorInvalidValue;
+    scan_cols_kernel<<<a.E, kScanThreads, 0, s>>>(a);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    scan_finalize_kernel<<<1, kScanThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -301,9 +316,9 @@ cudaError_t launch_combine(int dtype, const CombineArgs &a, int num_sms, cudaStr
     return cudaGetLastError();
 }
 
-cudaError_t launch_tile_table(const int32_t *offsets, int32_t *mt_prefix, int E, cudaStream_t s)
+cudaError_t launch_tile_table(const int32_t *offsets, int32_t *mt_prefix, int E, int tile_m, cudaStream_t s)
 {
-    tile_table_kernel<<<1, 32, 0, s>>>(offsets, mt_prefix, E);
+    tile_table_kernel<<<1, 32, 0, s>>>(offsets, mt_prefix, E, tile_m);
     return cudaGetLastError();
 }
 

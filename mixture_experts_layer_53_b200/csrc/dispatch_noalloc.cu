@@ -103,7 +103,7 @@ moe_status moe_dispatch_noalloc(const moe_config *cfg, const void *x, const int3
     sc.counts = counts;
     sc.offsets = offsets;
     if ((err = launch_scan(sc, s)) != cudaSuccess) return fail(err);
-    ScatterArgs sa{topk_ids, scratch, perm, inv_perm, cfg->N, cfg->E, cfg->k};
+    ScatterArgs sa{topk_ids, scratch, perm, inv_perm, cfg->N, cfg->E, cfg->k, offsets};
     if ((err = launch_scatter(sa, s)) != cudaSuccess) return fail(err);
     if (x) {
         int dev = 0, sms = 148;

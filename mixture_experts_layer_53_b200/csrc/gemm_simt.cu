@@ -3,8 +3,9 @@
 // The fp32 workload must match an fp64 oracle to 1e-5 relative, which the
 // tf32 tensor-core path cannot guarantee, so fp32 runs the same ragged tile
 // walk as the tcgen05 kernel (course module sec. 2.2: one product per expert
-// over its slice of x_sorted) with FFMA: 128x64 output tiles, 256 threads,
-// 8x4 outputs per thread, k-chunks of 16 staged in shared memory.
+// over its slice of x_sorted) with FFMA: each table tile of tile_m rows is
+// computed 128 rows x 64 columns at a time, 256 threads, 8x4 outputs per
+// thread, k-chunks of 16 staged in shared memory.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -24,7 +25,7 @@ struct SimtArgs {
     const int32_t *offsets;
     const int32_t *mt_prefix;
     int64_t rows;
-    int E, K, n_out, n_tiles, b_rows;
+    int E, K, n_out, n_tiles, b_rows, tile_m;
 };
 
 template <int EPI>
@@ -50,9 +51,12 @@ __global__ void __launch_bounds__(THREADS) simt_gemm_kernel(SimtArgs g)
         const int mt_e = g.mt_prefix[e + 1] - g.mt_prefix[e];
         const int local = t - g.mt_prefix[e] * g.n_tiles;
         const int m_tile = local % mt_e, n_tile = local / mt_e;
-        const int64_t row0 = g.offsets[e] + static_cast<int64_t>(m_tile) * TM;
         const int64_t row_end = g.offsets[e + 1];
         const int n0 = n_tile * TN;
+        // a tile of the table spans tile_m rows: walk it TM rows at a time
+        for (int part = 0; part * TM < g.tile_m; ++part) {
+        const int64_t row0 = g.offsets[e] + static_cast<int64_t>(m_tile) * g.tile_m + part * TM;
+        if (row0 >= row_end) break;  // uniform across the block
 
         float acc[8][4], acc3[8][4];
 #pragma unroll
@@ -113,6 +117,7 @@ __global__ void __launch_bounds__(THREADS) simt_gemm_kernel(SimtArgs g)
                 g.out[row * g.n_out + col] = v;
             }
         }
+        }
     }
 }
 
@@ -143,6 +148,7 @@ cudaError_t launch_ffn_f32_simt(const FfnArgs &a, int num_sms, cudaEvent_t mid, 
         g1.n_out = a.F;
         g1.n_tiles = (a.F + TN - 1) / TN;
         g1.b_rows = a.F;
+        g1.tile_m = a.tile_m;
         err = swiglu ? launch_simt<EPI_SWIGLU>(g1, num_sms, s) : launch_simt<EPI_GELU>(g1, num_sms, s);
         if (err != cudaSuccess) return err;
     }
@@ -161,6 +167,7 @@ cudaError_t launch_ffn_f32_simt(const FfnArgs &a, int num_sms, cudaEvent_t mid, 
         g2.n_out = a.d;
         g2.n_tiles = (a.d + TN - 1) / TN;
         g2.b_rows = a.d;
+        g2.tile_m = a.tile_m;
         err = launch_simt<EPI_LINEAR>(g2, num_sms, s);
     }
     return err;

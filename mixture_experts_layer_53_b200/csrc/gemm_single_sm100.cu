@@ -1,0 +1,385 @@
+// gemm_single_sm100.cu -- ragged grouped GEMM for the expert FFNs on single
+// CTAs (tcgen05 cta_group::1, 128 x 256 tiles), for experts with few rows.
+// The tile table it walks counts 128-row m-tiles; the CTA-pair kernel in
+// gemm_sm100.cu takes the experts with many rows.
+//
+// Course module "Mixture of Experts: routing, sorted dispatch, Switch aux
+// loss, aux-free bias", sec. 2.2: after the sorted dispatch "each expert runs
+// once on its slice" -- one matrix product per expert over rows
+// offsets[e] .. offsets[e+1]-1 of x_sorted, no padding to a capacity.
+//
+// GEMM1: h = act(x_sorted W1[e]^T (, x_sorted W3[e]^T))  [rows, d_ff]
+// GEMM2: y_sorted = h W2[e]^T (+ b2[e])                   [rows, d_model]
+//
+// When experts hold about 128 rows or fewer (fine-grained MoE such as the
+// DeepSeek-V3 shape), 256-row pair tiles would compute mostly rows of the next
+// expert; 128-row tiles waste less tensor work, which matters under the
+// power cap.  Tiles are 128 rows x 256 accumulator columns, k-blocks of 64.  The tile
+// list is (expert, n-tile, m-tile) with the m-tile innermost, so CTAs that run
+// at the same time share one expert's weight tile through L2.  The tile
+// count lives on the device (from the dispatch scan), so a persistent grid
+// of one CTA per SM walks it with no host synchronisation.
+//
+// Warp roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A and B tiles into a 4-stage shared-memory ring
+//   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma
+//               (M=128, N=256, K=16, bf16 -> fp32) and tcgen05.commit
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (one row per
+//               thread), fused activation / bias, bf16 stores
+// Accumulators are double-buffered in TMEM (2 x 256 columns) so the
+// epilogue of one tile overlaps the MMAs of the next.
+//
+// SwiGLU: the B tile holds 128 rows of W1 and the same 128 rows of W3, so
+// accumulator columns 0..127 are the gate and 128..255 the up projection of
+// 128 hidden units; the epilogue writes silu(gate) * up.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "host_util.h"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+
+enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_LINEAR = 2 };
+
+struct GemmArgs {
+    const int32_t *offsets;
+    const int32_t *mt_prefix;
+    __nv_bfloat16 *out;
+    int64_t ldo;
+    const __nv_bfloat16 *bias;  // [E, n_out] or null
+    int32_t *status;
+    int E, K, n_out, n_tiles, b_rows;
+};
+
+struct Ctl {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int off[kMaxE + 1];
+    int mt[kMaxE + 1];
+};
+
+constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(Ctl);
+
+struct Tile {
+    int e, m_tile, n_tile;
+};
+
+__device__ __forceinline__ Tile decode_tile(int t, const Ctl *c, int E, int n_tiles)
+{
+    const int q = t / n_tiles;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (c->mt[mid] <= q) lo = mid;
+        else hi = mid - 1;
+    }
+    const int mt_e = c->mt[lo + 1] - c->mt[lo];
+    const int local = t - c->mt[lo] * n_tiles;
+    return Tile{lo, local % mt_e, local / mt_e};
+}
+
+template <int EPI> __host__ __device__ constexpr int out_cols() { return EPI == EPI_SWIGLU ? 128 : 256; }
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase, int e, int row,
+                                              bool row_ok, int n0)
+{
+    __nv_bfloat16 *orow = g.out + static_cast<int64_t>(row) * g.ldo;
+    const __nv_bfloat16 *brow = g.bias ? g.bias + static_cast<int64_t>(e) * g.n_out : nullptr;
+#pragma unroll 1
+    for (int c = 0; c < out_cols<EPI>(); c += 32) {
+        uint32_t acc[32];
+        tmem_ld32(tbase + c, acc);
+        if constexpr (EPI == EPI_SWIGLU) {
+            uint32_t up[32];
+            tmem_ld32(tbase + 128 + c, up);
+            tmem_ld_wait();
+            if (row_ok) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const int col = n0 + c + v * 8;
+                    if (col < g.n_out) {
+                        float h[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            h[u] = silu(__uint_as_float(acc[v * 8 + u])) * __uint_as_float(up[v * 8 + u]);
+                        st16(orow + col, pack16(h, static_cast<const __nv_bfloat16 *>(nullptr)));
+                    }
+                }
+            }
+        } else {
+            tmem_ld_wait();
+            if (row_ok) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const int col = n0 + c + v * 8;
+                    if (col < g.n_out) {
+                        float o[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) o[u] = __uint_as_float(acc[v * 8 + u]);
+                        if (brow) {
+                            float b[8];
+                            unpack16(*reinterpret_cast<const uint4 *>(brow + col), b,
+                                     static_cast<const __nv_bfloat16 *>(nullptr));
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) o[u] += b[u];
+                        }
+                        if constexpr (EPI == EPI_GELU) {
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) o[u] = gelu_erf(o[u]);
+                        }
+                        st16(orow + col, pack16(o, static_cast<const __nv_bfloat16 *>(nullptr)));
+                    }
+                }
+            }
+        }
+    }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    ffn_gemm_single_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmB3, const GemmArgs g)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                 ~static_cast<uintptr_t>(1023));
+    Ctl *ctl = reinterpret_cast<Ctl *>(tiles + STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int *abort_flag = &ctl->abort;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->tfull[b], 1);
+            mbar_init(&ctl->tempty[b], 128);
+        }
+        mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    if (threadIdx.x == 32) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        if (EPI == EPI_SWIGLU) prefetch_tmap(&tmB3);
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    for (int i = threadIdx.x; i <= g.E; i += THREADS) {
+        ctl->off[i] = g.offsets[i];
+        ctl->mt[i] = g.mt_prefix[i];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem_base = ctl->tmem_base;
+    const int total = ctl->mt[g.E] * g.n_tiles;
+    const int num_kb = (g.K + BK - 1) / BK;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            int stage = 0;
+            uint32_t phase = 0, armed = 0, armed_parity = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const Tile ti = decode_tile(t, ctl, g.E, g.n_tiles);
+                const int row0 = ctl->off[ti.e] + ti.m_tile * BM;
+                const int brow = ti.e * g.b_rows + ti.n_tile * out_cols<EPI>();
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort_flag, g.status)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sA = tiles + stage * STAGE_BYTES;
+                    uint8_t *sB = sA + A_BYTES;
+                    mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
+                    armed |= 1u << stage;
+                    armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                    tma_load_2d(sA, &tmA, &ctl->full[stage], kb * BK, row0);
+                    if (EPI == EPI_SWIGLU) {
+                        tma_load_2d(sB, &tmB, &ctl->full[stage], kb * BK, brow);
+                        tma_load_2d(sB + B_BYTES / 2, &tmB3, &ctl->full[stage], kb * BK, brow);
+                    } else {
+                        tma_load_2d(sB, &tmB, &ctl->full[stage], kb * BK, brow);
+                    }
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (*abort_flag) {
+                // let every copy this thread started land before the CTA exits
+                for (int s = 0; s < STAGES; ++s)
+                    if ((armed >> s) & 1u)
+                        mbar_wait(&ctl->full[s], (armed_parity >> s) & 1u, abort_flag, g.status, false);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+            int stage = 0, buf = 0;
+            uint32_t phase = 0, tphase = 0;
+            bool ok = true, issued = false;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                if (!mbar_wait(&ctl->tempty[buf], tphase ^ 1u, abort_flag, g.status)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&ctl->full[stage], phase, abort_flag, g.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(tiles + stage * STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        umma_bf16(d_tmem, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32), idesc,
+                                  (kb | kk) != 0 ? 1u : 0u);
+                    issued = true;
+                    umma_commit(&ctl->empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&ctl->tfull[buf]);
+                if (++buf == 2) {
+                    buf = 0;
+                    tphase ^= 1u;
+                }
+            }
+            if (*abort_flag && issued) {
+                // wait for every MMA issued so far before TMEM is freed
+                umma_commit(&ctl->drain);
+                mbar_wait(&ctl->drain, 0, abort_flag, g.status, false);
+            }
+        }
+    } else {
+        // ---------------------------------------------------- epilogue
+        const int quarter = warp & 3;  // TMEM lanes this warp may access
+        const int row_in_tile = quarter * 32 + lane;
+        int buf = 0;
+        uint32_t tphase = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&ctl->tfull[buf], tphase, abort_flag, g.status));
+            if (!ok) break;
+            tc_fence_after();
+            const Tile ti = decode_tile(t, ctl, g.E, g.n_tiles);
+            const int row = ctl->off[ti.e] + ti.m_tile * BM + row_in_tile;
+            const bool row_ok = row < ctl->off[ti.e + 1];
+            const uint32_t tbase =
+                tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
+            epilogue_tile<EPI>(g, tbase, ti.e, row, row_ok, ti.n_tile * out_cols<EPI>());
+            tc_fence_before();
+            mbar_arrive(&ctl->tempty[buf]);
+            if (++buf == 2) {
+                buf = 0;
+                tphase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// --------------------------------------------------------------- host side
+
+template <int EPI>
+cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b3, const GemmArgs &g,
+                        int num_sms, cudaStream_t s)
+{
+    cudaError_t err =
+        ensure_smem_attr(reinterpret_cast<const void *>(&ffn_gemm_single_kernel<EPI>), static_cast<int>(kSmemBytes));
+    if (err != cudaSuccess) return err;
+    ffn_gemm_single_kernel<EPI><<<num_sms, THREADS, kSmemBytes, s>>>(a, b, b3, g);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_bf16_sm100_single(const FfnArgs &a, int num_sms, cudaEvent_t mid, cudaStream_t s)
+{
+    if (a.tile_m != BM) return cudaErrorInvalidValue;  // the tile table must count 128-row tiles
+    if (a.rows == 0) {
+        if (mid) return cudaEventRecord(mid, s);
+        return cudaSuccess;
+    }
+    const bool swiglu = a.act == kSwiglu;
+    const uint64_t rows = static_cast<uint64_t>(a.rows);
+    const uint64_t E = static_cast<uint64_t>(a.E);
+    CUtensorMap tA, tB, tB3, tH, tW2;
+    if (!make_tmap_bf16(&tA, a.x_sorted, a.d, rows, BM) ||
+        !make_tmap_bf16(&tB, a.W1, a.d, E * a.F, swiglu ? 128 : 256) ||
+        !make_tmap_bf16(&tB3, swiglu ? a.W3 : a.W1, a.d, E * a.F, swiglu ? 128 : 256) ||
+        !make_tmap_bf16(&tH, a.h, a.F, rows, BM) || !make_tmap_bf16(&tW2, a.W2, a.F, E * a.d, 256))
+        return cudaErrorInvalidValue;
+
+    GemmArgs g1{};
+    g1.offsets = a.offsets;
+    g1.mt_prefix = a.mt_prefix;
+    g1.out = static_cast<__nv_bfloat16 *>(a.h);
+    g1.ldo = a.F;
+    g1.bias = swiglu ? nullptr : static_cast<const __nv_bfloat16 *>(a.b1);
+    g1.status = a.status;
+    g1.E = a.E;
+    g1.K = a.d;
+    g1.n_out = a.F;
+    g1.n_tiles = (a.F + (swiglu ? 127 : 255)) / (swiglu ? 128 : 256);
+    g1.b_rows = a.F;
+    cudaError_t err = swiglu ? launch_gemm<EPI_SWIGLU>(tA, tB, tB3, g1, num_sms, s)
+                             : launch_gemm<EPI_GELU>(tA, tB, tB3, g1, num_sms, s);
+    if (err != cudaSuccess) return err;
+    if (mid && (err = cudaEventRecord(mid, s)) != cudaSuccess) return err;
+
+    GemmArgs g2{};
+    g2.offsets = a.offsets;
+    g2.mt_prefix = a.mt_prefix;
+    g2.out = static_cast<__nv_bfloat16 *>(a.y_sorted);
+    g2.ldo = a.d;
+    g2.bias = static_cast<const __nv_bfloat16 *>(a.b2);
+    g2.status = a.status;
+    g2.E = a.E;
+    g2.K = a.F;
+    g2.n_out = a.d;
+    g2.n_tiles = (a.d + 255) / 256;
+    g2.b_rows = a.d;
+    return launch_gemm<EPI_LINEAR>(tH, tW2, tW2, g2, num_sms, s);
+}
+
+}  // namespace moe

@@ -1,34 +1,34 @@
-// gemm_sm100.cu -- ragged grouped GEMM for the expert FFNs on the Blackwell
-// tensor cores (tcgen05, accumulators in TMEM, operands staged by TMA).
+// gemm_sm100.cu -- ragged grouped GEMM for the expert FFNs on CTA pairs
+// (tcgen05 cta_group::2): each pair computes a 256 x 256 tile.
 //
 // Course module "Mixture of Experts: routing, sorted dispatch, Switch aux
-// loss, aux-free bias", sec. 2.2: after the sorted dispatch "each expert runs
-// once on its slice" -- one matrix product per expert over rows
-// offsets[e] .. offsets[e+1]-1 of x_sorted, no padding to a capacity.
+// loss, aux-free bias", sec. 2.2: each expert runs once on its slice --
+// rows offsets[e] .. offsets[e+1]-1 of x_sorted, no padding to a capacity.
 //
 // GEMM1: h = act(x_sorted W1[e]^T (, x_sorted W3[e]^T))  [rows, d_ff]
 // GEMM2: y_sorted = h W2[e]^T (+ b2[e])                   [rows, d_model]
 //
-// Tiles are 128 rows x 256 accumulator columns, k-blocks of 64.  The tile
-// list is (expert, n-tile, m-tile) with the m-tile innermost, so CTAs that run
-// at the same time share one expert's weight tile through L2.  The tile
-// count lives on the device (from the dispatch scan), so a persistent grid
-// of one CTA per SM walks it with no host synchronisation.
+// A cluster of two CTAs (one SM pair) owns a tile of 256 rows x 256
+// accumulator columns.  Each CTA loads its own 128 rows of A and one half of
+// the B tile (128 of its 256 rows) with TMA into its own shared memory; the
+// even CTA issues tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16), which
+// reads A from each CTA and B from both, and accumulates each CTA's 128 rows
+// in that CTA's TMEM.  Per k-block each SM so moves 32 KB instead of the 48 KB
+// of a one-SM 128 x 256 tile, and a weight tile crosses L2 once per pair.
+// No TMA load uses multicast: each CTA fetches its own tiles.
 //
-// Warp roles (192 threads, one CTA per SM):
-//   warp 0      TMA producer: A and B tiles into a 4-stage shared-memory ring
-//   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma
-//               (M=128, N=256, K=16, bf16 -> fp32) and tcgen05.commit
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator (one row per
-//               thread), fused activation / bias, bf16 stores
-// Accumulators are double-buffered in TMEM (2 x 256 columns) so the
-// epilogue of one tile overlaps the MMAs of the next.
-//
-// SwiGLU: the B tile holds 128 rows of W1 and the same 128 rows of W3, so
-// accumulator columns 0..127 are the gate and 128..255 the up projection of
-// 128 hidden units; the epilogue writes silu(gate) * up.
+// Tiles are (expert, n-tile, m-tile of 256 rows), m-tile innermost, walked
+// by a persistent grid of one pair per two SMs.  Warp roles per CTA:
+//   warp 0     TMA producer (both CTAs; completion is counted on the even
+//              CTA's `full` barrier, which expects both CTAs' bytes)
+//   warp 1     TMEM allocation for the pair (both CTAs); in the even CTA one
+//              lane issues the MMAs and commits to both CTAs' barriers
+//   warps 2-5  epilogue on the CTA's own 128 rows (tcgen05.ld), fused
+//              activation / bias, bf16 stores
+// SwiGLU: the even CTA's B half holds 128 rows of W1 and the odd CTA's the
+// same 128 rows of W3, so accumulator columns 0..127 are the gate and
+// 128..255 the up projection of 128 hidden units.
 #include <cuda.h>
-#include <mutex>
 
 #include "common.cuh"
 #include "host_util.h"
@@ -40,15 +40,17 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;        // rows per CTA
+constexpr int PAIR_M = 256;    // rows per pair tile
+constexpr int BN = 256;        // accumulator columns
 constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * BK * 2;        // 16 KB
+constexpr int B_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's half of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
+
 
 enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_LINEAR = 2 };
 
@@ -63,10 +65,10 @@ struct GemmArgs {
 };
 
 struct Ctl {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
-    uint64_t tfull[2];
-    uint64_t tempty[2];
+    uint64_t full[STAGES];   // used in the even CTA: both CTAs' bytes
+    uint64_t empty[STAGES];  // each CTA: arrived by the even CTA's commit
+    uint64_t tfull[2];       // each CTA: arrived by the even CTA's commit
+    uint64_t tempty[2];      // even CTA: 4 epilogue warps x 2 CTAs
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -97,8 +99,8 @@ __device__ __forceinline__ Tile decode_tile(int t, const Ctl *c, int E, int n_ti
 template <int EPI> __host__ __device__ constexpr int out_cols() { return EPI == EPI_SWIGLU ? 128 : 256; }
 
 template <int EPI>
-__device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase, int e, int row,
-                                              bool row_ok, int n0)
+__device__ __forceinline__ void epilogue_rows(const GemmArgs &g, uint32_t tbase, int e, int row, bool row_ok,
+                                              int n0)
 {
     __nv_bfloat16 *orow = g.out + static_cast<int64_t>(row) * g.ldo;
     const __nv_bfloat16 *brow = g.bias ? g.bias + static_cast<int64_t>(e) * g.n_out : nullptr;
@@ -153,15 +155,17 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase,
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(THREADS, 1)
-    ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmB3, const GemmArgs g)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmB3, const GemmArgs g)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                  ~static_cast<uintptr_t>(1023));
     Ctl *ctl = reinterpret_cast<Ctl *>(tiles + STAGES * STAGE_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
     volatile int *abort_flag = &ctl->abort;
 
     if (threadIdx.x == 0) {
@@ -171,7 +175,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->tfull[b], 1);
-            mbar_init(&ctl->tempty[b], 128);
+            mbar_init(&ctl->tempty[b], 8);
         }
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
@@ -183,20 +187,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (EPI == EPI_SWIGLU) prefetch_tmap(&tmB3);
     }
     if (warp == 1) {
-        tmem_alloc(&ctl->tmem_base, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     for (int i = threadIdx.x; i <= g.E; i += THREADS) {
         ctl->off[i] = g.offsets[i];
         ctl->mt[i] = g.mt_prefix[i];
     }
     tc_fence_before();
-    __syncthreads();
+    // barriers of both CTAs are initialised before either CTA signals the other
+    cluster_sync();
     tc_fence_after();
 
     const uint32_t tmem_base = ctl->tmem_base;
     const int total = ctl->mt[g.E] * g.n_tiles;
     const int num_kb = (g.K + BK - 1) / BK;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -204,48 +210,53 @@ __global__ void __launch_bounds__(THREADS, 1)
             int stage = 0;
             uint32_t phase = 0, armed = 0, armed_parity = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (int t = pair; t < total && ok; t += npairs) {
                 const Tile ti = decode_tile(t, ctl, g.E, g.n_tiles);
-                const int row0 = ctl->off[ti.e] + ti.m_tile * BM;
-                const int brow = ti.e * g.b_rows + ti.n_tile * out_cols<EPI>();
+                const int row0 = ctl->off[ti.e] + ti.m_tile * PAIR_M + static_cast<int>(rank) * BM;
+                int brow;
+                const CUtensorMap *tb;
+                if (EPI == EPI_SWIGLU) {  // even CTA: W1 rows, odd CTA: the same rows of W3
+                    brow = ti.e * g.b_rows + ti.n_tile * 128;
+                    tb = rank ? &tmB3 : &tmB;
+                } else {
+                    brow = ti.e * g.b_rows + ti.n_tile * BN + static_cast<int>(rank) * (BN / 2);
+                    tb = &tmB;
+                }
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort_flag, g.status)) {
                         ok = false;
                         break;
                     }
                     uint8_t *sA = tiles + stage * STAGE_BYTES;
-                    uint8_t *sB = sA + A_BYTES;
-                    mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
-                    armed |= 1u << stage;
-                    armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-                    tma_load_2d(sA, &tmA, &ctl->full[stage], kb * BK, row0);
-                    if (EPI == EPI_SWIGLU) {
-                        tma_load_2d(sB, &tmB, &ctl->full[stage], kb * BK, brow);
-                        tma_load_2d(sB + B_BYTES / 2, &tmB3, &ctl->full[stage], kb * BK, brow);
-                    } else {
-                        tma_load_2d(sB, &tmB, &ctl->full[stage], kb * BK, brow);
+                    const uint32_t full_leader = mapa_shared(smem_u32(&ctl->full[stage]), 0);
+                    if (leader) {
+                        mbar_arrive_expect_tx(&ctl->full[stage], 2 * STAGE_BYTES);
+                        armed |= 1u << stage;
+                        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
                     }
+                    tma_load_2d_pair(sA, &tmA, full_leader, kb * BK, row0);
+                    tma_load_2d_pair(sA + A_BYTES, tb, full_leader, kb * BK, brow);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
-            if (*abort_flag) {
-                // let every copy this thread started land before the CTA exits
+            if (*abort_flag && leader) {
+                // both CTAs' copies land on these barriers: wait for them
                 for (int s = 0; s < STAGES; ++s)
                     if ((armed >> s) & 1u)
                         mbar_wait(&ctl->full[s], (armed_parity >> s) & 1u, abort_flag, g.status, false);
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && leader) {
             // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+            constexpr uint32_t idesc = idesc_bf16_f32(PAIR_M, BN);
             int stage = 0, buf = 0;
             uint32_t phase = 0, tphase = 0;
             bool ok = true, issued = false;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (int t = pair; t < total && ok; t += npairs) {
                 if (!mbar_wait(&ctl->tempty[buf], tphase ^ 1u, abort_flag, g.status)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
@@ -259,46 +270,48 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        umma_bf16(d_tmem, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32), idesc,
-                                  (kb | kk) != 0 ? 1u : 0u);
+                        umma_bf16_pair(d_tmem, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32), idesc,
+                                       (kb | kk) != 0 ? 1u : 0u);
                     issued = true;
-                    umma_commit(&ctl->empty[stage]);
+                    umma_commit_pair(&ctl->empty[stage], 0x3);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                umma_commit(&ctl->tfull[buf]);
+                umma_commit_pair(&ctl->tfull[buf], 0x3);
                 if (++buf == 2) {
                     buf = 0;
                     tphase ^= 1u;
                 }
             }
             if (*abort_flag && issued) {
-                // wait for every MMA issued so far before TMEM is freed
-                umma_commit(&ctl->drain);
+                umma_commit_pair(&ctl->drain, 0x1);
                 mbar_wait(&ctl->drain, 0, abort_flag, g.status, false);
             }
         }
     } else {
         // ---------------------------------------------------- epilogue
         const int quarter = warp & 3;  // TMEM lanes this warp may access
-        const int row_in_tile = quarter * 32 + lane;
+        const int row_in_cta = quarter * 32 + lane;
+        const uint32_t tempty_leader0 = mapa_shared(smem_u32(&ctl->tempty[0]), 0);
+        const uint32_t tempty_leader1 = mapa_shared(smem_u32(&ctl->tempty[1]), 0);
         int buf = 0;
         uint32_t tphase = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        for (int t = pair; t < total; t += npairs) {
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&ctl->tfull[buf], tphase, abort_flag, g.status));
             if (!ok) break;
             tc_fence_after();
             const Tile ti = decode_tile(t, ctl, g.E, g.n_tiles);
-            const int row = ctl->off[ti.e] + ti.m_tile * BM + row_in_tile;
+            const int row = ctl->off[ti.e] + ti.m_tile * PAIR_M + static_cast<int>(rank) * BM + row_in_cta;
             const bool row_ok = row < ctl->off[ti.e + 1];
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
-            epilogue_tile<EPI>(g, tbase, ti.e, row, row_ok, ti.n_tile * out_cols<EPI>());
+            epilogue_rows<EPI>(g, tbase, ti.e, row, row_ok, ti.n_tile * out_cols<EPI>());
             tc_fence_before();
-            mbar_arrive(&ctl->tempty[buf]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
             if (++buf == 2) {
                 buf = 0;
                 tphase ^= 1u;
@@ -308,61 +321,23 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    // neither CTA frees TMEM or leaves while its pair partner may still use it
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
     }
 }
 
-// --------------------------------------------------------------- host side
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
-                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                  CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-}  // namespace
-
-// bf16 matrix [outer, inner] (inner contiguous), box [box_outer, 64],
-// 128-byte swizzle, zero fill outside the matrix.
-bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_outer)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[2] = {inner, outer};
-    const cuuint64_t strides[1] = {inner * 2};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_outer};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-namespace {
-
 template <int EPI>
-cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b3, const GemmArgs &g,
+cudaError_t launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b3, const GemmArgs &g,
                         int num_sms, cudaStream_t s)
 {
-    cudaError_t err =
-        ensure_smem_attr(reinterpret_cast<const void *>(&ffn_gemm_kernel<EPI>), static_cast<int>(kSmemBytes));
+    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&ffn_gemm_pair_kernel<EPI>),
+                                       static_cast<int>(kSmemBytes));
     if (err != cudaSuccess) return err;
-    ffn_gemm_kernel<EPI><<<num_sms, THREADS, kSmemBytes, s>>>(a, b, b3, g);
+    const int grid = (num_sms / 2) * 2;
+    ffn_gemm_pair_kernel<EPI><<<grid, THREADS, kSmemBytes, s>>>(a, b, b3, g);
     return cudaGetLastError();
 }
 
@@ -370,6 +345,7 @@ cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtens
 
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid, cudaStream_t s)
 {
+    if (a.tile_m != PAIR_M) return cudaErrorInvalidValue;  // the tile table must count 256-row tiles
     if (a.rows == 0) {
         if (mid) return cudaEventRecord(mid, s);
         return cudaSuccess;
@@ -378,10 +354,10 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid
     const uint64_t rows = static_cast<uint64_t>(a.rows);
     const uint64_t E = static_cast<uint64_t>(a.E);
     CUtensorMap tA, tB, tB3, tH, tW2;
-    if (!make_tmap_bf16(&tA, a.x_sorted, a.d, rows, BM) ||
-        !make_tmap_bf16(&tB, a.W1, a.d, E * a.F, swiglu ? 128 : 256) ||
-        !make_tmap_bf16(&tB3, swiglu ? a.W3 : a.W1, a.d, E * a.F, swiglu ? 128 : 256) ||
-        !make_tmap_bf16(&tH, a.h, a.F, rows, BM) || !make_tmap_bf16(&tW2, a.W2, a.F, E * a.d, 256))
+    // each CTA loads 128 rows of A and 128 rows of B per k-block
+    if (!make_tmap_bf16(&tA, a.x_sorted, a.d, rows, BM) || !make_tmap_bf16(&tB, a.W1, a.d, E * a.F, 128) ||
+        !make_tmap_bf16(&tB3, swiglu ? a.W3 : a.W1, a.d, E * a.F, 128) ||
+        !make_tmap_bf16(&tH, a.h, a.F, rows, BM) || !make_tmap_bf16(&tW2, a.W2, a.F, E * a.d, 128))
         return cudaErrorInvalidValue;
 
     GemmArgs g1{};
@@ -396,8 +372,8 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid
     g1.n_out = a.F;
     g1.n_tiles = (a.F + (swiglu ? 127 : 255)) / (swiglu ? 128 : 256);
     g1.b_rows = a.F;
-    cudaError_t err = swiglu ? launch_gemm<EPI_SWIGLU>(tA, tB, tB3, g1, num_sms, s)
-                             : launch_gemm<EPI_GELU>(tA, tB, tB3, g1, num_sms, s);
+    cudaError_t err = swiglu ? launch_pair<EPI_SWIGLU>(tA, tB, tB3, g1, num_sms, s)
+                             : launch_pair<EPI_GELU>(tA, tB, tB3, g1, num_sms, s);
     if (err != cudaSuccess) return err;
     if (mid && (err = cudaEventRecord(mid, s)) != cudaSuccess) return err;
 
@@ -413,7 +389,7 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid
     g2.n_out = a.d;
     g2.n_tiles = (a.d + 255) / 256;
     g2.b_rows = a.d;
-    return launch_gemm<EPI_LINEAR>(tH, tW2, tW2, g2, num_sms, s);
+    return launch_pair<EPI_LINEAR>(tH, tW2, tW2, g2, num_sms, s);
 }
 
 }  // namespace moe

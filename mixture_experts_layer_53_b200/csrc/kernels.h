@@ -62,10 +62,11 @@ struct HistArgs {
 };
 cudaError_t launch_hist(const HistArgs &a, cudaStream_t s);
 
-// One CTA: counts, offsets, per-chunk bases (in place over hist), the GEMM
-// tile table, the Switch loss and the sign-rule bias step.
+// Counts, offsets, per-chunk bases inside each expert's slice (in place over
+// hist), the GEMM tile table, the Switch loss and the sign-rule bias step:
+// one CTA per expert, then one finalizing CTA.
 struct ScanArgs {
-    int32_t *hist;        // in: [chunks, E] counts; out: per-chunk slice bases
+    int32_t *hist;        // in: [chunks, E] counts; out: chunk bases within the expert's slice
     const float *psum;    // [chunks, E] or null (no loss then)
     int64_t chunks, N;
     int E, k;
@@ -75,16 +76,20 @@ struct ScanArgs {
     float *aux_out;       // scalar or null
     float gamma;
     float *b_e;           // [E] or null
+    double *pe;           // [E] scratch for P_e * N (needed when psum is given)
+    int tile_m;           // rows per m-tile of the tile table (when mt_prefix is given)
 };
 cudaError_t launch_scan(const ScanArgs &a, cudaStream_t s);
 
+// Sorted position of assignment a: offsets[e] + chunk base + rank in chunk.
 struct ScatterArgs {
     const int32_t *ids;
-    const int32_t *chunk_base;  // [chunks, E]
+    const int32_t *chunk_base;  // [chunks, E], relative to the slice start
     int32_t *perm;              // [N k] or null
     int32_t *inv_perm;          // [N k]
     int64_t N;
     int E, k;
+    const int32_t *offsets;     // [E+1]
 };
 cudaError_t launch_scatter(const ScatterArgs &a, cudaStream_t s);
 
@@ -107,8 +112,8 @@ struct CombineArgs {
 };
 cudaError_t launch_combine(int dtype, const CombineArgs &a, int num_sms, cudaStream_t s);
 
-// mt_prefix[e+1] = mt_prefix[e] + ceil((offsets[e+1] - offsets[e]) / 128).
-cudaError_t launch_tile_table(const int32_t *offsets, int32_t *mt_prefix, int E, cudaStream_t s);
+// mt_prefix[e+1] = mt_prefix[e] + ceil((offsets[e+1] - offsets[e]) / tile_m).
+cudaError_t launch_tile_table(const int32_t *offsets, int32_t *mt_prefix, int E, int tile_m, cudaStream_t s);
 
 struct FfnArgs {
     const void *x_sorted;      // [rows, d]
@@ -120,6 +125,7 @@ struct FfnArgs {
     int32_t *status;
     int64_t rows;              // N k
     int d, F, E, act;
+    int tile_m;                // m-tile rows of mt_prefix: 128 (single CTA) or 256 (CTA pair)
 };
 }  // namespace moe
 
@@ -132,7 +138,10 @@ namespace moe {
 bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_outer);
 
 // Both expert GEMMs; `mid` (may be null) is recorded between them.
+// CTA pairs, 256-row m-tiles:
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid, cudaStream_t s);
+// single CTAs, 128-row m-tiles:
+cudaError_t launch_ffn_bf16_sm100_single(const FfnArgs &a, int num_sms, cudaEvent_t mid, cudaStream_t s);
 cudaError_t launch_ffn_f32_simt(const FfnArgs &a, int num_sms, cudaEvent_t mid, cudaStream_t s);
 
 }  // namespace moe

@@ -60,7 +60,7 @@ moe_status validate(const moe_config *c)
 }
 
 struct Layout {
-    size_t hist, psum, logits, offsets, mt, counts, ids, w, perm, inv, xs, h, ys, total;
+    size_t hist, psum, logits, pe, offsets, mt, counts, ids, w, perm, inv, xs, h, ys, total;
 };
 
 size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
@@ -81,6 +81,7 @@ Layout layout(const moe_config *c)
     L.hist = take(C * E * 4);
     L.logits = take(static_cast<size_t>(c->N) * static_cast<size_t>(logits_ld(c->E)) * 4);
     L.psum = take(C * E * 4);
+    L.pe = take(E * 8);
     L.offsets = take((E + 1) * 4);
     L.mt = take((E + 1) * 4);
     L.counts = take(E * 4);
@@ -126,6 +127,16 @@ RouterArgs router_args(const moe_config *c, const void *x, const void *W_g, cons
     return r;
 }
 
+// Rows per m-tile of the expert GEMMs.  bf16: CTA pairs (256 rows) when the
+// experts hold many rows on average, single CTAs (128 rows) for fine-grained
+// experts, where 256-row tiles would mostly compute rows of the next expert.
+int ffn_tile_m(const moe_config *c)
+{
+    if (c->dtype != MOE_BF16) return 128;
+    const int64_t rows_per_expert = c->N * c->k / c->E;
+    return rows_per_expert > 192 ? 256 : 128;
+}
+
 FfnArgs ffn_args(const moe_config *c, const void *x_sorted, const int32_t *offsets, const int32_t *mt,
                  const void *W1, const void *b1, const void *W3, const void *W2, const void *b2, void *h,
                  void *y_sorted, int32_t *status)
@@ -147,6 +158,7 @@ FfnArgs ffn_args(const moe_config *c, const void *x_sorted, const int32_t *offse
     f.F = c->d_ff;
     f.E = c->E;
     f.act = c->act;
+    f.tile_m = ffn_tile_m(c);
     return f;
 }
 
@@ -176,8 +188,9 @@ cudaError_t launch_route(const moe_config *c, const RouterArgs &r, int32_t *stat
 
 cudaError_t launch_ffn(const moe_config *c, const FfnArgs &f, cudaEvent_t mid, cudaStream_t s)
 {
-    return c->dtype == MOE_BF16 ? launch_ffn_bf16_sm100(f, num_sms(), mid, s)
-                                : launch_ffn_f32_simt(f, num_sms(), mid, s);
+    if (c->dtype != MOE_BF16) return launch_ffn_f32_simt(f, num_sms(), mid, s);
+    return f.tile_m == 256 ? launch_ffn_bf16_sm100(f, num_sms(), mid, s)
+                           : launch_ffn_bf16_sm100_single(f, num_sms(), mid, s);
 }
 
 }  // namespace
@@ -251,7 +264,7 @@ moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *top
     sc.counts = counts;
     sc.offsets = offsets;
     if ((err = launch_scan(sc, s)) != cudaSuccess) return cuda_fail(err);
-    ScatterArgs sa{topk_ids, hist, perm, inv_perm, cfg->N, cfg->E, cfg->k};
+    ScatterArgs sa{topk_ids, hist, perm, inv_perm, cfg->N, cfg->E, cfg->k, offsets};
     if ((err = launch_scatter(sa, s)) != cudaSuccess) return cuda_fail(err);
     if (x) {
         GatherArgs ga{x, inv_perm, x_sorted, cfg->N, cfg->d_model, cfg->k};
@@ -275,7 +288,7 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_sorted, const int
     const Layout L = layout(cfg);
     int32_t *mt = at<int32_t>(ws, L.mt);
     cudaError_t err;
-    if ((err = launch_tile_table(offsets, mt, cfg->E, s)) != cudaSuccess) return cuda_fail(err);
+    if ((err = launch_tile_table(offsets, mt, cfg->E, ffn_tile_m(cfg), s)) != cudaSuccess) return cuda_fail(err);
     const FfnArgs f = ffn_args(cfg, x_sorted, offsets, mt, W1, b1, W3, W2, b2, at<void>(ws, L.h), y_sorted,
                                dev_status);
     if ((err = launch_ffn(cfg, f, nullptr, s)) != cudaSuccess) return cuda_fail(err);
@@ -314,6 +327,7 @@ moe_status moe_aux_loss(const moe_config *cfg, const float *probs, const int32_t
     ScanArgs sc{};
     sc.hist = hist;
     sc.psum = psum;
+    sc.pe = at<double>(ws, L.pe);
     sc.chunks = num_chunks(cfg->N);
     sc.N = cfg->N;
     sc.E = cfg->E;
@@ -370,6 +384,7 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const void *W_g, fl
     ScanArgs sc{};
     sc.hist = hist;
     sc.psum = psum;
+    sc.pe = at<double>(ws, L.pe);
     sc.chunks = num_chunks(cfg->N);
     sc.N = cfg->N;
     sc.E = cfg->E;
@@ -379,9 +394,10 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const void *W_g, fl
     sc.mt_prefix = mt;
     sc.aux_out = aux_out;
     sc.gamma = gamma;
+    sc.tile_m = ffn_tile_m(cfg);
     sc.b_e = b_e_inout;
     if ((err = launch_scan(sc, s)) != cudaSuccess) return cuda_fail(err);
-    ScatterArgs sa{ids, hist, nullptr, inv, cfg->N, cfg->E, cfg->k};
+    ScatterArgs sa{ids, hist, nullptr, inv, cfg->N, cfg->E, cfg->k, offsets};
     if ((err = launch_scatter(sa, s)) != cudaSuccess) return cuda_fail(err);
     GatherArgs ga{x, inv, xs, cfg->N, cfg->d_model, cfg->k};
     if ((err = launch_gather(cfg->dtype, ga, num_sms(), s)) != cudaSuccess) return cuda_fail(err);
