@@ -363,21 +363,32 @@ def run_native(args, wl):
         gemm1_flops = 2 * (2 if wl.act == "swiglu" else 1) * wl.d_model * wl.d_ff * wl.N * wl.k
         gemm1_s = stages["gemm1"] / 1000.0
         ffn_s = (stages["gemm1"] + stages["gemm2"]) / 1000.0
-        bf16_peak = peaks["bf16_tflops"]
+        # the GEMM is timed inside a run of back-to-back steps (the power cap
+        # engages within it), so the denominator is the sustained bf16 peak;
+        # the burst fraction is reported beside it
+        burst = peaks["bf16_tflops"]
+        sustained = peaks.get("bf16_tflops_sustained", burst)
         achieved = gemm1_flops / gemm1_s / 1e12
+        ffn_tflops = wl.expert_flops / ffn_s / 1e12
+        fp32 = wl.dtype == "f32"
+        kern = ("simt_gemm_kernel<GELU>" if fp32 else
+                ("ffn_gemm_pair_kernel" if wl.N * wl.k / wl.E > 192 else "ffn_gemm_single_kernel") +
+                ("<SwiGLU>" if wl.act == "swiglu" else "<GELU>")) + " (GEMM1)"
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
             "config": dict(describe(wl), l2=("inputs larger than L2 (expert weights %.2f GB)" % (weights_bytes(wl) / 1e9))
                            if big_inputs else "L2 flushed between steps (256 MiB write), per-step events"),
-            "roofline": {"kernel": "ffn_gemm_kernel<SwiGLU> (GEMM1)" if wl.act == "swiglu" else "ffn_gemm_kernel<GELU> (GEMM1)",
-                         "bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
-                         "frac": achieved / bf16_peak, "peak_source": f"{peak_src} bf16_tflops (burst)",
+            "roofline": {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": sustained,
+                         "unit": "TFLOP/s", "frac": achieved / sustained,
+                         "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a run of steps)",
+                         "frac_of_burst_peak": achieved / burst,
                          "traffic": traffic_for("gemm1", wl.name), "flops_per_launch": gemm1_flops},
-            "expert_ffn": {"tflops": wl.expert_flops / ffn_s / 1e12,
-                           "frac_of_measured_peak": wl.expert_flops / ffn_s / 1e12 / bf16_peak,
-                           "frac_of_datasheet_2250": wl.expert_flops / ffn_s / 1e12 / 2250.0},
+            "expert_ffn": {"tflops": ffn_tflops,
+                           "frac_of_measured_sustained": ffn_tflops / sustained,
+                           "frac_of_measured_burst": ffn_tflops / burst,
+                           "frac_of_datasheet_2250": ffn_tflops / 2250.0},
             "stages_ms": stages,
             "e2e": {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s",
                     "h2d_bytes_per_step": inp["x"].numel() * inp["x"].element_size(),

@@ -5,11 +5,12 @@
 // The stable sort of assignments a = n k + j by expert is a counting sort
 // over fixed chunks of 32 tokens:
 //   1. per-chunk expert histograms (from the router, or from the ids),
-//   2. one CTA scans them: counts, offsets = exclusive prefix of counts,
-//      and for every (chunk, expert) the first sorted position the chunk
-//      owns inside that expert's slice,
+//   2. one CTA per expert scans its column over the chunks: for every
+//      (chunk, expert) the first position the chunk owns inside the expert's
+//      slice, and the expert's count; one more CTA turns the counts into
+//      offsets = exclusive prefix (slice starts),
 //   3. each chunk ranks its own assignments in assignment order, so
-//      position = chunk base + rank is the stable order,
+//      position = offsets[e] + chunk base + rank is the stable order,
 //   4. rows are copied x -> x_sorted with 16-byte vectors, one warp per token
 //      (the token row is read once and written k times).
 // Every reduction runs in a fixed order, so results are bitwise repeatable.
@@ -122,10 +123,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_cols_kernel(ScanArgs a)
 // sign(N k - E count_e) (sec. 2.5).
 __global__ void __launch_bounds__(kScanThreads) scan_finalize_kernel(ScanArgs a)
 {
-    __shared__ int cnt_s[kMaxE];
     const int E = a.E, t = threadIdx.x;
     const int cnt = t < E ? a.offsets[t + 1] : 0;
-    if (t < E) cnt_s[t] = cnt;
     int total, mt_total;
     const int off = block_exclusive_scan(cnt, &total);
     const int mt = (t < E && a.mt_prefix) ? (cnt + a.tile_m - 1) / a.tile_m : 0;
@@ -142,14 +141,24 @@ __global__ void __launch_bounds__(kScanThreads) scan_finalize_kernel(ScanArgs a)
     if (t == 0) {
         a.offsets[E] = total;
         if (a.mt_prefix) a.mt_prefix[E] = mt_total;
-        if (a.aux_out && a.psum && a.pe) {
+    }
+    if (a.aux_out && a.psum && a.pe) {
+        // L = E / N^2 * sum_e count_e (N P_e): one term per thread, summed in a
+        // fixed tree (warp butterflies, then the 8 warp sums in order)
+        __shared__ double wsum[kScanThreads / 32];
+        double term = t < E ? static_cast<double>(cnt) * a.pe[t] : 0.0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) term += __shfl_xor_sync(0xffffffffu, term, o);
+        if ((t & 31) == 0) wsum[t >> 5] = term;
+        __syncthreads();
+        if (t == 0) {
             if (a.N == 0) {
                 *a.aux_out = 0.0f;  // no tokens: every sum is empty
             } else {
+                double s = 0.0;
+                for (int w = 0; w < kScanThreads / 32; ++w) s += wsum[w];
                 const double Nd = static_cast<double>(a.N);
-                double L = 0.0;
-                for (int q = 0; q < E; ++q) L += (static_cast<double>(cnt_s[q]) / Nd) * (a.pe[q] / Nd);
-                *a.aux_out = static_cast<float>(L * static_cast<double>(E));
+                *a.aux_out = static_cast<float>(s * static_cast<double>(E) / (Nd * Nd));
             }
         }
     }

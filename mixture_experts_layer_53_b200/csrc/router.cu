@@ -164,13 +164,25 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
     const int ntok = static_cast<int>(min64(kRT, a.N - tok0));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     SelectArgs sa{a.b_sel, a.ids, a.w, a.probs, E, k, a.router, a.norm_topk, a.scaling};
+    // software pipeline: the next token's row is loaded while this one is
+    // selected (one copy of the selection code)
+    float znext[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int e = lane + 32 * j;
+        znext[j] = (warp < ntok && j < EJ && e < E) ? a.logits[(tok0 + warp) * a.ld + e] : 0.f;
+    }
+#pragma unroll 1
     for (int t = warp; t < ntok; t += kSelWarps) {
         const int64_t n = tok0 + t;
         float z[8];
 #pragma unroll
+        for (int j = 0; j < 8; ++j) z[j] = znext[j];
+        const int tn = t + kSelWarps;
+#pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int e = lane + 32 * j;
-            z[j] = (j < EJ && e < E) ? a.logits[n * a.ld + e] : 0.f;
+            znext[j] = (tn < ntok && j < EJ && e < E) ? a.logits[(tok0 + tn) * a.ld + e] : 0.f;
         }
         int sel_ids[kMaxK];
         select_token(z, sa, n, true, sel_ids);

@@ -74,40 +74,47 @@ __device__ __forceinline__ void select_token(float (&z)[8], const SelectArgs &a,
     for (int o = 16; o > 0; o >>= 1) esum += __shfl_xor_sync(0xffffffffu, esum, o);
     const float inv_esum = 1.0f / esum;
 
-    // k rounds of a warp argmax under the (score desc, id asc) order
+    // k rounds of a warp argmax under the (score desc, id asc) order.  The
+    // round loop stays rolled (small code); results land in the register
+    // arrays through static-index selects.
     uint32_t taken = 0;
     float gsel[kMaxK];
 #pragma unroll
     for (int r = 0; r < kMaxK; ++r) {
         sel_ids[r] = 0;
         gsel[r] = 0.f;
-        if (r < k) {
-            float bv = -FLT_MAX, bg = 0.f;
-            int be = INT_MAX;
+    }
+#pragma unroll 1
+    for (int r = 0; r < k; ++r) {
+        float bv = -FLT_MAX, bg = 0.f;
+        int be = INT_MAX;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int e = lane + 32 * j;
-                if (j < EJ && e < E && !((taken >> j) & 1u) && rank_ahead(sel[j], e, bv, be)) {
-                    bv = sel[j];
-                    be = e;
-                    bg = graw[j];
-                }
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane + 32 * j;
+            if (j < EJ && e < E && !((taken >> j) & 1u) && rank_ahead(sel[j], e, bv, be)) {
+                bv = sel[j];
+                be = e;
+                bg = graw[j];
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                const float og = __shfl_xor_sync(0xffffffffu, bg, o);
-                if (rank_ahead(ov, oe, bv, be)) {
-                    bv = ov;
-                    be = oe;
-                    bg = og;
-                }
-            }
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            sel_ids[r] = be;
-            gsel[r] = bg;
         }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            const float og = __shfl_xor_sync(0xffffffffu, bg, o);
+            if (rank_ahead(ov, oe, bv, be)) {
+                bv = ov;
+                be = oe;
+                bg = og;
+            }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+            if (j == r) {
+                sel_ids[j] = be;
+                gsel[j] = bg;
+            }
     }
 
     float gs = 0.f;
