@@ -71,6 +71,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.oracle_aux_loss.restype = f64
     lib.oracle_bias_update.argtypes = [i64, i32, i32, _ip, f64, _dp]
     lib.oracle_bias_update.restype = None
+    lib.oracle_z_loss.argtypes = [i64, i32, _dp]
+    lib.oracle_z_loss.restype = f64
+    lib.oracle_shared_add.argtypes = [i64, i32, i32, i32, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
+    lib.oracle_shared_add.restype = i32
     return lib
 
 
@@ -245,6 +249,33 @@ def bias_update(b, counts, N: int, k: int, gamma: float,
     out = _f64(b).copy()
     counts = _i32(counts)
     L.oracle_bias_update(N, out.shape[0], k, _p(counts, _ip), float(gamma), _p(out, _dp))
+    return out
+
+
+def z_loss(logits, L: Optional[ctypes.CDLL] = None) -> float:
+    """Router z-loss: mean over tokens of (logsumexp of the logits)^2."""
+    L = L or lib()
+    z = _f64(logits)
+    N, E = z.shape
+    return float(L.oracle_z_loss(N, E, _p(z, _dp)))
+
+
+def shared_add(y, x, Ws1, Ws2, act="swiglu", Ws3=None, bs1=None, bs2=None,
+               L: Optional[ctypes.CDLL] = None) -> np.ndarray:
+    """Return y + Shared(x) (row by row); Ws1/Ws3 [Fs,d], Ws2 [d,Fs]."""
+    L = L or lib()
+    out = _f64(y).copy()
+    x = _f64(x)
+    Ws1 = _f64(Ws1)
+    Ws2 = _f64(Ws2)
+    Ws3 = None if Ws3 is None else _f64(Ws3)
+    bs1 = None if bs1 is None else _f64(bs1)
+    bs2 = None if bs2 is None else _f64(bs2)
+    N, d = x.shape
+    Fs = Ws1.shape[0]
+    rc = L.oracle_shared_add(N, d, Fs, ACTS[act], _p(x, _dp), _p(Ws1, _dp), _p(bs1, _dp), _p(Ws3, _dp),
+                             _p(Ws2, _dp), _p(bs2, _dp), _p(out, _dp))
+    _check(rc, "oracle_shared_add")
     return out
 
 

@@ -428,3 +428,50 @@ void oracle_bias_update(int64_t N, int E, int k, const int32_t *counts,
         b[e] += gamma * (double)s;
     }
 }
+
+/* ------------------------------------------------------ router z-loss, shared */
+
+/*
+ * Router z-loss ("nano-moe", "Router z-loss"; RustingBrain tutorial chapter
+ * "Mixture of Experts", sec. 15.3 "The z-loss"): the mean over tokens of the squared log-sum-exp of the
+ * router logits, (1/N) sum_n (log sum_e exp z_{n,e})^2.  logits is [N, E].
+ */
+double oracle_z_loss(int64_t N, int E, const double *logits)
+{
+    if (N <= 0 || E < 1) return N == 0 ? 0.0 : NAN;
+    double total = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+        const double *z = logits + n * E;
+        double zmax = z[0];
+        for (int e = 1; e < E; ++e) if (z[e] > zmax) zmax = z[e];
+        double s = 0.0;
+        for (int e = 0; e < E; ++e) s += exp(z[e] - zmax);
+        const double lse = zmax + log(s);
+        total += lse * lse;
+    }
+    return total / (double)N;
+}
+
+/*
+ * Shared expert (course module sec. 2.1: y_n = sum_{e in T_n} w_{n,e}
+ * Expert_e(x_n) + Shared(x_n); S shared experts of width f act as one FFN of
+ * width S f; RustingBrain chapter sec. 15.4 "The shared expert"): adds Shared(x_n) to y_n for every token, after the routed sum.
+ * Ws1/Ws3 are [Fs, d], Ws2 [d, Fs]; bs1 [Fs] (GELU only) and bs2 [d] may be
+ * NULL.
+ */
+int oracle_shared_add(int64_t N, int d, int Fs, int act, const double *x,
+                      const double *Ws1, const double *bs1, const double *Ws3,
+                      const double *Ws2, const double *bs2, double *y)
+{
+    if (N < 0 || d < 1 || Fs < 1) return ORC_ERR_ARG;
+    if (act == ORC_SWIGLU && !Ws3) return ORC_ERR_ARG;
+    double *h = malloc(sizeof(double) * Fs);
+    double *o = malloc(sizeof(double) * d);
+    if (!h || !o) { free(h); free(o); return ORC_ERR_ARG; }
+    for (int64_t n = 0; n < N; ++n) {
+        oracle_expert_ffn(d, Fs, act, x + n * d, Ws1, bs1, Ws3, Ws2, bs2, h, o);
+        for (int c = 0; c < d; ++c) y[n * d + c] += o[c];
+    }
+    free(h); free(o);
+    return ORC_OK;
+}

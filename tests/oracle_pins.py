@@ -410,4 +410,47 @@ def pin_rejects_bad_ids(L):
         raise AssertionError("dispatch accepted an expert id >= E")
 
 
+
+
+def pin_z_loss_closed_forms(L):
+    """Router z-loss = mean_n (logsumexp z_n)^2 ("nano-moe", router z-loss)."""
+    for E in (1, 4, 8):
+        _close(O.z_loss(np.zeros((5, E)), L=L), math.log(E) ** 2, 1e-14, f"zero logits, E={E}")
+    g = _golden("course_worked_example.json")
+    z = np.log(np.array([[float(v) for v in row] for row in g["logits_ln"]]))
+    # token 0: sum q = 8, token 1: sum q = 9
+    _close(O.z_loss(z, L=L), (math.log(8) ** 2 + math.log(9) ** 2) / 2, 1e-14, "worked-example logits")
+    zz = np.array([[1.5], [-2.0], [0.25]])
+    _close(O.z_loss(zz, L=L), float(np.mean(zz[:, 0] ** 2)), 1e-14, "one expert: lse = z")
+    rng = np.random.default_rng(31)
+    z = rng.standard_normal((6, 5)) * 3
+    lse = np.log(np.sum(np.exp(z), axis=1))
+    _close(O.z_loss(z + 7.0, L=L), float(np.mean((lse + 7.0) ** 2)), 1e-12, "shift by c moves lse by c")
+
+
+def pin_shared_expert_numpy(L):
+    """y_n = sum_j w_j Expert_j(x_n) + Shared(x_n) (course module sec. 2.1)."""
+    rng = np.random.default_rng(37)
+    for act, biases in (("swiglu", False), ("gelu", True)):
+        N, d, F, Fs, E, k = 7, 6, 9, 12, 4, 2
+        x, Wg, W1, W2, W3, b1, b2 = _rand_problem(rng, N, d, F, E, act, biases)
+        Ws1 = rng.standard_normal((Fs, d)) / math.sqrt(d)
+        Ws2 = rng.standard_normal((d, Fs)) / math.sqrt(Fs)
+        Ws3 = rng.standard_normal((Fs, d)) / math.sqrt(d) if act == "swiglu" else None
+        bs1 = rng.standard_normal(Fs) * 0.1 if biases else None
+        bs2 = rng.standard_normal(d) * 0.1 if biases else None
+        r = O.route(x, Wg, k, routed_scaling=2.5, L=L)
+        y = O.dense_forward(x, r["ids"], r["w"], W1, W2, act, W3, b1, b2, L=L)
+        y = O.shared_add(y, x, Ws1, Ws2, act, Ws3, bs1, bs2, L=L)
+        ref = sum(r["w"][:, j:j + 1] * np.stack([np_expert(x[n:n + 1], W1[r["ids"][n, j]], W2[r["ids"][n, j]],
+                                                           act, None if W3 is None else W3[r["ids"][n, j]],
+                                                           None if b1 is None else b1[r["ids"][n, j]],
+                                                           None if b2 is None else b2[r["ids"][n, j]])[0]
+                                                 for n in range(N)]) for j in range(k))
+        ref = ref + np_expert(x, Ws1, Ws2, act, Ws3, bs1, bs2)  # shared part carries no weight
+        _close(y, ref, 1e-12, f"routed sum + shared expert ({act})")
+    z = O.shared_add(np.ones((3, 4)), rng.standard_normal((3, 4)), np.zeros((5, 4)), np.zeros((4, 5)), "gelu", L=L)
+    _close(z, np.ones((3, 4)), 0.0, "zero shared expert adds nothing")
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

@@ -50,6 +50,9 @@ MUTANTS = {
     "softmax_no_normalise": ("for (int e = 0; e < E; ++e) p[e] /= denom;", ""),
     "wrong_expert_block": ("oracle_expert_ffn(d, F, act, xrow, W1 + (int64_t)e * F * d,",
                            "oracle_expert_ffn(d, F, act, xrow, W1 + (int64_t)(e ^ 1) * F * d,"),
+    "z_loss_not_squared": ("total += lse * lse;", "total += lse;"),
+    "z_loss_no_max_shift": ("const double lse = zmax + log(s);", "const double lse = log(s);"),
+    "shared_not_added": ("for (int c = 0; c < d; ++c) y[n * d + c] += o[c];", "for (int c = 0; c < d; ++c) y[n * d + c] = o[c];"),
     "combine_drops_last_slot": ("for (int j = 0; j < k; ++j) {\n            const double *src",
                                 "for (int j = 0; j + 1 < k; ++j) {\n            const double *src"),
 }
