@@ -33,9 +33,11 @@ METRIC = "MoE-layer tokens/sec (bf16, 1 B200); expert-GEMM TFLOPS as % of bf16 p
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
 # tokens of the workload the CPU oracle handles per reference step (about 1-3 s each)
-REF_TOKENS_PER_STEP = {"tiny_fp32": 64, "gpt2_moe": 32, "mixtral": 1, "deepseek_v3": 1, "qwen3_skew": 8}
+REF_TOKENS_PER_STEP = {"tiny_fp32": 64, "gpt2_moe": 32, "mixtral": 1, "deepseek_v3": 1, "qwen3_skew": 8,
+                       "deepseek_v3_shared": 1}
 # libmoe kernels per forward: router logits + selection (bf16; one fused router
-# kernel for fp32), scan, scatter, gather, GEMM1, GEMM2, combine
+# kernel for fp32), scan, scatter, gather, GEMM1, GEMM2, combine; a shared
+# expert adds its two GEMMs
 KERNELS_PER_STEP = {"bf16": 8, "f32": 7}
 
 
@@ -183,6 +185,9 @@ class OracleSample:
         self.Wg = r["W_g"].float().numpy().astype(np.float64)
         self.b = None if r["b_e"] is None else r["b_e"].numpy().astype(np.float64)
         self.L = O.lib()
+        sh = W.make_shared(wl)
+        self.shared = None if sh is None else {
+            k: (None if v is None else v.float().numpy().astype(np.float64)) for k, v in sh.items()}
         self.cache = {}
         self.cache_bytes = cache_bytes
 
@@ -213,6 +218,11 @@ class OracleSample:
                 t0 = time.perf_counter()
                 o = O.expert_ffn(x[s], ew["W1"], ew["W2"], wl.act, ew["b1"], ew["W3"], ew["b2"], L=self.L)
                 y += rt["w"][s, j] * o
+                spent += time.perf_counter() - t0
+            if self.shared is not None:
+                sw = self.shared
+                t0 = time.perf_counter()
+                y += O.expert_ffn(x[s], sw["W1"], sw["W2"], wl.act, sw["b1"], sw["W3"], sw["b2"], L=self.L)
                 spent += time.perf_counter() - t0
         return spent
 
@@ -278,7 +288,7 @@ def run_native(args, wl):
 
     M.library()
     cfg = M.make_config(wl.N, wl.d_model, wl.d_ff, wl.E, wl.k, wl.router, wl.norm_topk, wl.routed_scaling,
-                        wl.act, wl.dtype)
+                        wl.act, wl.dtype, wl.d_ff_shared)
     inp = W.make_inputs(wl.scaled(seed=wl.seed + 100 * rank) if rank else wl, dev)
     ws = M.workspace(cfg, dev)
     out = M.forward_outputs(cfg, dev)
@@ -289,7 +299,7 @@ def run_native(args, wl):
 
     def step(events=None):
         M.moe_forward(cfg, inp["x"], inp["W_g"], inp["W1"], inp["W2"], W3=inp["W3"], b1=inp["b1"], b2=inp["b2"],
-                      b_e=b_e, gamma=wl.gamma, ws=ws, out=out, stage_events=events)
+                      b_e=b_e, gamma=wl.gamma, ws=ws, out=out, stage_events=events, shared=inp["shared"])
 
     def barrier():
         if world > 1:
@@ -328,30 +338,32 @@ def run_native(args, wl):
             stages[k] += v / args.steps
     total_ms = max_over_ranks(local_ms, world, dev)
 
-    # end to end through the public call with host buffers: H2D of x, the
-    # forward, D2H of y and of the loss, every step
+    # end to end through the public call with host buffers: every step uploads
+    # its x from pinned host memory, runs the layer and downloads y and the
+    # loss; M.HostPipeline overlaps one step's copies with the neighbouring
+    # steps' forwards (upload and download streams, double-buffered tensors).
+    # The timed region starts before the first upload and ends after the last
+    # download (both joined to the compute stream).
     x_host = inp["x"].cpu().pin_memory()
     y_host = torch.empty_like(out["y"], device="cpu").pin_memory()
     aux_host = torch.empty(1, dtype=torch.float32).pin_memory()
-    x_dev = torch.empty_like(inp["x"])
-
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        M.moe_forward(cfg, x_dev, inp["W_g"], inp["W1"], inp["W2"], W3=inp["W3"], b1=inp["b1"], b2=inp["b2"],
-                      b_e=b_e, gamma=wl.gamma, ws=ws, out=out)
-        y_host.copy_(out["y"], non_blocking=True)
-        aux_host.copy_(out["aux"], non_blocking=True)
-
+    weights = {k: inp[k] for k in ("W_g", "W1", "W2", "W3", "b1", "b2")}
+    weights["b_e"] = b_e
+    weights["shared"] = inp["shared"]
+    pipe = M.HostPipeline(cfg, weights, gamma=wl.gamma, device=dev)
     for _ in range(max(1, args.warmup)):
-        e2e_step()
+        pipe.step(x_host, y_host, aux_host)
+    pipe.finish()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    pipe.upload.wait_stream(stream)
     for i in range(args.steps):
         if flush is not None:
             flush.fill_(i & 0xFF)
-        e2e_step()
+        pipe.step(x_host, y_host, aux_host)
+    stream.wait_stream(pipe.download)
     e1.record(stream)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
@@ -393,7 +405,7 @@ def run_native(args, wl):
             "e2e": {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s",
                     "h2d_bytes_per_step": inp["x"].numel() * inp["x"].element_size(),
                     "d2h_bytes_per_step": out["y"].numel() * out["y"].element_size() + 4},
-            "gpu_launches": KERNELS_PER_STEP[wl.dtype] * args.steps,
+            "gpu_launches": (KERNELS_PER_STEP[wl.dtype] + (2 if wl.d_ff_shared else 0)) * args.steps,
             "clocks": clocks.summary(),
         }
         if not args.no_cpu_baseline and world == 1:

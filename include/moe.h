@@ -97,13 +97,33 @@ typedef struct {
     float routed_scaling; /* every weight is multiplied by it (1.0 = off) */
     int32_t act;          /* moe_act */
     int32_t dtype;        /* moe_dtype */
+    int32_t d_ff_shared;  /* hidden width of the shared expert; 0 = none */
 } moe_config;
+
+/*
+ * Weights of the shared expert, the FFN every token passes through besides
+ * its k routed experts (course module sec. 2.1: y_n = sum_{e in T_n}
+ * w_{n,e} Expert_e(x_n) + Shared(x_n); S shared experts of width f are one
+ * FFN of width S f; RustingBrain chapter "Mixture of Experts", sec. 15.4).
+ * It has the routed experts' activation and dtype and width cfg->d_ff_shared
+ * (Fs): W1 and W3 [Fs, d_model], W2 [d_model, Fs], row-major; b1 [Fs]
+ * (GELU only) and b2 [d_model] may be NULL, W3 is SwiGLU only.  Its output
+ * carries no gate weight and no routed_scaling.  Device pointers, 16-byte
+ * aligned, owned by the caller.
+ */
+typedef struct {
+    const void *W1;
+    const void *b1;
+    const void *W3;
+    const void *W2;
+    const void *b2;
+} moe_shared_expert;
 
 /* Stage boundaries recorded by moe_forward when stage_events is given. */
 #define MOE_STAGE_ROUTE 0    /* router GEMM + scores + top-k + gates */
 #define MOE_STAGE_DISPATCH 1 /* counts/offsets/loss/bias rule, scatter, row gather */
 #define MOE_STAGE_GEMM1 2    /* x_sorted -> h (first expert GEMM + activation) */
-#define MOE_STAGE_GEMM2 3    /* h -> y_sorted (second expert GEMM + bias) */
+#define MOE_STAGE_GEMM2 3    /* h -> y_sorted (second expert GEMM + bias), then the shared expert's FFN */
 #define MOE_STAGE_COMBINE 4  /* weighted sum back in token order */
 #define MOE_NUM_STAGES 5
 
@@ -212,6 +232,42 @@ MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_sorted,
                        moe_stream_t stream);
 
 /*
+ * Shared expert over all N tokens (see moe_shared_expert):
+ * y_shared[n] = Shared(x[n]), [N, d_model] in cfg->dtype, on the same
+ * grouped-GEMM kernels as the routed experts (one slice of N rows).  Needs
+ * cfg->d_ff_shared > 0; the hidden activations live in the workspace.
+ */
+MOE_API moe_status moe_shared_ffn(const moe_config *cfg, const void *x,
+                          const moe_shared_expert *shared, void *y_shared,
+                          int32_t *dev_status, void *ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
+/*
+ * moe_combine plus the shared expert's output: y_n = sum_{j<k} topk_w[n, j]
+ * * y_sorted[inv_perm[n*k + j]] + y_shared[n] (course module sec. 2.1), with
+ * the shared row added after the routed sum, in fp32.  y_shared NULL gives
+ * moe_combine.  Needs no workspace.
+ */
+MOE_API moe_status moe_combine_shared(const moe_config *cfg, const void *y_sorted,
+                              const float *topk_w, const int32_t *inv_perm,
+                              const void *y_shared, void *y,
+                              moe_stream_t stream);
+
+/*
+ * Router z-loss ("nano-moe", "Router z-loss"; RustingBrain chapter sec. 15.3
+ * "The z-loss"): z = (1/N) sum_n (log sum_e exp z_{n,e})^2 over the router
+ * logits z_n = W_g x_n, written as float to the device scalar z_loss_out
+ * (per-token terms in fp32, summed in fp64 in a fixed order; 0 for N = 0).
+ * The raw value: the loss coefficient is the caller's.  Recomputes the
+ * routing into the workspace; moe_forward_ex returns the same value from its
+ * own routing pass at almost no cost.
+ */
+MOE_API moe_status moe_router_z_loss(const moe_config *cfg, const void *x,
+                             const void *W_g, float *z_loss_out,
+                             int32_t *dev_status, void *ws, size_t ws_bytes,
+                             moe_stream_t stream);
+
+/*
  * Switch load-balance loss: course module sec. 2.3 and the sec. 4
  * load_balance_loss:  L = E * sum_e f_e P_e with f_e = (assignments to e)/N
  * and P_e = mean_n probs[n, e]; written as float to the device scalar
@@ -227,8 +283,8 @@ MOE_API moe_status moe_aux_loss(const moe_config *cfg, const float *probs,
                         moe_stream_t stream);
 
 /*
- * The whole layer forward (course module sec. 4 MoE.forward, no shared
- * expert): route -> dispatch -> expert FFNs -> combine, plus the Switch loss
+ * The whole layer forward (course module sec. 4 MoE.forward; the shared
+ * expert and the z-loss are in moe_forward_ex): route -> dispatch -> expert FFNs -> combine, plus the Switch loss
  * (aux_out, may be NULL) and the assignment counts (counts, may be NULL; the
  * sec. 4 expert_load).  If gamma > 0 and b_e_inout is given (sigmoid
  * router), b_e is used for this forward's selection and then moved by one
@@ -245,6 +301,24 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const void 
                        float *topk_w, int32_t *counts, float *aux_out,
                        int32_t *dev_status, void *ws, size_t ws_bytes,
                        void *const *stage_events, moe_stream_t stream);
+
+/*
+ * moe_forward with the shared expert and the router z-loss (course module
+ * sec. 2.1; "nano-moe", "Router z-loss").  shared (NULL iff
+ * cfg->d_ff_shared == 0) adds Shared(x_n) to every output row after the
+ * routed sum; z_loss_out (may be NULL) receives the router z-loss as in
+ * moe_router_z_loss, taken from this forward's routing pass.  Every other
+ * argument is that of moe_forward, which is this call with shared and
+ * z_loss_out NULL (and rejects cfg->d_ff_shared > 0).
+ */
+MOE_API moe_status moe_forward_ex(const moe_config *cfg, const void *x, const void *W_g,
+                          float *b_e_inout, float gamma, const void *W1,
+                          const void *b1, const void *W3, const void *W2,
+                          const void *b2, const moe_shared_expert *shared,
+                          void *y, int32_t *topk_ids, float *topk_w,
+                          int32_t *counts, float *aux_out, float *z_loss_out,
+                          int32_t *dev_status, void *ws, size_t ws_bytes,
+                          void *const *stage_events, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -8,7 +8,10 @@ functions.  If the library is missing, every call raises.
 
 The functions carry the names of the C entry points in ``include/moe.h``:
 ``moe_route``, ``moe_dispatch``, ``moe_expert_ffn``, ``moe_combine``,
-``moe_aux_loss``, ``moe_forward`` and ``moe_workspace_size``.  Symbols follow
+``moe_aux_loss``, ``moe_forward`` and ``moe_workspace_size``, plus the
+shared expert (``moe_shared_ffn``, ``moe_combine_shared``) and the router
+z-loss (``moe_router_z_loss``; ``moe_forward`` with ``shared=`` or
+``z_loss=True`` calls ``moe_forward_ex``).  Symbols follow
 the course module "Mixture of Experts: routing, sorted dispatch, Switch aux
 loss, aux-free bias" (sec. 2): N, E, k, d_model, d_ff, W_g, b_e.
 """
@@ -33,7 +36,7 @@ NUM_STAGES = 5
 STAGE_NAMES = ("route", "dispatch", "gemm1", "gemm2", "combine")
 EXPORTS = ("moe_status_string", "moe_last_error", "moe_version", "moe_workspace_size", "moe_route",
            "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_combine", "moe_aux_loss",
-           "moe_forward")
+           "moe_forward", "moe_shared_ffn", "moe_combine_shared", "moe_router_z_loss", "moe_forward_ex")
 # ceil(N / 32) * E limit of moe_dispatch_noalloc (MOE_NOALLOC_DISPATCH_MAX_SLOTS)
 NOALLOC_DISPATCH_MAX_SLOTS = 1 << 19
 
@@ -43,11 +46,17 @@ class MoeConfig(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("d_model", ctypes.c_int32), ("d_ff", ctypes.c_int32),
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("router", ctypes.c_int32),
                 ("norm_topk", ctypes.c_int32), ("routed_scaling", ctypes.c_float),
-                ("act", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+                ("act", ctypes.c_int32), ("dtype", ctypes.c_int32), ("d_ff_shared", ctypes.c_int32)]
 
     @property
     def torch_dtype(self) -> torch.dtype:
         return torch.float32 if self.dtype == 0 else torch.bfloat16
+
+
+class SharedExpert(ctypes.Structure):
+    """Mirror of ``moe_shared_expert`` in include/moe.h (device pointers)."""
+    _fields_ = [("W1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("W3", ctypes.c_void_p),
+                ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p)]
 
 
 class MoeError(RuntimeError):
@@ -96,6 +105,16 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_forward.argtypes = [cfgp, vp, vp, f32p, ctypes.c_float, vp, vp, vp, vp, vp, vp, i32p, f32p, i32p,
                                 f32p, i32p, vp, sz, ctypes.c_void_p, vp]
     lib.moe_forward.restype = st
+    shp = ctypes.POINTER(SharedExpert)
+    lib.moe_shared_ffn.argtypes = [cfgp, vp, shp, vp, i32p, vp, sz, vp]
+    lib.moe_shared_ffn.restype = st
+    lib.moe_combine_shared.argtypes = [cfgp, vp, f32p, i32p, vp, vp, vp]
+    lib.moe_combine_shared.restype = st
+    lib.moe_router_z_loss.argtypes = [cfgp, vp, vp, f32p, i32p, vp, sz, vp]
+    lib.moe_router_z_loss.restype = st
+    lib.moe_forward_ex.argtypes = [cfgp, vp, vp, f32p, ctypes.c_float, vp, vp, vp, vp, vp, shp, vp, i32p, f32p,
+                                   i32p, f32p, f32p, i32p, vp, sz, ctypes.c_void_p, vp]
+    lib.moe_forward_ex.restype = st
     if path is None:
         _lib = lib
     return lib
@@ -103,9 +122,9 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
 
 def make_config(N: int, d_model: int, d_ff: int, E: int, k: int, router: str = "softmax_topk",
                 norm_topk: bool = True, routed_scaling: float = 1.0, act: str = "gelu",
-                dtype: str = "bf16") -> MoeConfig:
+                dtype: str = "bf16", d_ff_shared: int = 0) -> MoeConfig:
     return MoeConfig(int(N), int(d_model), int(d_ff), int(E), int(k), ROUTERS[router], int(bool(norm_topk)),
-                     float(routed_scaling), ACTS[act], DTYPES[dtype])
+                     float(routed_scaling), ACTS[act], DTYPES[dtype], int(d_ff_shared))
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -227,6 +246,49 @@ def moe_combine(cfg: MoeConfig, y_sorted: torch.Tensor, topk_w: torch.Tensor, in
     return y
 
 
+def _shared_struct(shared: Optional[Dict[str, Optional[torch.Tensor]]]):
+    """SharedExpert from {"W1", "W2", "W3"?, "b1"?, "b2"?} (None -> None)."""
+    if shared is None:
+        return None
+    ptr = lambda key: _ptr(shared.get(key)).value if shared.get(key) is not None else None
+    return SharedExpert(ptr("W1"), ptr("b1"), ptr("W3"), ptr("W2"), ptr("b2"))
+
+
+def moe_shared_ffn(cfg: MoeConfig, x: torch.Tensor, shared: Dict[str, Optional[torch.Tensor]],
+                   ws: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """y_shared [N, d_model] = Shared(x) (weights W1, W2 and W3 / b1 / b2 as the activation needs)."""
+    dev = x.device
+    ws = ws if ws is not None else workspace(cfg, dev)
+    y_shared = torch.empty((cfg.N, cfg.d_model), dtype=cfg.torch_dtype, device=dev)
+    sh = _shared_struct(shared)
+    rc = library().moe_shared_ffn(ctypes.byref(cfg), _ptr(x), ctypes.byref(sh), _ptr(y_shared), _ptr(status),
+                                  _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "moe_shared_ffn")
+    return y_shared
+
+
+def moe_combine_shared(cfg: MoeConfig, y_sorted: torch.Tensor, topk_w: torch.Tensor, inv_perm: torch.Tensor,
+                       y_shared: Optional[torch.Tensor], stream=None) -> torch.Tensor:
+    y = torch.empty((cfg.N, cfg.d_model), dtype=cfg.torch_dtype, device=y_sorted.device)
+    rc = library().moe_combine_shared(ctypes.byref(cfg), _ptr(y_sorted), _ptr(topk_w), _ptr(inv_perm),
+                                      _ptr(y_shared), _ptr(y), _stream(stream))
+    _check(rc, "moe_combine_shared")
+    return y
+
+
+def moe_router_z_loss(cfg: MoeConfig, x: torch.Tensor, W_g: torch.Tensor, ws: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """Router z-loss [1] f32: mean over tokens of (logsumexp of the router logits)^2."""
+    dev = x.device
+    ws = ws if ws is not None else workspace(cfg, dev)
+    z = torch.empty(1, dtype=torch.float32, device=dev)
+    rc = library().moe_router_z_loss(ctypes.byref(cfg), _ptr(x), _ptr(W_g), _ptr(z), None, _ptr(ws), ws.numel(),
+                                     _stream(stream))
+    _check(rc, "moe_router_z_loss")
+    return z
+
+
 def moe_aux_loss(cfg: MoeConfig, probs: torch.Tensor, topk_ids: torch.Tensor, gamma: float = 0.0,
                  b_e: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
     """Returns (aux [1] f32, counts [E] int32, status [1] int32); updates b_e in place if gamma > 0."""
@@ -264,23 +326,92 @@ def moe_forward(cfg: MoeConfig, x: torch.Tensor, W_g: torch.Tensor, W1: torch.Te
                 W3: Optional[torch.Tensor] = None, b1: Optional[torch.Tensor] = None,
                 b2: Optional[torch.Tensor] = None, b_e: Optional[torch.Tensor] = None, gamma: float = 0.0,
                 ws: Optional[torch.Tensor] = None, out: Optional[Dict[str, torch.Tensor]] = None,
-                stage_events: Optional[StageEvents] = None, stream=None) -> Dict[str, torch.Tensor]:
-    """The whole layer: y, topk_ids, topk_w, counts, aux (Switch loss), status.
+                stage_events: Optional[StageEvents] = None, stream=None,
+                shared: Optional[Dict[str, Optional[torch.Tensor]]] = None,
+                z_loss: bool = False) -> Dict[str, torch.Tensor]:
+    """The whole layer: y, topk_ids, topk_w, counts, aux (Switch loss), z (z-loss), status.
 
     b_e (sigmoid router) selects only; with gamma > 0 it is moved in place by one
     sign-rule step after the selection.  ``out`` may hold preallocated outputs.
+    ``shared`` (weights W1, W2, W3 / b1 / b2 of width cfg.d_ff_shared) adds the
+    shared expert; ``z_loss`` fills out["z"] with the router z-loss.  Either
+    goes through moe_forward_ex, otherwise moe_forward.
     """
     dev = x.device
     ws = ws if ws is not None else workspace(cfg, dev)
     if out is None:
         out = forward_outputs(cfg, dev)
-    rc = library().moe_forward(ctypes.byref(cfg), _ptr(x), _ptr(W_g), _ptr(b_e), float(gamma), _ptr(W1), _ptr(b1),
-                               _ptr(W3), _ptr(W2), _ptr(b2), _ptr(out["y"]), _ptr(out["topk_ids"]),
-                               _ptr(out["topk_w"]), _ptr(out["counts"]), _ptr(out["aux"]), _ptr(out["status"]),
-                               _ptr(ws), ws.numel(), stage_events.pointer if stage_events else None,
-                               _stream(stream))
-    _check(rc, "moe_forward")
+    events = stage_events.pointer if stage_events else None
+    if shared is None and not z_loss:
+        rc = library().moe_forward(ctypes.byref(cfg), _ptr(x), _ptr(W_g), _ptr(b_e), float(gamma), _ptr(W1),
+                                   _ptr(b1), _ptr(W3), _ptr(W2), _ptr(b2), _ptr(out["y"]), _ptr(out["topk_ids"]),
+                                   _ptr(out["topk_w"]), _ptr(out["counts"]), _ptr(out["aux"]),
+                                   _ptr(out["status"]), _ptr(ws), ws.numel(), events, _stream(stream))
+        _check(rc, "moe_forward")
+        return out
+    sh = _shared_struct(shared)
+    rc = library().moe_forward_ex(ctypes.byref(cfg), _ptr(x), _ptr(W_g), _ptr(b_e), float(gamma), _ptr(W1),
+                                  _ptr(b1), _ptr(W3), _ptr(W2), _ptr(b2), ctypes.byref(sh) if sh else None,
+                                  _ptr(out["y"]), _ptr(out["topk_ids"]), _ptr(out["topk_w"]), _ptr(out["counts"]),
+                                  _ptr(out["aux"]), _ptr(out["z"]) if z_loss else None, _ptr(out["status"]),
+                                  _ptr(ws), ws.numel(), events, _stream(stream))
+    _check(rc, "moe_forward_ex")
     return out
+
+
+class HostPipeline:
+    """moe_forward over batches that live in pinned host memory.
+
+    Each call of ``step(x_host, y_host)`` uploads one batch, runs the layer and
+    downloads y (and the Switch loss).  Uploads and downloads run on two copy
+    streams of their own, double-buffered, so batch i+1's upload and batch
+    i-1's download overlap batch i's forward on the compute stream.
+    ``finish()`` waits for the last download.  Only torch copies and CUDA
+    events are added around the library call; the layer is ``moe_forward``.
+    """
+
+    def __init__(self, cfg: MoeConfig, weights: Dict[str, Optional[torch.Tensor]], gamma: float = 0.0,
+                 device=None):
+        self.cfg = cfg
+        self.w = weights
+        self.gamma = gamma
+        dev = torch.device(device or "cuda")
+        self.compute = torch.cuda.current_stream(dev)
+        self.upload = torch.cuda.Stream(dev)
+        self.download = torch.cuda.Stream(dev)
+        self.ws = workspace(cfg, dev)
+        self.x = [torch.empty((cfg.N, cfg.d_model), dtype=cfg.torch_dtype, device=dev) for _ in range(2)]
+        self.out = [forward_outputs(cfg, dev) for _ in range(2)]
+        self.uploaded = [torch.cuda.Event() for _ in range(2)]
+        self.computed = [torch.cuda.Event() for _ in range(2)]
+        self.downloaded = [torch.cuda.Event() for _ in range(2)]
+        self.i = 0
+
+    def step(self, x_host: torch.Tensor, y_host: torch.Tensor, aux_host: Optional[torch.Tensor] = None):
+        b = self.i & 1
+        with torch.cuda.stream(self.upload):
+            # x buffer b was last read by the forward of step i-2
+            self.upload.wait_event(self.computed[b])
+            self.x[b].copy_(x_host, non_blocking=True)
+            self.uploaded[b].record(self.upload)
+        self.compute.wait_event(self.uploaded[b])
+        self.compute.wait_event(self.downloaded[b])  # outputs of step i-2 are on the host
+        w = self.w
+        moe_forward(self.cfg, self.x[b], w["W_g"], w["W1"], w["W2"], W3=w.get("W3"), b1=w.get("b1"),
+                    b2=w.get("b2"), b_e=w.get("b_e"), gamma=self.gamma, ws=self.ws, out=self.out[b],
+                    stream=self.compute, shared=w.get("shared"))
+        self.computed[b].record(self.compute)
+        with torch.cuda.stream(self.download):
+            self.download.wait_event(self.computed[b])
+            y_host.copy_(self.out[b]["y"], non_blocking=True)
+            if aux_host is not None:
+                aux_host.copy_(self.out[b]["aux"], non_blocking=True)
+            self.downloaded[b].record(self.download)
+        self.i += 1
+
+    def finish(self):
+        for e in self.downloaded:
+            e.synchronize()
 
 
 def forward_outputs(cfg: MoeConfig, device) -> Dict[str, torch.Tensor]:
@@ -290,10 +421,12 @@ def forward_outputs(cfg: MoeConfig, device) -> Dict[str, torch.Tensor]:
         "topk_w": torch.empty((cfg.N, cfg.k), dtype=torch.float32, device=device),
         "counts": torch.empty(cfg.E, dtype=torch.int32, device=device),
         "aux": torch.empty(1, dtype=torch.float32, device=device),
+        "z": torch.empty(1, dtype=torch.float32, device=device),
         "status": torch.zeros(1, dtype=torch.int32, device=device),
     }
 
 
-__all__ = ["MoeConfig", "MoeError", "make_config", "library", "workspace", "moe_workspace_size", "moe_route",
-           "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_aux_loss", "moe_forward", "forward_outputs",
-           "StageEvents", "EXPORTS", "LIB_PATH"]
+__all__ = ["MoeConfig", "SharedExpert", "MoeError", "make_config", "library", "workspace", "moe_workspace_size",
+           "moe_route", "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_combine", "moe_aux_loss",
+           "moe_forward", "moe_shared_ffn", "moe_combine_shared", "moe_router_z_loss", "forward_outputs",
+           "StageEvents", "HostPipeline", "EXPORTS", "LIB_PATH"]

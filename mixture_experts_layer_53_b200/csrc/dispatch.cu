@@ -117,6 +117,46 @@ __global__ void __launch_bounds__(kScanThreads) scan_cols_kernel(ScanArgs a)
     if (threadIdx.x == 0) a.offsets[e + 1] = total;
 }
 
+// Router z-loss ("nano-moe", "Router z-loss"): (1/N) sum_n (lse z_n)^2 from
+// the per-chunk sums, reduced in fp64 in a fixed order (strided per-thread
+// sums, warp butterflies, then the warp sums in order).  Called by every
+// thread of a kScanThreads block.
+__device__ __forceinline__ void reduce_z_loss(const float *zpart, int64_t chunks, int64_t N, float *z_out)
+{
+    __shared__ double zsum[kScanThreads / 32];
+    double s = 0.0;
+    for (int64_t c = threadIdx.x; c < chunks; c += kScanThreads) s += static_cast<double>(zpart[c]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if ((threadIdx.x & 31) == 0) zsum[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        for (int w = 0; w < kScanThreads / 32; ++w) t += zsum[w];
+        *z_out = N > 0 ? static_cast<float>(t / static_cast<double>(N)) : 0.0f;
+    }
+}
+
+__device__ __forceinline__ void write_dense_table(int32_t *offsets, int32_t *mt, int64_t N, int tile_m)
+{
+    offsets[0] = 0;
+    offsets[1] = static_cast<int32_t>(N);
+    if (mt) {
+        mt[0] = 0;
+        mt[1] = static_cast<int32_t>((N + tile_m - 1) / tile_m);
+    }
+}
+
+__global__ void __launch_bounds__(kScanThreads) z_loss_kernel(const float *zpart, int64_t N, float *z_out)
+{
+    reduce_z_loss(zpart, (N + kCT - 1) / kCT, N, z_out);
+}
+
+__global__ void dense_table_kernel(int32_t *offsets, int32_t *mt, int64_t N, int tile_m)
+{
+    if (threadIdx.x == 0 && blockIdx.x == 0) write_dense_table(offsets, mt, N, tile_m);
+}
+
 // One CTA (E <= 256 threads' worth): offsets = exclusive prefix of counts,
 // the GEMM tile table, the Switch loss L = E sum_e (count_e/N)(P_e/N) in fp64
 // (course module sec. 2.3) and the sign-rule step b_e += gamma *
@@ -141,7 +181,9 @@ __global__ void __launch_bounds__(kScanThreads) scan_finalize_kernel(ScanArgs a)
     if (t == 0) {
         a.offsets[E] = total;
         if (a.mt_prefix) a.mt_prefix[E] = mt_total;
+        if (a.dense_offsets) write_dense_table(a.dense_offsets, a.dense_mt, a.N, a.dense_tile_m);
     }
+    if (a.z_out && a.zpart) reduce_z_loss(a.zpart, a.chunks, a.N, a.z_out);  // block-uniform
     if (a.aux_out && a.psum && a.pe) {
         // L = E / N^2 * sum_e count_e (N P_e): one term per thread, summed in a
         // fixed tree (warp butterflies, then the 8 warp sums in order)
@@ -221,7 +263,8 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a)
 // ---------------------------------------------------------------- combine
 
 // y_n = sum_{j<k} w[n,j] * y_sorted[inv_perm[n k + j]], fp32 accumulation in
-// slot order (sec. 2.2); one warp per token, 16-byte vectors.
+// slot order (sec. 2.2), plus y_add[n] (the shared expert's output, sec. 2.1)
+// when given; one warp per token, 16-byte vectors.
 template <typename T>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
 {
@@ -252,6 +295,13 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
                          static_cast<const T *>(nullptr));
 #pragma unroll
                 for (int u = 0; u < V; ++u) acc[u] = fmaf(wj, f[u], acc[u]);
+            }
+            if (in_row && a.y_add) {  // + Shared(x_n), after the routed sum
+                float f[V];
+                unpack16(ld_stream16(static_cast<const char *>(a.y_add) + n * row_bytes + o), f,
+                         static_cast<const T *>(nullptr));
+#pragma unroll
+                for (int u = 0; u < V; ++u) acc[u] += f[u];
             }
             if (in_row) st16(y + n * row_bytes + o, pack16(acc, static_cast<const T *>(nullptr)));
         }
@@ -322,6 +372,18 @@ cudaError_t launch_combine(int dtype, const CombineArgs &a, int num_sms, cudaStr
     const int grid = warp_grid(a.N, num_sms);
     if (dtype == kF32) combine_kernel<float><<<grid, 256, 0, s>>>(a);
     else combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_z_loss(const float *zpart, int64_t N, float *z_out, cudaStream_t s)
+{
+    z_loss_kernel<<<1, kScanThreads, 0, s>>>(zpart, N, z_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dense_table(int32_t *offsets, int32_t *mt, int64_t N, int tile_m, cudaStream_t s)
+{
+    dense_table_kernel<<<1, 32, 0, s>>>(offsets, mt, N, tile_m);
     return cudaGetLastError();
 }
 

@@ -22,6 +22,7 @@ struct RouterArgs {
     float *probs;        // [N, E] or null
     int32_t *hist;       // [chunks, E] or null
     float *psum;         // [chunks, E] or null
+    float *zpart;        // [chunks] sum of the chunk's (lse z_n)^2, or null
     int64_t N;
     int d, E, k, router, norm_topk;
     float scaling;
@@ -43,6 +44,7 @@ struct SelectKernelArgs {
     float *probs;         // [N, E] or null
     int32_t *hist;        // [chunks, E] or null
     float *psum;          // [chunks, E] or null
+    float *zpart;         // [chunks] sum of the chunk's (lse z_n)^2, or null
     int64_t N;
     int ld, E, k, router, norm_topk;
     float scaling;
@@ -78,8 +80,20 @@ struct ScanArgs {
     float *b_e;           // [E] or null
     double *pe;           // [E] scratch for P_e * N (needed when psum is given)
     int tile_m;           // rows per m-tile of the tile table (when mt_prefix is given)
+    const float *zpart;   // [chunks] per-chunk z-loss sums, or null
+    float *z_out;         // router z-loss (scalar) or null; needs zpart
+    int32_t *dense_offsets;  // [2] or null: {0, N}, the one-slice table of the shared expert
+    int32_t *dense_mt;       // [2] or null: {0, ceil(N / dense_tile_m)}
+    int dense_tile_m;
 };
 cudaError_t launch_scan(const ScanArgs &a, cudaStream_t s);
+
+// Router z-loss from per-chunk sums: *z_out = (sum of zpart) / N in fp64.
+cudaError_t launch_z_loss(const float *zpart, int64_t N, float *z_out, cudaStream_t s);
+
+// One-slice tile table over all N rows (the shared expert's GEMMs):
+// offsets = {0, N}, mt = {0, ceil(N / tile_m)}.
+cudaError_t launch_dense_table(int32_t *offsets, int32_t *mt, int64_t N, int tile_m, cudaStream_t s);
 
 // Sorted position of assignment a: offsets[e] + chunk base + rank in chunk.
 struct ScatterArgs {
@@ -109,6 +123,7 @@ struct CombineArgs {
     void *y;
     int64_t N;
     int d, k;
+    const void *y_add;  // [N, d] or null: added after the weighted sum (shared expert)
 };
 cudaError_t launch_combine(int dtype, const CombineArgs &a, int num_sms, cudaStream_t s);
 

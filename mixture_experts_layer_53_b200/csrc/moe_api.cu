@@ -54,13 +54,15 @@ moe_status validate(const moe_config *c)
     if (c->norm_topk != 0 && c->norm_topk != 1) return MOE_ERR_INVALID_ARG;
     if (!std::isfinite(c->routed_scaling)) return MOE_ERR_INVALID_ARG;
     if (c->E > kMaxE || c->k > kMaxK) return MOE_ERR_UNSUPPORTED;
-    if (c->d_model % 8 != 0 || c->d_ff % 8 != 0) return MOE_ERR_UNSUPPORTED;
+    if (c->d_ff_shared < 0) return MOE_ERR_INVALID_ARG;
+    if (c->d_model % 8 != 0 || c->d_ff % 8 != 0 || c->d_ff_shared % 8 != 0) return MOE_ERR_UNSUPPORTED;
     if (c->N * static_cast<int64_t>(c->k) >= (static_cast<int64_t>(1) << 31)) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
 
 struct Layout {
-    size_t hist, psum, logits, pe, offsets, mt, counts, ids, w, perm, inv, xs, h, ys, total;
+    size_t hist, psum, zpart, logits, pe, offsets, mt, shoff, shmt, counts, ids, w, perm, inv, xs, h, ys, ysh,
+        total;
 };
 
 size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
@@ -81,17 +83,24 @@ Layout layout(const moe_config *c)
     L.hist = take(C * E * 4);
     L.logits = take(static_cast<size_t>(c->N) * static_cast<size_t>(logits_ld(c->E)) * 4);
     L.psum = take(C * E * 4);
+    L.zpart = take(C * 4);
     L.pe = take(E * 8);
     L.offsets = take((E + 1) * 4);
     L.mt = take((E + 1) * 4);
+    L.shoff = take(2 * 4);
+    L.shmt = take(2 * 4);
     L.counts = take(E * 4);
     L.ids = take(A * 4);
     L.w = take(A * 4);
     L.perm = take(A * 4);
     L.inv = take(A * 4);
     L.xs = take(A * c->d_model * es);
-    L.h = take(A * c->d_ff * es);
+    // h holds the routed experts' hidden rows, then (reused) the shared expert's
+    const size_t Nn = static_cast<size_t>(c->N);
+    const size_t h_rows_cols = A * c->d_ff > Nn * c->d_ff_shared ? A * c->d_ff : Nn * c->d_ff_shared;
+    L.h = take(h_rows_cols * es);
     L.ys = take(A * c->d_model * es);
+    L.ysh = take(c->d_ff_shared > 0 ? Nn * c->d_model * es : 0);
     L.total = o;
     return L;
 }
@@ -106,7 +115,7 @@ moe_status check_ws(const moe_config *c, const void *ws, size_t ws_bytes)
 }
 
 RouterArgs router_args(const moe_config *c, const void *x, const void *W_g, const float *b_e, int32_t *ids,
-                       float *w, float *probs, int32_t *hist, float *psum)
+                       float *w, float *probs, int32_t *hist, float *psum, float *zpart = nullptr)
 {
     RouterArgs r{};
     r.x = x;
@@ -117,6 +126,7 @@ RouterArgs router_args(const moe_config *c, const void *x, const void *W_g, cons
     r.probs = probs;
     r.hist = hist;
     r.psum = psum;
+    r.zpart = zpart;
     r.N = c->N;
     r.d = c->d_model;
     r.E = c->E;
@@ -135,6 +145,13 @@ int ffn_tile_m(const moe_config *c)
     if (c->dtype != MOE_BF16) return 128;
     const int64_t rows_per_expert = c->N * c->k / c->E;
     return rows_per_expert > 192 ? 256 : 128;
+}
+
+// The same rule for the shared expert, whose one slice holds all N rows.
+int shared_tile_m(const moe_config *c)
+{
+    if (c->dtype != MOE_BF16) return 128;
+    return c->N > 192 ? 256 : 128;
 }
 
 FfnArgs ffn_args(const moe_config *c, const void *x_sorted, const int32_t *offsets, const int32_t *mt,
@@ -181,8 +198,8 @@ cudaError_t launch_route(const moe_config *c, const RouterArgs &r, int32_t *stat
     if (c->dtype != MOE_BF16) return launch_router(c->dtype, r, s);
     cudaError_t err = launch_router_logits_sm100(r.x, r.Wg, logits, r.N, r.d, r.E, status, s);
     if (err != cudaSuccess) return err;
-    SelectKernelArgs sk{logits, r.b_sel, r.ids, r.w, r.probs, r.hist, r.psum, r.N, logits_ld(r.E), r.E, r.k,
-                        r.router, r.norm_topk, r.scaling};
+    SelectKernelArgs sk{logits, r.b_sel, r.ids, r.w, r.probs, r.hist, r.psum, r.zpart, r.N, logits_ld(r.E),
+                        r.E, r.k, r.router, r.norm_topk, r.scaling};
     return launch_select(sk, s);
 }
 
@@ -191,6 +208,40 @@ cudaError_t launch_ffn(const moe_config *c, const FfnArgs &f, cudaEvent_t mid, c
     if (c->dtype != MOE_BF16) return launch_ffn_f32_simt(f, num_sms(), mid, s);
     return f.tile_m == 256 ? launch_ffn_bf16_sm100(f, num_sms(), mid, s)
                            : launch_ffn_bf16_sm100_single(f, num_sms(), mid, s);
+}
+
+// The shared expert: cfg->d_ff_shared > 0 exactly when its weights are given.
+moe_status check_shared(const moe_config *c, const moe_shared_expert *sh)
+{
+    if ((c->d_ff_shared > 0) != (sh != nullptr)) return MOE_ERR_INVALID_ARG;
+    if (!sh) return MOE_OK;
+    return check_ffn_ptrs(c, sh->W1, sh->b1, sh->W3, sh->W2, sh->b2);
+}
+
+// Both GEMMs of the shared expert over the N rows of x into y_shared, with
+// the one-slice tile table at (offsets, mt) already written.
+cudaError_t launch_shared(const moe_config *c, const moe_shared_expert *sh, const void *x, const int32_t *offsets,
+                          const int32_t *mt, void *h, void *y_shared, int32_t *status, cudaStream_t s)
+{
+    FfnArgs f{};
+    f.x_sorted = x;
+    f.offsets = offsets;
+    f.mt_prefix = mt;
+    f.W1 = sh->W1;
+    f.b1 = c->act == MOE_ACT_GELU ? sh->b1 : nullptr;
+    f.W3 = sh->W3;
+    f.W2 = sh->W2;
+    f.b2 = sh->b2;
+    f.h = h;
+    f.y_sorted = y_shared;
+    f.status = status;
+    f.rows = c->N;
+    f.d = c->d_model;
+    f.F = c->d_ff_shared;
+    f.E = 1;
+    f.act = c->act;
+    f.tile_m = shared_tile_m(c);
+    return launch_ffn(c, f, nullptr, s);
 }
 
 }  // namespace
@@ -295,16 +346,64 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_sorted, const int
     return MOE_OK;
 }
 
-moe_status moe_combine(const moe_config *cfg, const void *y_sorted, const float *topk_w, const int32_t *inv_perm,
-                       void *y, moe_stream_t stream)
+moe_status moe_combine_shared(const moe_config *cfg, const void *y_sorted, const float *topk_w,
+                              const int32_t *inv_perm, const void *y_shared, void *y, moe_stream_t stream)
 {
     moe_status st = validate(cfg);
     if (st != MOE_OK) return st;
     if (cfg->N > 0 && (!y_sorted || !topk_w || !inv_perm || !y)) return MOE_ERR_INVALID_ARG;
-    if (!aligned16(y_sorted) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y_sorted) || !aligned16(y) || !aligned16(y_shared)) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    CombineArgs ca{y_sorted, topk_w, inv_perm, y, cfg->N, cfg->d_model, cfg->k};
+    CombineArgs ca{y_sorted, topk_w, inv_perm, y, cfg->N, cfg->d_model, cfg->k, y_shared};
     cudaError_t err = launch_combine(cfg->dtype, ca, num_sms(), s);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err);
+}
+
+moe_status moe_combine(const moe_config *cfg, const void *y_sorted, const float *topk_w, const int32_t *inv_perm,
+                       void *y, moe_stream_t stream)
+{
+    return moe_combine_shared(cfg, y_sorted, topk_w, inv_perm, nullptr, y, stream);
+}
+
+moe_status moe_shared_ffn(const moe_config *cfg, const void *x, const moe_shared_expert *shared, void *y_shared,
+                          int32_t *dev_status, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (cfg->d_ff_shared == 0 || !shared) return MOE_ERR_INVALID_ARG;
+    if (cfg->N > 0 && (!x || !y_shared)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y_shared)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_shared(cfg, shared)) != MOE_OK) return st;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Layout L = layout(cfg);
+    int32_t *off = at<int32_t>(ws, L.shoff), *mt = at<int32_t>(ws, L.shmt);
+    cudaError_t err;
+    if ((err = launch_dense_table(off, mt, cfg->N, shared_tile_m(cfg), s)) != cudaSuccess) return cuda_fail(err);
+    err = launch_shared(cfg, shared, x, off, mt, at<void>(ws, L.h), y_shared, dev_status, s);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err);
+}
+
+moe_status moe_router_z_loss(const moe_config *cfg, const void *x, const void *W_g, float *z_loss_out,
+                             int32_t *dev_status, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (!W_g || !z_loss_out || (cfg->N > 0 && !x)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W_g)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Layout L = layout(cfg);
+    float *zpart = at<float>(ws, L.zpart);
+    cudaError_t err;
+    if (cfg->N > 0) {
+        // the routing itself lands in the workspace; only the z-loss is kept
+        const RouterArgs r = router_args(cfg, x, W_g, nullptr, at<int32_t>(ws, L.ids), at<float>(ws, L.w),
+                                         nullptr, nullptr, nullptr, zpart);
+        if ((err = launch_route(cfg, r, dev_status, at<float>(ws, L.logits), s)) != cudaSuccess)
+            return cuda_fail(err);
+    }
+    err = launch_z_loss(zpart, cfg->N, z_loss_out, s);
     return err == cudaSuccess ? MOE_OK : cuda_fail(err);
 }
 
@@ -346,6 +445,16 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const void *W_g, fl
                        int32_t *topk_ids, float *topk_w, int32_t *counts, float *aux_out, int32_t *dev_status,
                        void *ws, size_t ws_bytes, void *const *stage_events, moe_stream_t stream)
 {
+    return moe_forward_ex(cfg, x, W_g, b_e_inout, gamma, W1, b1, W3, W2, b2, nullptr, y, topk_ids, topk_w, counts,
+                          aux_out, nullptr, dev_status, ws, ws_bytes, stage_events, stream);
+}
+
+moe_status moe_forward_ex(const moe_config *cfg, const void *x, const void *W_g, float *b_e_inout, float gamma,
+                          const void *W1, const void *b1, const void *W3, const void *W2, const void *b2,
+                          const moe_shared_expert *shared, void *y, int32_t *topk_ids, float *topk_w,
+                          int32_t *counts, float *aux_out, float *z_loss_out, int32_t *dev_status, void *ws,
+                          size_t ws_bytes, void *const *stage_events, moe_stream_t stream)
+{
     moe_status st = validate(cfg);
     if (st != MOE_OK) return st;
     if (!W_g || (cfg->N > 0 && (!x || !y))) return MOE_ERR_INVALID_ARG;  // N = 0: x, y may be NULL
@@ -353,6 +462,7 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const void *W_g, fl
     if (b_e_inout && cfg->router != MOE_ROUTER_SIGMOID) return MOE_ERR_INVALID_ARG;
     if (!(gamma >= 0.f) || !std::isfinite(gamma)) return MOE_ERR_INVALID_ARG;
     if ((st = check_ffn_ptrs(cfg, W1, b1, W3, W2, b2)) != MOE_OK) return st;
+    if ((st = check_shared(cfg, shared)) != MOE_OK) return st;
     if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -377,7 +487,9 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const void *W_g, fl
     if (dev_status && (err = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s)) != cudaSuccess)
         return cuda_fail(err);
     // route: logits, scores, top-k, gates, per-chunk histograms and P sums
-    const RouterArgs r = router_args(cfg, x, W_g, b_e_inout, ids, w, nullptr, hist, psum);
+    float *zpart = at<float>(ws, L.zpart);
+    const RouterArgs r = router_args(cfg, x, W_g, b_e_inout, ids, w, nullptr, hist, psum,
+                                     z_loss_out ? zpart : nullptr);
     if (cfg->N > 0 && (err = launch_route(cfg, r, dev_status, at<float>(ws, L.logits), s)) != cudaSuccess) return cuda_fail(err);
     if ((err = mark(1)) != cudaSuccess) return cuda_fail(err);
     // dispatch: counts, offsets, tile table, Switch loss, bias step; scatter; gather
@@ -396,6 +508,14 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const void *W_g, fl
     sc.gamma = gamma;
     sc.tile_m = ffn_tile_m(cfg);
     sc.b_e = b_e_inout;
+    sc.zpart = zpart;
+    sc.z_out = z_loss_out;
+    int32_t *shoff = at<int32_t>(ws, L.shoff), *shmt = at<int32_t>(ws, L.shmt);
+    if (shared) {
+        sc.dense_offsets = shoff;
+        sc.dense_mt = shmt;
+        sc.dense_tile_m = shared_tile_m(cfg);
+    }
     if ((err = launch_scan(sc, s)) != cudaSuccess) return cuda_fail(err);
     ScatterArgs sa{ids, hist, nullptr, inv, cfg->N, cfg->E, cfg->k, offsets};
     if ((err = launch_scatter(sa, s)) != cudaSuccess) return cuda_fail(err);
@@ -405,9 +525,14 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const void *W_g, fl
     // expert FFNs over the ragged slices
     const FfnArgs f = ffn_args(cfg, xs, offsets, mt, W1, b1, W3, W2, b2, at<void>(ws, L.h), ys, dev_status);
     if ((err = launch_ffn(cfg, f, ev[3], s)) != cudaSuccess) return cuda_fail(err);
+    // the shared expert over all N rows (its hidden rows reuse h)
+    void *ysh = shared ? at<void>(ws, L.ysh) : nullptr;
+    if (shared && (err = launch_shared(cfg, shared, x, shoff, shmt, at<void>(ws, L.h), ysh, dev_status, s)) !=
+                      cudaSuccess)
+        return cuda_fail(err);
     if ((err = mark(4)) != cudaSuccess) return cuda_fail(err);
-    // combine back in token order
-    CombineArgs ca{ys, w, inv, y, cfg->N, cfg->d_model, cfg->k};
+    // combine back in token order (+ the shared expert's rows)
+    CombineArgs ca{ys, w, inv, y, cfg->N, cfg->d_model, cfg->k, ysh};
     if ((err = launch_combine(cfg->dtype, ca, num_sms(), s)) != cudaSuccess) return cuda_fail(err);
     if ((err = mark(5)) != cudaSuccess) return cuda_fail(err);
     return MOE_OK;

@@ -49,6 +49,14 @@ template <> struct Load4<__nv_bfloat16> {
     }
 };
 
+// Sum of the chunk's per-token z-loss terms, in token order.
+__device__ __forceinline__ float chunk_sum(const float *zl, int ntok)
+{
+    float s = 0.f;
+    for (int t = 0; t < ntok; ++t) s += zl[t];
+    return s;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a)
 {
@@ -60,6 +68,7 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a)
     float *ws = xs + kRT * kKP;       // [E][kKP]
     float *zt = ws + E * kKP;         // [kRT][E+1]   probabilities p
     int *ids_s = reinterpret_cast<int *>(zt + kRT * ZS);  // [kRT][k]
+    float *zl = reinterpret_cast<float *>(ids_s + kRT * k);  // [kRT] lse^2
 
     const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kRT;
     const int ntok = static_cast<int>(min64(kRT, a.N - tok0));
@@ -118,7 +127,8 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a)
 #pragma unroll
         for (int j = 0; j < 8; ++j) z[j] = acc[i][j];
         int sel_ids[kMaxK];
-        select_token(z, sa, tok0 + t, true, sel_ids);
+        const float lse = select_token(z, sa, tok0 + t, true, sel_ids);
+        if (lane == 0) zl[t] = lse * lse;
 #pragma unroll
         for (int r = 0; r < kMaxK; ++r)
             if (r < k && lane == r) ids_s[t * k + r] = sel_ids[r];
@@ -129,6 +139,7 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a)
     __syncthreads();
 
     // ---- per-chunk statistics in a fixed order (deterministic)
+    if (a.zpart && tid == 0) a.zpart[blockIdx.x] = chunk_sum(zl, ntok);
     if (a.psum || a.hist) {
         for (int e = tid; e < E; e += kThreads) {
             if (a.psum) {
@@ -160,6 +171,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
     const int EJ = (E + 31) >> 5;
     float *pt = smem;                                     // [32][E+1] p
     int *ids_s = reinterpret_cast<int *>(pt + kRT * ZS);  // [32][k]
+    float *zl = reinterpret_cast<float *>(ids_s + kRT * k);  // [32] lse^2
     const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kRT;
     const int ntok = static_cast<int>(min64(kRT, a.N - tok0));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -185,7 +197,8 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
             znext[j] = (tn < ntok && j < EJ && e < E) ? a.logits[(tok0 + tn) * a.ld + e] : 0.f;
         }
         int sel_ids[kMaxK];
-        select_token(z, sa, n, true, sel_ids);
+        const float lse = select_token(z, sa, n, true, sel_ids);
+        if (lane == 0) zl[t] = lse * lse;
 #pragma unroll
         for (int r = 0; r < kMaxK; ++r)
             if (r < k && lane == r) ids_s[t * k + r] = sel_ids[r];
@@ -194,6 +207,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
             if (j < EJ && lane + 32 * j < E) pt[t * ZS + lane + 32 * j] = z[j];
     }
     __syncthreads();
+    if (a.zpart && threadIdx.x == 0) a.zpart[blockIdx.x] = chunk_sum(zl, ntok);
     for (int e = threadIdx.x; e < E; e += kSelWarps * 32) {
         if (a.psum) {
             float s = 0.f;
@@ -210,7 +224,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
 
 size_t router_smem_bytes(int E, int k)
 {
-    return sizeof(float) * (kRT * kKP + E * kKP + kRT * (E + 1)) + sizeof(int) * kRT * k;
+    return sizeof(float) * (kRT * kKP + E * kKP + kRT * (E + 1) + kRT) + sizeof(int) * kRT * k;
 }
 
 template <typename T> cudaError_t launch_router_t(const RouterArgs &a, cudaStream_t s)
@@ -232,7 +246,7 @@ cudaError_t launch_select(const SelectKernelArgs &a, cudaStream_t s)
 {
     const int64_t grid = num_chunks(a.N);
     if (grid == 0) return cudaSuccess;
-    const size_t smem = sizeof(float) * kRT * (a.E + 1) + sizeof(int) * kRT * a.k;
+    const size_t smem = sizeof(float) * kRT * (a.E + 2) + sizeof(int) * kRT * a.k;
     select_kernel<<<static_cast<unsigned>(grid), kSelWarps * 32, smem, s>>>(a);
     return cudaGetLastError();
 }

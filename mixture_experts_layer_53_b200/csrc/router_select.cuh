@@ -35,8 +35,10 @@ __device__ __forceinline__ bool rank_ahead(float v, int e, float bv, int be)
 
 // z[j] = logit of expert lane + 32 j (j < ceil(E/32) <= 8).  Writes the
 // token's ids / weights / probs rows (if `write`), returns p in z[] and the
-// chosen ids in sel_ids[0..k) (valid in every lane).
-__device__ __forceinline__ void select_token(float (&z)[8], const SelectArgs &a, int64_t n, bool write,
+// chosen ids in sel_ids[0..k) (valid in every lane).  The return value is
+// log sum_e exp z_e (every lane), the token's term of the router z-loss
+// ("nano-moe", "Router z-loss").
+__device__ __forceinline__ float select_token(float (&z)[8], const SelectArgs &a, int64_t n, bool write,
                                              int (&sel_ids)[kMaxK])
 {
     const int lane = threadIdx.x & 31;
@@ -140,6 +142,7 @@ __device__ __forceinline__ void select_token(float (&z)[8], const SelectArgs &a,
         z[j] = (j < EJ && e < E) ? ex[j] * inv_esum : 0.f;
         if (write && a.probs && j < EJ && e < E) a.probs[n * E + e] = z[j];
     }
+    return zmax + logf(esum);
 }
 
 }  // namespace moe

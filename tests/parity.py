@@ -12,7 +12,10 @@ Rules (the tolerance is the one the task fixes for this layer):
     because a single flipped near-tie moves L by ~E/N * dP;
   * y: max over tokens of ||y_n - r_n||_inf / ||r_n||_inf <= 1e-5 (fp32) or
     2e-2 (bf16, fp32 accumulation); L within 1e-5 absolute; gate weights
-    within 2e-5 absolute.
+    within 2e-5 absolute;
+  * router z-loss within 1e-5 relative (max(1, z) scale): each token's
+    log-sum-exp comes from fp32 logits of the same accuracy as the gates;
+  * the shared expert is part of y (same tolerance).
 """
 from __future__ import annotations
 
@@ -30,6 +33,7 @@ MARGIN = 1e-4
 TOL_Y = {"f32": 1e-5, "bf16": 2e-2}
 TOL_AUX = 1e-5
 TOL_W = 2e-5
+TOL_Z = 1e-5
 
 
 def np64(t: Optional[torch.Tensor]) -> Optional[np.ndarray]:
@@ -40,17 +44,19 @@ def np64(t: Optional[torch.Tensor]) -> Optional[np.ndarray]:
 
 def config_of(wl: W.Workload) -> M.MoeConfig:
     return M.make_config(wl.N, wl.d_model, wl.d_ff, wl.E, wl.k, wl.router, wl.norm_topk, wl.routed_scaling,
-                         wl.act, wl.dtype)
+                         wl.act, wl.dtype, wl.d_ff_shared)
 
 
-def gpu_forward(wl: W.Workload, inp: Dict[str, torch.Tensor]) -> Dict[str, np.ndarray]:
-    """One moe_forward on the device; returns host copies of every output."""
+def gpu_forward(wl: W.Workload, inp: Dict[str, torch.Tensor], z_loss: bool = True) -> Dict[str, np.ndarray]:
+    """One forward on the device (moe_forward_ex with the z-loss and any shared
+    expert; moe_forward when z_loss is False and there is no shared expert);
+    returns host copies of every output."""
     cfg = config_of(wl)
     b_e = inp["b_e"].clone() if inp["b_e"] is not None else None
     out = M.moe_forward(cfg, inp["x"], inp["W_g"], inp["W1"], inp["W2"], W3=inp["W3"], b1=inp["b1"],
-                        b2=inp["b2"], b_e=b_e, gamma=wl.gamma)
+                        b2=inp["b2"], b_e=b_e, gamma=wl.gamma, shared=inp.get("shared"), z_loss=z_loss)
     torch.cuda.synchronize()
-    res = {k: v.cpu().numpy() for k, v in out.items() if k != "y"}
+    res = {k: v.cpu().numpy() for k, v in out.items() if k != "y" and (k != "z" or z_loss)}
     res["y"] = np64(out["y"])
     res["b_e_after"] = None if b_e is None else b_e.cpu().numpy()
     return res
@@ -62,6 +68,7 @@ class Report:
     id_mismatch: int = 0
     y_err: float = 0.0
     aux_err: float = 0.0
+    z_err: float = 0.0
     w_err: float = 0.0
     tokens_checked_y: int = 0
 
@@ -121,6 +128,10 @@ def check_forward(wl: W.Workload, inp, gpu: Dict[str, np.ndarray], y_tokens: Opt
         aux_o, _ = O.aux_loss(rf["probs"], ids_g)
         rep.aux_err = abs(float(gpu["aux"][0]) - aux_o)
         assert rep.aux_err <= TOL_AUX, f"aux loss {gpu['aux'][0]} vs {aux_o}"
+    if "z" in gpu:
+        z_o = O.z_loss(r["logits"]) if wl.N else 0.0
+        rep.z_err = abs(float(gpu["z"][0]) - z_o) / max(1.0, abs(z_o))
+        assert rep.z_err <= TOL_Z, f"router z-loss {gpu['z'][0]} vs {z_o}"
 
     if inp["b_e"] is not None and wl.gamma > 0:
         want = O.bias_update(np64(inp["b_e"]), dp["counts"], wl.N, wl.k, wl.gamma)
@@ -131,11 +142,14 @@ def check_forward(wl: W.Workload, inp, gpu: Dict[str, np.ndarray], y_tokens: Opt
     if len(tokens):
         x = np64(inp["x"])
         if y_tokens is None:
-            g = expert_getter(inp)
             y_o = O.dense_forward(x, ids_g, rf["w"], np64(inp["W1"]), np64(inp["W2"]), wl.act,
                                   np64(inp["W3"]), np64(inp["b1"]), np64(inp["b2"]))
         else:
             y_o = O.forward_tokens(x[tokens], ids_g[tokens], rf["w"][tokens], expert_getter(inp), wl.act)
+        sh = inp.get("shared")
+        if sh is not None:
+            y_o = O.shared_add(y_o, x[tokens], np64(sh["W1"]), np64(sh["W2"]), wl.act, np64(sh["W3"]),
+                               np64(sh["b1"]), np64(sh["b2"]))
         y_g = gpu["y"][tokens]
         denom = np.max(np.abs(y_o), axis=1)
         denom = np.where(denom > 0, denom, 1.0)

@@ -47,20 +47,24 @@ def test_config_layout_matches_header(tmp_path):
 #include <stdio.h>
 #include "moe.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(moe_config),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(moe_config),
          offsetof(moe_config, N), offsetof(moe_config, d_model), offsetof(moe_config, d_ff),
          offsetof(moe_config, E), offsetof(moe_config, k), offsetof(moe_config, router),
          offsetof(moe_config, norm_topk), offsetof(moe_config, routed_scaling),
-         offsetof(moe_config, act), offsetof(moe_config, dtype));
+         offsetof(moe_config, act), offsetof(moe_config, dtype), offsetof(moe_config, d_ff_shared));
+  printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(moe_shared_expert), offsetof(moe_shared_expert, W1),
+         offsetof(moe_shared_expert, b1), offsetof(moe_shared_expert, W3), offsetof(moe_shared_expert, W2),
+         offsetof(moe_shared_expert, b2));
   return 0;
 }
 """)
     exe = tmp_path / "probe"
     subprocess.check_call(["gcc", "-std=c11", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)])
-    got = [int(v) for v in subprocess.check_output([str(exe)], text=True).split()]
-    C = M.MoeConfig
-    want = [ctypes.sizeof(C)] + [getattr(C, f).offset for f, _ in C._fields_]
-    assert got == want
+    lines = subprocess.check_output([str(exe)], text=True).splitlines()
+    for line, C in zip(lines, (M.MoeConfig, M.SharedExpert)):
+        got = [int(v) for v in line.split()]
+        want = [ctypes.sizeof(C)] + [getattr(C, f).offset for f, _ in C._fields_]
+        assert got == want, C.__name__
 
 
 def test_status_strings_and_version(lib):
@@ -78,7 +82,7 @@ def cfg(**kw):
 @pytest.mark.parametrize("bad,code", [
     (dict(k=5), 1), (dict(k=0), 1), (dict(E=0), 1), (dict(N=-1), 1), (dict(d_model=0), 1),
     (dict(E=257, k=2), 2), (dict(E=32, k=17), 2), (dict(d_model=60), 2), (dict(d_ff=100), 2),
-    (dict(N=2 ** 31, k=2), 2),
+    (dict(N=2 ** 31, k=2), 2), (dict(d_ff_shared=-8), 1), (dict(d_ff_shared=12), 2),
 ])
 def test_invalid_configs(lib, bad, code):
     c = cfg(**bad)
@@ -158,3 +162,47 @@ def test_workspace_grows_with_tokens(lib):
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(RuntimeError, match="missing"):
         M.library(str(tmp_path / "libmoe.so"))
+
+
+def test_shared_expert_needs_width_and_weights(lib):
+    a = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x100000)
+    big = ctypes.c_size_t(1 << 40)
+    sh = M.SharedExpert(0x10000, None, None, 0x10000, None)
+    c0, c1 = cfg(), cfg(d_ff_shared=64)
+    # moe_forward has no slot for shared weights
+    assert lib.moe_forward(ctypes.byref(c1), a, a, None, ctypes.c_float(0.0), a, None, None, a, None, a, None,
+                           None, None, None, None, ws, big, None, None) == 1
+    # weights without a width, a width without weights
+    args = lambda c, shp: (ctypes.byref(c), a, a, None, ctypes.c_float(0.0), a, None, None, a, None, shp, a, None,
+                           None, None, None, None, None, ws, big, None, None)
+    assert lib.moe_forward_ex(*args(c0, ctypes.byref(sh))) == 1
+    assert lib.moe_forward_ex(*args(c1, None)) == 1
+    assert lib.moe_shared_ffn(ctypes.byref(c0), a, ctypes.byref(sh), a, None, ws, big, None) == 1
+    assert lib.moe_shared_ffn(ctypes.byref(c1), a, None, a, None, ws, big, None) == 1
+    # SwiGLU shared expert without W3
+    c2 = cfg(act="swiglu", d_ff_shared=64)
+    assert lib.moe_shared_ffn(ctypes.byref(c2), a, ctypes.byref(sh), a, None, ws, big, None) == 1
+    # misaligned shared weight
+    bad = M.SharedExpert(0x10008, None, None, 0x10000, None)
+    assert lib.moe_shared_ffn(ctypes.byref(c1), a, ctypes.byref(bad), a, None, ws, big, None) == 1
+
+
+def test_z_loss_validation(lib):
+    a = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x100000)
+    big = ctypes.c_size_t(1 << 40)
+    c = cfg()
+    assert lib.moe_router_z_loss(ctypes.byref(c), a, a, None, None, ws, big, None) == 1
+    assert lib.moe_router_z_loss(ctypes.byref(c), a, None, a, None, ws, big, None) == 1
+    assert lib.moe_router_z_loss(ctypes.byref(c), a, a, a, None, None, big, None) == 4
+    assert lib.moe_combine_shared(ctypes.byref(c), a, a, a, ctypes.c_void_p(0x10004), a, None) == 1
+
+
+def test_workspace_holds_the_shared_expert(lib):
+    base = dict(N=1024, d_model=256, d_ff=128, E=8, k=2, dtype="bf16")
+    n0 = lib.moe_workspace_size(ctypes.byref(cfg(**base)))
+    n1 = lib.moe_workspace_size(ctypes.byref(cfg(**base, d_ff_shared=128)))
+    n2 = lib.moe_workspace_size(ctypes.byref(cfg(**base, d_ff_shared=1024)))
+    assert n1 - n0 >= 1024 * 256 * 2 - 256         # + y_shared [N, d] (an empty region still takes 256 B)
+    assert n2 >= n1 + 1024 * (1024 - 2 * 128) * 2  # h grows to N * Fs once that exceeds N k F

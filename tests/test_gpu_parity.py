@@ -34,6 +34,10 @@ SMALL = {
                                                          router="topk_softmax"),
     "sigmoid_no_norm_scaled": W.WORKLOADS["deepseek_v3"].scaled(N=96, d_model=128, d_ff=128, E=16, k=4,
                                                                norm_topk=False, routed_scaling=2.5),
+    # > 192 rows per expert: the CTA-pair GEMM (256-row tiles), ragged shapes
+    "pair_swiglu_odd": W.WORKLOADS["mixtral"].scaled(N=600, d_model=136, d_ff=200, E=3),
+    "pair_gelu_odd": W.WORKLOADS["gpt2_moe"].scaled(N=700, d_model=200, d_ff=328, E=3),
+    "pair_swiglu_tiles": W.WORKLOADS["mixtral"].scaled(N=1100, d_model=320, d_ff=640, E=4),
 }
 
 FULL_SAMPLES = {"tiny_fp32": None, "gpt2_moe": 24, "mixtral": 8, "deepseek_v3": 4, "qwen3_skew": 12}
@@ -121,12 +125,17 @@ def test_dispatch_reports_bad_expert_id():
     assert int(out["status"][0]) == 6
 
 
-@pytest.mark.parametrize("dtype,act", [("bf16", "swiglu"), ("bf16", "gelu"), ("f32", "gelu"), ("f32", "swiglu")])
-def test_expert_ffn_entry_point(dtype, act):
-    """Random ragged slices with idle experts; every row checked."""
+@pytest.mark.parametrize("dtype,act,big", [("bf16", "swiglu", False), ("bf16", "gelu", False),
+                                           ("f32", "gelu", False), ("f32", "swiglu", False),
+                                           ("bf16", "swiglu", True), ("bf16", "gelu", True)])
+def test_expert_ffn_entry_point(dtype, act, big):
+    """Random ragged slices with idle experts; every row checked.  `big`
+    slices (> 192 rows per expert on average) take the CTA-pair kernel."""
     rng = np.random.default_rng(3)
     E, d, F = 9, 200, 264
     counts = np.array([0, 130, 1, 0, 257, 5, 128, 0, 40], np.int32)
+    if big:
+        counts = np.array([0, 700, 1, 0, 257, 5, 513, 0, 300], np.int32)
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
     rows = int(offsets[-1])
     wl = W.Workload("ffn", N=rows, d_model=d, d_ff=F, E=E, k=1, act=act, router="softmax_topk",
@@ -225,3 +234,24 @@ def test_collapsed_routing_single_expert_gets_everything():
     gpu = gpu_forward(wl, inp)
     assert gpu["counts"][3] == 300 and gpu["counts"][6] == 300
     check_forward(wl, inp, gpu)
+
+
+def test_host_pipeline_matches_forward():
+    """Batches in pinned host memory through the overlapped copy pipeline give
+    the same y and loss as moe_forward on device tensors, batch by batch."""
+    wl = SMALL["mixtral_small"]
+    inp = W.make_inputs(wl, DEV)
+    cfg = config_of(wl)
+    weights = {k: inp[k] for k in ("W_g", "W1", "W2", "W3", "b1", "b2", "b_e")}
+    xs = [W.make_x(wl.scaled(seed=wl.seed + i)).pin_memory() for i in range(4)]
+    ys = [torch.empty((wl.N, wl.d_model), dtype=torch.bfloat16).pin_memory() for _ in range(4)]
+    auxs = [torch.empty(1, dtype=torch.float32).pin_memory() for _ in range(4)]
+    pipe = M.HostPipeline(cfg, weights, device=DEV)
+    for i in range(4):
+        pipe.step(xs[i], ys[i], auxs[i])
+    pipe.finish()
+    for i in range(4):
+        ref = M.moe_forward(cfg, xs[i].to(DEV), inp["W_g"], inp["W1"], inp["W2"], W3=inp["W3"])
+        torch.cuda.synchronize()
+        assert torch.equal(ys[i], ref["y"].cpu()), i
+        assert torch.equal(auxs[i], ref["aux"].cpu()), i

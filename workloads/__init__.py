@@ -67,6 +67,7 @@ class Workload:
     w_std: float = 0.02
     zipf: bool = False
     seed: int = 1000
+    d_ff_shared: int = 0     # width of the shared expert (0 = none)
 
     @property
     def mats(self) -> int:
@@ -74,8 +75,9 @@ class Workload:
 
     @property
     def expert_flops(self) -> int:
-        """Algorithmic FLOPs of the expert FFNs: 2 * mats * d * F per assignment."""
-        return 2 * self.mats * self.d_model * self.d_ff * self.N * self.k
+        """Algorithmic FLOPs of the expert FFNs: 2 * mats * d * F per assignment,
+        plus 2 * mats * d * Fs per token for the shared expert."""
+        return 2 * self.mats * self.d_model * (self.d_ff * self.N * self.k + self.d_ff_shared * self.N)
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -98,6 +100,12 @@ WORKLOADS: Dict[str, Workload] = {
                             gamma=1e-3, seed=1003),
     "qwen3_skew": Workload("qwen3_skew", N=16384, d_model=2048, d_ff=768, E=128, k=8,
                            act="swiglu", router="softmax_topk", dtype="bf16", zipf=True, seed=1004),
+    # DeepSeek-V3 as the course module's router table describes it: one
+    # shared expert of the routed width beside the 256 routed ones, and
+    # routed_scaling 2.5 (beyond the five configurations above)
+    "deepseek_v3_shared": Workload("deepseek_v3_shared", N=4096, d_model=7168, d_ff=2048, E=256, k=8,
+                                   act="swiglu", router="sigmoid", dtype="bf16", sel_bias=True,
+                                   gamma=1e-3, routed_scaling=2.5, d_ff_shared=2048, seed=1005),
 }
 
 
@@ -167,6 +175,27 @@ def make_expert(wl: Workload, e: int, device="cpu") -> Dict[str, Optional[torch.
     return out
 
 
+def make_shared(wl: Workload, device="cpu") -> Optional[Dict[str, Optional[torch.Tensor]]]:
+    """The shared expert: W1 [Fs,d], W3 [Fs,d] or None, W2 [d,Fs], b1 [Fs], b2 [d]; None if Fs = 0."""
+    if wl.d_ff_shared == 0:
+        return None
+    dev = torch.device(device)
+    Fs, d = wl.d_ff_shared, wl.d_model
+
+    def draw(tensor: int, shape):
+        g = _gen(_expert_seed(wl, tensor, 0x5A5A), dev)
+        t = torch.randn(shape, generator=g, device=dev, dtype=torch.float32)
+        return (t * wl.w_std).to(wl.torch_dtype)
+
+    out = {"W1": draw(11, (Fs, d)), "W2": draw(12, (d, Fs)), "W3": None, "b1": None, "b2": None}
+    if wl.act == "swiglu":
+        out["W3"] = draw(13, (Fs, d))
+    if wl.biases:
+        out["b1"] = draw(14, (Fs,))
+        out["b2"] = draw(15, (d,))
+    return out
+
+
 def make_experts(wl: Workload, device="cpu") -> Dict[str, Optional[torch.Tensor]]:
     """All expert weights stacked: W1 [E,F,d], W3 [E,F,d]|None, W2 [E,d,F], b1 [E,F]|None, b2 [E,d]|None."""
     dev = torch.device(device)
@@ -190,13 +219,14 @@ def make_experts(wl: Workload, device="cpu") -> Dict[str, Optional[torch.Tensor]
 
 
 def make_inputs(wl: Workload, device="cpu") -> Dict[str, Optional[torch.Tensor]]:
-    """Every input of one forward, on ``device``: x, W_g, b_e, W1, W3, W2, b1, b2."""
+    """Every input of one forward, on ``device``: x, W_g, b_e, W1, W3, W2, b1, b2, shared."""
     dev = torch.device(device)
     out = {"x": make_x(wl).to(dev)}
     r = make_router(wl)
     out["W_g"] = r["W_g"].to(dev)
     out["b_e"] = None if r["b_e"] is None else r["b_e"].to(dev)
     out.update(make_experts(wl, dev))
+    out["shared"] = make_shared(wl, dev)
     return out
 
 
@@ -207,8 +237,9 @@ def flush_bytes_for_l2() -> int:
 
 def describe(wl: Workload) -> Dict[str, object]:
     return {"workload": wl.name, "N": wl.N, "d_model": wl.d_model, "d_ff": wl.d_ff, "E": wl.E,
-            "k": wl.k, "act": wl.act, "router": wl.router, "dtype": wl.dtype}
+            "k": wl.k, "act": wl.act, "router": wl.router, "dtype": wl.dtype,
+            **({"d_ff_shared": wl.d_ff_shared, "routed_scaling": wl.routed_scaling} if wl.d_ff_shared else {})}
 
 
 __all__ = ["Workload", "WORKLOADS", "make_inputs", "make_x", "make_router", "make_expert",
-           "make_experts", "zipf_offsets", "describe"]
+           "make_experts", "make_shared", "zipf_offsets", "describe"]
