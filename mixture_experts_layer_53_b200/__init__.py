@@ -304,22 +304,35 @@ def moe_aux_loss(cfg: MoeConfig, probs: torch.Tensor, topk_ids: torch.Tensor, ga
 
 
 class StageEvents:
-    """MOE_NUM_STAGES + 1 CUDA events that moe_forward records at stage boundaries."""
+    """CUDA events that moe_forward records at stage boundaries.
 
-    def __init__(self):
-        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(NUM_STAGES + 1)]
+    ``which`` selects the boundaries (0 .. MOE_NUM_STAGES; default all); the
+    others are passed as NULL and not recorded.  An event between two of the
+    library's kernels stops the second from being scheduled early, so timing
+    loops record only the boundaries they need.
+    """
+
+    def __init__(self, which: Optional[Sequence[int]] = None):
+        which = range(NUM_STAGES + 1) if which is None else which
+        self.events = [torch.cuda.Event(enable_timing=True) if i in which else None
+                       for i in range(NUM_STAGES + 1)]
         for e in self.events:           # materialise the CUDA event handles
-            e.record()
-        self._arr = (ctypes.c_void_p * (NUM_STAGES + 1))(*[e.cuda_event for e in self.events])
+            if e is not None:
+                e.record()
+        self._arr = (ctypes.c_void_p * (NUM_STAGES + 1))(
+            *[e.cuda_event if e is not None else None for e in self.events])
 
     @property
     def pointer(self):
         return ctypes.cast(self._arr, ctypes.c_void_p)
 
     def elapsed_ms(self) -> Dict[str, float]:
-        """Per-stage milliseconds of the last recorded forward (synchronises)."""
-        self.events[-1].synchronize()
-        return {STAGE_NAMES[i]: self.events[i].elapsed_time(self.events[i + 1]) for i in range(NUM_STAGES)}
+        """Per-stage milliseconds of the last recorded forward (synchronises);
+        only stages whose two boundaries were recorded."""
+        last = [e for e in self.events if e is not None][-1]
+        last.synchronize()
+        return {STAGE_NAMES[i]: self.events[i].elapsed_time(self.events[i + 1]) for i in range(NUM_STAGES)
+                if self.events[i] is not None and self.events[i + 1] is not None}
 
 
 def moe_forward(cfg: MoeConfig, x: torch.Tensor, W_g: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor,

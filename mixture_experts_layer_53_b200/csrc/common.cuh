@@ -19,6 +19,19 @@ constexpr int kMaxK = 16;
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 __host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 
+// Programmatic dependent launch.  Every kernel of this library starts with
+// pdl_enter(): griddepcontrol.wait returns once the previous grid on the
+// stream has completed and its memory is visible (immediately if there is no
+// programmatic dependency), so nothing below it can race with the
+// predecessor; launch_dependents then lets the next kernel's CTAs be
+// scheduled while this grid runs, hiding the launch latency between the
+// kernels of one forward.
+__device__ __forceinline__ void pdl_enter()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // First error wins; later errors leave the word alone.
 __device__ __forceinline__ void set_status(int32_t *status, int32_t code)
 {

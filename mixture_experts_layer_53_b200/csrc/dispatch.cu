@@ -15,6 +15,7 @@
 //      (the token row is read once and written k times).
 // Every reduction runs in a fixed order, so results are bitwise repeatable.
 #include "common.cuh"
+#include "host_util.h"
 #include "kernels.h"
 
 namespace moe {
@@ -26,6 +27,7 @@ constexpr int kCT = kChunkTokens;
 
 __global__ void __launch_bounds__(256) hist_kernel(HistArgs a)
 {
+    pdl_enter();
     __shared__ int ids_s[kCT * kMaxK];
     const int64_t c = blockIdx.x;
     const int64_t tok0 = c * kCT;
@@ -85,6 +87,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *total)
 // P_e * N = sum over chunks of psum[c][e] in fp64 (fixed tree order).
 __global__ void __launch_bounds__(kScanThreads) scan_cols_kernel(ScanArgs a)
 {
+    pdl_enter();
     const int e = blockIdx.x, E = a.E;
     const int64_t C = a.chunks;
     const int64_t per = (C + kScanThreads - 1) / kScanThreads;
@@ -149,11 +152,13 @@ __device__ __forceinline__ void write_dense_table(int32_t *offsets, int32_t *mt,
 
 __global__ void __launch_bounds__(kScanThreads) z_loss_kernel(const float *zpart, int64_t N, float *z_out)
 {
+    pdl_enter();
     reduce_z_loss(zpart, (N + kCT - 1) / kCT, N, z_out);
 }
 
 __global__ void dense_table_kernel(int32_t *offsets, int32_t *mt, int64_t N, int tile_m)
 {
+    pdl_enter();
     if (threadIdx.x == 0 && blockIdx.x == 0) write_dense_table(offsets, mt, N, tile_m);
 }
 
@@ -163,6 +168,7 @@ __global__ void dense_table_kernel(int32_t *offsets, int32_t *mt, int64_t N, int
 // sign(N k - E count_e) (sec. 2.5).
 __global__ void __launch_bounds__(kScanThreads) scan_finalize_kernel(ScanArgs a)
 {
+    pdl_enter();
     const int E = a.E, t = threadIdx.x;
     const int cnt = t < E ? a.offsets[t + 1] : 0;
     int total, mt_total;
@@ -210,6 +216,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_finalize_kernel(ScanArgs a)
 
 __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a)
 {
+    pdl_enter();
     __shared__ int ids_s[kCT * kMaxK];
     const int64_t c = blockIdx.x;
     const int64_t a0 = c * kCT * a.k;
@@ -233,6 +240,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a)
 template <typename T>
 __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a)
 {
+    pdl_enter();
     const int lane = threadIdx.x & 31;
     const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
     const int64_t row_bytes = static_cast<int64_t>(a.d) * sizeof(T);
@@ -264,10 +272,15 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a)
 
 // y_n = sum_{j<k} w[n,j] * y_sorted[inv_perm[n k + j]], fp32 accumulation in
 // slot order (sec. 2.2), plus y_add[n] (the shared expert's output, sec. 2.1)
-// when given; one warp per token, 16-byte vectors.
+// when given; one warp per token, 16-byte vectors.  Each lane loads kCombU
+// vectors of a slot's row before accumulating them, so a warp keeps
+// kCombU x 512 bytes in flight per slot even when k is small.
+constexpr int kCombU = 4;
+
 template <typename T>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
 {
+    pdl_enter();
     constexpr int V = Vec16<T>::n;
     const int lane = threadIdx.x & 31;
     const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -279,31 +292,49 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
          n += warps) {
         const int src_l = lane < a.k ? a.inv_perm[n * a.k + lane] : 0;
         const float w_l = lane < a.k ? a.w[n * a.k + lane] : 0.f;
-        // warp-uniform trip count: every lane reaches every shuffle
-        for (int64_t ob = 0; ob < row_bytes; ob += 512) {
-            const int64_t o = ob + static_cast<int64_t>(lane) * 16;
-            const bool in_row = o < row_bytes;
-            float acc[V];
+        // warp-uniform trip counts: every lane reaches every shuffle
+        for (int64_t ob = 0; ob < row_bytes; ob += 512 * kCombU) {
+            float acc[kCombU][V];
 #pragma unroll
-            for (int u = 0; u < V; ++u) acc[u] = 0.f;
+            for (int u = 0; u < kCombU; ++u)
+#pragma unroll
+                for (int i = 0; i < V; ++i) acc[u][i] = 0.f;
             for (int j = 0; j < a.k; ++j) {
                 const int src = __shfl_sync(0xffffffffu, src_l, j);
                 const float wj = __shfl_sync(0xffffffffu, w_l, j);
-                if (!in_row || static_cast<uint32_t>(src) >= static_cast<uint32_t>(rows)) continue;
-                float f[V];
-                unpack16(ld_stream16(ys + static_cast<int64_t>(src) * row_bytes + o), f,
-                         static_cast<const T *>(nullptr));
+                // positions of assignments with an invalid expert id were
+                // never written; never let them address outside y_sorted
+                const bool ok = static_cast<uint32_t>(src) < static_cast<uint32_t>(rows);
+                const char *row = ys + static_cast<int64_t>(ok ? src : 0) * row_bytes;
+                uint4 v[kCombU];
 #pragma unroll
-                for (int u = 0; u < V; ++u) acc[u] = fmaf(wj, f[u], acc[u]);
-            }
-            if (in_row && a.y_add) {  // + Shared(x_n), after the routed sum
-                float f[V];
-                unpack16(ld_stream16(static_cast<const char *>(a.y_add) + n * row_bytes + o), f,
-                         static_cast<const T *>(nullptr));
+                for (int u = 0; u < kCombU; ++u) {
+                    const int64_t o = ob + u * 512 + static_cast<int64_t>(lane) * 16;
+                    v[u] = (ok && o < row_bytes) ? ld_stream16(row + o) : make_uint4(0, 0, 0, 0);
+                }
 #pragma unroll
-                for (int u = 0; u < V; ++u) acc[u] += f[u];
+                for (int u = 0; u < kCombU; ++u) {
+                    const int64_t o = ob + u * 512 + static_cast<int64_t>(lane) * 16;
+                    if (!ok || o >= row_bytes) continue;
+                    float f[V];
+                    unpack16(v[u], f, static_cast<const T *>(nullptr));
+#pragma unroll
+                    for (int i = 0; i < V; ++i) acc[u][i] = fmaf(wj, f[i], acc[u][i]);
+                }
             }
-            if (in_row) st16(y + n * row_bytes + o, pack16(acc, static_cast<const T *>(nullptr)));
+#pragma unroll
+            for (int u = 0; u < kCombU; ++u) {
+                const int64_t o = ob + u * 512 + static_cast<int64_t>(lane) * 16;
+                if (o >= row_bytes) continue;
+                if (a.y_add) {  // + Shared(x_n), after the routed sum
+                    float f[V];
+                    unpack16(ld_stream16(static_cast<const char *>(a.y_add) + n * row_bytes + o), f,
+                             static_cast<const T *>(nullptr));
+#pragma unroll
+                    for (int i = 0; i < V; ++i) acc[u][i] += f[i];
+                }
+                st16(y + n * row_bytes + o, pack16(acc[u], static_cast<const T *>(nullptr)));
+            }
         }
     }
 }
@@ -312,6 +343,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
 
 __global__ void tile_table_kernel(const int32_t *offsets, int32_t *mt_prefix, int E, int tile_m)
 {
+    pdl_enter();
     if (threadIdx.x == 0 && blockIdx.x == 0) {
         int mt = 0;
         mt_prefix[0] = 0;
@@ -335,62 +367,53 @@ cudaError_t launch_hist(const HistArgs &a, cudaStream_t s)
 {
     const int64_t grid = num_chunks(a.N);
     if (grid == 0) return cudaSuccess;
-    hist_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_k(hist_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, s, a);
 }
 
 cudaError_t launch_scan(const ScanArgs &a, cudaStream_t s)
 {
     if (a.E > kScanThreads) return cudaErrorInvalidValue;
-    scan_cols_kernel<<<a.E, kScanThreads, 0, s>>>(a);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_k(scan_cols_kernel, dim3(a.E), dim3(kScanThreads), 0, s, a);
     if (err != cudaSuccess) return err;
-    scan_finalize_kernel<<<1, kScanThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_k(scan_finalize_kernel, dim3(1), dim3(kScanThreads), 0, s, a);
 }
 
 cudaError_t launch_scatter(const ScatterArgs &a, cudaStream_t s)
 {
     const int64_t grid = num_chunks(a.N);
     if (grid == 0) return cudaSuccess;
-    scatter_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_k(scatter_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, s, a);
 }
 
 cudaError_t launch_gather(int dtype, const GatherArgs &a, int num_sms, cudaStream_t s)
 {
     if (a.N == 0) return cudaSuccess;
     const int grid = warp_grid(a.N, num_sms);
-    if (dtype == kF32) gather_kernel<float><<<grid, 256, 0, s>>>(a);
-    else gather_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
-    return cudaGetLastError();
+    if (dtype == kF32) return launch_k(gather_kernel<float>, dim3(grid), dim3(256), 0, s, a);
+    return launch_k(gather_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, a);
 }
 
 cudaError_t launch_combine(int dtype, const CombineArgs &a, int num_sms, cudaStream_t s)
 {
     if (a.N == 0) return cudaSuccess;
     const int grid = warp_grid(a.N, num_sms);
-    if (dtype == kF32) combine_kernel<float><<<grid, 256, 0, s>>>(a);
-    else combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
-    return cudaGetLastError();
+    if (dtype == kF32) return launch_k(combine_kernel<float>, dim3(grid), dim3(256), 0, s, a);
+    return launch_k(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, a);
 }
 
 cudaError_t launch_z_loss(const float *zpart, int64_t N, float *z_out, cudaStream_t s)
 {
-    z_loss_kernel<<<1, kScanThreads, 0, s>>>(zpart, N, z_out);
-    return cudaGetLastError();
+    return launch_k(z_loss_kernel, dim3(1), dim3(kScanThreads), 0, s, zpart, N, z_out);
 }
 
 cudaError_t launch_dense_table(int32_t *offsets, int32_t *mt, int64_t N, int tile_m, cudaStream_t s)
 {
-    dense_table_kernel<<<1, 32, 0, s>>>(offsets, mt, N, tile_m);
-    return cudaGetLastError();
+    return launch_k(dense_table_kernel, dim3(1), dim3(32), 0, s, offsets, mt, N, tile_m);
 }
 
 cudaError_t launch_tile_table(const int32_t *offsets, int32_t *mt_prefix, int E, int tile_m, cudaStream_t s)
 {
-    tile_table_kernel<<<1, 32, 0, s>>>(offsets, mt_prefix, E, tile_m);
-    return cudaGetLastError();
+    return launch_k(tile_table_kernel, dim3(1), dim3(32), 0, s, offsets, mt_prefix, E, tile_m);
 }
 
 }  // namespace moe

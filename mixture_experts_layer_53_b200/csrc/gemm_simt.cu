@@ -7,6 +7,7 @@
 // computed 128 rows x 64 columns at a time, 256 threads, 8x4 outputs per
 // thread, k-chunks of 16 staged in shared memory.
 #include "common.cuh"
+#include "host_util.h"
 #include "kernels.h"
 
 namespace moe {
@@ -31,6 +32,7 @@ struct SimtArgs {
 template <int EPI>
 __global__ void __launch_bounds__(THREADS) simt_gemm_kernel(SimtArgs g)
 {
+    pdl_enter();
     __shared__ float As[TK][TM + 4];
     __shared__ float Bs[TK][TN + 4];
     __shared__ float B3s[EPI == EPI_SWIGLU ? TK : 1][TN + 4];
@@ -123,8 +125,7 @@ __global__ void __launch_bounds__(THREADS) simt_gemm_kernel(SimtArgs g)
 
 template <int EPI> cudaError_t launch_simt(const SimtArgs &g, int num_sms, cudaStream_t s)
 {
-    simt_gemm_kernel<EPI><<<num_sms * 4, THREADS, 0, s>>>(g);
-    return cudaGetLastError();
+    return launch_k(simt_gemm_kernel<EPI>, dim3(num_sms * 4), dim3(THREADS), 0, s, g);
 }
 
 }  // namespace

@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     ffn_gemm_single_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmB3, const GemmArgs g)
 {
+    pdl_enter();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                  ~static_cast<uintptr_t>(1023));
@@ -327,8 +328,7 @@ cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtens
     cudaError_t err =
         ensure_smem_attr(reinterpret_cast<const void *>(&ffn_gemm_single_kernel<EPI>), static_cast<int>(kSmemBytes));
     if (err != cudaSuccess) return err;
-    ffn_gemm_single_kernel<EPI><<<num_sms, THREADS, kSmemBytes, s>>>(a, b, b3, g);
-    return cudaGetLastError();
+    return launch_k(ffn_gemm_single_kernel<EPI>, dim3(num_sms), dim3(THREADS), kSmemBytes, s, a, b, b3, g);
 }
 
 }  // namespace

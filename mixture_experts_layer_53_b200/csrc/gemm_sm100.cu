@@ -159,6 +159,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmB3, const GemmArgs g)
 {
+    pdl_enter();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                  ~static_cast<uintptr_t>(1023));
@@ -337,8 +338,7 @@ cudaError_t launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtens
                                        static_cast<int>(kSmemBytes));
     if (err != cudaSuccess) return err;
     const int grid = (num_sms / 2) * 2;
-    ffn_gemm_pair_kernel<EPI><<<grid, THREADS, kSmemBytes, s>>>(a, b, b3, g);
-    return cudaGetLastError();
+    return launch_k(ffn_gemm_pair_kernel<EPI>, dim3(grid), dim3(THREADS), kSmemBytes, s, a, b, b3, g);
 }
 
 }  // namespace

@@ -25,4 +25,24 @@ inline cudaError_t ensure_smem_attr(const void *func, int bytes)
     return err;
 }
 
+// Launch `kernel` on stream s with programmatic stream serialization, so that
+// its CTAs may be scheduled before the previous kernel on s has finished; the
+// kernel itself waits for that kernel's completion first (pdl_enter).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                            Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace moe

@@ -29,15 +29,17 @@ struct RouterArgs {
 };
 // CUDA-core router (fp32 path).
 cudaError_t launch_router(int dtype, const RouterArgs &a, cudaStream_t s);
-// tcgen05 router logits (bf16 path): logits [N, logits_ld(E)] fp32;
-// `status` receives device wait timeouts.
+// tcgen05 router logits (bf16 path): router_splits(N, d) partial sums over
+// d, logits [splits, N, logits_ld(E)] fp32; `status` receives device wait
+// timeouts.
 int logits_ld(int E);
+int router_splits(int64_t N, int d);
 cudaError_t launch_router_logits_sm100(const void *x, const void *W_g, float *logits, int64_t N, int d, int E,
                                        int32_t *status, cudaStream_t s);
 
 // Scores, top-k, gates and per-chunk statistics from fp32 logits.
 struct SelectKernelArgs {
-    const float *logits;  // [N, ld]
+    const float *logits;  // [splits, N, ld] partial logits, summed in split order
     const float *b_sel;   // [E] or null (sigmoid router only)
     int32_t *ids;
     float *w;
@@ -48,6 +50,7 @@ struct SelectKernelArgs {
     int64_t N;
     int ld, E, k, router, norm_topk;
     float scaling;
+    int splits;
 };
 cudaError_t launch_select(const SelectKernelArgs &a, cudaStream_t s);
 

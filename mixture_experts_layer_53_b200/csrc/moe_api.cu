@@ -81,7 +81,8 @@ Layout layout(const moe_config *c)
     const size_t A = static_cast<size_t>(c->N) * static_cast<size_t>(c->k);
     const size_t es = elem_size(c);
     L.hist = take(C * E * 4);
-    L.logits = take(static_cast<size_t>(c->N) * static_cast<size_t>(logits_ld(c->E)) * 4);
+    L.logits = take(static_cast<size_t>(router_splits(c->N, c->d_model)) * static_cast<size_t>(c->N) *
+                    static_cast<size_t>(logits_ld(c->E)) * 4);
     L.psum = take(C * E * 4);
     L.zpart = take(C * 4);
     L.pe = take(E * 8);
@@ -199,7 +200,7 @@ cudaError_t launch_route(const moe_config *c, const RouterArgs &r, int32_t *stat
     cudaError_t err = launch_router_logits_sm100(r.x, r.Wg, logits, r.N, r.d, r.E, status, s);
     if (err != cudaSuccess) return err;
     SelectKernelArgs sk{logits, r.b_sel, r.ids, r.w, r.probs, r.hist, r.psum, r.zpart, r.N, logits_ld(r.E),
-                        r.E, r.k, r.router, r.norm_topk, r.scaling};
+                        r.E, r.k, r.router, r.norm_topk, r.scaling, router_splits(r.N, r.d)};
     return launch_select(sk, s);
 }
 

@@ -7,7 +7,11 @@
 // tokens over every SM, one warp per token.
 //
 // The product is [N, d] x [d, E] with small E, so the kernel is bound by
-// reading x.  One CTA takes a tile of 128 tokens:
+// reading x.  To keep every SM streaming x even when N / 128 is small, the
+// reduction over d is split S ways (router_splits): CTA (tile, s) sums the
+// k-blocks of split s of a tile of 128 tokens and writes its own partial
+// logits [N, ld] at logits + s * N * ld; the selection kernel adds the S
+// partials in split order.  One CTA:
 //   warp 0      TMA: x tile (128 x 64) and W_g tile (E_pad x 64) per k-block
 //               into a shared-memory ring (up to 8 stages)
 //   warp 1      allocates TMEM, one lane issues tcgen05.mma M=128, N=E_pad
@@ -46,10 +50,10 @@ struct Ctl {
 };
 
 struct LArgs {
-    float *logits;  // [N, ld]
+    float *logits;  // [splits, N, ld]
     int32_t *status;
     int64_t N;
-    int d, E, E_pad, ld, stages;
+    int d, E, E_pad, ld, stages, splits;
     int nacc;            // TMEM accumulators, k-block kb -> kb % nacc
     uint32_t acc_cols;   // TMEM columns per accumulator (power of 2 >= E_pad)
     uint32_t tmem_cols;  // nacc * acc_cols
@@ -59,6 +63,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                          const LArgs a)
 {
+    pdl_enter();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                  ~static_cast<uintptr_t>(1023));
@@ -90,8 +95,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
 
     const uint32_t tmem_base = ctl->tmem_base;
-    const int num_kb = (a.d + BK - 1) / BK;
-    const int row0 = blockIdx.x * BM;
+    // this CTA: token tile blockIdx.x / splits, k-blocks [kb0, kb0 + num_kb)
+    const int all_kb = (a.d + BK - 1) / BK;
+    const int split = static_cast<int>(blockIdx.x % a.splits);
+    const int kb0 = split * all_kb / a.splits;
+    const int num_kb = (split + 1) * all_kb / a.splits - kb0;
+    const int row0 = static_cast<int>(blockIdx.x / a.splits) * BM;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -104,8 +113,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mbar_arrive_expect_tx(&ctl->full[stage], static_cast<uint32_t>(stage_bytes));
                 armed |= 1u << stage;
                 armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-                tma_load_2d(sA, &tmX, &ctl->full[stage], kb * BK, row0);
-                tma_load_2d(sA + A_BYTES, &tmW, &ctl->full[stage], kb * BK, 0);
+                tma_load_2d(sA, &tmX, &ctl->full[stage], (kb0 + kb) * BK, row0);
+                tma_load_2d(sA + A_BYTES, &tmW, &ctl->full[stage], (kb0 + kb) * BK, 0);
                 if (++stage == a.stages) {
                     stage = 0;
                     phase ^= 1u;
@@ -161,7 +170,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
             const int used = min(a.nacc, num_kb);
-            float *zrow = a.logits + n * a.ld;
+            float *zrow = a.logits + (static_cast<int64_t>(split) * a.N + n) * a.ld;
             for (int c0 = 0; c0 < a.E_pad; c0 += 32) {
                 uint32_t r[32], t[32];
                 tmem_ld32(taddr + c0, r);
@@ -197,6 +206,20 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 int logits_ld(int E) { return (E + 3) / 4 * 4; }
 
+// Splits of the d reduction: enough (tile, split) CTAs to cover the 148 SMs
+// of a B200 once, at most one per k-block and at most 8.  A fixed function of
+// the shape, so the workspace size does not depend on the device.
+int router_splits(int64_t N, int d)
+{
+    const int64_t tiles = (N + BM - 1) / BM;
+    const int64_t kbs = (d + BK - 1) / BK;
+    int64_t sp = tiles > 0 ? 148 / tiles : 1;
+    sp = sp < 1 ? 1 : sp;
+    sp = sp > 8 ? 8 : sp;
+    sp = sp > kbs ? kbs : sp;
+    return static_cast<int>(sp);
+}
+
 cudaError_t launch_router_logits_sm100(const void *x, const void *W_g, float *logits, int64_t N, int d, int E,
                                        int32_t *status, cudaStream_t s)
 {
@@ -209,6 +232,7 @@ cudaError_t launch_router_logits_sm100(const void *x, const void *W_g, float *lo
     a.E = E;
     a.E_pad = ((E + 15) / 16) * 16;
     a.ld = logits_ld(E);
+    a.splits = router_splits(N, d);
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(a.E_pad)) cols <<= 1;
     a.acc_cols = cols;
@@ -227,9 +251,8 @@ cudaError_t launch_router_logits_sm100(const void *x, const void *W_g, float *lo
     cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&router_logits_kernel),
                                        1024 + SMEM_TILE_BUDGET + static_cast<int>(sizeof(Ctl)));
     if (err != cudaSuccess) return err;
-    const int64_t grid = (N + BM - 1) / BM;
-    router_logits_kernel<<<static_cast<unsigned>(grid), THREADS, smem, s>>>(tX, tW, a);
-    return cudaGetLastError();
+    const int64_t grid = (N + BM - 1) / BM * a.splits;
+    return launch_k(router_logits_kernel, dim3(static_cast<unsigned>(grid)), dim3(THREADS), smem, s, tX, tW, a);
 }
 
 }  // namespace moe
