@@ -139,9 +139,10 @@ MOE_API int32_t moe_version(void);
 /*
  * Bytes of workspace that every entry point below accepts for `cfg` (the
  * largest need, that of moe_forward): per-chunk histograms and partial
- * probability sums, offsets, the GEMM tile table, perm / inv_perm, x_sorted,
- * the hidden activations h [N*k, d_ff] and y_sorted.  Returns 0 for an
- * invalid cfg.
+ * probability sums, router partial logits, offsets, the GEMM tile tables,
+ * perm / inv_perm, x_sorted, the hidden activations h [N*k, d_ff] (or
+ * [N, d_ff_shared] if larger), y_sorted and the shared expert's output.
+ * Returns 0 for an invalid cfg.
  */
 MOE_API size_t moe_workspace_size(const moe_config *cfg);
 

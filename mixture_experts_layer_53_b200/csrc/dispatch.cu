@@ -212,6 +212,91 @@ __global__ void __launch_bounds__(kScanThreads) scan_finalize_kernel(ScanArgs a)
     }
 }
 
+// For E <= 32 the whole of the above in one CTA: warp w scans the columns of
+// experts w, w+8, ... (chunk bases in place, count_e, P_e * N in fp64 with
+// fixed-order sums), then warp 0 does the finalizing step with lane e for
+// expert e.  One launch instead of two.
+__global__ void __launch_bounds__(kScanThreads) scan_small_kernel(ScanArgs a)
+{
+    pdl_enter();
+    __shared__ int cnt_s[32];
+    __shared__ double pe_s[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int E = a.E;
+    const int64_t C = a.chunks;
+    const int64_t per = (C + 31) / 32;
+    const int64_t c0 = min64(C, lane * per), c1 = min64(C, c0 + per);
+    for (int e = warp; e < E; e += kScanThreads / 32) {  // warp-uniform
+        int s = 0;
+        double p = 0.0;
+        for (int64_t c = c0; c < c1; ++c) {
+            s += a.hist[c * E + e];
+            if (a.psum) p += static_cast<double>(a.psum[c * E + e]);
+        }
+        int incl = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        int run = incl - s;
+        for (int64_t c = c0; c < c1; ++c) {
+            const int v = a.hist[c * E + e];
+            a.hist[c * E + e] = run;
+            run += v;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+        if (lane == 0) {
+            cnt_s[e] = total;
+            pe_s[e] = p;
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int cnt = lane < E ? cnt_s[lane] : 0;
+        const int mt = (lane < E && a.mt_prefix) ? (cnt + a.tile_m - 1) / a.tile_m : 0;
+        int incl = cnt, mincl = mt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, incl, o);
+            const int v = __shfl_up_sync(0xffffffffu, mincl, o);
+            if (lane >= o) {
+                incl += u;
+                mincl += v;
+            }
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        const int mt_total = __shfl_sync(0xffffffffu, mincl, 31);
+        if (lane < E) {
+            a.offsets[lane] = incl - cnt;
+            if (a.counts) a.counts[lane] = cnt;
+            if (a.mt_prefix) a.mt_prefix[lane] = mincl - mt;
+            if (a.b_e && a.gamma > 0.f) {
+                const long long diff = static_cast<long long>(a.N) * a.k - static_cast<long long>(E) * cnt;
+                a.b_e[lane] += a.gamma * static_cast<float>((diff > 0) - (diff < 0));
+            }
+        }
+        if (lane == 0) {
+            a.offsets[E] = total;
+            if (a.mt_prefix) a.mt_prefix[E] = mt_total;
+            if (a.dense_offsets) write_dense_table(a.dense_offsets, a.dense_mt, a.N, a.dense_tile_m);
+        }
+        if (a.aux_out && a.psum) {
+            // L = E / N^2 * sum_e count_e (N P_e), summed in a fixed butterfly
+            double term = lane < E ? static_cast<double>(cnt) * pe_s[lane] : 0.0;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) term += __shfl_xor_sync(0xffffffffu, term, o);
+            if (lane == 0) {
+                const double Nd = static_cast<double>(a.N);
+                *a.aux_out = a.N == 0 ? 0.0f : static_cast<float>(term * static_cast<double>(E) / (Nd * Nd));
+            }
+        }
+    }
+    if (a.z_out && a.zpart) reduce_z_loss(a.zpart, a.chunks, a.N, a.z_out);  // block-uniform
+}
+
 // ---------------------------------------------------------------- scatter
 
 __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a)
@@ -263,6 +348,65 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a)
                 // never written; never let them address outside x_sorted
                 if (in_row && static_cast<uint32_t>(dst) < static_cast<uint32_t>(rows))
                     st16(xs + static_cast<int64_t>(dst) * row_bytes + o, v);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------- scatter fused with gather
+
+// Positions and row copies in one pass, one warp per token n of chunk c:
+// the warp reads the chunk's ids (a few coalesced loads, shared through L1 by
+// the chunk's 32 warps), ranks each of its k assignments among the chunk's
+// earlier assignments to the same expert with ballots, so that
+// position = offsets[e] + chunk base + rank exactly as in scatter_kernel,
+// writes inv_perm (and perm), then stores the token's row at its k
+// positions.  An assignment with an invalid expert id gets inv_perm = -1 and
+// no row.
+template <typename T>
+__global__ void __launch_bounds__(256) dispatch_rows_kernel(DispatchRowsArgs a)
+{
+    pdl_enter();
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    const int64_t row_bytes = static_cast<int64_t>(a.d) * sizeof(T);
+    const char *x = static_cast<const char *>(a.x);
+    char *xs = static_cast<char *>(a.x_sorted);
+    const int k = a.k;
+    for (int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); n < a.N;
+         n += warps) {
+        const int64_t c = n / kCT;
+        const int64_t a0 = c * kCT * k;                                      // chunk's first assignment
+        const int nas = static_cast<int>(min64(kCT, a.N - c * kCT)) * k;     // chunk's assignments
+        const int e_l = lane < k ? a.ids[n * k + lane] : -1;
+        const int q_l = static_cast<int>(n * k + lane - a0);                 // this slot inside the chunk
+        const bool valid_l = lane < k && e_l >= 0 && e_l < a.E;
+        int rank_l = 0;
+        for (int base = 0; base < nas; base += 32) {  // warp-uniform
+            const int q = base + lane;
+            const int idq = q < nas ? a.ids[a0 + q] : -1;
+            for (int j = 0; j < k; ++j) {
+                const int ej = __shfl_sync(0xffffffffu, e_l, j);
+                const int qj = __shfl_sync(0xffffffffu, q_l, j);
+                const unsigned m = __ballot_sync(0xffffffffu, idq == ej && q < qj);
+                if (lane == j) rank_l += __popc(m);
+            }
+        }
+        int dst_l = -1;
+        if (valid_l) {
+            dst_l = a.offsets[e_l] + a.chunk_base[c * a.E + e_l] + rank_l;
+            if (a.perm) a.perm[dst_l] = static_cast<int32_t>(n * k + lane);
+        }
+        if (lane < k) a.inv_perm[n * k + lane] = dst_l;
+        const char *src = x + n * row_bytes;
+        for (int64_t ob = 0; ob < row_bytes; ob += 512) {  // warp-uniform
+            const int64_t o = ob + static_cast<int64_t>(lane) * 16;
+            const bool in_row = o < row_bytes;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (in_row) v = ld_stream16(src + o);
+            for (int j = 0; j < k; ++j) {
+                const int dst = __shfl_sync(0xffffffffu, dst_l, j);
+                if (in_row && dst >= 0) st16(xs + static_cast<int64_t>(dst) * row_bytes + o, v);
             }
         }
     }
@@ -373,6 +517,7 @@ cudaError_t launch_hist(const HistArgs &a, cudaStream_t s)
 cudaError_t launch_scan(const ScanArgs &a, cudaStream_t s)
 {
     if (a.E > kScanThreads) return cudaErrorInvalidValue;
+    if (a.E <= 32) return launch_k(scan_small_kernel, dim3(1), dim3(kScanThreads), 0, s, a);
     cudaError_t err = launch_k(scan_cols_kernel, dim3(a.E), dim3(kScanThreads), 0, s, a);
     if (err != cudaSuccess) return err;
     return launch_k(scan_finalize_kernel, dim3(1), dim3(kScanThreads), 0, s, a);
@@ -391,6 +536,14 @@ cudaError_t launch_gather(int dtype, const GatherArgs &a, int num_sms, cudaStrea
     const int grid = warp_grid(a.N, num_sms);
     if (dtype == kF32) return launch_k(gather_kernel<float>, dim3(grid), dim3(256), 0, s, a);
     return launch_k(gather_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, a);
+}
+
+cudaError_t launch_dispatch_rows(int dtype, const DispatchRowsArgs &a, int num_sms, cudaStream_t s)
+{
+    if (a.N == 0) return cudaSuccess;
+    const int grid = warp_grid(a.N, num_sms);
+    if (dtype == kF32) return launch_k(dispatch_rows_kernel<float>, dim3(grid), dim3(256), 0, s, a);
+    return launch_k(dispatch_rows_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, a);
 }
 
 cudaError_t launch_combine(int dtype, const CombineArgs &a, int num_sms, cudaStream_t s)

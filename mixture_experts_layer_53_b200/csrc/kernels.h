@@ -34,10 +34,16 @@ cudaError_t launch_router(int dtype, const RouterArgs &a, cudaStream_t s);
 // timeouts.
 int logits_ld(int E);
 int router_splits(int64_t N, int d);
+// clear_status: the kernel zeroes *status before anything else (used as the
+// first kernel of a forward instead of a memset).
 cudaError_t launch_router_logits_sm100(const void *x, const void *W_g, float *logits, int64_t N, int d, int E,
-                                       int32_t *status, cudaStream_t s);
+                                       int32_t *status, bool clear_status, cudaStream_t s);
+// E <= 32: logits, scores, top-k, gates and the per-chunk statistics of
+// RouterArgs in one tcgen05 kernel (clusters of router_splits CTAs).
+cudaError_t launch_router_fused_sm100(const RouterArgs &r, int32_t *status, bool clear_status, cudaStream_t s);
 
-// Scores, top-k, gates and per-chunk statistics from fp32 logits.
+// Scores, top-k, gates and per-chunk statistics from fp32 logits (E > 32;
+// smaller E selects inside launch_router_fused_sm100).
 struct SelectKernelArgs {
     const float *logits;  // [splits, N, ld] partial logits, summed in split order
     const float *b_sel;   // [E] or null (sigmoid router only)
@@ -118,6 +124,21 @@ struct GatherArgs {
     int d, k;
 };
 cudaError_t launch_gather(int dtype, const GatherArgs &a, int num_sms, cudaStream_t s);
+
+// Scatter and gather in one pass (positions as in ScatterArgs, rows as in
+// GatherArgs); invalid expert ids get inv_perm = -1.
+struct DispatchRowsArgs {
+    const int32_t *ids;         // [N k]
+    const int32_t *chunk_base;  // [chunks, E], relative to the slice start
+    const int32_t *offsets;     // [E+1]
+    int32_t *perm;              // [N k] or null
+    int32_t *inv_perm;          // [N k]
+    const void *x;              // [N, d]
+    void *x_sorted;             // [N k, d]
+    int64_t N;
+    int d, E, k;
+};
+cudaError_t launch_dispatch_rows(int dtype, const DispatchRowsArgs &a, int num_sms, cudaStream_t s);
 
 struct CombineArgs {
     const void *y_sorted;

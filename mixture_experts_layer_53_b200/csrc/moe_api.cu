@@ -194,10 +194,12 @@ moe_status check_ffn_ptrs(const moe_config *c, const void *W1, const void *b1, c
 
 // bf16 routes on the tensor cores; fp32 keeps the CUDA-core router (tf32
 // products would not meet the fp32 tolerance).
-cudaError_t launch_route(const moe_config *c, const RouterArgs &r, int32_t *status, float *logits, cudaStream_t s)
+cudaError_t launch_route(const moe_config *c, const RouterArgs &r, int32_t *status, float *logits, cudaStream_t s,
+                         bool clear_status = false)
 {
     if (c->dtype != MOE_BF16) return launch_router(c->dtype, r, s);
-    cudaError_t err = launch_router_logits_sm100(r.x, r.Wg, logits, r.N, r.d, r.E, status, s);
+    if (c->E <= 32) return launch_router_fused_sm100(r, status, clear_status, s);
+    cudaError_t err = launch_router_logits_sm100(r.x, r.Wg, logits, r.N, r.d, r.E, status, clear_status, s);
     if (err != cudaSuccess) return err;
     SelectKernelArgs sk{logits, r.b_sel, r.ids, r.w, r.probs, r.hist, r.psum, r.zpart, r.N, logits_ld(r.E),
                         r.E, r.k, r.router, r.norm_topk, r.scaling, router_splits(r.N, r.d)};
@@ -316,11 +318,13 @@ moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *top
     sc.counts = counts;
     sc.offsets = offsets;
     if ((err = launch_scan(sc, s)) != cudaSuccess) return cuda_fail(err);
-    ScatterArgs sa{topk_ids, hist, perm, inv_perm, cfg->N, cfg->E, cfg->k, offsets};
-    if ((err = launch_scatter(sa, s)) != cudaSuccess) return cuda_fail(err);
-    if (x) {
-        GatherArgs ga{x, inv_perm, x_sorted, cfg->N, cfg->d_model, cfg->k};
-        if ((err = launch_gather(cfg->dtype, ga, num_sms(), s)) != cudaSuccess) return cuda_fail(err);
+    if (x) {  // positions and rows in one pass
+        DispatchRowsArgs da{topk_ids, hist, offsets, perm, inv_perm, x, x_sorted, cfg->N, cfg->d_model, cfg->E,
+                            cfg->k};
+        if ((err = launch_dispatch_rows(cfg->dtype, da, num_sms(), s)) != cudaSuccess) return cuda_fail(err);
+    } else {
+        ScatterArgs sa{topk_ids, hist, perm, inv_perm, cfg->N, cfg->E, cfg->k, offsets};
+        if ((err = launch_scatter(sa, s)) != cudaSuccess) return cuda_fail(err);
     }
     return MOE_OK;
 }
@@ -480,18 +484,23 @@ moe_status moe_forward_ex(const moe_config *cfg, const void *x, const void *W_g,
     int32_t *ids = topk_ids ? topk_ids : at<int32_t>(ws, L.ids);
     float *w = topk_w ? topk_w : at<float>(ws, L.w);
     int32_t *inv = at<int32_t>(ws, L.inv);
-    void *xs = at<void>(ws, L.xs);
     void *ys = at<void>(ws, L.ys);
 
     cudaError_t err;
     if ((err = mark(0)) != cudaSuccess) return cuda_fail(err);
-    if (dev_status && (err = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s)) != cudaSuccess)
+    // dev_status is cleared by the bf16 router's first CTA (no memset between
+    // this forward's kernels and the previous ones); the fp32 path and N = 0
+    // clear it with a memset
+    const bool router_clears = cfg->dtype == MOE_BF16 && cfg->N > 0;
+    if (dev_status && !router_clears && (err = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s)) != cudaSuccess)
         return cuda_fail(err);
     // route: logits, scores, top-k, gates, per-chunk histograms and P sums
     float *zpart = at<float>(ws, L.zpart);
     const RouterArgs r = router_args(cfg, x, W_g, b_e_inout, ids, w, nullptr, hist, psum,
                                      z_loss_out ? zpart : nullptr);
-    if (cfg->N > 0 && (err = launch_route(cfg, r, dev_status, at<float>(ws, L.logits), s)) != cudaSuccess) return cuda_fail(err);
+    if (cfg->N > 0 && (err = launch_route(cfg, r, dev_status, at<float>(ws, L.logits), s, router_clears)) !=
+                          cudaSuccess)
+        return cuda_fail(err);
     if ((err = mark(1)) != cudaSuccess) return cuda_fail(err);
     // dispatch: counts, offsets, tile table, Switch loss, bias step; scatter; gather
     ScanArgs sc{};
@@ -518,10 +527,10 @@ moe_status moe_forward_ex(const moe_config *cfg, const void *x, const void *W_g,
         sc.dense_tile_m = shared_tile_m(cfg);
     }
     if ((err = launch_scan(sc, s)) != cudaSuccess) return cuda_fail(err);
-    ScatterArgs sa{ids, hist, nullptr, inv, cfg->N, cfg->E, cfg->k, offsets};
-    if ((err = launch_scatter(sa, s)) != cudaSuccess) return cuda_fail(err);
-    GatherArgs ga{x, inv, xs, cfg->N, cfg->d_model, cfg->k};
-    if ((err = launch_gather(cfg->dtype, ga, num_sms(), s)) != cudaSuccess) return cuda_fail(err);
+    // positions and rows in one pass
+    void *xs = at<void>(ws, L.xs);
+    DispatchRowsArgs da{ids, hist, offsets, nullptr, inv, x, xs, cfg->N, cfg->d_model, cfg->E, cfg->k};
+    if ((err = launch_dispatch_rows(cfg->dtype, da, num_sms(), s)) != cudaSuccess) return cuda_fail(err);
     if ((err = mark(2)) != cudaSuccess) return cuda_fail(err);
     // expert FFNs over the ragged slices
     const FfnArgs f = ffn_args(cfg, xs, offsets, mt, W1, b1, W3, W2, b2, at<void>(ws, L.h), ys, dev_status);

@@ -236,140 +236,6 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
     }
 }
 
-// The same for E <= EB <= 32: one thread per token, one warp per 32-token
-// chunk.  A token's E logits sit in its thread's registers, so softmax and the
-// k argmax rounds (score desc, id asc) run without shuffles; the chunk's
-// statistics are warp reductions in a fixed butterfly order.
-template <int EB>
-__global__ void __launch_bounds__(128) select_small_kernel(SelectKernelArgs a)
-{
-    pdl_enter();
-    const int lane = threadIdx.x & 31;
-    const int64_t chunk = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
-    if (chunk * kRT >= a.N) return;  // warp-uniform
-    const int64_t n = chunk * kRT + lane;
-    const bool live = n < a.N;
-    const int E = a.E, k = a.k;
-
-    float z[EB];
-#pragma unroll
-    for (int e = 0; e < EB; e += 4) {
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (live && e < E) {  // ld is a multiple of 4: rows are 16-byte aligned
-            const float *p = a.logits + n * a.ld + e;
-            v = *reinterpret_cast<const float4 *>(p);
-            for (int s = 1; s < a.splits; ++s) {
-                const float4 u = *reinterpret_cast<const float4 *>(p + s * a.N * a.ld);
-                v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
-            }
-        }
-        z[e] = v.x; z[e + 1] = v.y; z[e + 2] = v.z; z[e + 3] = v.w;
-    }
-    float zmax = -FLT_MAX;
-#pragma unroll
-    for (int e = 0; e < EB; ++e)
-        if (e < E) zmax = fmaxf(zmax, z[e]);
-    float ex[EB], sel[EB], graw[EB];
-    float esum = 0.f;
-#pragma unroll
-    for (int e = 0; e < EB; ++e) {
-        ex[e] = 0.f;
-        sel[e] = -FLT_MAX;
-        graw[e] = 0.f;
-        if (e < E) {
-            ex[e] = expf(z[e] - zmax);
-            esum += ex[e];
-            if (a.router == kSigmoid) {
-                const float sg = 1.0f / (1.0f + expf(-z[e]));
-                sel[e] = sg + (a.b_sel ? a.b_sel[e] : 0.f);
-                graw[e] = sg;
-            } else {
-                sel[e] = z[e];
-                graw[e] = ex[e];
-            }
-        }
-    }
-    const float inv_esum = 1.0f / esum;
-    const float lse = zmax + logf(esum);
-
-    uint32_t taken = 0;
-    int ids[kMaxK];
-    float gsel[kMaxK];
-#pragma unroll
-    for (int r = 0; r < kMaxK; ++r) {
-        ids[r] = 0;
-        gsel[r] = 0.f;
-    }
-#pragma unroll 1
-    for (int r = 0; r < k; ++r) {
-        float bv = -FLT_MAX, bg = 0.f;
-        int be = INT_MAX;
-#pragma unroll
-        for (int e = 0; e < EB; ++e) {
-            if (e < E && !((taken >> e) & 1u) && rank_ahead(sel[e], e, bv, be)) {
-                bv = sel[e];
-                be = e;
-                bg = graw[e];
-            }
-        }
-        taken |= 1u << be;
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
-            if (j == r) {
-                ids[j] = be;
-                gsel[j] = bg;
-            }
-    }
-    float gs = 0.f;
-#pragma unroll
-    for (int r = 0; r < kMaxK; ++r)
-        if (r < k) gs += gsel[r];
-    if (live) {
-#pragma unroll
-        for (int r = 0; r < kMaxK; ++r) {
-            if (r < k) {
-                float wr;
-                if (a.router == kSoftmaxTopk) wr = a.norm_topk ? gsel[r] / gs : gsel[r] * inv_esum;
-                else if (a.router == kTopkSoftmax) wr = gsel[r] / gs;
-                else wr = a.norm_topk ? gsel[r] / gs : gsel[r];
-                a.ids[n * k + r] = ids[r];
-                a.w[n * k + r] = wr * a.scaling;
-            }
-        }
-        if (a.probs) {
-#pragma unroll
-            for (int e = 0; e < EB; ++e)
-                if (e < E) a.probs[n * E + e] = ex[e] * inv_esum;
-        }
-    }
-
-    // chunk statistics; tokens past N contribute nothing
-#pragma unroll
-    for (int e = 0; e < EB; ++e) {
-        if (e >= E) break;
-        if (a.psum) {
-            float v = live ? ex[e] * inv_esum : 0.f;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == e) a.psum[chunk * E + e] = v;
-        }
-        if (a.hist) {
-            int c = 0;
-#pragma unroll
-            for (int r = 0; r < kMaxK; ++r)
-                if (r < k && live) c += (ids[r] == e);
-            c = __reduce_add_sync(0xffffffffu, c);
-            if (lane == e) a.hist[chunk * E + e] = c;
-        }
-    }
-    if (a.zpart) {
-        float v = live ? lse * lse : 0.f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) a.zpart[chunk] = v;
-    }
-}
-
 size_t router_smem_bytes(int E, int k)
 {
     return sizeof(float) * (kRT * kKP + E * kKP + kRT * (E + 1) + kRT) + sizeof(int) * kRT * k;
@@ -393,12 +259,6 @@ cudaError_t launch_select(const SelectKernelArgs &a, cudaStream_t s)
 {
     const int64_t grid = num_chunks(a.N);
     if (grid == 0) return cudaSuccess;
-    if (a.E <= 32) {  // one thread per token, four chunks per CTA
-        const dim3 g(static_cast<unsigned>((grid + 3) / 4));
-        if (a.E <= 8) return launch_k(select_small_kernel<8>, g, dim3(128), 0, s, a);
-        if (a.E <= 16) return launch_k(select_small_kernel<16>, g, dim3(128), 0, s, a);
-        return launch_k(select_small_kernel<32>, g, dim3(128), 0, s, a);
-    }
     const size_t smem = sizeof(float) * kRT * (a.E + 2) + sizeof(int) * kRT * a.k;
     return launch_k(select_kernel, dim3(static_cast<unsigned>(grid)), dim3(kSelWarps * 32), smem, s, a);
 }

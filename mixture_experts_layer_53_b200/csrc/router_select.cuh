@@ -145,4 +145,122 @@ __device__ __forceinline__ float select_token(float (&z)[8], const SelectArgs &a
     return zmax + logf(esum);
 }
 
+// One token per thread for E <= EB <= 32, called by all 32 lanes of a warp
+// that holds one 32-token chunk (lane = token; `live` is false past N).  z[e]
+// = logit of expert e.  Softmax, the k argmax rounds (score desc, id asc) and
+// the gates run in the thread's registers, without shuffles; the chunk's
+// sum of p, histogram and sum of (lse z_n)^2 are warp reductions in a fixed
+// butterfly order, written for `chunk` (each may be null).
+template <int EB>
+__device__ __forceinline__ void select_thread_chunk(float (&z)[EB], const SelectArgs &a, float *psum,
+                                                    int32_t *hist, float *zpart, int64_t n, bool live,
+                                                    int64_t chunk)
+{
+    const int lane = threadIdx.x & 31;
+    const int E = a.E, k = a.k;
+    float zmax = -FLT_MAX;
+#pragma unroll
+    for (int e = 0; e < EB; ++e)
+        if (e < E) zmax = fmaxf(zmax, z[e]);
+    float ex[EB], sel[EB], graw[EB];
+    float esum = 0.f;
+#pragma unroll
+    for (int e = 0; e < EB; ++e) {
+        ex[e] = 0.f;
+        sel[e] = -FLT_MAX;
+        graw[e] = 0.f;
+        if (e < E) {
+            ex[e] = expf(z[e] - zmax);
+            esum += ex[e];
+            if (a.router == kSigmoid) {
+                const float sg = 1.0f / (1.0f + expf(-z[e]));
+                sel[e] = sg + (a.b_sel ? a.b_sel[e] : 0.f);
+                graw[e] = sg;
+            } else {
+                sel[e] = z[e];
+                graw[e] = ex[e];
+            }
+        }
+    }
+    const float inv_esum = 1.0f / esum;
+    const float lse = zmax + logf(esum);
+
+    uint32_t taken = 0;
+    int ids[kMaxK];
+    float gsel[kMaxK];
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) {
+        ids[r] = 0;
+        gsel[r] = 0.f;
+    }
+#pragma unroll 1
+    for (int r = 0; r < k; ++r) {
+        float bv = -FLT_MAX, bg = 0.f;
+        int be = INT_MAX;
+#pragma unroll
+        for (int e = 0; e < EB; ++e) {
+            if (e < E && !((taken >> e) & 1u) && rank_ahead(sel[e], e, bv, be)) {
+                bv = sel[e];
+                be = e;
+                bg = graw[e];
+            }
+        }
+        taken |= 1u << be;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+            if (j == r) {
+                ids[j] = be;
+                gsel[j] = bg;
+            }
+    }
+    float gs = 0.f;
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r)
+        if (r < k) gs += gsel[r];
+    if (live) {
+#pragma unroll
+        for (int r = 0; r < kMaxK; ++r) {
+            if (r < k) {
+                float wr;
+                if (a.router == kSoftmaxTopk) wr = a.norm_topk ? gsel[r] / gs : gsel[r] * inv_esum;
+                else if (a.router == kTopkSoftmax) wr = gsel[r] / gs;
+                else wr = a.norm_topk ? gsel[r] / gs : gsel[r];
+                a.ids[n * k + r] = ids[r];
+                a.w[n * k + r] = wr * a.scaling;
+            }
+        }
+        if (a.probs) {
+#pragma unroll
+            for (int e = 0; e < EB; ++e)
+                if (e < E) a.probs[n * E + e] = ex[e] * inv_esum;
+        }
+    }
+
+    // chunk statistics; tokens past N contribute nothing
+#pragma unroll
+    for (int e = 0; e < EB; ++e) {
+        if (e >= E) break;
+        if (psum) {
+            float v = live ? ex[e] * inv_esum : 0.f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == e) psum[chunk * E + e] = v;
+        }
+        if (hist) {
+            int c = 0;
+#pragma unroll
+            for (int r = 0; r < kMaxK; ++r)
+                if (r < k && live) c += (ids[r] == e);
+            c = __reduce_add_sync(0xffffffffu, c);
+            if (lane == e) hist[chunk * E + e] = c;
+        }
+    }
+    if (zpart) {
+        float v = live ? lse * lse : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) zpart[chunk] = v;
+    }
+}
+
 }  // namespace moe

@@ -21,11 +21,19 @@
 // epilogue then adds in fp32 round-to-nearest: the tensor core's own running
 // sums are only num_kb / nacc steps deep, which keeps the logits close enough
 // to an fp32 dot product for the 1e-5 tolerance of the Switch loss.
+//
+// For E <= 32 (router_kernel_fused<EB>) the selection is fused in: the S
+// split CTAs of a tile form a thread-block cluster, each leaves its partial
+// rows in its own shared memory, and after a cluster barrier the epilogue
+// warp of chunk q in CTA q % S adds the S partials of its 32 tokens in split
+// order through distributed shared memory and runs one thread per token
+// (select_thread_chunk): no logits in HBM and no second kernel.
 #include <cuda.h>
 
 #include "common.cuh"
 #include "host_util.h"
 #include "kernels.h"
+#include "router_select.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -35,7 +43,13 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int MAX_STAGES = 8;
+#ifndef MOE_ROUTER_MAX_STAGES
+#define MOE_ROUTER_MAX_STAGES 8
+#endif
+#ifndef MOE_ROUTER_CTA_TARGET
+#define MOE_ROUTER_CTA_TARGET 148
+#endif
+constexpr int MAX_STAGES = MOE_ROUTER_MAX_STAGES;
 constexpr int THREADS = 192;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int SMEM_TILE_BUDGET = 196608;
@@ -50,25 +64,50 @@ struct Ctl {
 };
 
 struct LArgs {
-    float *logits;  // [splits, N, ld]
+    float *logits;  // [splits, N, ld] (unfused)
     int32_t *status;
+    int clear_status;  // CTA 0 zeroes *status first (the forward's first kernel)
     int64_t N;
     int d, E, E_pad, ld, stages, splits;
     int nacc;            // TMEM accumulators, k-block kb -> kb % nacc
     uint32_t acc_cols;   // TMEM columns per accumulator (power of 2 >= E_pad)
     uint32_t tmem_cols;  // nacc * acc_cols
+    // fused selection (E <= 32)
+    SelectArgs sel;
+    float *psum;
+    int32_t *hist;
+    float *zpart;
 };
 
+__device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// EB == 0: partial logits to HBM.  EB in {8, 16, 32}: fused selection for
+// E <= EB, launched as clusters of `splits` CTAs.
+template <int EB>
 __global__ void __launch_bounds__(THREADS, 1)
     router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                          const LArgs a)
 {
     pdl_enter();
+    // Clearing here instead of with a memset keeps the forward a chain of
+    // kernels.  Any other writer of *status in this grid is a wait that ran
+    // out after seconds, long after CTA 0 started.
+    if (a.clear_status && a.status && blockIdx.x == 0 && threadIdx.x == 0) *a.status = 0;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                  ~static_cast<uintptr_t>(1023));
     const int stage_bytes = A_BYTES + a.E_pad * BK * 2;
     Ctl *ctl = reinterpret_cast<Ctl *>(tiles + a.stages * stage_bytes);
+    // fused: partial rows [BM][E_pad] fp32 of this CTA's split
+    float *part = reinterpret_cast<float *>((reinterpret_cast<uintptr_t>(ctl + 1) + 15) & ~static_cast<uintptr_t>(15));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort_flag = &ctl->abort;
 
@@ -170,7 +209,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
             const int used = min(a.nacc, num_kb);
-            float *zrow = a.logits + (static_cast<int64_t>(split) * a.N + n) * a.ld;
+            float *zrow = EB == 0 ? a.logits + (static_cast<int64_t>(split) * a.N + n) * a.ld
+                                  : part + (q * 32 + lane) * a.E_pad;
             for (int c0 = 0; c0 < a.E_pad; c0 += 32) {
                 uint32_t r[32], t[32];
                 tmem_ld32(taddr + c0, r);
@@ -182,12 +222,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int u = 0; u < 32; ++u)
                         r[u] = __float_as_uint(__uint_as_float(r[u]) + __uint_as_float(t[u]));
                 }
-                if (n < a.N) {
+                if (EB == 0 && n < a.N) {
 #pragma unroll
                     for (int v = 0; v < 8; ++v) {
                         const int c = c0 + 4 * v;
                         if (c < a.ld)  // ld is a multiple of 4
                             st16(zrow + c, make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]));
+                    }
+                }
+                if (EB > 0) {  // the whole padded row into shared memory
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        const int c = c0 + 4 * v;
+                        if (c < a.E_pad)
+                            *reinterpret_cast<uint4 *>(zrow + c) =
+                                make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
                     }
                 }
             }
@@ -199,6 +248,36 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, a.tmem_cols);
+    }
+    if constexpr (EB > 0) {
+        cluster_sync();  // every split's partial rows are in place
+        if (warp >= 2) {
+            const int q = warp & 3;
+            // chunks past N (the last tile's tail) have no statistics slots
+            if (q % a.splits == static_cast<int>(cluster_ctarank()) &&
+                static_cast<int64_t>(row0) + q * 32 < a.N) {  // warp-uniform
+                const int t = q * 32 + lane;
+                const int64_t n = static_cast<int64_t>(row0) + t;
+                float z[EB];
+#pragma unroll
+                for (int e = 0; e < EB; ++e) z[e] = 0.f;
+                const uint32_t row_addr = smem_u32(part + t * a.E_pad);
+                for (int sp = 0; sp < a.splits; ++sp) {  // split order
+                    const uint32_t ra = mapa_shared(row_addr, static_cast<uint32_t>(sp));
+#pragma unroll
+                    for (int e = 0; e < EB; e += 4) {
+                        const float4 v = ld_shared_cluster_f4(ra + e * 4);
+                        z[e] += v.x;
+                        z[e + 1] += v.y;
+                        z[e + 2] += v.z;
+                        z[e + 3] += v.w;
+                    }
+                }
+                select_thread_chunk<EB>(z, a.sel, a.psum, a.hist, a.zpart, n, n < a.N,
+                                        static_cast<int64_t>(row0 / 32 + q));
+            }
+        }
+        cluster_sync();  // no CTA leaves while its rows may still be read
     }
 }
 
@@ -213,20 +292,21 @@ int router_splits(int64_t N, int d)
 {
     const int64_t tiles = (N + BM - 1) / BM;
     const int64_t kbs = (d + BK - 1) / BK;
-    int64_t sp = tiles > 0 ? 148 / tiles : 1;
+    int64_t sp = tiles > 0 ? MOE_ROUTER_CTA_TARGET / tiles : 1;
     sp = sp < 1 ? 1 : sp;
     sp = sp > 8 ? 8 : sp;
     sp = sp > kbs ? kbs : sp;
     return static_cast<int>(sp);
 }
 
-cudaError_t launch_router_logits_sm100(const void *x, const void *W_g, float *logits, int64_t N, int d, int E,
-                                       int32_t *status, cudaStream_t s)
+namespace {
+
+// Fills the shape-dependent fields of LArgs; false if the tensor maps fail.
+bool setup(LArgs &a, CUtensorMap &tX, CUtensorMap &tW, const void *x, const void *W_g, int64_t N, int d, int E,
+           int32_t *status, bool clear_status)
 {
-    if (N == 0) return cudaSuccess;
-    LArgs a{};
-    a.logits = logits;
     a.status = status;
+    a.clear_status = clear_status ? 1 : 0;
     a.N = N;
     a.d = d;
     a.E = E;
@@ -242,17 +322,60 @@ cudaError_t launch_router_logits_sm100(const void *x, const void *W_g, float *lo
     const int stage_bytes = A_BYTES + a.E_pad * BK * 2;
     a.stages = SMEM_TILE_BUDGET / stage_bytes;
     if (a.stages > MAX_STAGES) a.stages = MAX_STAGES;
+    return make_tmap_bf16(&tX, x, d, static_cast<uint64_t>(N), BM) &&
+           make_tmap_bf16(&tW, W_g, d, static_cast<uint64_t>(E), static_cast<uint32_t>(a.E_pad));
+}
 
+constexpr int kSmemMax = 1024 + SMEM_TILE_BUDGET + static_cast<int>(sizeof(Ctl)) + 16 + BM * 32 * 4;
+
+size_t smem_bytes(const LArgs &a, bool fused)
+{
+    const int stage_bytes = A_BYTES + a.E_pad * BK * 2;
+    return 1024 + static_cast<size_t>(a.stages) * stage_bytes + sizeof(Ctl) +
+           (fused ? 16 + static_cast<size_t>(BM) * a.E_pad * 4 : 0);
+}
+
+template <int EB>
+cudaError_t launch_fused(const CUtensorMap &tX, const CUtensorMap &tW, const LArgs &a, cudaStream_t s)
+{
+    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&router_logits_kernel<EB>), kSmemMax);
+    if (err != cudaSuccess) return err;
+    const int64_t grid = (a.N + BM - 1) / BM * a.splits;
+    return launch_k_cluster(router_logits_kernel<EB>, dim3(static_cast<unsigned>(grid)), dim3(THREADS),
+                            smem_bytes(a, true), s, static_cast<unsigned>(a.splits), tX, tW, a);
+}
+
+}  // namespace
+
+cudaError_t launch_router_logits_sm100(const void *x, const void *W_g, float *logits, int64_t N, int d, int E,
+                                       int32_t *status, bool clear_status, cudaStream_t s)
+{
+    if (N == 0) return cudaSuccess;
+    LArgs a{};
     CUtensorMap tX, tW;
-    if (!make_tmap_bf16(&tX, x, d, static_cast<uint64_t>(N), BM) ||
-        !make_tmap_bf16(&tW, W_g, d, static_cast<uint64_t>(E), static_cast<uint32_t>(a.E_pad)))
-        return cudaErrorInvalidValue;
-    const size_t smem = 1024 + static_cast<size_t>(a.stages) * stage_bytes + sizeof(Ctl);
-    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&router_logits_kernel),
-                                       1024 + SMEM_TILE_BUDGET + static_cast<int>(sizeof(Ctl)));
+    if (!setup(a, tX, tW, x, W_g, N, d, E, status, clear_status)) return cudaErrorInvalidValue;
+    a.logits = logits;
+    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&router_logits_kernel<0>), kSmemMax);
     if (err != cudaSuccess) return err;
     const int64_t grid = (N + BM - 1) / BM * a.splits;
-    return launch_k(router_logits_kernel, dim3(static_cast<unsigned>(grid)), dim3(THREADS), smem, s, tX, tW, a);
+    return launch_k(router_logits_kernel<0>, dim3(static_cast<unsigned>(grid)), dim3(THREADS), smem_bytes(a, false),
+                    s, tX, tW, a);
+}
+
+cudaError_t launch_router_fused_sm100(const RouterArgs &r, int32_t *status, bool clear_status, cudaStream_t s)
+{
+    if (r.N == 0) return cudaSuccess;
+    if (r.E > 32) return cudaErrorInvalidValue;
+    LArgs a{};
+    CUtensorMap tX, tW;
+    if (!setup(a, tX, tW, r.x, r.Wg, r.N, r.d, r.E, status, clear_status)) return cudaErrorInvalidValue;
+    a.sel = SelectArgs{r.b_sel, r.ids, r.w, r.probs, r.E, r.k, r.router, r.norm_topk, r.scaling};
+    a.psum = r.psum;
+    a.hist = r.hist;
+    a.zpart = r.zpart;
+    if (r.E <= 8) return launch_fused<8>(tX, tW, a, s);
+    if (r.E <= 16) return launch_fused<16>(tX, tW, a, s);
+    return launch_fused<32>(tX, tW, a, s);
 }
 
 }  // namespace moe

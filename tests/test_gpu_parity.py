@@ -38,6 +38,10 @@ SMALL = {
     "pair_swiglu_odd": W.WORKLOADS["mixtral"].scaled(N=600, d_model=136, d_ff=200, E=3),
     "pair_gelu_odd": W.WORKLOADS["gpt2_moe"].scaled(N=700, d_model=200, d_ff=328, E=3),
     "pair_swiglu_tiles": W.WORKLOADS["mixtral"].scaled(N=1100, d_model=320, d_ff=640, E=4),
+    # the fused tcgen05 router with 17..32 experts (32-wide registers), and a
+    # sigmoid router there
+    "fused_e24": W.WORKLOADS["mixtral"].scaled(N=333, d_model=256, d_ff=256, E=24, k=3),
+    "fused_e32_sigmoid": W.WORKLOADS["deepseek_v3"].scaled(N=130, d_model=192, d_ff=128, E=32, k=8),
 }
 
 FULL_SAMPLES = {"tiny_fp32": None, "gpt2_moe": 24, "mixtral": 8, "deepseek_v3": 4, "qwen3_skew": 12}
@@ -113,6 +117,19 @@ def test_dispatch_entry_point(E, k, N):
     assert int(out["status"][0]) == 0
 
 
+@pytest.mark.parametrize("E,k,N", [(4, 2, 64), (128, 8, 777), (6, 2, 1)])
+def test_dispatch_entry_point_without_rows(E, k, N):
+    """x = NULL: positions only (the scatter kernel instead of the fused row pass)."""
+    rng = np.random.default_rng(E * 1000 + k + 7)
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(N)]).astype(np.int32)
+    cfg = M.make_config(N, 64, 64, E, k, dtype="bf16")
+    out = M.moe_dispatch(cfg, torch.from_numpy(ids).to(DEV))
+    torch.cuda.synchronize()
+    want = O.dispatch(ids, E)
+    for key in ("perm", "inv_perm", "offsets", "counts"):
+        assert np.array_equal(out[key].cpu().numpy(), want[key]), key
+
+
 def test_dispatch_reports_bad_expert_id():
     N, E, k = 50, 8, 2
     ids = np.tile(np.array([[0, 1]], np.int32), (N, 1))
@@ -123,6 +140,15 @@ def test_dispatch_reports_bad_expert_id():
     out = M.moe_dispatch(cfg, torch.from_numpy(ids).to(DEV), x=x)
     torch.cuda.synchronize()
     assert int(out["status"][0]) == 6
+    # the valid assignments keep their stable positions; the two invalid ones
+    # get inv_perm = -1 and no row
+    inv = out["inv_perm"].cpu().numpy().reshape(N, k)
+    assert inv[7, 1] == -1 and inv[20, 0] == -1
+    valid = (ids >= 0) & (ids < E)
+    got_rows = x.float().cpu().numpy()[np.arange(N).repeat(k).reshape(N, k)[valid]]
+    xs = out["x_sorted"].float().cpu().numpy()
+    assert np.array_equal(xs[inv[valid]], got_rows)
+    assert len(set(inv[valid].tolist())) == int(valid.sum())
 
 
 @pytest.mark.parametrize("dtype,act,big", [("bf16", "swiglu", False), ("bf16", "gelu", False),
