@@ -170,55 +170,55 @@ __device__ __forceinline__ float logit_of(const SelectKernelArgs &a, int64_t n, 
 
 // Scores, top-k and gates from precomputed fp32 logits (the tcgen05 router
 // of the bf16 path writes them), for E > 32.  One CTA per 32-token dispatch
-// chunk, one warp per token (16 warps, 2 tokens each): thousands of
-// independent warps hide the shuffle latency of the selection, which is a
-// serial chain per token.  Also writes the chunk's expert histogram and sum
-// of p.
+// chunk, one warp per token (16 warps, 2 tokens each): the selection is a
+// serial shuffle chain per token, so many independent warps hide its
+// latency.  Each token's k choices go into a shared histogram (integer
+// atomics: order-free); the chunk's sum of p is then taken per expert in
+// token order.
 constexpr int kSelWarps = 16;
 
+template <int EJ>
 __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs a)
 {
     pdl_enter();
     extern __shared__ float smem[];
     const int E = a.E, k = a.k;
     const int ZS = E + 1;
-    const int EJ = (E + 31) >> 5;
-    float *pt = smem;                                     // [32][E+1] p
-    int *ids_s = reinterpret_cast<int *>(pt + kRT * ZS);  // [32][k]
-    float *zl = reinterpret_cast<float *>(ids_s + kRT * k);  // [32] lse^2
+    float *pt = smem;                                          // [32][E+1] p
+    int *hist_s = reinterpret_cast<int *>(pt + kRT * ZS);      // [E]
+    float *zl = reinterpret_cast<float *>(hist_s + kMaxE);     // [32] lse^2
     const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kRT;
     const int ntok = static_cast<int>(min64(kRT, a.N - tok0));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    SelectArgs sa{a.b_sel, a.ids, a.w, a.probs, E, k, a.router, a.norm_topk, a.scaling};
+    for (int e = threadIdx.x; e < E; e += kSelWarps * 32) hist_s[e] = 0;
+    __syncthreads();
+    const SelectArgs sa{a.b_sel, a.ids, a.w, a.probs, E, k, a.router, a.norm_topk, a.scaling};
     // software pipeline: the next token's row is loaded while this one is
-    // selected (one copy of the selection code)
-    float znext[8];
+    // selected
+    float znext[EJ];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < EJ; ++j) {
         const int e = lane + 32 * j;
-        znext[j] = (warp < ntok && j < EJ && e < E) ? logit_of(a, tok0 + warp, e) : 0.f;
+        znext[j] = (warp < ntok && e < E) ? logit_of(a, tok0 + warp, e) : 0.f;
     }
 #pragma unroll 1
     for (int t = warp; t < ntok; t += kSelWarps) {
-        const int64_t n = tok0 + t;
-        float z[8];
+        float z[EJ];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) z[j] = znext[j];
+        for (int j = 0; j < EJ; ++j) z[j] = znext[j];
         const int tn = t + kSelWarps;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < EJ; ++j) {
             const int e = lane + 32 * j;
-            znext[j] = (tn < ntok && j < EJ && e < E) ? logit_of(a, tok0 + tn, e) : 0.f;
+            znext[j] = (tn < ntok && e < E) ? logit_of(a, tok0 + tn, e) : 0.f;
         }
-        int sel_ids[kMaxK];
-        const float lse = select_token(z, sa, n, true, sel_ids);
+        int sel_id;
+        const float lse = select_token_keys<EJ>(z, sa, tok0 + t, true, &sel_id);
         if (lane == 0) zl[t] = lse * lse;
+        if (lane < k) atomicAdd(&hist_s[sel_id], 1);
 #pragma unroll
-        for (int r = 0; r < kMaxK; ++r)
-            if (r < k && lane == r) ids_s[t * k + r] = sel_ids[r];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (j < EJ && lane + 32 * j < E) pt[t * ZS + lane + 32 * j] = z[j];
+        for (int j = 0; j < EJ; ++j)
+            if (lane + 32 * j < E) pt[t * ZS + lane + 32 * j] = z[j];
     }
     __syncthreads();
     if (a.zpart && threadIdx.x == 0) a.zpart[blockIdx.x] = chunk_sum(zl, ntok);
@@ -228,11 +228,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
             for (int t = 0; t < ntok; ++t) s += pt[t * ZS + e];
             a.psum[static_cast<int64_t>(blockIdx.x) * E + e] = s;
         }
-        if (a.hist) {
-            int c = 0;
-            for (int q = 0; q < ntok * k; ++q) c += (ids_s[q] == e);
-            a.hist[static_cast<int64_t>(blockIdx.x) * E + e] = c;
-        }
+        if (a.hist) a.hist[static_cast<int64_t>(blockIdx.x) * E + e] = hist_s[e];
     }
 }
 
@@ -259,8 +255,11 @@ cudaError_t launch_select(const SelectKernelArgs &a, cudaStream_t s)
 {
     const int64_t grid = num_chunks(a.N);
     if (grid == 0) return cudaSuccess;
-    const size_t smem = sizeof(float) * kRT * (a.E + 2) + sizeof(int) * kRT * a.k;
-    return launch_k(select_kernel, dim3(static_cast<unsigned>(grid)), dim3(kSelWarps * 32), smem, s, a);
+    const size_t smem = sizeof(float) * (kRT * (a.E + 1) + kRT) + sizeof(int) * kMaxE;
+    const dim3 g(static_cast<unsigned>(grid)), b(kSelWarps * 32);
+    if (a.E <= 64) return launch_k(select_kernel<2>, g, b, smem, s, a);
+    if (a.E <= 128) return launch_k(select_kernel<4>, g, b, smem, s, a);
+    return launch_k(select_kernel<8>, g, b, smem, s, a);
 }
 
 cudaError_t launch_router(int dtype, const RouterArgs &a, cudaStream_t s)

@@ -145,6 +145,138 @@ __device__ __forceinline__ float select_token(float (&z)[8], const SelectArgs &a
     return zmax + logf(esum);
 }
 
+// Order-preserving 64-bit key of (selection score desc, expert id asc):
+// larger key = ranks ahead.  -0 is folded into +0 so that equal scores tie.
+__device__ __forceinline__ uint64_t rank_key(float score, int e)
+{
+    uint32_t u = __float_as_uint(score + 0.0f);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(0xFFFF - e);
+}
+
+// One token per warp for 32 < E <= 32 * EJ (lane l holds experts l + 32 j in
+// z[j]).  Softmax / sigmoid scores as select_token; each of the k rounds
+// takes every lane's best untaken candidate by its rank_key, a warp max of
+// the keys (xor butterfly), and the winner's gate from the winning lane.
+// Lane r < k ends with the r-th choice: writes ids / w for token n (if
+// `write`), probs (if given), and returns in z[] the token's p.  *sel_id /
+// *sel_gate: lane r's choice (lanes >= k: -1 / 0).  Returns log sum_e exp z.
+template <int EJ>
+__device__ __forceinline__ float select_token_keys(float (&z)[EJ], const SelectArgs &a, int64_t n, bool write,
+                                                   int *sel_id)
+{
+    const int lane = threadIdx.x & 31;
+    const int E = a.E, k = a.k;
+    float zmax = -FLT_MAX;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j)
+        if (lane + 32 * j < E) zmax = fmaxf(zmax, z[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
+    float ex[EJ], graw[EJ];
+    uint64_t key[EJ];
+    float esum = 0.f;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+        const int e = lane + 32 * j;
+        ex[j] = 0.f;
+        graw[j] = 0.f;
+        key[j] = 0;  // below every real key
+        if (e < E) {
+            ex[j] = expf(z[j] - zmax);
+            esum += ex[j];
+            if (a.router == kSigmoid) {
+                const float sg = 1.0f / (1.0f + expf(-z[j]));
+                key[j] = rank_key(sg + (a.b_sel ? a.b_sel[e] : 0.f), e);
+                graw[j] = sg;
+            } else {
+                key[j] = rank_key(z[j], e);
+                graw[j] = ex[j];
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) esum += __shfl_xor_sync(0xffffffffu, esum, o);
+    const float inv_esum = 1.0f / esum;
+
+    uint32_t taken = 0;
+    int my_id = -1;
+    float my_gate = 0.f;
+#pragma unroll 1
+    for (int r = 0; r < k; ++r) {
+        uint64_t best = 0;
+        float bg = 0.f;
+        int bj = 0;
+#pragma unroll
+        for (int j = 0; j < EJ; ++j) {
+            if (!((taken >> j) & 1u) && key[j] > best) {
+                best = key[j];
+                bg = graw[j];
+                bj = j;
+            }
+        }
+        uint64_t win = best;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint64_t other = __shfl_xor_sync(0xffffffffu, win, o);
+            win = other > win ? other : win;
+        }
+        const int e = 0xFFFF - static_cast<int>(win & 0xFFFFu);
+        const int owner = e & 31;
+        if (lane == owner) taken |= 1u << bj;  // the owner's best is the winner
+        const float g = __shfl_sync(0xffffffffu, bg, owner);
+        if (lane == r) {
+            my_id = e;
+            my_gate = g;
+        }
+    }
+    // sum of the k chosen gates, in a fixed butterfly order
+    float gs = lane < k ? my_gate : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
+    if (write && lane < k) {
+        float wr;
+        if (a.router == kSoftmaxTopk) wr = a.norm_topk ? my_gate / gs : my_gate * inv_esum;
+        else if (a.router == kTopkSoftmax) wr = my_gate / gs;
+        else wr = a.norm_topk ? my_gate / gs : my_gate;
+        a.ids[n * k + lane] = my_id;
+        a.w[n * k + lane] = wr * a.scaling;
+    }
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+        const int e = lane + 32 * j;
+        z[j] = e < E ? ex[j] * inv_esum : 0.f;
+        if (write && a.probs && e < E) a.probs[n * E + e] = z[j];
+    }
+    *sel_id = my_id;
+    return zmax + logf(esum);
+}
+
+// Sums v[e] over the 32 lanes of a warp for all EB (8, 16 or 32) values at
+// once, in a fixed order: at each step the lanes with bit o set keep the upper
+// half of their values and add their partner's copy of it, the others the
+// lower half.  After log2(EB) steps each lane holds one expert's partial,
+// expert lane / (32 / EB); a butterfly over the remaining lane bits completes
+// it.  EB + log2(32 / EB) - 1 shuffles instead of 5 EB.
+template <int EB>
+__device__ __forceinline__ float warp_reduce_scatter(float (&v)[EB], int lane)
+{
+    static_assert(EB == 8 || EB == 16 || EB == 32, "EB");
+#pragma unroll
+    for (int h = EB / 2, o = 16; h >= 1; h /= 2, o /= 2) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < h; ++i) {
+            const float send = up ? v[i] : v[i + h];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+            v[i] = (up ? v[i + h] : v[i]) + recv;
+        }
+    }
+#pragma unroll
+    for (int o = 16 * 2 / EB / 2; o >= 1; o /= 2) v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    return v[0];
+}
+
 // One token per thread for E <= EB <= 32, called by all 32 lanes of a warp
 // that holds one 32-token chunk (lane = token; `live` is false past N).  z[e]
 // = logit of expert e.  Softmax, the k argmax rounds (score desc, id asc) and
@@ -185,49 +317,45 @@ __device__ __forceinline__ void select_thread_chunk(float (&z)[EB], const Select
     const float inv_esum = 1.0f / esum;
     const float lse = zmax + logf(esum);
 
+    // k argmax rounds; the choices go to small per-thread arrays (indexed by
+    // the round, so they live in local memory: a few loads and stores)
     uint32_t taken = 0;
     int ids[kMaxK];
     float gsel[kMaxK];
+    float gs = 0.f;
+    int cnt[EB];
 #pragma unroll
-    for (int r = 0; r < kMaxK; ++r) {
-        ids[r] = 0;
-        gsel[r] = 0.f;
-    }
+    for (int e = 0; e < EB; ++e) cnt[e] = 0;
 #pragma unroll 1
     for (int r = 0; r < k; ++r) {
         float bv = -FLT_MAX, bg = 0.f;
-        int be = INT_MAX;
+        int be = 0;
+        bool found = false;
 #pragma unroll
         for (int e = 0; e < EB; ++e) {
-            if (e < E && !((taken >> e) & 1u) && rank_ahead(sel[e], e, bv, be)) {
+            if (e < E && !((taken >> e) & 1u) && (!found || sel[e] > bv)) {  // ascending e: ties keep the lower id
                 bv = sel[e];
                 be = e;
                 bg = graw[e];
+                found = true;
             }
         }
         taken |= 1u << be;
+        ids[r] = be;
+        gsel[r] = bg;
+        gs += bg;
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
-            if (j == r) {
-                ids[j] = be;
-                gsel[j] = bg;
-            }
+        for (int e = 0; e < EB; ++e) cnt[e] += (live && be == e) ? 1 : 0;
     }
-    float gs = 0.f;
-#pragma unroll
-    for (int r = 0; r < kMaxK; ++r)
-        if (r < k) gs += gsel[r];
     if (live) {
-#pragma unroll
-        for (int r = 0; r < kMaxK; ++r) {
-            if (r < k) {
-                float wr;
-                if (a.router == kSoftmaxTopk) wr = a.norm_topk ? gsel[r] / gs : gsel[r] * inv_esum;
-                else if (a.router == kTopkSoftmax) wr = gsel[r] / gs;
-                else wr = a.norm_topk ? gsel[r] / gs : gsel[r];
-                a.ids[n * k + r] = ids[r];
-                a.w[n * k + r] = wr * a.scaling;
-            }
+#pragma unroll 1
+        for (int r = 0; r < k; ++r) {
+            float wr;
+            if (a.router == kSoftmaxTopk) wr = a.norm_topk ? gsel[r] / gs : gsel[r] * inv_esum;
+            else if (a.router == kTopkSoftmax) wr = gsel[r] / gs;
+            else wr = a.norm_topk ? gsel[r] / gs : gsel[r];
+            a.ids[n * k + r] = ids[r];
+            a.w[n * k + r] = wr * a.scaling;
         }
         if (a.probs) {
 #pragma unroll
@@ -236,22 +364,22 @@ __device__ __forceinline__ void select_thread_chunk(float (&z)[EB], const Select
         }
     }
 
-    // chunk statistics; tokens past N contribute nothing
+    // chunk statistics; tokens past N contribute nothing.  Sums over the
+    // warp's 32 tokens for all EB experts at once: a reduce-scatter leaves
+    // expert e's total in lanes e * 32 / EB .. (e + 1) * 32 / EB - 1.
+    if (psum) {
+        float v[EB];
 #pragma unroll
-    for (int e = 0; e < EB; ++e) {
-        if (e >= E) break;
-        if (psum) {
-            float v = live ? ex[e] * inv_esum : 0.f;
+        for (int e = 0; e < EB; ++e) v[e] = live ? ex[e] * inv_esum : 0.f;
+        const float tot = warp_reduce_scatter<EB>(v, lane);
+        const int e = lane / (32 / EB);
+        if (lane % (32 / EB) == 0 && e < E) psum[chunk * E + e] = tot;
+    }
+    if (hist) {
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == e) psum[chunk * E + e] = v;
-        }
-        if (hist) {
-            int c = 0;
-#pragma unroll
-            for (int r = 0; r < kMaxK; ++r)
-                if (r < k && live) c += (ids[r] == e);
-            c = __reduce_add_sync(0xffffffffu, c);
+        for (int e = 0; e < EB; ++e) {
+            if (e >= E) break;
+            const int c = __reduce_add_sync(0xffffffffu, cnt[e]);
             if (lane == e) hist[chunk * E + e] = c;
         }
     }
