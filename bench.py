@@ -35,10 +35,17 @@ L2_BYTES = 126 * 1024 * 1024
 # tokens of the workload the CPU oracle handles per reference step (about 1-3 s each)
 REF_TOKENS_PER_STEP = {"tiny_fp32": 64, "gpt2_moe": 32, "mixtral": 1, "deepseek_v3": 1, "qwen3_skew": 8,
                        "deepseek_v3_shared": 1}
-# libmoe kernels per forward: router logits + selection (bf16; one fused router
-# kernel for fp32), scan, scatter, gather, GEMM1, GEMM2, combine; a shared
-# expert adds its two GEMMs
-KERNELS_PER_STEP = {"bf16": 8, "f32": 7}
+
+
+def kernels_per_step(wl) -> int:
+    """libmoe kernels one moe_forward launches: the router (bf16 and E <= 32:
+    one fused tcgen05 kernel; bf16 and E > 32: logits + selection; fp32: one
+    CUDA-core kernel), the scan (one CTA for E <= 32, else per-expert columns
+    + finalize), the row pass (scatter fused with the gather), GEMM1, GEMM2,
+    the combine, and a shared expert's two GEMMs."""
+    router = 2 if (wl.dtype == "bf16" and wl.E > 32) else 1
+    scan = 1 if wl.E <= 32 else 2
+    return router + scan + 1 + 2 + 1 + (2 if wl.d_ff_shared else 0)
 
 
 def parse_args():
@@ -442,7 +449,7 @@ def run_native(args, wl):
             "e2e": {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s",
                     "h2d_bytes_per_step": inp["x"].numel() * inp["x"].element_size(),
                     "d2h_bytes_per_step": out["y"].numel() * out["y"].element_size() + 4},
-            "gpu_launches": (KERNELS_PER_STEP[wl.dtype] + (2 if wl.d_ff_shared else 0)) * args.steps,
+            "gpu_launches": kernels_per_step(wl) * args.steps,
             "clocks": clocks.summary(),
         }
         if not args.no_cpu_baseline and world == 1:

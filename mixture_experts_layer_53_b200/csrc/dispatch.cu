@@ -14,6 +14,9 @@
 //   4. rows are copied x -> x_sorted with 16-byte vectors, one warp per token
 //      (the token row is read once and written k times).
 // Every reduction runs in a fixed order, so results are bitwise repeatable.
+#include <map>
+#include <mutex>
+
 #include "common.cuh"
 #include "host_util.h"
 #include "kernels.h"
@@ -229,9 +232,11 @@ __global__ void __launch_bounds__(kScanThreads) scan_small_kernel(ScanArgs a)
     for (int e = warp; e < E; e += kScanThreads / 32) {  // warp-uniform
         int s = 0;
         double p = 0.0;
-        for (int64_t c = c0; c < c1; ++c) {
-            s += a.hist[c * E + e];
-            if (a.psum) p += static_cast<double>(a.psum[c * E + e]);
+#pragma unroll 8
+        for (int64_t c = c0; c < c1; ++c) s += a.hist[c * E + e];
+        if (a.psum) {
+#pragma unroll 8
+            for (int64_t c = c0; c < c1; ++c) p += static_cast<double>(a.psum[c * E + e]);
         }
         int incl = s;
 #pragma unroll
@@ -363,6 +368,14 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a)
 // writes inv_perm (and perm), then stores the token's row at its k
 // positions.  An assignment with an invalid expert id gets inv_perm = -1 and
 // no row.
+// The row kernels walk their work with a warp stride over a grid of exactly
+// the CTAs that fit at once, so no partial wave trails.  Each lane moves kRowU
+// 16-byte vectors of a kRowBlock-byte block, loading all of them before
+// storing or accumulating.  dispatch_rows_kernel: one token per warp (its
+// ranks are computed once); combine_kernel: (token, block) items.
+constexpr int kRowU = 4;
+constexpr int kRowBlock = 512 * kRowU;
+
 template <typename T>
 __global__ void __launch_bounds__(256) dispatch_rows_kernel(DispatchRowsArgs a)
 {
@@ -370,16 +383,17 @@ __global__ void __launch_bounds__(256) dispatch_rows_kernel(DispatchRowsArgs a)
     const int lane = threadIdx.x & 31;
     const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
     const int64_t row_bytes = static_cast<int64_t>(a.d) * sizeof(T);
+    const int64_t nblk = (row_bytes + kRowBlock - 1) / kRowBlock;
     const char *x = static_cast<const char *>(a.x);
     char *xs = static_cast<char *>(a.x_sorted);
     const int k = a.k;
     for (int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); n < a.N;
          n += warps) {
         const int64_t c = n / kCT;
-        const int64_t a0 = c * kCT * k;                                      // chunk's first assignment
-        const int nas = static_cast<int>(min64(kCT, a.N - c * kCT)) * k;     // chunk's assignments
+        const int64_t a0 = c * kCT * k;                                   // chunk's first assignment
+        const int nas = static_cast<int>(min64(kCT, a.N - c * kCT)) * k;  // chunk's assignments
         const int e_l = lane < k ? a.ids[n * k + lane] : -1;
-        const int q_l = static_cast<int>(n * k + lane - a0);                 // this slot inside the chunk
+        const int q_l = static_cast<int>(n * k + lane - a0);              // this slot inside the chunk
         const bool valid_l = lane < k && e_l >= 0 && e_l < a.E;
         int rank_l = 0;
         for (int base = 0; base < nas; base += 32) {  // warp-uniform
@@ -393,20 +407,28 @@ __global__ void __launch_bounds__(256) dispatch_rows_kernel(DispatchRowsArgs a)
             }
         }
         int dst_l = -1;
-        if (valid_l) {
-            dst_l = a.offsets[e_l] + a.chunk_base[c * a.E + e_l] + rank_l;
-            if (a.perm) a.perm[dst_l] = static_cast<int32_t>(n * k + lane);
+        if (valid_l) dst_l = a.offsets[e_l] + a.chunk_base[c * a.E + e_l] + rank_l;
+        if (lane < k) {
+            a.inv_perm[n * k + lane] = dst_l;
+            if (valid_l && a.perm) a.perm[dst_l] = static_cast<int32_t>(n * k + lane);
         }
-        if (lane < k) a.inv_perm[n * k + lane] = dst_l;
         const char *src = x + n * row_bytes;
-        for (int64_t ob = 0; ob < row_bytes; ob += 512) {  // warp-uniform
-            const int64_t o = ob + static_cast<int64_t>(lane) * 16;
-            const bool in_row = o < row_bytes;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (in_row) v = ld_stream16(src + o);
+        for (int64_t ob = 0; ob < nblk * kRowBlock; ob += kRowBlock) {
+            uint4 v[kRowU];
+#pragma unroll
+            for (int u = 0; u < kRowU; ++u) {
+                const int64_t o = ob + u * 512 + static_cast<int64_t>(lane) * 16;
+                v[u] = o < row_bytes ? ld_stream16(src + o) : make_uint4(0, 0, 0, 0);
+            }
             for (int j = 0; j < k; ++j) {
                 const int dst = __shfl_sync(0xffffffffu, dst_l, j);
-                if (in_row && dst >= 0) st16(xs + static_cast<int64_t>(dst) * row_bytes + o, v);
+                if (dst < 0) continue;  // warp-uniform
+                char *drow = xs + static_cast<int64_t>(dst) * row_bytes;
+#pragma unroll
+                for (int u = 0; u < kRowU; ++u) {
+                    const int64_t o = ob + u * 512 + static_cast<int64_t>(lane) * 16;
+                    if (o < row_bytes) st16(drow + o, v[u]);
+                }
             }
         }
     }
@@ -416,11 +438,7 @@ __global__ void __launch_bounds__(256) dispatch_rows_kernel(DispatchRowsArgs a)
 
 // y_n = sum_{j<k} w[n,j] * y_sorted[inv_perm[n k + j]], fp32 accumulation in
 // slot order (sec. 2.2), plus y_add[n] (the shared expert's output, sec. 2.1)
-// when given; one warp per token, 16-byte vectors.  Each lane loads kCombU
-// vectors of a slot's row before accumulating them, so a warp keeps
-// kCombU x 512 bytes in flight per slot even when k is small.
-constexpr int kCombU = 4;
-
+// when given; work items as in dispatch_rows_kernel, 16-byte vectors.
 template <typename T>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
 {
@@ -429,56 +447,56 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
     const int lane = threadIdx.x & 31;
     const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
     const int64_t row_bytes = static_cast<int64_t>(a.d) * sizeof(T);
+    const int64_t nblk = (row_bytes + kRowBlock - 1) / kRowBlock;
     const char *ys = static_cast<const char *>(a.y_sorted);
     char *y = static_cast<char *>(a.y);
     const int64_t rows = a.N * a.k;
-    for (int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); n < a.N;
-         n += warps) {
+    for (int64_t it = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+         it < a.N * nblk; it += warps) {
+        const int64_t n = it / nblk;
+        const int64_t ob = (it - n * nblk) * kRowBlock;
         const int src_l = lane < a.k ? a.inv_perm[n * a.k + lane] : 0;
         const float w_l = lane < a.k ? a.w[n * a.k + lane] : 0.f;
-        // warp-uniform trip counts: every lane reaches every shuffle
-        for (int64_t ob = 0; ob < row_bytes; ob += 512 * kCombU) {
-            float acc[kCombU][V];
+        float acc[kRowU][V];
 #pragma unroll
-            for (int u = 0; u < kCombU; ++u)
+        for (int u = 0; u < kRowU; ++u)
 #pragma unroll
-                for (int i = 0; i < V; ++i) acc[u][i] = 0.f;
-            for (int j = 0; j < a.k; ++j) {
-                const int src = __shfl_sync(0xffffffffu, src_l, j);
-                const float wj = __shfl_sync(0xffffffffu, w_l, j);
-                // positions of assignments with an invalid expert id were
-                // never written; never let them address outside y_sorted
-                const bool ok = static_cast<uint32_t>(src) < static_cast<uint32_t>(rows);
-                const char *row = ys + static_cast<int64_t>(ok ? src : 0) * row_bytes;
-                uint4 v[kCombU];
+            for (int i = 0; i < V; ++i) acc[u][i] = 0.f;
+        for (int j = 0; j < a.k; ++j) {  // warp-uniform: every lane reaches every shuffle
+            const int src = __shfl_sync(0xffffffffu, src_l, j);
+            const float wj = __shfl_sync(0xffffffffu, w_l, j);
+            // positions of assignments with an invalid expert id were never
+            // written; never let them address outside y_sorted
+            const bool ok = static_cast<uint32_t>(src) < static_cast<uint32_t>(rows);
+            const char *row = ys + static_cast<int64_t>(ok ? src : 0) * row_bytes;
+            uint4 v[kRowU];
 #pragma unroll
-                for (int u = 0; u < kCombU; ++u) {
-                    const int64_t o = ob + u * 512 + static_cast<int64_t>(lane) * 16;
-                    v[u] = (ok && o < row_bytes) ? ld_stream16(row + o) : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int u = 0; u < kCombU; ++u) {
-                    const int64_t o = ob + u * 512 + static_cast<int64_t>(lane) * 16;
-                    if (!ok || o >= row_bytes) continue;
-                    float f[V];
-                    unpack16(v[u], f, static_cast<const T *>(nullptr));
-#pragma unroll
-                    for (int i = 0; i < V; ++i) acc[u][i] = fmaf(wj, f[i], acc[u][i]);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kCombU; ++u) {
+            for (int u = 0; u < kRowU; ++u) {
                 const int64_t o = ob + u * 512 + static_cast<int64_t>(lane) * 16;
-                if (o >= row_bytes) continue;
-                if (a.y_add) {  // + Shared(x_n), after the routed sum
-                    float f[V];
-                    unpack16(ld_stream16(static_cast<const char *>(a.y_add) + n * row_bytes + o), f,
-                             static_cast<const T *>(nullptr));
-#pragma unroll
-                    for (int i = 0; i < V; ++i) acc[u][i] += f[i];
-                }
-                st16(y + n * row_bytes + o, pack16(acc[u], static_cast<const T *>(nullptr)));
+                v[u] = (ok && o < row_bytes) ? ld_stream16(row + o) : make_uint4(0, 0, 0, 0);
             }
+#pragma unroll
+            for (int u = 0; u < kRowU; ++u) {
+                const int64_t o = ob + u * 512 + static_cast<int64_t>(lane) * 16;
+                if (!ok || o >= row_bytes) continue;
+                float f[V];
+                unpack16(v[u], f, static_cast<const T *>(nullptr));
+#pragma unroll
+                for (int i = 0; i < V; ++i) acc[u][i] = fmaf(wj, f[i], acc[u][i]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kRowU; ++u) {
+            const int64_t o = ob + u * 512 + static_cast<int64_t>(lane) * 16;
+            if (o >= row_bytes) continue;
+            if (a.y_add) {  // + Shared(x_n), after the routed sum
+                float f[V];
+                unpack16(ld_stream16(static_cast<const char *>(a.y_add) + n * row_bytes + o), f,
+                         static_cast<const T *>(nullptr));
+#pragma unroll
+                for (int i = 0; i < V; ++i) acc[u][i] += f[i];
+            }
+            st16(y + n * row_bytes + o, pack16(acc[u], static_cast<const T *>(nullptr)));
         }
     }
 }
@@ -496,6 +514,30 @@ __global__ void tile_table_kernel(const int32_t *offsets, int32_t *mt_prefix, in
             mt_prefix[e + 1] = mt;
         }
     }
+}
+
+// CTAs of `kernel` (256 threads) that fit on the device at once, capped by
+// the work: items / 8 (one item per warp).
+int row_grid(const void *kernel, int64_t items, int num_sms)
+{
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, int> occ;
+    int dev = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = occ.find({kernel, dev});
+        if (it != occ.end()) per_sm = it->second;
+    }
+    if (per_sm == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess || per_sm < 1)
+            per_sm = 1;
+        std::lock_guard<std::mutex> lock(mu);
+        occ[{kernel, dev}] = per_sm;
+    }
+    const int64_t want = (items + 7) / 8;
+    const int64_t cap = static_cast<int64_t>(num_sms) * per_sm;
+    return static_cast<int>(max64(1, min64(want, cap)));
 }
 
 int warp_grid(int64_t N, int num_sms)
@@ -538,20 +580,27 @@ cudaError_t launch_gather(int dtype, const GatherArgs &a, int num_sms, cudaStrea
     return launch_k(gather_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, a);
 }
 
+template <typename T>
+cudaError_t launch_rows(void (*kernel)(T), const T &a, int64_t items, int num_sms, cudaStream_t s)
+{
+    if (items == 0) return cudaSuccess;
+    const int grid = row_grid(reinterpret_cast<const void *>(kernel), items, num_sms);
+    return launch_k(kernel, dim3(grid), dim3(256), 0, s, a);
+}
+
+int64_t row_blocks(int dtype, int d) { return (static_cast<int64_t>(d) * (dtype == kF32 ? 4 : 2) + kRowBlock - 1) / kRowBlock; }
+
 cudaError_t launch_dispatch_rows(int dtype, const DispatchRowsArgs &a, int num_sms, cudaStream_t s)
 {
-    if (a.N == 0) return cudaSuccess;
-    const int grid = warp_grid(a.N, num_sms);
-    if (dtype == kF32) return launch_k(dispatch_rows_kernel<float>, dim3(grid), dim3(256), 0, s, a);
-    return launch_k(dispatch_rows_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, a);
+    if (dtype == kF32) return launch_rows(dispatch_rows_kernel<float>, a, a.N, num_sms, s);
+    return launch_rows(dispatch_rows_kernel<__nv_bfloat16>, a, a.N, num_sms, s);
 }
 
 cudaError_t launch_combine(int dtype, const CombineArgs &a, int num_sms, cudaStream_t s)
 {
-    if (a.N == 0) return cudaSuccess;
-    const int grid = warp_grid(a.N, num_sms);
-    if (dtype == kF32) return launch_k(combine_kernel<float>, dim3(grid), dim3(256), 0, s, a);
-    return launch_k(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, a);
+    const int64_t items = a.N * row_blocks(dtype, a.d);
+    if (dtype == kF32) return launch_rows(combine_kernel<float>, a, items, num_sms, s);
+    return launch_rows(combine_kernel<__nv_bfloat16>, a, items, num_sms, s);
 }
 
 cudaError_t launch_z_loss(const float *zpart, int64_t N, float *z_out, cudaStream_t s)
