@@ -75,6 +75,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.oracle_z_loss.restype = f64
     lib.oracle_shared_add.argtypes = [i64, i32, i32, i32, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
     lib.oracle_shared_add.restype = i32
+    lib.oracle_backward.argtypes = [i64, i32, i32, i32, i32, i32, i32, f64, i32, _dp, _dp, _dp, _dp, _dp, _dp,
+                                    _dp, _dp, i32, _dp, _dp, _dp, _dp, _dp, _dp, f64, f64, _ip, _u8p,
+                                    _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
+    lib.oracle_backward.restype = i32
     return lib
 
 
@@ -309,3 +313,42 @@ def forward_tokens(x_rows, ids, w, expert_weights: Callable[[int], Dict[str, Opt
         for j in range(k):
             y[s] += w[s, j] * outs[(s, j)]
     return y
+
+
+def backward(x, Wg, k: int, W1, W2, dy, router: str = "softmax_topk", norm_topk: bool = True,
+             routed_scaling: float = 1.0, act: str = "gelu", W3=None, b1=None, b2=None, b_sel=None,
+             shared: Optional[Dict[str, Optional[np.ndarray]]] = None, aux_coef: float = 0.0,
+             z_coef: float = 0.0, forced_ids=None, forced=None,
+             L: Optional[ctypes.CDLL] = None) -> Dict[str, np.ndarray]:
+    """Gradients of <dy, y> + aux_coef L_aux + z_coef L_z: dx, dW_g, dW1, db1, dW3, dW2, db2 and, with a
+    shared expert ({"W1","W2","W3"?,"b1"?,"b2"?}), dWs1, dbs1, dWs3, dWs2, dbs2."""
+    L = L or lib()
+    x, Wg, dy = _f64(x), _f64(Wg), _f64(dy)
+    W1, W2, W3, b1, b2 = _weights(W1, W2, W3, b1, b2)
+    N, d = x.shape
+    E = Wg.shape[0]
+    F = W1.shape[1]
+    b_sel = None if b_sel is None else _f64(b_sel)
+    sh = {kk: (None if v is None else _f64(v)) for kk, v in (shared or {}).items()}
+    Fs = sh["W1"].shape[0] if sh else 0
+    g = {"dx": np.zeros((N, d)), "dWg": np.zeros((E, d)), "dW1": np.zeros((E, F, d)),
+         "db1": np.zeros((E, F)) if b1 is not None else None,
+         "dW3": np.zeros((E, F, d)) if W3 is not None else None,
+         "dW2": np.zeros((E, d, F)), "db2": np.zeros((E, d)) if b2 is not None else None}
+    if Fs:
+        g.update({"dWs1": np.zeros((Fs, d)), "dbs1": np.zeros(Fs) if sh.get("b1") is not None else None,
+                  "dWs3": np.zeros((Fs, d)) if sh.get("W3") is not None else None,
+                  "dWs2": np.zeros((d, Fs)), "dbs2": np.zeros(d) if sh.get("b2") is not None else None})
+    fi = None if forced_ids is None else _i32(forced_ids)
+    fm = None if forced is None else np.ascontiguousarray(np.asarray(forced, dtype=np.uint8))
+    rc = L.oracle_backward(N, d, F, E, k, ROUTERS[router], int(bool(norm_topk)), float(routed_scaling), ACTS[act],
+                           _p(x, _dp), _p(Wg, _dp), _p(b_sel, _dp), _p(W1, _dp), _p(b1, _dp), _p(W3, _dp),
+                           _p(W2, _dp), _p(b2, _dp), Fs, _p(sh.get("W1"), _dp), _p(sh.get("b1"), _dp),
+                           _p(sh.get("W3"), _dp), _p(sh.get("W2"), _dp), _p(sh.get("b2"), _dp), _p(dy, _dp),
+                           float(aux_coef), float(z_coef), _p(fi, _ip), _p(fm, _u8p),
+                           _p(g["dx"], _dp), _p(g["dWg"], _dp), _p(g["dW1"], _dp), _p(g["db1"], _dp),
+                           _p(g["dW3"], _dp), _p(g["dW2"], _dp), _p(g["db2"], _dp), _p(g.get("dWs1"), _dp),
+                           _p(g.get("dbs1"), _dp), _p(g.get("dWs3"), _dp), _p(g.get("dWs2"), _dp),
+                           _p(g.get("dbs2"), _dp))
+    _check(rc, "oracle_backward")
+    return g

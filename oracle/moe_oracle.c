@@ -475,3 +475,219 @@ int oracle_shared_add(int64_t N, int d, int Fs, int act, const double *x,
     free(h); free(o);
     return ORC_OK;
 }
+
+/* --------------------------------------------------------------- backward */
+
+/*
+ * One FFN (an expert or the shared expert) on one token, backward: given the
+ * gradient `go` of its output o, adds the parameter gradients and the input
+ * gradient.  Recomputes the pre-activations from x.
+ *   GELU  : a = W1 x + b1, h = gelu(a), o = W2 h + b2;
+ *           gelu'(a) = Phi(a) + a phi(a)
+ *   SwiGLU: g = W1 x, u = W3 x, h = silu(g) u, o = W2 h (+ b2);
+ *           silu'(g) = s (1 + g (1 - s)), s = sigmoid(g)
+ * dh = W2^T go; dW2 += go h^T; db2 += go; then da (dg, du) through the
+ * activation; dW1 += da x^T (dW3 += du x^T); db1 += da; dx += W1^T da
+ * (+ W3^T du).  Gradient pointers other than dx may be NULL (not wanted).
+ */
+static void ffn_backward(int d, int F, int act, const double *x, const double *W1, const double *b1,
+                         const double *W3, const double *W2, const double *go, double *dW1, double *db1,
+                         double *dW3, double *dW2, double *db2, double *dx, double *scratch)
+{
+    double *a = scratch, *u = scratch + F, *h = scratch + 2 * F, *dh = scratch + 3 * F;
+    for (int f = 0; f < F; ++f) {
+        double g = 0.0;
+        for (int i = 0; i < d; ++i) g += W1[(int64_t)f * d + i] * x[i];
+        if (act == ORC_SWIGLU) {
+            double v = 0.0;
+            for (int i = 0; i < d; ++i) v += W3[(int64_t)f * d + i] * x[i];
+            a[f] = g;
+            u[f] = v;
+            h[f] = silu(g) * v;
+        } else {
+            if (b1 != NULL) g += b1[f];
+            a[f] = g;
+            h[f] = gelu_exact(g);
+        }
+    }
+    for (int f = 0; f < F; ++f) {
+        double s = 0.0;
+        for (int c = 0; c < d; ++c) s += W2[(int64_t)c * F + f] * go[c];
+        dh[f] = s;
+    }
+    if (dW2)
+        for (int c = 0; c < d; ++c)
+            for (int f = 0; f < F; ++f) dW2[(int64_t)c * F + f] += go[c] * h[f];
+    if (db2) for (int c = 0; c < d; ++c) db2[c] += go[c];
+    for (int f = 0; f < F; ++f) {
+        double da, du = 0.0;
+        if (act == ORC_SWIGLU) {
+            const double sg = sigmoid(a[f]);
+            da = dh[f] * u[f] * sg * (1.0 + a[f] * (1.0 - sg));
+            du = dh[f] * silu(a[f]);
+        } else {
+            const double Phi = 0.5 * (1.0 + erf(a[f] / sqrt(2.0)));
+            const double phi = exp(-0.5 * a[f] * a[f]) / sqrt(2.0 * acos(-1.0));
+            da = dh[f] * (Phi + a[f] * phi);
+            if (db1) db1[f] += da;
+        }
+        for (int i = 0; i < d; ++i) {
+            if (dW1) dW1[(int64_t)f * d + i] += da * x[i];
+            dx[i] += W1[(int64_t)f * d + i] * da;
+            if (act == ORC_SWIGLU) {
+                if (dW3) dW3[(int64_t)f * d + i] += du * x[i];
+                dx[i] += W3[(int64_t)f * d + i] * du;
+            }
+        }
+    }
+}
+
+/*
+ * Backward of the layer (course module sec. 2.1 forward with the sec. 2.3
+ * Switch loss; "nano-moe" router z-loss) for the scalar
+ *   loss = <dy, y> + aux_coef * L_aux + z_coef * L_z,
+ * y = sum_j w_j Expert_{T_n[j]}(x_n) + Shared(x_n).  The expert choice and
+ * f_e = count_e / N are piecewise constant (no gradient); the selection bias
+ * b_sel selects only.  Per token:
+ *   dw_j = <dy_n, o_j> for the j-th expert output o_j; the expert gets the
+ *   output gradient w_j dy_n; the shared expert gets dy_n;
+ *   gates w_j = routed_scaling * g_{T[j]}:
+ *     softmax_topk: g_e = p_e (/ S, S = sum_T p, if norm_topk)
+ *     topk_softmax: g = softmax over z_T
+ *     sigmoid:      g_e = s_e = sigmoid(z_e) (/ sum_T s, if norm_topk)
+ *   L_aux = E sum_e f_e P_e gives dL_aux/dp_{n,e} = E f_e / N (sec. 2.3,
+ *   through P_e = mean_n p_{n,e}, p = softmax(z) for every router);
+ *   L_z = mean_n lse(z_n)^2 gives dL_z/dz_{n,e} = 2 lse(z_n) p_{n,e} / N;
+ *   through p = softmax(z): dz = p (dp - <p, dp>);
+ *   dW_g += dz x_n^T; dx_n += W_g^T dz.
+ * forced_ids / forced replay the routing as in oracle_route.  Every gradient
+ * is zeroed first; shared-expert pointers are NULL when Fs = 0; dWs*, db*
+ * may be NULL where the activation has no such parameter.
+ */
+int oracle_backward(int64_t N, int d, int F, int E, int k, int router, int norm_topk,
+                    double routed_scaling, int act, const double *x, const double *Wg,
+                    const double *b_sel, const double *W1, const double *b1,
+                    const double *W3, const double *W2, const double *b2, int Fs,
+                    const double *Ws1, const double *bs1, const double *Ws3,
+                    const double *Ws2, const double *bs2, const double *dy,
+                    double aux_coef, double z_coef, const int32_t *forced_ids,
+                    const uint8_t *forced, double *dx, double *dWg, double *dW1,
+                    double *db1, double *dW3, double *dW2, double *db2, double *dWs1,
+                    double *dbs1, double *dWs3, double *dWs2, double *dbs2)
+{
+    if (N < 0 || d < 1 || F < 1 || E < 1 || k < 1 || k > E || Fs < 0) return ORC_ERR_ARG;
+    if (act == ORC_SWIGLU && (!W3 || !dW3)) return ORC_ERR_ARG;
+    if (Fs > 0 && (!Ws1 || !Ws2 || !dWs1 || !dWs2 || (act == ORC_SWIGLU && (!Ws3 || !dWs3)))) return ORC_ERR_ARG;
+    memset(dx, 0, sizeof(double) * N * d);
+    memset(dWg, 0, sizeof(double) * E * d);
+    memset(dW1, 0, sizeof(double) * E * F * d);
+    memset(dW2, 0, sizeof(double) * E * d * F);
+    if (dW3) memset(dW3, 0, sizeof(double) * E * F * d);
+    if (db1) memset(db1, 0, sizeof(double) * E * F);
+    if (db2) memset(db2, 0, sizeof(double) * E * d);
+    if (Fs > 0) {
+        memset(dWs1, 0, sizeof(double) * Fs * d);
+        memset(dWs2, 0, sizeof(double) * d * Fs);
+        if (dWs3) memset(dWs3, 0, sizeof(double) * Fs * d);
+        if (dbs1) memset(dbs1, 0, sizeof(double) * Fs);
+        if (dbs2) memset(dbs2, 0, sizeof(double) * d);
+    }
+    if (N == 0) return ORC_OK;
+
+    int32_t *ids = malloc(sizeof(int32_t) * N * k);
+    double *w = malloc(sizeof(double) * N * k);
+    double *probs = malloc(sizeof(double) * N * E);
+    double *logits = malloc(sizeof(double) * N * E);
+    double *cnt = calloc(E, sizeof(double));
+    int Fmax = F > Fs ? F : Fs;
+    double *scratch = malloc(sizeof(double) * 4 * Fmax);
+    double *hbuf = malloc(sizeof(double) * F);
+    double *o = malloc(sizeof(double) * d);
+    double *go = malloc(sizeof(double) * d);
+    double *dp = malloc(sizeof(double) * E);
+    double *dz = malloc(sizeof(double) * E);
+    double *dg = malloc(sizeof(double) * E);
+    if (!ids || !w || !probs || !logits || !cnt || !scratch || !hbuf || !o || !go || !dp || !dz || !dg) {
+        free(ids); free(w); free(probs); free(logits); free(cnt); free(scratch); free(hbuf);
+        free(o); free(go); free(dp); free(dz); free(dg);
+        return ORC_ERR_ARG;
+    }
+    int rc = oracle_route(N, d, E, k, router, norm_topk, routed_scaling, x, Wg, b_sel, forced_ids, forced,
+                          ids, w, probs, logits, NULL);
+    if (rc == ORC_OK) {
+        for (int64_t a = 0; a < N * k; ++a) cnt[ids[a]] += 1.0;
+        for (int64_t n = 0; n < N; ++n) {
+            const double *xn = x + n * d, *dyn = dy + n * d, *p = probs + n * E, *z = logits + n * E;
+            const int32_t *idn = ids + n * k;
+            double *dxn = dx + n * d;
+            for (int e = 0; e < E; ++e) dg[e] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                const int e = idn[j];
+                expert_on_token(d, F, act, e, xn, W1, b1, W3, W2, b2, hbuf, o);
+                double dwj = 0.0;
+                for (int c = 0; c < d; ++c) dwj += dyn[c] * o[c];
+                dg[e] += routed_scaling * dwj;  /* gradient of the unscaled gate */
+                for (int c = 0; c < d; ++c) go[c] = w[n * k + j] * dyn[c];
+                ffn_backward(d, F, act, xn, W1 + (int64_t)e * F * d, b1 ? b1 + (int64_t)e * F : NULL,
+                             W3 ? W3 + (int64_t)e * F * d : NULL, W2 + (int64_t)e * d * F, go,
+                             dW1 + (int64_t)e * F * d, db1 ? db1 + (int64_t)e * F : NULL,
+                             dW3 ? dW3 + (int64_t)e * F * d : NULL, dW2 + (int64_t)e * d * F,
+                             db2 ? db2 + (int64_t)e * d : NULL, dxn, scratch);
+            }
+            if (Fs > 0)
+                ffn_backward(d, Fs, act, xn, Ws1, bs1, Ws3, Ws2, dyn, dWs1, dbs1, dWs3, dWs2, dbs2, dxn,
+                             scratch);
+
+            /* gates -> dp (softmax probabilities) and dz (direct) */
+            for (int e = 0; e < E; ++e) { dp[e] = 0.0; dz[e] = 0.0; }
+            if (router == ORC_SOFTMAX_TOPK) {
+                if (norm_topk) {
+                    double S = 0.0, gp = 0.0;
+                    for (int j = 0; j < k; ++j) { S += p[idn[j]]; gp += dg[idn[j]] * p[idn[j]]; }
+                    for (int j = 0; j < k; ++j) dp[idn[j]] += dg[idn[j]] / S - gp / (S * S);
+                } else {
+                    for (int j = 0; j < k; ++j) dp[idn[j]] += dg[idn[j]];
+                }
+            } else if (router == ORC_TOPK_SOFTMAX) {
+                double cmax = z[idn[0]], s = 0.0, gdot = 0.0;
+                for (int j = 1; j < k; ++j) if (z[idn[j]] > cmax) cmax = z[idn[j]];
+                for (int j = 0; j < k; ++j) s += exp(z[idn[j]] - cmax);
+                for (int j = 0; j < k; ++j) gdot += exp(z[idn[j]] - cmax) / s * dg[idn[j]];
+                for (int j = 0; j < k; ++j) {
+                    const double gj = exp(z[idn[j]] - cmax) / s;
+                    dz[idn[j]] += gj * (dg[idn[j]] - gdot);
+                }
+            } else {
+                double S = 0.0, gs = 0.0;
+                for (int j = 0; j < k; ++j) { S += sigmoid(z[idn[j]]); gs += dg[idn[j]] * sigmoid(z[idn[j]]); }
+                for (int j = 0; j < k; ++j) {
+                    const int e = idn[j];
+                    const double s = sigmoid(z[e]);
+                    const double ds = norm_topk ? dg[e] / S - gs / (S * S) : dg[e];
+                    dz[e] += ds * s * (1.0 - s);
+                }
+            }
+            /* Switch loss through P_e = mean_n p_{n,e} */
+            for (int e = 0; e < E; ++e) dp[e] += aux_coef * (double)E * (cnt[e] / (double)N) / (double)N;
+            double pdp = 0.0;
+            for (int e = 0; e < E; ++e) pdp += p[e] * dp[e];
+            for (int e = 0; e < E; ++e) dz[e] += p[e] * (dp[e] - pdp);
+            /* router z-loss */
+            if (z_coef != 0.0) {
+                double zmax = z[0], s = 0.0;
+                for (int e = 1; e < E; ++e) if (z[e] > zmax) zmax = z[e];
+                for (int e = 0; e < E; ++e) s += exp(z[e] - zmax);
+                const double lse_n = zmax + log(s);
+                for (int e = 0; e < E; ++e) dz[e] += z_coef * 2.0 * lse_n * p[e] / (double)N;
+            }
+            for (int e = 0; e < E; ++e)
+                for (int i = 0; i < d; ++i) {
+                    dWg[(int64_t)e * d + i] += dz[e] * xn[i];
+                    dxn[i] += Wg[(int64_t)e * d + i] * dz[e];
+                }
+        }
+    }
+    free(ids); free(w); free(probs); free(logits); free(cnt); free(scratch); free(hbuf);
+    free(o); free(go); free(dp); free(dz); free(dg);
+    return rc;
+}

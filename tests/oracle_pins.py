@@ -453,4 +453,91 @@ def pin_shared_expert_numpy(L):
     _close(z, np.ones((3, 4)), 0.0, "zero shared expert adds nothing")
 
 
+
+def _fd_case(L, rng, N, d, F, E, k, act, router, norm_topk, scaling, biases, shared_F, sel_bias, aux_coef, z_coef):
+    """Central finite differences of the oracle's own forward loss
+    <dy, y> + aux_coef L_aux + z_coef L_z against oracle_backward, for every
+    entry of every input and parameter (ids held at the unperturbed routing)."""
+    x, Wg, W1, W2, W3, b1, b2 = _rand_problem(rng, N, d, F, E, act, biases)
+    b_sel = rng.uniform(-0.1, 0.1, E) if sel_bias else None
+    sh = None
+    if shared_F:
+        sh = {"W1": rng.standard_normal((shared_F, d)) / math.sqrt(d),
+              "W2": rng.standard_normal((d, shared_F)) / math.sqrt(shared_F),
+              "W3": rng.standard_normal((shared_F, d)) / math.sqrt(d) if act == "swiglu" else None,
+              "b1": rng.standard_normal(shared_F) * 0.1 if (biases and act == "gelu") else None,
+              "b2": rng.standard_normal(d) * 0.1 if biases else None}
+    dy = rng.standard_normal((N, d))
+    r0 = O.route(x, Wg, k, router, norm_topk, scaling, b_sel=b_sel, L=L)
+    assert np.min(r0["margin"]) > 1e-4, "pick a seed with clear routing"
+    ids0 = r0["ids"]
+    forced = np.ones(N, np.uint8)
+    P = {"x": x, "Wg": Wg, "W1": W1, "W2": W2, "W3": W3, "b1": b1, "b2": b2}
+    if sh:
+        P.update({"Ws1": sh["W1"], "Ws2": sh["W2"], "Ws3": sh["W3"], "bs1": sh["b1"], "bs2": sh["b2"]})
+
+    def loss():
+        r = O.route(P["x"], P["Wg"], k, router, norm_topk, scaling, b_sel=b_sel, forced_ids=ids0, forced=forced, L=L)
+        y = O.dense_forward(P["x"], ids0, r["w"], P["W1"], P["W2"], act, P["W3"], P["b1"], P["b2"], L=L)
+        if sh:
+            y = O.shared_add(y, P["x"], P["Ws1"], P["Ws2"], act, P["Ws3"], P["bs1"], P["bs2"], L=L)
+        aux, _ = O.aux_loss(r["probs"], ids0, L=L)
+        return float(np.sum(dy * y)) + aux_coef * aux + z_coef * O.z_loss(r["logits"], L=L)
+
+    shared = None if not sh else {"W1": P["Ws1"], "W2": P["Ws2"], "W3": P["Ws3"], "b1": P["bs1"], "b2": P["bs2"]}
+    g = O.backward(x, Wg, k, W1, W2, dy, router, norm_topk, scaling, act, W3, b1, b2, b_sel, shared,
+                   aux_coef, z_coef, L=L)
+    names = {"x": "dx", "Wg": "dWg", "W1": "dW1", "W2": "dW2", "W3": "dW3", "b1": "db1", "b2": "db2",
+             "Ws1": "dWs1", "Ws2": "dWs2", "Ws3": "dWs3", "bs1": "dbs1", "bs2": "dbs2"}
+    h = 1e-5
+    for pname, arr in P.items():
+        if arr is None:
+            continue
+        fd = np.zeros_like(arr)
+        flat = arr.reshape(-1)
+        for i in range(flat.size):
+            v = flat[i]
+            flat[i] = v + h
+            lp = loss()
+            flat[i] = v - h
+            lm = loss()
+            flat[i] = v
+            fd.reshape(-1)[i] = (lp - lm) / (2 * h)
+        an = g[names[pname]]
+        assert an is not None and an.shape == arr.shape, pname
+        err = float(np.max(np.abs(fd - an) / np.maximum(1.0, np.abs(an))))
+        assert err <= 1e-6, f"{router}/{act}: d{pname} off by {err:.2e} (finite differences)"
+
+
+def pin_backward_finite_differences(L):
+    """Every gradient of oracle_backward equals the central difference of the
+    forward loss (routing held fixed: the choice and f_e are piecewise
+    constant), for each router, both activations, biases, a shared expert,
+    routed_scaling, the aux-free bias, the Switch loss and the router z-loss."""
+    rng = np.random.default_rng(91)
+    _fd_case(L, rng, 4, 4, 5, 4, 2, "gelu", "softmax_topk", True, 1.0, True, 3, False, 0.3, 0.2)
+    _fd_case(L, rng, 4, 4, 3, 5, 2, "swiglu", "sigmoid", True, 2.5, False, 3, True, 0.5, 0.1)
+    _fd_case(L, rng, 3, 4, 3, 4, 3, "swiglu", "topk_softmax", True, 1.0, False, 0, False, 1.0, 0.0)
+    _fd_case(L, rng, 4, 3, 4, 4, 2, "gelu", "softmax_topk", False, 1.0, False, 0, False, 0.7, 0.3)
+    _fd_case(L, rng, 3, 3, 3, 3, 3, "gelu", "sigmoid", False, 1.0, True, 0, True, 0.4, 0.0)
+
+
+def pin_aux_gradient_is_E_f_over_N(L):
+    """[course] sec. 2.3: dL_aux / dp_{n,e} = E f_e / N.  With dy = 0 and only
+    the Switch loss, dW_g = sum_n (J_softmax(z_n) c) x_n^T, c_e = E f_e / N."""
+    rng = np.random.default_rng(93)
+    N, d, E, k = 7, 5, 6, 2
+    x = rng.standard_normal((N, d))
+    Wg = rng.standard_normal((E, d))
+    W1 = rng.standard_normal((E, 3, d))
+    W2 = rng.standard_normal((E, d, 3))
+    r = O.route(x, Wg, k, L=L)
+    f = np.bincount(r["ids"].reshape(-1), minlength=E) / N
+    c = E * f / N
+    p = r["probs"]
+    dz = p * (c[None, :] - (p @ c)[:, None])
+    g = O.backward(x, Wg, k, W1, W2, np.zeros((N, d)), aux_coef=1.0, L=L)
+    _close(g["dWg"], dz.T @ x, 1e-12, "dW_g of the Switch loss")
+    _close(g["dW1"], np.zeros_like(W1), 0.0, "no expert gradient without dy")
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

@@ -53,6 +53,19 @@ MUTANTS = {
     "z_loss_not_squared": ("total += lse * lse;", "total += lse;"),
     "z_loss_no_max_shift": ("const double lse = zmax + log(s);", "const double lse = log(s);"),
     "shared_not_added": ("for (int c = 0; c < d; ++c) y[n * d + c] += o[c];", "for (int c = 0; c < d; ++c) y[n * d + c] = o[c];"),
+    "bwd_softmax_jacobian_no_mean": ("for (int e = 0; e < E; ++e) dz[e] += p[e] * (dp[e] - pdp);",
+                                     "for (int e = 0; e < E; ++e) dz[e] += p[e] * dp[e];"),
+    "bwd_silu_derivative_short": ("da = dh[f] * u[f] * sg * (1.0 + a[f] * (1.0 - sg));", "da = dh[f] * u[f] * sg;"),
+    "bwd_gelu_derivative_short": ("da = dh[f] * (Phi + a[f] * phi);", "da = dh[f] * Phi;"),
+    "bwd_aux_missing_E": ("dp[e] += aux_coef * (double)E * (cnt[e] / (double)N) / (double)N;",
+                          "dp[e] += aux_coef * (cnt[e] / (double)N) / (double)N;"),
+    "bwd_z_loss_not_doubled": ("dz[e] += z_coef * 2.0 * lse_n * p[e] / (double)N;",
+                               "dz[e] += z_coef * lse_n * p[e] / (double)N;"),
+    "bwd_gate_scaling_dropped": ("dg[e] += routed_scaling * dwj;", "dg[e] += dwj;"),
+    "bwd_norm_term_dropped": ("for (int j = 0; j < k; ++j) dp[idn[j]] += dg[idn[j]] / S - gp / (S * S);",
+                              "for (int j = 0; j < k; ++j) dp[idn[j]] += dg[idn[j]] / S;"),
+    "bwd_W2_grad_transposed": ("for (int f = 0; f < F; ++f) dW2[(int64_t)c * F + f] += go[c] * h[f];",
+                               "for (int f = 0; f < F; ++f) dW2[(int64_t)c * F + f] += go[f % d] * h[c % F];"),
     "combine_drops_last_slot": ("for (int j = 0; j < k; ++j) {\n            const double *src",
                                 "for (int j = 0; j + 1 < k; ++j) {\n            const double *src"),
 }
