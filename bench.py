@@ -57,6 +57,8 @@ def parse_args():
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--tokens", type=int, default=0, help="override N (small profiling cases)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
+                   help="backward: time moe_backward (fp32 gradients of <dy, y> + losses) instead")
     return p.parse_args()
 
 
@@ -464,6 +466,84 @@ def run_native(args, wl):
         dist.destroy_process_group()
 
 
+def backward_flops(wl) -> int:
+    """Algorithmic FLOPs of one moe_backward: the recomputed pre-activations
+    (mats - 1 products), dh = dy_s W2, dx_s (mats - 1), the weight gradients
+    (mats), for N k rows of d x d_ff each; the router's 2 dz products; the
+    shared expert's 3 mats - 1 products over N rows."""
+    m = wl.mats
+    rows = wl.N * wl.k
+    per = 2 * wl.d_model * wl.d_ff
+    expert = rows * per * ((m - 1) + 1 + (m - 1) + m)
+    router = 2 * 2 * wl.N * wl.E * wl.d_model
+    shared = wl.N * 2 * wl.d_model * wl.d_ff_shared * (3 * m - 1) if wl.d_ff_shared else 0
+    return expert + router + shared
+
+
+def run_backward(args, wl):
+    """Times moe_backward; its products run on the CUDA cores, so the roofline
+    is the fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x the sampled clock."""
+    import ctypes
+
+    import torch
+
+    import mixture_experts_layer_53_b200 as M
+    import workloads as W
+
+    rank, local_rank, world = dist_env()
+    if rank != 0:
+        return
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    M.library()
+    cfg = M.make_config(wl.N, wl.d_model, wl.d_ff, wl.E, wl.k, wl.router, wl.norm_topk, wl.routed_scaling,
+                        wl.act, wl.dtype, wl.d_ff_shared)
+    inp = W.make_inputs(wl, dev)
+    g = torch.Generator().manual_seed(wl.seed * 7 + 9)
+    dy = torch.randn((wl.N, wl.d_model), generator=g).to(wl.torch_dtype).to(dev)
+    n = int(M.library().moe_backward_workspace_size(ctypes.byref(cfg)))
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=dev)
+    ws = ws[(-ws.data_ptr()) % 256:][:n]
+
+    def step(out=None):
+        return M.moe_backward(cfg, inp["x"], inp["W_g"], inp["W1"], inp["W2"], dy, W3=inp["W3"], b1=inp["b1"],
+                              b2=inp["b2"], b_e=inp["b_e"], shared=inp["shared"], aux_coef=1e-2, z_coef=1e-3,
+                              ws=ws, out=out)
+
+    out = step()
+    for _ in range(max(0, args.warmup - 1)):
+        step(out)
+    torch.cuda.synchronize()
+    assert int(out["status"][0]) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        w0 = time.monotonic()
+        e0.record()
+        for _ in range(args.steps):
+            step(out)
+        e1.record()
+        torch.cuda.synchronize()
+        clocks.mark(w0, time.monotonic())
+    ms = e0.elapsed_time(e1) / args.steps
+    cl = clocks.summary()
+    flops = backward_flops(wl)
+    achieved = flops / (ms / 1000.0) / 1e12
+    mhz = cl.get("sm_mhz") or 1965.0
+    peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+    line = {
+        "metric": "MoE-layer backward tokens/sec (fp32 gradients, 1 B200)", "value": wl.N / (ms / 1000.0),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "config": describe(wl),
+        "roofline": {"kernel": "gemm_generic_kernel (all backward products)", "bound": "alu", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x sampled SM clock",
+                     "flops_per_step": flops},
+        "clocks": cl,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     import workloads as W
@@ -472,6 +552,8 @@ def main():
         wl = wl.scaled(N=args.tokens)
     if args.impl == "reference":
         run_reference(args, wl)
+    elif args.which == "backward":
+        run_backward(args, wl)
     else:
         run_native(args, wl)
 

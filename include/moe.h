@@ -321,6 +321,60 @@ MOE_API moe_status moe_forward_ex(const moe_config *cfg, const void *x, const vo
                           int32_t *dev_status, void *ws, size_t ws_bytes,
                           void *const *stage_events, moe_stream_t stream);
 
+/*
+ * Gradients written by moe_backward: fp32, row-major, caller-owned device
+ * memory, each overwritten (not accumulated).  Shapes as the parameters:
+ * dx [N, d_model], dW_g [E, d_model], dW1 / dW3 [E, d_ff, d_model],
+ * db1 [E, d_ff], dW2 [E, d_model, d_ff], db2 [E, d_model]; the shared
+ * expert's dWs1 / dWs3 [d_ff_shared, d_model], dbs1 [d_ff_shared],
+ * dWs2 [d_model, d_ff_shared], dbs2 [d_model].  A gradient whose parameter
+ * is absent (dW3 for GELU, db1 without b1, ...) is ignored and may be NULL;
+ * dx, dW_g, dW1, dW2 (and dW3 for SwiGLU, dWs1 / dWs2 (/ dWs3) with a shared
+ * expert) are required.
+ */
+typedef struct {
+    float *dx;
+    float *dW_g;
+    float *dW1;
+    float *db1;
+    float *dW3;
+    float *dW2;
+    float *db2;
+    float *dWs1;
+    float *dbs1;
+    float *dWs3;
+    float *dWs2;
+    float *dbs2;
+} moe_grads;
+
+/* Workspace bytes moe_backward needs for cfg (0 for an invalid cfg). */
+MOE_API size_t moe_backward_workspace_size(const moe_config *cfg);
+
+/*
+ * Backward of the layer for an upstream gradient dy [N, d_model] (layer
+ * dtype): the gradients of
+ *   loss = <dy, y> + aux_coef * L_aux + z_coef * L_z
+ * with y, L_aux (Switch loss, course module sec. 2.3) and L_z (router
+ * z-loss, "nano-moe") as moe_forward_ex computes them from the same inputs.
+ * b_e must be the selection bias the forward selected with (before its
+ * sign-rule step).  The expert choice and f_e = count_e / N are piecewise
+ * constant and carry no gradient (course module sec. 2.4); the bias selects
+ * only.  Per token: the
+ * gate of expert e gets <dy_n, Expert_e(x_n)>, the expert the output
+ * gradient w dy_n, the shared expert dy_n; the Switch loss reaches the
+ * router through dL_aux / dp_{n,e} = E f_e / N (course module sec. 2.3),
+ * the z-loss through 2 lse(z_n) p_n / N.  The routing and the
+ * expert pre-activations are recomputed (same kernels as the forward, so the
+ * same expert choice); all products accumulate in fp32.  Enqueues only.
+ */
+MOE_API moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g,
+                        const float *b_e, const void *W1, const void *b1,
+                        const void *W3, const void *W2, const void *b2,
+                        const moe_shared_expert *shared, const void *dy,
+                        float aux_coef, float z_coef, const moe_grads *grads,
+                        int32_t *dev_status, void *ws, size_t ws_bytes,
+                        moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

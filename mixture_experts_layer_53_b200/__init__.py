@@ -36,7 +36,8 @@ NUM_STAGES = 5
 STAGE_NAMES = ("route", "dispatch", "gemm1", "gemm2", "combine")
 EXPORTS = ("moe_status_string", "moe_last_error", "moe_version", "moe_workspace_size", "moe_route",
            "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_combine", "moe_aux_loss",
-           "moe_forward", "moe_shared_ffn", "moe_combine_shared", "moe_router_z_loss", "moe_forward_ex")
+           "moe_forward", "moe_shared_ffn", "moe_combine_shared", "moe_router_z_loss", "moe_forward_ex",
+           "moe_backward_workspace_size", "moe_backward")
 # ceil(N / 32) * E limit of moe_dispatch_noalloc (MOE_NOALLOC_DISPATCH_MAX_SLOTS)
 NOALLOC_DISPATCH_MAX_SLOTS = 1 << 19
 
@@ -57,6 +58,12 @@ class SharedExpert(ctypes.Structure):
     """Mirror of ``moe_shared_expert`` in include/moe.h (device pointers)."""
     _fields_ = [("W1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("W3", ctypes.c_void_p),
                 ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p)]
+
+
+class MoeGrads(ctypes.Structure):
+    """Mirror of ``moe_grads`` in include/moe.h (fp32 device pointers)."""
+    _fields_ = [(name, ctypes.c_void_p) for name in
+                ("dx", "dW_g", "dW1", "db1", "dW3", "dW2", "db2", "dWs1", "dbs1", "dWs3", "dWs2", "dbs2")]
 
 
 class MoeError(RuntimeError):
@@ -115,6 +122,11 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_forward_ex.argtypes = [cfgp, vp, vp, f32p, ctypes.c_float, vp, vp, vp, vp, vp, shp, vp, i32p, f32p,
                                    i32p, f32p, f32p, i32p, vp, sz, ctypes.c_void_p, vp]
     lib.moe_forward_ex.restype = st
+    lib.moe_backward_workspace_size.argtypes = [cfgp]
+    lib.moe_backward_workspace_size.restype = sz
+    lib.moe_backward.argtypes = [cfgp, vp, vp, f32p, vp, vp, vp, vp, vp, shp, vp, ctypes.c_float, ctypes.c_float,
+                                 ctypes.POINTER(MoeGrads), i32p, vp, sz, vp]
+    lib.moe_backward.restype = st
     if path is None:
         _lib = lib
     return lib
@@ -303,6 +315,46 @@ def moe_aux_loss(cfg: MoeConfig, probs: torch.Tensor, topk_ids: torch.Tensor, ga
     return aux, counts, status
 
 
+def moe_backward(cfg: MoeConfig, x: torch.Tensor, W_g: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor,
+                 dy: torch.Tensor, W3: Optional[torch.Tensor] = None, b1: Optional[torch.Tensor] = None,
+                 b2: Optional[torch.Tensor] = None, b_e: Optional[torch.Tensor] = None,
+                 shared: Optional[Dict[str, Optional[torch.Tensor]]] = None, aux_coef: float = 0.0,
+                 z_coef: float = 0.0, ws: Optional[torch.Tensor] = None,
+                 out: Optional[Dict[str, torch.Tensor]] = None, stream=None) -> Dict[str, torch.Tensor]:
+    """fp32 gradients of <dy, y> + aux_coef L_aux + z_coef L_z (moe_backward): dx, dW_g, dW1, dW2 and, as
+    the layer has them, db1, dW3, db2 and the shared expert's dWs1, dbs1, dWs3, dWs2, dbs2; plus status."""
+    dev = x.device
+    if ws is None:
+        n = int(library().moe_backward_workspace_size(ctypes.byref(cfg)))
+        if n == 0:
+            raise MoeError(1, "moe_backward_workspace_size")
+        raw = torch.empty(n + 256, dtype=torch.uint8, device=dev)
+        off = (-raw.data_ptr()) % 256
+        ws = raw[off:off + n]
+    f32 = dict(dtype=torch.float32, device=dev)
+    N, d, F, E, Fs = cfg.N, cfg.d_model, cfg.d_ff, cfg.E, cfg.d_ff_shared
+    if out is None:
+        out = {"dx": torch.empty((N, d), **f32), "dW_g": torch.empty((E, d), **f32),
+               "dW1": torch.empty((E, F, d), **f32), "dW2": torch.empty((E, d, F), **f32),
+               "db1": torch.empty((E, F), **f32) if b1 is not None else None,
+               "dW3": torch.empty((E, F, d), **f32) if W3 is not None else None,
+               "db2": torch.empty((E, d), **f32) if b2 is not None else None}
+        if shared is not None:
+            out.update({"dWs1": torch.empty((Fs, d), **f32), "dWs2": torch.empty((d, Fs), **f32),
+                        "dWs3": torch.empty((Fs, d), **f32) if shared.get("W3") is not None else None,
+                        "dbs1": torch.empty(Fs, **f32) if shared.get("b1") is not None else None,
+                        "dbs2": torch.empty(d, **f32) if shared.get("b2") is not None else None})
+        out["status"] = torch.zeros(1, dtype=torch.int32, device=dev)
+    g = MoeGrads(*[(_ptr(out.get(k)).value if out.get(k) is not None else None) for k, _ in MoeGrads._fields_])
+    sh = _shared_struct(shared)
+    rc = library().moe_backward(ctypes.byref(cfg), _ptr(x), _ptr(W_g), _ptr(b_e), _ptr(W1), _ptr(b1), _ptr(W3),
+                                _ptr(W2), _ptr(b2), ctypes.byref(sh) if sh else None, _ptr(dy), float(aux_coef),
+                                float(z_coef), ctypes.byref(g), _ptr(out["status"]), _ptr(ws), ws.numel(),
+                                _stream(stream))
+    _check(rc, "moe_backward")
+    return out
+
+
 class StageEvents:
     """CUDA events that moe_forward records at stage boundaries.
 
@@ -441,5 +493,6 @@ def forward_outputs(cfg: MoeConfig, device) -> Dict[str, torch.Tensor]:
 
 __all__ = ["MoeConfig", "SharedExpert", "MoeError", "make_config", "library", "workspace", "moe_workspace_size",
            "moe_route", "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_combine", "moe_aux_loss",
-           "moe_forward", "moe_shared_ffn", "moe_combine_shared", "moe_router_z_loss", "forward_outputs",
+           "moe_forward", "moe_shared_ffn", "moe_combine_shared", "moe_router_z_loss", "moe_backward",
+           "MoeGrads", "forward_outputs",
            "StageEvents", "HostPipeline", "EXPORTS", "LIB_PATH"]

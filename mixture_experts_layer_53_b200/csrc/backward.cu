@@ -1,0 +1,261 @@
+// backward.cu -- element-wise and per-token kernels of the layer backward.
+//
+// The scalar differentiated is loss = <dy, y> + aux_coef L_aux + z_coef L_z
+// for the forward of the course module (sec. 2.1 with the sec. 2.3 Switch
+// loss) and the "nano-moe" router z-loss.  The expert choice and f_e are
+// piecewise constant; the selection bias only selects.  Everything here is
+// fp32; the products between these kernels run on gemm_generic_kernel.
+#include <float.h>
+
+#include "common.cuh"
+#include "host_util.h"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+__device__ __forceinline__ float sigmoidf_(float v) { return 1.0f / (1.0f + expf(-v)); }
+
+// Element i of a layer-dtype array (bf16 or fp32).
+__device__ __forceinline__ float ldv(const void *p, int64_t i, int bf16)
+{
+    return bf16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]) : static_cast<const float *>(p)[i];
+}
+
+// Per sorted row r: its token, gate weight and expert (from perm and the
+// routing); thread 0 of block 0 also stores the constant 1.0 that the bias
+// gradients use as a one-element B operand.
+__global__ void rows_prep_kernel(BwdRowsArgs a)
+{
+    pdl_enter();
+    if (blockIdx.x == 0 && threadIdx.x == 0) *a.one = 1.0f;
+    for (int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; r < a.rows;
+         r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int32_t asg = a.perm[r];
+        a.row_tok[r] = asg / a.k;
+        a.row_w[r] = a.w[asg];
+        a.row_e[r] = a.ids[asg];
+    }
+}
+
+// Pre-activations a (+ b1 for GELU) and the hidden activations h.
+__global__ void act_forward_kernel(BwdActArgs a)
+{
+    pdl_enter();
+    const int64_t total = a.rows * a.F;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = i / a.F;
+        const int f = static_cast<int>(i - r * a.F);
+        float v = a.pre[i];
+        if (a.act == kSwiglu) {
+            a.h[i] = silu(v) * a.up[i];
+        } else {
+            if (a.b1) {
+                const int e = a.row_e ? a.row_e[r] : 0;
+                v += ldv(a.b1, static_cast<int64_t>(e) * a.F + f, a.bf16);
+                a.pre[i] = v;
+            }
+            a.h[i] = gelu_erf(v);
+        }
+    }
+}
+
+// One warp per sorted row r, given dh_raw = dy_s W2[e] (the output gradient
+// before the gate weight):
+//   dw_r = <dh_raw_r, h_r> + <dy_s r, b2[e]>     (= <dy_n, Expert_e(x_n)>)
+//   dh = w_r dh_raw_r through the activation: pre <- da, up <- du, and
+//   h <- w_r h (the right operand of dW2 = dy_s^T (w h)).
+// Without a weight array (the shared expert) w_r = 1 and dw is not kept.
+__global__ void __launch_bounds__(256) row_backward_kernel(BwdActArgs a)
+{
+    pdl_enter();
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < a.rows;
+         r += warps) {
+        const float wr = a.row_w ? a.row_w[r] : 1.0f;
+        const int e = a.row_e ? a.row_e[r] : 0;
+        float* pre = a.pre + r * a.F;
+        float* up = a.up ? a.up + r * a.F : nullptr;
+        float* h = a.h + r * a.F;
+        const float* dh = a.dh + r * a.F;
+        if (a.dw) {
+            float s = 0.f;
+            for (int f = lane; f < a.F; f += 32) s += dh[f] * h[f];
+            if (a.b2) {
+                for (int c = lane; c < a.d; c += 32)
+                    s += ldv(a.dy_s, r * a.d + c, a.bf16) * ldv(a.b2, static_cast<int64_t>(e) * a.d + c, a.bf16);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            if (lane == 0) a.dw[a.perm[r]] = s;
+        }
+        for (int f = lane; f < a.F; f += 32) {
+            const float g = wr * dh[f];
+            const float v = pre[f];
+            if (a.act == kSwiglu) {
+                const float sg = sigmoidf_(v);
+                const float u = up[f];
+                pre[f] = g * u * sg * (1.0f + v * (1.0f - sg));
+                up[f] = g * v * sg;
+            } else {
+                const float Phi = 0.5f * (1.0f + erff(v * 0.70710678118654752f));
+                const float phi = 0.39894228040143268f * expf(-0.5f * v * v);
+                pre[f] = g * (Phi + v * phi);
+            }
+            h[f] *= wr;
+        }
+    }
+}
+
+// dx_n = sum_j dx_s[inv_perm[n k + j]] (fp32), one warp per token.
+__global__ void __launch_bounds__(256) gather_sum_kernel(BwdGatherSumArgs a)
+{
+    pdl_enter();
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); n < a.N;
+         n += warps) {
+        const int src_l = lane < a.k ? a.inv_perm[n * a.k + lane] : 0;
+        for (int c0 = 0; c0 < a.d; c0 += 32) {  // warp-uniform
+            const int c = c0 + lane;
+            float s = 0.f;
+            for (int j = 0; j < a.k; ++j) {
+                const int src = __shfl_sync(0xffffffffu, src_l, j);
+                if (c < a.d) s += a.dxs[static_cast<int64_t>(src) * a.d + c];
+            }
+            if (c < a.d) a.dx[n * a.d + c] = s;
+        }
+    }
+}
+
+// Router backward, one warp per token (lane l holds experts l + 32 j).
+// dg_e = routed_scaling dw_j for the chosen experts; then per router
+//   softmax_topk: dp = dg (/ S - <dg, p>_T / S^2 with norm_topk)
+//   topk_softmax: dz_T = g (dg - <g, dg>_T), g = p / S over the chosen
+//   sigmoid:      ds = dg (/ S - <dg, s>_T / S^2), dz = ds s (1 - s),
+//                 s = sigmoid(z), z = log p + lse
+// plus dp_e += aux_coef E f_e / N (Switch loss through P_e), dz += p (dp -
+// <p, dp>) (softmax), dz += z_coef 2 lse p / N (z-loss).
+__global__ void __launch_bounds__(256) router_backward_kernel(BwdRouterArgs a)
+{
+    pdl_enter();
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    const int E = a.E, k = a.k;
+    const float invN = 1.0f / static_cast<float>(a.N);
+    for (int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); n < a.N;
+         n += warps) {
+        const float *p = a.probs + n * E;
+        const float lse = a.lse[n];
+        // the k choices: lane j < k holds id, p, dg and (sigmoid) s
+        const int id_l = lane < k ? a.ids[n * k + lane] : 0;
+        const float p_l = lane < k ? p[id_l] : 0.f;
+        const float dg_l = lane < k ? a.scaling * a.dw[n * k + lane] : 0.f;
+        const float s_l = (lane < k && a.router == kSigmoid) ? sigmoidf_(logf(p_l) + lse) : 0.f;
+        float S = 0.f, gdot = 0.f;
+        if (a.router == kSigmoid) {
+            S = s_l;
+            gdot = dg_l * s_l;
+        } else {
+            S = p_l;
+            gdot = dg_l * p_l;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            S += __shfl_xor_sync(0xffffffffu, S, o);
+            gdot += __shfl_xor_sync(0xffffffffu, gdot, o);
+        }
+        // per chosen expert: its dp (softmax path) or its direct dz
+        float dp_l = 0.f, dzd_l = 0.f;
+        if (lane < k) {
+            if (a.router == kSoftmaxTopk) {
+                dp_l = a.norm_topk ? dg_l / S - gdot / (S * S) : dg_l;
+            } else if (a.router == kTopkSoftmax) {
+                const float g = p_l / S;
+                dzd_l = g * (dg_l - gdot / S);
+            } else {
+                const float ds = a.norm_topk ? dg_l / S - gdot / (S * S) : dg_l;
+                dzd_l = ds * s_l * (1.0f - s_l);
+            }
+        }
+        // expert e's dp and direct dz, <p, dp>; the shuffles run in every
+        // lane (warp-uniform loops), only the accumulation is per lane
+        float dp[8], dzd[8], pdp = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            dp[j] = 0.f;
+            dzd[j] = 0.f;
+        }
+        for (int q = 0; q < k; ++q) {
+            const int idq = __shfl_sync(0xffffffffu, id_l, q);
+            const float dpq = __shfl_sync(0xffffffffu, dp_l, q);
+            const float dzq = __shfl_sync(0xffffffffu, dzd_l, q);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (idq == lane + 32 * j) {
+                    dp[j] += dpq;
+                    dzd[j] += dzq;
+                }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) {
+                dp[j] += a.aux_coef * static_cast<float>(E) * (static_cast<float>(a.counts[e]) * invN) * invN;
+                pdp += p[e] * dp[j];
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pdp += __shfl_xor_sync(0xffffffffu, pdp, o);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) {
+                float dz = dzd[j] + p[e] * (dp[j] - pdp);
+                if (a.z_coef != 0.f) dz += a.z_coef * 2.0f * lse * p[e] * invN;
+                a.dz[n * E + e] = dz;
+            }
+        }
+    }
+}
+
+int grid_for(int64_t work, int per_block, int num_sms)
+{
+    const int64_t want = (work + per_block - 1) / per_block;
+    return static_cast<int>(max64(1, min64(want, static_cast<int64_t>(num_sms) * 16)));
+}
+
+}  // namespace
+
+cudaError_t launch_rows_prep(const BwdRowsArgs &a, int num_sms, cudaStream_t s)
+{
+    return launch_k(rows_prep_kernel, dim3(grid_for(max64(a.rows, 1), 256, num_sms)), dim3(256), 0, s, a);
+}
+
+cudaError_t launch_act_forward(const BwdActArgs &a, int num_sms, cudaStream_t s)
+{
+    if (a.rows == 0) return cudaSuccess;
+    return launch_k(act_forward_kernel, dim3(grid_for(a.rows * a.F, 256, num_sms)), dim3(256), 0, s, a);
+}
+
+cudaError_t launch_row_backward(const BwdActArgs &a, int num_sms, cudaStream_t s)
+{
+    if (a.rows == 0) return cudaSuccess;
+    return launch_k(row_backward_kernel, dim3(grid_for(a.rows, 8, num_sms)), dim3(256), 0, s, a);
+}
+
+cudaError_t launch_gather_sum(const BwdGatherSumArgs &a, int num_sms, cudaStream_t s)
+{
+    if (a.N == 0) return cudaSuccess;
+    return launch_k(gather_sum_kernel, dim3(grid_for(a.N, 8, num_sms)), dim3(256), 0, s, a);
+}
+
+cudaError_t launch_router_backward(const BwdRouterArgs &a, int num_sms, cudaStream_t s)
+{
+    if (a.N == 0) return cudaSuccess;
+    return launch_k(router_backward_kernel, dim3(grid_for(a.N, 8, num_sms)), dim3(256), 0, s, a);
+}
+
+}  // namespace moe

@@ -26,6 +26,7 @@ struct RouterArgs {
     int64_t N;
     int d, E, k, router, norm_topk;
     float scaling;
+    float *lse;          // [N] per-token log-sum-exp of the logits, or null
 };
 // CUDA-core router (fp32 path).
 cudaError_t launch_router(int dtype, const RouterArgs &a, cudaStream_t s);
@@ -57,6 +58,7 @@ struct SelectKernelArgs {
     int ld, E, k, router, norm_topk;
     float scaling;
     int splits;
+    float *lse;           // [N] or null
 };
 cudaError_t launch_select(const SelectKernelArgs &a, cudaStream_t s);
 
@@ -153,6 +155,78 @@ cudaError_t launch_combine(int dtype, const CombineArgs &a, int num_sms, cudaStr
 
 // mt_prefix[e+1] = mt_prefix[e] + ceil((offsets[e+1] - offsets[e]) / tile_m).
 cudaError_t launch_tile_table(const int32_t *offsets, int32_t *mt_prefix, int E, int tile_m, cudaStream_t s);
+
+// Strided grouped GEMM on the CUDA cores, fp32 out (backward products):
+// C_g(m, n) (+)= sum_k A(m, k) B_g(k, n), A(m, k) = A[m sam + k sak],
+// B_g(k, n) = B[g sbg + k sbk + n sbn], C_g(m, n) = C[g scg + m scm + n scn].
+// ragged_k = 0: group g owns rows offsets[g] .. offsets[g+1]-1 of A and C
+// (mt_prefix: the per-group 64-row tile prefix, launch with an upper bound
+// on the tiles); ragged_k = 1: group g sums k over offsets[g] ..
+// offsets[g+1]-1.
+struct GenericGemmArgs {
+    const void *A;
+    int64_t sam, sak;
+    const void *B;
+    int64_t sbk, sbn, sbg;
+    float *C;
+    int64_t scm, scn, scg;
+    const int32_t *offsets;
+    const int32_t *mt_prefix;
+    int G;
+    int ragged_k;
+    int64_t M, N, K;
+    int accumulate, a_bf16, b_bf16;
+};
+constexpr int kGenericTileM = 64;
+cudaError_t launch_gemm_generic(const GenericGemmArgs &g, int64_t max_tiles_m, cudaStream_t s);
+
+// ---- backward (backward.cu)
+struct BwdRowsArgs {
+    const int32_t *perm, *ids;  // sorted position -> assignment; [N k]
+    const float *w;             // [N k] gate weights
+    int64_t rows;
+    int k;
+    int32_t *row_tok, *row_e;   // [rows]
+    float *row_w;               // [rows]
+    float *one;                 // receives 1.0f
+};
+cudaError_t launch_rows_prep(const BwdRowsArgs &a, int num_sms, cudaStream_t s);
+
+struct BwdActArgs {
+    int64_t rows;
+    int F, d, act, bf16;   // bf16: the layer dtype of b1, b2, dy_s
+    float *pre, *up, *h;   // [rows, F]: pre-activations, SwiGLU up, h
+    const float *dh;       // [rows, F]: dy_s W2[e]
+    const void *b1, *b2;   // [E, F], [E, d] or null
+    const int32_t *row_e;  // [rows] or null (expert 0)
+    const float *row_w;    // [rows] or null (weight 1)
+    float *dw;             // [N k] or null: <dy_n, Expert(x_n)> per assignment
+    const int32_t *perm;   // [rows] (with dw)
+    const void *dy_s;      // [rows, d] (with dw and b2)
+};
+cudaError_t launch_act_forward(const BwdActArgs &a, int num_sms, cudaStream_t s);
+cudaError_t launch_row_backward(const BwdActArgs &a, int num_sms, cudaStream_t s);
+
+struct BwdGatherSumArgs {
+    const float *dxs;          // [N k, d]
+    const int32_t *inv_perm;   // [N k]
+    float *dx;                 // [N, d]
+    int64_t N;
+    int d, k;
+};
+cudaError_t launch_gather_sum(const BwdGatherSumArgs &a, int num_sms, cudaStream_t s);
+
+struct BwdRouterArgs {
+    const float *probs, *lse;  // [N, E], [N]
+    const int32_t *ids;        // [N k]
+    const float *dw;           // [N k]
+    const int32_t *counts;     // [E]
+    float *dz;                 // [N, E]
+    int64_t N;
+    int E, k, router, norm_topk;
+    float scaling, aux_coef, z_coef;
+};
+cudaError_t launch_router_backward(const BwdRouterArgs &a, int num_sms, cudaStream_t s);
 
 struct FfnArgs {
     const void *x_sorted;      // [rows, d]

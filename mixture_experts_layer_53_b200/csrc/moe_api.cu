@@ -202,7 +202,7 @@ cudaError_t launch_route(const moe_config *c, const RouterArgs &r, int32_t *stat
     cudaError_t err = launch_router_logits_sm100(r.x, r.Wg, logits, r.N, r.d, r.E, status, clear_status, s);
     if (err != cudaSuccess) return err;
     SelectKernelArgs sk{logits, r.b_sel, r.ids, r.w, r.probs, r.hist, r.psum, r.zpart, r.N, logits_ld(r.E),
-                        r.E, r.k, r.router, r.norm_topk, r.scaling, router_splits(r.N, r.d)};
+                        r.E, r.k, r.router, r.norm_topk, r.scaling, router_splits(r.N, r.d), r.lse};
     return launch_select(sk, s);
 }
 
@@ -245,6 +245,105 @@ cudaError_t launch_shared(const moe_config *c, const moe_shared_expert *sh, cons
     f.act = c->act;
     f.tile_m = shared_tile_m(c);
     return launch_ffn(c, f, nullptr, s);
+}
+
+// ------------------------------------------------------------- backward
+
+struct BwdLayout {
+    size_t hist, logits, offsets, mt64, counts, ids, w, perm, inv, probs, lse, xs, dys, row_tok, row_e, row_w,
+        pre, up, h, dh, dxs, dw, dz, doff, dmt, one, spre, sup, sh, sdh, total;
+};
+
+BwdLayout bwd_layout(const moe_config *c)
+{
+    BwdLayout L{};
+    size_t o = 0;
+    auto take = [&o](size_t bytes) {
+        const size_t at = o;
+        o += align256(bytes > 0 ? bytes : 1);
+        return at;
+    };
+    const size_t C = static_cast<size_t>(num_chunks(c->N));
+    const size_t E = static_cast<size_t>(c->E);
+    const size_t Nn = static_cast<size_t>(c->N);
+    const size_t A = Nn * static_cast<size_t>(c->k);
+    const size_t es = elem_size(c);
+    const size_t d = static_cast<size_t>(c->d_model), F = static_cast<size_t>(c->d_ff);
+    const size_t Fs = static_cast<size_t>(c->d_ff_shared);
+    const bool swiglu = c->act == MOE_ACT_SWIGLU;
+    L.hist = take(C * E * 4);
+    L.logits = take(static_cast<size_t>(router_splits(c->N, c->d_model)) * Nn * logits_ld(c->E) * 4);
+    L.offsets = take((E + 1) * 4);
+    L.mt64 = take((E + 1) * 4);
+    L.counts = take(E * 4);
+    L.ids = take(A * 4);
+    L.w = take(A * 4);
+    L.perm = take(A * 4);
+    L.inv = take(A * 4);
+    L.probs = take(Nn * E * 4);
+    L.lse = take(Nn * 4);
+    L.xs = take(A * d * es);
+    L.dys = take(A * d * es);
+    L.row_tok = take(A * 4);
+    L.row_e = take(A * 4);
+    L.row_w = take(A * 4);
+    L.pre = take(A * F * 4);
+    L.up = take(swiglu ? A * F * 4 : 0);
+    L.h = take(A * F * 4);
+    L.dh = take(A * F * 4);
+    L.dxs = take(A * d * 4);
+    L.dw = take(A * 4);
+    L.dz = take(Nn * E * 4);
+    L.doff = take(2 * 4);
+    L.dmt = take(2 * 4);
+    L.one = take(4);
+    L.spre = take(Nn * Fs * 4);
+    L.sup = take(swiglu ? Nn * Fs * 4 : 0);
+    L.sh = take(Nn * Fs * 4);
+    L.sdh = take(Nn * Fs * 4);
+    L.total = o;
+    return L;
+}
+
+// One strided product on gemm_generic_kernel (see kernels.h).
+struct GG {
+    GenericGemmArgs g{};
+    GG &a(const void *p, int64_t sm, int64_t sk, bool bf16)
+    {
+        g.A = p; g.sam = sm; g.sak = sk; g.a_bf16 = bf16 ? 1 : 0;
+        return *this;
+    }
+    GG &b(const void *p, int64_t sk, int64_t sn, int64_t sg, bool bf16)
+    {
+        g.B = p; g.sbk = sk; g.sbn = sn; g.sbg = sg; g.b_bf16 = bf16 ? 1 : 0;
+        return *this;
+    }
+    GG &c(float *p, int64_t sm, int64_t sn, int64_t sg, bool acc = false)
+    {
+        g.C = p; g.scm = sm; g.scn = sn; g.scg = sg; g.accumulate = acc ? 1 : 0;
+        return *this;
+    }
+    // rows offsets[gi] .. offsets[gi+1]-1 of A and C per group; N columns, K depth
+    cudaError_t rows(const int32_t *off, const int32_t *mt, int G, int64_t rows_total, int64_t N, int64_t K,
+                     cudaStream_t s)
+    {
+        g.offsets = off; g.mt_prefix = mt; g.G = G; g.ragged_k = 0; g.N = N; g.K = K;
+        return launch_gemm_generic(g, (rows_total + kGenericTileM - 1) / kGenericTileM + G, s);
+    }
+    // per group an M x N result summed over rows offsets[gi] .. offsets[gi+1]-1
+    cudaError_t sum_rows(const int32_t *off, int G, int64_t M, int64_t N, cudaStream_t s)
+    {
+        g.offsets = off; g.mt_prefix = nullptr; g.G = G; g.ragged_k = 1; g.M = M; g.N = N;
+        return launch_gemm_generic(g, 0, s);
+    }
+};
+
+moe_status check_grads(const moe_config *c, const moe_grads *gr, bool shared)
+{
+    if (!gr || (c->N > 0 && !gr->dx) || !gr->dW_g || !gr->dW1 || !gr->dW2) return MOE_ERR_INVALID_ARG;
+    if (c->act == MOE_ACT_SWIGLU && !gr->dW3) return MOE_ERR_INVALID_ARG;
+    if (shared && (!gr->dWs1 || !gr->dWs2 || (c->act == MOE_ACT_SWIGLU && !gr->dWs3))) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
 }
 
 }  // namespace
@@ -545,6 +644,165 @@ moe_status moe_forward_ex(const moe_config *cfg, const void *x, const void *W_g,
     CombineArgs ca{ys, w, inv, y, cfg->N, cfg->d_model, cfg->k, ysh};
     if ((err = launch_combine(cfg->dtype, ca, num_sms(), s)) != cudaSuccess) return cuda_fail(err);
     if ((err = mark(5)) != cudaSuccess) return cuda_fail(err);
+    return MOE_OK;
+}
+
+size_t moe_backward_workspace_size(const moe_config *cfg)
+{
+    if (validate(cfg) != MOE_OK) return 0;
+    return bwd_layout(cfg).total;
+}
+
+moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, const float *b_e, const void *W1,
+                        const void *b1, const void *W3, const void *W2, const void *b2,
+                        const moe_shared_expert *shared, const void *dy, float aux_coef, float z_coef,
+                        const moe_grads *grads, int32_t *dev_status, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (!W_g || (cfg->N > 0 && (!x || !dy))) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W_g) || !aligned16(dy)) return MOE_ERR_INVALID_ARG;
+    if (b_e && cfg->router != MOE_ROUTER_SIGMOID) return MOE_ERR_INVALID_ARG;
+    if (!std::isfinite(aux_coef) || !std::isfinite(z_coef)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ffn_ptrs(cfg, W1, b1, W3, W2, b2)) != MOE_OK) return st;
+    if ((st = check_shared(cfg, shared)) != MOE_OK) return st;
+    if ((st = check_grads(cfg, grads, shared != nullptr)) != MOE_OK) return st;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < bwd_layout(cfg).total)
+        return MOE_ERR_WORKSPACE;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const BwdLayout L = bwd_layout(cfg);
+    const int64_t N = cfg->N, rows = N * cfg->k;
+    const int E = cfg->E, k = cfg->k, d = cfg->d_model, F = cfg->d_ff, Fs = cfg->d_ff_shared;
+    const bool bf = cfg->dtype == MOE_BF16, swiglu = cfg->act == MOE_ACT_SWIGLU;
+    const moe_grads &gr = *grads;
+    cudaError_t err;
+#define MOE_TRY(call)                                   \
+    do {                                                \
+        if ((err = (call)) != cudaSuccess) return cuda_fail(err); \
+    } while (0)
+    if (dev_status) MOE_TRY(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s));
+    if (N == 0) {  // empty sums: every parameter gradient is zero
+        MOE_TRY(cudaMemsetAsync(gr.dW_g, 0, sizeof(float) * E * d, s));
+        MOE_TRY(cudaMemsetAsync(gr.dW1, 0, sizeof(float) * E * F * d, s));
+        MOE_TRY(cudaMemsetAsync(gr.dW2, 0, sizeof(float) * E * d * F, s));
+        if (swiglu) MOE_TRY(cudaMemsetAsync(gr.dW3, 0, sizeof(float) * E * F * d, s));
+        if (b1 && gr.db1) MOE_TRY(cudaMemsetAsync(gr.db1, 0, sizeof(float) * E * F, s));
+        if (b2 && gr.db2) MOE_TRY(cudaMemsetAsync(gr.db2, 0, sizeof(float) * E * d, s));
+        if (shared) {
+            MOE_TRY(cudaMemsetAsync(gr.dWs1, 0, sizeof(float) * Fs * d, s));
+            MOE_TRY(cudaMemsetAsync(gr.dWs2, 0, sizeof(float) * d * Fs, s));
+            if (swiglu) MOE_TRY(cudaMemsetAsync(gr.dWs3, 0, sizeof(float) * Fs * d, s));
+            if (shared->b1 && gr.dbs1) MOE_TRY(cudaMemsetAsync(gr.dbs1, 0, sizeof(float) * Fs, s));
+            if (shared->b2 && gr.dbs2) MOE_TRY(cudaMemsetAsync(gr.dbs2, 0, sizeof(float) * d, s));
+        }
+        return MOE_OK;
+    }
+    const int sms = num_sms();
+    int32_t *hist = at<int32_t>(ws, L.hist), *offsets = at<int32_t>(ws, L.offsets), *mt = at<int32_t>(ws, L.mt64);
+    int32_t *counts = at<int32_t>(ws, L.counts), *ids = at<int32_t>(ws, L.ids), *perm = at<int32_t>(ws, L.perm);
+    int32_t *inv = at<int32_t>(ws, L.inv), *doff = at<int32_t>(ws, L.doff), *dmt = at<int32_t>(ws, L.dmt);
+    float *w = at<float>(ws, L.w), *probs = at<float>(ws, L.probs), *lse = at<float>(ws, L.lse);
+    void *xs = at<void>(ws, L.xs), *dys = at<void>(ws, L.dys);
+    float *row_w = at<float>(ws, L.row_w), *pre = at<float>(ws, L.pre), *up = swiglu ? at<float>(ws, L.up) : nullptr;
+    float *h = at<float>(ws, L.h), *dh = at<float>(ws, L.dh), *dxs = at<float>(ws, L.dxs), *dw = at<float>(ws, L.dw);
+    float *dz = at<float>(ws, L.dz), *one = at<float>(ws, L.one);
+
+    // ---- recompute: routing (with p and lse), counts, slices, x_sorted
+    RouterArgs r = router_args(cfg, x, W_g, b_e, ids, w, probs, hist, nullptr);
+    r.lse = lse;
+    MOE_TRY(launch_route(cfg, r, dev_status, at<float>(ws, L.logits), s));
+    ScanArgs sc{};
+    sc.hist = hist;
+    sc.chunks = num_chunks(N);
+    sc.N = N;
+    sc.E = E;
+    sc.k = k;
+    sc.counts = counts;
+    sc.offsets = offsets;
+    sc.mt_prefix = mt;
+    sc.tile_m = kGenericTileM;
+    sc.dense_offsets = doff;  // {0, N}: one group of all tokens
+    sc.dense_mt = dmt;
+    sc.dense_tile_m = kGenericTileM;
+    MOE_TRY(launch_scan(sc, s));
+    DispatchRowsArgs da{ids, hist, offsets, perm, inv, x, xs, N, d, E, k};
+    MOE_TRY(launch_dispatch_rows(cfg->dtype, da, sms, s));
+    BwdRowsArgs ra{perm, ids, w, rows, k, at<int32_t>(ws, L.row_tok), at<int32_t>(ws, L.row_e), row_w, one};
+    MOE_TRY(launch_rows_prep(ra, sms, s));
+    GatherArgs gd{dy, inv, dys, N, d, k};  // dy_s[r] = dy[token of r]
+    MOE_TRY(launch_gather(cfg->dtype, gd, sms, s));
+
+    // ---- expert pre-activations and h (fp32)
+    MOE_TRY(GG().a(xs, d, 1, bf).b(W1, 1, d, static_cast<int64_t>(F) * d, bf).c(pre, F, 1, 0)
+                .rows(offsets, mt, E, rows, F, d, s));
+    if (swiglu)
+        MOE_TRY(GG().a(xs, d, 1, bf).b(W3, 1, d, static_cast<int64_t>(F) * d, bf).c(up, F, 1, 0)
+                    .rows(offsets, mt, E, rows, F, d, s));
+    BwdActArgs act{rows, F, d, cfg->act, bf ? 1 : 0, pre, up, h, dh, swiglu ? nullptr : b1, b2,
+                   at<int32_t>(ws, L.row_e), row_w, dw, perm, dys};
+    MOE_TRY(launch_act_forward(act, sms, s));
+
+    // ---- output side: dh = dy_s W2[e]; gates, activation backward
+    MOE_TRY(GG().a(dys, d, 1, bf).b(W2, F, 1, static_cast<int64_t>(d) * F, bf).c(dh, F, 1, 0)
+                .rows(offsets, mt, E, rows, F, d, s));
+    MOE_TRY(launch_row_backward(act, sms, s));
+    // dW2[e] = dy_s^T (w h), db2[e] = sum_r w_r dy_s r
+    MOE_TRY(GG().a(dys, 1, d, bf).b(h, F, 1, 0, false).c(gr.dW2, F, 1, static_cast<int64_t>(d) * F)
+                .sum_rows(offsets, E, d, F, s));
+    if (b2 && gr.db2)
+        MOE_TRY(GG().a(dys, 1, d, bf).b(row_w, 1, 0, 0, false).c(gr.db2, 1, 0, d).sum_rows(offsets, E, d, 1, s));
+
+    // ---- input side: dx_s = da W1[e] (+ du W3[e]); dW1, dW3, db1
+    MOE_TRY(GG().a(pre, F, 1, false).b(W1, d, 1, static_cast<int64_t>(F) * d, bf).c(dxs, d, 1, 0)
+                .rows(offsets, mt, E, rows, d, F, s));
+    if (swiglu)
+        MOE_TRY(GG().a(up, F, 1, false).b(W3, d, 1, static_cast<int64_t>(F) * d, bf).c(dxs, d, 1, 0, true)
+                    .rows(offsets, mt, E, rows, d, F, s));
+    MOE_TRY(GG().a(pre, 1, F, false).b(xs, d, 1, 0, bf).c(gr.dW1, d, 1, static_cast<int64_t>(F) * d)
+                .sum_rows(offsets, E, F, d, s));
+    if (swiglu)
+        MOE_TRY(GG().a(up, 1, F, false).b(xs, d, 1, 0, bf).c(gr.dW3, d, 1, static_cast<int64_t>(F) * d)
+                    .sum_rows(offsets, E, F, d, s));
+    if (!swiglu && b1 && gr.db1)
+        MOE_TRY(GG().a(pre, 1, F, false).b(one, 0, 0, 0, false).c(gr.db1, 1, 0, F).sum_rows(offsets, E, F, 1, s));
+    BwdGatherSumArgs gs{dxs, inv, gr.dx, N, d, k};
+    MOE_TRY(launch_gather_sum(gs, sms, s));
+
+    // ---- router: dz, dW_g = dz^T x, dx += dz W_g
+    BwdRouterArgs rb{probs, lse, ids, dw, counts, dz, N, E, k, cfg->router, cfg->norm_topk, cfg->routed_scaling,
+                     aux_coef, z_coef};
+    MOE_TRY(launch_router_backward(rb, sms, s));
+    MOE_TRY(GG().a(dz, 1, E, false).b(x, d, 1, 0, bf).c(gr.dW_g, d, 1, 0).sum_rows(doff, 1, E, d, s));
+    MOE_TRY(GG().a(dz, E, 1, false).b(W_g, d, 1, 0, bf).c(gr.dx, d, 1, 0, true).rows(doff, dmt, 1, N, d, E, s));
+
+    // ---- shared expert: the same with weight 1 over all N rows of x
+    if (shared) {
+        float *spre = at<float>(ws, L.spre), *sup = swiglu ? at<float>(ws, L.sup) : nullptr;
+        float *sh = at<float>(ws, L.sh), *sdh = at<float>(ws, L.sdh);
+        MOE_TRY(GG().a(x, d, 1, bf).b(shared->W1, 1, d, 0, bf).c(spre, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
+        if (swiglu)
+            MOE_TRY(GG().a(x, d, 1, bf).b(shared->W3, 1, d, 0, bf).c(sup, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
+        BwdActArgs sa{N, Fs, d, cfg->act, bf ? 1 : 0, spre, sup, sh, sdh, swiglu ? nullptr : shared->b1, nullptr,
+                      nullptr, nullptr, nullptr, nullptr, nullptr};
+        MOE_TRY(launch_act_forward(sa, sms, s));
+        MOE_TRY(GG().a(dy, d, 1, bf).b(shared->W2, Fs, 1, 0, bf).c(sdh, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
+        MOE_TRY(launch_row_backward(sa, sms, s));
+        MOE_TRY(GG().a(dy, 1, d, bf).b(sh, Fs, 1, 0, false).c(gr.dWs2, Fs, 1, 0).sum_rows(doff, 1, d, Fs, s));
+        if (shared->b2 && gr.dbs2)
+            MOE_TRY(GG().a(dy, 1, d, bf).b(one, 0, 0, 0, false).c(gr.dbs2, 1, 0, 0).sum_rows(doff, 1, d, 1, s));
+        MOE_TRY(GG().a(spre, 1, Fs, false).b(x, d, 1, 0, bf).c(gr.dWs1, d, 1, 0).sum_rows(doff, 1, Fs, d, s));
+        if (swiglu)
+            MOE_TRY(GG().a(sup, 1, Fs, false).b(x, d, 1, 0, bf).c(gr.dWs3, d, 1, 0).sum_rows(doff, 1, Fs, d, s));
+        if (!swiglu && shared->b1 && gr.dbs1)
+            MOE_TRY(GG().a(spre, 1, Fs, false).b(one, 0, 0, 0, false).c(gr.dbs1, 1, 0, 0).sum_rows(doff, 1, Fs, 1, s));
+        MOE_TRY(GG().a(spre, Fs, 1, false).b(shared->W1, d, 1, 0, bf).c(gr.dx, d, 1, 0, true)
+                    .rows(doff, dmt, 1, N, d, Fs, s));
+        if (swiglu)
+            MOE_TRY(GG().a(sup, Fs, 1, false).b(shared->W3, d, 1, 0, bf).c(gr.dx, d, 1, 0, true)
+                        .rows(doff, dmt, 1, N, d, Fs, s));
+    }
+#undef MOE_TRY
     return MOE_OK;
 }
 

@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a)
     }
 
     // ---- scores, top-k and gates, one token at a time per warp
-    SelectArgs sa{a.b_sel, a.ids, a.w, a.probs, E, k, a.router, a.norm_topk, a.scaling};
+    SelectArgs sa{a.b_sel, a.ids, a.w, a.probs, E, k, a.router, a.norm_topk, a.scaling, a.lse};
 #pragma unroll 1
     for (int i = 0; i < 4; ++i) {
         const int t = warp + 8 * i;
@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int e = threadIdx.x; e < E; e += kSelWarps * 32) hist_s[e] = 0;
     __syncthreads();
-    const SelectArgs sa{a.b_sel, a.ids, a.w, a.probs, E, k, a.router, a.norm_topk, a.scaling};
+    const SelectArgs sa{a.b_sel, a.ids, a.w, a.probs, E, k, a.router, a.norm_topk, a.scaling, a.lse};
     // software pipeline: the next token's row is loaded while this one is
     // selected
     float znext[EJ];

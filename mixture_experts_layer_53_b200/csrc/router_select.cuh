@@ -25,6 +25,7 @@ struct SelectArgs {
     float *probs;        // [N, E] or null
     int E, k, router, norm_topk;
     float scaling;
+    float *lse;          // [N] log-sum-exp of each token's logits, or null
 };
 
 // (value desc, id asc): does (v, e) rank ahead of (bv, be)?
@@ -123,6 +124,7 @@ __device__ __forceinline__ float select_token(float (&z)[8], const SelectArgs &a
 #pragma unroll
     for (int r = 0; r < kMaxK; ++r)
         if (r < k) gs += gsel[r];
+    if (write && a.lse && lane == 0) a.lse[n] = zmax + logf(esum);
     if (write) {
 #pragma unroll
         for (int r = 0; r < kMaxK; ++r) {
@@ -234,6 +236,7 @@ __device__ __forceinline__ float select_token_keys(float (&z)[EJ], const SelectA
     float gs = lane < k ? my_gate : 0.f;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
+    if (write && a.lse && lane == 0) a.lse[n] = zmax + logf(esum);
     if (write && lane < k) {
         float wr;
         if (a.router == kSoftmaxTopk) wr = a.norm_topk ? my_gate / gs : my_gate * inv_esum;
@@ -348,6 +351,7 @@ __device__ __forceinline__ void select_thread_chunk(float (&z)[EB], const Select
         for (int e = 0; e < EB; ++e) cnt[e] += (live && be == e) ? 1 : 0;
     }
     if (live) {
+        if (a.lse) a.lse[n] = lse;
 #pragma unroll 1
         for (int r = 0; r < k; ++r) {
             float wr;

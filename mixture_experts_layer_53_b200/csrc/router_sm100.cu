@@ -369,7 +369,7 @@ cudaError_t launch_router_fused_sm100(const RouterArgs &r, int32_t *status, bool
     LArgs a{};
     CUtensorMap tX, tW;
     if (!setup(a, tX, tW, r.x, r.Wg, r.N, r.d, r.E, status, clear_status)) return cudaErrorInvalidValue;
-    a.sel = SelectArgs{r.b_sel, r.ids, r.w, r.probs, r.E, r.k, r.router, r.norm_topk, r.scaling};
+    a.sel = SelectArgs{r.b_sel, r.ids, r.w, r.probs, r.E, r.k, r.router, r.norm_topk, r.scaling, r.lse};
     a.psum = r.psum;
     a.hist = r.hist;
     a.zpart = r.zpart;

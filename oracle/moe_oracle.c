@@ -547,8 +547,8 @@ static void ffn_backward(int d, int F, int act, const double *x, const double *W
  * Switch loss; "nano-moe" router z-loss) for the scalar
  *   loss = <dy, y> + aux_coef * L_aux + z_coef * L_z,
  * y = sum_j w_j Expert_{T_n[j]}(x_n) + Shared(x_n).  The expert choice and
- * f_e = count_e / N are piecewise constant (no gradient); the selection bias
- * b_sel selects only.  Per token:
+ * f_e = count_e / N are piecewise constant (no gradient, sec. 2.4); the
+ * selection bias b_sel selects only.  Per token:
  *   dw_j = <dy_n, o_j> for the j-th expert output o_j; the expert gets the
  *   output gradient w_j dy_n; the shared expert gets dy_n;
  *   gates w_j = routed_scaling * g_{T[j]}:

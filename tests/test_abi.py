@@ -55,13 +55,18 @@ int main(void) {
   printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(moe_shared_expert), offsetof(moe_shared_expert, W1),
          offsetof(moe_shared_expert, b1), offsetof(moe_shared_expert, W3), offsetof(moe_shared_expert, W2),
          offsetof(moe_shared_expert, b2));
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(moe_grads), offsetof(moe_grads, dx),
+         offsetof(moe_grads, dW_g), offsetof(moe_grads, dW1), offsetof(moe_grads, db1), offsetof(moe_grads, dW3),
+         offsetof(moe_grads, dW2), offsetof(moe_grads, db2), offsetof(moe_grads, dWs1), offsetof(moe_grads, dbs1),
+         offsetof(moe_grads, dWs3), offsetof(moe_grads, dWs2), offsetof(moe_grads, dbs2));
   return 0;
 }
 """)
     exe = tmp_path / "probe"
     subprocess.check_call(["gcc", "-std=c11", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)])
     lines = subprocess.check_output([str(exe)], text=True).splitlines()
-    for line, C in zip(lines, (M.MoeConfig, M.SharedExpert)):
+    assert len(lines) == 3
+    for line, C in zip(lines, (M.MoeConfig, M.SharedExpert, M.MoeGrads)):
         got = [int(v) for v in line.split()]
         want = [ctypes.sizeof(C)] + [getattr(C, f).offset for f, _ in C._fields_]
         assert got == want, C.__name__
@@ -206,3 +211,23 @@ def test_workspace_holds_the_shared_expert(lib):
     n2 = lib.moe_workspace_size(ctypes.byref(cfg(**base, d_ff_shared=1024)))
     assert n1 - n0 >= 1024 * 256 * 2 - 256         # + y_shared [N, d] (an empty region still takes 256 B)
     assert n2 >= n1 + 1024 * (1024 - 2 * 128) * 2  # h grows to N * Fs once that exceeds N k F
+
+
+def test_backward_validation(lib):
+    a = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x100000)
+    big = ctypes.c_size_t(1 << 40)
+    c = cfg(act="swiglu")
+    assert lib.moe_backward_workspace_size(ctypes.byref(c)) > lib.moe_workspace_size(ctypes.byref(c))
+    full = M.MoeGrads(*([0x20000] * 12))
+    no_dw3 = M.MoeGrads(0x20000, 0x20000, 0x20000, None, None, 0x20000, None, None, None, None, None, None)
+    args = lambda g, dy=a, aux=0.0: (ctypes.byref(c), a, a, None, a, None, a, a, None, None, dy, ctypes.c_float(aux),
+                                     ctypes.c_float(0.0), ctypes.byref(g) if g is not None else None, None, ws, big,
+                                     None)
+    assert lib.moe_backward(*args(no_dw3)) == 1          # SwiGLU needs dW3
+    assert lib.moe_backward(*args(None)) == 1            # no gradient struct
+    assert lib.moe_backward(*args(full, dy=None)) == 1   # dy missing
+    assert lib.moe_backward(*args(full, aux=float("inf"))) == 1
+    small = ctypes.c_size_t(lib.moe_workspace_size(ctypes.byref(c)))
+    assert lib.moe_backward(ctypes.byref(c), a, a, None, a, None, a, a, None, None, a, ctypes.c_float(0.0),
+                            ctypes.c_float(0.0), ctypes.byref(full), None, ws, small, None) == 4
