@@ -23,8 +23,9 @@
 //              CTA's `full` barrier, which expects both CTAs' bytes)
 //   warp 1     TMEM allocation for the pair (both CTAs); in the even CTA one
 //              lane issues the MMAs and commits to both CTAs' barriers
-//   warps 2-5  epilogue on the CTA's own 128 rows (tcgen05.ld), fused
-//              activation / bias, bf16 stores
+//   warps 2-9  epilogue on the CTA's own 128 rows (tcgen05.ld), two warps
+//              per TMEM lane quarter, each on half of the tile's output
+//              columns; fused activation / bias, bf16 stores
 // SwiGLU: the even CTA's B half holds 128 rows of W1 and the odd CTA's the
 // same 128 rows of W3, so accumulator columns 0..127 are the gate and
 // 128..255 the up projection of 128 hidden units.
@@ -48,7 +49,8 @@ constexpr int STAGES = 6;
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int B_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's half of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;  // two per TMEM lane quarter, each on half of the columns
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 
 
@@ -98,14 +100,15 @@ __device__ __forceinline__ Tile decode_tile(int t, const Ctl *c, int E, int n_ti
 
 template <int EPI> __host__ __device__ constexpr int out_cols() { return EPI == EPI_SWIGLU ? 128 : 256; }
 
+// Output columns [c_begin, c_end) of one accumulator row (this thread's row).
 template <int EPI>
 __device__ __forceinline__ void epilogue_rows(const GemmArgs &g, uint32_t tbase, int e, int row, bool row_ok,
-                                              int n0)
+                                              int n0, int c_begin, int c_end)
 {
     __nv_bfloat16 *orow = g.out + static_cast<int64_t>(row) * g.ldo;
     const __nv_bfloat16 *brow = g.bias ? g.bias + static_cast<int64_t>(e) * g.n_out : nullptr;
 #pragma unroll 1
-    for (int c = 0; c < out_cols<EPI>(); c += 32) {
+    for (int c = c_begin; c < c_end; c += 32) {
         uint32_t acc[32];
         tmem_ld32(tbase + c, acc);
         if constexpr (EPI == EPI_SWIGLU) {
@@ -176,7 +179,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->tfull[b], 1);
-            mbar_init(&ctl->tempty[b], 8);
+            mbar_init(&ctl->tempty[b], 2 * EPI_WARPS);  // every epilogue warp of both CTAs
         }
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
@@ -295,6 +298,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     } else {
         // ---------------------------------------------------- epilogue
         const int quarter = warp & 3;  // TMEM lanes this warp may access
+        const int half = (warp - 2) / 4;  // which half of the output columns
         const int row_in_cta = quarter * 32 + lane;
         const uint32_t tempty_leader0 = mapa_shared(smem_u32(&ctl->tempty[0]), 0);
         const uint32_t tempty_leader1 = mapa_shared(smem_u32(&ctl->tempty[1]), 0);
@@ -309,7 +313,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const bool row_ok = row < ctl->off[ti.e + 1];
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
-            epilogue_rows<EPI>(g, tbase, ti.e, row, row_ok, ti.n_tile * out_cols<EPI>());
+            epilogue_rows<EPI>(g, tbase, ti.e, row, row_ok, ti.n_tile * out_cols<EPI>(), half * out_cols<EPI>() / 2,
+                               (half + 1) * out_cols<EPI>() / 2);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
