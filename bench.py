@@ -481,8 +481,9 @@ def backward_flops(wl) -> int:
 
 
 def run_backward(args, wl):
-    """Times moe_backward; its products run on the CUDA cores, so the roofline
-    is the fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x the sampled clock."""
+    """Times moe_backward.  bf16: the expert products run on the tensor cores
+    (roofline: the measured sustained bf16 peak); fp32: on the CUDA cores
+    (roofline: 148 SMs x 128 fp32 lanes x 2 FLOP x the sampled SM clock)."""
     import ctypes
 
     import torch
@@ -529,16 +530,24 @@ def run_backward(args, wl):
     flops = backward_flops(wl)
     achieved = flops / (ms / 1000.0) / 1e12
     mhz = cl.get("sm_mhz") or 1965.0
-    peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+    if wl.dtype == "bf16":
+        peaks, peak_src = load_peaks()
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        bound, kern = "tensor", "ffn_gemm_single_kernel<F32> (expert dgrad / wgrad products)"
+        src = f"{peak_src} bf16_tflops_sustained"
+    else:
+        peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+        bound, kern = "alu", "gemm_generic_kernel (all backward products)"
+        src = "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x sampled SM clock"
     line = {
         "metric": "MoE-layer backward tokens/sec (fp32 gradients, 1 B200)", "value": wl.N / (ms / 1000.0),
         "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
         "config": describe(wl),
-        "roofline": {"kernel": "gemm_generic_kernel (all backward products)", "bound": "alu", "achieved": achieved,
-                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x sampled SM clock",
-                     "flops_per_step": flops},
+        "roofline": {"kernel": kern, "bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_source": src, "flops_per_step": flops,
+                     "note": "achieved = all backward FLOPs over the whole step (transposes, element-wise and "
+                             "router kernels included)"},
         "clocks": cl,
     }
     print(json.dumps(line), flush=True)

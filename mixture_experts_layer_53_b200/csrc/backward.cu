@@ -221,6 +221,88 @@ __global__ void __launch_bounds__(256) router_backward_kernel(BwdRouterArgs a)
     }
 }
 
+__global__ void pad_offsets_kernel(const int32_t *counts, int32_t *kpad, int E)
+{
+    pdl_enter();
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        int32_t o = 0;
+        for (int e = 0; e < E; ++e) {
+            kpad[e] = o;
+            o += (counts[e] + 63) / 64 * 64;
+        }
+        kpad[E] = o;
+    }
+}
+
+// 32 x 32 tiles through shared memory: coalesced reads along C, writes along
+// the (padded) row positions.
+template <bool BF16_IN>
+__global__ void __launch_bounds__(256) transpose_rows_kernel(const void *src, __nv_bfloat16 *dst, int64_t rows, int C,
+                                                             int64_t ld_dst, const int32_t *row_e,
+                                                             const int32_t *offsets, const int32_t *kpad)
+{
+    pdl_enter();
+    __shared__ float tile[32][33];
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 32;
+    const int c0 = blockIdx.x * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 8 rows of 32 per pass
+    for (int i = ty; i < 32; i += 8) {
+        const int64_t r = r0 + i;
+        const int c = c0 + tx;
+        float v = 0.f;
+        if (r < rows && c < C) {
+            v = BF16_IN ? __bfloat162float(static_cast<const __nv_bfloat16 *>(src)[r * C + c])
+                        : static_cast<const float *>(src)[r * C + c];
+        }
+        tile[i][tx] = v;
+    }
+    __syncthreads();
+    for (int i = ty; i < 32; i += 8) {
+        const int c = c0 + i;
+        const int64_t r = r0 + tx;
+        if (r < rows && c < C) {
+            const int e = row_e[r];
+            const int64_t col = kpad[e] + (r - offsets[e]);
+            dst[static_cast<int64_t>(c) * ld_dst + col] = __float2bfloat16_rn(tile[tx][i]);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) transpose_weights_kernel(const __nv_bfloat16 *src, __nv_bfloat16 *dst, int R,
+                                                                int C, int64_t ld_dst, int col0)
+{
+    pdl_enter();
+    __shared__ __nv_bfloat16 tile[32][34];
+    const int e = blockIdx.z;
+    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    const __nv_bfloat16 *s = src + static_cast<int64_t>(e) * R * C;
+    __nv_bfloat16 *d = dst + static_cast<int64_t>(e) * C * ld_dst;
+    for (int i = ty; i < 32; i += 8) {
+        const int r = r0 + i, c = c0 + tx;
+        if (r < R && c < C) tile[i][tx] = s[static_cast<int64_t>(r) * C + c];
+    }
+    __syncthreads();
+    for (int i = ty; i < 32; i += 8) {
+        const int c = c0 + i, r = r0 + tx;
+        if (r < R && c < C) d[static_cast<int64_t>(c) * ld_dst + col0 + r] = tile[tx][i];
+    }
+}
+
+__global__ void to_bf16_cat_kernel(const float *a, const float *b, __nv_bfloat16 *dst, int64_t rows, int F)
+{
+    pdl_enter();
+    const int W = b ? 2 * F : F;
+    const int64_t total = rows * W;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = i / W;
+        const int c = static_cast<int>(i - r * W);
+        const float v = c < F ? a[r * F + c] : b[r * F + (c - F)];
+        dst[i] = __float2bfloat16_rn(v);
+    }
+}
+
 int grid_for(int64_t work, int per_block, int num_sms)
 {
     const int64_t want = (work + per_block - 1) / per_block;
@@ -228,6 +310,42 @@ int grid_for(int64_t work, int per_block, int num_sms)
 }
 
 }  // namespace
+
+cudaError_t launch_pad_offsets(const int32_t *counts, int32_t *kpad, int E, cudaStream_t s)
+{
+    return launch_k(pad_offsets_kernel, dim3(1), dim3(32), 0, s, counts, kpad, E);
+}
+
+cudaError_t launch_transpose_rows(const void *src, int src_bf16, __nv_bfloat16 *dst, int64_t rows, int C,
+                                  int64_t ld_dst, const int32_t *row_e, const int32_t *offsets,
+                                  const int32_t *kpad, cudaStream_t s)
+{
+    if (rows == 0 || C == 0) return cudaSuccess;
+    const dim3 grid(static_cast<unsigned>((C + 31) / 32), static_cast<unsigned>((rows + 31) / 32));
+    if (src_bf16)
+        return launch_k(transpose_rows_kernel<true>, grid, dim3(256), 0, s, src, dst, rows, C, ld_dst, row_e, offsets,
+                        kpad);
+    return launch_k(transpose_rows_kernel<false>, grid, dim3(256), 0, s, src, dst, rows, C, ld_dst, row_e, offsets,
+                    kpad);
+}
+
+cudaError_t launch_transpose_weights(const void *src, __nv_bfloat16 *dst, int E, int R, int C, int64_t ld_dst,
+                                     int col0, cudaStream_t s)
+{
+    const dim3 grid(static_cast<unsigned>((C + 31) / 32), static_cast<unsigned>((R + 31) / 32),
+                    static_cast<unsigned>(E));
+    return launch_k(transpose_weights_kernel, grid, dim3(256), 0, s, static_cast<const __nv_bfloat16 *>(src), dst, R,
+                    C, ld_dst, col0);
+}
+
+cudaError_t launch_to_bf16_cat(const float *a, const float *b, __nv_bfloat16 *dst, int64_t rows, int F,
+                               cudaStream_t s)
+{
+    if (rows == 0) return cudaSuccess;
+    const int64_t total = rows * (b ? 2 * F : F);
+    const int grid = static_cast<int>(min64((total + 255) / 256, 148 * 16));
+    return launch_k(to_bf16_cat_kernel, dim3(grid), dim3(256), 0, s, a, b, dst, rows, F);
+}
 
 cudaError_t launch_rows_prep(const BwdRowsArgs &a, int num_sms, cudaStream_t s)
 {

@@ -54,7 +54,7 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 
-enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_LINEAR = 2 };
+enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_LINEAR = 2, EPI_F32 = 3 };
 
 struct GemmArgs {
     const int32_t *offsets;
@@ -64,6 +64,14 @@ struct GemmArgs {
     const __nv_bfloat16 *bias;  // [E, n_out] or null
     int32_t *status;
     int E, K, n_out, n_tiles, b_rows;
+    // EPI_F32: plain fp32 stores to out_f32 (the backward's products)
+    float *out_f32;
+    // ragged_k: the reduction of expert e runs over columns offsets[e] ..
+    // offsets[e+1]-1 of A and B (multiples of BK, zero-padded); A rows are
+    // the m_total result rows (m_tiles tiles of BM), B rows the n_out result
+    // columns; expert e's result starts at out_f32 + e * c_stride
+    int ragged_k, m_tiles;
+    int64_t m_total, c_stride;
 };
 
 struct Ctl {
@@ -100,10 +108,43 @@ __device__ __forceinline__ Tile decode_tile(int t, const Ctl *c, int E, int n_ti
 
 template <int EPI> __host__ __device__ constexpr int out_cols() { return EPI == EPI_SWIGLU ? 128 : 256; }
 
+// Tile t of either schedule: the forward's ragged-M table, or (ragged_k)
+// experts x m-tiles x n-tiles with m innermost.
+__device__ __forceinline__ Tile tile_of(int t, const Ctl *c, const GemmArgs &g)
+{
+    if (!g.ragged_k) return decode_tile(t, c, g.E, g.n_tiles);
+    const int per = g.m_tiles * g.n_tiles;
+    const int e = t / per, local = t - e * per;
+    return Tile{e, local % g.m_tiles, local / g.m_tiles};
+}
+
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase, int e, int row,
-                                              bool row_ok, int n0)
+                                              bool row_ok, int n0, bool zero = false)
 {
+    if constexpr (EPI == EPI_F32) {
+        // zero: the expert had no rows (no MMA wrote the accumulator)
+        float *orow = g.out_f32 + (g.ragged_k ? static_cast<int64_t>(e) * g.c_stride : 0) +
+                      static_cast<int64_t>(row) * g.ldo;
+#pragma unroll 1
+        for (int c = 0; c < 256; c += 32) {
+            uint32_t acc[32];
+            tmem_ld32(tbase + c, acc);
+            tmem_ld_wait();
+            if (row_ok) {
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const int col = n0 + c + v * 4;
+                    if (col < g.n_out) {  // n_out is a multiple of 4 (16-byte stores)
+                        const uint4 q = zero ? make_uint4(0, 0, 0, 0)
+                                             : make_uint4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+                        st16(orow + col, q);
+                    }
+                }
+            }
+        }
+        return;
+    }
     __nv_bfloat16 *orow = g.out + static_cast<int64_t>(row) * g.ldo;
     const __nv_bfloat16 *brow = g.bias ? g.bias + static_cast<int64_t>(e) * g.n_out : nullptr;
 #pragma unroll 1
@@ -193,15 +234,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int i = threadIdx.x; i <= g.E; i += THREADS) {
         ctl->off[i] = g.offsets[i];
-        ctl->mt[i] = g.mt_prefix[i];
+        ctl->mt[i] = g.mt_prefix ? g.mt_prefix[i] : 0;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
     const uint32_t tmem_base = ctl->tmem_base;
-    const int total = ctl->mt[g.E] * g.n_tiles;
+    const int total = g.ragged_k ? g.E * g.m_tiles * g.n_tiles : ctl->mt[g.E] * g.n_tiles;
     const int num_kb = (g.K + BK - 1) / BK;
+    // k-blocks of a tile and the column they start at
+    auto kblocks = [&](int e) { return g.ragged_k ? (ctl->off[e + 1] - ctl->off[e]) / BK : num_kb; };
+    auto kstart = [&](int e) { return g.ragged_k ? ctl->off[e] : 0; };
 
     if (warp == 0) {
         if (lane == 0) {
@@ -210,10 +254,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t phase = 0, armed = 0, armed_parity = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const Tile ti = decode_tile(t, ctl, g.E, g.n_tiles);
-                const int row0 = ctl->off[ti.e] + ti.m_tile * BM;
-                const int brow = ti.e * g.b_rows + ti.n_tile * out_cols<EPI>();
-                for (int kb = 0; kb < num_kb; ++kb) {
+                const Tile ti = tile_of(t, ctl, g);
+                const int row0 = g.ragged_k ? ti.m_tile * BM : ctl->off[ti.e] + ti.m_tile * BM;
+                const int brow = g.ragged_k ? ti.n_tile * out_cols<EPI>()
+                                            : ti.e * g.b_rows + ti.n_tile * out_cols<EPI>();
+                const int nkb = kblocks(ti.e), k0 = kstart(ti.e);
+                for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort_flag, g.status)) {
                         ok = false;
                         break;
@@ -223,12 +269,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                     mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
                     armed |= 1u << stage;
                     armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-                    tma_load_2d(sA, &tmA, &ctl->full[stage], kb * BK, row0);
+                    tma_load_2d(sA, &tmA, &ctl->full[stage], k0 + kb * BK, row0);
                     if (EPI == EPI_SWIGLU) {
                         tma_load_2d(sB, &tmB, &ctl->full[stage], kb * BK, brow);
                         tma_load_2d(sB + B_BYTES / 2, &tmB3, &ctl->full[stage], kb * BK, brow);
                     } else {
-                        tma_load_2d(sB, &tmB, &ctl->full[stage], kb * BK, brow);
+                        tma_load_2d(sB, &tmB, &ctl->full[stage], k0 + kb * BK, brow);
                     }
                     if (++stage == STAGES) {
                         stage = 0;
@@ -254,7 +300,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (!mbar_wait(&ctl->tempty[buf], tphase ^ 1u, abort_flag, g.status)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-                for (int kb = 0; kb < num_kb; ++kb) {
+                const int nkb = kblocks(tile_of(t, ctl, g).e);
+                for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&ctl->full[stage], phase, abort_flag, g.status)) {
                         ok = false;
                         break;
@@ -296,12 +343,19 @@ __global__ void __launch_bounds__(THREADS, 1)
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&ctl->tfull[buf], tphase, abort_flag, g.status));
             if (!ok) break;
             tc_fence_after();
-            const Tile ti = decode_tile(t, ctl, g.E, g.n_tiles);
-            const int row = ctl->off[ti.e] + ti.m_tile * BM + row_in_tile;
-            const bool row_ok = row < ctl->off[ti.e + 1];
+            const Tile ti = tile_of(t, ctl, g);
+            int row;
+            bool row_ok;
+            if (g.ragged_k) {  // result row m of expert e
+                row = ti.m_tile * BM + row_in_tile;
+                row_ok = row < g.m_total;
+            } else {
+                row = ctl->off[ti.e] + ti.m_tile * BM + row_in_tile;
+                row_ok = row < ctl->off[ti.e + 1];
+            }
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
-            epilogue_tile<EPI>(g, tbase, ti.e, row, row_ok, ti.n_tile * out_cols<EPI>());
+            epilogue_tile<EPI>(g, tbase, ti.e, row, row_ok, ti.n_tile * out_cols<EPI>(), kblocks(ti.e) == 0);
             tc_fence_before();
             mbar_arrive(&ctl->tempty[buf]);
             if (++buf == 2) {
@@ -332,6 +386,30 @@ cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtens
 }
 
 }  // namespace
+
+cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s)
+{
+    if (t.ragged_k ? (t.m_total == 0 || t.n_out == 0) : (t.a_rows == 0 || t.n_out == 0)) return cudaSuccess;
+    CUtensorMap tA, tB;
+    if (!make_tmap_bf16(&tA, t.A, t.a_cols, t.a_rows, BM) || !make_tmap_bf16(&tB, t.B, t.b_cols, t.b_rows, 256))
+        return cudaErrorInvalidValue;
+    GemmArgs g{};
+    g.offsets = t.offsets;
+    g.mt_prefix = t.mt_prefix;
+    g.out_f32 = t.C;
+    g.ldo = t.ldc;
+    g.status = t.status;
+    g.E = t.E;
+    g.K = t.K;
+    g.n_out = t.n_out;
+    g.n_tiles = (t.n_out + 255) / 256;
+    g.b_rows = t.n_out;
+    g.ragged_k = t.ragged_k;
+    g.m_tiles = static_cast<int>((t.m_total + BM - 1) / BM);
+    g.m_total = t.m_total;
+    g.c_stride = t.c_stride;
+    return launch_gemm<EPI_F32>(tA, tB, tB, g, num_sms, s);
+}
 
 cudaError_t launch_ffn_bf16_sm100_single(const FfnArgs &a, int num_sms, cudaEvent_t mid, cudaStream_t s)
 {

@@ -1,6 +1,7 @@
 // kernels.h -- host-side launchers of the MoE kernels (internal to libmoe).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -228,6 +229,21 @@ struct BwdRouterArgs {
 };
 cudaError_t launch_router_backward(const BwdRouterArgs &a, int num_sms, cudaStream_t s);
 
+// Layout helpers of the tensor-core backward (bf16 operands):
+// padded column starts kpad[e] = sum_{e' < e} roundup64(counts[e']);
+cudaError_t launch_pad_offsets(const int32_t *counts, int32_t *kpad, int E, cudaStream_t s);
+// dst[c, kpad[e_r] + r - offsets[e_r]] = src[r, c] (bf16; src fp32 or bf16),
+// dst [C, ld_dst] zero elsewhere (the caller clears it first);
+cudaError_t launch_transpose_rows(const void *src, int src_bf16, __nv_bfloat16 *dst, int64_t rows, int C,
+                                  int64_t ld_dst, const int32_t *row_e, const int32_t *offsets,
+                                  const int32_t *kpad, cudaStream_t s);
+// per expert e: dst[e, c, col0 + r] = src[e, r, c] for src [E, R, C] (bf16);
+cudaError_t launch_transpose_weights(const void *src, __nv_bfloat16 *dst, int E, int R, int C, int64_t ld_dst,
+                                     int col0, cudaStream_t s);
+// dst[r, 0..F) = bf16(a[r]), dst[r, F..2F) = bf16(b[r]) (b may be null: [rows, F]).
+cudaError_t launch_to_bf16_cat(const float *a, const float *b, __nv_bfloat16 *dst, int64_t rows, int F,
+                               cudaStream_t s);
+
 struct FfnArgs {
     const void *x_sorted;      // [rows, d]
     const int32_t *offsets;    // [E+1]
@@ -249,6 +265,28 @@ namespace moe {
 // TMA descriptor of a bf16 matrix [outer, inner] (inner contiguous) with a
 // box of [box_outer, 64] elements, 128-byte swizzle, zero fill outside.
 bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_outer);
+
+// C (fp32) = A B^T on tcgen05 with bf16 operands, both K-major (the
+// backward's products on the tensor cores), 128 x 256 tiles:
+//   ragged_k = 0: rows offsets[e] .. offsets[e+1]-1 of A and C belong to
+//     expert e (mt_prefix: its 128-row tile prefix), B = [E * n_out, K];
+//   ragged_k = 1: expert e's result (m_total x n_out, at C + e * c_stride)
+//     sums columns offsets[e] .. offsets[e+1]-1 of A [m_total, cols] and
+//     B [n_out, cols]; the offsets are multiples of 64 and the columns
+//     between an expert's rows and the next offset are zero.
+struct TcGemmArgs {
+    const void *A;
+    uint64_t a_rows, a_cols;
+    const void *B;
+    uint64_t b_rows, b_cols;
+    float *C;
+    int64_t ldc, c_stride;
+    const int32_t *offsets, *mt_prefix;
+    int E, ragged_k, K, n_out;
+    int64_t m_total;
+    int32_t *status;
+};
+cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s);
 
 // Both expert GEMMs; `mid` (may be null) is recorded between them.
 // CTA pairs, 256-row m-tiles:

@@ -251,8 +251,19 @@ cudaError_t launch_shared(const moe_config *c, const moe_shared_expert *sh, cons
 
 struct BwdLayout {
     size_t hist, logits, offsets, mt64, counts, ids, w, perm, inv, probs, lse, xs, dys, row_tok, row_e, row_w,
-        pre, up, h, dh, dxs, dw, dz, doff, dmt, one, spre, sup, sh, sdh, total;
+        pre, up, h, dh, dxs, dw, dz, doff, dmt, one, spre, sup, sh, sdh;
+    // bf16 path (tensor cores): 128-row tile prefix, padded column starts,
+    // transposed weights, the bf16 [da | du], transposed activations
+    size_t mt128, kpad, w2t, wcat, dacat, dysT, xsT, hwT, daT, duT, total;
+    int64_t kp;  // columns of the transposed activations
 };
+
+// Columns of the transposed, per-expert padded activations: every expert's
+// rows rounded up to 64.
+int64_t bwd_kp(const moe_config *c)
+{
+    return (c->N * c->k + 64LL * c->E + 63) / 64 * 64;
+}
 
 BwdLayout bwd_layout(const moe_config *c)
 {
@@ -301,6 +312,20 @@ BwdLayout bwd_layout(const moe_config *c)
     L.sup = take(swiglu ? Nn * Fs * 4 : 0);
     L.sh = take(Nn * Fs * 4);
     L.sdh = take(Nn * Fs * 4);
+    const bool tc = c->dtype == MOE_BF16;
+    const size_t m = swiglu ? 2 : 1;
+    L.kp = bwd_kp(c);
+    const size_t kp = static_cast<size_t>(L.kp);
+    L.mt128 = take((E + 1) * 4);
+    L.kpad = take((E + 1) * 4);
+    L.w2t = take(tc ? E * F * d * 2 : 0);
+    L.wcat = take(tc ? E * d * m * F * 2 : 0);
+    L.dacat = take(tc ? A * m * F * 2 : 0);
+    L.dysT = take(tc ? d * kp * 2 : 0);
+    L.xsT = take(tc ? d * kp * 2 : 0);
+    L.hwT = take(tc ? F * kp * 2 : 0);
+    L.daT = take(tc ? F * kp * 2 : 0);
+    L.duT = take(tc && swiglu ? F * kp * 2 : 0);
     L.total = o;
     return L;
 }
@@ -733,37 +758,94 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
     GatherArgs gd{dy, inv, dys, N, d, k};  // dy_s[r] = dy[token of r]
     MOE_TRY(launch_gather(cfg->dtype, gd, sms, s));
 
-    // ---- expert pre-activations and h (fp32)
-    MOE_TRY(GG().a(xs, d, 1, bf).b(W1, 1, d, static_cast<int64_t>(F) * d, bf).c(pre, F, 1, 0)
-                .rows(offsets, mt, E, rows, F, d, s));
-    if (swiglu)
-        MOE_TRY(GG().a(xs, d, 1, bf).b(W3, 1, d, static_cast<int64_t>(F) * d, bf).c(up, F, 1, 0)
-                    .rows(offsets, mt, E, rows, F, d, s));
     BwdActArgs act{rows, F, d, cfg->act, bf ? 1 : 0, pre, up, h, dh, swiglu ? nullptr : b1, b2,
                    at<int32_t>(ws, L.row_e), row_w, dw, perm, dys};
-    MOE_TRY(launch_act_forward(act, sms, s));
-
-    // ---- output side: dh = dy_s W2[e]; gates, activation backward
-    MOE_TRY(GG().a(dys, d, 1, bf).b(W2, F, 1, static_cast<int64_t>(d) * F, bf).c(dh, F, 1, 0)
-                .rows(offsets, mt, E, rows, F, d, s));
-    MOE_TRY(launch_row_backward(act, sms, s));
-    // dW2[e] = dy_s^T (w h), db2[e] = sum_r w_r dy_s r
-    MOE_TRY(GG().a(dys, 1, d, bf).b(h, F, 1, 0, false).c(gr.dW2, F, 1, static_cast<int64_t>(d) * F)
-                .sum_rows(offsets, E, d, F, s));
+    const int m = swiglu ? 2 : 1;
+    if (bf) {
+        // ---- bf16: every expert product on the tensor cores (fp32 results);
+        // dgrad against transposed weights, wgrad over transposed activations
+        // whose per-expert column blocks start at multiples of 64
+        int32_t *mt128 = at<int32_t>(ws, L.mt128), *kpad = at<int32_t>(ws, L.kpad);
+        auto *w2t = at<__nv_bfloat16>(ws, L.w2t), *wcat = at<__nv_bfloat16>(ws, L.wcat);
+        auto *dacat = at<__nv_bfloat16>(ws, L.dacat);
+        auto *dysT = at<__nv_bfloat16>(ws, L.dysT), *xsT = at<__nv_bfloat16>(ws, L.xsT);
+        auto *hwT = at<__nv_bfloat16>(ws, L.hwT), *daT = at<__nv_bfloat16>(ws, L.daT);
+        auto *duT = swiglu ? at<__nv_bfloat16>(ws, L.duT) : nullptr;
+        const int64_t kp = L.kp;
+        const int32_t *row_e = at<int32_t>(ws, L.row_e);
+        auto ragged_m = [&](const void *A, int64_t K, const void *B, int n_out, float *C) {
+            TcGemmArgs t{};
+            t.A = A; t.a_rows = static_cast<uint64_t>(rows); t.a_cols = static_cast<uint64_t>(K);
+            t.B = B; t.b_rows = static_cast<uint64_t>(E) * n_out; t.b_cols = static_cast<uint64_t>(K);
+            t.C = C; t.ldc = n_out; t.offsets = offsets; t.mt_prefix = mt128; t.E = E; t.K = static_cast<int>(K);
+            t.n_out = n_out; t.status = dev_status;
+            return launch_gemm_tc_f32(t, sms, s);
+        };
+        auto ragged_k = [&](const void *A, int64_t m_total, const void *B, int n_out, float *C) {
+            TcGemmArgs t{};
+            t.A = A; t.a_rows = static_cast<uint64_t>(m_total); t.a_cols = static_cast<uint64_t>(kp);
+            t.B = B; t.b_rows = static_cast<uint64_t>(n_out); t.b_cols = static_cast<uint64_t>(kp);
+            t.C = C; t.ldc = n_out; t.c_stride = m_total * n_out; t.offsets = kpad; t.E = E; t.ragged_k = 1;
+            t.n_out = n_out; t.m_total = m_total; t.status = dev_status;
+            return launch_gemm_tc_f32(t, sms, s);
+        };
+        MOE_TRY(launch_tile_table(offsets, mt128, E, 128, s));
+        MOE_TRY(launch_pad_offsets(counts, kpad, E, s));
+        MOE_TRY(ragged_m(xs, d, W1, F, pre));
+        if (swiglu) MOE_TRY(ragged_m(xs, d, W3, F, up));
+        MOE_TRY(launch_act_forward(act, sms, s));
+        MOE_TRY(launch_transpose_weights(W2, w2t, E, d, F, d, 0, s));  // W2[e]^T: [F, d]
+        MOE_TRY(ragged_m(dys, d, w2t, F, dh));
+        MOE_TRY(launch_row_backward(act, sms, s));
+        // dx_s = [da | du] [W1[e] ; W3[e]]: one product with K = m F
+        MOE_TRY(launch_to_bf16_cat(pre, up, dacat, rows, F, s));
+        MOE_TRY(launch_transpose_weights(W1, wcat, E, F, d, static_cast<int64_t>(m) * F, 0, s));
+        if (swiglu) MOE_TRY(launch_transpose_weights(W3, wcat, E, F, d, 2LL * F, F, s));
+        MOE_TRY(ragged_m(dacat, static_cast<int64_t>(m) * F, wcat, d, dxs));
+        // weight gradients over the transposed, padded activations
+        MOE_TRY(cudaMemsetAsync(dysT, 0, sizeof(__nv_bfloat16) * d * kp, s));
+        MOE_TRY(cudaMemsetAsync(xsT, 0, sizeof(__nv_bfloat16) * d * kp, s));
+        MOE_TRY(cudaMemsetAsync(hwT, 0, sizeof(__nv_bfloat16) * F * kp, s));
+        MOE_TRY(cudaMemsetAsync(daT, 0, sizeof(__nv_bfloat16) * F * kp, s));
+        if (swiglu) MOE_TRY(cudaMemsetAsync(duT, 0, sizeof(__nv_bfloat16) * F * kp, s));
+        MOE_TRY(launch_transpose_rows(dys, 1, dysT, rows, d, kp, row_e, offsets, kpad, s));
+        MOE_TRY(launch_transpose_rows(xs, 1, xsT, rows, d, kp, row_e, offsets, kpad, s));
+        MOE_TRY(launch_transpose_rows(h, 0, hwT, rows, F, kp, row_e, offsets, kpad, s));
+        MOE_TRY(launch_transpose_rows(pre, 0, daT, rows, F, kp, row_e, offsets, kpad, s));
+        if (swiglu) MOE_TRY(launch_transpose_rows(up, 0, duT, rows, F, kp, row_e, offsets, kpad, s));
+        MOE_TRY(ragged_k(dysT, d, hwT, F, gr.dW2));   // dW2[e] = dy_s^T (w h)
+        MOE_TRY(ragged_k(daT, F, xsT, d, gr.dW1));    // dW1[e] = da^T x_s
+        if (swiglu) MOE_TRY(ragged_k(duT, F, xsT, d, gr.dW3));
+    } else {
+        // ---- fp32: the same products on the CUDA cores
+        MOE_TRY(GG().a(xs, d, 1, bf).b(W1, 1, d, static_cast<int64_t>(F) * d, bf).c(pre, F, 1, 0)
+                    .rows(offsets, mt, E, rows, F, d, s));
+        if (swiglu)
+            MOE_TRY(GG().a(xs, d, 1, bf).b(W3, 1, d, static_cast<int64_t>(F) * d, bf).c(up, F, 1, 0)
+                        .rows(offsets, mt, E, rows, F, d, s));
+        MOE_TRY(launch_act_forward(act, sms, s));
+        // output side: dh = dy_s W2[e]; gates, activation backward
+        MOE_TRY(GG().a(dys, d, 1, bf).b(W2, F, 1, static_cast<int64_t>(d) * F, bf).c(dh, F, 1, 0)
+                    .rows(offsets, mt, E, rows, F, d, s));
+        MOE_TRY(launch_row_backward(act, sms, s));
+        // dW2[e] = dy_s^T (w h)
+        MOE_TRY(GG().a(dys, 1, d, bf).b(h, F, 1, 0, false).c(gr.dW2, F, 1, static_cast<int64_t>(d) * F)
+                    .sum_rows(offsets, E, d, F, s));
+        // input side: dx_s = da W1[e] (+ du W3[e]); dW1, dW3
+        MOE_TRY(GG().a(pre, F, 1, false).b(W1, d, 1, static_cast<int64_t>(F) * d, bf).c(dxs, d, 1, 0)
+                    .rows(offsets, mt, E, rows, d, F, s));
+        if (swiglu)
+            MOE_TRY(GG().a(up, F, 1, false).b(W3, d, 1, static_cast<int64_t>(F) * d, bf).c(dxs, d, 1, 0, true)
+                        .rows(offsets, mt, E, rows, d, F, s));
+        MOE_TRY(GG().a(pre, 1, F, false).b(xs, d, 1, 0, bf).c(gr.dW1, d, 1, static_cast<int64_t>(F) * d)
+                    .sum_rows(offsets, E, F, d, s));
+        if (swiglu)
+            MOE_TRY(GG().a(up, 1, F, false).b(xs, d, 1, 0, bf).c(gr.dW3, d, 1, static_cast<int64_t>(F) * d)
+                        .sum_rows(offsets, E, F, d, s));
+    }
+    // bias gradients: db2[e] = sum_r w_r dy_s r, db1[e] = sum_r da_r
     if (b2 && gr.db2)
         MOE_TRY(GG().a(dys, 1, d, bf).b(row_w, 1, 0, 0, false).c(gr.db2, 1, 0, d).sum_rows(offsets, E, d, 1, s));
-
-    // ---- input side: dx_s = da W1[e] (+ du W3[e]); dW1, dW3, db1
-    MOE_TRY(GG().a(pre, F, 1, false).b(W1, d, 1, static_cast<int64_t>(F) * d, bf).c(dxs, d, 1, 0)
-                .rows(offsets, mt, E, rows, d, F, s));
-    if (swiglu)
-        MOE_TRY(GG().a(up, F, 1, false).b(W3, d, 1, static_cast<int64_t>(F) * d, bf).c(dxs, d, 1, 0, true)
-                    .rows(offsets, mt, E, rows, d, F, s));
-    MOE_TRY(GG().a(pre, 1, F, false).b(xs, d, 1, 0, bf).c(gr.dW1, d, 1, static_cast<int64_t>(F) * d)
-                .sum_rows(offsets, E, F, d, s));
-    if (swiglu)
-        MOE_TRY(GG().a(up, 1, F, false).b(xs, d, 1, 0, bf).c(gr.dW3, d, 1, static_cast<int64_t>(F) * d)
-                    .sum_rows(offsets, E, F, d, s));
     if (!swiglu && b1 && gr.db1)
         MOE_TRY(GG().a(pre, 1, F, false).b(one, 0, 0, 0, false).c(gr.db1, 1, 0, F).sum_rows(offsets, E, F, 1, s));
     BwdGatherSumArgs gs{dxs, inv, gr.dx, N, d, k};

@@ -2,7 +2,8 @@
 
 The scalar is <dy, y> + aux_coef L_aux + z_coef L_z (course module sec. 2.1,
 2.3 and 2.4; "nano-moe" router z-loss).  The GPU recomputes the routing with
-the forward's kernels; tokens whose top-k margin is under 1e-4 are replayed
+the forward's kernels (bf16: expert products on the tensor cores, fp32: on
+the CUDA cores); tokens whose top-k margin is under 1e-4 are replayed
 in the oracle with the GPU's choice, as in the forward parity.  Every
 gradient is compared normwise: max |g - r| / max |r| per tensor.
 """
@@ -18,8 +19,10 @@ from parity import MARGIN, config_of, np64
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
-# every product accumulates in fp32 from inputs the oracle sees exactly: errors are fp32 rounding
-TOL_G = {"f32": 1e-5, "bf16": 1e-5}
+# fp32: every product accumulates in fp32 from inputs the oracle sees exactly (errors are fp32
+# rounding).  bf16: the expert products run on the tensor cores, whose operands da, du and w h are
+# rounded to bf16 (2^-9 relative) before the fp32 accumulation.
+TOL_G = {"f32": 1e-5, "bf16": 1e-2}
 
 CASES = {
     "fp32_gelu_bias": (W.WORKLOADS["tiny_fp32"].scaled(N=97, d_model=40, d_ff=48, E=5, k=2, x_std=1.0), 0.3, 0.2),
