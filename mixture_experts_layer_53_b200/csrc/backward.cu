@@ -62,27 +62,69 @@ __global__ void act_forward_kernel(BwdActArgs a)
 }
 
 // One warp per sorted row r, given dh_raw = dy_s W2[e] (the output gradient
-// before the gate weight):
+// before the gate weight), in one pass over the row with 4-float vectors:
 //   dw_r = <dh_raw_r, h_r> + <dy_s r, b2[e]>     (= <dy_n, Expert_e(x_n)>)
 //   dh = w_r dh_raw_r through the activation: pre <- da, up <- du, and
-//   h <- w_r h (the right operand of dW2 = dy_s^T (w h)).
+//   h <- w_r h (the right operand of dW2 = dy_s^T (w h)); with dcat also the
+//   bf16 copies [da | du] that the tensor-core dgrad reads.
 // Without a weight array (the shared expert) w_r = 1 and dw is not kept.
 __global__ void __launch_bounds__(256) row_backward_kernel(BwdActArgs a)
 {
     pdl_enter();
     const int lane = threadIdx.x & 31;
     const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    const bool swiglu = a.act == kSwiglu;
+    const int64_t wcat = swiglu ? 2LL * a.F : a.F;
     for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < a.rows;
          r += warps) {
         const float wr = a.row_w ? a.row_w[r] : 1.0f;
         const int e = a.row_e ? a.row_e[r] : 0;
-        float* pre = a.pre + r * a.F;
-        float* up = a.up ? a.up + r * a.F : nullptr;
-        float* h = a.h + r * a.F;
-        const float* dh = a.dh + r * a.F;
+        float *pre = a.pre + r * a.F;
+        float *up = swiglu ? a.up + r * a.F : nullptr;
+        float *h = a.h + r * a.F;
+        const float *dh = a.dh + r * a.F;
+        float s = 0.f;
+        for (int f = lane * 4; f < a.F; f += 128) {  // F is a multiple of 8
+            const float4 dh4 = *reinterpret_cast<const float4 *>(dh + f);
+            float4 h4 = *reinterpret_cast<const float4 *>(h + f);
+            float4 p4 = *reinterpret_cast<const float4 *>(pre + f);
+            float4 u4 = swiglu ? *reinterpret_cast<const float4 *>(up + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+            float dhv[4] = {dh4.x, dh4.y, dh4.z, dh4.w}, hv[4] = {h4.x, h4.y, h4.z, h4.w};
+            float pv[4] = {p4.x, p4.y, p4.z, p4.w}, uv[4] = {u4.x, u4.y, u4.z, u4.w};
+            float da[4], du[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                s += dhv[q] * hv[q];
+                const float g = wr * dhv[q];
+                const float v = pv[q];
+                if (swiglu) {
+                    const float sg = sigmoidf_(v);
+                    da[q] = g * uv[q] * sg * (1.0f + v * (1.0f - sg));
+                    du[q] = g * v * sg;
+                } else {
+                    const float Phi = 0.5f * (1.0f + erff(v * 0.70710678118654752f));
+                    const float phi = 0.39894228040143268f * expf(-0.5f * v * v);
+                    da[q] = g * (Phi + v * phi);
+                    du[q] = 0.f;
+                }
+                hv[q] *= wr;
+            }
+            *reinterpret_cast<float4 *>(pre + f) = make_float4(da[0], da[1], da[2], da[3]);
+            if (swiglu) *reinterpret_cast<float4 *>(up + f) = make_float4(du[0], du[1], du[2], du[3]);
+            *reinterpret_cast<float4 *>(h + f) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+            if (a.dcat) {
+                __nv_bfloat16 b4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) b4[q] = __float2bfloat16_rn(da[q]);
+                *reinterpret_cast<uint2 *>(a.dcat + r * wcat + f) = *reinterpret_cast<const uint2 *>(b4);
+                if (swiglu) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) b4[q] = __float2bfloat16_rn(du[q]);
+                    *reinterpret_cast<uint2 *>(a.dcat + r * wcat + a.F + f) = *reinterpret_cast<const uint2 *>(b4);
+                }
+            }
+        }
         if (a.dw) {
-            float s = 0.f;
-            for (int f = lane; f < a.F; f += 32) s += dh[f] * h[f];
             if (a.b2) {
                 for (int c = lane; c < a.d; c += 32)
                     s += ldv(a.dy_s, r * a.d + c, a.bf16) * ldv(a.b2, static_cast<int64_t>(e) * a.d + c, a.bf16);
@@ -90,21 +132,6 @@ __global__ void __launch_bounds__(256) row_backward_kernel(BwdActArgs a)
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
             if (lane == 0) a.dw[a.perm[r]] = s;
-        }
-        for (int f = lane; f < a.F; f += 32) {
-            const float g = wr * dh[f];
-            const float v = pre[f];
-            if (a.act == kSwiglu) {
-                const float sg = sigmoidf_(v);
-                const float u = up[f];
-                pre[f] = g * u * sg * (1.0f + v * (1.0f - sg));
-                up[f] = g * v * sg;
-            } else {
-                const float Phi = 0.5f * (1.0f + erff(v * 0.70710678118654752f));
-                const float phi = 0.39894228040143268f * expf(-0.5f * v * v);
-                pre[f] = g * (Phi + v * phi);
-            }
-            h[f] *= wr;
         }
     }
 }
@@ -234,72 +261,88 @@ __global__ void pad_offsets_kernel(const int32_t *counts, int32_t *kpad, int E)
     }
 }
 
-// 32 x 32 tiles through shared memory: coalesced reads along C, writes along
-// the (padded) row positions.
+// Transposes in 64 x 64 tiles through shared memory with 16-byte vectors on
+// both sides.  transpose_rows_kernel walks the padded column space of the
+// result: a 64-column tile lies inside one expert's block (its start kpad[e]
+// is a multiple of 64), so its source rows are contiguous; columns past the
+// expert's rows are written as zeros.
 template <bool BF16_IN>
-__global__ void __launch_bounds__(256) transpose_rows_kernel(const void *src, __nv_bfloat16 *dst, int64_t rows, int C,
-                                                             int64_t ld_dst, const int32_t *row_e,
-                                                             const int32_t *offsets, const int32_t *kpad)
+__global__ void __launch_bounds__(256) transpose_rows_kernel(TransposeRowsArgs a)
 {
     pdl_enter();
-    __shared__ float tile[32][33];
-    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 32;
-    const int c0 = blockIdx.x * 32;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 8 rows of 32 per pass
-    for (int i = ty; i < 32; i += 8) {
+    __shared__ __nv_bfloat16 tile[64][72];
+    const int64_t pc0 = static_cast<int64_t>(blockIdx.y) * 64;  // padded column of the tile
+    if (pc0 >= a.kpad[a.E]) return;                              // block-uniform: past every expert
+    int lo = 0, hi = a.E - 1;                                    // expert whose block holds pc0
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.kpad[mid] <= pc0) lo = mid;
+        else hi = mid - 1;
+    }
+    const int64_t r0 = a.offsets[lo] + (pc0 - a.kpad[lo]);  // first source row
+    const int64_t r_end = a.offsets[lo + 1];
+    const int c0 = blockIdx.x * 64;
+    const int t = threadIdx.x;
+    // load: 64 rows x 64 columns, 8 columns per thread and step
+    for (int idx = t; idx < 64 * 8; idx += 256) {
+        const int i = idx >> 3, cv = (idx & 7) * 8;
         const int64_t r = r0 + i;
-        const int c = c0 + tx;
-        float v = 0.f;
-        if (r < rows && c < C) {
-            v = BF16_IN ? __bfloat162float(static_cast<const __nv_bfloat16 *>(src)[r * C + c])
-                        : static_cast<const float *>(src)[r * C + c];
+        const int c = c0 + cv;
+        float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (r < r_end && c < a.C) {  // C is a multiple of 8
+            if (BF16_IN) {
+                unpack16(*reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.src) + r * a.ld_src + c),
+                         f, static_cast<const __nv_bfloat16 *>(nullptr));
+            } else {
+                const float *p = static_cast<const float *>(a.src) + r * a.ld_src + c;
+                const float4 u = *reinterpret_cast<const float4 *>(p), w = *reinterpret_cast<const float4 *>(p + 4);
+                f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w; f[4] = w.x; f[5] = w.y; f[6] = w.z; f[7] = w.w;
+            }
         }
-        tile[i][tx] = v;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) tile[i][cv + j] = __float2bfloat16_rn(f[j]);
     }
     __syncthreads();
-    for (int i = ty; i < 32; i += 8) {
-        const int c = c0 + i;
-        const int64_t r = r0 + tx;
-        if (r < rows && c < C) {
-            const int e = row_e[r];
-            const int64_t col = kpad[e] + (r - offsets[e]);
-            dst[static_cast<int64_t>(c) * ld_dst + col] = __float2bfloat16_rn(tile[tx][i]);
-        }
+    // store: row c of the result gets 64 consecutive columns, 8 per vector
+    for (int idx = t; idx < 64 * 8; idx += 256) {
+        const int cl = idx >> 3, rv = (idx & 7) * 8;
+        const int c = c0 + cl;
+        if (c >= a.C) continue;
+        __nv_bfloat16 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = tile[rv + j][cl];
+        *reinterpret_cast<uint4 *>(a.dst + static_cast<int64_t>(c) * a.ld_dst + pc0 + rv) =
+            *reinterpret_cast<const uint4 *>(v);
     }
 }
 
+// dst[e, c, col0 + r] = src[e, r, c]; R, C, ld_dst and col0 are multiples of 8.
 __global__ void __launch_bounds__(256) transpose_weights_kernel(const __nv_bfloat16 *src, __nv_bfloat16 *dst, int R,
                                                                 int C, int64_t ld_dst, int col0)
 {
     pdl_enter();
-    __shared__ __nv_bfloat16 tile[32][34];
+    __shared__ __nv_bfloat16 tile[64][72];
     const int e = blockIdx.z;
-    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-    const __nv_bfloat16 *s = src + static_cast<int64_t>(e) * R * C;
-    __nv_bfloat16 *d = dst + static_cast<int64_t>(e) * C * ld_dst;
-    for (int i = ty; i < 32; i += 8) {
-        const int r = r0 + i, c = c0 + tx;
-        if (r < R && c < C) tile[i][tx] = s[static_cast<int64_t>(r) * C + c];
+    const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
+    const int t = threadIdx.x;
+    const __nv_bfloat16 *sp = src + static_cast<int64_t>(e) * R * C;
+    __nv_bfloat16 *dp = dst + static_cast<int64_t>(e) * C * ld_dst;
+    for (int idx = t; idx < 64 * 8; idx += 256) {
+        const int i = idx >> 3, cv = (idx & 7) * 8;
+        const int r = r0 + i, c = c0 + cv;
+        uint4 q = make_uint4(0, 0, 0, 0);
+        if (r < R && c < C) q = *reinterpret_cast<const uint4 *>(sp + static_cast<int64_t>(r) * C + c);
+        *reinterpret_cast<uint4 *>(&tile[i][cv]) = q;
     }
     __syncthreads();
-    for (int i = ty; i < 32; i += 8) {
-        const int c = c0 + i, r = r0 + tx;
-        if (r < R && c < C) d[static_cast<int64_t>(c) * ld_dst + col0 + r] = tile[tx][i];
-    }
-}
-
-__global__ void to_bf16_cat_kernel(const float *a, const float *b, __nv_bfloat16 *dst, int64_t rows, int F)
-{
-    pdl_enter();
-    const int W = b ? 2 * F : F;
-    const int64_t total = rows * W;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t r = i / W;
-        const int c = static_cast<int>(i - r * W);
-        const float v = c < F ? a[r * F + c] : b[r * F + (c - F)];
-        dst[i] = __float2bfloat16_rn(v);
+    for (int idx = t; idx < 64 * 8; idx += 256) {
+        const int cl = idx >> 3, rv = (idx & 7) * 8;
+        const int c = c0 + cl, r = r0 + rv;
+        if (c >= C || r >= R) continue;
+        __nv_bfloat16 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = tile[rv + j][cl];
+        *reinterpret_cast<uint4 *>(dp + static_cast<int64_t>(c) * ld_dst + col0 + r) = *reinterpret_cast<const uint4 *>(v);
     }
 }
 
@@ -316,35 +359,22 @@ cudaError_t launch_pad_offsets(const int32_t *counts, int32_t *kpad, int E, cuda
     return launch_k(pad_offsets_kernel, dim3(1), dim3(32), 0, s, counts, kpad, E);
 }
 
-cudaError_t launch_transpose_rows(const void *src, int src_bf16, __nv_bfloat16 *dst, int64_t rows, int C,
-                                  int64_t ld_dst, const int32_t *row_e, const int32_t *offsets,
-                                  const int32_t *kpad, cudaStream_t s)
+cudaError_t launch_transpose_rows(const TransposeRowsArgs &a, int64_t kp_max, cudaStream_t s)
 {
-    if (rows == 0 || C == 0) return cudaSuccess;
-    const dim3 grid(static_cast<unsigned>((C + 31) / 32), static_cast<unsigned>((rows + 31) / 32));
-    if (src_bf16)
-        return launch_k(transpose_rows_kernel<true>, grid, dim3(256), 0, s, src, dst, rows, C, ld_dst, row_e, offsets,
-                        kpad);
-    return launch_k(transpose_rows_kernel<false>, grid, dim3(256), 0, s, src, dst, rows, C, ld_dst, row_e, offsets,
-                    kpad);
+    if (kp_max == 0 || a.C == 0) return cudaSuccess;
+    if (kp_max / 64 > 65535) return cudaErrorInvalidValue;
+    const dim3 grid(static_cast<unsigned>((a.C + 63) / 64), static_cast<unsigned>(kp_max / 64));
+    if (a.src_bf16) return launch_k(transpose_rows_kernel<true>, grid, dim3(256), 0, s, a);
+    return launch_k(transpose_rows_kernel<false>, grid, dim3(256), 0, s, a);
 }
 
 cudaError_t launch_transpose_weights(const void *src, __nv_bfloat16 *dst, int E, int R, int C, int64_t ld_dst,
                                      int col0, cudaStream_t s)
 {
-    const dim3 grid(static_cast<unsigned>((C + 31) / 32), static_cast<unsigned>((R + 31) / 32),
+    const dim3 grid(static_cast<unsigned>((C + 63) / 64), static_cast<unsigned>((R + 63) / 64),
                     static_cast<unsigned>(E));
     return launch_k(transpose_weights_kernel, grid, dim3(256), 0, s, static_cast<const __nv_bfloat16 *>(src), dst, R,
                     C, ld_dst, col0);
-}
-
-cudaError_t launch_to_bf16_cat(const float *a, const float *b, __nv_bfloat16 *dst, int64_t rows, int F,
-                               cudaStream_t s)
-{
-    if (rows == 0) return cudaSuccess;
-    const int64_t total = rows * (b ? 2 * F : F);
-    const int grid = static_cast<int>(min64((total + 255) / 256, 148 * 16));
-    return launch_k(to_bf16_cat_kernel, dim3(grid), dim3(256), 0, s, a, b, dst, rows, F);
 }
 
 cudaError_t launch_rows_prep(const BwdRowsArgs &a, int num_sms, cudaStream_t s)

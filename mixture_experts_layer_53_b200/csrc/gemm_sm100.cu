@@ -23,9 +23,10 @@
 //              CTA's `full` barrier, which expects both CTAs' bytes)
 //   warp 1     TMEM allocation for the pair (both CTAs); in the even CTA one
 //              lane issues the MMAs and commits to both CTAs' barriers
-//   warps 2-9  epilogue on the CTA's own 128 rows (tcgen05.ld), two warps
-//              per TMEM lane quarter, each on half of the tile's output
-//              columns; fused activation / bias, bf16 stores
+//   warps 2-   epilogue on the CTA's own 128 rows (tcgen05.ld), one or
+//              (GELU) two warps per TMEM lane quarter, the latter each on
+//              half of the tile's output columns; fused activation / bias,
+//              bf16 stores
 // SwiGLU: the even CTA's B half holds 128 rows of W1 and the odd CTA's the
 // same 128 rows of W3, so accumulator columns 0..127 are the gate and
 // 128..255 the up projection of 128 hidden units.
@@ -49,12 +50,17 @@ constexpr int STAGES = 6;
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int B_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's half of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int EPI_WARPS = 8;  // two per TMEM lane quarter, each on half of the columns
-constexpr int THREADS = 64 + 32 * EPI_WARPS;
+// Epilogue warps: one per TMEM lane quarter, or (GELU, whose erf epilogue
+// outlasts a short k-loop) two per quarter, each on half of the columns.
+// More epilogue warps let the pairs run further apart, which costs L2 reuse
+// of the weight tiles: SwiGLU and the linear GEMM keep four.
+template <int EPI> __host__ __device__ constexpr int epi_warps();
+template <int EPI> __host__ __device__ constexpr int threads_of() { return 64 + 32 * epi_warps<EPI>(); }
 constexpr uint32_t TMEM_COLS = 512;
 
 
 enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_LINEAR = 2 };
+template <int EPI> __host__ __device__ constexpr int epi_warps() { return EPI == EPI_GELU ? 8 : 4; }
 
 struct GemmArgs {
     const int32_t *offsets;
@@ -158,7 +164,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &g, uint32_t tbase,
 }
 
 template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmB3, const GemmArgs g)
 {
@@ -179,7 +185,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->tfull[b], 1);
-            mbar_init(&ctl->tempty[b], 2 * EPI_WARPS);  // every epilogue warp of both CTAs
+            mbar_init(&ctl->tempty[b], 2 * epi_warps<EPI>());  // every epilogue warp of both CTAs
         }
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
@@ -194,7 +200,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
         tmem_relinquish_pair();
     }
-    for (int i = threadIdx.x; i <= g.E; i += THREADS) {
+    for (int i = threadIdx.x; i <= g.E; i += threads_of<EPI>()) {
         ctl->off[i] = g.offsets[i];
         ctl->mt[i] = g.mt_prefix[i];
     }
@@ -298,7 +304,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     } else {
         // ---------------------------------------------------- epilogue
         const int quarter = warp & 3;  // TMEM lanes this warp may access
-        const int half = (warp - 2) / 4;  // which half of the output columns
+        constexpr int parts = epi_warps<EPI>() / 4;  // warps per TMEM lane quarter
+        const int part = (warp - 2) / 4;            // which part of the output columns
         const int row_in_cta = quarter * 32 + lane;
         const uint32_t tempty_leader0 = mapa_shared(smem_u32(&ctl->tempty[0]), 0);
         const uint32_t tempty_leader1 = mapa_shared(smem_u32(&ctl->tempty[1]), 0);
@@ -313,8 +320,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const bool row_ok = row < ctl->off[ti.e + 1];
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
-            epilogue_rows<EPI>(g, tbase, ti.e, row, row_ok, ti.n_tile * out_cols<EPI>(), half * out_cols<EPI>() / 2,
-                               (half + 1) * out_cols<EPI>() / 2);
+            epilogue_rows<EPI>(g, tbase, ti.e, row, row_ok, ti.n_tile * out_cols<EPI>(),
+                               part * out_cols<EPI>() / parts, (part + 1) * out_cols<EPI>() / parts);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
@@ -343,7 +350,7 @@ cudaError_t launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtens
                                        static_cast<int>(kSmemBytes));
     if (err != cudaSuccess) return err;
     const int grid = (num_sms / 2) * 2;
-    return launch_k(ffn_gemm_pair_kernel<EPI>, dim3(grid), dim3(THREADS), kSmemBytes, s, a, b, b3, g);
+    return launch_k(ffn_gemm_pair_kernel<EPI>, dim3(grid), dim3(threads_of<EPI>()), kSmemBytes, s, a, b, b3, g);
 }
 
 }  // namespace

@@ -204,6 +204,7 @@ struct BwdActArgs {
     float *dw;             // [N k] or null: <dy_n, Expert(x_n)> per assignment
     const int32_t *perm;   // [rows] (with dw)
     const void *dy_s;      // [rows, d] (with dw and b2)
+    __nv_bfloat16 *dcat;   // [rows, m F] or null: bf16 copies [da | du] (the tensor-core dgrad operand)
 };
 cudaError_t launch_act_forward(const BwdActArgs &a, int num_sms, cudaStream_t s);
 cudaError_t launch_row_backward(const BwdActArgs &a, int num_sms, cudaStream_t s);
@@ -232,17 +233,23 @@ cudaError_t launch_router_backward(const BwdRouterArgs &a, int num_sms, cudaStre
 // Layout helpers of the tensor-core backward (bf16 operands):
 // padded column starts kpad[e] = sum_{e' < e} roundup64(counts[e']);
 cudaError_t launch_pad_offsets(const int32_t *counts, int32_t *kpad, int E, cudaStream_t s);
-// dst[c, kpad[e_r] + r - offsets[e_r]] = src[r, c] (bf16; src fp32 or bf16),
-// dst [C, ld_dst] zero elsewhere (the caller clears it first);
-cudaError_t launch_transpose_rows(const void *src, int src_bf16, __nv_bfloat16 *dst, int64_t rows, int C,
-                                  int64_t ld_dst, const int32_t *row_e, const int32_t *offsets,
-                                  const int32_t *kpad, cudaStream_t s);
+// dst[c, kpad[e] + r - offsets[e]] = src[r, c] for the rows r of expert e
+// (bf16; src fp32 or bf16 with row stride ld_src), and zeros in
+// dst[c, kpad[e] + count_e .. kpad[e+1]); columns from kpad[E] on are not
+// written.  kp_max: an upper bound of kpad[E] (a multiple of 64).
+struct TransposeRowsArgs {
+    const void *src;
+    int src_bf16;
+    int64_t ld_src;
+    __nv_bfloat16 *dst;
+    int64_t ld_dst;
+    int C, E;
+    const int32_t *offsets, *kpad;
+};
+cudaError_t launch_transpose_rows(const TransposeRowsArgs &a, int64_t kp_max, cudaStream_t s);
 // per expert e: dst[e, c, col0 + r] = src[e, r, c] for src [E, R, C] (bf16);
 cudaError_t launch_transpose_weights(const void *src, __nv_bfloat16 *dst, int E, int R, int C, int64_t ld_dst,
                                      int col0, cudaStream_t s);
-// dst[r, 0..F) = bf16(a[r]), dst[r, F..2F) = bf16(b[r]) (b may be null: [rows, F]).
-cudaError_t launch_to_bf16_cat(const float *a, const float *b, __nv_bfloat16 *dst, int64_t rows, int F,
-                               cudaStream_t s);
 
 struct FfnArgs {
     const void *x_sorted;      // [rows, d]

@@ -759,7 +759,7 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
     MOE_TRY(launch_gather(cfg->dtype, gd, sms, s));
 
     BwdActArgs act{rows, F, d, cfg->act, bf ? 1 : 0, pre, up, h, dh, swiglu ? nullptr : b1, b2,
-                   at<int32_t>(ws, L.row_e), row_w, dw, perm, dys};
+                   at<int32_t>(ws, L.row_e), row_w, dw, perm, dys, nullptr};
     const int m = swiglu ? 2 : 1;
     if (bf) {
         // ---- bf16: every expert product on the tensor cores (fp32 results);
@@ -772,7 +772,6 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
         auto *hwT = at<__nv_bfloat16>(ws, L.hwT), *daT = at<__nv_bfloat16>(ws, L.daT);
         auto *duT = swiglu ? at<__nv_bfloat16>(ws, L.duT) : nullptr;
         const int64_t kp = L.kp;
-        const int32_t *row_e = at<int32_t>(ws, L.row_e);
         auto ragged_m = [&](const void *A, int64_t K, const void *B, int n_out, float *C) {
             TcGemmArgs t{};
             t.A = A; t.a_rows = static_cast<uint64_t>(rows); t.a_cols = static_cast<uint64_t>(K);
@@ -796,23 +795,22 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
         MOE_TRY(launch_act_forward(act, sms, s));
         MOE_TRY(launch_transpose_weights(W2, w2t, E, d, F, d, 0, s));  // W2[e]^T: [F, d]
         MOE_TRY(ragged_m(dys, d, w2t, F, dh));
+        act.dcat = dacat;  // [da | du] in bf16 as well
         MOE_TRY(launch_row_backward(act, sms, s));
         // dx_s = [da | du] [W1[e] ; W3[e]]: one product with K = m F
-        MOE_TRY(launch_to_bf16_cat(pre, up, dacat, rows, F, s));
         MOE_TRY(launch_transpose_weights(W1, wcat, E, F, d, static_cast<int64_t>(m) * F, 0, s));
         if (swiglu) MOE_TRY(launch_transpose_weights(W3, wcat, E, F, d, 2LL * F, F, s));
         MOE_TRY(ragged_m(dacat, static_cast<int64_t>(m) * F, wcat, d, dxs));
         // weight gradients over the transposed, padded activations
-        MOE_TRY(cudaMemsetAsync(dysT, 0, sizeof(__nv_bfloat16) * d * kp, s));
-        MOE_TRY(cudaMemsetAsync(xsT, 0, sizeof(__nv_bfloat16) * d * kp, s));
-        MOE_TRY(cudaMemsetAsync(hwT, 0, sizeof(__nv_bfloat16) * F * kp, s));
-        MOE_TRY(cudaMemsetAsync(daT, 0, sizeof(__nv_bfloat16) * F * kp, s));
-        if (swiglu) MOE_TRY(cudaMemsetAsync(duT, 0, sizeof(__nv_bfloat16) * F * kp, s));
-        MOE_TRY(launch_transpose_rows(dys, 1, dysT, rows, d, kp, row_e, offsets, kpad, s));
-        MOE_TRY(launch_transpose_rows(xs, 1, xsT, rows, d, kp, row_e, offsets, kpad, s));
-        MOE_TRY(launch_transpose_rows(h, 0, hwT, rows, F, kp, row_e, offsets, kpad, s));
-        MOE_TRY(launch_transpose_rows(pre, 0, daT, rows, F, kp, row_e, offsets, kpad, s));
-        if (swiglu) MOE_TRY(launch_transpose_rows(up, 0, duT, rows, F, kp, row_e, offsets, kpad, s));
+        auto tr = [&](const void *src, int bf_in, int64_t ld_src, __nv_bfloat16 *dst, int C) {
+            TransposeRowsArgs t{src, bf_in, ld_src, dst, kp, C, E, offsets, kpad};
+            return launch_transpose_rows(t, kp, s);
+        };
+        MOE_TRY(tr(dys, 1, d, dysT, d));
+        MOE_TRY(tr(xs, 1, d, xsT, d));
+        MOE_TRY(tr(h, 0, F, hwT, F));
+        MOE_TRY(tr(dacat, 1, static_cast<int64_t>(m) * F, daT, F));
+        if (swiglu) MOE_TRY(tr(dacat + F, 1, 2LL * F, duT, F));
         MOE_TRY(ragged_k(dysT, d, hwT, F, gr.dW2));   // dW2[e] = dy_s^T (w h)
         MOE_TRY(ragged_k(daT, F, xsT, d, gr.dW1));    // dW1[e] = da^T x_s
         if (swiglu) MOE_TRY(ragged_k(duT, F, xsT, d, gr.dW3));
@@ -866,7 +864,7 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
         if (swiglu)
             MOE_TRY(GG().a(x, d, 1, bf).b(shared->W3, 1, d, 0, bf).c(sup, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
         BwdActArgs sa{N, Fs, d, cfg->act, bf ? 1 : 0, spre, sup, sh, sdh, swiglu ? nullptr : shared->b1, nullptr,
-                      nullptr, nullptr, nullptr, nullptr, nullptr};
+                      nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
         MOE_TRY(launch_act_forward(sa, sms, s));
         MOE_TRY(GG().a(dy, d, 1, bf).b(shared->W2, Fs, 1, 0, bf).c(sdh, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
         MOE_TRY(launch_row_backward(sa, sms, s));
