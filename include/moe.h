@@ -365,7 +365,11 @@ MOE_API size_t moe_backward_workspace_size(const moe_config *cfg);
  * router through dL_aux / dp_{n,e} = E f_e / N (course module sec. 2.3),
  * the z-loss through 2 lse(z_n) p_n / N.  The routing and the
  * expert pre-activations are recomputed (same kernels as the forward, so the
- * same expert choice); all products accumulate in fp32.  Enqueues only.
+ * same expert choice); all products accumulate in fp32.  bf16: the expert
+ * products run on the tensor cores, with the intermediate gradients (da,
+ * du, w h) rounded to bf16 as operands; fp32: on the CUDA cores throughout.
+ * Workspace: moe_backward_workspace_size(cfg) bytes (it holds transposed
+ * copies of the expert weights and activations).  Enqueues only.
  */
 MOE_API moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g,
                         const float *b_e, const void *W1, const void *b1,
