@@ -379,6 +379,16 @@ MOE_API moe_status moe_backward(const moe_config *cfg, const void *x, const void
                         int32_t *dev_status, void *ws, size_t ws_bytes,
                         moe_stream_t stream);
 
+/*
+ * Failure-detection check (the pages have no counterpart): launches one CTA
+ * that waits on an mbarrier nothing ever arrives at, through the same
+ * bounded wait every tcgen05 kernel of the library uses.  After the wait
+ * limit (2 s of %globaltimer) the kernel writes MOE_ERR_TIMEOUT to
+ * *dev_status (cleared first) and returns; the context stays usable.
+ * Enqueues only: synchronise the stream, then read *dev_status.
+ */
+MOE_API moe_status moe_selftest_wait_timeout(int32_t *dev_status, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -37,7 +37,7 @@ STAGE_NAMES = ("route", "dispatch", "gemm1", "gemm2", "combine")
 EXPORTS = ("moe_status_string", "moe_last_error", "moe_version", "moe_workspace_size", "moe_route",
            "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_combine", "moe_aux_loss",
            "moe_forward", "moe_shared_ffn", "moe_combine_shared", "moe_router_z_loss", "moe_forward_ex",
-           "moe_backward_workspace_size", "moe_backward")
+           "moe_backward_workspace_size", "moe_backward", "moe_selftest_wait_timeout")
 # ceil(N / 32) * E limit of moe_dispatch_noalloc (MOE_NOALLOC_DISPATCH_MAX_SLOTS)
 NOALLOC_DISPATCH_MAX_SLOTS = 1 << 19
 
@@ -127,6 +127,8 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_backward.argtypes = [cfgp, vp, vp, f32p, vp, vp, vp, vp, vp, shp, vp, ctypes.c_float, ctypes.c_float,
                                  ctypes.POINTER(MoeGrads), i32p, vp, sz, vp]
     lib.moe_backward.restype = st
+    lib.moe_selftest_wait_timeout.argtypes = [i32p, vp]
+    lib.moe_selftest_wait_timeout.restype = st
     if path is None:
         _lib = lib
     return lib
@@ -353,6 +355,16 @@ def moe_backward(cfg: MoeConfig, x: torch.Tensor, W_g: torch.Tensor, W1: torch.T
                                 _stream(stream))
     _check(rc, "moe_backward")
     return out
+
+
+def moe_selftest_wait_timeout(stream=None) -> int:
+    """Runs the library's bounded device wait on a barrier nothing arrives at
+    and returns the status word it leaves (5, MOE_ERR_TIMEOUT); synchronises."""
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = library().moe_selftest_wait_timeout(_ptr(st), _stream(stream))
+    _check(rc, "moe_selftest_wait_timeout")
+    torch.cuda.synchronize()
+    return int(st[0])
 
 
 class StageEvents:
