@@ -38,26 +38,36 @@ __global__ void rows_prep_kernel(BwdRowsArgs a)
     }
 }
 
-// Pre-activations a (+ b1 for GELU) and the hidden activations h.
+// Pre-activations a (+ b1 for GELU) and the hidden activations h, four
+// elements per thread (F is a multiple of 8).
 __global__ void act_forward_kernel(BwdActArgs a)
 {
     pdl_enter();
-    const int64_t total = a.rows * a.F;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t r = i / a.F;
-        const int f = static_cast<int>(i - r * a.F);
-        float v = a.pre[i];
-        if (a.act == kSwiglu) {
-            a.h[i] = silu(v) * a.up[i];
+    const int64_t total4 = a.rows * a.F / 4;
+    const bool swiglu = a.act == kSwiglu;
+    for (int64_t i4 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i4 < total4;
+         i4 += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t i = i4 * 4;
+        float4 p = *reinterpret_cast<const float4 *>(a.pre + i);
+        float v[4] = {p.x, p.y, p.z, p.w}, h[4];
+        if (swiglu) {
+            const float4 u = *reinterpret_cast<const float4 *>(a.up + i);
+            const float uv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) h[q] = silu(v[q]) * uv[q];
         } else {
             if (a.b1) {
+                const int64_t r = i / a.F;
+                const int f = static_cast<int>(i - r * a.F);
                 const int e = a.row_e ? a.row_e[r] : 0;
-                v += ldv(a.b1, static_cast<int64_t>(e) * a.F + f, a.bf16);
-                a.pre[i] = v;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) v[q] += ldv(a.b1, static_cast<int64_t>(e) * a.F + f + q, a.bf16);
+                *reinterpret_cast<float4 *>(a.pre + i) = make_float4(v[0], v[1], v[2], v[3]);
             }
-            a.h[i] = gelu_erf(v);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) h[q] = gelu_erf(v[q]);
         }
+        *reinterpret_cast<float4 *>(a.h + i) = make_float4(h[0], h[1], h[2], h[3]);
     }
 }
 
@@ -385,7 +395,7 @@ cudaError_t launch_rows_prep(const BwdRowsArgs &a, int num_sms, cudaStream_t s)
 cudaError_t launch_act_forward(const BwdActArgs &a, int num_sms, cudaStream_t s)
 {
     if (a.rows == 0) return cudaSuccess;
-    return launch_k(act_forward_kernel, dim3(grid_for(a.rows * a.F, 256, num_sms)), dim3(256), 0, s, a);
+    return launch_k(act_forward_kernel, dim3(grid_for(a.rows * a.F / 4, 256, num_sms)), dim3(256), 0, s, a);
 }
 
 cudaError_t launch_row_backward(const BwdActArgs &a, int num_sms, cudaStream_t s)

@@ -38,12 +38,19 @@ __global__ void __launch_bounds__(THREADS) gemm_generic_kernel(GenericGemmArgs g
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;  // rows ty*4.., cols tx*4..
     int grp;
     int64_t m0, m_end, k_lo, k_hi;
+    int split = 0;
     if (g.ragged_k) {
-        grp = blockIdx.z;
+        grp = blockIdx.z / g.ksplit;
+        split = blockIdx.z - grp * g.ksplit;
         m0 = static_cast<int64_t>(blockIdx.x) * TM;
         m_end = g.M;
         k_lo = g.offsets[grp];
         k_hi = g.offsets[grp + 1];
+        if (g.ksplit > 1) {  // this CTA's share of the reduction, whole k-chunks
+            const int64_t chunk = ((k_hi - k_lo + g.ksplit - 1) / g.ksplit + TK - 1) / TK * TK;
+            k_lo = min64(k_hi, k_lo + split * chunk);
+            k_hi = min64(k_hi, k_lo + chunk);
+        }
     } else {
         // tile -> (group, m-tile) through the per-group tile prefix
         const int t = blockIdx.x;
@@ -62,7 +69,12 @@ __global__ void __launch_bounds__(THREADS) gemm_generic_kernel(GenericGemmArgs g
     }
     const int64_t n0 = static_cast<int64_t>(blockIdx.y) * TN;
     const int64_t boff = static_cast<int64_t>(grp) * g.sbg;
-    float *C = g.C + static_cast<int64_t>(grp) * g.scg;
+    // split reductions write dense partials [G * ksplit][M][N], summed in
+    // split order by split_reduce_kernel
+    const bool partial = g.ragged_k && g.ksplit > 1;
+    float *C = partial ? g.partial + (static_cast<int64_t>(grp) * g.ksplit + split) * g.M * g.N
+                       : g.C + static_cast<int64_t>(grp) * g.scg;
+    const int64_t scm = partial ? g.N : g.scm, scn = partial ? 1 : g.scn;
 
     float acc[4][4];
 #pragma unroll
@@ -104,9 +116,25 @@ __global__ void __launch_bounds__(THREADS) gemm_generic_kernel(GenericGemmArgs g
         for (int j = 0; j < 4; ++j) {
             const int64_t n = n0 + tx * 4 + j;
             if (n >= g.N) continue;
-            float *cp = C + m * g.scm + n * g.scn;
-            *cp = g.accumulate ? *cp + acc[i][j] : acc[i][j];
+            float *cp = C + m * scm + n * scn;
+            *cp = (g.accumulate && !partial) ? *cp + acc[i][j] : acc[i][j];
         }
+    }
+}
+
+// C_g(m, n) (+)= sum over splits, in split order.
+__global__ void __launch_bounds__(256) split_reduce_kernel(GenericGemmArgs g)
+{
+    pdl_enter();
+    const int64_t total = static_cast<int64_t>(g.G) * g.M * g.N;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t grp = i / (g.M * g.N), mn = i - grp * g.M * g.N;
+        const int64_t m = mn / g.N, n = mn - m * g.N;
+        float s = 0.f;
+        for (int sp = 0; sp < g.ksplit; ++sp) s += g.partial[(grp * g.ksplit + sp) * g.M * g.N + mn];
+        float *cp = g.C + grp * g.scg + m * g.scm + n * g.scn;
+        *cp = g.accumulate ? *cp + s : s;
     }
 }
 
@@ -116,13 +144,18 @@ cudaError_t launch_gemm_generic(const GenericGemmArgs &g, int64_t max_tiles_m, c
 {
     dim3 grid;
     if (g.ragged_k) grid = dim3(static_cast<unsigned>((g.M + TM - 1) / TM), static_cast<unsigned>((g.N + TN - 1) / TN),
-                                static_cast<unsigned>(g.G));
+                                static_cast<unsigned>(g.G * max(g.ksplit, 1)));
     else grid = dim3(static_cast<unsigned>(max_tiles_m), static_cast<unsigned>((g.N + TN - 1) / TN), 1);
     if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
-    if (g.a_bf16 && g.b_bf16) return launch_k(gemm_generic_kernel<true, true>, grid, dim3(THREADS), 0, s, g);
-    if (g.a_bf16) return launch_k(gemm_generic_kernel<true, false>, grid, dim3(THREADS), 0, s, g);
-    if (g.b_bf16) return launch_k(gemm_generic_kernel<false, true>, grid, dim3(THREADS), 0, s, g);
-    return launch_k(gemm_generic_kernel<false, false>, grid, dim3(THREADS), 0, s, g);
+    cudaError_t err;
+    if (g.a_bf16 && g.b_bf16) err = launch_k(gemm_generic_kernel<true, true>, grid, dim3(THREADS), 0, s, g);
+    else if (g.a_bf16) err = launch_k(gemm_generic_kernel<true, false>, grid, dim3(THREADS), 0, s, g);
+    else if (g.b_bf16) err = launch_k(gemm_generic_kernel<false, true>, grid, dim3(THREADS), 0, s, g);
+    else err = launch_k(gemm_generic_kernel<false, false>, grid, dim3(THREADS), 0, s, g);
+    if (err != cudaSuccess || !g.ragged_k || g.ksplit <= 1) return err;
+    const int64_t total = static_cast<int64_t>(g.G) * g.M * g.N;
+    const int rgrid = static_cast<int>(min64((total + 255) / 256, 148 * 8));
+    return launch_k(split_reduce_kernel, dim3(rgrid), dim3(256), 0, s, g);
 }
 
 }  // namespace moe

@@ -177,8 +177,13 @@ struct GenericGemmArgs {
     int ragged_k;
     int64_t M, N, K;
     int accumulate, a_bf16, b_bf16;
+    // ragged_k only: split each reduction ksplit ways (> 1: dense partials
+    // [G * ksplit][M][N] in `partial`, then summed in split order)
+    int ksplit;
+    float *partial;
 };
 constexpr int kGenericTileM = 64;
+constexpr int64_t kGenericPartialFloats = 4 << 20;  // workspace floats for split partials
 cudaError_t launch_gemm_generic(const GenericGemmArgs &g, int64_t max_tiles_m, cudaStream_t s);
 
 // ---- backward (backward.cu)

@@ -254,7 +254,7 @@ struct BwdLayout {
         pre, up, h, dh, dxs, dw, dz, doff, dmt, one, spre, sup, sh, sdh;
     // bf16 path (tensor cores): 128-row tile prefix, padded column starts,
     // transposed weights, the bf16 [da | du], transposed activations
-    size_t mt128, kpad, w2t, wcat, dacat, dysT, xsT, hwT, daT, duT, total;
+    size_t mt128, kpad, w2t, wcat, dacat, dysT, xsT, hwT, daT, duT, partial, total;
     int64_t kp;  // columns of the transposed activations
 };
 
@@ -326,6 +326,7 @@ BwdLayout bwd_layout(const moe_config *c)
     L.hwT = take(tc ? F * kp * 2 : 0);
     L.daT = take(tc ? F * kp * 2 : 0);
     L.duT = take(tc && swiglu ? F * kp * 2 : 0);
+    L.partial = take(static_cast<size_t>(kGenericPartialFloats) * 4);
     L.total = o;
     return L;
 }
@@ -333,6 +334,7 @@ BwdLayout bwd_layout(const moe_config *c)
 // One strided product on gemm_generic_kernel (see kernels.h).
 struct GG {
     GenericGemmArgs g{};
+    float *partial = nullptr;  // workspace for split reductions (sum_rows)
     GG &a(const void *p, int64_t sm, int64_t sk, bool bf16)
     {
         g.A = p; g.sam = sm; g.sak = sk; g.a_bf16 = bf16 ? 1 : 0;
@@ -356,10 +358,23 @@ struct GG {
         return launch_gemm_generic(g, (rows_total + kGenericTileM - 1) / kGenericTileM + G, s);
     }
     // per group an M x N result summed over rows offsets[gi] .. offsets[gi+1]-1
+    // Few output tiles (the router's dW_g, the shared expert): the sums are
+    // split so that about four CTAs per SM run, partials fixed-order reduced.
     cudaError_t sum_rows(const int32_t *off, int G, int64_t M, int64_t N, cudaStream_t s)
     {
         g.offsets = off; g.mt_prefix = nullptr; g.G = G; g.ragged_k = 1; g.M = M; g.N = N;
+        const int64_t tiles = ((M + 63) / 64) * ((N + 63) / 64) * G;
+        int64_t ks = tiles > 0 ? (148 * 4) / tiles : 1;
+        ks = ks > 32 ? 32 : (ks < 1 ? 1 : ks);
+        while (ks > 1 && ks * G * M * N > kGenericPartialFloats) --ks;
+        g.ksplit = partial ? static_cast<int>(ks) : 1;
+        g.partial = partial;
         return launch_gemm_generic(g, 0, s);
+    }
+    GG &split(float *p)
+    {
+        partial = p;
+        return *this;
     }
 };
 
@@ -731,7 +746,7 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
     void *xs = at<void>(ws, L.xs), *dys = at<void>(ws, L.dys);
     float *row_w = at<float>(ws, L.row_w), *pre = at<float>(ws, L.pre), *up = swiglu ? at<float>(ws, L.up) : nullptr;
     float *h = at<float>(ws, L.h), *dh = at<float>(ws, L.dh), *dxs = at<float>(ws, L.dxs), *dw = at<float>(ws, L.dw);
-    float *dz = at<float>(ws, L.dz), *one = at<float>(ws, L.one);
+    float *dz = at<float>(ws, L.dz), *one = at<float>(ws, L.one), *partial = at<float>(ws, L.partial);
 
     // ---- recompute: routing (with p and lse), counts, slices, x_sorted
     RouterArgs r = router_args(cfg, x, W_g, b_e, ids, w, probs, hist, nullptr);
@@ -853,7 +868,7 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
     BwdRouterArgs rb{probs, lse, ids, dw, counts, dz, N, E, k, cfg->router, cfg->norm_topk, cfg->routed_scaling,
                      aux_coef, z_coef};
     MOE_TRY(launch_router_backward(rb, sms, s));
-    MOE_TRY(GG().a(dz, 1, E, false).b(x, d, 1, 0, bf).c(gr.dW_g, d, 1, 0).sum_rows(doff, 1, E, d, s));
+    MOE_TRY(GG().split(partial).a(dz, 1, E, false).b(x, d, 1, 0, bf).c(gr.dW_g, d, 1, 0).sum_rows(doff, 1, E, d, s));
     MOE_TRY(GG().a(dz, E, 1, false).b(W_g, d, 1, 0, bf).c(gr.dx, d, 1, 0, true).rows(doff, dmt, 1, N, d, E, s));
 
     // ---- shared expert: the same with weight 1 over all N rows of x
@@ -868,14 +883,14 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
         MOE_TRY(launch_act_forward(sa, sms, s));
         MOE_TRY(GG().a(dy, d, 1, bf).b(shared->W2, Fs, 1, 0, bf).c(sdh, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
         MOE_TRY(launch_row_backward(sa, sms, s));
-        MOE_TRY(GG().a(dy, 1, d, bf).b(sh, Fs, 1, 0, false).c(gr.dWs2, Fs, 1, 0).sum_rows(doff, 1, d, Fs, s));
+        MOE_TRY(GG().split(partial).a(dy, 1, d, bf).b(sh, Fs, 1, 0, false).c(gr.dWs2, Fs, 1, 0).sum_rows(doff, 1, d, Fs, s));
         if (shared->b2 && gr.dbs2)
-            MOE_TRY(GG().a(dy, 1, d, bf).b(one, 0, 0, 0, false).c(gr.dbs2, 1, 0, 0).sum_rows(doff, 1, d, 1, s));
-        MOE_TRY(GG().a(spre, 1, Fs, false).b(x, d, 1, 0, bf).c(gr.dWs1, d, 1, 0).sum_rows(doff, 1, Fs, d, s));
+            MOE_TRY(GG().split(partial).a(dy, 1, d, bf).b(one, 0, 0, 0, false).c(gr.dbs2, 1, 0, 0).sum_rows(doff, 1, d, 1, s));
+        MOE_TRY(GG().split(partial).a(spre, 1, Fs, false).b(x, d, 1, 0, bf).c(gr.dWs1, d, 1, 0).sum_rows(doff, 1, Fs, d, s));
         if (swiglu)
-            MOE_TRY(GG().a(sup, 1, Fs, false).b(x, d, 1, 0, bf).c(gr.dWs3, d, 1, 0).sum_rows(doff, 1, Fs, d, s));
+            MOE_TRY(GG().split(partial).a(sup, 1, Fs, false).b(x, d, 1, 0, bf).c(gr.dWs3, d, 1, 0).sum_rows(doff, 1, Fs, d, s));
         if (!swiglu && shared->b1 && gr.dbs1)
-            MOE_TRY(GG().a(spre, 1, Fs, false).b(one, 0, 0, 0, false).c(gr.dbs1, 1, 0, 0).sum_rows(doff, 1, Fs, 1, s));
+            MOE_TRY(GG().split(partial).a(spre, 1, Fs, false).b(one, 0, 0, 0, false).c(gr.dbs1, 1, 0, 0).sum_rows(doff, 1, Fs, 1, s));
         MOE_TRY(GG().a(spre, Fs, 1, false).b(shared->W1, d, 1, 0, bf).c(gr.dx, d, 1, 0, true)
                     .rows(doff, dmt, 1, N, d, Fs, s));
         if (swiglu)
