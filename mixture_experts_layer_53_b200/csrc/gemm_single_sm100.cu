@@ -72,6 +72,7 @@ struct GemmArgs {
     // columns; expert e's result starts at out_f32 + e * c_stride
     int ragged_k, m_tiles;
     int64_t m_total, c_stride;
+    int accumulate;  // EPI_F32: add to the existing result instead of overwriting
 };
 
 struct Ctl {
@@ -136,9 +137,15 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase,
                 for (int v = 0; v < 8; ++v) {
                     const int col = n0 + c + v * 4;
                     if (col < g.n_out) {  // n_out is a multiple of 4 (16-byte stores)
-                        const uint4 q = zero ? make_uint4(0, 0, 0, 0)
-                                             : make_uint4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
-                        st16(orow + col, q);
+                        float4 q = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                        : make_float4(__uint_as_float(acc[4 * v]), __uint_as_float(acc[4 * v + 1]),
+                                                      __uint_as_float(acc[4 * v + 2]),
+                                                      __uint_as_float(acc[4 * v + 3]));
+                        if (g.accumulate) {
+                            const float4 o = *reinterpret_cast<const float4 *>(orow + col);
+                            q.x += o.x; q.y += o.y; q.z += o.z; q.w += o.w;
+                        }
+                        *reinterpret_cast<float4 *>(orow + col) = q;
                     }
                 }
             }
@@ -408,6 +415,7 @@ cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s)
     g.m_tiles = static_cast<int>((t.m_total + BM - 1) / BM);
     g.m_total = t.m_total;
     g.c_stride = t.c_stride;
+    g.accumulate = t.accumulate;
     return launch_gemm<EPI_F32>(tA, tB, tB, g, num_sms, s);
 }
 

@@ -297,6 +297,7 @@ struct TcGemmArgs {
     int E, ragged_k, K, n_out;
     int64_t m_total;
     int32_t *status;
+    int accumulate;  // add to C instead of overwriting it
 };
 cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s);
 

@@ -254,8 +254,11 @@ struct BwdLayout {
         pre, up, h, dh, dxs, dw, dz, doff, dmt, one, spre, sup, sh, sdh;
     // bf16 path (tensor cores): 128-row tile prefix, padded column starts,
     // transposed weights, the bf16 [da | du], transposed activations
-    size_t mt128, kpad, w2t, wcat, dacat, dysT, xsT, hwT, daT, duT, partial, total;
-    int64_t kp;  // columns of the transposed activations
+    size_t mt128, kpad, w2t, wcat, dacat, dysT, xsT, hwT, daT, duT, partial;
+    // bf16 shared expert on the tensor cores: the same over one group of N rows
+    size_t smt128, skpad, ws2t, swcat, sdcat, dyT, xT, shT, sdaT, sduT, total;
+    int64_t kp;   // columns of the transposed activations
+    int64_t skp;  // the same for the shared expert's N rows
 };
 
 // Columns of the transposed, per-expert padded activations: every expert's
@@ -327,6 +330,19 @@ BwdLayout bwd_layout(const moe_config *c)
     L.daT = take(tc ? F * kp * 2 : 0);
     L.duT = take(tc && swiglu ? F * kp * 2 : 0);
     L.partial = take(static_cast<size_t>(kGenericPartialFloats) * 4);
+    const bool stc = tc && Fs > 0;
+    L.skp = (c->N + 64 + 63) / 64 * 64;
+    const size_t skp = static_cast<size_t>(L.skp);
+    L.smt128 = take(2 * 4);
+    L.skpad = take(2 * 4);
+    L.ws2t = take(stc ? Fs * d * 2 : 0);
+    L.swcat = take(stc ? d * m * Fs * 2 : 0);
+    L.sdcat = take(stc ? Nn * m * Fs * 2 : 0);
+    L.dyT = take(stc ? d * skp * 2 : 0);
+    L.xT = take(stc ? d * skp * 2 : 0);
+    L.shT = take(stc ? Fs * skp * 2 : 0);
+    L.sdaT = take(stc ? Fs * skp * 2 : 0);
+    L.sduT = take(stc && swiglu ? Fs * skp * 2 : 0);
     L.total = o;
     return L;
 }
@@ -773,6 +789,27 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
     GatherArgs gd{dy, inv, dys, N, d, k};  // dy_s[r] = dy[token of r]
     MOE_TRY(launch_gather(cfg->dtype, gd, sms, s));
 
+    // tensor-core products: rows offsets[g] .. of A and C per group (B per
+    // group n_out rows of K), or (tc_sum_rows) per group a sum over the
+    // group's padded columns of A [m_total, cols] and B [n_out, cols]
+    auto tc_rows = [&](const void *A, int64_t nrows, int64_t K, const void *B, int n_out, float *C,
+                       const int32_t *off, const int32_t *mt_, int G, bool accumulate) {
+        TcGemmArgs t{};
+        t.A = A; t.a_rows = static_cast<uint64_t>(nrows); t.a_cols = static_cast<uint64_t>(K);
+        t.B = B; t.b_rows = static_cast<uint64_t>(G) * n_out; t.b_cols = static_cast<uint64_t>(K);
+        t.C = C; t.ldc = n_out; t.offsets = off; t.mt_prefix = mt_; t.E = G; t.K = static_cast<int>(K);
+        t.n_out = n_out; t.status = dev_status; t.accumulate = accumulate ? 1 : 0;
+        return launch_gemm_tc_f32(t, sms, s);
+    };
+    auto tc_sum_rows = [&](const void *A, int64_t m_total, const void *B, int n_out, float *C, const int32_t *kp_off,
+                           int G, int64_t cols) {
+        TcGemmArgs t{};
+        t.A = A; t.a_rows = static_cast<uint64_t>(m_total); t.a_cols = static_cast<uint64_t>(cols);
+        t.B = B; t.b_rows = static_cast<uint64_t>(n_out); t.b_cols = static_cast<uint64_t>(cols);
+        t.C = C; t.ldc = n_out; t.c_stride = m_total * n_out; t.offsets = kp_off; t.E = G; t.ragged_k = 1;
+        t.n_out = n_out; t.m_total = m_total; t.status = dev_status;
+        return launch_gemm_tc_f32(t, sms, s);
+    };
     BwdActArgs act{rows, F, d, cfg->act, bf ? 1 : 0, pre, up, h, dh, swiglu ? nullptr : b1, b2,
                    at<int32_t>(ws, L.row_e), row_w, dw, perm, dys, nullptr};
     const int m = swiglu ? 2 : 1;
@@ -788,20 +825,10 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
         auto *duT = swiglu ? at<__nv_bfloat16>(ws, L.duT) : nullptr;
         const int64_t kp = L.kp;
         auto ragged_m = [&](const void *A, int64_t K, const void *B, int n_out, float *C) {
-            TcGemmArgs t{};
-            t.A = A; t.a_rows = static_cast<uint64_t>(rows); t.a_cols = static_cast<uint64_t>(K);
-            t.B = B; t.b_rows = static_cast<uint64_t>(E) * n_out; t.b_cols = static_cast<uint64_t>(K);
-            t.C = C; t.ldc = n_out; t.offsets = offsets; t.mt_prefix = mt128; t.E = E; t.K = static_cast<int>(K);
-            t.n_out = n_out; t.status = dev_status;
-            return launch_gemm_tc_f32(t, sms, s);
+            return tc_rows(A, rows, K, B, n_out, C, offsets, mt128, E, false);
         };
         auto ragged_k = [&](const void *A, int64_t m_total, const void *B, int n_out, float *C) {
-            TcGemmArgs t{};
-            t.A = A; t.a_rows = static_cast<uint64_t>(m_total); t.a_cols = static_cast<uint64_t>(kp);
-            t.B = B; t.b_rows = static_cast<uint64_t>(n_out); t.b_cols = static_cast<uint64_t>(kp);
-            t.C = C; t.ldc = n_out; t.c_stride = m_total * n_out; t.offsets = kpad; t.E = E; t.ragged_k = 1;
-            t.n_out = n_out; t.m_total = m_total; t.status = dev_status;
-            return launch_gemm_tc_f32(t, sms, s);
+            return tc_sum_rows(A, m_total, B, n_out, C, kpad, E, kp);
         };
         MOE_TRY(launch_tile_table(offsets, mt128, E, 128, s));
         MOE_TRY(launch_pad_offsets(counts, kpad, E, s));
@@ -875,27 +902,66 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
     if (shared) {
         float *spre = at<float>(ws, L.spre), *sup = swiglu ? at<float>(ws, L.sup) : nullptr;
         float *sh = at<float>(ws, L.sh), *sdh = at<float>(ws, L.sdh);
-        MOE_TRY(GG().a(x, d, 1, bf).b(shared->W1, 1, d, 0, bf).c(spre, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
-        if (swiglu)
-            MOE_TRY(GG().a(x, d, 1, bf).b(shared->W3, 1, d, 0, bf).c(sup, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
         BwdActArgs sa{N, Fs, d, cfg->act, bf ? 1 : 0, spre, sup, sh, sdh, swiglu ? nullptr : shared->b1, nullptr,
                       nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
-        MOE_TRY(launch_act_forward(sa, sms, s));
-        MOE_TRY(GG().a(dy, d, 1, bf).b(shared->W2, Fs, 1, 0, bf).c(sdh, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
-        MOE_TRY(launch_row_backward(sa, sms, s));
-        MOE_TRY(GG().split(partial).a(dy, 1, d, bf).b(sh, Fs, 1, 0, false).c(gr.dWs2, Fs, 1, 0).sum_rows(doff, 1, d, Fs, s));
-        if (shared->b2 && gr.dbs2)
-            MOE_TRY(GG().split(partial).a(dy, 1, d, bf).b(one, 0, 0, 0, false).c(gr.dbs2, 1, 0, 0).sum_rows(doff, 1, d, 1, s));
-        MOE_TRY(GG().split(partial).a(spre, 1, Fs, false).b(x, d, 1, 0, bf).c(gr.dWs1, d, 1, 0).sum_rows(doff, 1, Fs, d, s));
-        if (swiglu)
-            MOE_TRY(GG().split(partial).a(sup, 1, Fs, false).b(x, d, 1, 0, bf).c(gr.dWs3, d, 1, 0).sum_rows(doff, 1, Fs, d, s));
-        if (!swiglu && shared->b1 && gr.dbs1)
-            MOE_TRY(GG().split(partial).a(spre, 1, Fs, false).b(one, 0, 0, 0, false).c(gr.dbs1, 1, 0, 0).sum_rows(doff, 1, Fs, 1, s));
-        MOE_TRY(GG().a(spre, Fs, 1, false).b(shared->W1, d, 1, 0, bf).c(gr.dx, d, 1, 0, true)
-                    .rows(doff, dmt, 1, N, d, Fs, s));
-        if (swiglu)
-            MOE_TRY(GG().a(sup, Fs, 1, false).b(shared->W3, d, 1, 0, bf).c(gr.dx, d, 1, 0, true)
+        if (bf) {  // tensor cores, one group of N rows
+            int32_t *smt = at<int32_t>(ws, L.smt128), *skpad = at<int32_t>(ws, L.skpad);
+            auto *ws2t = at<__nv_bfloat16>(ws, L.ws2t), *swcat = at<__nv_bfloat16>(ws, L.swcat);
+            auto *sdcat = at<__nv_bfloat16>(ws, L.sdcat);
+            auto *dyT = at<__nv_bfloat16>(ws, L.dyT), *xT = at<__nv_bfloat16>(ws, L.xT);
+            auto *shT = at<__nv_bfloat16>(ws, L.shT), *sdaT = at<__nv_bfloat16>(ws, L.sdaT);
+            auto *sduT = swiglu ? at<__nv_bfloat16>(ws, L.sduT) : nullptr;
+            const int64_t skp = L.skp;
+            MOE_TRY(launch_tile_table(doff, smt, 1, 128, s));
+            MOE_TRY(launch_pad_offsets(doff + 1, skpad, 1, s));  // the one group's count is N
+            MOE_TRY(tc_rows(x, N, d, shared->W1, Fs, spre, doff, smt, 1, false));
+            if (swiglu) MOE_TRY(tc_rows(x, N, d, shared->W3, Fs, sup, doff, smt, 1, false));
+            MOE_TRY(launch_act_forward(sa, sms, s));
+            MOE_TRY(launch_transpose_weights(shared->W2, ws2t, 1, d, Fs, d, 0, s));
+            MOE_TRY(tc_rows(dy, N, d, ws2t, Fs, sdh, doff, smt, 1, false));
+            sa.dcat = sdcat;
+            MOE_TRY(launch_row_backward(sa, sms, s));
+            MOE_TRY(launch_transpose_weights(shared->W1, swcat, 1, Fs, d, static_cast<int64_t>(m) * Fs, 0, s));
+            if (swiglu) MOE_TRY(launch_transpose_weights(shared->W3, swcat, 1, Fs, d, 2LL * Fs, Fs, s));
+            MOE_TRY(tc_rows(sdcat, N, static_cast<int64_t>(m) * Fs, swcat, d, gr.dx, doff, smt, 1, true));
+            auto tr = [&](const void *src, int bf_in, int64_t ld_src, __nv_bfloat16 *dst, int C) {
+                TransposeRowsArgs t{src, bf_in, ld_src, dst, skp, C, 1, doff, skpad};
+                return launch_transpose_rows(t, skp, s);
+            };
+            MOE_TRY(tr(dy, 1, d, dyT, d));
+            MOE_TRY(tr(x, 1, d, xT, d));
+            MOE_TRY(tr(sh, 0, Fs, shT, Fs));
+            MOE_TRY(tr(sdcat, 1, static_cast<int64_t>(m) * Fs, sdaT, Fs));
+            if (swiglu) MOE_TRY(tr(sdcat + Fs, 1, 2LL * Fs, sduT, Fs));
+            MOE_TRY(tc_sum_rows(dyT, d, shT, Fs, gr.dWs2, skpad, 1, skp));
+            MOE_TRY(tc_sum_rows(sdaT, Fs, xT, d, gr.dWs1, skpad, 1, skp));
+            if (swiglu) MOE_TRY(tc_sum_rows(sduT, Fs, xT, d, gr.dWs3, skpad, 1, skp));
+        } else {
+            MOE_TRY(GG().a(x, d, 1, bf).b(shared->W1, 1, d, 0, bf).c(spre, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
+            if (swiglu)
+                MOE_TRY(GG().a(x, d, 1, bf).b(shared->W3, 1, d, 0, bf).c(sup, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
+            MOE_TRY(launch_act_forward(sa, sms, s));
+            MOE_TRY(GG().a(dy, d, 1, bf).b(shared->W2, Fs, 1, 0, bf).c(sdh, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
+            MOE_TRY(launch_row_backward(sa, sms, s));
+            MOE_TRY(GG().split(partial).a(dy, 1, d, bf).b(sh, Fs, 1, 0, false).c(gr.dWs2, Fs, 1, 0)
+                        .sum_rows(doff, 1, d, Fs, s));
+            MOE_TRY(GG().split(partial).a(spre, 1, Fs, false).b(x, d, 1, 0, bf).c(gr.dWs1, d, 1, 0)
+                        .sum_rows(doff, 1, Fs, d, s));
+            if (swiglu)
+                MOE_TRY(GG().split(partial).a(sup, 1, Fs, false).b(x, d, 1, 0, bf).c(gr.dWs3, d, 1, 0)
+                            .sum_rows(doff, 1, Fs, d, s));
+            MOE_TRY(GG().a(spre, Fs, 1, false).b(shared->W1, d, 1, 0, bf).c(gr.dx, d, 1, 0, true)
                         .rows(doff, dmt, 1, N, d, Fs, s));
+            if (swiglu)
+                MOE_TRY(GG().a(sup, Fs, 1, false).b(shared->W3, d, 1, 0, bf).c(gr.dx, d, 1, 0, true)
+                            .rows(doff, dmt, 1, N, d, Fs, s));
+        }
+        if (shared->b2 && gr.dbs2)
+            MOE_TRY(GG().split(partial).a(dy, 1, d, bf).b(one, 0, 0, 0, false).c(gr.dbs2, 1, 0, 0)
+                        .sum_rows(doff, 1, d, 1, s));
+        if (!swiglu && shared->b1 && gr.dbs1)
+            MOE_TRY(GG().split(partial).a(spre, 1, Fs, false).b(one, 0, 0, 0, false).c(gr.dbs1, 1, 0, 0)
+                        .sum_rows(doff, 1, Fs, 1, s));
     }
 #undef MOE_TRY
     return MOE_OK;

@@ -36,6 +36,8 @@ CASES = {
                                                               norm_topk=False), 1.0, 0.05),
     "bf16_deepseek_shared": (W.WORKLOADS["deepseek_v3_shared"].scaled(N=128, d_model=192, d_ff=64, E=64,
                                                                       d_ff_shared=64), 0.1, 0.01),
+    "bf16_gpt2_shared_bias": (W.WORKLOADS["gpt2_moe"].scaled(N=150, d_model=128, d_ff=128, d_ff_shared=96),
+                              0.05, 0.01),
     "one_token": (W.WORKLOADS["mixtral"].scaled(N=1, d_model=64, d_ff=64), 0.5, 0.5),
 }
 
