@@ -4,7 +4,8 @@
 // for the forward of the course module (sec. 2.1 with the sec. 2.3 Switch
 // loss) and the "nano-moe" router z-loss.  The expert choice and f_e are
 // piecewise constant; the selection bias only selects.  Everything here is
-// fp32; the products between these kernels run on gemm_generic_kernel.
+// fp32; the products between these kernels run on the tensor-core GEMM
+// (bf16 layers) or gemm_generic_kernel (fp32 layers).
 #include <float.h>
 
 #include "common.cuh"
@@ -326,36 +327,6 @@ __global__ void __launch_bounds__(256) transpose_rows_kernel(TransposeRowsArgs a
     }
 }
 
-// dst[e, c, col0 + r] = src[e, r, c]; R, C, ld_dst and col0 are multiples of 8.
-__global__ void __launch_bounds__(256) transpose_weights_kernel(const __nv_bfloat16 *src, __nv_bfloat16 *dst, int R,
-                                                                int C, int64_t ld_dst, int col0)
-{
-    pdl_enter();
-    __shared__ __nv_bfloat16 tile[64][72];
-    const int e = blockIdx.z;
-    const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
-    const int t = threadIdx.x;
-    const __nv_bfloat16 *sp = src + static_cast<int64_t>(e) * R * C;
-    __nv_bfloat16 *dp = dst + static_cast<int64_t>(e) * C * ld_dst;
-    for (int idx = t; idx < 64 * 8; idx += 256) {
-        const int i = idx >> 3, cv = (idx & 7) * 8;
-        const int r = r0 + i, c = c0 + cv;
-        uint4 q = make_uint4(0, 0, 0, 0);
-        if (r < R && c < C) q = *reinterpret_cast<const uint4 *>(sp + static_cast<int64_t>(r) * C + c);
-        *reinterpret_cast<uint4 *>(&tile[i][cv]) = q;
-    }
-    __syncthreads();
-    for (int idx = t; idx < 64 * 8; idx += 256) {
-        const int cl = idx >> 3, rv = (idx & 7) * 8;
-        const int c = c0 + cl, r = r0 + rv;
-        if (c >= C || r >= R) continue;
-        __nv_bfloat16 v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = tile[rv + j][cl];
-        *reinterpret_cast<uint4 *>(dp + static_cast<int64_t>(c) * ld_dst + col0 + r) = *reinterpret_cast<const uint4 *>(v);
-    }
-}
-
 int grid_for(int64_t work, int per_block, int num_sms)
 {
     const int64_t want = (work + per_block - 1) / per_block;
@@ -376,15 +347,6 @@ cudaError_t launch_transpose_rows(const TransposeRowsArgs &a, int64_t kp_max, cu
     const dim3 grid(static_cast<unsigned>((a.C + 63) / 64), static_cast<unsigned>(kp_max / 64));
     if (a.src_bf16) return launch_k(transpose_rows_kernel<true>, grid, dim3(256), 0, s, a);
     return launch_k(transpose_rows_kernel<false>, grid, dim3(256), 0, s, a);
-}
-
-cudaError_t launch_transpose_weights(const void *src, __nv_bfloat16 *dst, int E, int R, int C, int64_t ld_dst,
-                                     int col0, cudaStream_t s)
-{
-    const dim3 grid(static_cast<unsigned>((C + 63) / 64), static_cast<unsigned>((R + 63) / 64),
-                    static_cast<unsigned>(E));
-    return launch_k(transpose_weights_kernel, grid, dim3(256), 0, s, static_cast<const __nv_bfloat16 *>(src), dst, R,
-                    C, ld_dst, col0);
 }
 
 cudaError_t launch_rows_prep(const BwdRowsArgs &a, int num_sms, cudaStream_t s)

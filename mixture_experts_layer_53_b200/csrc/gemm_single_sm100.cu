@@ -73,6 +73,10 @@ struct GemmArgs {
     int ragged_k, m_tiles;
     int64_t m_total, c_stride;
     int accumulate;  // EPI_F32: add to the existing result instead of overwriting
+    // MN-major B (kernel template BMN): k-blocks 0..kb1-1 read tmB rows
+    // kb * BK of expert e with A columns kb * BK; k-blocks kb1..kb_total-1
+    // read tmB3 with A columns a_col2 + (kb - kb1) * BK
+    int kb1, kb_total, a_col2;
 };
 
 struct Ctl {
@@ -204,7 +208,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase,
     }
 }
 
-template <int EPI>
+// BMN (EPI_F32, ragged M): B tiles are MN-major -- four 64-column x 64-row
+// boxes of the [E][K][n_out] weights, 8 KB apart -- so the backward's
+// products against W^T need no transposed copy of the weights.
+template <int EPI, bool BMN = false>
 __global__ void __launch_bounds__(THREADS, 1)
     ffn_gemm_single_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmB3, const GemmArgs g)
@@ -233,7 +240,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (threadIdx.x == 32) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
-        if (EPI == EPI_SWIGLU) prefetch_tmap(&tmB3);
+        if (EPI == EPI_SWIGLU || BMN) prefetch_tmap(&tmB3);
     }
     if (warp == 1) {
         tmem_alloc(&ctl->tmem_base, TMEM_COLS);
@@ -249,7 +256,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     const uint32_t tmem_base = ctl->tmem_base;
     const int total = g.ragged_k ? g.E * g.m_tiles * g.n_tiles : ctl->mt[g.E] * g.n_tiles;
-    const int num_kb = (g.K + BK - 1) / BK;
+    const int num_kb = BMN ? g.kb_total : (g.K + BK - 1) / BK;
     // k-blocks of a tile and the column they start at
     auto kblocks = [&](int e) { return g.ragged_k ? (ctl->off[e + 1] - ctl->off[e]) / BK : num_kb; };
     auto kstart = [&](int e) { return g.ragged_k ? ctl->off[e] : 0; };
@@ -273,6 +280,26 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                     uint8_t *sA = tiles + stage * STAGE_BYTES;
                     uint8_t *sB = sA + A_BYTES;
+                    if constexpr (BMN) {
+                        // boxes wholly past n_out are not loaded: their
+                        // accumulator columns are never stored
+                        const int n0 = ti.n_tile * BN;
+                        const int boxes = min(BN / 64, (g.n_out - n0 + 63) / 64);
+                        mbar_arrive_expect_tx(&ctl->full[stage], A_BYTES + boxes * (B_BYTES / 4));
+                        armed |= 1u << stage;
+                        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                        const bool second = kb >= g.kb1;
+                        const int kk0 = (second ? kb - g.kb1 : kb) * BK;
+                        tma_load_2d(sA, &tmA, &ctl->full[stage], (second ? g.a_col2 : 0) + kk0, row0);
+                        const CUtensorMap *mb = second ? &tmB3 : &tmB;
+                        for (int c = 0; c < boxes; ++c)
+                            tma_load_3d(sB + c * (B_BYTES / 4), mb, &ctl->full[stage], n0 + c * 64, kk0, ti.e);
+                        if (++stage == STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                        continue;
+                    }
                     mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
                     armed |= 1u << stage;
                     armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -299,7 +326,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+            constexpr uint32_t idesc = BMN ? idesc_bf16_f32_bmn(BM, BN) : idesc_bf16_f32(BM, BN);
             int stage = 0, buf = 0;
             uint32_t phase = 0, tphase = 0;
             bool ok = true, issued = false;
@@ -317,9 +344,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint32_t a_addr = smem_u32(tiles + stage * STAGE_BYTES);
                     const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        umma_bf16(d_tmem, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32), idesc,
-                                  (kb | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        // K-major: 16 columns are 32 B inside each 128-B row;
+                        // MN-major: 16 K rows are two whole swizzle atoms
+                        const uint64_t bd = BMN ? desc_sw128_mn(b_addr + kk * 2048, B_BYTES / 4)
+                                                : desc_sw128(b_addr + kk * 32);
+                        umma_bf16(d_tmem, desc_sw128(a_addr + kk * 32), bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
                     issued = true;
                     umma_commit(&ctl->empty[stage]);
                     if (++stage == STAGES) {
@@ -382,14 +413,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // --------------------------------------------------------------- host side
 
-template <int EPI>
+template <int EPI, bool BMN = false>
 cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b3, const GemmArgs &g,
                         int num_sms, cudaStream_t s)
 {
-    cudaError_t err =
-        ensure_smem_attr(reinterpret_cast<const void *>(&ffn_gemm_single_kernel<EPI>), static_cast<int>(kSmemBytes));
+    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&ffn_gemm_single_kernel<EPI, BMN>),
+                                       static_cast<int>(kSmemBytes));
     if (err != cudaSuccess) return err;
-    return launch_k(ffn_gemm_single_kernel<EPI>, dim3(num_sms), dim3(THREADS), kSmemBytes, s, a, b, b3, g);
+    return launch_k(ffn_gemm_single_kernel<EPI, BMN>, dim3(num_sms), dim3(THREADS), kSmemBytes, s, a, b, b3, g);
 }
 
 }  // namespace
@@ -397,9 +428,19 @@ cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtens
 cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s)
 {
     if (t.ragged_k ? (t.m_total == 0 || t.n_out == 0) : (t.a_rows == 0 || t.n_out == 0)) return cudaSuccess;
-    CUtensorMap tA, tB;
-    if (!make_tmap_bf16(&tA, t.A, t.a_cols, t.a_rows, BM) || !make_tmap_bf16(&tB, t.B, t.b_cols, t.b_rows, 256))
+    if (t.b_mn && (t.ragged_k || t.k1 <= 0 || t.k2 < 0 || (t.k2 > 0) != (t.B2 != nullptr) ||
+                   static_cast<uint64_t>(t.k1 + t.k2) != t.a_cols || t.k1 % 8 != 0 || t.n_out % 8 != 0))
+        return cudaErrorInvalidValue;  // A's second column block must start on a 16-byte boundary
+    CUtensorMap tA, tB, tB3;
+    if (!make_tmap_bf16(&tA, t.A, t.a_cols, t.a_rows, BM)) return cudaErrorInvalidValue;
+    if (t.b_mn) {
+        const uint64_t n = static_cast<uint64_t>(t.n_out), G = static_cast<uint64_t>(t.E);
+        if (!make_tmap_bf16_mn(&tB, t.B, n, static_cast<uint64_t>(t.k1), G) ||
+            !make_tmap_bf16_mn(&tB3, t.B2 ? t.B2 : t.B, n, static_cast<uint64_t>(t.B2 ? t.k2 : t.k1), G))
+            return cudaErrorInvalidValue;
+    } else if (!make_tmap_bf16(&tB, t.B, t.b_cols, t.b_rows, 256)) {
         return cudaErrorInvalidValue;
+    }
     GemmArgs g{};
     g.offsets = t.offsets;
     g.mt_prefix = t.mt_prefix;
@@ -416,6 +457,12 @@ cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s)
     g.m_total = t.m_total;
     g.c_stride = t.c_stride;
     g.accumulate = t.accumulate;
+    if (t.b_mn) {
+        g.kb1 = static_cast<int>((t.k1 + BK - 1) / BK);
+        g.kb_total = g.kb1 + static_cast<int>((t.k2 + BK - 1) / BK);
+        g.a_col2 = static_cast<int>(t.k1);
+        return launch_gemm<EPI_F32, true>(tA, tB, tB3, g, num_sms, s);
+    }
     return launch_gemm<EPI_F32>(tA, tB, tB, g, num_sms, s);
 }
 

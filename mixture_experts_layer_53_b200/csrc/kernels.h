@@ -252,9 +252,6 @@ struct TransposeRowsArgs {
     const int32_t *offsets, *kpad;
 };
 cudaError_t launch_transpose_rows(const TransposeRowsArgs &a, int64_t kp_max, cudaStream_t s);
-// per expert e: dst[e, c, col0 + r] = src[e, r, c] for src [E, R, C] (bf16);
-cudaError_t launch_transpose_weights(const void *src, __nv_bfloat16 *dst, int E, int R, int C, int64_t ld_dst,
-                                     int col0, cudaStream_t s);
 
 struct FfnArgs {
     const void *x_sorted;      // [rows, d]
@@ -277,6 +274,7 @@ namespace moe {
 // TMA descriptor of a bf16 matrix [outer, inner] (inner contiguous) with a
 // box of [box_outer, 64] elements, 128-byte swizzle, zero fill outside.
 bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_outer);
+bool make_tmap_bf16_mn(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t groups);
 
 // C (fp32) = A B^T on tcgen05 with bf16 operands, both K-major (the
 // backward's products on the tensor cores), 128 x 256 tiles:
@@ -298,6 +296,13 @@ struct TcGemmArgs {
     int64_t m_total;
     int32_t *status;
     int accumulate;  // add to C instead of overwriting it
+    // b_mn (ragged M only): B is E matrices [k1 rows][n_out] with n_out
+    // contiguous, read as an MN-major operand (no transposed copy); A's
+    // columns 0..k1-1 pair with B, columns k1..k1+k2-1 with B2 (same layout,
+    // k2 rows; k2 = 0 and B2 = null without it)
+    int b_mn;
+    const void *B2;
+    int64_t k1, k2;
 };
 cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s);
 

@@ -254,9 +254,9 @@ struct BwdLayout {
         pre, up, h, dh, dxs, dw, dz, doff, dmt, one, spre, sup, sh, sdh;
     // bf16 path (tensor cores): 128-row tile prefix, padded column starts,
     // transposed weights, the bf16 [da | du], transposed activations
-    size_t mt128, kpad, w2t, wcat, dacat, dysT, xsT, hwT, daT, duT, partial;
+    size_t mt128, kpad, dacat, dysT, xsT, hwT, daT, duT, partial;
     // bf16 shared expert on the tensor cores: the same over one group of N rows
-    size_t smt128, skpad, ws2t, swcat, sdcat, dyT, xT, shT, sdaT, sduT, total;
+    size_t smt128, skpad, sdcat, dyT, xT, shT, sdaT, sduT, total;
     int64_t kp;   // columns of the transposed activations
     int64_t skp;  // the same for the shared expert's N rows
 };
@@ -321,8 +321,6 @@ BwdLayout bwd_layout(const moe_config *c)
     const size_t kp = static_cast<size_t>(L.kp);
     L.mt128 = take((E + 1) * 4);
     L.kpad = take((E + 1) * 4);
-    L.w2t = take(tc ? E * F * d * 2 : 0);
-    L.wcat = take(tc ? E * d * m * F * 2 : 0);
     L.dacat = take(tc ? A * m * F * 2 : 0);
     L.dysT = take(tc ? d * kp * 2 : 0);
     L.xsT = take(tc ? d * kp * 2 : 0);
@@ -335,8 +333,6 @@ BwdLayout bwd_layout(const moe_config *c)
     const size_t skp = static_cast<size_t>(L.skp);
     L.smt128 = take(2 * 4);
     L.skpad = take(2 * 4);
-    L.ws2t = take(stc ? Fs * d * 2 : 0);
-    L.swcat = take(stc ? d * m * Fs * 2 : 0);
     L.sdcat = take(stc ? Nn * m * Fs * 2 : 0);
     L.dyT = take(stc ? d * skp * 2 : 0);
     L.xT = take(stc ? d * skp * 2 : 0);
@@ -810,15 +806,26 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
         t.n_out = n_out; t.m_total = m_total; t.status = dev_status;
         return launch_gemm_tc_f32(t, sms, s);
     };
+    // the same with B = G matrices [K rows][n_out] read MN-major in place:
+    // A's columns 0..k1-1 against B1, k1..k1+k2-1 against B2
+    auto tc_rows_mn = [&](const void *A, int64_t nrows, const void *B1, int64_t k1, const void *B2, int64_t k2,
+                          int n_out, float *C, const int32_t *off, const int32_t *mt_, int G, bool accumulate) {
+        TcGemmArgs t{};
+        t.A = A; t.a_rows = static_cast<uint64_t>(nrows); t.a_cols = static_cast<uint64_t>(k1 + k2);
+        t.B = B1; t.B2 = B2; t.k1 = k1; t.k2 = k2; t.b_mn = 1;
+        t.C = C; t.ldc = n_out; t.offsets = off; t.mt_prefix = mt_; t.E = G; t.K = static_cast<int>(k1 + k2);
+        t.n_out = n_out; t.status = dev_status; t.accumulate = accumulate ? 1 : 0;
+        return launch_gemm_tc_f32(t, sms, s);
+    };
     BwdActArgs act{rows, F, d, cfg->act, bf ? 1 : 0, pre, up, h, dh, swiglu ? nullptr : b1, b2,
                    at<int32_t>(ws, L.row_e), row_w, dw, perm, dys, nullptr};
     const int m = swiglu ? 2 : 1;
     if (bf) {
         // ---- bf16: every expert product on the tensor cores (fp32 results);
-        // dgrad against transposed weights, wgrad over transposed activations
-        // whose per-expert column blocks start at multiples of 64
+        // dgrad with the weights read as MN-major operands in place, wgrad
+        // over transposed activations whose per-expert column blocks start
+        // at multiples of 64
         int32_t *mt128 = at<int32_t>(ws, L.mt128), *kpad = at<int32_t>(ws, L.kpad);
-        auto *w2t = at<__nv_bfloat16>(ws, L.w2t), *wcat = at<__nv_bfloat16>(ws, L.wcat);
         auto *dacat = at<__nv_bfloat16>(ws, L.dacat);
         auto *dysT = at<__nv_bfloat16>(ws, L.dysT), *xsT = at<__nv_bfloat16>(ws, L.xsT);
         auto *hwT = at<__nv_bfloat16>(ws, L.hwT), *daT = at<__nv_bfloat16>(ws, L.daT);
@@ -835,14 +842,12 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
         MOE_TRY(ragged_m(xs, d, W1, F, pre));
         if (swiglu) MOE_TRY(ragged_m(xs, d, W3, F, up));
         MOE_TRY(launch_act_forward(act, sms, s));
-        MOE_TRY(launch_transpose_weights(W2, w2t, E, d, F, d, 0, s));  // W2[e]^T: [F, d]
-        MOE_TRY(ragged_m(dys, d, w2t, F, dh));
+        MOE_TRY(tc_rows_mn(dys, rows, W2, d, nullptr, 0, F, dh, offsets, mt128, E, false));  // dh = dy_s W2[e]
         act.dcat = dacat;  // [da | du] in bf16 as well
         MOE_TRY(launch_row_backward(act, sms, s));
         // dx_s = [da | du] [W1[e] ; W3[e]]: one product with K = m F
-        MOE_TRY(launch_transpose_weights(W1, wcat, E, F, d, static_cast<int64_t>(m) * F, 0, s));
-        if (swiglu) MOE_TRY(launch_transpose_weights(W3, wcat, E, F, d, 2LL * F, F, s));
-        MOE_TRY(ragged_m(dacat, static_cast<int64_t>(m) * F, wcat, d, dxs));
+        MOE_TRY(tc_rows_mn(dacat, rows, W1, F, swiglu ? W3 : nullptr, swiglu ? F : 0, d, dxs, offsets, mt128, E,
+                           false));
         // weight gradients over the transposed, padded activations
         auto tr = [&](const void *src, int bf_in, int64_t ld_src, __nv_bfloat16 *dst, int C) {
             TransposeRowsArgs t{src, bf_in, ld_src, dst, kp, C, E, offsets, kpad};
@@ -906,7 +911,6 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
                       nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
         if (bf) {  // tensor cores, one group of N rows
             int32_t *smt = at<int32_t>(ws, L.smt128), *skpad = at<int32_t>(ws, L.skpad);
-            auto *ws2t = at<__nv_bfloat16>(ws, L.ws2t), *swcat = at<__nv_bfloat16>(ws, L.swcat);
             auto *sdcat = at<__nv_bfloat16>(ws, L.sdcat);
             auto *dyT = at<__nv_bfloat16>(ws, L.dyT), *xT = at<__nv_bfloat16>(ws, L.xT);
             auto *shT = at<__nv_bfloat16>(ws, L.shT), *sdaT = at<__nv_bfloat16>(ws, L.sdaT);
@@ -917,13 +921,11 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
             MOE_TRY(tc_rows(x, N, d, shared->W1, Fs, spre, doff, smt, 1, false));
             if (swiglu) MOE_TRY(tc_rows(x, N, d, shared->W3, Fs, sup, doff, smt, 1, false));
             MOE_TRY(launch_act_forward(sa, sms, s));
-            MOE_TRY(launch_transpose_weights(shared->W2, ws2t, 1, d, Fs, d, 0, s));
-            MOE_TRY(tc_rows(dy, N, d, ws2t, Fs, sdh, doff, smt, 1, false));
+            MOE_TRY(tc_rows_mn(dy, N, shared->W2, d, nullptr, 0, Fs, sdh, doff, smt, 1, false));
             sa.dcat = sdcat;
             MOE_TRY(launch_row_backward(sa, sms, s));
-            MOE_TRY(launch_transpose_weights(shared->W1, swcat, 1, Fs, d, static_cast<int64_t>(m) * Fs, 0, s));
-            if (swiglu) MOE_TRY(launch_transpose_weights(shared->W3, swcat, 1, Fs, d, 2LL * Fs, Fs, s));
-            MOE_TRY(tc_rows(sdcat, N, static_cast<int64_t>(m) * Fs, swcat, d, gr.dx, doff, smt, 1, true));
+            MOE_TRY(tc_rows_mn(sdcat, N, shared->W1, Fs, swiglu ? shared->W3 : nullptr, swiglu ? Fs : 0, d, gr.dx,
+                               doff, smt, 1, true));
             auto tr = [&](const void *src, int bf_in, int64_t ld_src, __nv_bfloat16 *dst, int C) {
                 TransposeRowsArgs t{src, bf_in, ld_src, dst, skp, C, 1, doff, skpad};
                 return launch_transpose_rows(t, skp, s);

@@ -49,4 +49,20 @@ bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t o
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 tensor [groups][rows][inner] (inner contiguous) read as MN-major
+// operand tiles: box {64 inner, 64 rows, 1 group}, 128-byte swizzle, zero
+// fill past the inner extent and past each group's rows.
+bool make_tmap_bf16_mn(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t groups)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {inner, rows, groups};
+    const cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(BK), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace moe
