@@ -546,7 +546,7 @@ def run_backward(args, wl):
         "config": describe(wl),
         "roofline": {"kernel": kern, "bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "peak_source": src, "flops_per_step": flops,
-                     "note": "achieved = all backward FLOPs over the whole step (transposes, element-wise and "
+                     "note": "achieved = all backward FLOPs over the whole step (recomputation, element-wise and "
                              "router kernels included)"},
         "clocks": cl,
     }

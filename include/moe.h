@@ -368,9 +368,9 @@ MOE_API size_t moe_backward_workspace_size(const moe_config *cfg);
  * same expert choice); all products accumulate in fp32.  bf16: the expert
  * products run on the tensor cores, with the intermediate gradients (da,
  * du, w h) rounded to bf16 as operands; fp32: on the CUDA cores throughout.
- * Workspace: moe_backward_workspace_size(cfg) bytes (it holds the
- * recomputed activations and, for bf16, transposed copies of them; the
- * weights are read in place).  Enqueues only.
+ * Workspace: moe_backward_workspace_size(cfg) bytes (the recomputed
+ * activations and the intermediate gradients; weights and activations are
+ * read in place by the tensor-core products).  Enqueues only.
  */
 MOE_API moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g,
                         const float *b_e, const void *W1, const void *b1,

@@ -76,8 +76,9 @@ __global__ void act_forward_kernel(BwdActArgs a)
 // before the gate weight), in one pass over the row with 4-float vectors:
 //   dw_r = <dh_raw_r, h_r> + <dy_s r, b2[e]>     (= <dy_n, Expert_e(x_n)>)
 //   dh = w_r dh_raw_r through the activation: pre <- da, up <- du, and
-//   h <- w_r h (the right operand of dW2 = dy_s^T (w h)); with dcat also the
-//   bf16 copies [da | du] that the tensor-core dgrad reads.
+//   h <- w_r h (the right operand of dW2 = dy_s^T (w h)); with dcat and
+//   hw_bf also the bf16 copies [da | du] and w h that the tensor-core
+//   products read (fp32 results in skip_f32 are then not written back).
 // Without a weight array (the shared expert) w_r = 1 and dw is not kept.
 __global__ void __launch_bounds__(256) row_backward_kernel(BwdActArgs a)
 {
@@ -120,9 +121,16 @@ __global__ void __launch_bounds__(256) row_backward_kernel(BwdActArgs a)
                 }
                 hv[q] *= wr;
             }
-            *reinterpret_cast<float4 *>(pre + f) = make_float4(da[0], da[1], da[2], da[3]);
-            if (swiglu) *reinterpret_cast<float4 *>(up + f) = make_float4(du[0], du[1], du[2], du[3]);
-            *reinterpret_cast<float4 *>(h + f) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+            if (!(a.skip_f32 & kSkipPre)) *reinterpret_cast<float4 *>(pre + f) = make_float4(da[0], da[1], da[2], da[3]);
+            if (swiglu && !(a.skip_f32 & kSkipUp))
+                *reinterpret_cast<float4 *>(up + f) = make_float4(du[0], du[1], du[2], du[3]);
+            if (!(a.skip_f32 & kSkipH)) *reinterpret_cast<float4 *>(h + f) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+            if (a.hw_bf) {
+                __nv_bfloat16 b4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) b4[q] = __float2bfloat16_rn(hv[q]);
+                *reinterpret_cast<uint2 *>(a.hw_bf + r * a.F + f) = *reinterpret_cast<const uint2 *>(b4);
+            }
             if (a.dcat) {
                 __nv_bfloat16 b4[4];
 #pragma unroll
@@ -259,74 +267,6 @@ __global__ void __launch_bounds__(256) router_backward_kernel(BwdRouterArgs a)
     }
 }
 
-__global__ void pad_offsets_kernel(const int32_t *counts, int32_t *kpad, int E)
-{
-    pdl_enter();
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        int32_t o = 0;
-        for (int e = 0; e < E; ++e) {
-            kpad[e] = o;
-            o += (counts[e] + 63) / 64 * 64;
-        }
-        kpad[E] = o;
-    }
-}
-
-// Transposes in 64 x 64 tiles through shared memory with 16-byte vectors on
-// both sides.  transpose_rows_kernel walks the padded column space of the
-// result: a 64-column tile lies inside one expert's block (its start kpad[e]
-// is a multiple of 64), so its source rows are contiguous; columns past the
-// expert's rows are written as zeros.
-template <bool BF16_IN>
-__global__ void __launch_bounds__(256) transpose_rows_kernel(TransposeRowsArgs a)
-{
-    pdl_enter();
-    __shared__ __nv_bfloat16 tile[64][72];
-    const int64_t pc0 = static_cast<int64_t>(blockIdx.y) * 64;  // padded column of the tile
-    if (pc0 >= a.kpad[a.E]) return;                              // block-uniform: past every expert
-    int lo = 0, hi = a.E - 1;                                    // expert whose block holds pc0
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (a.kpad[mid] <= pc0) lo = mid;
-        else hi = mid - 1;
-    }
-    const int64_t r0 = a.offsets[lo] + (pc0 - a.kpad[lo]);  // first source row
-    const int64_t r_end = a.offsets[lo + 1];
-    const int c0 = blockIdx.x * 64;
-    const int t = threadIdx.x;
-    // load: 64 rows x 64 columns, 8 columns per thread and step
-    for (int idx = t; idx < 64 * 8; idx += 256) {
-        const int i = idx >> 3, cv = (idx & 7) * 8;
-        const int64_t r = r0 + i;
-        const int c = c0 + cv;
-        float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (r < r_end && c < a.C) {  // C is a multiple of 8
-            if (BF16_IN) {
-                unpack16(*reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.src) + r * a.ld_src + c),
-                         f, static_cast<const __nv_bfloat16 *>(nullptr));
-            } else {
-                const float *p = static_cast<const float *>(a.src) + r * a.ld_src + c;
-                const float4 u = *reinterpret_cast<const float4 *>(p), w = *reinterpret_cast<const float4 *>(p + 4);
-                f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w; f[4] = w.x; f[5] = w.y; f[6] = w.z; f[7] = w.w;
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) tile[i][cv + j] = __float2bfloat16_rn(f[j]);
-    }
-    __syncthreads();
-    // store: row c of the result gets 64 consecutive columns, 8 per vector
-    for (int idx = t; idx < 64 * 8; idx += 256) {
-        const int cl = idx >> 3, rv = (idx & 7) * 8;
-        const int c = c0 + cl;
-        if (c >= a.C) continue;
-        __nv_bfloat16 v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = tile[rv + j][cl];
-        *reinterpret_cast<uint4 *>(a.dst + static_cast<int64_t>(c) * a.ld_dst + pc0 + rv) =
-            *reinterpret_cast<const uint4 *>(v);
-    }
-}
-
 int grid_for(int64_t work, int per_block, int num_sms)
 {
     const int64_t want = (work + per_block - 1) / per_block;
@@ -334,20 +274,6 @@ int grid_for(int64_t work, int per_block, int num_sms)
 }
 
 }  // namespace
-
-cudaError_t launch_pad_offsets(const int32_t *counts, int32_t *kpad, int E, cudaStream_t s)
-{
-    return launch_k(pad_offsets_kernel, dim3(1), dim3(32), 0, s, counts, kpad, E);
-}
-
-cudaError_t launch_transpose_rows(const TransposeRowsArgs &a, int64_t kp_max, cudaStream_t s)
-{
-    if (kp_max == 0 || a.C == 0) return cudaSuccess;
-    if (kp_max / 64 > 65535) return cudaErrorInvalidValue;
-    const dim3 grid(static_cast<unsigned>((a.C + 63) / 64), static_cast<unsigned>(kp_max / 64));
-    if (a.src_bf16) return launch_k(transpose_rows_kernel<true>, grid, dim3(256), 0, s, a);
-    return launch_k(transpose_rows_kernel<false>, grid, dim3(256), 0, s, a);
-}
 
 cudaError_t launch_rows_prep(const BwdRowsArgs &a, int num_sms, cudaStream_t s)
 {

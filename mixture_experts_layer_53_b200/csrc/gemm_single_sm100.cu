@@ -55,6 +55,15 @@ constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 
 enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_LINEAR = 2, EPI_F32 = 3 };
+// Operand layouts (kernel template OPS):
+//   OPS_KK    A and B K-major (the forward, the recomputed pre-activations)
+//   OPS_K_MN  B MN-major: [E][K][n_out] weights read in place by 64 x 64
+//             boxes (the dgrad products against W^T); ragged M
+//   OPS_MN_MN A and B MN-major: row-major activations [rows][M] and
+//             [rows][n_out]; expert e sums its own rows offsets[e] ..
+//             offsets[e+1]-1 (the weight gradients); ragged K
+enum { OPS_KK = 0, OPS_K_MN = 1, OPS_MN_MN = 2 };
+constexpr int BOX_BYTES = 64 * 64 * 2;  // one 64 x 64 MN-major box
 
 struct GemmArgs {
     const int32_t *offsets;
@@ -73,9 +82,9 @@ struct GemmArgs {
     int ragged_k, m_tiles;
     int64_t m_total, c_stride;
     int accumulate;  // EPI_F32: add to the existing result instead of overwriting
-    // MN-major B (kernel template BMN): k-blocks 0..kb1-1 read tmB rows
-    // kb * BK of expert e with A columns kb * BK; k-blocks kb1..kb_total-1
-    // read tmB3 with A columns a_col2 + (kb - kb1) * BK
+    // OPS_K_MN: k-blocks 0..kb1-1 read tmB rows kb * BK of expert e with A
+    // columns kb * BK; k-blocks kb1..kb_total-1 read tmB3 with A columns
+    // a_col2 + (kb - kb1) * BK
     int kb1, kb_total, a_col2;
 };
 
@@ -208,10 +217,12 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase,
     }
 }
 
-// BMN (EPI_F32, ragged M): B tiles are MN-major -- four 64-column x 64-row
-// boxes of the [E][K][n_out] weights, 8 KB apart -- so the backward's
-// products against W^T need no transposed copy of the weights.
-template <int EPI, bool BMN = false>
+// MN-major operand tiles (OPS_K_MN, OPS_MN_MN; EPI_F32 only) are 64-column
+// x 64-row boxes 8 KB apart, so the backward's products against W^T and
+// over token rows need no transposed copies.  In OPS_MN_MN the last k-block
+// of an expert can hold rows of the next one: the MMA warp zeroes those rows
+// of both tiles in shared memory before the MMA reads them.
+template <int EPI, int OPS = OPS_KK>
 __global__ void __launch_bounds__(THREADS, 1)
     ffn_gemm_single_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmB3, const GemmArgs g)
@@ -240,7 +251,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (threadIdx.x == 32) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
-        if (EPI == EPI_SWIGLU || BMN) prefetch_tmap(&tmB3);
+        if (EPI == EPI_SWIGLU || OPS == OPS_K_MN) prefetch_tmap(&tmB3);
     }
     if (warp == 1) {
         tmem_alloc(&ctl->tmem_base, TMEM_COLS);
@@ -256,9 +267,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     const uint32_t tmem_base = ctl->tmem_base;
     const int total = g.ragged_k ? g.E * g.m_tiles * g.n_tiles : ctl->mt[g.E] * g.n_tiles;
-    const int num_kb = BMN ? g.kb_total : (g.K + BK - 1) / BK;
-    // k-blocks of a tile and the column they start at
-    auto kblocks = [&](int e) { return g.ragged_k ? (ctl->off[e + 1] - ctl->off[e]) / BK : num_kb; };
+    const int num_kb = OPS == OPS_K_MN ? g.kb_total : (g.K + BK - 1) / BK;
+    // k-blocks of a tile and the column (OPS_MN_MN: row) they start at
+    auto kblocks = [&](int e) {
+        if (OPS == OPS_MN_MN) return (ctl->off[e + 1] - ctl->off[e] + BK - 1) / BK;
+        return g.ragged_k ? (ctl->off[e + 1] - ctl->off[e]) / BK : num_kb;
+    };
     auto kstart = [&](int e) { return g.ragged_k ? ctl->off[e] : 0; };
 
     if (warp == 0) {
@@ -280,12 +294,32 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                     uint8_t *sA = tiles + stage * STAGE_BYTES;
                     uint8_t *sB = sA + A_BYTES;
-                    if constexpr (BMN) {
+                    if constexpr (OPS == OPS_MN_MN) {
+                        // boxes wholly past m_total / n_out are not loaded:
+                        // their accumulator rows / columns are never stored
+                        const int m0 = ti.m_tile * BM, n0 = ti.n_tile * BN;
+                        const int aboxes = min(BM / 64, static_cast<int>((g.m_total - m0 + 63) / 64));
+                        const int bboxes = min(BN / 64, (g.n_out - n0 + 63) / 64);
+                        mbar_arrive_expect_tx(&ctl->full[stage], (aboxes + bboxes) * BOX_BYTES);
+                        armed |= 1u << stage;
+                        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                        const int r = k0 + kb * BK;
+                        for (int c = 0; c < aboxes; ++c)
+                            tma_load_2d(sA + c * BOX_BYTES, &tmA, &ctl->full[stage], m0 + c * 64, r);
+                        for (int c = 0; c < bboxes; ++c)
+                            tma_load_2d(sB + c * BOX_BYTES, &tmB, &ctl->full[stage], n0 + c * 64, r);
+                        if (++stage == STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                        continue;
+                    }
+                    if constexpr (OPS == OPS_K_MN) {
                         // boxes wholly past n_out are not loaded: their
                         // accumulator columns are never stored
                         const int n0 = ti.n_tile * BN;
                         const int boxes = min(BN / 64, (g.n_out - n0 + 63) / 64);
-                        mbar_arrive_expect_tx(&ctl->full[stage], A_BYTES + boxes * (B_BYTES / 4));
+                        mbar_arrive_expect_tx(&ctl->full[stage], A_BYTES + boxes * BOX_BYTES);
                         armed |= 1u << stage;
                         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
                         const bool second = kb >= g.kb1;
@@ -293,7 +327,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         tma_load_2d(sA, &tmA, &ctl->full[stage], (second ? g.a_col2 : 0) + kk0, row0);
                         const CUtensorMap *mb = second ? &tmB3 : &tmB;
                         for (int c = 0; c < boxes; ++c)
-                            tma_load_3d(sB + c * (B_BYTES / 4), mb, &ctl->full[stage], n0 + c * 64, kk0, ti.e);
+                            tma_load_3d(sB + c * BOX_BYTES, mb, &ctl->full[stage], n0 + c * 64, kk0, ti.e);
                         if (++stage == STAGES) {
                             stage = 0;
                             phase ^= 1u;
@@ -324,48 +358,80 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc = BMN ? idesc_bf16_f32_bmn(BM, BN) : idesc_bf16_f32(BM, BN);
+        // ---------------------------------------------------- MMA issuer
+        // One lane issues; with OPS_MN_MN the whole warp runs the loop and
+        // zeroes the rows past an expert's end before the MMA reads them.
+        constexpr bool kWarp = OPS == OPS_MN_MN;
+        if (kWarp || lane == 0) {
+            constexpr uint32_t idesc = OPS == OPS_MN_MN   ? idesc_bf16_f32_mn(BM, BN)
+                                       : OPS == OPS_K_MN ? idesc_bf16_f32_bmn(BM, BN)
+                                                         : idesc_bf16_f32(BM, BN);
+            auto wait = [&](uint64_t *bar, uint32_t parity) {
+                const bool w = mbar_wait(bar, parity, abort_flag, g.status);
+                return kWarp ? __all_sync(0xffffffffu, w) : w;
+            };
             int stage = 0, buf = 0;
             uint32_t phase = 0, tphase = 0;
             bool ok = true, issued = false;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                if (!mbar_wait(&ctl->tempty[buf], tphase ^ 1u, abort_flag, g.status)) break;
+                if (!wait(&ctl->tempty[buf], tphase ^ 1u)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-                const int nkb = kblocks(tile_of(t, ctl, g).e);
+                const int e = tile_of(t, ctl, g).e;
+                const int nkb = kblocks(e);
                 for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&ctl->full[stage], phase, abort_flag, g.status)) {
+                    if (!wait(&ctl->full[stage], phase)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(tiles + stage * STAGE_BYTES);
-                    const uint32_t b_addr = a_addr + A_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        // K-major: 16 columns are 32 B inside each 128-B row;
-                        // MN-major: 16 K rows are two whole swizzle atoms
-                        const uint64_t bd = BMN ? desc_sw128_mn(b_addr + kk * 2048, B_BYTES / 4)
-                                                : desc_sw128(b_addr + kk * 32);
-                        umma_bf16(d_tmem, desc_sw128(a_addr + kk * 32), bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    uint8_t *st = tiles + stage * STAGE_BYTES;
+                    if constexpr (kWarp) {
+                        // rows v..63 of every box (2 of A, 4 of B) belong to
+                        // the next expert; whole 128-B rows, so the swizzle
+                        // does not matter
+                        const int v = ctl->off[e + 1] - ctl->off[e] - kb * BK;
+                        if (v < BK) {
+                            const int per_box = (BK - v) * 8;  // 16-B chunks
+                            for (int i = lane; i < 6 * per_box; i += 32) {
+                                const int box = i / per_box, j = i - box * per_box;
+                                *reinterpret_cast<uint4 *>(st + box * BOX_BYTES + v * 128 + j * 16) =
+                                    make_uint4(0u, 0u, 0u, 0u);
+                            }
+                            fence_proxy_async_smem();
+                        }
+                        __syncwarp();
                     }
-                    issued = true;
-                    umma_commit(&ctl->empty[stage]);
+                    if (!kWarp || lane == 0) {
+                        const uint32_t a_addr = smem_u32(st);
+                        const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            // K-major: 16 columns are 32 B inside each 128-B
+                            // row; MN-major: 16 K rows are two whole swizzle atoms
+                            const uint64_t ad = OPS == OPS_MN_MN ? desc_sw128_mn(a_addr + kk * 2048, BOX_BYTES)
+                                                                 : desc_sw128(a_addr + kk * 32);
+                            const uint64_t bd = OPS != OPS_KK ? desc_sw128_mn(b_addr + kk * 2048, BOX_BYTES)
+                                                              : desc_sw128(b_addr + kk * 32);
+                            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        }
+                        issued = true;
+                        umma_commit(&ctl->empty[stage]);
+                    }
+                    if (kWarp) __syncwarp();
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                umma_commit(&ctl->tfull[buf]);
+                if (!kWarp || lane == 0) umma_commit(&ctl->tfull[buf]);
                 if (++buf == 2) {
                     buf = 0;
                     tphase ^= 1u;
                 }
             }
-            if (*abort_flag && issued) {
+            if ((!kWarp || lane == 0) && *abort_flag && issued) {
                 // wait for every MMA issued so far before TMEM is freed
                 umma_commit(&ctl->drain);
                 mbar_wait(&ctl->drain, 0, abort_flag, g.status, false);
@@ -413,14 +479,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // --------------------------------------------------------------- host side
 
-template <int EPI, bool BMN = false>
+template <int EPI, int OPS = OPS_KK>
 cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b3, const GemmArgs &g,
                         int num_sms, cudaStream_t s)
 {
-    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&ffn_gemm_single_kernel<EPI, BMN>),
+    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&ffn_gemm_single_kernel<EPI, OPS>),
                                        static_cast<int>(kSmemBytes));
     if (err != cudaSuccess) return err;
-    return launch_k(ffn_gemm_single_kernel<EPI, BMN>, dim3(num_sms), dim3(THREADS), kSmemBytes, s, a, b, b3, g);
+    return launch_k(ffn_gemm_single_kernel<EPI, OPS>, dim3(num_sms), dim3(THREADS), kSmemBytes, s, a, b, b3, g);
 }
 
 }  // namespace
@@ -431,6 +497,32 @@ cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s)
     if (t.b_mn && (t.ragged_k || t.k1 <= 0 || t.k2 < 0 || (t.k2 > 0) != (t.B2 != nullptr) ||
                    static_cast<uint64_t>(t.k1 + t.k2) != t.a_cols || t.k1 % 8 != 0 || t.n_out % 8 != 0))
         return cudaErrorInvalidValue;  // A's second column block must start on a 16-byte boundary
+    if (t.rows_mn) {
+        // row strides and inner extents in whole 16-byte units (tensor map rules)
+        if (!t.ragged_k || t.b_mn || t.lda % 8 != 0 || t.ldb % 8 != 0 || t.m_total % 8 != 0 || t.n_out % 8 != 0 ||
+            t.m_total > t.lda || t.n_out > t.ldb)
+            return cudaErrorInvalidValue;
+        CUtensorMap tA, tB;
+        if (!make_tmap_bf16_mn_rows(&tA, t.A, static_cast<uint64_t>(t.m_total), t.a_rows,
+                                    static_cast<uint64_t>(t.lda)) ||
+            !make_tmap_bf16_mn_rows(&tB, t.B, static_cast<uint64_t>(t.n_out), t.a_rows,
+                                    static_cast<uint64_t>(t.ldb)))
+            return cudaErrorInvalidValue;
+        GemmArgs g{};
+        g.offsets = t.offsets;
+        g.out_f32 = t.C;
+        g.ldo = t.ldc;
+        g.status = t.status;
+        g.E = t.E;
+        g.n_out = t.n_out;
+        g.n_tiles = (t.n_out + 255) / 256;
+        g.ragged_k = 1;
+        g.m_tiles = static_cast<int>((t.m_total + BM - 1) / BM);
+        g.m_total = t.m_total;
+        g.c_stride = t.c_stride;
+        g.accumulate = t.accumulate;
+        return launch_gemm<EPI_F32, OPS_MN_MN>(tA, tB, tB, g, num_sms, s);
+    }
     CUtensorMap tA, tB, tB3;
     if (!make_tmap_bf16(&tA, t.A, t.a_cols, t.a_rows, BM)) return cudaErrorInvalidValue;
     if (t.b_mn) {
@@ -461,7 +553,7 @@ cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s)
         g.kb1 = static_cast<int>((t.k1 + BK - 1) / BK);
         g.kb_total = g.kb1 + static_cast<int>((t.k2 + BK - 1) / BK);
         g.a_col2 = static_cast<int>(t.k1);
-        return launch_gemm<EPI_F32, true>(tA, tB, tB3, g, num_sms, s);
+        return launch_gemm<EPI_F32, OPS_K_MN>(tA, tB, tB3, g, num_sms, s);
     }
     return launch_gemm<EPI_F32>(tA, tB, tB, g, num_sms, s);
 }

@@ -210,7 +210,10 @@ struct BwdActArgs {
     const int32_t *perm;   // [rows] (with dw)
     const void *dy_s;      // [rows, d] (with dw and b2)
     __nv_bfloat16 *dcat;   // [rows, m F] or null: bf16 copies [da | du] (the tensor-core dgrad operand)
+    __nv_bfloat16 *hw_bf;  // [rows, F] or null: bf16 copy of w h (the tensor-core dW2 operand)
+    int skip_f32;          // row_backward: fp32 results not written back (kSkip* bits)
 };
+constexpr int kSkipPre = 1, kSkipUp = 2, kSkipH = 4;
 cudaError_t launch_act_forward(const BwdActArgs &a, int num_sms, cudaStream_t s);
 cudaError_t launch_row_backward(const BwdActArgs &a, int num_sms, cudaStream_t s);
 
@@ -235,24 +238,6 @@ struct BwdRouterArgs {
 };
 cudaError_t launch_router_backward(const BwdRouterArgs &a, int num_sms, cudaStream_t s);
 
-// Layout helpers of the tensor-core backward (bf16 operands):
-// padded column starts kpad[e] = sum_{e' < e} roundup64(counts[e']);
-cudaError_t launch_pad_offsets(const int32_t *counts, int32_t *kpad, int E, cudaStream_t s);
-// dst[c, kpad[e] + r - offsets[e]] = src[r, c] for the rows r of expert e
-// (bf16; src fp32 or bf16 with row stride ld_src), and zeros in
-// dst[c, kpad[e] + count_e .. kpad[e+1]); columns from kpad[E] on are not
-// written.  kp_max: an upper bound of kpad[E] (a multiple of 64).
-struct TransposeRowsArgs {
-    const void *src;
-    int src_bf16;
-    int64_t ld_src;
-    __nv_bfloat16 *dst;
-    int64_t ld_dst;
-    int C, E;
-    const int32_t *offsets, *kpad;
-};
-cudaError_t launch_transpose_rows(const TransposeRowsArgs &a, int64_t kp_max, cudaStream_t s);
-
 struct FfnArgs {
     const void *x_sorted;      // [rows, d]
     const int32_t *offsets;    // [E+1]
@@ -275,6 +260,7 @@ namespace moe {
 // box of [box_outer, 64] elements, 128-byte swizzle, zero fill outside.
 bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_outer);
 bool make_tmap_bf16_mn(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t groups);
+bool make_tmap_bf16_mn_rows(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t ld);
 
 // C (fp32) = A B^T on tcgen05 with bf16 operands, both K-major (the
 // backward's products on the tensor cores), 128 x 256 tiles:
@@ -303,6 +289,12 @@ struct TcGemmArgs {
     int b_mn;
     const void *B2;
     int64_t k1, k2;
+    // rows_mn (ragged K only): A and B are row-major [a_rows][lda] and
+    // [a_rows][ldb] whose columns 0..m_total-1 and 0..n_out-1 are the result
+    // rows and columns; expert e sums rows offsets[e] .. offsets[e+1]-1 (no
+    // padding; the result of an expert without rows is zero)
+    int rows_mn;
+    int64_t lda, ldb;
 };
 cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s);
 

@@ -252,21 +252,12 @@ cudaError_t launch_shared(const moe_config *c, const moe_shared_expert *sh, cons
 struct BwdLayout {
     size_t hist, logits, offsets, mt64, counts, ids, w, perm, inv, probs, lse, xs, dys, row_tok, row_e, row_w,
         pre, up, h, dh, dxs, dw, dz, doff, dmt, one, spre, sup, sh, sdh;
-    // bf16 path (tensor cores): 128-row tile prefix, padded column starts,
-    // transposed weights, the bf16 [da | du], transposed activations
-    size_t mt128, kpad, dacat, dysT, xsT, hwT, daT, duT, partial;
+    // bf16 path (tensor cores): 128-row tile prefix, the bf16 [da | du] and
+    // w h operands
+    size_t mt128, dacat, hwb, partial;
     // bf16 shared expert on the tensor cores: the same over one group of N rows
-    size_t smt128, skpad, sdcat, dyT, xT, shT, sdaT, sduT, total;
-    int64_t kp;   // columns of the transposed activations
-    int64_t skp;  // the same for the shared expert's N rows
+    size_t smt128, sdcat, shb, total;
 };
-
-// Columns of the transposed, per-expert padded activations: every expert's
-// rows rounded up to 64.
-int64_t bwd_kp(const moe_config *c)
-{
-    return (c->N * c->k + 64LL * c->E + 63) / 64 * 64;
-}
 
 BwdLayout bwd_layout(const moe_config *c)
 {
@@ -317,28 +308,14 @@ BwdLayout bwd_layout(const moe_config *c)
     L.sdh = take(Nn * Fs * 4);
     const bool tc = c->dtype == MOE_BF16;
     const size_t m = swiglu ? 2 : 1;
-    L.kp = bwd_kp(c);
-    const size_t kp = static_cast<size_t>(L.kp);
     L.mt128 = take((E + 1) * 4);
-    L.kpad = take((E + 1) * 4);
     L.dacat = take(tc ? A * m * F * 2 : 0);
-    L.dysT = take(tc ? d * kp * 2 : 0);
-    L.xsT = take(tc ? d * kp * 2 : 0);
-    L.hwT = take(tc ? F * kp * 2 : 0);
-    L.daT = take(tc ? F * kp * 2 : 0);
-    L.duT = take(tc && swiglu ? F * kp * 2 : 0);
+    L.hwb = take(tc ? A * F * 2 : 0);
     L.partial = take(static_cast<size_t>(kGenericPartialFloats) * 4);
     const bool stc = tc && Fs > 0;
-    L.skp = (c->N + 64 + 63) / 64 * 64;
-    const size_t skp = static_cast<size_t>(L.skp);
     L.smt128 = take(2 * 4);
-    L.skpad = take(2 * 4);
     L.sdcat = take(stc ? Nn * m * Fs * 2 : 0);
-    L.dyT = take(stc ? d * skp * 2 : 0);
-    L.xT = take(stc ? d * skp * 2 : 0);
-    L.shT = take(stc ? Fs * skp * 2 : 0);
-    L.sdaT = take(stc ? Fs * skp * 2 : 0);
-    L.sduT = take(stc && swiglu ? Fs * skp * 2 : 0);
+    L.shb = take(stc ? Nn * Fs * 2 : 0);
     L.total = o;
     return L;
 }
@@ -797,12 +774,13 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
         t.n_out = n_out; t.status = dev_status; t.accumulate = accumulate ? 1 : 0;
         return launch_gemm_tc_f32(t, sms, s);
     };
-    auto tc_sum_rows = [&](const void *A, int64_t m_total, const void *B, int n_out, float *C, const int32_t *kp_off,
-                           int G, int64_t cols) {
+    // C_g [m_total, n_out] = sum over rows off[g] .. off[g+1]-1 of A[r, :m_total]^T B[r, :n_out]
+    // (row-major A [nrows][lda], B [nrows][ldb], both read MN-major in place)
+    auto tc_sum_rows = [&](const void *A, int64_t lda, int64_t m_total, const void *B, int64_t ldb, int n_out, float *C,
+                           const int32_t *off, int G, int64_t nrows) {
         TcGemmArgs t{};
-        t.A = A; t.a_rows = static_cast<uint64_t>(m_total); t.a_cols = static_cast<uint64_t>(cols);
-        t.B = B; t.b_rows = static_cast<uint64_t>(n_out); t.b_cols = static_cast<uint64_t>(cols);
-        t.C = C; t.ldc = n_out; t.c_stride = m_total * n_out; t.offsets = kp_off; t.E = G; t.ragged_k = 1;
+        t.A = A; t.a_rows = static_cast<uint64_t>(nrows); t.lda = lda; t.B = B; t.ldb = ldb; t.rows_mn = 1;
+        t.C = C; t.ldc = n_out; t.c_stride = m_total * n_out; t.offsets = off; t.E = G; t.ragged_k = 1;
         t.n_out = n_out; t.m_total = m_total; t.status = dev_status;
         return launch_gemm_tc_f32(t, sms, s);
     };
@@ -821,46 +799,31 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
                    at<int32_t>(ws, L.row_e), row_w, dw, perm, dys, nullptr};
     const int m = swiglu ? 2 : 1;
     if (bf) {
-        // ---- bf16: every expert product on the tensor cores (fp32 results);
-        // dgrad with the weights read as MN-major operands in place, wgrad
-        // over transposed activations whose per-expert column blocks start
-        // at multiples of 64
-        int32_t *mt128 = at<int32_t>(ws, L.mt128), *kpad = at<int32_t>(ws, L.kpad);
-        auto *dacat = at<__nv_bfloat16>(ws, L.dacat);
-        auto *dysT = at<__nv_bfloat16>(ws, L.dysT), *xsT = at<__nv_bfloat16>(ws, L.xsT);
-        auto *hwT = at<__nv_bfloat16>(ws, L.hwT), *daT = at<__nv_bfloat16>(ws, L.daT);
-        auto *duT = swiglu ? at<__nv_bfloat16>(ws, L.duT) : nullptr;
-        const int64_t kp = L.kp;
+        // ---- bf16: every expert product on the tensor cores (fp32 results),
+        // every operand read in place: dgrad with the weights MN-major, wgrad
+        // over each expert's token rows of the activations (MN-major)
+        int32_t *mt128 = at<int32_t>(ws, L.mt128);
+        auto *dacat = at<__nv_bfloat16>(ws, L.dacat), *hwb = at<__nv_bfloat16>(ws, L.hwb);
         auto ragged_m = [&](const void *A, int64_t K, const void *B, int n_out, float *C) {
             return tc_rows(A, rows, K, B, n_out, C, offsets, mt128, E, false);
         };
-        auto ragged_k = [&](const void *A, int64_t m_total, const void *B, int n_out, float *C) {
-            return tc_sum_rows(A, m_total, B, n_out, C, kpad, E, kp);
-        };
         MOE_TRY(launch_tile_table(offsets, mt128, E, 128, s));
-        MOE_TRY(launch_pad_offsets(counts, kpad, E, s));
         MOE_TRY(ragged_m(xs, d, W1, F, pre));
         if (swiglu) MOE_TRY(ragged_m(xs, d, W3, F, up));
         MOE_TRY(launch_act_forward(act, sms, s));
         MOE_TRY(tc_rows_mn(dys, rows, W2, d, nullptr, 0, F, dh, offsets, mt128, E, false));  // dh = dy_s W2[e]
-        act.dcat = dacat;  // [da | du] in bf16 as well
+        act.dcat = dacat;  // [da | du] and w h in bf16; fp32 da only for db1
+        act.hw_bf = hwb;
+        act.skip_f32 = kSkipUp | kSkipH | ((!swiglu && b1 && gr.db1) ? 0 : kSkipPre);
         MOE_TRY(launch_row_backward(act, sms, s));
         // dx_s = [da | du] [W1[e] ; W3[e]]: one product with K = m F
         MOE_TRY(tc_rows_mn(dacat, rows, W1, F, swiglu ? W3 : nullptr, swiglu ? F : 0, d, dxs, offsets, mt128, E,
                            false));
-        // weight gradients over the transposed, padded activations
-        auto tr = [&](const void *src, int bf_in, int64_t ld_src, __nv_bfloat16 *dst, int C) {
-            TransposeRowsArgs t{src, bf_in, ld_src, dst, kp, C, E, offsets, kpad};
-            return launch_transpose_rows(t, kp, s);
-        };
-        MOE_TRY(tr(dys, 1, d, dysT, d));
-        MOE_TRY(tr(xs, 1, d, xsT, d));
-        MOE_TRY(tr(h, 0, F, hwT, F));
-        MOE_TRY(tr(dacat, 1, static_cast<int64_t>(m) * F, daT, F));
-        if (swiglu) MOE_TRY(tr(dacat + F, 1, 2LL * F, duT, F));
-        MOE_TRY(ragged_k(dysT, d, hwT, F, gr.dW2));   // dW2[e] = dy_s^T (w h)
-        MOE_TRY(ragged_k(daT, F, xsT, d, gr.dW1));    // dW1[e] = da^T x_s
-        if (swiglu) MOE_TRY(ragged_k(duT, F, xsT, d, gr.dW3));
+        // weight gradients, each expert over its own rows
+        const int64_t ldcat = static_cast<int64_t>(m) * F;
+        MOE_TRY(tc_sum_rows(dys, d, d, hwb, F, F, gr.dW2, offsets, E, rows));          // dW2[e] = dy_s^T (w h)
+        MOE_TRY(tc_sum_rows(dacat, ldcat, F, xs, d, d, gr.dW1, offsets, E, rows));     // dW1[e] = da^T x_s
+        if (swiglu) MOE_TRY(tc_sum_rows(dacat + F, ldcat, F, xs, d, d, gr.dW3, offsets, E, rows));
     } else {
         // ---- fp32: the same products on the CUDA cores
         MOE_TRY(GG().a(xs, d, 1, bf).b(W1, 1, d, static_cast<int64_t>(F) * d, bf).c(pre, F, 1, 0)
@@ -910,34 +873,23 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
         BwdActArgs sa{N, Fs, d, cfg->act, bf ? 1 : 0, spre, sup, sh, sdh, swiglu ? nullptr : shared->b1, nullptr,
                       nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
         if (bf) {  // tensor cores, one group of N rows
-            int32_t *smt = at<int32_t>(ws, L.smt128), *skpad = at<int32_t>(ws, L.skpad);
-            auto *sdcat = at<__nv_bfloat16>(ws, L.sdcat);
-            auto *dyT = at<__nv_bfloat16>(ws, L.dyT), *xT = at<__nv_bfloat16>(ws, L.xT);
-            auto *shT = at<__nv_bfloat16>(ws, L.shT), *sdaT = at<__nv_bfloat16>(ws, L.sdaT);
-            auto *sduT = swiglu ? at<__nv_bfloat16>(ws, L.sduT) : nullptr;
-            const int64_t skp = L.skp;
+            int32_t *smt = at<int32_t>(ws, L.smt128);
+            auto *sdcat = at<__nv_bfloat16>(ws, L.sdcat), *shb = at<__nv_bfloat16>(ws, L.shb);
             MOE_TRY(launch_tile_table(doff, smt, 1, 128, s));
-            MOE_TRY(launch_pad_offsets(doff + 1, skpad, 1, s));  // the one group's count is N
             MOE_TRY(tc_rows(x, N, d, shared->W1, Fs, spre, doff, smt, 1, false));
             if (swiglu) MOE_TRY(tc_rows(x, N, d, shared->W3, Fs, sup, doff, smt, 1, false));
             MOE_TRY(launch_act_forward(sa, sms, s));
             MOE_TRY(tc_rows_mn(dy, N, shared->W2, d, nullptr, 0, Fs, sdh, doff, smt, 1, false));
             sa.dcat = sdcat;
+            sa.hw_bf = shb;
+            sa.skip_f32 = kSkipUp | kSkipH | ((!swiglu && shared->b1 && gr.dbs1) ? 0 : kSkipPre);
             MOE_TRY(launch_row_backward(sa, sms, s));
             MOE_TRY(tc_rows_mn(sdcat, N, shared->W1, Fs, swiglu ? shared->W3 : nullptr, swiglu ? Fs : 0, d, gr.dx,
                                doff, smt, 1, true));
-            auto tr = [&](const void *src, int bf_in, int64_t ld_src, __nv_bfloat16 *dst, int C) {
-                TransposeRowsArgs t{src, bf_in, ld_src, dst, skp, C, 1, doff, skpad};
-                return launch_transpose_rows(t, skp, s);
-            };
-            MOE_TRY(tr(dy, 1, d, dyT, d));
-            MOE_TRY(tr(x, 1, d, xT, d));
-            MOE_TRY(tr(sh, 0, Fs, shT, Fs));
-            MOE_TRY(tr(sdcat, 1, static_cast<int64_t>(m) * Fs, sdaT, Fs));
-            if (swiglu) MOE_TRY(tr(sdcat + Fs, 1, 2LL * Fs, sduT, Fs));
-            MOE_TRY(tc_sum_rows(dyT, d, shT, Fs, gr.dWs2, skpad, 1, skp));
-            MOE_TRY(tc_sum_rows(sdaT, Fs, xT, d, gr.dWs1, skpad, 1, skp));
-            if (swiglu) MOE_TRY(tc_sum_rows(sduT, Fs, xT, d, gr.dWs3, skpad, 1, skp));
+            const int64_t ldcat = static_cast<int64_t>(m) * Fs;
+            MOE_TRY(tc_sum_rows(dy, d, d, shb, Fs, Fs, gr.dWs2, doff, 1, N));
+            MOE_TRY(tc_sum_rows(sdcat, ldcat, Fs, x, d, d, gr.dWs1, doff, 1, N));
+            if (swiglu) MOE_TRY(tc_sum_rows(sdcat + Fs, ldcat, Fs, x, d, d, gr.dWs3, doff, 1, N));
         } else {
             MOE_TRY(GG().a(x, d, 1, bf).b(shared->W1, 1, d, 0, bf).c(spre, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
             if (swiglu)

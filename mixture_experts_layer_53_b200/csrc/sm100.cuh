@@ -323,8 +323,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N)
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// The same with B MN-major (bit 16 set).
+// The same with B MN-major (bit 16 set), and with A and B MN-major (bits 15
+// and 16 set).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) { return idesc_bf16_f32(M, N) | (1u << 16); }
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_mn(int M, int N)
+{
+    return idesc_bf16_f32(M, N) | (1u << 15) | (1u << 16);
+}
+
+// Orders this thread's generic-proxy writes to shared memory before later
+// async-proxy reads of it (tcgen05.mma operands, TMA stores).
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 }  // namespace sm100
 }  // namespace moe
