@@ -98,7 +98,12 @@ struct Ctl {
     int abort;
     int off[kMaxE + 1];
     int mt[kMaxE + 1];
+    // EPI_F32: per epilogue warp, a 32 x 32 fp32 chunk of its rows on the
+    // way from TMEM (one row per lane) to global memory (whole 128-B rows);
+    // rows padded to 36 floats so both sides are free of bank conflicts
+    alignas(16) float stage[4][32][36];
 };
+static_assert(1024 + STAGES * STAGE_BYTES + sizeof(Ctl) <= 232448, "shared memory per CTA");
 
 constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(Ctl);
 
@@ -132,39 +137,54 @@ __device__ __forceinline__ Tile tile_of(int t, const Ctl *c, const GemmArgs &g)
     return Tile{e, local % g.m_tiles, local / g.m_tiles};
 }
 
+// The warp's rows are row_first .. row_first + 31 (lane l holds TMEM lane
+// row_first + l); rows from row_end on are not stored.
 template <int EPI>
-__device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase, int e, int row,
-                                              bool row_ok, int n0, bool zero = false)
+__device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase, int e, int row_first,
+                                              int64_t row_end, int n0, float (*stage)[36], bool zero = false)
 {
+    const int lane = threadIdx.x & 31;
     if constexpr (EPI == EPI_F32) {
-        // zero: the expert had no rows (no MMA wrote the accumulator)
-        float *orow = g.out_f32 + (g.ragged_k ? static_cast<int64_t>(e) * g.c_stride : 0) +
-                      static_cast<int64_t>(row) * g.ldo;
+        // zero: the expert had no rows (no MMA wrote the accumulator).
+        // Each 32-column chunk goes through `stage`: lane l writes its row,
+        // then lanes 8j .. 8j+7 store 128 B of row 4q + j (q = 0..7).
+        float *out = g.out_f32 + (g.ragged_k ? static_cast<int64_t>(e) * g.c_stride : 0);
+        const int sub = lane >> 3, cq = (lane & 7) * 4;
 #pragma unroll 1
         for (int c = 0; c < 256; c += 32) {
             uint32_t acc[32];
             tmem_ld32(tbase + c, acc);
             tmem_ld_wait();
-            if (row_ok) {
 #pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    const int col = n0 + c + v * 4;
-                    if (col < g.n_out) {  // n_out is a multiple of 4 (16-byte stores)
-                        float4 q = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
-                                        : make_float4(__uint_as_float(acc[4 * v]), __uint_as_float(acc[4 * v + 1]),
-                                                      __uint_as_float(acc[4 * v + 2]),
-                                                      __uint_as_float(acc[4 * v + 3]));
+            for (int v = 0; v < 8; ++v)
+                *reinterpret_cast<float4 *>(&stage[lane][4 * v]) =
+                    zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                         : make_float4(__uint_as_float(acc[4 * v]), __uint_as_float(acc[4 * v + 1]),
+                                       __uint_as_float(acc[4 * v + 2]), __uint_as_float(acc[4 * v + 3]));
+            __syncwarp();
+            const int col = n0 + c + cq;
+            if (col < g.n_out) {  // n_out is a multiple of 4 (16-byte stores)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int r = 4 * q + sub;
+                    const int64_t row = static_cast<int64_t>(row_first) + r;
+                    if (row < row_end) {
+                        float4 v4 = *reinterpret_cast<const float4 *>(&stage[r][cq]);
+                        float *dst = out + row * g.ldo + col;
                         if (g.accumulate) {
-                            const float4 o = *reinterpret_cast<const float4 *>(orow + col);
-                            q.x += o.x; q.y += o.y; q.z += o.z; q.w += o.w;
+                            const float4 o = *reinterpret_cast<const float4 *>(dst);
+                            v4.x += o.x; v4.y += o.y; v4.z += o.z; v4.w += o.w;
                         }
-                        *reinterpret_cast<float4 *>(orow + col) = q;
+                        *reinterpret_cast<float4 *>(dst) = v4;
                     }
                 }
             }
+            __syncwarp();
         }
         return;
     }
+    const int row = row_first + lane;
+    const bool row_ok = row < row_end;
     __nv_bfloat16 *orow = g.out + static_cast<int64_t>(row) * g.ldo;
     const __nv_bfloat16 *brow = g.bias ? g.bias + static_cast<int64_t>(e) * g.n_out : nullptr;
 #pragma unroll 1
@@ -440,7 +460,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else {
         // ---------------------------------------------------- epilogue
         const int quarter = warp & 3;  // TMEM lanes this warp may access
-        const int row_in_tile = quarter * 32 + lane;
         int buf = 0;
         uint32_t tphase = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
@@ -448,18 +467,19 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!ok) break;
             tc_fence_after();
             const Tile ti = tile_of(t, ctl, g);
-            int row;
-            bool row_ok;
+            int row_first;  // the warp's first row
+            int64_t row_end;
             if (g.ragged_k) {  // result row m of expert e
-                row = ti.m_tile * BM + row_in_tile;
-                row_ok = row < g.m_total;
+                row_first = ti.m_tile * BM + quarter * 32;
+                row_end = g.m_total;
             } else {
-                row = ctl->off[ti.e] + ti.m_tile * BM + row_in_tile;
-                row_ok = row < ctl->off[ti.e + 1];
+                row_first = ctl->off[ti.e] + ti.m_tile * BM + quarter * 32;
+                row_end = ctl->off[ti.e + 1];
             }
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
-            epilogue_tile<EPI>(g, tbase, ti.e, row, row_ok, ti.n_tile * out_cols<EPI>(), kblocks(ti.e) == 0);
+            epilogue_tile<EPI>(g, tbase, ti.e, row_first, row_end, ti.n_tile * out_cols<EPI>(), ctl->stage[quarter],
+                               kblocks(ti.e) == 0);
             tc_fence_before();
             mbar_arrive(&ctl->tempty[buf]);
             if (++buf == 2) {
