@@ -323,7 +323,8 @@ MOE_API moe_status moe_forward_ex(const moe_config *cfg, const void *x, const vo
 
 /*
  * Gradients written by moe_backward: fp32, row-major, caller-owned device
- * memory, each overwritten (not accumulated).  Shapes as the parameters:
+ * memory, 16-byte aligned (else MOE_ERR_INVALID_ARG), each overwritten (not
+ * accumulated).  Shapes as the parameters:
  * dx [N, d_model], dW_g [E, d_model], dW1 / dW3 [E, d_ff, d_model],
  * db1 [E, d_ff], dW2 [E, d_model, d_ff], db2 [E, d_model]; the shared
  * expert's dWs1 / dWs3 [d_ff_shared, d_model], dbs1 [d_ff_shared],

@@ -89,6 +89,12 @@ struct GemmArgs {
 };
 
 struct Ctl {
+    // EPI_F32: per epilogue warp, a 32 x 32 fp32 chunk of its rows on the
+    // way from TMEM (one row per lane) to global memory.  Ragged M: rows
+    // padded to 36 floats (no bank conflicts) and stored back by the lanes in
+    // whole 128-B rows; OPS_MN_MN: 4 KB per warp in the 128-byte swizzled
+    // layout of a TMA store box (also free of bank conflicts).
+    alignas(1024) float stage[4][32][36];
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t tfull[2];
@@ -98,11 +104,8 @@ struct Ctl {
     int abort;
     int off[kMaxE + 1];
     int mt[kMaxE + 1];
-    // EPI_F32: per epilogue warp, a 32 x 32 fp32 chunk of its rows on the
-    // way from TMEM (one row per lane) to global memory (whole 128-B rows);
-    // rows padded to 36 floats so both sides are free of bank conflicts
-    alignas(16) float stage[4][32][36];
 };
+static_assert(sizeof(float) * 4 * 32 * 36 >= 4 * 4096, "TMA store staging fits");
 static_assert(1024 + STAGES * STAGE_BYTES + sizeof(Ctl) <= 232448, "shared memory per CTA");
 
 constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(Ctl);
@@ -237,11 +240,46 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase,
     }
 }
 
+// EPI_F32 with OPS_MN_MN: expert e's [m_total, n_out] result goes out
+// through TMA stores of 32 x 32 boxes (tm_out = {n_out, m_total, E}, clipped
+// at the edges), so the short per-expert reductions of the weight gradients
+// are not held up by thread stores.  buf: this warp's 4 KB, 1024-aligned.
+__device__ __forceinline__ void epilogue_tile_tma(const GemmArgs &g, const CUtensorMap *tm_out, uint32_t tbase,
+                                                  int e, int row_first, int n0, uint8_t *buf, bool zero)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll 1
+    for (int c = 0; c < 256; c += 32) {
+        uint32_t acc[32];
+        tmem_ld32(tbase + c, acc);
+        tmem_ld_wait();
+        const int col = n0 + c;
+        if (row_first >= g.m_total || col >= g.n_out) continue;  // warp-uniform: nothing to store
+        if (lane == 0) bulk_wait_read_all();  // the previous store has read buf
+        __syncwarp();
+        // row `lane`; its 16-B piece j sits at piece j ^ (lane & 7) of the row
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4 *>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                     : make_float4(__uint_as_float(acc[4 * j]), __uint_as_float(acc[4 * j + 1]),
+                                   __uint_as_float(acc[4 * j + 2]), __uint_as_float(acc[4 * j + 3]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_3d(tm_out, buf, col, row_first, e);
+            bulk_commit();
+        }
+    }
+}
+
 // MN-major operand tiles (OPS_K_MN, OPS_MN_MN; EPI_F32 only) are 64-column
 // x 64-row boxes 8 KB apart, so the backward's products against W^T and
 // over token rows need no transposed copies.  In OPS_MN_MN the last k-block
 // of an expert can hold rows of the next one: the MMA warp zeroes those rows
 // of both tiles in shared memory before the MMA reads them.
+// The third tensor map is W3 (SwiGLU), the second B (OPS_K_MN) or the fp32
+// result (OPS_MN_MN).
 template <int EPI, int OPS = OPS_KK>
 __global__ void __launch_bounds__(THREADS, 1)
     ffn_gemm_single_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -271,7 +309,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (threadIdx.x == 32) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
-        if (EPI == EPI_SWIGLU || OPS == OPS_K_MN) prefetch_tmap(&tmB3);
+        if (EPI == EPI_SWIGLU || OPS != OPS_KK) prefetch_tmap(&tmB3);
     }
     if (warp == 1) {
         tmem_alloc(&ctl->tmem_base, TMEM_COLS);
@@ -478,8 +516,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
-            epilogue_tile<EPI>(g, tbase, ti.e, row_first, row_end, ti.n_tile * out_cols<EPI>(), ctl->stage[quarter],
-                               kblocks(ti.e) == 0);
+            if constexpr (EPI == EPI_F32 && OPS == OPS_MN_MN)
+                epilogue_tile_tma(g, &tmB3, tbase, ti.e, row_first, ti.n_tile * BN,
+                                  reinterpret_cast<uint8_t *>(ctl->stage) + quarter * 4096, kblocks(ti.e) == 0);
+            else
+                epilogue_tile<EPI>(g, tbase, ti.e, row_first, row_end, ti.n_tile * out_cols<EPI>(),
+                                   ctl->stage[quarter], kblocks(ti.e) == 0);
             tc_fence_before();
             mbar_arrive(&ctl->tempty[buf]);
             if (++buf == 2) {
@@ -487,6 +529,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tphase ^= 1u;
             }
         }
+        // the staging buffers stay valid until this warp's stores are done
+        if (EPI == EPI_F32 && OPS == OPS_MN_MN && lane == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -522,11 +566,16 @@ cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s)
         if (!t.ragged_k || t.b_mn || t.lda % 8 != 0 || t.ldb % 8 != 0 || t.m_total % 8 != 0 || t.n_out % 8 != 0 ||
             t.m_total > t.lda || t.n_out > t.ldb)
             return cudaErrorInvalidValue;
-        CUtensorMap tA, tB;
+        // the result goes out through TMA stores: [E][m_total][n_out], 16-byte aligned
+        if (t.ldc != t.n_out || t.c_stride != t.m_total * t.n_out || (reinterpret_cast<uintptr_t>(t.C) & 15u) != 0)
+            return cudaErrorInvalidValue;
+        CUtensorMap tA, tB, tOut;
         if (!make_tmap_bf16_mn_rows(&tA, t.A, static_cast<uint64_t>(t.m_total), t.a_rows,
                                     static_cast<uint64_t>(t.lda)) ||
             !make_tmap_bf16_mn_rows(&tB, t.B, static_cast<uint64_t>(t.n_out), t.a_rows,
-                                    static_cast<uint64_t>(t.ldb)))
+                                    static_cast<uint64_t>(t.ldb)) ||
+            !make_tmap_f32_store(&tOut, t.C, static_cast<uint64_t>(t.n_out), static_cast<uint64_t>(t.m_total),
+                                 static_cast<uint64_t>(t.E)))
             return cudaErrorInvalidValue;
         GemmArgs g{};
         g.offsets = t.offsets;
@@ -541,7 +590,7 @@ cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s)
         g.m_total = t.m_total;
         g.c_stride = t.c_stride;
         g.accumulate = t.accumulate;
-        return launch_gemm<EPI_F32, OPS_MN_MN>(tA, tB, tB, g, num_sms, s);
+        return launch_gemm<EPI_F32, OPS_MN_MN>(tA, tB, tOut, g, num_sms, s);
     }
     CUtensorMap tA, tB, tB3;
     if (!make_tmap_bf16(&tA, t.A, t.a_cols, t.a_rows, BM)) return cudaErrorInvalidValue;

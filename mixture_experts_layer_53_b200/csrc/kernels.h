@@ -261,6 +261,7 @@ namespace moe {
 bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_outer);
 bool make_tmap_bf16_mn(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t groups);
 bool make_tmap_bf16_mn_rows(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t ld);
+bool make_tmap_f32_store(CUtensorMap *m, void *base, uint64_t inner, uint64_t rows, uint64_t groups);
 
 // C (fp32) = A B^T on tcgen05 with bf16 operands, both K-major (the
 // backward's products on the tensor cores), 128 x 256 tiles:

@@ -372,6 +372,11 @@ moe_status check_grads(const moe_config *c, const moe_grads *gr, bool shared)
     if (!gr || (c->N > 0 && !gr->dx) || !gr->dW_g || !gr->dW1 || !gr->dW2) return MOE_ERR_INVALID_ARG;
     if (c->act == MOE_ACT_SWIGLU && !gr->dW3) return MOE_ERR_INVALID_ARG;
     if (shared && (!gr->dWs1 || !gr->dWs2 || (c->act == MOE_ACT_SWIGLU && !gr->dWs3))) return MOE_ERR_INVALID_ARG;
+    // the gradient kernels store 16-byte vectors (and the tensor-core
+    // weight gradients go out through TMA stores)
+    for (const float *p : {gr->dx, gr->dW_g, gr->dW1, gr->db1, gr->dW3, gr->dW2, gr->db2, gr->dWs1, gr->dbs1,
+                           gr->dWs3, gr->dWs2, gr->dbs2})
+        if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
 
