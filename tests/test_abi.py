@@ -228,6 +228,8 @@ def test_backward_validation(lib):
     assert lib.moe_backward(*args(None)) == 1            # no gradient struct
     assert lib.moe_backward(*args(full, dy=None)) == 1   # dy missing
     assert lib.moe_backward(*args(full, aux=float("inf"))) == 1
+    misaligned = M.MoeGrads(*([0x20000] * 5 + [0x20004] + [0x20000] * 6))  # dW2 off a 16-byte boundary
+    assert lib.moe_backward(*args(misaligned)) == 1
     small = ctypes.c_size_t(lib.moe_workspace_size(ctypes.byref(c)))
     assert lib.moe_backward(ctypes.byref(c), a, a, None, a, None, a, a, None, None, a, ctypes.c_float(0.0),
                             ctypes.c_float(0.0), ctypes.byref(full), None, ws, small, None) == 4
