@@ -37,6 +37,7 @@
 #include "common.cuh"
 #include "host_util.h"
 #include "kernels.h"
+#include "epilogue_f32.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -148,42 +149,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase,
 {
     const int lane = threadIdx.x & 31;
     if constexpr (EPI == EPI_F32) {
-        // zero: the expert had no rows (no MMA wrote the accumulator).
-        // Each 32-column chunk goes through `stage`: lane l writes its row,
-        // then lanes 8j .. 8j+7 store 128 B of row 4q + j (q = 0..7).
         float *out = g.out_f32 + (g.ragged_k ? static_cast<int64_t>(e) * g.c_stride : 0);
-        const int sub = lane >> 3, cq = (lane & 7) * 4;
-#pragma unroll 1
-        for (int c = 0; c < 256; c += 32) {
-            uint32_t acc[32];
-            tmem_ld32(tbase + c, acc);
-            tmem_ld_wait();
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-                *reinterpret_cast<float4 *>(&stage[lane][4 * v]) =
-                    zero ? make_float4(0.f, 0.f, 0.f, 0.f)
-                         : make_float4(__uint_as_float(acc[4 * v]), __uint_as_float(acc[4 * v + 1]),
-                                       __uint_as_float(acc[4 * v + 2]), __uint_as_float(acc[4 * v + 3]));
-            __syncwarp();
-            const int col = n0 + c + cq;
-            if (col < g.n_out) {  // n_out is a multiple of 4 (16-byte stores)
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int r = 4 * q + sub;
-                    const int64_t row = static_cast<int64_t>(row_first) + r;
-                    if (row < row_end) {
-                        float4 v4 = *reinterpret_cast<const float4 *>(&stage[r][cq]);
-                        float *dst = out + row * g.ldo + col;
-                        if (g.accumulate) {
-                            const float4 o = *reinterpret_cast<const float4 *>(dst);
-                            v4.x += o.x; v4.y += o.y; v4.z += o.z; v4.w += o.w;
-                        }
-                        *reinterpret_cast<float4 *>(dst) = v4;
-                    }
-                }
-            }
-            __syncwarp();
-        }
+        epilogue_f32_rows(out, g.ldo, g.n_out, tbase, row_first, row_end, n0, stage, zero, g.accumulate != 0);
         return;
     }
     const int row = row_first + lane;

@@ -30,9 +30,16 @@
 // SwiGLU: the even CTA's B half holds 128 rows of W1 and the odd CTA's the
 // same 128 rows of W3, so accumulator columns 0..127 are the gate and
 // 128..255 the up projection of 128 hidden units.
+//
+// The backward's ragged-M products use the same kernel with fp32 results
+// (EPI_F32): the recomputed pre-activations x_s W1[e]^T (K-major B) and the
+// dgrad products dy_s W2[e], [da | du] [W1[e]; W3[e]] (OPS_K_MN: each CTA
+// loads its 128 result columns of the [E][K][n_out] weights as two 64 x 64
+// MN-major boxes, so no transposed copy of the weights is made).
 #include <cuda.h>
 
 #include "common.cuh"
+#include "epilogue_f32.cuh"
 #include "host_util.h"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -59,7 +66,9 @@ template <int EPI> __host__ __device__ constexpr int threads_of() { return 64 + 
 constexpr uint32_t TMEM_COLS = 512;
 
 
-enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_LINEAR = 2 };
+enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_LINEAR = 2, EPI_F32 = 3 };
+enum { OPS_KK = 0, OPS_K_MN = 1 };  // B K-major / MN-major (A K-major in both)
+constexpr int BOX_BYTES = 64 * 64 * 2;  // one 64 x 64 MN-major box
 template <int EPI> __host__ __device__ constexpr int epi_warps() { return EPI == EPI_GELU ? 8 : 4; }
 
 struct GemmArgs {
@@ -70,9 +79,17 @@ struct GemmArgs {
     const __nv_bfloat16 *bias;  // [E, n_out] or null
     int32_t *status;
     int E, K, n_out, n_tiles, b_rows;
+    float *out_f32;  // EPI_F32: the result, ldo floats per row
+    int accumulate;  // EPI_F32: add to the existing result
+    // OPS_K_MN: k-blocks 0..kb1-1 read tmB rows kb * BK of expert e with A
+    // columns kb * BK; k-blocks kb1..kb_total-1 read tmB3 with A columns
+    // a_col2 + (kb - kb1) * BK
+    int kb1, kb_total, a_col2;
 };
 
 struct Ctl {
+    // EPI_F32: per epilogue warp, a 32 x 32 chunk on its way to global memory
+    alignas(1024) float stage[4][32][36];
     uint64_t full[STAGES];   // used in the even CTA: both CTAs' bytes
     uint64_t empty[STAGES];  // each CTA: arrived by the even CTA's commit
     uint64_t tfull[2];       // each CTA: arrived by the even CTA's commit
@@ -85,6 +102,7 @@ struct Ctl {
 };
 
 constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(Ctl);
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 struct Tile {
     int e, m_tile, n_tile;
@@ -163,7 +181,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &g, uint32_t tbase,
     }
 }
 
-template <int EPI>
+template <int EPI, int OPS = OPS_KK>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmB3, const GemmArgs g)
@@ -194,7 +212,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
     if (threadIdx.x == 32) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
-        if (EPI == EPI_SWIGLU) prefetch_tmap(&tmB3);
+        if (EPI == EPI_SWIGLU || OPS == OPS_K_MN) prefetch_tmap(&tmB3);
     }
     if (warp == 1) {
         tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
@@ -211,7 +229,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
 
     const uint32_t tmem_base = ctl->tmem_base;
     const int total = ctl->mt[g.E] * g.n_tiles;
-    const int num_kb = (g.K + BK - 1) / BK;
+    const int num_kb = OPS == OPS_K_MN ? g.kb_total : (g.K + BK - 1) / BK;
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (warp == 0) {
@@ -232,6 +250,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                     brow = ti.e * g.b_rows + ti.n_tile * BN + static_cast<int>(rank) * (BN / 2);
                     tb = &tmB;
                 }
+                // OPS_K_MN: this CTA's 128 result columns as two boxes; boxes
+                // wholly past n_out are not loaded (their columns are never
+                // stored), and the even CTA expects both CTAs' bytes
+                const int nc0 = ti.n_tile * BN + static_cast<int>(rank) * (BN / 2);
+                auto boxes_of = [&](int r) {
+                    const int left = g.n_out - (ti.n_tile * BN + r * (BN / 2));
+                    return left <= 0 ? 0 : min(2, (left + 63) / 64);
+                };
+                const int my_boxes = boxes_of(static_cast<int>(rank));
+                const uint32_t pair_bytes = OPS == OPS_K_MN
+                                                ? 2u * A_BYTES + static_cast<uint32_t>(boxes_of(0) + boxes_of(1)) * BOX_BYTES
+                                                : 2u * STAGE_BYTES;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort_flag, g.status)) {
                         ok = false;
@@ -239,6 +269,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                     }
                     uint8_t *sA = tiles + stage * STAGE_BYTES;
                     const uint32_t full_leader = mapa_shared(smem_u32(&ctl->full[stage]), 0);
+                    if constexpr (OPS == OPS_K_MN) {
+                        if (leader) {
+                            mbar_arrive_expect_tx(&ctl->full[stage], pair_bytes);
+                            armed |= 1u << stage;
+                            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                        }
+                        const bool second = kb >= g.kb1;
+                        const int kk0 = (second ? kb - g.kb1 : kb) * BK;
+                        tma_load_2d_pair(sA, &tmA, full_leader, (second ? g.a_col2 : 0) + kk0, row0);
+                        const CUtensorMap *mb = second ? &tmB3 : &tmB;
+                        for (int c = 0; c < my_boxes; ++c)
+                            tma_load_3d_pair(sA + A_BYTES + c * BOX_BYTES, mb, full_leader, nc0 + c * 64, kk0, ti.e);
+                        if (++stage == STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                        continue;
+                    }
                     if (leader) {
                         mbar_arrive_expect_tx(&ctl->full[stage], 2 * STAGE_BYTES);
                         armed |= 1u << stage;
@@ -262,7 +310,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc = idesc_bf16_f32(PAIR_M, BN);
+            constexpr uint32_t idesc = OPS == OPS_K_MN ? idesc_bf16_f32_bmn(PAIR_M, BN) : idesc_bf16_f32(PAIR_M, BN);
             int stage = 0, buf = 0;
             uint32_t phase = 0, tphase = 0;
             bool ok = true, issued = false;
@@ -279,9 +327,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                     const uint32_t a_addr = smem_u32(tiles + stage * STAGE_BYTES);
                     const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        umma_bf16_pair(d_tmem, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32), idesc,
-                                       (kb | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        // MN-major B: 16 K rows are two whole swizzle atoms;
+                        // each CTA's 128 columns are two chunks BOX_BYTES apart
+                        const uint64_t bd = OPS == OPS_K_MN ? desc_sw128_mn(b_addr + kk * 2048, BOX_BYTES)
+                                                            : desc_sw128(b_addr + kk * 32);
+                        umma_bf16_pair(d_tmem, desc_sw128(a_addr + kk * 32), bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
                     issued = true;
                     umma_commit_pair(&ctl->empty[stage], 0x3);
                     if (++stage == STAGES) {
@@ -320,8 +372,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             const bool row_ok = row < ctl->off[ti.e + 1];
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
-            epilogue_rows<EPI>(g, tbase, ti.e, row, row_ok, ti.n_tile * out_cols<EPI>(),
-                               part * out_cols<EPI>() / parts, (part + 1) * out_cols<EPI>() / parts);
+            if constexpr (EPI == EPI_F32)
+                epilogue_f32_rows(g.out_f32, g.ldo, g.n_out, tbase, row - lane, ctl->off[ti.e + 1], ti.n_tile * BN,
+                                  ctl->stage[quarter], false, g.accumulate != 0);
+            else
+                epilogue_rows<EPI>(g, tbase, ti.e, row, row_ok, ti.n_tile * out_cols<EPI>(),
+                                   part * out_cols<EPI>() / parts, (part + 1) * out_cols<EPI>() / parts);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
@@ -342,18 +398,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
     }
 }
 
-template <int EPI>
+template <int EPI, int OPS = OPS_KK>
 cudaError_t launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b3, const GemmArgs &g,
                         int num_sms, cudaStream_t s)
 {
-    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&ffn_gemm_pair_kernel<EPI>),
+    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&ffn_gemm_pair_kernel<EPI, OPS>),
                                        static_cast<int>(kSmemBytes));
     if (err != cudaSuccess) return err;
     const int grid = (num_sms / 2) * 2;
-    return launch_k(ffn_gemm_pair_kernel<EPI>, dim3(grid), dim3(threads_of<EPI>()), kSmemBytes, s, a, b, b3, g);
+    return launch_k(ffn_gemm_pair_kernel<EPI, OPS>, dim3(grid), dim3(threads_of<EPI>()), kSmemBytes, s, a, b, b3,
+                    g);
 }
 
 }  // namespace
+
+cudaError_t launch_gemm_tc_f32_pair(const TcGemmArgs &t, int num_sms, cudaStream_t s)
+{
+    if (t.ragged_k || t.rows_mn) return cudaErrorInvalidValue;  // ragged M only
+    if (t.a_rows == 0 || t.n_out == 0) return cudaSuccess;
+    if (t.b_mn && (t.k1 <= 0 || t.k2 < 0 || (t.k2 > 0) != (t.B2 != nullptr) ||
+                   static_cast<uint64_t>(t.k1 + t.k2) != t.a_cols || t.k1 % 8 != 0 || t.n_out % 8 != 0))
+        return cudaErrorInvalidValue;  // A's second column block must start on a 16-byte boundary
+    CUtensorMap tA, tB, tB3;
+    if (!make_tmap_bf16(&tA, t.A, t.a_cols, t.a_rows, BM)) return cudaErrorInvalidValue;
+    if (t.b_mn) {
+        const uint64_t n = static_cast<uint64_t>(t.n_out), G = static_cast<uint64_t>(t.E);
+        if (!make_tmap_bf16_mn(&tB, t.B, n, static_cast<uint64_t>(t.k1), G) ||
+            !make_tmap_bf16_mn(&tB3, t.B2 ? t.B2 : t.B, n, static_cast<uint64_t>(t.B2 ? t.k2 : t.k1), G))
+            return cudaErrorInvalidValue;
+    } else if (!make_tmap_bf16(&tB, t.B, t.b_cols, t.b_rows, 128)) {
+        return cudaErrorInvalidValue;
+    }
+    GemmArgs g{};
+    g.offsets = t.offsets;
+    g.mt_prefix = t.mt_prefix;
+    g.out_f32 = t.C;
+    g.ldo = t.ldc;
+    g.status = t.status;
+    g.E = t.E;
+    g.K = t.K;
+    g.n_out = t.n_out;
+    g.n_tiles = (t.n_out + BN - 1) / BN;
+    g.b_rows = t.n_out;
+    g.accumulate = t.accumulate;
+    if (t.b_mn) {
+        g.kb1 = static_cast<int>((t.k1 + BK - 1) / BK);
+        g.kb_total = g.kb1 + static_cast<int>((t.k2 + BK - 1) / BK);
+        g.a_col2 = static_cast<int>(t.k1);
+        return launch_pair<EPI_F32, OPS_K_MN>(tA, tB, tB3, g, num_sms, s);
+    }
+    return launch_pair<EPI_F32>(tA, tB, tB, g, num_sms, s);
+}
 
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid, cudaStream_t s)
 {

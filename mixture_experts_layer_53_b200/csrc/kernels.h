@@ -298,6 +298,9 @@ struct TcGemmArgs {
     int64_t lda, ldb;
 };
 cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s);
+// The same on CTA pairs (256 x 256 tiles) for ragged-M products; mt_prefix
+// must count 256-row tiles.
+cudaError_t launch_gemm_tc_f32_pair(const TcGemmArgs &t, int num_sms, cudaStream_t s);
 
 // Both expert GEMMs; `mid` (may be null) is recorded between them.
 // CTA pairs, 256-row m-tiles:

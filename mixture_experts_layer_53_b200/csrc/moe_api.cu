@@ -252,11 +252,11 @@ cudaError_t launch_shared(const moe_config *c, const moe_shared_expert *sh, cons
 struct BwdLayout {
     size_t hist, logits, offsets, mt64, counts, ids, w, perm, inv, probs, lse, xs, dys, row_tok, row_e, row_w,
         pre, up, h, dh, dxs, dw, dz, doff, dmt, one, spre, sup, sh, sdh;
-    // bf16 path (tensor cores): 128-row tile prefix, the bf16 [da | du] and
-    // w h operands
-    size_t mt128, dacat, hwb, partial;
+    // bf16 path (tensor cores): 128- or 256-row tile prefix, the bf16
+    // [da | du] and w h operands
+    size_t mtc, dacat, hwb, partial;
     // bf16 shared expert on the tensor cores: the same over one group of N rows
-    size_t smt128, sdcat, shb, total;
+    size_t smtc, sdcat, shb, total;
 };
 
 BwdLayout bwd_layout(const moe_config *c)
@@ -308,12 +308,12 @@ BwdLayout bwd_layout(const moe_config *c)
     L.sdh = take(Nn * Fs * 4);
     const bool tc = c->dtype == MOE_BF16;
     const size_t m = swiglu ? 2 : 1;
-    L.mt128 = take((E + 1) * 4);
+    L.mtc = take((E + 1) * 4);
     L.dacat = take(tc ? A * m * F * 2 : 0);
     L.hwb = take(tc ? A * F * 2 : 0);
     L.partial = take(static_cast<size_t>(kGenericPartialFloats) * 4);
     const bool stc = tc && Fs > 0;
-    L.smt128 = take(2 * 4);
+    L.smtc = take(2 * 4);
     L.sdcat = take(stc ? Nn * m * Fs * 2 : 0);
     L.shb = take(stc ? Nn * Fs * 2 : 0);
     L.total = o;
@@ -770,14 +770,19 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
     // tensor-core products: rows offsets[g] .. of A and C per group (B per
     // group n_out rows of K), or (tc_sum_rows) per group a sum over the
     // group's padded columns of A [m_total, cols] and B [n_out, cols]
+    // (ragged M: CTA pairs with 256-row tiles where the groups average more
+    // than 192 rows, as in the forward; the tile prefix mt_ counts tile_m rows)
+    auto tc_launch = [&](const TcGemmArgs &t, int tile_m) {
+        return tile_m == 256 ? launch_gemm_tc_f32_pair(t, sms, s) : launch_gemm_tc_f32(t, sms, s);
+    };
     auto tc_rows = [&](const void *A, int64_t nrows, int64_t K, const void *B, int n_out, float *C,
-                       const int32_t *off, const int32_t *mt_, int G, bool accumulate) {
+                       const int32_t *off, const int32_t *mt_, int tile_m, int G, bool accumulate) {
         TcGemmArgs t{};
         t.A = A; t.a_rows = static_cast<uint64_t>(nrows); t.a_cols = static_cast<uint64_t>(K);
         t.B = B; t.b_rows = static_cast<uint64_t>(G) * n_out; t.b_cols = static_cast<uint64_t>(K);
         t.C = C; t.ldc = n_out; t.offsets = off; t.mt_prefix = mt_; t.E = G; t.K = static_cast<int>(K);
         t.n_out = n_out; t.status = dev_status; t.accumulate = accumulate ? 1 : 0;
-        return launch_gemm_tc_f32(t, sms, s);
+        return tc_launch(t, tile_m);
     };
     // C_g [m_total, n_out] = sum over rows off[g] .. off[g+1]-1 of A[r, :m_total]^T B[r, :n_out]
     // (row-major A [nrows][lda], B [nrows][ldb], both read MN-major in place)
@@ -792,13 +797,14 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
     // the same with B = G matrices [K rows][n_out] read MN-major in place:
     // A's columns 0..k1-1 against B1, k1..k1+k2-1 against B2
     auto tc_rows_mn = [&](const void *A, int64_t nrows, const void *B1, int64_t k1, const void *B2, int64_t k2,
-                          int n_out, float *C, const int32_t *off, const int32_t *mt_, int G, bool accumulate) {
+                          int n_out, float *C, const int32_t *off, const int32_t *mt_, int tile_m, int G,
+                          bool accumulate) {
         TcGemmArgs t{};
         t.A = A; t.a_rows = static_cast<uint64_t>(nrows); t.a_cols = static_cast<uint64_t>(k1 + k2);
         t.B = B1; t.B2 = B2; t.k1 = k1; t.k2 = k2; t.b_mn = 1;
         t.C = C; t.ldc = n_out; t.offsets = off; t.mt_prefix = mt_; t.E = G; t.K = static_cast<int>(k1 + k2);
         t.n_out = n_out; t.status = dev_status; t.accumulate = accumulate ? 1 : 0;
-        return launch_gemm_tc_f32(t, sms, s);
+        return tc_launch(t, tile_m);
     };
     BwdActArgs act{rows, F, d, cfg->act, bf ? 1 : 0, pre, up, h, dh, swiglu ? nullptr : b1, b2,
                    at<int32_t>(ws, L.row_e), row_w, dw, perm, dys, nullptr};
@@ -807,22 +813,23 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
         // ---- bf16: every expert product on the tensor cores (fp32 results),
         // every operand read in place: dgrad with the weights MN-major, wgrad
         // over each expert's token rows of the activations (MN-major)
-        int32_t *mt128 = at<int32_t>(ws, L.mt128);
+        const int tm = ffn_tile_m(cfg);
+        int32_t *mtc = at<int32_t>(ws, L.mtc);
         auto *dacat = at<__nv_bfloat16>(ws, L.dacat), *hwb = at<__nv_bfloat16>(ws, L.hwb);
         auto ragged_m = [&](const void *A, int64_t K, const void *B, int n_out, float *C) {
-            return tc_rows(A, rows, K, B, n_out, C, offsets, mt128, E, false);
+            return tc_rows(A, rows, K, B, n_out, C, offsets, mtc, tm, E, false);
         };
-        MOE_TRY(launch_tile_table(offsets, mt128, E, 128, s));
+        MOE_TRY(launch_tile_table(offsets, mtc, E, tm, s));
         MOE_TRY(ragged_m(xs, d, W1, F, pre));
         if (swiglu) MOE_TRY(ragged_m(xs, d, W3, F, up));
         MOE_TRY(launch_act_forward(act, sms, s));
-        MOE_TRY(tc_rows_mn(dys, rows, W2, d, nullptr, 0, F, dh, offsets, mt128, E, false));  // dh = dy_s W2[e]
+        MOE_TRY(tc_rows_mn(dys, rows, W2, d, nullptr, 0, F, dh, offsets, mtc, tm, E, false));  // dh = dy_s W2[e]
         act.dcat = dacat;  // [da | du] and w h in bf16; fp32 da only for db1
         act.hw_bf = hwb;
         act.skip_f32 = kSkipUp | kSkipH | ((!swiglu && b1 && gr.db1) ? 0 : kSkipPre);
         MOE_TRY(launch_row_backward(act, sms, s));
         // dx_s = [da | du] [W1[e] ; W3[e]]: one product with K = m F
-        MOE_TRY(tc_rows_mn(dacat, rows, W1, F, swiglu ? W3 : nullptr, swiglu ? F : 0, d, dxs, offsets, mt128, E,
+        MOE_TRY(tc_rows_mn(dacat, rows, W1, F, swiglu ? W3 : nullptr, swiglu ? F : 0, d, dxs, offsets, mtc, tm, E,
                            false));
         // weight gradients, each expert over its own rows
         const int64_t ldcat = static_cast<int64_t>(m) * F;
@@ -878,19 +885,20 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
         BwdActArgs sa{N, Fs, d, cfg->act, bf ? 1 : 0, spre, sup, sh, sdh, swiglu ? nullptr : shared->b1, nullptr,
                       nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
         if (bf) {  // tensor cores, one group of N rows
-            int32_t *smt = at<int32_t>(ws, L.smt128);
+            const int stm = shared_tile_m(cfg);
+            int32_t *smt = at<int32_t>(ws, L.smtc);
             auto *sdcat = at<__nv_bfloat16>(ws, L.sdcat), *shb = at<__nv_bfloat16>(ws, L.shb);
-            MOE_TRY(launch_tile_table(doff, smt, 1, 128, s));
-            MOE_TRY(tc_rows(x, N, d, shared->W1, Fs, spre, doff, smt, 1, false));
-            if (swiglu) MOE_TRY(tc_rows(x, N, d, shared->W3, Fs, sup, doff, smt, 1, false));
+            MOE_TRY(launch_tile_table(doff, smt, 1, stm, s));
+            MOE_TRY(tc_rows(x, N, d, shared->W1, Fs, spre, doff, smt, stm, 1, false));
+            if (swiglu) MOE_TRY(tc_rows(x, N, d, shared->W3, Fs, sup, doff, smt, stm, 1, false));
             MOE_TRY(launch_act_forward(sa, sms, s));
-            MOE_TRY(tc_rows_mn(dy, N, shared->W2, d, nullptr, 0, Fs, sdh, doff, smt, 1, false));
+            MOE_TRY(tc_rows_mn(dy, N, shared->W2, d, nullptr, 0, Fs, sdh, doff, smt, stm, 1, false));
             sa.dcat = sdcat;
             sa.hw_bf = shb;
             sa.skip_f32 = kSkipUp | kSkipH | ((!swiglu && shared->b1 && gr.dbs1) ? 0 : kSkipPre);
             MOE_TRY(launch_row_backward(sa, sms, s));
             MOE_TRY(tc_rows_mn(sdcat, N, shared->W1, Fs, swiglu ? shared->W3 : nullptr, swiglu ? Fs : 0, d, gr.dx,
-                               doff, smt, 1, true));
+                               doff, smt, stm, 1, true));
             const int64_t ldcat = static_cast<int64_t>(m) * Fs;
             MOE_TRY(tc_sum_rows(dy, d, d, shb, Fs, Fs, gr.dWs2, doff, 1, N));
             MOE_TRY(tc_sum_rows(sdcat, ldcat, Fs, x, d, d, gr.dWs1, doff, 1, N));

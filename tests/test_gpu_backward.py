@@ -38,6 +38,11 @@ CASES = {
                                                                       d_ff_shared=64), 0.1, 0.01),
     "bf16_gpt2_shared_bias": (W.WORKLOADS["gpt2_moe"].scaled(N=150, d_model=128, d_ff=128, d_ff_shared=96),
                               0.05, 0.01),
+    # more than 192 rows per group: the ragged-M products run on CTA pairs
+    # (d_model 320 and d_ff 384 leave partial 256-column tiles)
+    "bf16_mixtral_pairs": (W.WORKLOADS["mixtral"].scaled(N=1100, d_model=320, d_ff=384), 0.5, 0.1),
+    "bf16_gpt2_shared_pairs": (W.WORKLOADS["gpt2_moe"].scaled(N=420, d_model=128, d_ff=128, d_ff_shared=96),
+                               0.05, 0.01),
     "one_token": (W.WORKLOADS["mixtral"].scaled(N=1, d_model=64, d_ff=64), 0.5, 0.5),
 }
 
