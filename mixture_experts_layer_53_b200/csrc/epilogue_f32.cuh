@@ -57,5 +57,43 @@ __device__ __forceinline__ void epilogue_f32_rows(float *out, int64_t ldo, int n
     }
 }
 
+// The same warp's rows written by TMA stores instead (the weight gradients,
+// whose short per-expert reductions would otherwise wait on thread stores):
+// the result is [E][m_total][n_out] behind tm_out ({n_out, m_total, E},
+// 32 x 32 boxes, 128-byte swizzle, clipped at the edges); this is group e,
+// rows row_first .. row_first + 31.  buf: the warp's 4 KB, 1024-byte aligned,
+// written in the box's swizzled layout (16-byte piece j of row r at piece
+// j ^ (r & 7)), which is also free of bank conflicts.  Lane 0 owns the
+// stores: it waits for the previous one to have read buf before buf is
+// rewritten, and the caller waits for all of them (bulk_wait_all) before
+// the CTA exits.
+__device__ __forceinline__ void epilogue_f32_tma(const CUtensorMap *tm_out, uint32_t tbase, int e, int row_first,
+                                                 int64_t m_total, int n0, int n_out, uint8_t *buf, bool zero)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll 1
+    for (int c = 0; c < 256; c += 32) {
+        uint32_t acc[32];
+        tmem_ld32(tbase + c, acc);
+        tmem_ld_wait();
+        const int col = n0 + c;
+        if (row_first >= m_total || col >= n_out) continue;  // warp-uniform: nothing to store
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4 *>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                     : make_float4(__uint_as_float(acc[4 * j]), __uint_as_float(acc[4 * j + 1]),
+                                   __uint_as_float(acc[4 * j + 2]), __uint_as_float(acc[4 * j + 3]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_3d(tm_out, buf, col, row_first, e);
+            bulk_commit();
+        }
+    }
+}
+
 }  // namespace sm100
 }  // namespace moe

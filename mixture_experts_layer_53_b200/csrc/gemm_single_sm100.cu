@@ -207,39 +207,6 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase,
     }
 }
 
-// EPI_F32 with OPS_MN_MN: expert e's [m_total, n_out] result goes out
-// through TMA stores of 32 x 32 boxes (tm_out = {n_out, m_total, E}, clipped
-// at the edges), so the short per-expert reductions of the weight gradients
-// are not held up by thread stores.  buf: this warp's 4 KB, 1024-aligned.
-__device__ __forceinline__ void epilogue_tile_tma(const GemmArgs &g, const CUtensorMap *tm_out, uint32_t tbase,
-                                                  int e, int row_first, int n0, uint8_t *buf, bool zero)
-{
-    const int lane = threadIdx.x & 31;
-#pragma unroll 1
-    for (int c = 0; c < 256; c += 32) {
-        uint32_t acc[32];
-        tmem_ld32(tbase + c, acc);
-        tmem_ld_wait();
-        const int col = n0 + c;
-        if (row_first >= g.m_total || col >= g.n_out) continue;  // warp-uniform: nothing to store
-        if (lane == 0) bulk_wait_read_all();  // the previous store has read buf
-        __syncwarp();
-        // row `lane`; its 16-B piece j sits at piece j ^ (lane & 7) of the row
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<float4 *>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                zero ? make_float4(0.f, 0.f, 0.f, 0.f)
-                     : make_float4(__uint_as_float(acc[4 * j]), __uint_as_float(acc[4 * j + 1]),
-                                   __uint_as_float(acc[4 * j + 2]), __uint_as_float(acc[4 * j + 3]));
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-            tma_store_3d(tm_out, buf, col, row_first, e);
-            bulk_commit();
-        }
-    }
-}
-
 // MN-major operand tiles (OPS_K_MN, OPS_MN_MN; EPI_F32 only) are 64-column
 // x 64-row boxes 8 KB apart, so the backward's products against W^T and
 // over token rows need no transposed copies.  In OPS_MN_MN the last k-block
@@ -484,8 +451,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
             if constexpr (EPI == EPI_F32 && OPS == OPS_MN_MN)
-                epilogue_tile_tma(g, &tmB3, tbase, ti.e, row_first, ti.n_tile * BN,
-                                  reinterpret_cast<uint8_t *>(ctl->stage) + quarter * 4096, kblocks(ti.e) == 0);
+                epilogue_f32_tma(&tmB3, tbase, ti.e, row_first, g.m_total, ti.n_tile * BN, g.n_out,
+                                 reinterpret_cast<uint8_t *>(ctl->stage) + quarter * 4096, kblocks(ti.e) == 0);
             else
                 epilogue_tile<EPI>(g, tbase, ti.e, row_first, row_end, ti.n_tile * out_cols<EPI>(),
                                    ctl->stage[quarter], kblocks(ti.e) == 0);
