@@ -533,7 +533,8 @@ def run_backward(args, wl):
     if wl.dtype == "bf16":
         peaks, peak_src = load_peaks()
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        bound, kern = "tensor", "ffn_gemm_single_kernel<F32> (expert dgrad / wgrad products)"
+        bound, kern = "tensor", ("ffn_gemm_pair_kernel<F32> / ffn_gemm_single_kernel<F32> (expert recompute, dgrad "
+                                 "and wgrad products)")
         src = f"{peak_src} bf16_tflops_sustained"
     else:
         peak = 148 * 128 * 2 * mhz * 1e6 / 1e12

@@ -164,14 +164,20 @@ __global__ void __launch_bounds__(256) gather_sum_kernel(BwdGatherSumArgs a)
     for (int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); n < a.N;
          n += warps) {
         const int src_l = lane < a.k ? a.inv_perm[n * a.k + lane] : 0;
-        for (int c0 = 0; c0 < a.d; c0 += 32) {  // warp-uniform
-            const int c = c0 + lane;
-            float s = 0.f;
-            for (int j = 0; j < a.k; ++j) {
+        for (int c0 = 0; c0 < a.d; c0 += 128) {  // warp-uniform; 4 columns per lane (d is a multiple of 8)
+            const int c = c0 + lane * 4;
+            float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < a.k; ++j) {  // fixed order over the token's k rows
                 const int src = __shfl_sync(0xffffffffu, src_l, j);
-                if (c < a.d) s += a.dxs[static_cast<int64_t>(src) * a.d + c];
+                if (c < a.d) {
+                    const float4 v = *reinterpret_cast<const float4 *>(a.dxs + static_cast<int64_t>(src) * a.d + c);
+                    s.x += v.x;
+                    s.y += v.y;
+                    s.z += v.z;
+                    s.w += v.w;
+                }
             }
-            if (c < a.d) a.dx[n * a.d + c] = s;
+            if (c < a.d) *reinterpret_cast<float4 *>(a.dx + n * a.d + c) = s;
         }
     }
 }
