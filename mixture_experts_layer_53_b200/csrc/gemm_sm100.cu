@@ -31,11 +31,20 @@
 // same 128 rows of W3, so accumulator columns 0..127 are the gate and
 // 128..255 the up projection of 128 hidden units.
 //
-// The backward's ragged-M products use the same kernel with fp32 results
-// (EPI_F32): the recomputed pre-activations x_s W1[e]^T (K-major B) and the
-// dgrad products dy_s W2[e], [da | du] [W1[e]; W3[e]] (OPS_K_MN: each CTA
-// loads its 128 result columns of the [E][K][n_out] weights as two 64 x 64
-// MN-major boxes, so no transposed copy of the weights is made).
+// The backward's products use the same kernel with fp32 results (EPI_F32):
+// the recomputed pre-activations x_s W1[e]^T (K-major B); the dgrad
+// products dy_s W2[e], [da | du] [W1[e]; W3[e]] (OPS_K_MN: each CTA loads
+// its 128 result columns of the [E][K][n_out] weights as two 64 x 64
+// MN-major boxes, so no transposed copy of the weights is made); and the
+// weight gradients (OPS_MN_MN, ragged K): tile (expert, m-tile of 256,
+// n-tile) sums its expert's own rows of two row-major activations, each CTA
+// loading its 128 columns of both as MN-major boxes.  Only an expert's last
+// k-block, which also holds rows of the next expert, needs more than the
+// forward's protocol: there each CTA loads onto its own `tail_full`
+// barrier, zeroes those rows in its own shared memory, fences, and arrives
+// on the even CTA's `ready` barrier, which the even CTA waits on (cluster
+// scope) before the MMA; the even CTA's `full` barrier gets a 0-byte arrival
+// so that its phases stay in step.  The results leave through TMA stores.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -67,7 +76,8 @@ constexpr uint32_t TMEM_COLS = 512;
 
 
 enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_LINEAR = 2, EPI_F32 = 3 };
-enum { OPS_KK = 0, OPS_K_MN = 1 };  // B K-major / MN-major (A K-major in both)
+// B K-major / B MN-major (A K-major in both) / A and B MN-major, ragged K
+enum { OPS_KK = 0, OPS_K_MN = 1, OPS_MN_MN = 2 };
 constexpr int BOX_BYTES = 64 * 64 * 2;  // one 64 x 64 MN-major box
 template <int EPI> __host__ __device__ constexpr int epi_warps() { return EPI == EPI_GELU ? 8 : 4; }
 
@@ -85,6 +95,10 @@ struct GemmArgs {
     // columns kb * BK; k-blocks kb1..kb_total-1 read tmB3 with A columns
     // a_col2 + (kb - kb1) * BK
     int kb1, kb_total, a_col2;
+    // OPS_MN_MN: expert e sums rows offsets[e] .. offsets[e+1]-1; the result
+    // [E][m_total][n_out] has m_tiles tiles of 256 rows
+    int m_tiles;
+    int64_t m_total;
 };
 
 struct Ctl {
@@ -95,6 +109,8 @@ struct Ctl {
     uint64_t tfull[2];       // each CTA: arrived by the even CTA's commit
     uint64_t tempty[2];      // even CTA: 4 epilogue warps x 2 CTAs
     uint64_t drain;
+    uint64_t tail_full[STAGES];  // OPS_MN_MN, each CTA: its own copies of an expert's last k-block
+    uint64_t ready[STAGES];      // OPS_MN_MN, even CTA: both CTAs zeroed that k-block's extra rows
     uint32_t tmem_base;
     int abort;
     int off[kMaxE + 1];
@@ -123,6 +139,27 @@ __device__ __forceinline__ Tile decode_tile(int t, const Ctl *c, int E, int n_ti
 }
 
 template <int EPI> __host__ __device__ constexpr int out_cols() { return EPI == EPI_SWIGLU ? 128 : 256; }
+
+// Tile t: the ragged-M tile table, or (OPS_MN_MN) experts x n-tiles x
+// m-tiles with m innermost.
+template <int OPS> __device__ __forceinline__ Tile tile_at(int t, const Ctl *c, const GemmArgs &g)
+{
+    if constexpr (OPS != OPS_MN_MN) {
+        return decode_tile(t, c, g.E, g.n_tiles);
+    } else {
+        const int per = g.m_tiles * g.n_tiles;
+        const int e = t / per, local = t - e * per;
+        return Tile{e, local % g.m_tiles, local / g.m_tiles};
+    }
+}
+
+// OPS_MN_MN: 64-column boxes CTA r of the pair loads for a 256-wide range
+// starting at `base` of an extent (0 past the end).
+__device__ __forceinline__ int half_boxes(int r, int64_t extent, int base)
+{
+    const int64_t left = extent - (base + r * 128);
+    return left <= 0 ? 0 : static_cast<int>(min64(2, (left + 63) / 64));
+}
 
 // Output columns [c_begin, c_end) of one accumulator row (this thread's row).
 template <int EPI>
@@ -206,13 +243,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             mbar_init(&ctl->tempty[b], 2 * epi_warps<EPI>());  // every epilogue warp of both CTAs
         }
         mbar_init(&ctl->drain, 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&ctl->tail_full[s], 1);
+            mbar_init(&ctl->ready[s], 2);
+        }
         ctl->abort = 0;
         fence_mbar_init();
     }
     if (threadIdx.x == 32) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
-        if (EPI == EPI_SWIGLU || OPS == OPS_K_MN) prefetch_tmap(&tmB3);
+        if (EPI == EPI_SWIGLU || OPS != OPS_KK) prefetch_tmap(&tmB3);
     }
     if (warp == 1) {
         tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
@@ -220,7 +261,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
     }
     for (int i = threadIdx.x; i <= g.E; i += threads_of<EPI>()) {
         ctl->off[i] = g.offsets[i];
-        ctl->mt[i] = g.mt_prefix[i];
+        ctl->mt[i] = OPS == OPS_MN_MN ? 0 : g.mt_prefix[i];
     }
     tc_fence_before();
     // barriers of both CTAs are initialised before either CTA signals the other
@@ -228,8 +269,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
     tc_fence_after();
 
     const uint32_t tmem_base = ctl->tmem_base;
-    const int total = ctl->mt[g.E] * g.n_tiles;
+    const int total = OPS == OPS_MN_MN ? g.E * g.m_tiles * g.n_tiles : ctl->mt[g.E] * g.n_tiles;
     const int num_kb = OPS == OPS_K_MN ? g.kb_total : (g.K + BK - 1) / BK;
+    // OPS_MN_MN: an expert's rows in k-blocks of BK
+    auto mn_kblocks = [&](int e) { return (ctl->off[e + 1] - ctl->off[e] + BK - 1) / BK; };
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (warp == 0) {
@@ -237,9 +280,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             // ------------------------------------------------ TMA producer
             int stage = 0;
             uint32_t phase = 0, armed = 0, armed_parity = 0;
+            uint32_t tpar = 0, tarmed = 0, tarmed_parity = 0;  // OPS_MN_MN tail_full phases per stage
             bool ok = true;
             for (int t = pair; t < total && ok; t += npairs) {
-                const Tile ti = decode_tile(t, ctl, g.E, g.n_tiles);
+                const Tile ti = tile_at<OPS>(t, ctl, g);
+                if constexpr (OPS == OPS_MN_MN) {
+                    const int mrow = ti.m_tile * PAIR_M, ncol = ti.n_tile * BN;
+                    const int ab0 = half_boxes(0, g.m_total, mrow), ab1 = half_boxes(1, g.m_total, mrow);
+                    const int bb0 = half_boxes(0, g.n_out, ncol), bb1 = half_boxes(1, g.n_out, ncol);
+                    const int ab = rank ? ab1 : ab0, bb = rank ? bb1 : bb0;
+                    const uint32_t both_bytes = static_cast<uint32_t>(ab0 + bb0 + ab1 + bb1) * BOX_BYTES;
+                    const uint32_t my_bytes = static_cast<uint32_t>(ab + bb) * BOX_BYTES;
+                    const int m0 = mrow + static_cast<int>(rank) * BM, n0 = ncol + static_cast<int>(rank) * (BN / 2);
+                    const int cnt = ctl->off[ti.e + 1] - ctl->off[ti.e], nkb = mn_kblocks(ti.e);
+                    for (int kb = 0; kb < nkb; ++kb) {
+                        if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort_flag, g.status)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t *sA = tiles + stage * STAGE_BYTES;
+                        const int r = ctl->off[ti.e] + kb * BK;
+                        const bool tail = cnt - kb * BK < BK;
+                        if (leader) {  // a tail k-block only completes the phase
+                            mbar_arrive_expect_tx(&ctl->full[stage], tail ? 0u : both_bytes);
+                            armed |= 1u << stage;
+                            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                        }
+                        if (!tail) {
+                            const uint32_t full_leader = mapa_shared(smem_u32(&ctl->full[stage]), 0);
+                            for (int c = 0; c < ab; ++c)
+                                tma_load_2d_pair(sA + c * BOX_BYTES, &tmA, full_leader, m0 + c * 64, r);
+                            for (int c = 0; c < bb; ++c)
+                                tma_load_2d_pair(sA + A_BYTES + c * BOX_BYTES, &tmB, full_leader, n0 + c * 64, r);
+                        } else {
+                            const uint32_t tp = (tpar >> stage) & 1u;
+                            mbar_arrive_expect_tx(&ctl->tail_full[stage], my_bytes);
+                            tarmed |= 1u << stage;
+                            tarmed_parity = (tarmed_parity & ~(1u << stage)) | (tp << stage);
+                            for (int c = 0; c < ab; ++c)
+                                tma_load_2d(sA + c * BOX_BYTES, &tmA, &ctl->tail_full[stage], m0 + c * 64, r);
+                            for (int c = 0; c < bb; ++c)
+                                tma_load_2d(sA + A_BYTES + c * BOX_BYTES, &tmB, &ctl->tail_full[stage], n0 + c * 64,
+                                            r);
+                            tpar ^= 1u << stage;
+                        }
+                        if (++stage == STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                    continue;
+                }
                 const int row0 = ctl->off[ti.e] + ti.m_tile * PAIR_M + static_cast<int>(rank) * BM;
                 int brow;
                 const CUtensorMap *tb;
@@ -306,6 +397,90 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                     if ((armed >> s) & 1u)
                         mbar_wait(&ctl->full[s], (armed_parity >> s) & 1u, abort_flag, g.status, false);
             }
+            if (*abort_flag) {
+                // OPS_MN_MN: this CTA's own copies of tail k-blocks
+                for (int s = 0; s < STAGES; ++s)
+                    if ((tarmed >> s) & 1u)
+                        mbar_wait(&ctl->tail_full[s], (tarmed_parity >> s) & 1u, abort_flag, g.status, false);
+            }
+        }
+    } else if (warp == 1 && OPS == OPS_MN_MN) {
+        // ------------------------ OPS_MN_MN: MMA issuer (even CTA) and the
+        // tail k-blocks' zeroing (both CTAs, the whole warp)
+        constexpr uint32_t idesc = idesc_bf16_f32_mn(PAIR_M, BN);
+        auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, g.status));
+        };
+        int stage = 0, buf = 0;
+        uint32_t phase = 0, tphase = 0, tpar = 0;
+        bool ok = true, issued = false;
+        for (int t = pair; t < total && ok; t += npairs) {
+            const int e = tile_at<OPS>(t, ctl, g).e;
+            const int nkb = mn_kblocks(e), cnt = ctl->off[e + 1] - ctl->off[e];
+            if (leader) {
+                if (!wait_all(&ctl->tempty[buf], tphase ^ 1u)) break;
+                tc_fence_after();
+            }
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+            for (int kb = 0; kb < nkb; ++kb) {
+                uint8_t *st = tiles + stage * STAGE_BYTES;
+                const int v = cnt - kb * BK;  // rows of the expert in this k-block
+                const bool tail = v < BK;
+                const uint32_t tp = (tpar >> stage) & 1u;
+                if (tail) {
+                    if (!wait_all(&ctl->tail_full[stage], tp)) {
+                        ok = false;
+                        break;
+                    }
+                    // rows v..63 of the four boxes (whole 128-B rows)
+                    const int per_box = (BK - v) * 8;  // 16-B pieces
+                    for (int i = lane; i < 4 * per_box; i += 32) {
+                        const int box = i / per_box, j = i - box * per_box;
+                        *reinterpret_cast<uint4 *>(st + box * BOX_BYTES + v * 128 + j * 16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->ready[stage]), 0));
+                    tpar ^= 1u << stage;
+                }
+                if (leader) {
+                    const bool w = tail ? __all_sync(0xffffffffu, mbar_wait<true>(&ctl->ready[stage], tp, abort_flag,
+                                                                                 g.status))
+                                        : wait_all(&ctl->full[stage], phase);
+                    if (!w) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t a_addr = smem_u32(st);
+                        const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            umma_bf16_pair(d_tmem, desc_sw128_mn(a_addr + kk * 2048, BOX_BYTES),
+                                           desc_sw128_mn(b_addr + kk * 2048, BOX_BYTES), idesc,
+                                           (kb | kk) != 0 ? 1u : 0u);
+                        issued = true;
+                        umma_commit_pair(&ctl->empty[stage], 0x3);
+                    }
+                    __syncwarp();
+                }
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (leader && lane == 0) umma_commit_pair(&ctl->tfull[buf], 0x3);
+            if (++buf == 2) {
+                buf = 0;
+                tphase ^= 1u;
+            }
+        }
+        if (leader && lane == 0 && *abort_flag && issued) {
+            umma_commit_pair(&ctl->drain, 0x1);
+            mbar_wait(&ctl->drain, 0, abort_flag, g.status, false);
         }
     } else if (warp == 1) {
         if (lane == 0 && leader) {
@@ -367,12 +542,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&ctl->tfull[buf], tphase, abort_flag, g.status));
             if (!ok) break;
             tc_fence_after();
-            const Tile ti = decode_tile(t, ctl, g.E, g.n_tiles);
+            const Tile ti = tile_at<OPS>(t, ctl, g);
             const int row = ctl->off[ti.e] + ti.m_tile * PAIR_M + static_cast<int>(rank) * BM + row_in_cta;
             const bool row_ok = row < ctl->off[ti.e + 1];
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
-            if constexpr (EPI == EPI_F32)
+            if constexpr (EPI == EPI_F32 && OPS == OPS_MN_MN)
+                epilogue_f32_tma(&tmB3, tbase, ti.e, ti.m_tile * PAIR_M + static_cast<int>(rank) * BM + quarter * 32,
+                                 g.m_total, ti.n_tile * BN, g.n_out,
+                                 reinterpret_cast<uint8_t *>(ctl->stage) + quarter * 4096, mn_kblocks(ti.e) == 0);
+            else if constexpr (EPI == EPI_F32)
                 epilogue_f32_rows(g.out_f32, g.ldo, g.n_out, tbase, row - lane, ctl->off[ti.e + 1], ti.n_tile * BN,
                                   ctl->stage[quarter], false, g.accumulate != 0);
             else
@@ -386,6 +565,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                 tphase ^= 1u;
             }
         }
+        // the staging buffers stay valid until this warp's stores are done
+        if (EPI == EPI_F32 && OPS == OPS_MN_MN && lane == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -414,7 +595,33 @@ cudaError_t launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtens
 
 cudaError_t launch_gemm_tc_f32_pair(const TcGemmArgs &t, int num_sms, cudaStream_t s)
 {
-    if (t.ragged_k || t.rows_mn) return cudaErrorInvalidValue;  // ragged M only
+    if (t.rows_mn) {
+        // weight gradients: ragged K over each group's rows, A and B read
+        // MN-major in place, the result out through TMA stores
+        if (!t.ragged_k || t.b_mn || t.lda % 8 != 0 || t.ldb % 8 != 0 || t.m_total % 8 != 0 || t.n_out % 8 != 0 ||
+            t.m_total > t.lda || t.n_out > t.ldb || t.ldc != t.n_out || t.c_stride != t.m_total * t.n_out ||
+            (reinterpret_cast<uintptr_t>(t.C) & 15u) != 0)
+            return cudaErrorInvalidValue;
+        if (t.m_total == 0 || t.n_out == 0) return cudaSuccess;
+        CUtensorMap tA, tB, tOut;
+        if (!make_tmap_bf16_mn_rows(&tA, t.A, static_cast<uint64_t>(t.m_total), t.a_rows,
+                                    static_cast<uint64_t>(t.lda)) ||
+            !make_tmap_bf16_mn_rows(&tB, t.B, static_cast<uint64_t>(t.n_out), t.a_rows,
+                                    static_cast<uint64_t>(t.ldb)) ||
+            !make_tmap_f32_store(&tOut, t.C, static_cast<uint64_t>(t.n_out), static_cast<uint64_t>(t.m_total),
+                                 static_cast<uint64_t>(t.E)))
+            return cudaErrorInvalidValue;
+        GemmArgs g{};
+        g.offsets = t.offsets;
+        g.status = t.status;
+        g.E = t.E;
+        g.n_out = t.n_out;
+        g.n_tiles = (t.n_out + BN - 1) / BN;
+        g.m_tiles = static_cast<int>((t.m_total + PAIR_M - 1) / PAIR_M);
+        g.m_total = t.m_total;
+        return launch_pair<EPI_F32, OPS_MN_MN>(tA, tB, tOut, g, num_sms, s);
+    }
+    if (t.ragged_k) return cudaErrorInvalidValue;  // ragged K only with rows_mn
     if (t.a_rows == 0 || t.n_out == 0) return cudaSuccess;
     if (t.b_mn && (t.k1 <= 0 || t.k2 < 0 || (t.k2 > 0) != (t.B2 != nullptr) ||
                    static_cast<uint64_t>(t.k1 + t.k2) != t.a_cols || t.k1 % 8 != 0 || t.n_out % 8 != 0))

@@ -786,13 +786,14 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
     };
     // C_g [m_total, n_out] = sum over rows off[g] .. off[g+1]-1 of A[r, :m_total]^T B[r, :n_out]
     // (row-major A [nrows][lda], B [nrows][ldb], both read MN-major in place)
+    // (CTA pairs under the same rule as the ragged-M products)
     auto tc_sum_rows = [&](const void *A, int64_t lda, int64_t m_total, const void *B, int64_t ldb, int n_out, float *C,
-                           const int32_t *off, int G, int64_t nrows) {
+                           const int32_t *off, int tile_m, int G, int64_t nrows) {
         TcGemmArgs t{};
         t.A = A; t.a_rows = static_cast<uint64_t>(nrows); t.lda = lda; t.B = B; t.ldb = ldb; t.rows_mn = 1;
         t.C = C; t.ldc = n_out; t.c_stride = m_total * n_out; t.offsets = off; t.E = G; t.ragged_k = 1;
         t.n_out = n_out; t.m_total = m_total; t.status = dev_status;
-        return launch_gemm_tc_f32(t, sms, s);
+        return tile_m == 256 ? launch_gemm_tc_f32_pair(t, sms, s) : launch_gemm_tc_f32(t, sms, s);
     };
     // the same with B = G matrices [K rows][n_out] read MN-major in place:
     // A's columns 0..k1-1 against B1, k1..k1+k2-1 against B2
@@ -833,9 +834,9 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
                            false));
         // weight gradients, each expert over its own rows
         const int64_t ldcat = static_cast<int64_t>(m) * F;
-        MOE_TRY(tc_sum_rows(dys, d, d, hwb, F, F, gr.dW2, offsets, E, rows));          // dW2[e] = dy_s^T (w h)
-        MOE_TRY(tc_sum_rows(dacat, ldcat, F, xs, d, d, gr.dW1, offsets, E, rows));     // dW1[e] = da^T x_s
-        if (swiglu) MOE_TRY(tc_sum_rows(dacat + F, ldcat, F, xs, d, d, gr.dW3, offsets, E, rows));
+        MOE_TRY(tc_sum_rows(dys, d, d, hwb, F, F, gr.dW2, offsets, tm, E, rows));          // dW2[e] = dy_s^T (w h)
+        MOE_TRY(tc_sum_rows(dacat, ldcat, F, xs, d, d, gr.dW1, offsets, tm, E, rows));     // dW1[e] = da^T x_s
+        if (swiglu) MOE_TRY(tc_sum_rows(dacat + F, ldcat, F, xs, d, d, gr.dW3, offsets, tm, E, rows));
     } else {
         // ---- fp32: the same products on the CUDA cores
         MOE_TRY(GG().a(xs, d, 1, bf).b(W1, 1, d, static_cast<int64_t>(F) * d, bf).c(pre, F, 1, 0)
@@ -900,9 +901,9 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
             MOE_TRY(tc_rows_mn(sdcat, N, shared->W1, Fs, swiglu ? shared->W3 : nullptr, swiglu ? Fs : 0, d, gr.dx,
                                doff, smt, stm, 1, true));
             const int64_t ldcat = static_cast<int64_t>(m) * Fs;
-            MOE_TRY(tc_sum_rows(dy, d, d, shb, Fs, Fs, gr.dWs2, doff, 1, N));
-            MOE_TRY(tc_sum_rows(sdcat, ldcat, Fs, x, d, d, gr.dWs1, doff, 1, N));
-            if (swiglu) MOE_TRY(tc_sum_rows(sdcat + Fs, ldcat, Fs, x, d, d, gr.dWs3, doff, 1, N));
+            MOE_TRY(tc_sum_rows(dy, d, d, shb, Fs, Fs, gr.dWs2, doff, stm, 1, N));
+            MOE_TRY(tc_sum_rows(sdcat, ldcat, Fs, x, d, d, gr.dWs1, doff, stm, 1, N));
+            if (swiglu) MOE_TRY(tc_sum_rows(sdcat + Fs, ldcat, Fs, x, d, d, gr.dWs3, doff, stm, 1, N));
         } else {
             MOE_TRY(GG().a(x, d, 1, bf).b(shared->W1, 1, d, 0, bf).c(spre, Fs, 1, 0).rows(doff, dmt, 1, N, Fs, d, s));
             if (swiglu)

@@ -64,17 +64,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// The same with cluster-scope acquire: for phases completed by arrivals
+// (release.cluster) from the other CTA of a pair.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false when
 // the CTA's abort flag is raised or the time limit passes (then it raises the
 // flag and records kDevTimeout).  `honour_abort` = false is used while
-// draining after an abort.
+// draining after an abort.  kCluster: cluster-scope acquire.
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                           int32_t *status, bool honour_abort = true)
 {
-    if (mbar_try_wait(bar, parity)) return true;
+    auto try_wait = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+    if (try_wait()) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (try_wait()) return true;
         if ((i & 31u) == 0) {
             if (honour_abort && *abort_flag) return false;
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
