@@ -76,9 +76,9 @@ struct GemmArgs {
     int E, K, n_out, n_tiles, b_rows;
     // EPI_F32: plain fp32 stores to out_f32 (the backward's products)
     float *out_f32;
-    // ragged_k: the reduction of expert e runs over columns offsets[e] ..
-    // offsets[e+1]-1 of A and B (multiples of BK, zero-padded); A rows are
-    // the m_total result rows (m_tiles tiles of BM), B rows the n_out result
+    // ragged_k (OPS_MN_MN): the reduction of expert e runs over rows
+    // offsets[e] .. offsets[e+1]-1 of the activations; A's columns are the
+    // m_total result rows (m_tiles tiles of BM), B's the n_out result
     // columns; expert e's result starts at out_f32 + e * c_stride
     int ragged_k, m_tiles;
     int64_t m_total, c_stride;
@@ -261,11 +261,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int total = g.ragged_k ? g.E * g.m_tiles * g.n_tiles : ctl->mt[g.E] * g.n_tiles;
     const int num_kb = OPS == OPS_K_MN ? g.kb_total : (g.K + BK - 1) / BK;
     // k-blocks of a tile and the column (OPS_MN_MN: row) they start at
-    auto kblocks = [&](int e) {
-        if (OPS == OPS_MN_MN) return (ctl->off[e + 1] - ctl->off[e] + BK - 1) / BK;
-        return g.ragged_k ? (ctl->off[e + 1] - ctl->off[e]) / BK : num_kb;
-    };
-    auto kstart = [&](int e) { return g.ragged_k ? ctl->off[e] : 0; };
+    auto kblocks = [&](int e) { return OPS == OPS_MN_MN ? (ctl->off[e + 1] - ctl->off[e] + BK - 1) / BK : num_kb; };
+    auto kstart = [&](int e) { return OPS == OPS_MN_MN ? ctl->off[e] : 0; };
 
     if (warp == 0) {
         if (lane == 0) {
@@ -275,9 +272,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 const Tile ti = tile_of(t, ctl, g);
-                const int row0 = g.ragged_k ? ti.m_tile * BM : ctl->off[ti.e] + ti.m_tile * BM;
-                const int brow = g.ragged_k ? ti.n_tile * out_cols<EPI>()
-                                            : ti.e * g.b_rows + ti.n_tile * out_cols<EPI>();
+                // ragged M (the OPS_MN_MN branch below places its own boxes)
+                const int row0 = ctl->off[ti.e] + ti.m_tile * BM;
+                const int brow = ti.e * g.b_rows + ti.n_tile * out_cols<EPI>();
                 const int nkb = kblocks(ti.e), k0 = kstart(ti.e);
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort_flag, g.status)) {
@@ -491,6 +488,7 @@ cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtens
 
 cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s)
 {
+    if (t.ragged_k != t.rows_mn) return cudaErrorInvalidValue;  // ragged K always reads the rows MN-major
     if (t.ragged_k ? (t.m_total == 0 || t.n_out == 0) : (t.a_rows == 0 || t.n_out == 0)) return cudaSuccess;
     if (t.b_mn && (t.ragged_k || t.k1 <= 0 || t.k2 < 0 || (t.k2 > 0) != (t.B2 != nullptr) ||
                    static_cast<uint64_t>(t.k1 + t.k2) != t.a_cols || t.k1 % 8 != 0 || t.n_out % 8 != 0))
@@ -547,10 +545,6 @@ cudaError_t launch_gemm_tc_f32(const TcGemmArgs &t, int num_sms, cudaStream_t s)
     g.n_out = t.n_out;
     g.n_tiles = (t.n_out + 255) / 256;
     g.b_rows = t.n_out;
-    g.ragged_k = t.ragged_k;
-    g.m_tiles = static_cast<int>((t.m_total + BM - 1) / BM);
-    g.m_total = t.m_total;
-    g.c_stride = t.c_stride;
     g.accumulate = t.accumulate;
     if (t.b_mn) {
         g.kb1 = static_cast<int>((t.k1 + BK - 1) / BK);

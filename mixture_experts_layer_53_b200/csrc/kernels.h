@@ -263,14 +263,15 @@ bool make_tmap_bf16_mn(CUtensorMap *m, const void *base, uint64_t inner, uint64_
 bool make_tmap_bf16_mn_rows(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t ld);
 bool make_tmap_f32_store(CUtensorMap *m, void *base, uint64_t inner, uint64_t rows, uint64_t groups);
 
-// C (fp32) = A B^T on tcgen05 with bf16 operands, both K-major (the
-// backward's products on the tensor cores), 128 x 256 tiles:
-//   ragged_k = 0: rows offsets[e] .. offsets[e+1]-1 of A and C belong to
-//     expert e (mt_prefix: its 128-row tile prefix), B = [E * n_out, K];
-//   ragged_k = 1: expert e's result (m_total x n_out, at C + e * c_stride)
-//     sums columns offsets[e] .. offsets[e+1]-1 of A [m_total, cols] and
-//     B [n_out, cols]; the offsets are multiples of 64 and the columns
-//     between an expert's rows and the next offset are zero.
+// C (fp32) from bf16 operands on tcgen05 (the backward's products on the
+// tensor cores), 128 x 256 tiles:
+//   ragged M (ragged_k = 0): rows offsets[e] .. offsets[e+1]-1 of A
+//     [a_rows, K] (K-major) and of C belong to group e (mt_prefix: its
+//     128-row tile prefix); B is K-major [E * n_out, K] (C = A B^T), or with
+//     b_mn the MN-major weights below (C = A B);
+//   ragged K (ragged_k = rows_mn = 1): group e's result (m_total x n_out at
+//     C + e * c_stride) sums over rows offsets[e] .. offsets[e+1]-1 of the
+//     two row-major activations below, both read MN-major.
 struct TcGemmArgs {
     const void *A;
     uint64_t a_rows, a_cols;
