@@ -382,6 +382,19 @@ MOE_API moe_status moe_backward(const moe_config *cfg, const void *x, const void
                         moe_stream_t stream);
 
 /*
+ * Row permutation, the regrouping step of expert parallelism (course module
+ * "Going further": experts on different GPUs, tokens moved by all-to-all;
+ * the rows one rank receives arrive grouped by sending rank and are
+ * regrouped by expert): dst[dst_row[i]] = src[i] for i < rows, rows of d
+ * elements of `dtype`.  dst_row should be a permutation of 0..rows-1; an
+ * entry outside that range is skipped (that source row is not copied).
+ * src, dst: device, 16-byte aligned, not overlapping; d > 0 and a multiple
+ * of 8; rows < 2^31.  Enqueues only.
+ */
+MOE_API moe_status moe_permute_rows(int32_t dtype, const void *src, const int32_t *dst_row,
+                                    void *dst, int64_t rows, int32_t d, moe_stream_t stream);
+
+/*
  * Failure-detection check (the pages have no counterpart): launches one CTA
  * that waits on an mbarrier nothing ever arrives at, through the same
  * bounded wait every tcgen05 kernel of the library uses.  After the wait

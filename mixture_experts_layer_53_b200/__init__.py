@@ -37,7 +37,7 @@ STAGE_NAMES = ("route", "dispatch", "gemm1", "gemm2", "combine")
 EXPORTS = ("moe_status_string", "moe_last_error", "moe_version", "moe_workspace_size", "moe_route",
            "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_combine", "moe_aux_loss",
            "moe_forward", "moe_shared_ffn", "moe_combine_shared", "moe_router_z_loss", "moe_forward_ex",
-           "moe_backward_workspace_size", "moe_backward", "moe_selftest_wait_timeout")
+           "moe_backward_workspace_size", "moe_backward", "moe_permute_rows", "moe_selftest_wait_timeout")
 # ceil(N / 32) * E limit of moe_dispatch_noalloc (MOE_NOALLOC_DISPATCH_MAX_SLOTS)
 NOALLOC_DISPATCH_MAX_SLOTS = 1 << 19
 
@@ -127,6 +127,8 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_backward.argtypes = [cfgp, vp, vp, f32p, vp, vp, vp, vp, vp, shp, vp, ctypes.c_float, ctypes.c_float,
                                  ctypes.POINTER(MoeGrads), i32p, vp, sz, vp]
     lib.moe_backward.restype = st
+    lib.moe_permute_rows.argtypes = [ctypes.c_int32, vp, i32p, vp, ctypes.c_int64, ctypes.c_int32, vp]
+    lib.moe_permute_rows.restype = st
     lib.moe_selftest_wait_timeout.argtypes = [i32p, vp]
     lib.moe_selftest_wait_timeout.restype = st
     if path is None:
@@ -258,6 +260,21 @@ def moe_combine(cfg: MoeConfig, y_sorted: torch.Tensor, topk_w: torch.Tensor, in
                                _stream(stream))
     _check(rc, "moe_combine")
     return y
+
+
+def moe_permute_rows(src: torch.Tensor, dst_row: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """out[dst_row[i]] = src[i] for the rows of src [rows, d] (f32 or bf16); dst_row [rows] int32."""
+    dtype = {torch.float32: "f32", torch.bfloat16: "bf16"}.get(src.dtype)
+    if dtype is None or src.dim() != 2 or dst_row.dtype != torch.int32 or dst_row.numel() != src.shape[0]:
+        raise ValueError("moe_permute_rows: src [rows, d] f32/bf16 and dst_row [rows] int32")
+    out = out if out is not None else torch.empty_like(src)
+    if src.shape[0] == 0:
+        return out
+    rc = library().moe_permute_rows(DTYPES[dtype], _ptr(src), _ptr(dst_row), _ptr(out), src.shape[0], src.shape[1],
+                                    _stream(stream))
+    _check(rc, "moe_permute_rows")
+    return out
 
 
 def _shared_struct(shared: Optional[Dict[str, Optional[torch.Tensor]]]):

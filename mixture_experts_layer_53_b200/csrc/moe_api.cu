@@ -681,6 +681,19 @@ moe_status moe_forward_ex(const moe_config *cfg, const void *x, const void *W_g,
     return MOE_OK;
 }
 
+moe_status moe_permute_rows(int32_t dtype, const void *src, const int32_t *dst_row, void *dst, int64_t rows,
+                            int32_t d, moe_stream_t stream)
+{
+    if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (rows < 0 || d <= 0 || d % 8 != 0 || rows >= (static_cast<int64_t>(1) << 31)) return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (!src || !dst_row || !dst || !aligned16(src) || !aligned16(dst)) return MOE_ERR_INVALID_ARG;
+    // the dispatch's row copy with one slot per row: dst[dst_row[i]] = src[i]
+    GatherArgs ga{src, dst_row, dst, rows, d, 1};
+    const cudaError_t err = launch_gather(dtype, ga, num_sms(), reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err);
+}
+
 size_t moe_backward_workspace_size(const moe_config *cfg)
 {
     if (validate(cfg) != MOE_OK) return 0;

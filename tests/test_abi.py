@@ -233,3 +233,14 @@ def test_backward_validation(lib):
     small = ctypes.c_size_t(lib.moe_workspace_size(ctypes.byref(c)))
     assert lib.moe_backward(ctypes.byref(c), a, a, None, a, None, a, a, None, None, a, ctypes.c_float(0.0),
                             ctypes.c_float(0.0), ctypes.byref(full), None, ws, small, None) == 4
+
+
+def test_permute_rows_validation(lib):
+    a = ctypes.c_void_p(0x10000)
+    idx = ctypes.cast(ctypes.c_void_p(0x20000), ctypes.POINTER(ctypes.c_int32))
+    assert lib.moe_permute_rows(2, a, idx, a, 4, 8, None) == 1                       # no such dtype
+    assert lib.moe_permute_rows(1, a, idx, a, 4, 12, None) == 1                      # d not a multiple of 8
+    assert lib.moe_permute_rows(1, None, idx, a, 4, 8, None) == 1                    # src missing
+    assert lib.moe_permute_rows(1, ctypes.c_void_p(0x10008), idx, a, 4, 8, None) == 1  # src misaligned
+    assert lib.moe_permute_rows(1, a, idx, a, -1, 8, None) == 1                      # negative rows
+    assert lib.moe_permute_rows(1, None, None, None, 0, 8, None) == 0                # nothing to move
