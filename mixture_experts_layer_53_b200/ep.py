@@ -118,7 +118,11 @@ class ExpertParallelMoE:
     def forward(self, x: torch.Tensor, W_g: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor,
                 W3: Optional[torch.Tensor] = None, b1: Optional[torch.Tensor] = None,
                 b2: Optional[torch.Tensor] = None, b_e: Optional[torch.Tensor] = None):
-        """Returns (y [N, d_model], aux [1] f32: this rank's Switch loss)."""
+        """Returns (y [N, d_model], aux [1] f32: this rank's Switch loss).
+
+        b_e (sigmoid router) selects as in moe_forward; its sign-rule step
+        is left to the caller (moe_aux_loss with gamma and b_e, on this
+        rank's counts or on counts all-reduced over the group)."""
         cfg, world, E_r, g = self.cfg, self.world, self.E_r, self.group
         dev = x.device
         ids, w, probs = moe_route(cfg, x, W_g, b_e, want_probs=True)
