@@ -102,8 +102,23 @@ __device__ __forceinline__ void st16(void *p, const uint4 &v)
     *reinterpret_cast<uint4 *>(p) = v;
 }
 
-// Exact GELU (erf form) and SiLU, fp32.
-__device__ __forceinline__ float gelu_erf(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
+// erf(x) by Abramowitz & Stegun, Handbook of Mathematical Functions, formula
+// 7.1.26: for a = |x|, erf(a) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5))))
+// exp(-a^2) with t = 1 / (1 + p a), |error| <= 1.5e-7; erf is odd.  A few
+// fused multiply-adds, one fast reciprocal and one fast exponential: the
+// GELU epilogues of the expert GEMMs (results rounded to bf16) are bound by
+// this function when the k-loop is short.
+__device__ __forceinline__ float erf_as7126(float x)
+{
+    const float a = fabsf(x);
+    const float t = __fdividef(1.0f, fmaf(0.3275911f, a, 1.0f));
+    const float poly =
+        t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f), -0.284496736f), 0.254829592f);
+    return copysignf(fmaf(-poly, __expf(-a * a), 1.0f), x);
+}
+
+// GELU (erf form) and SiLU, fp32.
+__device__ __forceinline__ float gelu_erf(float v) { return 0.5f * v * (1.0f + erf_as7126(v * 0.70710678118654752f)); }
 __device__ __forceinline__ float silu(float v) { return v / (1.0f + expf(-v)); }
 
 }  // namespace moe
