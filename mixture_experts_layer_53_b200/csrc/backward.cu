@@ -155,7 +155,8 @@ __global__ void __launch_bounds__(256) row_backward_kernel(BwdActArgs a)
     }
 }
 
-// dx_n = sum_j dx_s[inv_perm[n k + j]] (fp32), one warp per token.
+// dx_n = sum_j dx_s[inv_perm[n k + j]] (+ sum_e dz[n, e] W_g[e, :]) (fp32),
+// one warp per token.
 __global__ void __launch_bounds__(256) gather_sum_kernel(BwdGatherSumArgs a)
 {
     pdl_enter();
@@ -164,6 +165,7 @@ __global__ void __launch_bounds__(256) gather_sum_kernel(BwdGatherSumArgs a)
     for (int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); n < a.N;
          n += warps) {
         const int src_l = lane < a.k ? a.inv_perm[n * a.k + lane] : 0;
+        const float dz_l = (a.dz && lane < a.E) ? a.dz[n * a.E + lane] : 0.f;
         for (int c0 = 0; c0 < a.d; c0 += 128) {  // warp-uniform; 4 columns per lane (d is a multiple of 8)
             const int c = c0 + lane * 4;
             float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -175,6 +177,27 @@ __global__ void __launch_bounds__(256) gather_sum_kernel(BwdGatherSumArgs a)
                     s.y += v.y;
                     s.z += v.z;
                     s.w += v.w;
+                }
+            }
+            if (a.dz) {
+                for (int e = 0; e < a.E; ++e) {  // fixed order over the experts
+                    const float z = __shfl_sync(0xffffffffu, dz_l, e);
+                    if (c < a.d) {
+                        const int64_t o = static_cast<int64_t>(e) * a.d + c;
+                        float4 wv;
+                        if (a.bf16) {
+                            const uint2 q = *reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(a.W_g) + o);
+                            const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&q.x);
+                            const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&q.y);
+                            wv = make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
+                        } else {
+                            wv = *reinterpret_cast<const float4 *>(static_cast<const float *>(a.W_g) + o);
+                        }
+                        s.x = fmaf(z, wv.x, s.x);
+                        s.y = fmaf(z, wv.y, s.y);
+                        s.z = fmaf(z, wv.z, s.z);
+                        s.w = fmaf(z, wv.w, s.w);
+                    }
                 }
             }
             if (c < a.d) *reinterpret_cast<float4 *>(a.dx + n * a.d + c) = s;

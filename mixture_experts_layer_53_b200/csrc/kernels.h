@@ -223,6 +223,11 @@ struct BwdGatherSumArgs {
     float *dx;                 // [N, d]
     int64_t N;
     int d, k;
+    // with dz (E <= 32): also dx_n += sum_e dz[n, e] W_g[e, :], the router's
+    // input gradient (W_g [E, d] in the layer dtype)
+    const float *dz;
+    const void *W_g;
+    int E, bf16;
 };
 cudaError_t launch_gather_sum(const BwdGatherSumArgs &a, int num_sms, cudaStream_t s);
 

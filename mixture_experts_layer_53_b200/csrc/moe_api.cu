@@ -882,15 +882,16 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *W_g, c
         MOE_TRY(GG().a(dys, 1, d, bf).b(row_w, 1, 0, 0, false).c(gr.db2, 1, 0, d).sum_rows(offsets, E, d, 1, s));
     if (!swiglu && b1 && gr.db1)
         MOE_TRY(GG().a(pre, 1, F, false).b(one, 0, 0, 0, false).c(gr.db1, 1, 0, F).sum_rows(offsets, E, F, 1, s));
-    BwdGatherSumArgs gs{dxs, inv, gr.dx, N, d, k};
-    MOE_TRY(launch_gather_sum(gs, sms, s));
-
-    // ---- router: dz, dW_g = dz^T x, dx += dz W_g
+    // ---- router: dz; dx = sum_j dx_s (+ dz W_g, folded in for E <= 32); dW_g = dz^T x
     BwdRouterArgs rb{probs, lse, ids, dw, counts, dz, N, E, k, cfg->router, cfg->norm_topk, cfg->routed_scaling,
                      aux_coef, z_coef};
     MOE_TRY(launch_router_backward(rb, sms, s));
+    const bool fold_router_dx = E <= 32;
+    BwdGatherSumArgs gs{dxs, inv, gr.dx, N, d, k, fold_router_dx ? dz : nullptr, W_g, E, bf ? 1 : 0};
+    MOE_TRY(launch_gather_sum(gs, sms, s));
     MOE_TRY(GG().split(partial).a(dz, 1, E, false).b(x, d, 1, 0, bf).c(gr.dW_g, d, 1, 0).sum_rows(doff, 1, E, d, s));
-    MOE_TRY(GG().a(dz, E, 1, false).b(W_g, d, 1, 0, bf).c(gr.dx, d, 1, 0, true).rows(doff, dmt, 1, N, d, E, s));
+    if (!fold_router_dx)
+        MOE_TRY(GG().a(dz, E, 1, false).b(W_g, d, 1, 0, bf).c(gr.dx, d, 1, 0, true).rows(doff, dmt, 1, N, d, E, s));
 
     // ---- shared expert: the same with weight 1 over all N rows of x
     if (shared) {
