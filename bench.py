@@ -110,70 +110,116 @@ def traffic_for(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 50 ms, kept for the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clocks and clock-event (throttle) reasons of one GPU, polled through
+    NVML from a background thread every `interval_ms` (default 2 ms, so that
+    even a timed region of a few tens of milliseconds holds ten or more
+    samples); `mark(t0, t1)` keeps the samples of the timed region.  Falls
+    back to `nvidia-smi -lms` when NVML is unavailable.  Reads only."""
+    SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event bits (hw_slowdown includes the power brake)
+    REASONS = (("hw_slowdown", 0x88), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
 
-    def __init__(self, gpu_index: int, interval_ms: int = 50):
-        self.gpu = gpu_index
+    def __init__(self, cuda_index: int, interval_ms: float = 2.0):
+        self.cuda_index = cuda_index
         self.interval_ms = interval_ms
-        self.proc = None
-        self.lines = []
+        self.samples = []      # (time.monotonic(), sm_mhz, reasons bitmask)
+        self.sm_max = None
+        self.source = None
         self.window = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        idx = self.cuda_index
+        try:
+            import torch
+            idx = torch.cuda._get_nvml_device_index(self.cuda_index)
+        except Exception:
+            pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(idx)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms",
-                 str(self.interval_ms), "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except OSError:
-            self.proc = None
+            nv, h = self._nvml_handle()
+            self.sm_max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.source = "nvml"
+
+            def poll():
+                while not self._stop.is_set():
+                    try:
+                        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                        self.samples.append((time.monotonic(), sm, rs))
+                    except Exception:
+                        pass
+                    time.sleep(self.interval_ms / 1000.0)
+
+            self._thread = threading.Thread(target=poll, daemon=True)
+            self._thread.start()
+        except Exception:
+            self._start_smi()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append((time.monotonic(), line.strip()))
+    def _start_smi(self):
+        try:
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.SMI_FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", str(self.cuda_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi"
+
+            def read():
+                for line in self._proc.stdout:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) < 9:
+                        continue
+                    try:
+                        sm, smax = float(parts[1]), float(parts[2])
+                    except ValueError:
+                        continue
+                    self.sm_max = smax
+                    rs = 0
+                    for (name, bit), val in zip(self.REASONS, parts[5:9]):
+                        if val.lower().startswith("active"):
+                            rs |= bit
+                    self.samples.append((time.monotonic(), sm, rs))
+
+            self._thread = threading.Thread(target=read, daemon=True)
+            self._thread.start()
+        except OSError:
+            self._proc = None
 
     def mark(self, t0: float, t1: float):
         """The timed region in time.monotonic() seconds; samples outside it are ignored."""
         self.window = (t0, t1)
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+        self._stop.set()
+        if self._proc is not None:
+            self._proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                self._proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
+                self._proc.kill()
+        if self._thread is not None and self._proc is None:
+            self._thread.join(timeout=1)
 
     def summary(self):
-        sm, smax, reasons = [], None, set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        lines = self.lines
+        samples = list(self.samples)
         if self.window is not None:
             t0, t1 = self.window
-            inside = [(t, l) for t, l in lines if t0 <= t <= t1 + self.interval_ms / 1000.0]
-            lines = inside if inside else lines
-        for _, line in lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+            samples = [s for s in samples if t0 <= s[0] <= t1]
+        if not samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.sm_max, "reasons": [], "samples": 0, "source": self.source}
+        reasons = sorted({name for _, _, rs in samples for name, bit in self.REASONS if rs & bit})
+        return {"sm_mhz": statistics.median(s[1] for s in samples), "sm_max_mhz": self.sm_max, "reasons": reasons,
+                "samples": len(samples), "source": self.source,
+                "interval_ms": self.interval_ms if self.source == "nvml" else 50}
 
 
 class OracleSample:
@@ -236,10 +282,44 @@ class OracleSample:
         return spent
 
 
+def host_info():
+    """Host core count and CPU model, reported beside every CPU timing."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model}
+
+
+class PinnedToOneCore:
+    """Runs the enclosed code with this process pinned to one host core (the
+    lowest core it may use), restoring the previous affinity afterwards."""
+
+    def __enter__(self):
+        self.core = None
+        self.prev = None
+        if hasattr(os, "sched_getaffinity"):
+            self.prev = os.sched_getaffinity(0)
+            self.core = min(self.prev)
+            os.sched_setaffinity(0, {self.core})
+        return self
+
+    def __exit__(self, *exc):
+        if self.prev is not None:
+            os.sched_setaffinity(0, self.prev)
+
+
 def cpu_baseline(wl, tokens: int):
-    """Oracle tokens/s on the first `tokens` tokens of the workload (one host core)."""
-    t = OracleSample(wl).run(list(range(tokens)))
-    return tokens / t, t
+    """Oracle tokens/s on the first `tokens` tokens of the workload, pinned to one host core."""
+    sample = OracleSample(wl)
+    with PinnedToOneCore() as pin:
+        t = sample.run(list(range(tokens)))
+    return tokens / t, t, pin.core
 
 
 def run_reference(args, wl):
@@ -256,44 +336,96 @@ def run_reference(args, wl):
         nxt += per
         return toks
 
-    for _ in range(args.warmup):
-        sampler.run(take())
-    total_t = 0.0
-    for _ in range(args.steps):
-        total_t += sampler.run(take())
+    with PinnedToOneCore() as pin:
+        for _ in range(args.warmup):
+            sampler.run(take())
+        total_t = 0.0
+        for _ in range(args.steps):
+            total_t += sampler.run(take())
     value = per * args.steps / total_t
-    sample = (f"first {per} tokens of the {wl.name} workload per step (routing + per-token expert FFNs, "
-              f"fp64, single thread); value = tokens/s over {args.steps} steps")
+    sample = (f"{per} token(s) of the {wl.name} workload per step (routing + per-token expert FFNs, "
+              f"fp64, single thread pinned to core {pin.core}); value = tokens/s over {args.steps} steps")
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": describe(wl),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": dict({"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample,
+                              "pinned_core": pin.core}, **host_info()),
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": "the fp64 oracle on the host cores of the GPU box (rank 0 only); n_gpus is the launch's size",
     }
     print(json.dumps(line), flush=True)
 
 
-def hbm_stages(wl, stages, hbm_gbs):
-    """Algorithmic bytes of the HBM-bound stages over their event-timed
-    durations (every boundary recorded: no early scheduling across them, so
-    the fractions are conservative).  route: x and W_g read, ids and weights
-    written; dispatch: x read, x_sorted written, ids read, inv_perm written;
-    combine: y_sorted, weights and inv_perm read, y written."""
+def stage_bytes(wl):
+    """Algorithmic bytes of the HBM-bound stages.  route: x and W_g read, ids
+    and weights written; dispatch: x read, x_sorted written, ids read,
+    inv_perm written; combine: y_sorted, weights and inv_perm read, y
+    written."""
     es = 4 if wl.dtype == "f32" else 2
     A = wl.N * wl.k
-    nbytes = {
+    return {
         "route": wl.N * wl.d_model * es + wl.E * wl.d_model * es + A * 8,
         "dispatch": wl.N * wl.d_model * es + A * wl.d_model * es + A * 8,
         "combine": A * wl.d_model * es + A * 8 + wl.N * wl.d_model * es,
     }
+
+
+def hbm_fracs(wl, times_us, hbm_gbs):
+    """Algorithmic bytes over measured microseconds, against the copy bandwidth."""
     out = {}
-    for k, b in nbytes.items():
-        ms = stages.get(k, 0.0)
-        gbs = b / (ms / 1000.0) / 1e9 if ms > 0 else 0.0
-        out[k] = {"bytes": b, "ms": ms, "GB/s": gbs, "frac": gbs / hbm_gbs}
+    for k, b in stage_bytes(wl).items():
+        us = times_us.get(k, 0.0)
+        gbs = b / (us / 1e6) / 1e9 if us > 0 else 0.0
+        out[k] = {"bytes": b, "us": us, "GB/s": gbs, "frac": gbs / hbm_gbs}
     return out
+
+
+def isolated_stage_times(M, cfg, wl, inp, dev, reps: int = 20, warm: int = 3):
+    """The HBM-bound entry points each timed alone: moe_route, moe_dispatch
+    (histogram, scan, row pass) and moe_combine, with L2 flushed (a 2x L2
+    write) before every launch and CUDA events right around it, so that the
+    bytes they move come from and go to HBM.  Returns mean microseconds per
+    call, over `reps` rounds after `warm` untimed ones."""
+    import ctypes
+
+    import torch
+    L = M.library()
+    A, d = wl.N * wl.k, wl.d_model
+    i32 = dict(dtype=torch.int32, device=dev)
+    ws = M.workspace(cfg, dev)
+    ids = torch.empty((wl.N, wl.k), **i32)
+    w = torch.empty((wl.N, wl.k), dtype=torch.float32, device=dev)
+    xs = torch.empty((A, d), dtype=wl.torch_dtype, device=dev)
+    inv, offsets, counts, status = (torch.empty(A, **i32), torch.empty(wl.E + 1, **i32), torch.empty(wl.E, **i32),
+                                    torch.zeros(1, **i32))
+    ys = torch.randn((A, d), device=dev).to(wl.torch_dtype)
+    y = torch.empty((wl.N, d), dtype=wl.torch_dtype, device=dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    P, st, cfgp = M._ptr, M._stream(), ctypes.byref(cfg)
+    calls = {
+        "route": lambda: L.moe_route(cfgp, P(inp["x"]), P(inp["W_g"]), P(inp["b_e"]), P(ids), P(w), None, P(ws),
+                                     ws.numel(), st),
+        "dispatch": lambda: L.moe_dispatch(cfgp, P(inp["x"]), P(ids), P(xs), None, P(inv), P(offsets), P(counts),
+                                           P(status), P(ws), ws.numel(), st),
+        "combine": lambda: L.moe_combine(cfgp, P(ys), P(w), P(inv), P(y), st),
+    }
+    ev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)] for k in calls}
+    for i in range(warm + reps):
+        for name, call in calls.items():
+            flush.fill_(i & 0xFF)
+            if i >= warm:
+                ev[name][i - warm][0].record()
+            rc = call()
+            if rc != 0:
+                raise RuntimeError(f"{name}: status {rc}")
+            if i >= warm:
+                ev[name][i - warm][1].record()
+    torch.cuda.synchronize()
+    assert int(status[0]) == 0
+    return {k: 1000.0 * sum(a.elapsed_time(b) for a, b in v) / reps for k, v in ev.items()}
 
 
 def describe(wl):
@@ -413,6 +545,9 @@ def run_native(args, wl):
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
 
+    # route, dispatch and combine each alone, L2 flushed before each launch
+    kernel_us = isolated_stage_times(M, cfg, wl, inp, dev)
+
     if rank == 0:
         peaks, peak_src = load_peaks()
         tokens = wl.N * args.steps * world
@@ -420,9 +555,9 @@ def run_native(args, wl):
         gemm1_flops = 2 * (2 if wl.act == "swiglu" else 1) * wl.d_model * wl.d_ff * wl.N * wl.k
         gemm1_s = gemm1_ms / 1000.0
         ffn_s = (stages["gemm1"] + stages["gemm2"]) / 1000.0
-        # the GEMM is timed inside a run of back-to-back steps (the power cap
-        # engages within it), so the denominator is the sustained bf16 peak;
-        # the burst fraction is reported beside it
+        # the timed region lasts well under the seconds it takes the power cap
+        # to settle, so the denominator is the burst bf16 peak; the sustained
+        # fraction is reported beside it
         burst = peaks["bf16_tflops"]
         sustained = peaks.get("bf16_tflops_sustained", burst)
         achieved = gemm1_flops / gemm1_s / 1e12
@@ -437,17 +572,23 @@ def run_native(args, wl):
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
             "config": dict(describe(wl), l2=("inputs larger than L2 (expert weights %.2f GB)" % (weights_bytes(wl) / 1e9))
                            if big_inputs else "L2 flushed between steps (256 MiB write), per-step events"),
-            "roofline": {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": sustained,
-                         "unit": "TFLOP/s", "frac": achieved / sustained,
-                         "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a run of steps)",
-                         "frac_of_burst_peak": achieved / burst,
+            "roofline": {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": burst,
+                         "unit": "TFLOP/s", "frac": achieved / burst,
+                         "peak_source": f"{peak_src} bf16_tflops (burst; timed region {total_ms:.0f} ms)",
+                         "frac_of_sustained_peak": achieved / sustained,
                          "traffic": traffic_for("gemm1", wl.name), "flops_per_launch": gemm1_flops},
             "expert_ffn": {"tflops": ffn_tflops,
                            "frac_of_measured_sustained": ffn_tflops / sustained,
                            "frac_of_measured_burst": ffn_tflops / burst,
                            "frac_of_datasheet_2250": ffn_tflops / 2250.0},
             "stages_ms": stages,
-            "hbm_stages": hbm_stages(wl, stages, peaks["hbm_gbs"]),
+            # each stage inside a forward, every boundary recorded (launch
+            # latency included, L2 left warm by the previous stage)
+            "hbm_stages": hbm_fracs(wl, {k: 1000.0 * v for k, v in stages.items()}, peaks["hbm_gbs"]),
+            # each entry point alone, L2 flushed before it: moe_route (one
+            # kernel for E <= 32), moe_dispatch (histogram + scan + row pass),
+            # moe_combine
+            "hbm_kernels": hbm_fracs(wl, kernel_us, peaks["hbm_gbs"]),
             "e2e": {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s",
                     "h2d_bytes_per_step": inp["x"].numel() * inp["x"].element_size(),
                     "d2h_bytes_per_step": out["y"].numel() * out["y"].element_size() + 4},
@@ -456,10 +597,11 @@ def run_native(args, wl):
         }
         if not args.no_cpu_baseline and world == 1:
             per = min(REF_TOKENS_PER_STEP.get(wl.name, 4) * 16, wl.N)
-            v, dt = cpu_baseline(wl, per)
-            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                    "sample": f"first {per} tokens of the workload, routing + per-token expert "
-                                              f"FFNs in fp64 on one host core ({dt:.1f} s)"}
+            v, dt, core = cpu_baseline(wl, per)
+            line["cpu_baseline"] = dict({
+                "value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "pinned_core": core,
+                "sample": f"first {per} tokens of the workload, routing + per-token expert FFNs in fp64, one "
+                          f"thread pinned to host core {core} ({dt:.1f} s)"}, **host_info())
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -554,8 +696,26 @@ def run_backward(args, wl):
     print(json.dumps(line), flush=True)
 
 
+def relaunch_under_torchrun(args) -> int:
+    """`--gpus N` (N > 1) outside torchrun: run this script again as N ranks
+    on this node, one per GPU, and return their exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     args = parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch_under_torchrun(args))
+    _, _, world = dist_env()
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE {world}; reporting the launched {world}",
+              file=sys.stderr)
     import workloads as W
     wl = W.WORKLOADS[args.workload]
     if args.tokens:

@@ -40,9 +40,13 @@
  *   clears it itself).  The library never traps.
  * Limits.  1 <= k <= min(E, 16); E <= 256; d_model and d_ff multiples of 8;
  *   N*k < 2^31; every pointer 16-byte aligned.
- * Threading.  No global mutable state besides a per-device attribute cache;
- *   calls on different streams may run concurrently with separate
- *   workspaces.
+ * Threading.  Host-side state is limited to caches filled on first use and
+ *   guarded by mutexes: per-device attributes (SM count, shared-memory
+ *   opt-ins, occupancy), the driver entry points, and the device address of
+ *   moe_dispatch_noalloc's scratch array.  Calls on different streams may run
+ *   concurrently with separate workspaces.  The one piece of global DEVICE
+ *   state is that scratch array: moe_dispatch_noalloc calls share it (see
+ *   there); every other entry point touches only the caller's memory.
  */
 #ifndef MOE_H
 #define MOE_H
@@ -153,9 +157,11 @@ MOE_API size_t moe_workspace_size(const moe_config *cfg);
  * selection score first (ties: lowest id), and their weights (times
  * routed_scaling).  b_e (sigmoid router only, may be NULL) enters the
  * selection score only, never the weights (sec. 2.5).  probs [N, E] (may be
- * NULL) receives softmax(z_n) for every router.  The workspace holds the
- * bf16 path's fp32 logits between its two kernels (tensor-core logits, then
- * one warp per token for scores, top-k and gates).
+ * NULL) receives softmax(z_n) for every router.  bf16 with E <= 32 runs as
+ * one kernel (tensor-core logits split over d across a thread-block cluster,
+ * selection fused); bf16 with E > 32 keeps partial logits in the workspace
+ * between the logits kernel and the selection kernel; fp32 runs one CUDA-core
+ * kernel.
  */
 MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const void *W_g,
                      const float *b_e, int32_t *topk_ids, float *topk_w,
@@ -169,8 +175,9 @@ MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const void *W
  * x_sorted[i] = x[perm[i] / k], counts[e] = assignments to e,
  * offsets[e] = start of expert e's slice (offsets[0] = 0, offsets[E] = N*k).
  * perm, x and x_sorted may be NULL (then that output is skipped).  An
- * expert id outside [0, E) sets MOE_ERR_BAD_EXPERT_ID in dev_status; the
- * outputs are then unspecified.
+ * expert id outside [0, E) sets MOE_ERR_BAD_EXPERT_ID in dev_status; that
+ * assignment is left out of counts and offsets, gets inv_perm = -1 and no
+ * row, and every valid assignment keeps its stable position.
  */
 MOE_API moe_status moe_dispatch(const moe_config *cfg, const void *x,
                         const int32_t *topk_ids, void *x_sorted, int32_t *perm,
@@ -197,11 +204,14 @@ MOE_API moe_status moe_dispatch(const moe_config *cfg, const void *x,
  * library until the process exits); a larger problem returns
  * MOE_ERR_WORKSPACE and enqueues nothing.  Nothing is allocated, here or
  * later.  The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it: make that
- * first call before any stream capture.  Every call uses the same array, so
- * calls whose work overlaps on the GPU (e.g. on two streams) race: order them.
- * Each call overwrites all the scratch it later reads, so earlier contents
- * never matter.
+ * (cudaGetSymbolAddress, with that device current) and caches it with the
+ * id of the device's context: make that first call before any stream
+ * capture.  A call that finds a different context current (after
+ * cudaDeviceReset) looks the address up again; so does every call made from
+ * a thread on which no context is current yet.  Every call uses the same
+ * array, so calls whose work overlaps on the GPU (e.g. on two streams) race:
+ * order them.  Each call overwrites all the scratch it later reads, so
+ * earlier contents never matter.
  */
 MOE_API moe_status moe_dispatch_noalloc(const moe_config *cfg, const void *x,
                                 const int32_t *topk_ids, void *x_sorted,

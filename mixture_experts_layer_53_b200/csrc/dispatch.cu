@@ -316,7 +316,10 @@ __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a)
     __syncthreads();
     for (int q = threadIdx.x; q < nas; q += blockDim.x) {
         const int e = ids_s[q];
-        if (e < 0 || e >= a.E) continue;  // reported by the histogram pass
+        if (e < 0 || e >= a.E) {  // reported by the histogram pass; no position
+            a.inv_perm[a0 + q] = -1;
+            continue;
+        }
         int rank = 0;
         for (int r = 0; r < q; ++r) rank += (ids_s[r] == e);
         const int pos = a.offsets[e] + a.chunk_base[c * a.E + e] + rank;

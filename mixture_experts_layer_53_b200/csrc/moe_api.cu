@@ -9,22 +9,23 @@
 #include <string>
 
 #include "../../include/moe.h"
+#include "api_internal.h"
 #include "common.cuh"
 #include "kernels.h"
 
 namespace {
-
-using namespace moe;
-
 thread_local std::string g_last_error;
+}  // namespace
 
-moe_status cuda_fail(cudaError_t err)
+namespace moe {
+
+moe_status record_cuda_error(cudaError_t err)
 {
     g_last_error = cudaGetErrorString(err);
     return MOE_ERR_CUDA;
 }
 
-int num_sms()
+int device_sms()
 {
     static std::mutex mu;
     static int cache[64] = {0};
@@ -39,11 +40,7 @@ int num_sms()
     return cache[dev];
 }
 
-size_t elem_size(const moe_config *c) { return c->dtype == MOE_F32 ? 4 : 2; }
-
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-moe_status validate(const moe_config *c)
+moe_status validate_config(const moe_config *c)
 {
     if (!c) return MOE_ERR_INVALID_ARG;
     if (c->N < 0 || c->d_model <= 0 || c->d_ff <= 0 || c->E <= 0 || c->k <= 0) return MOE_ERR_INVALID_ARG;
@@ -59,6 +56,56 @@ moe_status validate(const moe_config *c)
     if (c->N * static_cast<int64_t>(c->k) >= (static_cast<int64_t>(1) << 31)) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
+
+namespace {
+bool aligned16_(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+}  // namespace
+
+moe_status check_dispatch_args(const moe_config *c, const void *x, const int32_t *topk_ids, const void *x_sorted,
+                               const int32_t *inv_perm, const int32_t *offsets, const int32_t *counts)
+{
+    const bool empty = c->N == 0;
+    if (!offsets || !counts || (!empty && (!topk_ids || !inv_perm))) return MOE_ERR_INVALID_ARG;
+    if ((x == nullptr) != (x_sorted == nullptr)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16_(x) || !aligned16_(x_sorted)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+cudaError_t enqueue_dispatch(const moe_config *c, const void *x, const int32_t *topk_ids, void *x_sorted,
+                             int32_t *perm, int32_t *inv_perm, int32_t *offsets, int32_t *counts,
+                             int32_t *dev_status, int32_t *hist, cudaStream_t s)
+{
+    cudaError_t err;
+    HistArgs h{topk_ids, nullptr, hist, nullptr, dev_status, c->N, c->E, c->k};
+    if ((err = launch_hist(h, s)) != cudaSuccess) return err;
+    ScanArgs sc{};
+    sc.hist = hist;
+    sc.chunks = num_chunks(c->N);
+    sc.N = c->N;
+    sc.E = c->E;
+    sc.k = c->k;
+    sc.counts = counts;
+    sc.offsets = offsets;
+    if ((err = launch_scan(sc, s)) != cudaSuccess) return err;
+    if (x) {  // positions and rows in one pass
+        DispatchRowsArgs da{topk_ids, hist, offsets, perm, inv_perm, x, x_sorted, c->N, c->d_model, c->E, c->k};
+        return launch_dispatch_rows(c->dtype, da, device_sms(), s);
+    }
+    ScatterArgs sa{topk_ids, hist, perm, inv_perm, c->N, c->E, c->k, offsets};
+    return launch_scatter(sa, s);
+}
+
+}  // namespace moe
+
+namespace {
+
+using namespace moe;
+
+moe_status cuda_fail(cudaError_t err) { return record_cuda_error(err); }
+int num_sms() { return device_sms(); }
+moe_status validate(const moe_config *c) { return validate_config(c); }
+size_t elem_size(const moe_config *c) { return c->dtype == MOE_F32 ? 4 : 2; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct Layout {
     size_t hist, psum, zpart, logits, pe, offsets, mt, shoff, shmt, counts, ids, w, perm, inv, xs, h, ys, ysh,
@@ -431,35 +478,11 @@ moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *top
 {
     moe_status st = validate(cfg);
     if (st != MOE_OK) return st;
-    const bool empty = cfg->N == 0;
-    if (!offsets || !counts || (!empty && (!topk_ids || !inv_perm))) return MOE_ERR_INVALID_ARG;
-    if ((x == nullptr) != (x_sorted == nullptr)) return MOE_ERR_INVALID_ARG;
-    if ((x && !aligned16(x)) || (x_sorted && !aligned16(x_sorted))) return MOE_ERR_INVALID_ARG;
+    if ((st = check_dispatch_args(cfg, x, topk_ids, x_sorted, inv_perm, offsets, counts)) != MOE_OK) return st;
     if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const Layout L = layout(cfg);
-    int32_t *hist = at<int32_t>(ws, L.hist);
-    cudaError_t err;
-    HistArgs h{topk_ids, nullptr, hist, nullptr, dev_status, cfg->N, cfg->E, cfg->k};
-    if ((err = launch_hist(h, s)) != cudaSuccess) return cuda_fail(err);
-    ScanArgs sc{};
-    sc.hist = hist;
-    sc.chunks = num_chunks(cfg->N);
-    sc.N = cfg->N;
-    sc.E = cfg->E;
-    sc.k = cfg->k;
-    sc.counts = counts;
-    sc.offsets = offsets;
-    if ((err = launch_scan(sc, s)) != cudaSuccess) return cuda_fail(err);
-    if (x) {  // positions and rows in one pass
-        DispatchRowsArgs da{topk_ids, hist, offsets, perm, inv_perm, x, x_sorted, cfg->N, cfg->d_model, cfg->E,
-                            cfg->k};
-        if ((err = launch_dispatch_rows(cfg->dtype, da, num_sms(), s)) != cudaSuccess) return cuda_fail(err);
-    } else {
-        ScatterArgs sa{topk_ids, hist, perm, inv_perm, cfg->N, cfg->E, cfg->k, offsets};
-        if ((err = launch_scatter(sa, s)) != cudaSuccess) return cuda_fail(err);
-    }
-    return MOE_OK;
+    const cudaError_t err = enqueue_dispatch(cfg, x, topk_ids, x_sorted, perm, inv_perm, offsets, counts, dev_status,
+                                             at<int32_t>(ws, layout(cfg).hist), reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err);
 }
 
 moe_status moe_expert_ffn(const moe_config *cfg, const void *x_sorted, const int32_t *offsets, const void *W1,

@@ -23,6 +23,8 @@ What pins what:
                                          E=k=1 plain FFN
   brute force over all subsets           selection on tiny random cases
   invariants                             sum w, counts, bijection, stability
+  C per-token loop and numpy             forward_tokens (sampled-token y at
+                                         full size), bit for bit / to 1e-12
 """
 from __future__ import annotations
 
@@ -539,5 +541,46 @@ def pin_aux_gradient_is_E_f_over_N(L):
     g = O.backward(x, Wg, k, W1, W2, np.zeros((N, d)), aux_coef=1.0, L=L)
     _close(g["dWg"], dz.T @ x, 1e-12, "dW_g of the Switch loss")
     _close(g["dW1"], np.zeros_like(W1), 0.0, "no expert gradient without dy")
+
+def pin_forward_tokens(L, forward_tokens=None):
+    """The per-token loop for sampled tokens (``oracle.forward_tokens``, the
+    oracle of y at full size) equals the C per-token loop
+    ``oracle_dense_forward`` bit for bit, and numpy's float64 restatement
+    y_n = sum_j w_nj Expert_{e_nj}(x_n) (course module sec. 2.1) to 1e-12.
+    Problems: k = 8 with experts shared across tokens and one idle expert, a
+    GELU layer with biases, a single token with k = 1, and slot weights that
+    differ per slot (so a slot swap shows)."""
+    fwd = forward_tokens or O.forward_tokens
+    rng = np.random.default_rng(29)
+    cases = (("swiglu", False, 9, 10, 8), ("gelu", True, 6, 7, 3), ("swiglu", True, 1, 4, 1))
+    for act, biases, S, E, k in cases:
+        d, F = 12, 10
+        x, _, W1, W2, W3, b1, b2 = _rand_problem(rng, S, d, F, E, act, biases)
+        if act == "swiglu":
+            b1 = None  # SwiGLU experts carry no hidden bias
+        idle = E // 2
+        pool = [e for e in range(E) if e != idle]
+        ids = np.stack([rng.permutation(pool)[:k] for _ in range(S)]).astype(np.int32)
+        w = rng.uniform(0.05, 1.0, (S, k))
+        fetched = []
+
+        def getter(e):
+            fetched.append(e)
+            return {"W1": W1[e], "W2": W2[e], "W3": None if W3 is None else W3[e],
+                    "b1": None if b1 is None else b1[e], "b2": None if b2 is None else b2[e]}
+
+        got = fwd(x, ids, w, getter, act, L=L)
+        assert idle not in fetched, "an expert no token chose was evaluated"
+        want = O.dense_forward(x, ids, w, W1, W2, act, W3, b1, b2, L=L)
+        assert np.array_equal(got, want), f"forward_tokens != dense_forward bitwise ({act}, k={k})"
+        ref = np.zeros((S, d))
+        for s_ in range(S):
+            for j in range(k):
+                e = int(ids[s_, j])
+                ref[s_] += w[s_, j] * np_expert(x[s_:s_ + 1], W1[e], W2[e], act, None if W3 is None else W3[e],
+                                                None if b1 is None else b1[e], None if b2 is None else b2[e])[0]
+        scale = np.max(np.abs(ref))
+        _close(got / scale, ref / scale, 1e-12, f"forward_tokens vs numpy ({act}, k={k})")
+
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

@@ -90,6 +90,50 @@ def expert_getter(inp):
     return get
 
 
+def ffn_tile_m(wl: W.Workload) -> int:
+    """Rows per m-tile of the library's expert GEMMs for this workload: 256
+    (CTA pairs) for bf16 when the experts average more than 192 rows, else
+    128 (the rule the library states for its grouped GEMM)."""
+    return 256 if wl.dtype == "bf16" and wl.N * wl.k / wl.E > 192 else 128
+
+
+def tile_rows(offsets: np.ndarray, tile_m: int) -> np.ndarray:
+    """Sorted rows that start every (expert, m-tile) of the grouped GEMM's
+    tile schedule -- tile t of expert e starts at offsets[e] + t * tile_m --
+    plus each non-empty expert's last row."""
+    rows = []
+    for e in range(len(offsets) - 1):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi > lo:
+            rows.extend(range(lo, hi, tile_m))
+            rows.append(hi - 1)
+    return np.unique(np.asarray(rows, dtype=np.int64))
+
+
+def covering_tokens(ids: np.ndarray, E: int, tile_m: int, budget: int) -> np.ndarray:
+    """Tokens whose routed rows touch as many (expert, m-tile) pairs of the
+    tile schedule as possible, at most `budget` of them (greedy set cover;
+    ties to the lowest token).  Each token's k rows sit at their sorted
+    positions; a tile counts as touched by any of its rows."""
+    dp = O.dispatch(ids, E)
+    N, k = ids.shape
+    inv = dp["inv_perm"].reshape(N, k)
+    off = dp["offsets"]
+    expert_of = np.searchsorted(off, inv, side="right") - 1
+    tile_of = expert_of.astype(np.int64) * (1 << 32) + (inv - off[expert_of]) // tile_m
+    need = set(np.unique(tile_of).tolist())
+    chosen = []
+    covers = [set(tile_of[n].tolist()) for n in range(N)]
+    while need and len(chosen) < budget:
+        best = max(range(N), key=lambda n: (len(covers[n] & need), -n))
+        gain = covers[best] & need
+        if not gain:
+            break
+        chosen.append(best)
+        need -= gain
+    return np.unique(np.asarray(chosen, dtype=np.int64))
+
+
 def sample_tokens(N: int, count: int, seed: int = 0) -> np.ndarray:
     if count >= N:
         return np.arange(N)

@@ -14,8 +14,8 @@ import torch
 import mixture_experts_layer_53_b200 as M
 import oracle as O
 import workloads as W
-from parity import (MARGIN, TOL_Y, check_forward, config_of, gpu_forward, np64, oracle_routing,
-                    sample_tokens)
+from parity import (MARGIN, TOL_Y, check_forward, config_of, covering_tokens, ffn_tile_m, gpu_forward, np64,
+                    oracle_routing, tile_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -44,7 +44,10 @@ SMALL = {
     "fused_e32_sigmoid": W.WORKLOADS["deepseek_v3"].scaled(N=130, d_model=192, d_ff=128, E=32, k=8),
 }
 
-FULL_SAMPLES = {"tiny_fp32": None, "gpt2_moe": 24, "mixtral": 8, "deepseek_v3": 4, "qwen3_skew": 12}
+# Token budgets for y at full size: tokens are chosen so that their routed
+# rows touch as many (expert, m-tile) pairs of the GEMM tile schedule as the
+# budget allows (None: every token).
+FULL_BUDGET = {"tiny_fp32": None, "gpt2_moe": 48, "mixtral": 40, "deepseek_v3": 48, "qwen3_skew": 96}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -69,11 +72,52 @@ def test_forward_full_size(name):
     wl = W.WORKLOADS[name]
     inp = W.make_inputs(wl, DEV)
     gpu = gpu_forward(wl, inp)
-    n = FULL_SAMPLES[name]
-    tokens = None if n is None else sample_tokens(wl.N, n, seed=wl.seed)
+    n = FULL_BUDGET[name]
+    tokens = None
+    if n is not None:
+        tokens = covering_tokens(gpu["topk_ids"], wl.E, ffn_tile_m(wl), n)
+        tokens = np.union1d(tokens, [0, wl.N - 1])
     rep = check_forward(wl, inp, gpu, y_tokens=tokens)
     print(name, rep.as_dict())
     del inp
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["gpt2_moe", "mixtral", "deepseek_v3", "qwen3_skew"])
+def test_expert_ffn_full_size_rows(name):
+    """moe_expert_ffn at full size on the forward's own x_sorted and offsets
+    (moe_route + moe_dispatch), in the tile configuration the benchmark runs:
+    the first row of every (expert, m-tile) and each expert's last row are
+    compared with the oracle's expert FFN, row by row."""
+    wl = W.WORKLOADS[name]
+    inp = W.make_inputs(wl, DEV)
+    cfg = config_of(wl)
+    ws = M.workspace(cfg, DEV)
+    ids, _, _ = M.moe_route(cfg, inp["x"], inp["W_g"], b_e=inp["b_e"], ws=ws)
+    d = M.moe_dispatch(cfg, ids, x=inp["x"], ws=ws)
+    ys = M.moe_expert_ffn(cfg, d["x_sorted"], d["offsets"], inp["W1"], inp["W2"], b1=inp["b1"], W3=inp["W3"],
+                          b2=inp["b2"], ws=ws)
+    torch.cuda.synchronize()
+    offsets = d["offsets"].cpu().numpy()
+    rows = tile_rows(offsets, ffn_tile_m(wl))
+    expert_of = np.searchsorted(offsets, rows, side="right") - 1
+    worst, checked = 0.0, 0
+    for e in np.unique(expert_of):
+        sel = rows[expert_of == e]
+        ew = {"W1": np64(inp["W1"][e]), "W2": np64(inp["W2"][e]),
+              "W3": None if inp["W3"] is None else np64(inp["W3"][e]),
+              "b1": None if inp["b1"] is None else np64(inp["b1"][e]),
+              "b2": None if inp["b2"] is None else np64(inp["b2"][e])}
+        xr = np64(d["x_sorted"][torch.from_numpy(sel).to(DEV)])
+        yr = np64(ys[torch.from_numpy(sel).to(DEV)])
+        for i in range(len(sel)):
+            ref = O.expert_ffn(xr[i], ew["W1"], ew["W2"], wl.act, ew["b1"], ew["W3"], ew["b2"])
+            worst = max(worst, float(np.max(np.abs(yr[i] - ref)) / max(np.max(np.abs(ref)), 1e-30)))
+            checked += 1
+    print(name, {"rows_checked": checked, "tile_m": ffn_tile_m(wl), "max_rel_err": worst})
+    assert checked == len(rows)
+    assert worst <= TOL_Y[wl.dtype], worst
+    del inp, ws, ys, d
     torch.cuda.empty_cache()
 
 

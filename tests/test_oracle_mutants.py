@@ -10,13 +10,15 @@ tanh GELU, the wrong SwiGLU operand, an unstable sort, a wrong P).
 The planted copies are compiled to a temporary directory on the CPU; the
 oracle under ``oracle/`` is never modified.
 """
+import inspect
 import os
 import subprocess
+import textwrap
 
 import pytest
 
 import oracle as O
-from oracle_pins import ALL_PINS
+from oracle_pins import ALL_PINS, pin_forward_tokens
 
 SRC = os.path.join(os.path.dirname(O.__file__), "moe_oracle.c")
 
@@ -99,3 +101,28 @@ def test_mutant_is_caught(name, source, tmp_path):
         except (AssertionError, O.OracleError, FloatingPointError, ValueError, IndexError):
             failed.append(pin.__name__)
     assert failed, f"mutant {name} passed every pin"
+
+
+# Mistakes planted in a copy of oracle.forward_tokens (plain Python): the
+# per-token loop the full-size parity tests use for y on sampled tokens.
+FORWARD_TOKENS_MUTANTS = {
+    "slot_weights_swapped": ("y[s] += w[s, j] * outs[(s, j)]", "y[s] += w[s, k - 1 - j] * outs[(s, j)]"),
+    "other_slot_output": ("y[s] += w[s, j] * outs[(s, j)]", "y[s] += w[s, j] * outs[(s, (j + 1) % k)]"),
+    "wrong_expert_fetched": ("ew = expert_weights(e)", "ew = expert_weights(sorted(by_expert)[0])"),
+    "wrong_token_row": ("outs[(s, j)] = expert_ffn(x_rows[s],", "outs[(s, j)] = expert_ffn(x_rows[(s + 1) % S],"),
+    "key_transposed": ("by_expert.setdefault(int(ids[s, j]), []).append((s, j))",
+                       "by_expert.setdefault(int(ids[s, j]), []).append((j % S, s % k))"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FORWARD_TOKENS_MUTANTS))
+def test_forward_tokens_mutant_is_caught(name):
+    old, new = FORWARD_TOKENS_MUTANTS[name]
+    src = textwrap.dedent(inspect.getsource(O.forward_tokens))
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    scope = dict(vars(O))
+    exec(compile(src.replace(old, new), "<mutant>", "exec"), scope)
+    L = O.load()
+    pin_forward_tokens(L)  # the real function passes
+    with pytest.raises((AssertionError, KeyError, IndexError, ValueError)):
+        pin_forward_tokens(L, forward_tokens=scope["forward_tokens"])
