@@ -332,6 +332,45 @@ MOE_API moe_status moe_forward_ex(const moe_config *cfg, const void *x, const vo
                           void *const *stage_events, moe_stream_t stream);
 
 /*
+ * The forward of one data-parallel rank (course module sec. 2.3 and 2.5: the
+ * Switch loss and the sign rule are defined over the whole batch, which a
+ * data-parallel layer splits across ranks).  Runs the layer like
+ * moe_forward_ex on this call's N tokens and, instead of the local loss,
+ * returns the two partials the whole-batch loss is made of:
+ *   counts   [E] int32   assignments to each expert (required),
+ *   psum_out [E] float64 sum over this call's tokens of p_{n,e} = softmax(z_n)
+ *                        (required, 8-byte aligned; summed in fp64 in a fixed
+ *                        order).
+ * Summed over the ranks (an all-reduce of each; sums of integers and of the
+ * rank totals), they go to moe_aux_from_partials.  b_e (sigmoid router, may
+ * be NULL) selects only and is not moved here: its sign-rule step needs the
+ * whole batch's load.  Every other argument is that of moe_forward_ex.
+ */
+MOE_API moe_status moe_forward_partials(const moe_config *cfg, const void *x, const void *W_g,
+                                        const float *b_e, const void *W1, const void *b1,
+                                        const void *W3, const void *W2, const void *b2,
+                                        const moe_shared_expert *shared, void *y,
+                                        int32_t *topk_ids, float *topk_w, int32_t *counts,
+                                        double *psum_out, float *z_loss_out, int32_t *dev_status,
+                                        void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * The whole batch's Switch loss and sign-rule step from partials summed over
+ * forwards (course module sec. 2.3, sec. 2.5): with counts [E] int32 and
+ * psum [E] float64 (8-byte aligned) the sums over every rank's
+ * moe_forward_partials, N = sum_e counts[e] / k (each token makes exactly k
+ * assignments) and
+ *   aux_out   = E sum_e counts[e] psum[e] / N^2   (float; 0 when N = 0),
+ *   b_e_inout += gamma sign(N k - E counts[e])    (if gamma > 0 and given).
+ * Either output may be NULL, not both.  Device pointers; one small kernel on
+ * `stream`, reduced in fp64 in a fixed order, so ranks that pass the same
+ * sums get the same bits.  Limits as moe_config (E <= 256, k <= min(E, 16)).
+ */
+MOE_API moe_status moe_aux_from_partials(int32_t E, int32_t k, const int32_t *counts,
+                                         const double *psum, float *aux_out, float gamma,
+                                         float *b_e_inout, moe_stream_t stream);
+
+/*
  * Gradients written by moe_backward: fp32, row-major, caller-owned device
  * memory, 16-byte aligned (else MOE_ERR_INVALID_ARG), each overwritten (not
  * accumulated).  Shapes as the parameters:

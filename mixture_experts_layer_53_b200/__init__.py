@@ -37,7 +37,8 @@ STAGE_NAMES = ("route", "dispatch", "gemm1", "gemm2", "combine")
 EXPORTS = ("moe_status_string", "moe_last_error", "moe_version", "moe_workspace_size", "moe_route",
            "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_combine", "moe_aux_loss",
            "moe_forward", "moe_shared_ffn", "moe_combine_shared", "moe_router_z_loss", "moe_forward_ex",
-           "moe_backward_workspace_size", "moe_backward", "moe_permute_rows", "moe_selftest_wait_timeout")
+           "moe_backward_workspace_size", "moe_backward", "moe_permute_rows", "moe_selftest_wait_timeout",
+           "moe_forward_partials", "moe_aux_from_partials")
 # ceil(N / 32) * E limit of moe_dispatch_noalloc (MOE_NOALLOC_DISPATCH_MAX_SLOTS)
 NOALLOC_DISPATCH_MAX_SLOTS = 1 << 19
 
@@ -122,6 +123,11 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_forward_ex.argtypes = [cfgp, vp, vp, f32p, ctypes.c_float, vp, vp, vp, vp, vp, shp, vp, i32p, f32p,
                                    i32p, f32p, f32p, i32p, vp, sz, ctypes.c_void_p, vp]
     lib.moe_forward_ex.restype = st
+    lib.moe_forward_partials.argtypes = [cfgp, vp, vp, f32p, vp, vp, vp, vp, vp, shp, vp, i32p, f32p, i32p, vp,
+                                         f32p, i32p, vp, sz, vp]
+    lib.moe_forward_partials.restype = st
+    lib.moe_aux_from_partials.argtypes = [ctypes.c_int32, ctypes.c_int32, i32p, vp, f32p, ctypes.c_float, f32p, vp]
+    lib.moe_aux_from_partials.restype = st
     lib.moe_backward_workspace_size.argtypes = [cfgp]
     lib.moe_backward_workspace_size.restype = sz
     lib.moe_backward.argtypes = [cfgp, vp, vp, f32p, vp, vp, vp, vp, vp, shp, vp, ctypes.c_float, ctypes.c_float,
@@ -508,6 +514,46 @@ class HostPipeline:
             e.synchronize()
 
 
+def moe_forward_partials(cfg: MoeConfig, x: torch.Tensor, W_g: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor,
+                         W3: Optional[torch.Tensor] = None, b1: Optional[torch.Tensor] = None,
+                         b2: Optional[torch.Tensor] = None, b_e: Optional[torch.Tensor] = None,
+                         ws: Optional[torch.Tensor] = None, out: Optional[Dict[str, torch.Tensor]] = None,
+                         stream=None, shared: Optional[Dict[str, Optional[torch.Tensor]]] = None,
+                         z_loss: bool = False) -> Dict[str, torch.Tensor]:
+    """One data-parallel rank's forward: y, topk_ids, topk_w, status, (z) and
+    the Switch-loss partials counts [E] int32 and psum [E] float64 (sum over
+    this call's tokens of softmax(z_n)).  b_e selects only and is not moved."""
+    dev = x.device
+    ws = ws if ws is not None else workspace(cfg, dev)
+    if out is None:
+        out = forward_outputs(cfg, dev)
+    if "psum" not in out:
+        out["psum"] = torch.empty(cfg.E, dtype=torch.float64, device=dev)
+    sh = _shared_struct(shared)
+    rc = library().moe_forward_partials(ctypes.byref(cfg), _ptr(x), _ptr(W_g), _ptr(b_e), _ptr(W1), _ptr(b1),
+                                        _ptr(W3), _ptr(W2), _ptr(b2), ctypes.byref(sh) if sh else None,
+                                        _ptr(out["y"]), _ptr(out["topk_ids"]), _ptr(out["topk_w"]),
+                                        _ptr(out["counts"]), _ptr(out["psum"]), _ptr(out["z"]) if z_loss else None,
+                                        _ptr(out["status"]), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "moe_forward_partials")
+    return out
+
+
+def moe_aux_from_partials(E: int, k: int, counts: torch.Tensor, psum: torch.Tensor, gamma: float = 0.0,
+                          b_e: Optional[torch.Tensor] = None, aux: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """Whole-batch Switch loss [1] f32 from summed partials (counts int32 [E],
+    psum float64 [E]); with gamma > 0 moves b_e in place by the sign rule on
+    the whole batch's load."""
+    if counts.dtype != torch.int32 or psum.dtype != torch.float64:
+        raise ValueError("moe_aux_from_partials: counts int32 [E] and psum float64 [E]")
+    aux = aux if aux is not None else torch.empty(1, dtype=torch.float32, device=counts.device)
+    rc = library().moe_aux_from_partials(int(E), int(k), _ptr(counts), _ptr(psum), _ptr(aux), float(gamma),
+                                         _ptr(b_e), _stream(stream))
+    _check(rc, "moe_aux_from_partials")
+    return aux
+
+
 def forward_outputs(cfg: MoeConfig, device) -> Dict[str, torch.Tensor]:
     return {
         "y": torch.empty((cfg.N, cfg.d_model), dtype=cfg.torch_dtype, device=device),
@@ -523,5 +569,6 @@ def forward_outputs(cfg: MoeConfig, device) -> Dict[str, torch.Tensor]:
 __all__ = ["MoeConfig", "SharedExpert", "MoeError", "make_config", "library", "workspace", "moe_workspace_size",
            "moe_route", "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_combine", "moe_aux_loss",
            "moe_forward", "moe_shared_ffn", "moe_combine_shared", "moe_router_z_loss", "moe_backward",
+           "moe_forward_partials", "moe_aux_from_partials",
            "MoeGrads", "forward_outputs",
            "StageEvents", "HostPipeline", "EXPORTS", "LIB_PATH"]

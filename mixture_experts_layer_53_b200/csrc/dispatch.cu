@@ -277,6 +277,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_small_kernel(ScanArgs a)
         if (lane < E) {
             a.offsets[lane] = incl - cnt;
             if (a.counts) a.counts[lane] = cnt;
+            if (a.psum && a.pe) a.pe[lane] = pe_s[lane];
             if (a.mt_prefix) a.mt_prefix[lane] = mincl - mt;
             if (a.b_e && a.gamma > 0.f) {
                 const long long diff = static_cast<long long>(a.N) * a.k - static_cast<long long>(E) * cnt;
@@ -300,6 +301,45 @@ __global__ void __launch_bounds__(kScanThreads) scan_small_kernel(ScanArgs a)
         }
     }
     if (a.z_out && a.zpart) reduce_z_loss(a.zpart, a.chunks, a.N, a.z_out);  // block-uniform
+}
+
+// Switch loss and sign-rule step from partials summed over several forwards
+// (course module sec. 2.3: L = E sum_e f_e P_e over the whole batch; sec.
+// 2.5: the sign rule on the whole batch's load).  One CTA; the same fixed
+// reduction order as scan_finalize_kernel.
+__global__ void __launch_bounds__(kScanThreads) aux_partials_kernel(AuxPartialsArgs a)
+{
+    pdl_enter();
+    const int E = a.E, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int cnt = t < E ? a.counts[t] : 0;
+    __shared__ long long csum[kScanThreads / 32];
+    __shared__ double wsum[kScanThreads / 32];
+    long long c = cnt;
+    double term = t < E ? static_cast<double>(cnt) * a.psum[t] : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        c += __shfl_xor_sync(0xffffffffu, c, o);
+        term += __shfl_xor_sync(0xffffffffu, term, o);
+    }
+    if (lane == 0) {
+        csum[warp] = c;
+        wsum[warp] = term;
+    }
+    __syncthreads();
+    long long total = 0;  // N k assignments
+    double s = 0.0;
+    for (int w = 0; w < kScanThreads / 32; ++w) {
+        total += csum[w];
+        s += wsum[w];
+    }
+    if (t < E && a.b_e && a.gamma > 0.f) {
+        const long long diff = total - static_cast<long long>(E) * cnt;
+        a.b_e[t] += a.gamma * static_cast<float>((diff > 0) - (diff < 0));
+    }
+    if (t == 0 && a.aux_out) {
+        const double Nd = static_cast<double>(total) / static_cast<double>(a.k);
+        *a.aux_out = total == 0 ? 0.0f : static_cast<float>(s * static_cast<double>(E) / (Nd * Nd));
+    }
 }
 
 // ---------------------------------------------------------------- scatter
@@ -566,6 +606,12 @@ cudaError_t launch_scan(const ScanArgs &a, cudaStream_t s)
     cudaError_t err = launch_k(scan_cols_kernel, dim3(a.E), dim3(kScanThreads), 0, s, a);
     if (err != cudaSuccess) return err;
     return launch_k(scan_finalize_kernel, dim3(1), dim3(kScanThreads), 0, s, a);
+}
+
+cudaError_t launch_aux_partials(const AuxPartialsArgs &a, cudaStream_t s)
+{
+    if (a.E > kScanThreads) return cudaErrorInvalidValue;
+    return launch_k(aux_partials_kernel, dim3(1), dim3(kScanThreads), 0, s, a);
 }
 
 cudaError_t launch_scatter(const ScatterArgs &a, cudaStream_t s)

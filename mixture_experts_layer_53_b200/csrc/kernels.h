@@ -90,7 +90,7 @@ struct ScanArgs {
     float *aux_out;       // scalar or null
     float gamma;
     float *b_e;           // [E] or null
-    double *pe;           // [E] scratch for P_e * N (needed when psum is given)
+    double *pe;           // [E] P_e * N = sum_n p_{n,e} in fp64 (needed when psum is given; written)
     int tile_m;           // rows per m-tile of the tile table (when mt_prefix is given)
     const float *zpart;   // [chunks] per-chunk z-loss sums, or null
     float *z_out;         // router z-loss (scalar) or null; needs zpart
@@ -99,6 +99,20 @@ struct ScanArgs {
     int dense_tile_m;
 };
 cudaError_t launch_scan(const ScanArgs &a, cudaStream_t s);
+
+// The Switch loss and the sign-rule step from assignment counts and
+// probability sums added up over several forwards (the ranks of a
+// data-parallel layer): N = sum_e counts[e] / k, L = E sum_e counts[e]
+// psum[e] / N^2, b_e += gamma sign(sum counts - E counts[e]).
+struct AuxPartialsArgs {
+    const int32_t *counts;  // [E]
+    const double *psum;     // [E] sum over tokens of p_{n,e}
+    float *aux_out;         // scalar or null
+    float gamma;
+    float *b_e;             // [E] or null
+    int E, k;
+};
+cudaError_t launch_aux_partials(const AuxPartialsArgs &a, cudaStream_t s);
 
 // Router z-loss from per-chunk sums: *z_out = (sum of zpart) / N in fp64.
 cudaError_t launch_z_loss(const float *zpart, int64_t N, float *z_out, cudaStream_t s);

@@ -610,11 +610,17 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const void *W_g, fl
                           aux_out, nullptr, dev_status, ws, ws_bytes, stage_events, stream);
 }
 
-moe_status moe_forward_ex(const moe_config *cfg, const void *x, const void *W_g, float *b_e_inout, float gamma,
-                          const void *W1, const void *b1, const void *W3, const void *W2, const void *b2,
-                          const moe_shared_expert *shared, void *y, int32_t *topk_ids, float *topk_w,
-                          int32_t *counts, float *aux_out, float *z_loss_out, int32_t *dev_status, void *ws,
-                          size_t ws_bytes, void *const *stage_events, moe_stream_t stream)
+}  // extern "C"
+
+namespace {
+
+// The layer forward behind moe_forward, moe_forward_ex and
+// moe_forward_partials; psum_out (may be NULL) receives sum_n p_{n,e}.
+moe_status forward_impl(const moe_config *cfg, const void *x, const void *W_g, float *b_e_inout, float gamma,
+                        const void *W1, const void *b1, const void *W3, const void *W2, const void *b2,
+                        const moe_shared_expert *shared, void *y, int32_t *topk_ids, float *topk_w,
+                        int32_t *counts, float *aux_out, float *z_loss_out, double *psum_out, int32_t *dev_status,
+                        void *ws, size_t ws_bytes, void *const *stage_events, moe_stream_t stream)
 {
     moe_status st = validate(cfg);
     if (st != MOE_OK) return st;
@@ -662,7 +668,7 @@ moe_status moe_forward_ex(const moe_config *cfg, const void *x, const void *W_g,
     ScanArgs sc{};
     sc.hist = hist;
     sc.psum = psum;
-    sc.pe = at<double>(ws, L.pe);
+    sc.pe = psum_out ? psum_out : at<double>(ws, L.pe);
     sc.chunks = num_chunks(cfg->N);
     sc.N = cfg->N;
     sc.E = cfg->E;
@@ -702,6 +708,46 @@ moe_status moe_forward_ex(const moe_config *cfg, const void *x, const void *W_g,
     if ((err = launch_combine(cfg->dtype, ca, num_sms(), s)) != cudaSuccess) return cuda_fail(err);
     if ((err = mark(5)) != cudaSuccess) return cuda_fail(err);
     return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_forward_ex(const moe_config *cfg, const void *x, const void *W_g, float *b_e_inout, float gamma,
+                          const void *W1, const void *b1, const void *W3, const void *W2, const void *b2,
+                          const moe_shared_expert *shared, void *y, int32_t *topk_ids, float *topk_w,
+                          int32_t *counts, float *aux_out, float *z_loss_out, int32_t *dev_status, void *ws,
+                          size_t ws_bytes, void *const *stage_events, moe_stream_t stream)
+{
+    return forward_impl(cfg, x, W_g, b_e_inout, gamma, W1, b1, W3, W2, b2, shared, y, topk_ids, topk_w, counts,
+                        aux_out, z_loss_out, nullptr, dev_status, ws, ws_bytes, stage_events, stream);
+}
+
+moe_status moe_forward_partials(const moe_config *cfg, const void *x, const void *W_g, const float *b_e,
+                                const void *W1, const void *b1, const void *W3, const void *W2, const void *b2,
+                                const moe_shared_expert *shared, void *y, int32_t *topk_ids, float *topk_w,
+                                int32_t *counts, double *psum_out, float *z_loss_out, int32_t *dev_status,
+                                void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    if (!counts || !psum_out) return MOE_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(psum_out) & 7u) return MOE_ERR_INVALID_ARG;
+    // the selection bias is read, never moved: its step needs the global load
+    return forward_impl(cfg, x, W_g, const_cast<float *>(b_e), 0.0f, W1, b1, W3, W2, b2, shared, y, topk_ids,
+                        topk_w, counts, nullptr, z_loss_out, psum_out, dev_status, ws, ws_bytes, nullptr, stream);
+}
+
+moe_status moe_aux_from_partials(int32_t E, int32_t k, const int32_t *counts, const double *psum, float *aux_out,
+                                 float gamma, float *b_e_inout, moe_stream_t stream)
+{
+    if (E <= 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+    if (E > kMaxE || k > kMaxK) return MOE_ERR_UNSUPPORTED;
+    if (!counts || !psum || (!aux_out && !b_e_inout)) return MOE_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(psum) & 7u) return MOE_ERR_INVALID_ARG;
+    if (!(gamma >= 0.f) || !std::isfinite(gamma)) return MOE_ERR_INVALID_ARG;
+    AuxPartialsArgs a{counts, psum, aux_out, gamma, b_e_inout, E, k};
+    const cudaError_t err = launch_aux_partials(a, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err);
 }
 
 moe_status moe_permute_rows(int32_t dtype, const void *src, const int32_t *dst_row, void *dst, int64_t rows,

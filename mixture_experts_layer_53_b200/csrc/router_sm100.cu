@@ -70,8 +70,8 @@ struct LArgs {
     int64_t N;
     int d, E, E_pad, ld, stages, splits;
     int nacc;            // TMEM accumulators, k-block kb -> kb % nacc
-    uint32_t acc_cols;   // TMEM columns per accumulator (power of 2 >= E_pad)
-    uint32_t tmem_cols;  // nacc * acc_cols
+    uint32_t acc_cols;   // TMEM columns between accumulators (power of 2 >= max(E_pad, 32))
+    uint32_t tmem_cols;  // nacc * acc_cols rounded up to a power of 2
     // fused selection (E <= 32)
     SelectArgs sel;
     float *psum;
@@ -205,22 +205,60 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int64_t n = static_cast<int64_t>(row0) + q * 32 + lane;
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&ctl->tfull, 0, abort_flag, a.status));
-        if (ok && num_kb > 0) {
+        if (ok && num_kb > 0 && EB > 0 && EB <= 16) {
+            // E_pad = 16: the first 16 columns of each accumulator; the loads
+            // of up to four accumulators are in flight at once, then added in
+            // accumulator order
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+            const int used = min(a.nacc, num_kb);
+            float zs[16];
+            for (int s0 = 0; s0 < used; s0 += 4) {
+                uint32_t t[4][16];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (s0 + i < used) tmem_ld16(taddr + static_cast<uint32_t>(s0 + i) * a.acc_cols, t[i]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (s0 + i >= used) break;
+#pragma unroll
+                    for (int u = 0; u < 16; ++u)
+                        zs[u] = (s0 + i == 0) ? __uint_as_float(t[i][u]) : zs[u] + __uint_as_float(t[i][u]);
+                }
+            }
+            float *zrow = part + (q * 32 + lane) * a.E_pad;
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+                *reinterpret_cast<float4 *>(zrow + 4 * v) = make_float4(zs[4 * v], zs[4 * v + 1], zs[4 * v + 2],
+                                                                        zs[4 * v + 3]);
+        } else if (ok && num_kb > 0) {
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
             const int used = min(a.nacc, num_kb);
             float *zrow = EB == 0 ? a.logits + (static_cast<int64_t>(split) * a.N + n) * a.ld
                                   : part + (q * 32 + lane) * a.E_pad;
             for (int c0 = 0; c0 < a.E_pad; c0 += 32) {
-                uint32_t r[32], t[32];
-                tmem_ld32(taddr + c0, r);
-                tmem_ld_wait();
-                for (int s = 1; s < used; ++s) {
-                    tmem_ld32(taddr + static_cast<uint32_t>(s) * a.acc_cols + c0, t);
+                uint32_t r[32];
+                for (int s0 = 0; s0 < used; s0 += 2) {
+                    // two accumulators' loads in flight, added in order
+                    uint32_t t[32];
+                    if (s0 == 0) tmem_ld32(taddr + c0, r);
+                    else tmem_ld32(taddr + static_cast<uint32_t>(s0) * a.acc_cols + c0, t);
+                    uint32_t t2[32];
+                    const bool two = s0 + 1 < used;
+                    if (two) tmem_ld32(taddr + static_cast<uint32_t>(s0 + 1) * a.acc_cols + c0, t2);
                     tmem_ld_wait();
+                    if (s0 != 0) {
 #pragma unroll
-                    for (int u = 0; u < 32; ++u)
-                        r[u] = __float_as_uint(__uint_as_float(r[u]) + __uint_as_float(t[u]));
+                        for (int u = 0; u < 32; ++u)
+                            r[u] = __float_as_uint(__uint_as_float(r[u]) + __uint_as_float(t[u]));
+                    }
+                    if (two) {
+#pragma unroll
+                        for (int u = 0; u < 32; ++u)
+                            r[u] = __float_as_uint(__uint_as_float(r[u]) + __uint_as_float(t2[u]));
+                    }
                 }
                 if (EB == 0 && n < a.N) {
 #pragma unroll
@@ -313,12 +351,21 @@ bool setup(LArgs &a, CUtensorMap &tX, CUtensorMap &tW, const void *x, const void
     a.E_pad = ((E + 15) / 16) * 16;
     a.ld = logits_ld(E);
     a.splits = router_splits(N, d);
+    // accumulators 32-column aligned (a power of 2 >= E_pad, >= 32), k-blocks
+    // dealt round-robin so that each sums at most 4 of the CTA's k-blocks
+    // (the tensor core's own running sums stay short), at most 8 and as many
+    // as fit in 512 columns
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(a.E_pad)) cols <<= 1;
     a.acc_cols = cols;
-    a.nacc = static_cast<int>(512 / cols);
+    const int kb_per_cta = ((d + BK - 1) / BK + a.splits - 1) / a.splits;
+    a.nacc = (kb_per_cta + 3) / 4;
     if (a.nacc > 8) a.nacc = 8;
-    a.tmem_cols = cols * static_cast<uint32_t>(a.nacc);
+    if (a.nacc > static_cast<int>(512 / cols)) a.nacc = static_cast<int>(512 / cols);
+    if (a.nacc < 1) a.nacc = 1;
+    uint32_t tcols = 32;
+    while (tcols < cols * static_cast<uint32_t>(a.nacc)) tcols <<= 1;
+    a.tmem_cols = tcols;
     const int stage_bytes = A_BYTES + a.E_pad * BK * 2;
     a.stages = SMEM_TILE_BUDGET / stage_bytes;
     if (a.stages > MAX_STAGES) a.stages = MAX_STAGES;

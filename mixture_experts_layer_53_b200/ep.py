@@ -89,22 +89,34 @@ def exchange(t: torch.Tensor, send_rows: List[int], recv_rows: List[int], group=
     return out
 
 
+class DispatchState(NamedTuple):
+    """What a rank keeps between its dispatch and its combine."""
+    ids: torch.Tensor       # [N, k] int32
+    w: torch.Tensor         # [N, k] f32
+    probs: torch.Tensor     # [N, E] f32
+    x_sorted: torch.Tensor  # [N k, d_model], grouped by expert
+    inv_perm: torch.Tensor  # [N k] int32
+    counts: torch.Tensor    # [E] int32
+
+
 class ExpertParallelMoE:
     """One rank's share of an expert-parallel layer (see the module docstring).
 
     cfg: the layer's configuration with this rank's token count N and all E
     experts.  The rank's expert weights follow the layer layout restricted
     to its experts: W1 / W3 [E_r, d_ff, d_model], W2 [E_r, d_model, d_ff],
-    b1 [E_r, d_ff], b2 [E_r, d_model].
+    b1 [E_r, d_ff], b2 [E_r, d_model].  ``world`` and ``rank`` default to
+    the process group's; given explicitly (with no group), the phases below
+    can be driven by a caller that moves the rows itself.
     """
 
-    def __init__(self, cfg: MoeConfig, group=None):
+    def __init__(self, cfg: MoeConfig, group=None, world: Optional[int] = None, rank: Optional[int] = None):
         if cfg.d_ff_shared != 0:
             raise ValueError("the shared expert is not part of the expert-parallel exchange")
         self.cfg = cfg
         self.group = group
-        self.world = dist.get_world_size(group)
-        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group) if world is None else int(world)
+        self.rank = dist.get_rank(group) if rank is None else int(rank)
         if cfg.E % self.world != 0:
             raise ValueError(f"{cfg.E} experts do not split over {self.world} ranks")
         self.E_r = cfg.E // self.world
@@ -115,6 +127,39 @@ class ExpertParallelMoE:
         return make_config(rows, c.d_model, c.d_ff, self.E_r, 1, act=("gelu", "swiglu")[c.act],
                            dtype=("f32", "bf16")[c.dtype])
 
+    # -- the three compute phases; the exchanges sit between them
+
+    def dispatch_phase(self, x: torch.Tensor, W_g: torch.Tensor, b_e: Optional[torch.Tensor] = None) -> DispatchState:
+        """Step 1: route and dispatch this rank's tokens."""
+        ids, w, probs = moe_route(self.cfg, x, W_g, b_e, want_probs=True)
+        dsp = moe_dispatch(self.cfg, ids, x)
+        return DispatchState(ids, w, probs, dsp["x_sorted"], dsp["inv_perm"], dsp["counts"])
+
+    def expert_phase(self, x_recv: torch.Tensor, p: EPPlan, W1: torch.Tensor, W2: torch.Tensor,
+                     W3: Optional[torch.Tensor] = None, b1: Optional[torch.Tensor] = None,
+                     b2: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Step 3: the received rows, in (source rank, local expert) order,
+        regrouped by local expert, through the local experts and back to the
+        received order."""
+        rows = x_recv.shape[0]
+        y_recv = torch.empty_like(x_recv)
+        if rows > 0:
+            dev = x_recv.device
+            regroup = torch.from_numpy(p.regroup).to(dev)
+            back = np.empty_like(p.regroup)
+            back[p.regroup] = np.arange(rows, dtype=np.int32)
+            x_local = moe_permute_rows(x_recv, regroup)
+            y_local = moe_expert_ffn(self.local_config(rows), x_local, torch.from_numpy(p.offsets).to(dev), W1, W2,
+                                     b1=b1, W3=W3, b2=b2)
+            moe_permute_rows(y_local, torch.from_numpy(back).to(dev), out=y_recv)
+        return y_recv
+
+    def combine_phase(self, st: DispatchState, y_sorted: torch.Tensor):
+        """Step 4: the rank's rows back in token order, and its Switch loss."""
+        y = moe_combine(self.cfg, y_sorted, st.w, st.inv_perm)
+        aux, _, _ = moe_aux_loss(self.cfg, st.probs, st.ids)
+        return y, aux
+
     def forward(self, x: torch.Tensor, W_g: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor,
                 W3: Optional[torch.Tensor] = None, b1: Optional[torch.Tensor] = None,
                 b2: Optional[torch.Tensor] = None, b_e: Optional[torch.Tensor] = None):
@@ -124,25 +169,11 @@ class ExpertParallelMoE:
         is left to the caller (moe_aux_loss with gamma and b_e, on this
         rank's counts or on counts all-reduced over the group)."""
         cfg, world, E_r, g = self.cfg, self.world, self.E_r, self.group
-        dev = x.device
-        ids, w, probs = moe_route(cfg, x, W_g, b_e, want_probs=True)
-        dsp = moe_dispatch(cfg, ids, x)
-        counts = dsp["counts"]
-        recv_counts = exchange(counts, [E_r] * world, [E_r] * world, g)
-        host = torch.cat([counts, recv_counts]).cpu().numpy()
+        st = self.dispatch_phase(x, W_g, b_e)
+        recv_counts = exchange(st.counts, [E_r] * world, [E_r] * world, g)
+        host = torch.cat([st.counts, recv_counts]).cpu().numpy()
         p = plan(host[:cfg.E], host[cfg.E:].reshape(world, E_r), world)
-        x_recv = exchange(dsp["x_sorted"], p.send_rows, p.recv_rows, g)
-        rows = x_recv.shape[0]
-        y_recv = torch.empty_like(x_recv)
-        if rows > 0:
-            regroup = torch.from_numpy(p.regroup).to(dev)
-            back = np.empty_like(p.regroup)
-            back[p.regroup] = np.arange(rows, dtype=np.int32)
-            x_local = moe_permute_rows(x_recv, regroup)
-            y_local = moe_expert_ffn(self.local_config(rows), x_local, torch.from_numpy(p.offsets).to(dev), W1, W2,
-                                     b1=b1, W3=W3, b2=b2)
-            moe_permute_rows(y_local, torch.from_numpy(back).to(dev), out=y_recv)
+        x_recv = exchange(st.x_sorted, p.send_rows, p.recv_rows, g)
+        y_recv = self.expert_phase(x_recv, p, W1, W2, W3=W3, b1=b1, b2=b2)
         y_sorted = exchange(y_recv, p.recv_rows, p.send_rows, g)
-        y = moe_combine(cfg, y_sorted, w, dsp["inv_perm"])
-        aux, _, _ = moe_aux_loss(cfg, probs, ids)
-        return y, aux
+        return self.combine_phase(st, y_sorted)

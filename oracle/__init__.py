@@ -69,6 +69,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.oracle_sorted_forward.restype = i32
     lib.oracle_aux_loss.argtypes = [i64, i32, i32, _dp, _ip, _ip]
     lib.oracle_aux_loss.restype = f64
+    lib.oracle_aux_from_partials.argtypes = [i32, i32, _ip, _dp]
+    lib.oracle_aux_from_partials.restype = f64
     lib.oracle_bias_update.argtypes = [i64, i32, i32, _ip, f64, _dp]
     lib.oracle_bias_update.restype = None
     lib.oracle_z_loss.argtypes = [i64, i32, _dp]
@@ -244,6 +246,17 @@ def aux_loss(probs, ids, L: Optional[ctypes.CDLL] = None) -> Tuple[float, np.nda
     counts = np.zeros(E, np.int32)
     val = L.oracle_aux_loss(N, E, k, _p(probs, _dp), _p(ids, _ip), _p(counts, _ip))
     return float(val), counts
+
+
+def aux_from_partials(counts, psum, k: int, L: Optional[ctypes.CDLL] = None) -> float:
+    """Switch loss of a whole batch from its parts' summed counts [E] and
+    probability sums [E] (N = sum(counts) / k)."""
+    L = L or lib()
+    counts = _i32(counts)
+    psum = _f64(psum)
+    E = counts.shape[0]
+    assert psum.shape == (E,)
+    return float(L.oracle_aux_from_partials(E, int(k), _p(counts, _ip), _p(psum, _dp)))
 
 
 def bias_update(b, counts, N: int, k: int, gamma: float,

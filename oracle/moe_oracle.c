@@ -416,6 +416,31 @@ double oracle_aux_loss(int64_t N, int E, int k, const double *probs,
 }
 
 /*
+ * The Switch loss of a batch split into parts (course module sec. 2.3: f_e
+ * and P_e are averages over the whole batch of N tokens), from each part's
+ * assignment counts and probability sums added up over the parts:
+ * counts[e] = assignments to e in the whole batch, psum[e] = sum over the
+ * whole batch of p_{n,e}.  Every token makes k assignments, so
+ * N = (sum_e counts[e]) / k; then f_e = counts[e] / N, P_e = psum[e] / N and
+ * L = E sum_e f_e P_e as in oracle_aux_loss.  0 for an empty batch.
+ */
+double oracle_aux_from_partials(int E, int k, const int32_t *counts, const double *psum)
+{
+    if (E < 1 || k < 1) return NAN;
+    int64_t total = 0;
+    for (int e = 0; e < E; ++e) total += counts[e];
+    if (total == 0) return 0.0;
+    const double N = (double)total / (double)k;
+    double L = 0.0;
+    for (int e = 0; e < E; ++e) {
+        double f = (double)counts[e] / N;
+        double Pe = psum[e] / N;
+        L += f * Pe;
+    }
+    return L * (double)E;
+}
+
+/*
  * Aux-free bias rule (sec. 2.5): b_e <- b_e + gamma sign(mean load - load_e)
  * with mean load = N k / E, i.e. the sign of the integer N k - E count_e.
  */

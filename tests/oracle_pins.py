@@ -25,6 +25,9 @@ What pins what:
   invariants                             sum w, counts, bijection, stability
   C per-token loop and numpy             forward_tokens (sampled-token y at
                                          full size), bit for bit / to 1e-12
+  batch split into parts                 L from summed counts and P sums
+                                         equals the whole batch's; = k at
+                                         balance
 """
 from __future__ import annotations
 
@@ -581,6 +584,46 @@ def pin_forward_tokens(L, forward_tokens=None):
                                                 None if b1 is None else b1[e], None if b2 is None else b2[e])[0]
         scale = np.max(np.abs(ref))
         _close(got / scale, ref / scale, 1e-12, f"forward_tokens vs numpy ({act}, k={k})")
+
+
+def pin_loss_from_partials(L):
+    """A batch split into parts (course module sec. 2.3: f and P are averages
+    over the whole batch): summing each part's counts and probability sums
+    and applying the loss gives the whole batch's L to rounding; at the
+    circulant router's perfect balance it is k; with one part it is the
+    part's own L; an empty batch gives 0."""
+    rng = np.random.default_rng(31)
+    for router, E, k, parts in (("softmax_topk", 8, 2, (13, 1, 30)), ("sigmoid", 16, 4, (20, 20)),
+                                ("topk_softmax", 5, 5, (7,))):
+        N = sum(parts)
+        x, Wg, *_ = _rand_problem(rng, N, 9, 4, E, "gelu", False)
+        bsel = rng.uniform(-0.1, 0.1, E) if router == "sigmoid" else None
+        r = O.route(x, Wg, k, router, b_sel=bsel, L=L)
+        whole, whole_counts = O.aux_loss(r["probs"], r["ids"], L=L)
+        counts = np.zeros(E, np.int64)
+        psum = np.zeros(E)
+        lo = 0
+        for n in parts:
+            part_counts = np.bincount(r["ids"][lo:lo + n].reshape(-1), minlength=E)
+            counts += part_counts
+            psum += r["probs"][lo:lo + n].sum(axis=0)
+            if len(parts) == 1:
+                own, _ = O.aux_loss(r["probs"][lo:lo + n], r["ids"][lo:lo + n], L=L)
+                _close(O.aux_from_partials(part_counts, r["probs"][lo:lo + n].sum(axis=0), k, L=L), own, 1e-14,
+                       "one part: its own L")
+            lo += n
+        _eq(counts, whole_counts, "summed counts are the whole batch's")
+        _close(O.aux_from_partials(counts, psum, k, L=L), whole, 1e-13, f"L from partials ({router})")
+    E, k = 8, 3
+    v = np.array([1.5, -0.5, 0.75, 0.0, -1.25, 0.5, 1.0, -0.25])
+    x = np.eye(E)
+    Wg = np.array([[v[(e - n) % E] for n in range(E)] for e in range(E)])
+    r = O.route(x, Wg, k, L=L)
+    halves = [slice(0, 3), slice(3, E)]
+    counts = sum(np.bincount(r["ids"][h].reshape(-1), minlength=E) for h in halves)
+    psum = sum(r["probs"][h].sum(axis=0) for h in halves)
+    _close(O.aux_from_partials(counts, psum, k, L=L), k, 1e-12, "balanced split batch: L = k")
+    assert O.aux_from_partials(np.zeros(E, np.int32), np.zeros(E), k, L=L) == 0.0, "empty batch"
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

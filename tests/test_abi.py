@@ -244,3 +244,26 @@ def test_permute_rows_validation(lib):
     assert lib.moe_permute_rows(1, ctypes.c_void_p(0x10008), idx, a, 4, 8, None) == 1  # src misaligned
     assert lib.moe_permute_rows(1, a, idx, a, -1, 8, None) == 1                      # negative rows
     assert lib.moe_permute_rows(1, None, None, None, 0, 8, None) == 0                # nothing to move
+
+
+def test_data_parallel_partials_validation(lib):
+    """moe_forward_partials needs counts and an 8-byte aligned psum_out;
+    moe_aux_from_partials checks E, k, its outputs and gamma -- all before
+    any launch."""
+    c = M.make_config(64, 64, 128, 8, 2, act="swiglu", dtype="bf16")
+    fwd = lambda counts, psum: lib.moe_forward_partials(ctypes.byref(c), BAD, BAD, None, BAD, None, BAD, BAD, None,
+                                                        None, BAD, None, None, counts, psum, None, None, BAD, 1 << 30,
+                                                        None)
+    assert fwd(None, ctypes.c_void_p(0x2000)) == 1                   # counts missing
+    assert fwd(ctypes.c_void_p(0x2000), None) == 1                   # psum_out missing
+    assert fwd(ctypes.c_void_p(0x2000), ctypes.c_void_p(0x2004)) == 1  # psum_out not 8-byte aligned
+    cnt, ps, a = ctypes.c_void_p(0x3000), ctypes.c_void_p(0x4000), ctypes.c_void_p(0x5000)
+    fin = lib.moe_aux_from_partials
+    assert fin(8, 9, cnt, ps, a, 0.0, None, None) == 1                       # k > E
+    assert fin(0, 1, cnt, ps, a, 0.0, None, None) == 1                       # E < 1
+    assert fin(512, 2, cnt, ps, a, 0.0, None, None) == 2                     # E > 256
+    assert fin(64, 17, cnt, ps, a, 0.0, None, None) == 2                     # k > 16
+    assert fin(8, 2, None, ps, a, 0.0, None, None) == 1                      # counts missing
+    assert fin(8, 2, cnt, ctypes.c_void_p(0x4004), a, 0.0, None, None) == 1  # psum misaligned
+    assert fin(8, 2, cnt, ps, None, 0.0, None, None) == 1                    # no output at all
+    assert fin(8, 2, cnt, ps, a, float("nan"), None, None) == 1              # gamma not finite

@@ -2,8 +2,9 @@
 
 * bench.py's max-over-ranks reduction of the timed region;
 * the layer is token-parallel: tokens sharded over ranks give the same
-  outputs as the whole batch, and an all-reduce of the per-rank assignment
-  counts and probability sums gives the whole batch's Switch loss
+  outputs as the whole batch, and the data-parallel layer's exchange
+  (``dp.all_reduce_partials``: int32 counts and float64 probability sums,
+  the inputs of moe_aux_from_partials) gives the whole batch's Switch loss
   (course module sec. 2.3: L = E sum_e f_e P_e over all N tokens).
 The layer math here is the fp64 oracle (no GPU on this path).
 """
@@ -50,11 +51,14 @@ def _rank_main(rank, world, port, results):
         f64 = lambda t: None if t is None else t.float().numpy().astype(np.float64)
         y = O.dense_forward(x[lo:hi], r["ids"], r["w"], f64(inp["W1"]), f64(inp["W2"]), wl.act, None,
                             f64(inp["b1"]), f64(inp["b2"]))
-        counts = torch.from_numpy(np.bincount(r["ids"].reshape(-1), minlength=wl.E).astype(np.int64))
+        # the partials moe_forward_partials returns, exchanged by the
+        # data-parallel layer's own all-reduce step, then the whole batch's
+        # loss from them (the oracle's statement of moe_aux_from_partials)
+        from mixture_experts_layer_53_b200 import dp as DP
+        counts = torch.from_numpy(np.bincount(r["ids"].reshape(-1), minlength=wl.E).astype(np.int32))
         psum = torch.from_numpy(r["probs"].sum(axis=0))
-        dist.all_reduce(counts)
-        dist.all_reduce(psum)
-        L = wl.E * float(np.sum((counts.numpy() / wl.N) * (psum.numpy() / wl.N)))
+        DP.all_reduce_partials(counts, psum)
+        L = O.aux_from_partials(counts.numpy(), psum.numpy(), wl.k)
         ys = [torch.zeros(0)] * world
         dist.all_gather_object(ys, y)
         if rank == 0:

@@ -68,6 +68,9 @@ MUTANTS = {
                               "for (int j = 0; j < k; ++j) dp[idn[j]] += dg[idn[j]] / S;"),
     "bwd_W2_grad_transposed": ("for (int f = 0; f < F; ++f) dW2[(int64_t)c * F + f] += go[c] * h[f];",
                                "for (int f = 0; f < F; ++f) dW2[(int64_t)c * F + f] += go[f % d] * h[c % F];"),
+    "partials_N_not_over_k": ("const double N = (double)total / (double)k;", "const double N = (double)total;"),
+    "partials_P_unnormalised": ("double Pe = psum[e] / N;\n        L += f * Pe;\n    }\n    return L * (double)E;",
+                                "double Pe = psum[e];\n        L += f * Pe;\n    }\n    return L * (double)E;"),
     "combine_drops_last_slot": ("for (int j = 0; j < k; ++j) {\n            const double *src",
                                 "for (int j = 0; j + 1 < k; ++j) {\n            const double *src"),
 }
