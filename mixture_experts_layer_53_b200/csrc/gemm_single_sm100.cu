@@ -37,6 +37,7 @@
 #include "common.cuh"
 #include "host_util.h"
 #include "kernels.h"
+#include "epilogue_bf16.cuh"
 #include "epilogue_f32.cuh"
 #include "sm100.cuh"
 
@@ -87,6 +88,8 @@ struct GemmArgs {
     // columns kb * BK; k-blocks kb1..kb_total-1 read tmB3 with A columns
     // a_col2 + (kb - kb1) * BK
     int kb1, kb_total, a_col2;
+    const int32_t *slot;  // EPI_LINEAR: row r -> output row slot[r], scaled by slot_w[slot[r]]
+    const float *slot_w;
 };
 
 struct Ctl {
@@ -95,7 +98,7 @@ struct Ctl {
     // padded to 36 floats (no bank conflicts) and stored back by the lanes in
     // whole 128-B rows; OPS_MN_MN: 4 KB per warp in the 128-byte swizzled
     // layout of a TMA store box (also free of bank conflicts).
-    alignas(1024) float stage[4][32][36];
+    alignas(1024) float stage[4][32][36];  // bf16 results: kBf16StageBytes per warp at its start
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t tfull[2];
@@ -147,64 +150,14 @@ template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase, int e, int row_first,
                                               int64_t row_end, int n0, float (*stage)[36], bool zero = false)
 {
-    const int lane = threadIdx.x & 31;
     if constexpr (EPI == EPI_F32) {
         float *out = g.out_f32 + (g.ragged_k ? static_cast<int64_t>(e) * g.c_stride : 0);
         epilogue_f32_rows(out, g.ldo, g.n_out, tbase, row_first, row_end, n0, stage, zero, g.accumulate != 0);
         return;
     }
-    const int row = row_first + lane;
-    const bool row_ok = row < row_end;
-    __nv_bfloat16 *orow = g.out + static_cast<int64_t>(row) * g.ldo;
-    const __nv_bfloat16 *brow = g.bias ? g.bias + static_cast<int64_t>(e) * g.n_out : nullptr;
-#pragma unroll 1
-    for (int c = 0; c < out_cols<EPI>(); c += 32) {
-        uint32_t acc[32];
-        tmem_ld32(tbase + c, acc);
-        if constexpr (EPI == EPI_SWIGLU) {
-            uint32_t up[32];
-            tmem_ld32(tbase + 128 + c, up);
-            tmem_ld_wait();
-            if (row_ok) {
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const int col = n0 + c + v * 8;
-                    if (col < g.n_out) {
-                        float h[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            h[u] = silu(__uint_as_float(acc[v * 8 + u])) * __uint_as_float(up[v * 8 + u]);
-                        st16(orow + col, pack16(h, static_cast<const __nv_bfloat16 *>(nullptr)));
-                    }
-                }
-            }
-        } else {
-            tmem_ld_wait();
-            if (row_ok) {
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const int col = n0 + c + v * 8;
-                    if (col < g.n_out) {
-                        float o[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) o[u] = __uint_as_float(acc[v * 8 + u]);
-                        if (brow) {
-                            float b[8];
-                            unpack16(*reinterpret_cast<const uint4 *>(brow + col), b,
-                                     static_cast<const __nv_bfloat16 *>(nullptr));
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) o[u] += b[u];
-                        }
-                        if constexpr (EPI == EPI_GELU) {
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) o[u] = gelu_erf(o[u]);
-                        }
-                        st16(orow + col, pack16(o, static_cast<const __nv_bfloat16 *>(nullptr)));
-                    }
-                }
-            }
-        }
-    }
+    epilogue_bf16_rows<EPI>(g.out, g.ldo, g.n_out, g.bias ? g.bias + static_cast<int64_t>(e) * g.n_out : nullptr,
+                            tbase, row_first, row_end, n0, 0, out_cols<EPI>(), reinterpret_cast<uint8_t *>(stage),
+                            g.slot, g.slot_w);
 }
 
 // MN-major operand tiles (OPS_K_MN, OPS_MN_MN; EPI_F32 only) are 64-column
@@ -601,6 +554,8 @@ cudaError_t launch_ffn_bf16_sm100_single(const FfnArgs &a, int num_sms, cudaEven
     g2.n_out = a.d;
     g2.n_tiles = (a.d + 255) / 256;
     g2.b_rows = a.d;
+    g2.slot = a.slot;
+    g2.slot_w = a.slot_w;
     return launch_gemm<EPI_LINEAR>(tH, tW2, tW2, g2, num_sms, s);
 }
 

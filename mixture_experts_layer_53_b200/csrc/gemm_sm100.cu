@@ -48,6 +48,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "epilogue_bf16.cuh"
 #include "epilogue_f32.cuh"
 #include "host_util.h"
 #include "kernels.h"
@@ -99,11 +100,17 @@ struct GemmArgs {
     // [E][m_total][n_out] has m_tiles tiles of 256 rows
     int m_tiles;
     int64_t m_total;
+    const int32_t *slot;  // EPI_LINEAR: row r -> output row slot[r], scaled by slot_w[slot[r]]
+    const float *slot_w;
 };
 
+// Staging for the epilogue warps: EPI_F32, a 32 x 32 fp32 chunk per warp
+// (rows padded to 36 floats, or 4 KB in the TMA store box's layout); bf16,
+// kBf16StageBytes per warp (up to 8 warps).
+constexpr int kStageRaw = 8 * kBf16StageBytes > 4 * 32 * 36 * 4 ? 8 * kBf16StageBytes : 4 * 32 * 36 * 4;
+
 struct Ctl {
-    // EPI_F32: per epilogue warp, a 32 x 32 chunk on its way to global memory
-    alignas(1024) float stage[4][32][36];
+    alignas(1024) uint8_t stage[kStageRaw];
     uint64_t full[STAGES];   // used in the even CTA: both CTAs' bytes
     uint64_t empty[STAGES];  // each CTA: arrived by the even CTA's commit
     uint64_t tfull[2];       // each CTA: arrived by the even CTA's commit
@@ -159,63 +166,6 @@ __device__ __forceinline__ int half_boxes(int r, int64_t extent, int base)
 {
     const int64_t left = extent - (base + r * 128);
     return left <= 0 ? 0 : static_cast<int>(min64(2, (left + 63) / 64));
-}
-
-// Output columns [c_begin, c_end) of one accumulator row (this thread's row).
-template <int EPI>
-__device__ __forceinline__ void epilogue_rows(const GemmArgs &g, uint32_t tbase, int e, int row, bool row_ok,
-                                              int n0, int c_begin, int c_end)
-{
-    __nv_bfloat16 *orow = g.out + static_cast<int64_t>(row) * g.ldo;
-    const __nv_bfloat16 *brow = g.bias ? g.bias + static_cast<int64_t>(e) * g.n_out : nullptr;
-#pragma unroll 1
-    for (int c = c_begin; c < c_end; c += 32) {
-        uint32_t acc[32];
-        tmem_ld32(tbase + c, acc);
-        if constexpr (EPI == EPI_SWIGLU) {
-            uint32_t up[32];
-            tmem_ld32(tbase + 128 + c, up);
-            tmem_ld_wait();
-            if (row_ok) {
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const int col = n0 + c + v * 8;
-                    if (col < g.n_out) {
-                        float h[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            h[u] = silu(__uint_as_float(acc[v * 8 + u])) * __uint_as_float(up[v * 8 + u]);
-                        st16(orow + col, pack16(h, static_cast<const __nv_bfloat16 *>(nullptr)));
-                    }
-                }
-            }
-        } else {
-            tmem_ld_wait();
-            if (row_ok) {
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const int col = n0 + c + v * 8;
-                    if (col < g.n_out) {
-                        float o[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) o[u] = __uint_as_float(acc[v * 8 + u]);
-                        if (brow) {
-                            float b[8];
-                            unpack16(*reinterpret_cast<const uint4 *>(brow + col), b,
-                                     static_cast<const __nv_bfloat16 *>(nullptr));
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) o[u] += b[u];
-                        }
-                        if constexpr (EPI == EPI_GELU) {
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) o[u] = gelu_erf(o[u]);
-                        }
-                        st16(orow + col, pack16(o, static_cast<const __nv_bfloat16 *>(nullptr)));
-                    }
-                }
-            }
-        }
-    }
 }
 
 template <int EPI, int OPS = OPS_KK>
@@ -544,19 +494,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             tc_fence_after();
             const Tile ti = tile_at<OPS>(t, ctl, g);
             const int row = ctl->off[ti.e] + ti.m_tile * PAIR_M + static_cast<int>(rank) * BM + row_in_cta;
-            const bool row_ok = row < ctl->off[ti.e + 1];
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
             if constexpr (EPI == EPI_F32 && OPS == OPS_MN_MN)
                 epilogue_f32_tma(&tmB3, tbase, ti.e, ti.m_tile * PAIR_M + static_cast<int>(rank) * BM + quarter * 32,
-                                 g.m_total, ti.n_tile * BN, g.n_out,
-                                 reinterpret_cast<uint8_t *>(ctl->stage) + quarter * 4096, mn_kblocks(ti.e) == 0);
+                                 g.m_total, ti.n_tile * BN, g.n_out, ctl->stage + quarter * 4096,
+                                 mn_kblocks(ti.e) == 0);
             else if constexpr (EPI == EPI_F32)
                 epilogue_f32_rows(g.out_f32, g.ldo, g.n_out, tbase, row - lane, ctl->off[ti.e + 1], ti.n_tile * BN,
-                                  ctl->stage[quarter], false, g.accumulate != 0);
+                                  reinterpret_cast<float(*)[36]>(ctl->stage + quarter * (32 * 36 * 4)), false,
+                                  g.accumulate != 0);
             else
-                epilogue_rows<EPI>(g, tbase, ti.e, row, row_ok, ti.n_tile * out_cols<EPI>(),
-                                   part * out_cols<EPI>() / parts, (part + 1) * out_cols<EPI>() / parts);
+                epilogue_bf16_rows<EPI>(g.out, g.ldo, g.n_out,
+                                        g.bias ? g.bias + static_cast<int64_t>(ti.e) * g.n_out : nullptr, tbase,
+                                        row - lane, ctl->off[ti.e + 1], ti.n_tile * out_cols<EPI>(),
+                                        part * out_cols<EPI>() / parts, (part + 1) * out_cols<EPI>() / parts,
+                                        ctl->stage + (warp - 2) * kBf16StageBytes, g.slot, g.slot_w);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
@@ -703,6 +656,8 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid
     g2.n_out = a.d;
     g2.n_tiles = (a.d + 255) / 256;
     g2.b_rows = a.d;
+    g2.slot = a.slot;
+    g2.slot_w = a.slot_w;
     return launch_pair<EPI_LINEAR>(tH, tW2, tW2, g2, num_sms, s);
 }
 

@@ -159,8 +159,8 @@ cudaError_t launch_dispatch_rows(int dtype, const DispatchRowsArgs &a, int num_s
 
 struct CombineArgs {
     const void *y_sorted;
-    const float *w;
-    const int32_t *inv_perm;
+    const float *w;             // null: every weight 1
+    const int32_t *inv_perm;    // null: slot n k + j is row n k + j
     void *y;
     int64_t N;
     int d, k;
@@ -268,6 +268,10 @@ struct FfnArgs {
     int64_t rows;              // N k
     int d, F, E, act;
     int tile_m;                // m-tile rows of mt_prefix: 128 (single CTA) or 256 (CTA pair)
+    // optional (the forward): GEMM2 row r is scaled by slot_w[slot[r]] and
+    // written to row slot[r] of y_sorted (assignment order) instead of row r
+    const int32_t *slot;       // [rows] (perm) or null
+    const float *slot_w;       // [rows] gate weights by assignment
 };
 }  // namespace moe
 

@@ -21,7 +21,15 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 # fp32: every product accumulates in fp32 from inputs the oracle sees exactly (errors are fp32
 # rounding).  bf16: the expert products run on the tensor cores, whose operands da, du and w h are
-# rounded to bf16 (2^-9 relative) before the fp32 accumulation.
+# rounded to bf16 (2^-9 = 1.95e-3 relative per element) before the fp32 accumulation.  Per gradient,
+# normwise against max |r|:
+#   dW2 = dy_s^T (w h):        one bf16 operand rounding (w h)           -> about 2^-9 of a typical term
+#   dW1, dW3 = [da | du]^T x_s: da / du rounded once, and they carry h's recomputation from the
+#                              bf16 pre-activations                      -> 2-3 x 2^-9
+#   dx = sum_j [da | du] W:    the same da / du roundings                 -> 2-3 x 2^-9
+#   dW_g, db: fp32 operands (CUDA-core products)                        -> fp32 rounding
+# Measured worst cases are 1.5e-3 .. 2.6e-3; 1e-2 (about 5 x 2^-9) bounds a sum of a few such
+# roundings with no cancellation, and is half the forward's bf16 output tolerance of 2e-2.
 TOL_G = {"f32": 1e-5, "bf16": 1e-2}
 
 CASES = {
