@@ -382,50 +382,66 @@ def hbm_fracs(wl, times_us, hbm_gbs):
     return out
 
 
-def isolated_stage_times(M, cfg, wl, inp, dev, reps: int = 20, warm: int = 3):
+def isolated_stage_times(M, cfg, wl, inp, dev, rounds: int = 6, warm: int = 2):
     """The HBM-bound entry points each timed alone: moe_route, moe_dispatch
-    (histogram, scan, row pass) and moe_combine, with L2 flushed (a 2x L2
-    write) before every launch and CUDA events right around it, so that the
-    bytes they move come from and go to HBM.  Returns mean microseconds per
-    call, over `reps` rounds after `warm` untimed ones."""
+    (histogram, scan, row pass) and moe_combine.  Each call reads its own
+    copy of its inputs, rotating over enough copies that they span more than
+    twice L2, so every call reads from HBM, and the calls of one stage run
+    back to back between one pair of CUDA events (launch gaps hidden as in a
+    forward).  Returns mean microseconds per call."""
     import ctypes
 
     import torch
     L = M.library()
     A, d = wl.N * wl.k, wl.d_model
+    es = 4 if wl.dtype == "f32" else 2
     i32 = dict(dtype=torch.int32, device=dev)
+
+    def copies(nbytes):
+        return int(max(2, min(8, -(-2 * L2_BYTES // max(nbytes, 1)) + 1)))
+
     ws = M.workspace(cfg, dev)
-    ids = torch.empty((wl.N, wl.k), **i32)
+    R_x = copies(wl.N * d * es)
+    xs_in = [inp["x"].clone() for _ in range(R_x)]
+    ids = [torch.empty((wl.N, wl.k), **i32) for _ in range(R_x)]
     w = torch.empty((wl.N, wl.k), dtype=torch.float32, device=dev)
-    xs = torch.empty((A, d), dtype=wl.torch_dtype, device=dev)
+    x_sorted = torch.empty((A, d), dtype=wl.torch_dtype, device=dev)
     inv, offsets, counts, status = (torch.empty(A, **i32), torch.empty(wl.E + 1, **i32), torch.empty(wl.E, **i32),
                                     torch.zeros(1, **i32))
-    ys = torch.randn((A, d), device=dev).to(wl.torch_dtype)
+    R_y = copies(A * d * es)
+    ys = [torch.randn((A, d), device=dev).to(wl.torch_dtype) for _ in range(R_y)]
     y = torch.empty((wl.N, d), dtype=wl.torch_dtype, device=dev)
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     P, st, cfgp = M._ptr, M._stream(), ctypes.byref(cfg)
-    calls = {
-        "route": lambda: L.moe_route(cfgp, P(inp["x"]), P(inp["W_g"]), P(inp["b_e"]), P(ids), P(w), None, P(ws),
-                                     ws.numel(), st),
-        "dispatch": lambda: L.moe_dispatch(cfgp, P(inp["x"]), P(ids), P(xs), None, P(inv), P(offsets), P(counts),
-                                           P(status), P(ws), ws.numel(), st),
-        "combine": lambda: L.moe_combine(cfgp, P(ys), P(w), P(inv), P(y), st),
-    }
-    ev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(reps)] for k in calls}
-    for i in range(warm + reps):
-        for name, call in calls.items():
-            flush.fill_(i & 0xFF)
-            if i >= warm:
-                ev[name][i - warm][0].record()
-            rc = call()
-            if rc != 0:
-                raise RuntimeError(f"{name}: status {rc}")
-            if i >= warm:
-                ev[name][i - warm][1].record()
-    torch.cuda.synchronize()
+
+    def route(i):
+        return L.moe_route(cfgp, P(xs_in[i % R_x]), P(inp["W_g"]), P(inp["b_e"]), P(ids[i % R_x]), P(w), None,
+                           P(ws), ws.numel(), st)
+
+    def dispatch(i):
+        return L.moe_dispatch(cfgp, P(xs_in[i % R_x]), P(ids[i % R_x]), P(x_sorted), None, P(inv), P(offsets),
+                              P(counts), P(status), P(ws), ws.numel(), st)
+
+    def combine(i):
+        return L.moe_combine(cfgp, P(ys[i % R_y]), P(w), P(inv), P(y), st)
+
+    for i in range(R_x):  # every copy of x gets its routing before the dispatch reads it
+        if route(i) != 0:
+            raise RuntimeError("moe_route")
+    out = {}
+    for name, call, R in (("route", route, R_x), ("dispatch", dispatch, R_x), ("combine", combine, R_y)):
+        for i in range(warm * R):
+            if call(i) != 0:
+                raise RuntimeError(name)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(rounds * R):
+            call(i)
+        e1.record()
+        torch.cuda.synchronize()
+        out[name] = 1000.0 * e0.elapsed_time(e1) / (rounds * R)
     assert int(status[0]) == 0
-    return {k: 1000.0 * sum(a.elapsed_time(b) for a, b in v) / reps for k, v in ev.items()}
+    del xs_in, ys
+    return out
 
 
 def describe(wl):
@@ -545,7 +561,7 @@ def run_native(args, wl):
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
 
-    # route, dispatch and combine each alone, L2 flushed before each launch
+    # route, dispatch and combine each alone, inputs rotated past L2
     kernel_us = isolated_stage_times(M, cfg, wl, inp, dev)
 
     if rank == 0:
@@ -585,9 +601,9 @@ def run_native(args, wl):
             # each stage inside a forward, every boundary recorded (launch
             # latency included, L2 left warm by the previous stage)
             "hbm_stages": hbm_fracs(wl, {k: 1000.0 * v for k, v in stages.items()}, peaks["hbm_gbs"]),
-            # each entry point alone, L2 flushed before it: moe_route (one
-            # kernel for E <= 32), moe_dispatch (histogram + scan + row pass),
-            # moe_combine
+            # each entry point alone, back to back over input copies larger
+            # than L2: moe_route (one kernel for E <= 32), moe_dispatch
+            # (histogram + scan + row pass), moe_combine
             "hbm_kernels": hbm_fracs(wl, kernel_us, peaks["hbm_gbs"]),
             "e2e": {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s",
                     "h2d_bytes_per_step": inp["x"].numel() * inp["x"].element_size(),

@@ -498,8 +498,8 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
          it < a.N * nblk; it += warps) {
         const int64_t n = it / nblk;
         const int64_t ob = (it - n * nblk) * kRowBlock;
-        const int src_l = lane < a.k ? (a.inv_perm ? a.inv_perm[n * a.k + lane] : static_cast<int>(n * a.k + lane)) : 0;
-        const float w_l = lane < a.k ? (a.w ? a.w[n * a.k + lane] : 1.f) : 0.f;
+        const int src_l = lane < a.k ? a.inv_perm[n * a.k + lane] : 0;
+        const float w_l = lane < a.k ? a.w[n * a.k + lane] : 0.f;
         float acc[kRowU][V];
 #pragma unroll
         for (int u = 0; u < kRowU; ++u)

@@ -24,8 +24,7 @@ constexpr int kBf16StageBytes = 32 * kBf16StageRowBytes;
 // gelu_erf(acc + b); linear: acc + b (b = bias[col], absent if bias null).
 template <int EPI>
 __device__ __forceinline__ void epi_bf16_math(const uint32_t (&acc)[32], const uint32_t (&up)[32],
-                                              const __nv_bfloat16 *bias, int col0, int n_out, float scale,
-                                              uint32_t (&p)[16])
+                                              const __nv_bfloat16 *bias, int col0, int n_out, uint32_t (&p)[16])
 {
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
@@ -47,10 +46,6 @@ __device__ __forceinline__ void epi_bf16_math(const uint32_t (&acc)[32], const u
 #pragma unroll
                 for (int u = 0; u < 8; ++u) o[u] = gelu_erf(o[u]);
             }
-            if constexpr (EPI == EPIB_LINEAR) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) o[u] *= scale;
-            }
         }
         const uint4 q = pack16(o, static_cast<const __nv_bfloat16 *>(nullptr));
         p[v * 4 + 0] = q.x;
@@ -64,10 +59,9 @@ __device__ __forceinline__ void epi_bf16_math(const uint32_t (&acc)[32], const u
 // into `stage`, then each store instruction writes 8 whole 64-B row
 // segments (lanes 4r .. 4r+3: 16 B each of row r).  Rows from row_end on
 // and columns from n_out on are not stored (n_out is a multiple of 8).
-// dst_l >= 0: lane l's row goes to output row dst_l instead of its own.
 __device__ __forceinline__ void epi_bf16_store_chunk(const uint32_t (&p)[16], uint8_t *stage, __nv_bfloat16 *out,
                                                      int64_t ldo, int64_t row_first, int64_t row_end, int col0,
-                                                     int n_out, int dst_l)
+                                                     int n_out)
 {
     const int lane = threadIdx.x & 31;
 #pragma unroll
@@ -77,16 +71,13 @@ __device__ __forceinline__ void epi_bf16_store_chunk(const uint32_t (&p)[16], ui
     __syncwarp();
     const int piece = lane & 3;
     const int col = col0 + piece * 8;
-    int dst[4];  // destination rows of the 4 rows this lane stores (all lanes shuffle)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = __shfl_sync(0xffffffffu, dst_l, (lane >> 2) + 8 * i);
     if (col < n_out) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int r = (lane >> 2) + 8 * i;
             const int64_t row = row_first + r;
             if (row < row_end)
-                st16(out + (dst[i] >= 0 ? static_cast<int64_t>(dst[i]) : row) * ldo + col,
+                st16(out + row * ldo + col,
                      *reinterpret_cast<const uint4 *>(stage + r * kBf16StageRowBytes + piece * 16));
         }
     }
@@ -98,22 +89,11 @@ __device__ __forceinline__ void epi_bf16_store_chunk(const uint32_t (&p)[16], ui
 // the tile, a multiple of 64 wide; result column n0 + c.  The TMEM loads of
 // the next 32-column chunk are in flight while the current one is computed
 // and stored.  `stage`: the warp's kBf16StageBytes, 16-byte aligned.
-// slot (linear only, may be null): row r of the result is scaled by
-// slot_w[slot[r]] and stored as output row slot[r] (the combine's
-// assignment order) instead of row r.
 template <int EPI>
 __device__ __forceinline__ void epilogue_bf16_rows(__nv_bfloat16 *out, int64_t ldo, int n_out,
                                                    const __nv_bfloat16 *bias_row, uint32_t tbase, int64_t row_first,
-                                                   int64_t row_end, int n0, int c_begin, int c_end, uint8_t *stage,
-                                                   const int32_t *slot = nullptr, const float *slot_w = nullptr)
+                                                   int64_t row_end, int n0, int c_begin, int c_end, uint8_t *stage)
 {
-    const int lane = threadIdx.x & 31;
-    int dst_l = -1;
-    float scale = 1.f;
-    if (EPI == EPIB_LINEAR && slot && row_first + lane < row_end) {
-        dst_l = slot[row_first + lane];
-        scale = slot_w[dst_l];
-    }
     uint32_t a0[32], a1[32], u0[32], u1[32];
     auto load = [&](uint32_t (&acc)[32], uint32_t (&up)[32], int c) {
         tmem_ld32(tbase + c, acc);
@@ -125,12 +105,12 @@ __device__ __forceinline__ void epilogue_bf16_rows(__nv_bfloat16 *out, int64_t l
     for (int c = c_begin; c < c_end; c += 64) {
         uint32_t p[16];
         load(a1, u1, c + 32);
-        epi_bf16_math<EPI>(a0, u0, bias_row, n0 + c, n_out, scale, p);
-        epi_bf16_store_chunk(p, stage, out, ldo, row_first, row_end, n0 + c, n_out, dst_l);
+        epi_bf16_math<EPI>(a0, u0, bias_row, n0 + c, n_out, p);
+        epi_bf16_store_chunk(p, stage, out, ldo, row_first, row_end, n0 + c, n_out);
         tmem_ld_wait();
         if (c + 64 < c_end) load(a0, u0, c + 64);
-        epi_bf16_math<EPI>(a1, u1, bias_row, n0 + c + 32, n_out, scale, p);
-        epi_bf16_store_chunk(p, stage, out, ldo, row_first, row_end, n0 + c + 32, n_out, dst_l);
+        epi_bf16_math<EPI>(a1, u1, bias_row, n0 + c + 32, n_out, p);
+        epi_bf16_store_chunk(p, stage, out, ldo, row_first, row_end, n0 + c + 32, n_out);
         tmem_ld_wait();
     }
 }

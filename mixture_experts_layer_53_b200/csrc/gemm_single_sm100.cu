@@ -88,8 +88,6 @@ struct GemmArgs {
     // columns kb * BK; k-blocks kb1..kb_total-1 read tmB3 with A columns
     // a_col2 + (kb - kb1) * BK
     int kb1, kb_total, a_col2;
-    const int32_t *slot;  // EPI_LINEAR: row r -> output row slot[r], scaled by slot_w[slot[r]]
-    const float *slot_w;
 };
 
 struct Ctl {
@@ -156,8 +154,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase,
         return;
     }
     epilogue_bf16_rows<EPI>(g.out, g.ldo, g.n_out, g.bias ? g.bias + static_cast<int64_t>(e) * g.n_out : nullptr,
-                            tbase, row_first, row_end, n0, 0, out_cols<EPI>(), reinterpret_cast<uint8_t *>(stage),
-                            g.slot, g.slot_w);
+                            tbase, row_first, row_end, n0, 0, out_cols<EPI>(), reinterpret_cast<uint8_t *>(stage));
 }
 
 // MN-major operand tiles (OPS_K_MN, OPS_MN_MN; EPI_F32 only) are 64-column
@@ -554,8 +551,6 @@ cudaError_t launch_ffn_bf16_sm100_single(const FfnArgs &a, int num_sms, cudaEven
     g2.n_out = a.d;
     g2.n_tiles = (a.d + 255) / 256;
     g2.b_rows = a.d;
-    g2.slot = a.slot;
-    g2.slot_w = a.slot_w;
     return launch_gemm<EPI_LINEAR>(tH, tW2, tW2, g2, num_sms, s);
 }
 

@@ -100,8 +100,6 @@ struct GemmArgs {
     // [E][m_total][n_out] has m_tiles tiles of 256 rows
     int m_tiles;
     int64_t m_total;
-    const int32_t *slot;  // EPI_LINEAR: row r -> output row slot[r], scaled by slot_w[slot[r]]
-    const float *slot_w;
 };
 
 // Staging for the epilogue warps: EPI_F32, a 32 x 32 fp32 chunk per warp
@@ -509,7 +507,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                                         g.bias ? g.bias + static_cast<int64_t>(ti.e) * g.n_out : nullptr, tbase,
                                         row - lane, ctl->off[ti.e + 1], ti.n_tile * out_cols<EPI>(),
                                         part * out_cols<EPI>() / parts, (part + 1) * out_cols<EPI>() / parts,
-                                        ctl->stage + (warp - 2) * kBf16StageBytes, g.slot, g.slot_w);
+                                        ctl->stage + (warp - 2) * kBf16StageBytes);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
@@ -656,8 +654,6 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid
     g2.n_out = a.d;
     g2.n_tiles = (a.d + 255) / 256;
     g2.b_rows = a.d;
-    g2.slot = a.slot;
-    g2.slot_w = a.slot_w;
     return launch_pair<EPI_LINEAR>(tH, tW2, tW2, g2, num_sms, s);
 }
 

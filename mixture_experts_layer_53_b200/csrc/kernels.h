@@ -43,6 +43,9 @@ cudaError_t launch_router_logits_sm100(const void *x, const void *W_g, float *lo
 // E <= 32: logits, scores, top-k, gates and the per-chunk statistics of
 // RouterArgs in one tcgen05 kernel (clusters of router_splits CTAs).
 cudaError_t launch_router_fused_sm100(const RouterArgs &r, int32_t *status, bool clear_status, cudaStream_t s);
+// E <= 32: the same in one streaming kernel, one CTA per 32-token chunk,
+// warps over column ranges of d, warp-level MMAs (router_mma.cu).
+cudaError_t launch_router_stream(const RouterArgs &r, int32_t *status, bool clear_status, cudaStream_t s);
 
 // Scores, top-k, gates and per-chunk statistics from fp32 logits (E > 32;
 // smaller E selects inside launch_router_fused_sm100).
@@ -159,8 +162,8 @@ cudaError_t launch_dispatch_rows(int dtype, const DispatchRowsArgs &a, int num_s
 
 struct CombineArgs {
     const void *y_sorted;
-    const float *w;             // null: every weight 1
-    const int32_t *inv_perm;    // null: slot n k + j is row n k + j
+    const float *w;
+    const int32_t *inv_perm;
     void *y;
     int64_t N;
     int d, k;
@@ -268,10 +271,6 @@ struct FfnArgs {
     int64_t rows;              // N k
     int d, F, E, act;
     int tile_m;                // m-tile rows of mt_prefix: 128 (single CTA) or 256 (CTA pair)
-    // optional (the forward): GEMM2 row r is scaled by slot_w[slot[r]] and
-    // written to row slot[r] of y_sorted (assignment order) instead of row r
-    const int32_t *slot;       // [rows] (perm) or null
-    const float *slot_w;       // [rows] gate weights by assignment
 };
 }  // namespace moe
 
