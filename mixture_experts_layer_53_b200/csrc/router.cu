@@ -157,25 +157,19 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a)
     }
 }
 
-// Logit z_{n,e}: the tcgen05 router's partial sums over d, added in split
-// order.
-__device__ __forceinline__ float logit_of(const SelectKernelArgs &a, int64_t n, int e)
-{
-    const float *p = a.logits + n * a.ld + e;
-    const int64_t stride = a.N * a.ld;
-    float z = p[0];
-    for (int s = 1; s < a.splits; ++s) z += p[s * stride];
-    return z;
-}
-
 // Scores, top-k and gates from precomputed fp32 logits (the tcgen05 router
 // of the bf16 path writes them), for E > 32.  One CTA per 32-token dispatch
-// chunk, one warp per token (16 warps, 2 tokens each): the selection is a
-// serial shuffle chain per token, so many independent warps hide its
-// latency.  Each token's k choices go into a shared histogram (integer
-// atomics: order-free); the chunk's sum of p is then taken per expert in
-// token order.
-constexpr int kSelWarps = 16;
+// chunk; a group of 8 lanes owns one token (4 tokens per warp, 8 warps), and
+// lane q of the group holds a contiguous block of EJ = E_pad / 8 of its
+// experts.  Each expert gets the 64-bit rank key of (selection score desc,
+// id asc) (rank_key), so the k rounds of the selection are: every lane takes
+// its largest key below the previous round's winner, then a 3-step xor
+// butterfly over the group's 8 lanes; the winner's logit travels with its
+// key, from which every lane of the group forms the gate.  The chunk's
+// histogram uses integer shared-memory atomics (order-free); its sum of p is
+// taken per expert in token order.
+constexpr int kSelWarps = 8;
+constexpr int kGroup = 8;  // lanes per token
 
 template <int EJ>
 __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs a)
@@ -189,43 +183,153 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
     float *zl = reinterpret_cast<float *>(hist_s + kMaxE);     // [32] lse^2
     const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kRT;
     const int ntok = static_cast<int>(min64(kRT, a.N - tok0));
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, q = lane & (kGroup - 1);
+    const int t = threadIdx.x / kGroup;  // token of this lane's group, 0..31
+    const bool live = t < ntok;
+    const int64_t n = tok0 + t;
+    const int e0 = q * EJ;  // this lane's experts e0 .. e0 + EJ - 1
     for (int e = threadIdx.x; e < E; e += kSelWarps * 32) hist_s[e] = 0;
-    __syncthreads();
-    const SelectArgs sa{a.b_sel, a.ids, a.w, a.probs, E, k, a.router, a.norm_topk, a.scaling, a.lse};
-    // software pipeline: the next token's row is loaded while this one is
-    // selected
-    float znext[EJ];
+
+    // logits: the splits' partial sums in split order
+    float z[EJ];
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) z[j] = 0.f;
+    if (live) {
+        const float *row = a.logits + n * a.ld;
+        const int64_t stride = a.N * a.ld;
+        for (int sp = 0; sp < a.splits; ++sp) {
+#pragma unroll
+            for (int j = 0; j < EJ; j += 4) {
+                if (e0 + j < a.ld) {  // ld and EJ are multiples of 4: whole float4s in or out
+                    const float4 v = *reinterpret_cast<const float4 *>(row + sp * stride + e0 + j);
+                    z[j] += v.x;
+                    z[j + 1] += v.y;
+                    z[j + 2] += v.z;
+                    z[j + 3] += v.w;
+                }
+            }
+        }
+    }
+    // softmax over all E (p = exp(z - max) / sum), in the group
+    float zmax = -FLT_MAX;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j)
+        if (e0 + j < E) zmax = fmaxf(zmax, z[j]);
+#pragma unroll
+    for (int o = 1; o < kGroup; o <<= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
+    float ex[EJ], esum = 0.f;
 #pragma unroll
     for (int j = 0; j < EJ; ++j) {
-        const int e = lane + 32 * j;
-        znext[j] = (warp < ntok && e < E) ? logit_of(a, tok0 + warp, e) : 0.f;
+        ex[j] = e0 + j < E ? expf(z[j] - zmax) : 0.f;
+        esum += ex[j];
     }
-#pragma unroll 1
-    for (int t = warp; t < ntok; t += kSelWarps) {
-        float z[EJ];
 #pragma unroll
-        for (int j = 0; j < EJ; ++j) z[j] = znext[j];
-        const int tn = t + kSelWarps;
+    for (int o = 1; o < kGroup; o <<= 1) esum += __shfl_xor_sync(0xffffffffu, esum, o);
+    const float inv_esum = 1.0f / esum;
+    const float lse = zmax + logf(esum);
+    // selection keys (0: below every real key)
+    uint64_t key[EJ];
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+        const int e = e0 + j;
+        key[j] = 0ull;
+        if (e < E) {
+            float sc = z[j];
+            if (a.router == kSigmoid) sc = 1.0f / (1.0f + expf(-z[j])) + (a.b_sel ? a.b_sel[e] : 0.f);
+            key[j] = rank_key(sc, e);
+        }
+    }
+    // k rounds: the group's largest key below the previous winner
+    uint64_t bound = ~0ull;
+    int my_id = -1;        // lane q < k (and q + 8 < k): the q-th (q + 8-th) choice
+    float my_z = 0.f, my_z2 = 0.f;
+    int my_id2 = -1;
+    float zsel[kMaxK];
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) zsel[r] = 0.f;
+#pragma unroll 1
+    for (int r = 0; r < k; ++r) {
+        uint64_t best = 0;
+        float bz = 0.f;
 #pragma unroll
         for (int j = 0; j < EJ; ++j) {
-            const int e = lane + 32 * j;
-            znext[j] = (tn < ntok && e < E) ? logit_of(a, tok0 + tn, e) : 0.f;
+            if (key[j] < bound && key[j] > best) {
+                best = key[j];
+                bz = z[j];
+            }
         }
-        int sel_id;
-        const float lse = select_token_keys<EJ>(z, sa, tok0 + t, true, &sel_id);
-        if (lane == 0) zl[t] = lse * lse;
-        if (lane < k) atomicAdd(&hist_s[sel_id], 1);
 #pragma unroll
-        for (int j = 0; j < EJ; ++j)
-            if (lane + 32 * j < E) pt[t * ZS + lane + 32 * j] = z[j];
+        for (int o = 1; o < kGroup; o <<= 1) {
+            const uint64_t ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
+            if (ob > best) {
+                best = ob;
+                bz = oz;
+            }
+        }
+        bound = best;
+        const int e = 0xFFFF - static_cast<int>(best & 0xFFFFu);
+#pragma unroll
+        for (int i = 0; i < kMaxK; ++i)
+            if (i == r) zsel[i] = bz;
+        if (q == r) {
+            my_id = e;
+            my_z = bz;
+        }
+        if (q + kGroup == r) {
+            my_id2 = e;
+            my_z2 = bz;
+        }
+    }
+    // gates: raw gate of each choice, their sum in choice order, then this
+    // lane's one or two outputs
+    auto raw_gate = [&](float zr) {
+        return a.router == kSigmoid ? 1.0f / (1.0f + expf(-zr)) : expf(zr - zmax);
+    };
+    float gs = 0.f;
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r)
+        if (r < k) gs += raw_gate(zsel[r]);
+    auto weight = [&](float zr) {
+        const float g = raw_gate(zr);
+        float wr;
+        if (a.router == kSoftmaxTopk) wr = a.norm_topk ? g / gs : g * inv_esum;
+        else if (a.router == kTopkSoftmax) wr = g / gs;
+        else wr = a.norm_topk ? g / gs : g;
+        return wr * a.scaling;
+    };
+    if (live) {
+        if (q < k) {
+            a.ids[n * k + q] = my_id;
+            a.w[n * k + q] = weight(my_z);
+            atomicAdd(&hist_s[my_id], 1);
+        }
+        if (q + kGroup < k) {
+            a.ids[n * k + q + kGroup] = my_id2;
+            a.w[n * k + q + kGroup] = weight(my_z2);
+            atomicAdd(&hist_s[my_id2], 1);
+        }
+        if (q == 0) {
+            zl[t] = lse * lse;
+            if (a.lse) a.lse[n] = lse;
+        }
+    }
+    // p for the chunk's sums (and probs if asked for)
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+        const int e = e0 + j;
+        if (e < E) {
+            const float p = live ? ex[j] * inv_esum : 0.f;
+            pt[t * ZS + e] = p;
+            if (live && a.probs) a.probs[n * E + e] = p;
+        }
     }
     __syncthreads();
     if (a.zpart && threadIdx.x == 0) a.zpart[blockIdx.x] = chunk_sum(zl, ntok);
     for (int e = threadIdx.x; e < E; e += kSelWarps * 32) {
         if (a.psum) {
             float s = 0.f;
-            for (int t = 0; t < ntok; ++t) s += pt[t * ZS + e];
+            for (int tt = 0; tt < ntok; ++tt) s += pt[tt * ZS + e];
             a.psum[static_cast<int64_t>(blockIdx.x) * E + e] = s;
         }
         if (a.hist) a.hist[static_cast<int64_t>(blockIdx.x) * E + e] = hist_s[e];
@@ -255,11 +359,15 @@ cudaError_t launch_select(const SelectKernelArgs &a, cudaStream_t s)
 {
     const int64_t grid = num_chunks(a.N);
     if (grid == 0) return cudaSuccess;
+    // EJ: experts per lane (8 lanes cover 64, 128 or 256 experts); logits
+    // rows of ld >= E columns, a multiple of 4 (columns E .. ld-1 are read
+    // as whole float4s and ignored)
+    if (a.ld % 4 != 0 || a.ld < a.E || a.E > kMaxE) return cudaErrorInvalidValue;
     const size_t smem = sizeof(float) * (kRT * (a.E + 1) + kRT) + sizeof(int) * kMaxE;
     const dim3 g(static_cast<unsigned>(grid)), b(kSelWarps * 32);
-    if (a.E <= 64) return launch_k(select_kernel<2>, g, b, smem, s, a);
-    if (a.E <= 128) return launch_k(select_kernel<4>, g, b, smem, s, a);
-    return launch_k(select_kernel<8>, g, b, smem, s, a);
+    if (a.E <= 64) return launch_k(select_kernel<8>, g, b, smem, s, a);
+    if (a.E <= 128) return launch_k(select_kernel<16>, g, b, smem, s, a);
+    return launch_k(select_kernel<32>, g, b, smem, s, a);
 }
 
 cudaError_t launch_router(int dtype, const RouterArgs &a, cudaStream_t s)

@@ -42,6 +42,10 @@ SMALL = {
     # sigmoid router there
     "fused_e24": W.WORKLOADS["mixtral"].scaled(N=333, d_model=256, d_ff=256, E=24, k=3),
     "fused_e32_sigmoid": W.WORKLOADS["deepseek_v3"].scaled(N=130, d_model=192, d_ff=128, E=32, k=8),
+    # the E > 32 selection: k > 8 (two choices per lane of a token's group),
+    # E not a multiple of 4 (padded logit rows), a 200-expert sigmoid router
+    "select_e50_k10": W.WORKLOADS["qwen3_skew"].scaled(N=161, d_model=136, d_ff=64, E=50, k=10, zipf=False),
+    "select_e200_k16_sigmoid": W.WORKLOADS["deepseek_v3"].scaled(N=97, d_model=128, d_ff=64, E=200, k=16),
 }
 
 # Token budgets for y at full size: tokens are chosen so that their routed
