@@ -102,23 +102,40 @@ __device__ __forceinline__ void st16(void *p, const uint4 &v)
     *reinterpret_cast<uint4 *>(p) = v;
 }
 
-// erf(x) by Abramowitz & Stegun, Handbook of Mathematical Functions, formula
-// 7.1.26: for a = |x|, erf(a) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5))))
-// exp(-a^2) with t = 1 / (1 + p a), |error| <= 1.5e-7; erf is odd.  A few
-// fused multiply-adds, one fast reciprocal and one fast exponential: the
-// GELU epilogues of the expert GEMMs (results rounded to bf16) are bound by
-// this function when the k-loop is short.
-__device__ __forceinline__ float erf_as7126(float x)
+// 2^x and 1/x by the special-function unit (PTX ex2.approx.ftz /
+// rcp.approx.ftz: about 2 ulp, subnormal results flushed to zero).
+__device__ __forceinline__ float ex2_approx(float x)
 {
-    const float a = fabsf(x);
-    const float t = __fdividef(1.0f, fmaf(0.3275911f, a, 1.0f));
-    const float poly =
-        t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f), -0.284496736f), 0.254829592f);
-    return copysignf(fmaf(-poly, __expf(-a * a), 1.0f), x);
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x)
+{
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
-// GELU (erf form) and SiLU, fp32.
-__device__ __forceinline__ float gelu_erf(float v) { return 0.5f * v * (1.0f + erf_as7126(v * 0.70710678118654752f)); }
+// GELU (erf form), fp32: gelu(v) = v Phi(v) with Phi the standard normal
+// distribution function, taken from Abramowitz & Stegun, Handbook of
+// Mathematical Functions, formula 26.2.17: for x >= 0, 1 - Phi(x) =
+// Z(x) t (b1 + t (b2 + t (b3 + t (b4 + t b5)))), t = 1 / (1 + p x), Z the
+// normal density, |error| < 7.5e-8; Phi(-x) = 1 - Phi(x).  The b_i below
+// carry Z's factor 1/sqrt(2 pi), and Z's exponential is 2^(-x^2 log2(e) / 2):
+// eleven multiply-adds, a select and two special-function operations per
+// value.  This is the same approximation as formula 7.1.26 for erf (whose
+// |error| 1.5e-7 halves on Phi).  The GELU epilogues of the expert GEMMs
+// (results rounded to bf16) are bound by this function when the k-loop is
+// short.  Large |v|: the exponential flushes to 0 and Phi to 0 or 1.
+__device__ __forceinline__ float gelu_erf(float v)
+{
+    const float t = rcp_approx(fmaf(0.2316419f, fabsf(v), 1.0f));
+    const float poly =
+        t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 0.530702710f, -0.726576030f), 0.710706890f), -0.142248362f), 0.127414793f);
+    const float q = poly * ex2_approx(v * (v * -0.72134752f));  // 1 - Phi(|v|)
+    return v * (v >= 0.0f ? 1.0f - q : q);
+}
 __device__ __forceinline__ float silu(float v) { return v / (1.0f + expf(-v)); }
 
 }  // namespace moe

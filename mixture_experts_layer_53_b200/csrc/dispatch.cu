@@ -218,25 +218,51 @@ __global__ void __launch_bounds__(kScanThreads) scan_finalize_kernel(ScanArgs a)
 // For E <= 32 the whole of the above in one CTA: warp w scans the columns of
 // experts w, w+8, ... (chunk bases in place, count_e, P_e * N in fp64 with
 // fixed-order sums), then warp 0 does the finalizing step with lane e for
-// expert e.  One launch instead of two.
+// expert e.  One launch instead of two.  STAGED (chunks * E <= kScanStage,
+// chunks <= kScanStageZ): the histograms, probability sums and z-loss sums
+// are first copied into shared memory with coalesced loads (one round trip
+// instead of a chain of strided ones per lane), scanned there, and the
+// chunk bases copied back; the sums are taken in the same order either way.
+constexpr int kScanStage = 4096;
+constexpr int kScanStageZ = 1024;
+
+template <bool STAGED>
 __global__ void __launch_bounds__(kScanThreads) scan_small_kernel(ScanArgs a)
 {
     pdl_enter();
     __shared__ int cnt_s[32];
     __shared__ double pe_s[32];
+    __shared__ int h_s[STAGED ? kScanStage : 1];
+    __shared__ float p_s[STAGED ? kScanStage : 1];
+    __shared__ float z_s[STAGED ? kScanStageZ : 1];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int E = a.E;
     const int64_t C = a.chunks;
+    int *hist = a.hist;
+    const float *psum = a.psum;
+    const float *zpart = a.zpart;
+    if constexpr (STAGED) {
+        for (int i = threadIdx.x; i < C * E; i += kScanThreads) {
+            h_s[i] = a.hist[i];
+            if (a.psum) p_s[i] = a.psum[i];
+        }
+        if (a.z_out && a.zpart)
+            for (int i = threadIdx.x; i < C; i += kScanThreads) z_s[i] = a.zpart[i];
+        __syncthreads();
+        hist = h_s;
+        psum = a.psum ? p_s : nullptr;
+        zpart = z_s;
+    }
     const int64_t per = (C + 31) / 32;
     const int64_t c0 = min64(C, lane * per), c1 = min64(C, c0 + per);
     for (int e = warp; e < E; e += kScanThreads / 32) {  // warp-uniform
         int s = 0;
         double p = 0.0;
 #pragma unroll 8
-        for (int64_t c = c0; c < c1; ++c) s += a.hist[c * E + e];
-        if (a.psum) {
+        for (int64_t c = c0; c < c1; ++c) s += hist[c * E + e];
+        if (psum) {
 #pragma unroll 8
-            for (int64_t c = c0; c < c1; ++c) p += static_cast<double>(a.psum[c * E + e]);
+            for (int64_t c = c0; c < c1; ++c) p += static_cast<double>(psum[c * E + e]);
         }
         int incl = s;
 #pragma unroll
@@ -247,8 +273,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_small_kernel(ScanArgs a)
         const int total = __shfl_sync(0xffffffffu, incl, 31);
         int run = incl - s;
         for (int64_t c = c0; c < c1; ++c) {
-            const int v = a.hist[c * E + e];
-            a.hist[c * E + e] = run;
+            const int v = hist[c * E + e];
+            hist[c * E + e] = run;
             run += v;
         }
 #pragma unroll
@@ -300,7 +326,9 @@ __global__ void __launch_bounds__(kScanThreads) scan_small_kernel(ScanArgs a)
             }
         }
     }
-    if (a.z_out && a.zpart) reduce_z_loss(a.zpart, a.chunks, a.N, a.z_out);  // block-uniform
+    if (a.z_out && a.zpart) reduce_z_loss(zpart, a.chunks, a.N, a.z_out);  // block-uniform
+    if constexpr (STAGED)  // the chunk bases back to the workspace (after the barrier above)
+        for (int i = threadIdx.x; i < C * E; i += kScanThreads) a.hist[i] = h_s[i];
 }
 
 // Switch loss and sign-rule step from partials summed over several forwards
@@ -602,7 +630,11 @@ cudaError_t launch_hist(const HistArgs &a, cudaStream_t s)
 cudaError_t launch_scan(const ScanArgs &a, cudaStream_t s)
 {
     if (a.E > kScanThreads) return cudaErrorInvalidValue;
-    if (a.E <= 32) return launch_k(scan_small_kernel, dim3(1), dim3(kScanThreads), 0, s, a);
+    if (a.E <= 32) {
+        if (a.chunks * a.E <= kScanStage && a.chunks <= kScanStageZ)
+            return launch_k(scan_small_kernel<true>, dim3(1), dim3(kScanThreads), 0, s, a);
+        return launch_k(scan_small_kernel<false>, dim3(1), dim3(kScanThreads), 0, s, a);
+    }
     cudaError_t err = launch_k(scan_cols_kernel, dim3(a.E), dim3(kScanThreads), 0, s, a);
     if (err != cudaSuccess) return err;
     return launch_k(scan_finalize_kernel, dim3(1), dim3(kScanThreads), 0, s, a);

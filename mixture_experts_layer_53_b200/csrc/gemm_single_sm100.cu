@@ -153,8 +153,9 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &g, uint32_t tbase,
         epilogue_f32_rows(out, g.ldo, g.n_out, tbase, row_first, row_end, n0, stage, zero, g.accumulate != 0);
         return;
     }
-    epilogue_bf16_rows<EPI>(g.out, g.ldo, g.n_out, g.bias ? g.bias + static_cast<int64_t>(e) * g.n_out : nullptr,
-                            tbase, row_first, row_end, n0, 0, out_cols<EPI>(), reinterpret_cast<uint8_t *>(stage));
+    epilogue_bf16_rows<EPI>(nullptr, g.out, g.ldo, g.n_out, g.bias ? g.bias + static_cast<int64_t>(e) * g.n_out : nullptr,
+                            tbase, row_first, row_end, n0, 0, out_cols<EPI>(), reinterpret_cast<uint8_t *>(stage),
+                            [] {});
 }
 
 // MN-major operand tiles (OPS_K_MN, OPS_MN_MN; EPI_F32 only) are 64-column

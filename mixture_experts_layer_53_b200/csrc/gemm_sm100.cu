@@ -63,14 +63,16 @@ constexpr int BM = 128;        // rows per CTA
 constexpr int PAIR_M = 256;    // rows per pair tile
 constexpr int BN = 256;        // accumulator columns
 constexpr int BK = 64;
-constexpr int STAGES = 6;
+constexpr int STAGES = 6;  // the most k-block stages a kernel uses
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int B_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's half of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 // Epilogue warps: one per TMEM lane quarter, or (GELU, whose erf epilogue
-// outlasts a short k-loop) two per quarter, each on half of the columns.
-// More epilogue warps let the pairs run further apart, which costs L2 reuse
-// of the weight tiles: SwiGLU and the linear GEMM keep four.
+// outlasts a short k-loop) four per quarter, each on a quarter of the
+// columns, one 32-column chunk at a time; that kernel keeps five k-block
+// stages so that its staging buffers fit.  More epilogue warps let the pairs
+// run further apart, which costs L2 reuse of the weight tiles: SwiGLU and
+// the linear GEMM keep four.
 template <int EPI> __host__ __device__ constexpr int epi_warps();
 template <int EPI> __host__ __device__ constexpr int threads_of() { return 64 + 32 * epi_warps<EPI>(); }
 constexpr uint32_t TMEM_COLS = 512;
@@ -80,7 +82,9 @@ enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_LINEAR = 2, EPI_F32 = 3 };
 // B K-major / B MN-major (A K-major in both) / A and B MN-major, ragged K
 enum { OPS_KK = 0, OPS_K_MN = 1, OPS_MN_MN = 2 };
 constexpr int BOX_BYTES = 64 * 64 * 2;  // one 64 x 64 MN-major box
-template <int EPI> __host__ __device__ constexpr int epi_warps() { return EPI == EPI_GELU ? 8 : 4; }
+template <int EPI> __host__ __device__ constexpr int epi_warps() { return EPI == EPI_GELU ? 16 : 4; }
+template <int EPI> __host__ __device__ constexpr int stages_of() { return epi_warps<EPI>() > 8 ? 5 : STAGES; }
+template <int EPI> __host__ __device__ constexpr int bias_floats() { return 4 * BN / epi_warps<EPI>(); }
 
 struct GemmArgs {
     const int32_t *offsets;
@@ -102,13 +106,18 @@ struct GemmArgs {
     int64_t m_total;
 };
 
-// Staging for the epilogue warps: EPI_F32, a 32 x 32 fp32 chunk per warp
-// (rows padded to 36 floats, or 4 KB in the TMA store box's layout); bf16,
-// kBf16StageBytes per warp (up to 8 warps).
-constexpr int kStageRaw = 8 * kBf16StageBytes > 4 * 32 * 36 * 4 ? 8 * kBf16StageBytes : 4 * 32 * 36 * 4;
+// Staging for the epilogue warps, after the k-block stages: EPI_F32, a
+// 32 x 32 fp32 chunk per warp (rows padded to 36 floats, or 4 KB in the TMA
+// store box's layout); bf16, kBf16StageBytes per warp (each buffer 2 KB-aligned).
+// Lean epilogues (more than 8 warps) add each warp's fp32 bias values for
+// its share of the columns.
+template <int EPI> __host__ __device__ constexpr int stage_bytes_of()
+{
+    return EPI == EPI_F32 ? 4 * 32 * 36 * 4
+                          : epi_warps<EPI>() * (kBf16StageBytes + (epi_warps<EPI>() > 8 ? bias_floats<EPI>() * 4 : 0));
+}
 
 struct Ctl {
-    alignas(1024) uint8_t stage[kStageRaw];
     uint64_t full[STAGES];   // used in the even CTA: both CTAs' bytes
     uint64_t empty[STAGES];  // each CTA: arrived by the even CTA's commit
     uint64_t tfull[2];       // each CTA: arrived by the even CTA's commit
@@ -122,8 +131,13 @@ struct Ctl {
     int mt[kMaxE + 1];
 };
 
-constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(Ctl);
-static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+template <int EPI> constexpr size_t smem_bytes_of()
+{
+    return 1024 + stages_of<EPI>() * STAGE_BYTES + stage_bytes_of<EPI>() + sizeof(Ctl);
+}
+static_assert(smem_bytes_of<EPI_SWIGLU>() <= 232448 && smem_bytes_of<EPI_GELU>() <= 232448 &&
+                  smem_bytes_of<EPI_LINEAR>() <= 232448 && smem_bytes_of<EPI_F32>() <= 232448,
+              "shared memory per CTA");
 
 struct Tile {
     int e, m_tile, n_tile;
@@ -169,20 +183,23 @@ __device__ __forceinline__ int half_boxes(int r, int64_t extent, int base)
 template <int EPI, int OPS = OPS_KK>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                         const __grid_constant__ CUtensorMap tmB3, const GemmArgs g)
+                         const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ CUtensorMap tmOut,
+                         const GemmArgs g)
 {
     pdl_enter();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                  ~static_cast<uintptr_t>(1023));
-    Ctl *ctl = reinterpret_cast<Ctl *>(tiles + STAGES * STAGE_BYTES);
+    constexpr int NST = stages_of<EPI>();
+    uint8_t *stage_base = tiles + NST * STAGE_BYTES;
+    Ctl *ctl = reinterpret_cast<Ctl *>(stage_base + stage_bytes_of<EPI>());
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
     volatile int *abort_flag = &ctl->abort;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(&ctl->full[s], 1);
             mbar_init(&ctl->empty[s], 1);
         }
@@ -191,7 +208,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             mbar_init(&ctl->tempty[b], 2 * epi_warps<EPI>());  // every epilogue warp of both CTAs
         }
         mbar_init(&ctl->drain, 1);
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(&ctl->tail_full[s], 1);
             mbar_init(&ctl->ready[s], 2);
         }
@@ -202,6 +219,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
         if (EPI == EPI_SWIGLU || OPS != OPS_KK) prefetch_tmap(&tmB3);
+        if (EPI != EPI_F32) prefetch_tmap(&tmOut);
     }
     if (warp == 1) {
         tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
@@ -272,7 +290,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                                             r);
                             tpar ^= 1u << stage;
                         }
-                        if (++stage == STAGES) {
+                        if (++stage == NST) {
                             stage = 0;
                             phase ^= 1u;
                         }
@@ -320,7 +338,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                         const CUtensorMap *mb = second ? &tmB3 : &tmB;
                         for (int c = 0; c < my_boxes; ++c)
                             tma_load_3d_pair(sA + A_BYTES + c * BOX_BYTES, mb, full_leader, nc0 + c * 64, kk0, ti.e);
-                        if (++stage == STAGES) {
+                        if (++stage == NST) {
                             stage = 0;
                             phase ^= 1u;
                         }
@@ -333,7 +351,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                     }
                     tma_load_2d_pair(sA, &tmA, full_leader, kb * BK, row0);
                     tma_load_2d_pair(sA + A_BYTES, tb, full_leader, kb * BK, brow);
-                    if (++stage == STAGES) {
+                    if (++stage == NST) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -341,13 +359,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             }
             if (*abort_flag && leader) {
                 // both CTAs' copies land on these barriers: wait for them
-                for (int s = 0; s < STAGES; ++s)
+                for (int s = 0; s < NST; ++s)
                     if ((armed >> s) & 1u)
                         mbar_wait(&ctl->full[s], (armed_parity >> s) & 1u, abort_flag, g.status, false);
             }
             if (*abort_flag) {
                 // OPS_MN_MN: this CTA's own copies of tail k-blocks
-                for (int s = 0; s < STAGES; ++s)
+                for (int s = 0; s < NST; ++s)
                     if ((tarmed >> s) & 1u)
                         mbar_wait(&ctl->tail_full[s], (tarmed_parity >> s) & 1u, abort_flag, g.status, false);
             }
@@ -414,7 +432,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                     }
                     __syncwarp();
                 }
-                if (++stage == STAGES) {
+                if (++stage == NST) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -459,7 +477,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                     }
                     issued = true;
                     umma_commit_pair(&ctl->empty[stage], 0x3);
-                    if (++stage == STAGES) {
+                    if (++stage == NST) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -494,30 +512,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             const int row = ctl->off[ti.e] + ti.m_tile * PAIR_M + static_cast<int>(rank) * BM + row_in_cta;
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
-            if constexpr (EPI == EPI_F32 && OPS == OPS_MN_MN)
+            // the MMA warp may refill this accumulator once every epilogue
+            // warp of both CTAs has read its part of it (the loads have
+            // completed, tcgen05.wait::ld, before this runs)
+            auto release = [&] {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster_cta(buf ? tempty_leader1 : tempty_leader0);
+            };
+            if constexpr (EPI == EPI_F32 && OPS == OPS_MN_MN) {
                 epilogue_f32_tma(&tmB3, tbase, ti.e, ti.m_tile * PAIR_M + static_cast<int>(rank) * BM + quarter * 32,
-                                 g.m_total, ti.n_tile * BN, g.n_out, ctl->stage + quarter * 4096,
+                                 g.m_total, ti.n_tile * BN, g.n_out, stage_base + quarter * 4096,
                                  mn_kblocks(ti.e) == 0);
-            else if constexpr (EPI == EPI_F32)
+                release();
+            } else if constexpr (EPI == EPI_F32) {
                 epilogue_f32_rows(g.out_f32, g.ldo, g.n_out, tbase, row - lane, ctl->off[ti.e + 1], ti.n_tile * BN,
-                                  reinterpret_cast<float(*)[36]>(ctl->stage + quarter * (32 * 36 * 4)), false,
+                                  reinterpret_cast<float(*)[36]>(stage_base + quarter * (32 * 36 * 4)), false,
                                   g.accumulate != 0);
-            else
-                epilogue_bf16_rows<EPI>(g.out, g.ldo, g.n_out,
+                release();
+            } else {
+                epilogue_bf16_rows<EPI, (epi_warps<EPI>() > 8)>(&tmOut, g.out, g.ldo, g.n_out,
                                         g.bias ? g.bias + static_cast<int64_t>(ti.e) * g.n_out : nullptr, tbase,
                                         row - lane, ctl->off[ti.e + 1], ti.n_tile * out_cols<EPI>(),
                                         part * out_cols<EPI>() / parts, (part + 1) * out_cols<EPI>() / parts,
-                                        ctl->stage + (warp - 2) * kBf16StageBytes);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
+                                        stage_base + (warp - 2) * kBf16StageBytes, release,
+                                        reinterpret_cast<float *>(stage_base + epi_warps<EPI>() * kBf16StageBytes) +
+                                            (warp - 2) * bias_floats<EPI>());
+            }
             if (++buf == 2) {
                 buf = 0;
                 tphase ^= 1u;
             }
         }
         // the staging buffers stay valid until this warp's stores are done
-        if (EPI == EPI_F32 && OPS == OPS_MN_MN && lane == 0) bulk_wait_all();
+        if ((EPI != EPI_F32 || OPS == OPS_MN_MN) && lane == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -531,15 +559,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
 }
 
 template <int EPI, int OPS = OPS_KK>
-cudaError_t launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b3, const GemmArgs &g,
-                        int num_sms, cudaStream_t s)
+cudaError_t launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b3, const CUtensorMap &out,
+                        const GemmArgs &g, int num_sms, cudaStream_t s)
 {
     cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&ffn_gemm_pair_kernel<EPI, OPS>),
-                                       static_cast<int>(kSmemBytes));
+                                       static_cast<int>(smem_bytes_of<EPI>()));
     if (err != cudaSuccess) return err;
     const int grid = (num_sms / 2) * 2;
-    return launch_k(ffn_gemm_pair_kernel<EPI, OPS>, dim3(grid), dim3(threads_of<EPI>()), kSmemBytes, s, a, b, b3,
-                    g);
+    return launch_k(ffn_gemm_pair_kernel<EPI, OPS>, dim3(grid), dim3(threads_of<EPI>()), smem_bytes_of<EPI>(), s, a, b, b3,
+                    out, g);
 }
 
 }  // namespace
@@ -570,7 +598,7 @@ cudaError_t launch_gemm_tc_f32_pair(const TcGemmArgs &t, int num_sms, cudaStream
         g.n_tiles = (t.n_out + BN - 1) / BN;
         g.m_tiles = static_cast<int>((t.m_total + PAIR_M - 1) / PAIR_M);
         g.m_total = t.m_total;
-        return launch_pair<EPI_F32, OPS_MN_MN>(tA, tB, tOut, g, num_sms, s);
+        return launch_pair<EPI_F32, OPS_MN_MN>(tA, tB, tOut, tOut, g, num_sms, s);
     }
     if (t.ragged_k) return cudaErrorInvalidValue;  // ragged K only with rows_mn
     if (t.a_rows == 0 || t.n_out == 0) return cudaSuccess;
@@ -603,9 +631,9 @@ cudaError_t launch_gemm_tc_f32_pair(const TcGemmArgs &t, int num_sms, cudaStream
         g.kb1 = static_cast<int>((t.k1 + BK - 1) / BK);
         g.kb_total = g.kb1 + static_cast<int>((t.k2 + BK - 1) / BK);
         g.a_col2 = static_cast<int>(t.k1);
-        return launch_pair<EPI_F32, OPS_K_MN>(tA, tB, tB3, g, num_sms, s);
+        return launch_pair<EPI_F32, OPS_K_MN>(tA, tB, tB3, tB3, g, num_sms, s);
     }
-    return launch_pair<EPI_F32>(tA, tB, tB, g, num_sms, s);
+    return launch_pair<EPI_F32>(tA, tB, tB, tB, g, num_sms, s);
 }
 
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid, cudaStream_t s)
@@ -618,11 +646,13 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid
     const bool swiglu = a.act == kSwiglu;
     const uint64_t rows = static_cast<uint64_t>(a.rows);
     const uint64_t E = static_cast<uint64_t>(a.E);
-    CUtensorMap tA, tB, tB3, tH, tW2;
-    // each CTA loads 128 rows of A and 128 rows of B per k-block
+    CUtensorMap tA, tB, tB3, tH, tW2, tHout, tYout;
+    // each CTA loads 128 rows of A and 128 rows of B per k-block; h and
+    // y_sorted are written through 32 x 32 store boxes
     if (!make_tmap_bf16(&tA, a.x_sorted, a.d, rows, BM) || !make_tmap_bf16(&tB, a.W1, a.d, E * a.F, 128) ||
         !make_tmap_bf16(&tB3, swiglu ? a.W3 : a.W1, a.d, E * a.F, 128) ||
-        !make_tmap_bf16(&tH, a.h, a.F, rows, BM) || !make_tmap_bf16(&tW2, a.W2, a.F, E * a.d, 128))
+        !make_tmap_bf16(&tH, a.h, a.F, rows, BM) || !make_tmap_bf16(&tW2, a.W2, a.F, E * a.d, 128) ||
+        !make_tmap_bf16_store(&tHout, a.h, a.F, rows) || !make_tmap_bf16_store(&tYout, a.y_sorted, a.d, rows))
         return cudaErrorInvalidValue;
 
     GemmArgs g1{};
@@ -637,8 +667,8 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid
     g1.n_out = a.F;
     g1.n_tiles = (a.F + (swiglu ? 127 : 255)) / (swiglu ? 128 : 256);
     g1.b_rows = a.F;
-    cudaError_t err = swiglu ? launch_pair<EPI_SWIGLU>(tA, tB, tB3, g1, num_sms, s)
-                             : launch_pair<EPI_GELU>(tA, tB, tB3, g1, num_sms, s);
+    cudaError_t err = swiglu ? launch_pair<EPI_SWIGLU>(tA, tB, tB3, tHout, g1, num_sms, s)
+                             : launch_pair<EPI_GELU>(tA, tB, tB3, tHout, g1, num_sms, s);
     if (err != cudaSuccess) return err;
     if (mid && (err = cudaEventRecord(mid, s)) != cudaSuccess) return err;
 
@@ -654,7 +684,7 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs &a, int num_sms, cudaEvent_t mid
     g2.n_out = a.d;
     g2.n_tiles = (a.d + 255) / 256;
     g2.b_rows = a.d;
-    return launch_pair<EPI_LINEAR>(tH, tW2, tW2, g2, num_sms, s);
+    return launch_pair<EPI_LINEAR>(tH, tW2, tW2, tYout, g2, num_sms, s);
 }
 
 }  // namespace moe

@@ -284,6 +284,7 @@ bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t o
 bool make_tmap_bf16_mn(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t groups);
 bool make_tmap_bf16_mn_rows(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t ld);
 bool make_tmap_f32_store(CUtensorMap *m, void *base, uint64_t inner, uint64_t rows, uint64_t groups);
+bool make_tmap_bf16_store(CUtensorMap *m, void *base, uint64_t inner, uint64_t rows);
 
 // C (fp32) from bf16 operands on tcgen05 (the backward's products on the
 // tensor cores), 128 x 256 tiles:

@@ -135,6 +135,14 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *m
 
 // 3-D tiled store of one box from shared memory (bulk async-group); the
 // box is clipped at the tensor's extents.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *smem_src, int32_t c0, int32_t c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(smem_u32(smem_src)), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *m, const void *smem_src, int32_t c0, int32_t c1,
                                              int32_t c2)
 {
@@ -274,6 +282,15 @@ __device__ __forceinline__ void cluster_sync()
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Arrival on an mbarrier of either CTA of the pair that orders nothing but
+// this thread's own earlier operations (CTA-scope release): for signals
+// whose payload is already complete in program order, such as "this warp's
+// TMEM loads have finished" after tcgen05.wait::ld.
+__device__ __forceinline__ void mbar_arrive_cluster_cta(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // Tile load into this CTA's shared memory whose completion is signalled on an

@@ -81,6 +81,22 @@ bool make_tmap_bf16_mn_rows(CUtensorMap *m, const void *base, uint64_t inner, ui
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 matrix [rows][inner] (inner contiguous) written by 32 x 32 boxes
+// from shared memory in the 64-byte swizzled layout (16-byte piece j of box
+// row r at piece j ^ ((r >> 1) & 3)); stores are clipped at the extents.
+bool make_tmap_bf16_store(CUtensorMap *m, void *base, uint64_t inner, uint64_t rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint32_t box[2] = {32, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 // fp32 tensor [groups][rows][inner] (inner contiguous) written by 32 x 32
 // boxes from 128-byte-swizzled shared memory; stores are clipped at the
 // extents.
