@@ -159,36 +159,54 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a)
 
 // Scores, top-k and gates from precomputed fp32 logits (the tcgen05 router
 // of the bf16 path writes them), for E > 32.  One CTA per 32-token dispatch
-// chunk; a group of 8 lanes owns one token (4 tokens per warp, 8 warps), and
-// lane q of the group holds a contiguous block of EJ = E_pad / 8 of its
-// experts.  Each expert gets the 64-bit rank key of (selection score desc,
-// id asc) (rank_key), so the k rounds of the selection are: every lane takes
-// its largest key below the previous round's winner, then a 3-step xor
-// butterfly over the group's 8 lanes; the winner's logit travels with its
-// key, from which every lane of the group forms the gate.  The chunk's
-// histogram uses integer shared-memory atomics (order-free); its sum of p is
-// taken per expert in token order.
-constexpr int kSelWarps = 8;
-constexpr int kGroup = 8;  // lanes per token
+// chunk; a group of G lanes owns one token, and lane q of the group holds a
+// contiguous block of EJ = E_pad / G of its experts.  Each expert gets the
+// 64-bit rank key of (selection score desc, id asc) (rank_key); every lane
+// first sorts its EJ keys, descending, with a bitonic network.  Each of the
+// k rounds is then a group max of the lanes' first keys (xor butterfly over
+// the G lanes) after which the lane holding the winner drops it (its list
+// moves up by one): k short rounds instead of k scans of all EJ keys.  The
+// winner's logit is read back from shared memory, where the group left its
+// logits; the gates' sum is formed round by round in choice order.  The
+// chunk's histogram uses integer shared-memory atomics (order-free); its
+// sum of p is taken per expert in token order.
+template <int N> __device__ __forceinline__ void bitonic_sort_desc(uint64_t (&v)[N])
+{
+#pragma unroll
+    for (int blk = 2; blk <= N; blk <<= 1)
+#pragma unroll
+        for (int j = blk >> 1; j > 0; j >>= 1)
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const uint64_t a = v[i], b = v[l];
+                    const bool sw = (i & blk) == 0 ? a < b : a > b;  // this block descending, or ascending
+                    v[i] = sw ? b : a;
+                    v[l] = sw ? a : b;
+                }
+            }
+}
 
-template <int EJ>
-__global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs a)
+template <int EJ, int G>
+__global__ void __launch_bounds__(kRT * G) select_kernel(SelectKernelArgs a)
 {
     pdl_enter();
     extern __shared__ float smem[];
     const int E = a.E, k = a.k;
     const int ZS = E + 1;
-    float *pt = smem;                                          // [32][E+1] p
+    float *pt = smem;                                          // [32][E+1] z, then p
     int *hist_s = reinterpret_cast<int *>(pt + kRT * ZS);      // [E]
     float *zl = reinterpret_cast<float *>(hist_s + kMaxE);     // [32] lse^2
     const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kRT;
     const int ntok = static_cast<int>(min64(kRT, a.N - tok0));
-    const int lane = threadIdx.x & 31, q = lane & (kGroup - 1);
-    const int t = threadIdx.x / kGroup;  // token of this lane's group, 0..31
+    const int lane = threadIdx.x & 31, q = lane & (G - 1);
+    const int t = threadIdx.x / G;  // token of this lane's group, 0..31
     const bool live = t < ntok;
     const int64_t n = tok0 + t;
     const int e0 = q * EJ;  // this lane's experts e0 .. e0 + EJ - 1
-    for (int e = threadIdx.x; e < E; e += kSelWarps * 32) hist_s[e] = 0;
+    float *zrow = pt + t * ZS;
+    for (int e = threadIdx.x; e < E; e += kRT * G) hist_s[e] = 0;
 
     // logits: the splits' partial sums in split order
     float z[EJ];
@@ -216,7 +234,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
     for (int j = 0; j < EJ; ++j)
         if (e0 + j < E) zmax = fmaxf(zmax, z[j]);
 #pragma unroll
-    for (int o = 1; o < kGroup; o <<= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
+    for (int o = 1; o < G; o <<= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
     float ex[EJ], esum = 0.f;
 #pragma unroll
     for (int j = 0; j < EJ; ++j) {
@@ -224,10 +242,11 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
         esum += ex[j];
     }
 #pragma unroll
-    for (int o = 1; o < kGroup; o <<= 1) esum += __shfl_xor_sync(0xffffffffu, esum, o);
+    for (int o = 1; o < G; o <<= 1) esum += __shfl_xor_sync(0xffffffffu, esum, o);
     const float inv_esum = 1.0f / esum;
     const float lse = zmax + logf(esum);
-    // selection keys (0: below every real key)
+    // selection keys (0: below every real key), sorted; the logits to shared
+    // memory for the gates
     uint64_t key[EJ];
 #pragma unroll
     for (int j = 0; j < EJ; ++j) {
@@ -237,59 +256,44 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
             float sc = z[j];
             if (a.router == kSigmoid) sc = 1.0f / (1.0f + expf(-z[j])) + (a.b_sel ? a.b_sel[e] : 0.f);
             key[j] = rank_key(sc, e);
+            zrow[e] = z[j];
         }
     }
-    // k rounds: the group's largest key below the previous winner
-    uint64_t bound = ~0ull;
-    int my_id = -1;        // lane q < k (and q + 8 < k): the q-th (q + 8-th) choice
-    float my_z = 0.f, my_z2 = 0.f;
-    int my_id2 = -1;
-    float zsel[kMaxK];
-#pragma unroll
-    for (int r = 0; r < kMaxK; ++r) zsel[r] = 0.f;
-#pragma unroll 1
-    for (int r = 0; r < k; ++r) {
-        uint64_t best = 0;
-        float bz = 0.f;
-#pragma unroll
-        for (int j = 0; j < EJ; ++j) {
-            if (key[j] < bound && key[j] > best) {
-                best = key[j];
-                bz = z[j];
-            }
-        }
-#pragma unroll
-        for (int o = 1; o < kGroup; o <<= 1) {
-            const uint64_t ob = __shfl_xor_sync(0xffffffffu, best, o);
-            const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
-            if (ob > best) {
-                best = ob;
-                bz = oz;
-            }
-        }
-        bound = best;
-        const int e = 0xFFFF - static_cast<int>(best & 0xFFFFu);
-#pragma unroll
-        for (int i = 0; i < kMaxK; ++i)
-            if (i == r) zsel[i] = bz;
-        if (q == r) {
-            my_id = e;
-            my_z = bz;
-        }
-        if (q + kGroup == r) {
-            my_id2 = e;
-            my_z2 = bz;
-        }
-    }
-    // gates: raw gate of each choice, their sum in choice order, then this
-    // lane's one or two outputs
+    bitonic_sort_desc(key);
+    __syncwarp();
     auto raw_gate = [&](float zr) {
         return a.router == kSigmoid ? 1.0f / (1.0f + expf(-zr)) : expf(zr - zmax);
     };
-    float gs = 0.f;
+    // k rounds: the group's largest remaining key
+    int my_id = -1, my_id2 = -1;  // lane q < k (and q + G < k): the q-th (q + G-th) choice
+    float my_z = 0.f, my_z2 = 0.f, gs = 0.f;
+#pragma unroll 1
+    for (int r = 0; r < k; ++r) {
+        uint64_t best = key[0];
 #pragma unroll
-    for (int r = 0; r < kMaxK; ++r)
-        if (r < k) gs += raw_gate(zsel[r]);
+        for (int o = 1; o < G; o <<= 1) {
+            const uint64_t ob = __shfl_xor_sync(0xffffffffu, best, o);
+            best = ob > best ? ob : best;
+        }
+        if (key[0] == best) {  // the winner's lane (keys are unique)
+#pragma unroll
+            for (int j = 0; j + 1 < EJ; ++j) key[j] = key[j + 1];
+            key[EJ - 1] = 0ull;
+        }
+        const int e = 0xFFFF - static_cast<int>(best & 0xFFFFu);
+        const float ez = zrow[e];
+        gs += raw_gate(ez);
+        if (q == r) {
+            my_id = e;
+            my_z = ez;
+        }
+        if (q + G == r) {
+            my_id2 = e;
+            my_z2 = ez;
+        }
+    }
+    // gates: raw gate of each choice over their sum (in choice order), then
+    // this lane's one or two outputs
     auto weight = [&](float zr) {
         const float g = raw_gate(zr);
         float wr;
@@ -304,9 +308,9 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
             a.w[n * k + q] = weight(my_z);
             atomicAdd(&hist_s[my_id], 1);
         }
-        if (q + kGroup < k) {
-            a.ids[n * k + q + kGroup] = my_id2;
-            a.w[n * k + q + kGroup] = weight(my_z2);
+        if (q + G < k) {
+            a.ids[n * k + q + G] = my_id2;
+            a.w[n * k + q + G] = weight(my_z2);
             atomicAdd(&hist_s[my_id2], 1);
         }
         if (q == 0) {
@@ -314,19 +318,20 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectKernelArgs
             if (a.lse) a.lse[n] = lse;
         }
     }
+    __syncwarp();  // the group's logits have been read: p replaces them
     // p for the chunk's sums (and probs if asked for)
 #pragma unroll
     for (int j = 0; j < EJ; ++j) {
         const int e = e0 + j;
         if (e < E) {
             const float p = live ? ex[j] * inv_esum : 0.f;
-            pt[t * ZS + e] = p;
+            zrow[e] = p;
             if (live && a.probs) a.probs[n * E + e] = p;
         }
     }
     __syncthreads();
     if (a.zpart && threadIdx.x == 0) a.zpart[blockIdx.x] = chunk_sum(zl, ntok);
-    for (int e = threadIdx.x; e < E; e += kSelWarps * 32) {
+    for (int e = threadIdx.x; e < E; e += kRT * G) {
         if (a.psum) {
             float s = 0.f;
             for (int tt = 0; tt < ntok; ++tt) s += pt[tt * ZS + e];
@@ -359,15 +364,15 @@ cudaError_t launch_select(const SelectKernelArgs &a, cudaStream_t s)
 {
     const int64_t grid = num_chunks(a.N);
     if (grid == 0) return cudaSuccess;
-    // EJ: experts per lane (8 lanes cover 64, 128 or 256 experts); logits
-    // rows of ld >= E columns, a multiple of 4 (columns E .. ld-1 are read
-    // as whole float4s and ignored)
+    // logits rows of ld >= E columns, a multiple of 4 (columns E .. ld-1 are
+    // read as whole float4s and ignored)
     if (a.ld % 4 != 0 || a.ld < a.E || a.E > kMaxE) return cudaErrorInvalidValue;
     const size_t smem = sizeof(float) * (kRT * (a.E + 1) + kRT) + sizeof(int) * kMaxE;
-    const dim3 g(static_cast<unsigned>(grid)), b(kSelWarps * 32);
-    if (a.E <= 64) return launch_k(select_kernel<8>, g, b, smem, s, a);
-    if (a.E <= 128) return launch_k(select_kernel<16>, g, b, smem, s, a);
-    return launch_k(select_kernel<32>, g, b, smem, s, a);
+    // experts per lane x lanes per token: 8 x 8, 16 x 8 or 16 x 16
+    const dim3 g(static_cast<unsigned>(grid));
+    if (a.E <= 64) return launch_k(select_kernel<8, 8>, g, dim3(kRT * 8), smem, s, a);
+    if (a.E <= 128) return launch_k(select_kernel<16, 8>, g, dim3(kRT * 8), smem, s, a);
+    return launch_k(select_kernel<16, 16>, g, dim3(kRT * 16), smem, s, a);
 }
 
 cudaError_t launch_router(int dtype, const RouterArgs &a, cudaStream_t s)
