@@ -102,11 +102,20 @@ def traffic_for(kernel: str, workload: str):
     ent = table.get(f"{kernel}:{workload}")
     if not ent:
         return None
-    src = os.path.join(ROOT, ent["source"])
-    if not os.path.exists(src):
-        return None
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return ent["bytes_per_launch"] if h == ent["source_sha256_16"] else None
+    h = sources_hash(ent["sources"])
+    return ent["bytes_per_launch"] if h is not None and h == ent["sources_sha256_16"] else None
+
+
+def sources_hash(sources):
+    """sha256 (first 16 hex digits) of the given repository files, concatenated in order."""
+    hasher = hashlib.sha256()
+    for rel in sources:
+        src = os.path.join(ROOT, rel)
+        if not os.path.exists(src):
+            return None
+        with open(src, "rb") as f:
+            hasher.update(f.read())
+    return hasher.hexdigest()[:16]
 
 
 class ClockSampler:

@@ -158,10 +158,11 @@ MOE_API size_t moe_workspace_size(const moe_config *cfg);
  * routed_scaling).  b_e (sigmoid router only, may be NULL) enters the
  * selection score only, never the weights (sec. 2.5).  probs [N, E] (may be
  * NULL) receives softmax(z_n) for every router.  bf16 with E <= 32 runs as
- * one kernel (tensor-core logits split over d across a thread-block cluster,
- * selection fused); bf16 with E > 32 keeps partial logits in the workspace
- * between the logits kernel and the selection kernel; fp32 runs one CUDA-core
- * kernel.
+ * one streaming kernel (each CTA reads the rows of x of its 32 tokens once,
+ * the products on warp-level tensor-core MMAs, the selection fused); bf16
+ * with E > 32 keeps the logits (partial sums over d when the reduction is
+ * split) in the workspace between the tcgen05 logits kernel and the
+ * selection kernel; fp32 runs one CUDA-core kernel.
  */
 MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const void *W_g,
                      const float *b_e, int32_t *topk_ids, float *topk_w,

@@ -41,14 +41,12 @@ int router_splits(int64_t N, int d);
 cudaError_t launch_router_logits_sm100(const void *x, const void *W_g, float *logits, int64_t N, int d, int E,
                                        int32_t *status, bool clear_status, cudaStream_t s);
 // E <= 32: logits, scores, top-k, gates and the per-chunk statistics of
-// RouterArgs in one tcgen05 kernel (clusters of router_splits CTAs).
-cudaError_t launch_router_fused_sm100(const RouterArgs &r, int32_t *status, bool clear_status, cudaStream_t s);
-// E <= 32: the same in one streaming kernel, one CTA per 32-token chunk,
-// warps over column ranges of d, warp-level MMAs (router_mma.cu).
+// RouterArgs in one streaming kernel, one CTA per 32-token chunk, warps over
+// column ranges of d, warp-level MMAs (router_mma.cu).
 cudaError_t launch_router_stream(const RouterArgs &r, int32_t *status, bool clear_status, cudaStream_t s);
 
 // Scores, top-k, gates and per-chunk statistics from fp32 logits (E > 32;
-// smaller E selects inside launch_router_fused_sm100).
+// smaller E selects inside launch_router_stream).
 struct SelectKernelArgs {
     const float *logits;  // [splits, N, ld] partial logits, summed in split order
     const float *b_sel;   // [E] or null (sigmoid router only)

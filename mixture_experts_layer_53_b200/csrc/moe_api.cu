@@ -4,7 +4,6 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
-#include <cstdlib>
 #include <cstdint>
 #include <mutex>
 #include <string>
@@ -246,12 +245,7 @@ cudaError_t launch_route(const moe_config *c, const RouterArgs &r, int32_t *stat
                          bool clear_status = false)
 {
     if (c->dtype != MOE_BF16) return launch_router(c->dtype, r, s);
-    static const bool tc_router = [] {
-        const char *v = getenv("MOE_ROUTER_TC");
-        return v && v[0] == '1';
-    }();
-    if (c->E <= 32) return tc_router ? launch_router_fused_sm100(r, status, clear_status, s)
-                                     : launch_router_stream(r, status, clear_status, s);
+    if (c->E <= 32) return launch_router_stream(r, status, clear_status, s);
     cudaError_t err = launch_router_logits_sm100(r.x, r.Wg, logits, r.N, r.d, r.E, status, clear_status, s);
     if (err != cudaSuccess) return err;
     SelectKernelArgs sk{logits, r.b_sel, r.ids, r.w, r.probs, r.hist, r.psum, r.zpart, r.N, logits_ld(r.E),

@@ -3,8 +3,8 @@
 //
 // Course module "Mixture of Experts: routing, sorted dispatch, Switch aux
 // loss, aux-free bias", sec. 2 symbol table: z_n = W_g x_n.  The scores,
-// top-k and gates follow in select_kernel (router.cu), which spreads the
-// tokens over every SM, one warp per token.
+// top-k and gates follow in select_kernel (router.cu); E <= 32 uses the
+// streaming router of router_mma.cu instead.
 //
 // The product is [N, d] x [d, E] with small E, so the kernel is bound by
 // reading x.  To keep every SM streaming x even when N / 128 is small, the
@@ -22,18 +22,11 @@
 // sums are only num_kb / nacc steps deep, which keeps the logits close enough
 // to an fp32 dot product for the 1e-5 tolerance of the Switch loss.
 //
-// For E <= 32 (router_kernel_fused<EB>) the selection is fused in: the S
-// split CTAs of a tile form a thread-block cluster, each leaves its partial
-// rows in its own shared memory, and after a cluster barrier the epilogue
-// warp of chunk q in CTA q % S adds the S partials of its 32 tokens in split
-// order through distributed shared memory and runs one thread per token
-// (select_thread_chunk): no logits in HBM and no second kernel.
 #include <cuda.h>
 
 #include "common.cuh"
 #include "host_util.h"
 #include "kernels.h"
-#include "router_select.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -72,26 +65,8 @@ struct LArgs {
     int nacc;            // TMEM accumulators, k-block kb -> kb % nacc
     uint32_t acc_cols;   // TMEM columns between accumulators (power of 2 >= max(E_pad, 32))
     uint32_t tmem_cols;  // nacc * acc_cols rounded up to a power of 2
-    // fused selection (E <= 32)
-    SelectArgs sel;
-    float *psum;
-    int32_t *hist;
-    float *zpart;
 };
 
-__device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t addr)
-{
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
-}
-
-// EB == 0: partial logits to HBM.  EB in {8, 16, 32}: fused selection for
-// E <= EB, launched as clusters of `splits` CTAs.
-template <int EB>
 __global__ void __launch_bounds__(THREADS, 1)
     router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                          const LArgs a)
@@ -106,8 +81,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                                                  ~static_cast<uintptr_t>(1023));
     const int stage_bytes = A_BYTES + a.E_pad * BK * 2;
     Ctl *ctl = reinterpret_cast<Ctl *>(tiles + a.stages * stage_bytes);
-    // fused: partial rows [BM][E_pad] fp32 of this CTA's split
-    float *part = reinterpret_cast<float *>((reinterpret_cast<uintptr_t>(ctl + 1) + 15) & ~static_cast<uintptr_t>(15));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort_flag = &ctl->abort;
 
@@ -205,39 +178,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int64_t n = static_cast<int64_t>(row0) + q * 32 + lane;
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&ctl->tfull, 0, abort_flag, a.status));
-        if (ok && num_kb > 0 && EB > 0 && EB <= 16) {
-            // E_pad = 16: the first 16 columns of each accumulator; the loads
-            // of up to four accumulators are in flight at once, then added in
-            // accumulator order
+        if (ok && num_kb > 0) {
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
             const int used = min(a.nacc, num_kb);
-            float zs[16];
-            for (int s0 = 0; s0 < used; s0 += 4) {
-                uint32_t t[4][16];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    if (s0 + i < used) tmem_ld16(taddr + static_cast<uint32_t>(s0 + i) * a.acc_cols, t[i]);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    if (s0 + i >= used) break;
-#pragma unroll
-                    for (int u = 0; u < 16; ++u)
-                        zs[u] = (s0 + i == 0) ? __uint_as_float(t[i][u]) : zs[u] + __uint_as_float(t[i][u]);
-                }
-            }
-            float *zrow = part + (q * 32 + lane) * a.E_pad;
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-                *reinterpret_cast<float4 *>(zrow + 4 * v) = make_float4(zs[4 * v], zs[4 * v + 1], zs[4 * v + 2],
-                                                                        zs[4 * v + 3]);
-        } else if (ok && num_kb > 0) {
-            tc_fence_after();
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-            const int used = min(a.nacc, num_kb);
-            float *zrow = EB == 0 ? a.logits + (static_cast<int64_t>(split) * a.N + n) * a.ld
-                                  : part + (q * 32 + lane) * a.E_pad;
+            float *zrow = a.logits + (static_cast<int64_t>(split) * a.N + n) * a.ld;
             for (int c0 = 0; c0 < a.E_pad; c0 += 32) {
                 uint32_t r[32];
                 for (int s0 = 0; s0 < used; s0 += 2) {
@@ -260,21 +205,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                             r[u] = __float_as_uint(__uint_as_float(r[u]) + __uint_as_float(t2[u]));
                     }
                 }
-                if (EB == 0 && n < a.N) {
+                if (n < a.N) {
 #pragma unroll
                     for (int v = 0; v < 8; ++v) {
                         const int c = c0 + 4 * v;
                         if (c < a.ld)  // ld is a multiple of 4
                             st16(zrow + c, make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]));
-                    }
-                }
-                if (EB > 0) {  // the whole padded row into shared memory
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        const int c = c0 + 4 * v;
-                        if (c < a.E_pad)
-                            *reinterpret_cast<uint4 *>(zrow + c) =
-                                make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
                     }
                 }
             }
@@ -286,36 +222,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, a.tmem_cols);
-    }
-    if constexpr (EB > 0) {
-        cluster_sync();  // every split's partial rows are in place
-        if (warp >= 2) {
-            const int q = warp & 3;
-            // chunks past N (the last tile's tail) have no statistics slots
-            if (q % a.splits == static_cast<int>(cluster_ctarank()) &&
-                static_cast<int64_t>(row0) + q * 32 < a.N) {  // warp-uniform
-                const int t = q * 32 + lane;
-                const int64_t n = static_cast<int64_t>(row0) + t;
-                float z[EB];
-#pragma unroll
-                for (int e = 0; e < EB; ++e) z[e] = 0.f;
-                const uint32_t row_addr = smem_u32(part + t * a.E_pad);
-                for (int sp = 0; sp < a.splits; ++sp) {  // split order
-                    const uint32_t ra = mapa_shared(row_addr, static_cast<uint32_t>(sp));
-#pragma unroll
-                    for (int e = 0; e < EB; e += 4) {
-                        const float4 v = ld_shared_cluster_f4(ra + e * 4);
-                        z[e] += v.x;
-                        z[e + 1] += v.y;
-                        z[e + 2] += v.z;
-                        z[e + 3] += v.w;
-                    }
-                }
-                select_thread_chunk<EB>(z, a.sel, a.psum, a.hist, a.zpart, n, n < a.N,
-                                        static_cast<int64_t>(row0 / 32 + q));
-            }
-        }
-        cluster_sync();  // no CTA leaves while its rows may still be read
     }
 }
 
@@ -373,23 +279,12 @@ bool setup(LArgs &a, CUtensorMap &tX, CUtensorMap &tW, const void *x, const void
            make_tmap_bf16(&tW, W_g, d, static_cast<uint64_t>(E), static_cast<uint32_t>(a.E_pad));
 }
 
-constexpr int kSmemMax = 1024 + SMEM_TILE_BUDGET + static_cast<int>(sizeof(Ctl)) + 16 + BM * 32 * 4;
+constexpr int kSmemMax = 1024 + SMEM_TILE_BUDGET + static_cast<int>(sizeof(Ctl));
 
-size_t smem_bytes(const LArgs &a, bool fused)
+size_t smem_bytes(const LArgs &a)
 {
     const int stage_bytes = A_BYTES + a.E_pad * BK * 2;
-    return 1024 + static_cast<size_t>(a.stages) * stage_bytes + sizeof(Ctl) +
-           (fused ? 16 + static_cast<size_t>(BM) * a.E_pad * 4 : 0);
-}
-
-template <int EB>
-cudaError_t launch_fused(const CUtensorMap &tX, const CUtensorMap &tW, const LArgs &a, cudaStream_t s)
-{
-    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&router_logits_kernel<EB>), kSmemMax);
-    if (err != cudaSuccess) return err;
-    const int64_t grid = (a.N + BM - 1) / BM * a.splits;
-    return launch_k_cluster(router_logits_kernel<EB>, dim3(static_cast<unsigned>(grid)), dim3(THREADS),
-                            smem_bytes(a, true), s, static_cast<unsigned>(a.splits), tX, tW, a);
+    return 1024 + static_cast<size_t>(a.stages) * stage_bytes + sizeof(Ctl);
 }
 
 }  // namespace
@@ -402,27 +297,11 @@ cudaError_t launch_router_logits_sm100(const void *x, const void *W_g, float *lo
     CUtensorMap tX, tW;
     if (!setup(a, tX, tW, x, W_g, N, d, E, status, clear_status)) return cudaErrorInvalidValue;
     a.logits = logits;
-    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&router_logits_kernel<0>), kSmemMax);
+    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void *>(&router_logits_kernel), kSmemMax);
     if (err != cudaSuccess) return err;
     const int64_t grid = (N + BM - 1) / BM * a.splits;
-    return launch_k(router_logits_kernel<0>, dim3(static_cast<unsigned>(grid)), dim3(THREADS), smem_bytes(a, false),
-                    s, tX, tW, a);
-}
-
-cudaError_t launch_router_fused_sm100(const RouterArgs &r, int32_t *status, bool clear_status, cudaStream_t s)
-{
-    if (r.N == 0) return cudaSuccess;
-    if (r.E > 32) return cudaErrorInvalidValue;
-    LArgs a{};
-    CUtensorMap tX, tW;
-    if (!setup(a, tX, tW, r.x, r.Wg, r.N, r.d, r.E, status, clear_status)) return cudaErrorInvalidValue;
-    a.sel = SelectArgs{r.b_sel, r.ids, r.w, r.probs, r.E, r.k, r.router, r.norm_topk, r.scaling, r.lse};
-    a.psum = r.psum;
-    a.hist = r.hist;
-    a.zpart = r.zpart;
-    if (r.E <= 8) return launch_fused<8>(tX, tW, a, s);
-    if (r.E <= 16) return launch_fused<16>(tX, tW, a, s);
-    return launch_fused<32>(tX, tW, a, s);
+    return launch_k(router_logits_kernel, dim3(static_cast<unsigned>(grid)), dim3(THREADS), smem_bytes(a), s, tX,
+                    tW, a);
 }
 
 }  // namespace moe
