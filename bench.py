@@ -100,7 +100,7 @@ def traffic_for(kernel: str, workload: str):
     with open(path) as f:
         table = json.load(f)
     ent = table.get(f"{kernel}:{workload}")
-    if not ent:
+    if not ent or "sources" not in ent:
         return None
     h = sources_hash(ent["sources"])
     return ent["bytes_per_launch"] if h is not None and h == ent["sources_sha256_16"] else None
