@@ -31,6 +31,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/sec (bf16, 1 B200); expert-GEMM TFLOPS as % of bf16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# timed regions at least this long are held against the sustained bf16 peak
+# (the power cap has settled: median SM clocks near 1.1-1.3 GHz were seen
+# from about half a second of back-to-back expert GEMMs on)
+SUSTAINED_REGION_MS = 250.0
 L2_BYTES = 126 * 1024 * 1024
 # tokens of the workload the CPU oracle handles per reference step (about 1-3 s each)
 REF_TOKENS_PER_STEP = {"tiny_fp32": 64, "gpt2_moe": 32, "mixtral": 1, "deepseek_v3": 1, "qwen3_skew": 8,
@@ -580,11 +584,13 @@ def run_native(args, wl):
         gemm1_flops = 2 * (2 if wl.act == "swiglu" else 1) * wl.d_model * wl.d_ff * wl.N * wl.k
         gemm1_s = gemm1_ms / 1000.0
         ffn_s = (stages["gemm1"] + stages["gemm2"]) / 1000.0
-        # the timed region lasts well under the seconds it takes the power cap
-        # to settle, so the denominator is the burst bf16 peak; the sustained
-        # fraction is reported beside it
+        # a timed region well under the time the power cap takes to settle is
+        # held against the burst bf16 peak, a longer one against the
+        # sustained peak; the other fraction is reported beside it
         burst = peaks["bf16_tflops"]
         sustained = peaks.get("bf16_tflops_sustained", burst)
+        long_region = total_ms >= SUSTAINED_REGION_MS
+        peak = sustained if long_region else burst
         achieved = gemm1_flops / gemm1_s / 1e12
         ffn_tflops = wl.expert_flops / ffn_s / 1e12
         fp32 = wl.dtype == "f32"
@@ -597,9 +603,12 @@ def run_native(args, wl):
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
             "config": dict(describe(wl), l2=("inputs larger than L2 (expert weights %.2f GB)" % (weights_bytes(wl) / 1e9))
                            if big_inputs else "L2 flushed between steps (256 MiB write), per-step events"),
-            "roofline": {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": burst,
-                         "unit": "TFLOP/s", "frac": achieved / burst,
-                         "peak_source": f"{peak_src} bf16_tflops (burst; timed region {total_ms:.0f} ms)",
+            "roofline": {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": (f"{peak_src} bf16_tflops_sustained (timed region {total_ms:.0f} ms)"
+                                         if long_region else
+                                         f"{peak_src} bf16_tflops (burst; timed region {total_ms:.0f} ms)"),
+                         "frac_of_burst_peak": achieved / burst,
                          "frac_of_sustained_peak": achieved / sustained,
                          "traffic": traffic_for("gemm1", wl.name), "flops_per_launch": gemm1_flops},
             "expert_ffn": {"tflops": ffn_tflops,
