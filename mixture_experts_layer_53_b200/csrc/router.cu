@@ -159,8 +159,8 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a)
 
 // Scores, top-k and gates from precomputed fp32 logits (the tcgen05 router
 // of the bf16 path writes them), for E > 32.  One CTA per 32-token dispatch
-// chunk; a group of G lanes owns one token, and lane q of the group holds a
-// contiguous block of EJ = E_pad / G of its experts.  Each expert gets the
+// chunk; a group of G lanes (up to a whole warp) owns one token, and lane q
+// of the group holds a contiguous block of EJ = E_pad / G of its experts.  Each expert gets the
 // 64-bit rank key of (selection score desc, id asc) (rank_key); every lane
 // first sorts its EJ keys, descending, with a bitonic network.  Each of the
 // k rounds is then a group max of the lanes' first keys (xor butterfly over
@@ -368,11 +368,12 @@ cudaError_t launch_select(const SelectKernelArgs &a, cudaStream_t s)
     // read as whole float4s and ignored)
     if (a.ld % 4 != 0 || a.ld < a.E || a.E > kMaxE) return cudaErrorInvalidValue;
     const size_t smem = sizeof(float) * (kRT * (a.E + 1) + kRT) + sizeof(int) * kMaxE;
-    // experts per lane x lanes per token: 8 x 8, 16 x 8 or 16 x 16
+    // experts per lane x lanes per token: 8 x 8, 8 x 16 or 8 x 32 (eight keys
+    // per lane keep the registers low enough for 32 warps per SM)
     const dim3 g(static_cast<unsigned>(grid));
     if (a.E <= 64) return launch_k(select_kernel<8, 8>, g, dim3(kRT * 8), smem, s, a);
-    if (a.E <= 128) return launch_k(select_kernel<16, 8>, g, dim3(kRT * 8), smem, s, a);
-    return launch_k(select_kernel<16, 16>, g, dim3(kRT * 16), smem, s, a);
+    if (a.E <= 128) return launch_k(select_kernel<8, 16>, g, dim3(kRT * 16), smem, s, a);
+    return launch_k(select_kernel<8, 32>, g, dim3(kRT * 32), smem, s, a);
 }
 
 cudaError_t launch_router(int dtype, const RouterArgs &a, cudaStream_t s)
