@@ -1,0 +1,67 @@
+"""Host-side logic of bench.py (no GPU): the roofline denominators and the
+measured-traffic table keyed by a hash of the kernel's sources."""
+import json
+import os
+
+import pytest
+
+import bench
+
+
+def _root(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    return tmp_path
+
+
+def test_peaks_fallback_without_file(tmp_path, monkeypatch):
+    _root(tmp_path, monkeypatch)
+    peaks, src = bench.load_peaks()
+    assert src == "fallback"
+    assert peaks == bench.FALLBACK_PEAKS
+
+
+def test_peaks_from_file_and_partial_file(tmp_path, monkeypatch):
+    root = _root(tmp_path, monkeypatch)
+    full = {"hbm_gbs": 6452.8, "bf16_tflops": 1662.0, "bf16_tflops_sustained": 1383.8, "note": "x"}
+    (root / "MEASURED_PEAKS.json").write_text(json.dumps(full))
+    peaks, src = bench.load_peaks()
+    assert src == "measured"
+    assert peaks["bf16_tflops"] == 1662.0 and peaks["hbm_gbs"] == 6452.8
+    (root / "MEASURED_PEAKS.json").write_text(json.dumps({"bf16_tflops": 1700}))
+    peaks, src = bench.load_peaks()
+    assert src == "measured (partly fallback)"
+    assert peaks["bf16_tflops"] == 1700.0
+    assert peaks["hbm_gbs"] == bench.FALLBACK_PEAKS["hbm_gbs"]
+    (root / "MEASURED_PEAKS.json").write_text("not json")
+    assert bench.load_peaks()[1] == "fallback"
+
+
+@pytest.mark.parametrize("region_ms,sustained", [(46.0, False), (249.9, False), (250.0, True), (554.0, True)])
+def test_tensor_peak_by_region(region_ms, sustained):
+    peaks = {"hbm_gbs": 1.0, "bf16_tflops": 1662.0, "bf16_tflops_sustained": 1383.8}
+    peak, name = bench.tensor_peak(peaks, region_ms)
+    assert peak == (1383.8 if sustained else 1662.0)
+    assert ("sustained" in name) == sustained
+
+
+def test_traffic_only_while_sources_unchanged(tmp_path, monkeypatch):
+    root = _root(tmp_path, monkeypatch)
+    srcs = ["a.cu", "b.cuh"]
+    (root / "a.cu").write_text("kernel a")
+    (root / "b.cuh").write_text("header b")
+    table = {"gemm1:mixtral": {"bytes_per_launch": 123, "sources": srcs,
+                               "sources_sha256_16": bench.sources_hash(srcs)}}
+    (root / "profiles" / "traffic.json").write_text(json.dumps(table))
+    assert bench.traffic_for("gemm1", "mixtral") == 123
+    assert bench.traffic_for("gemm1", "qwen3_skew") is None
+    (root / "b.cuh").write_text("header b, edited")
+    assert bench.traffic_for("gemm1", "mixtral") is None
+    os.remove(root / "a.cu")
+    assert bench.traffic_for("gemm1", "mixtral") is None
+
+
+def test_traffic_entry_without_sources_is_ignored(tmp_path, monkeypatch):
+    root = _root(tmp_path, monkeypatch)
+    (root / "profiles" / "traffic.json").write_text(json.dumps({"gemm1:mixtral": {"bytes_per_launch": 1}}))
+    assert bench.traffic_for("gemm1", "mixtral") is None
