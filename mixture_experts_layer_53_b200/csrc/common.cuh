@@ -137,5 +137,13 @@ __device__ __forceinline__ float gelu_erf(float v)
     return v * (v >= 0.0f ? 1.0f - q : q);
 }
 __device__ __forceinline__ float silu(float v) { return v / (1.0f + expf(-v)); }
+// The same on the special-function unit, for results rounded to bf16:
+// v / (1 + 2^(-v log2 e)) with ex2.approx and rcp.approx (relative error a
+// few 1e-7; large negative v: the exponential overflows to +inf and the
+// reciprocal to 0, so silu -> -0).
+__device__ __forceinline__ float silu_approx(float v)
+{
+    return v * rcp_approx(1.0f + ex2_approx(v * -1.44269504f));
+}
 
 }  // namespace moe

@@ -44,7 +44,8 @@ __device__ __forceinline__ void epi_bf16_math(const uint32_t (&acc)[32], const u
         float o[8];
         if constexpr (EPI == EPIB_SWIGLU) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) o[u] = silu(__uint_as_float(acc[v * 8 + u])) * __uint_as_float(up[v * 8 + u]);
+            for (int u = 0; u < 8; ++u)
+                o[u] = silu_approx(__uint_as_float(acc[v * 8 + u])) * __uint_as_float(up[v * 8 + u]);
         } else {
 #pragma unroll
             for (int u = 0; u < 8; ++u) o[u] = __uint_as_float(acc[v * 8 + u]);
