@@ -156,105 +156,6 @@ __device__ __forceinline__ uint64_t rank_key(float score, int e)
     return (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(0xFFFF - e);
 }
 
-// One token per warp for 32 < E <= 32 * EJ (lane l holds experts l + 32 j in
-// z[j]).  Softmax / sigmoid scores as select_token; each of the k rounds
-// takes every lane's best untaken candidate by its rank_key, a warp max of
-// the keys (xor butterfly), and the winner's gate from the winning lane.
-// Lane r < k ends with the r-th choice: writes ids / w for token n (if
-// `write`), probs (if given), and returns in z[] the token's p.  *sel_id /
-// *sel_gate: lane r's choice (lanes >= k: -1 / 0).  Returns log sum_e exp z.
-template <int EJ>
-__device__ __forceinline__ float select_token_keys(float (&z)[EJ], const SelectArgs &a, int64_t n, bool write,
-                                                   int *sel_id)
-{
-    const int lane = threadIdx.x & 31;
-    const int E = a.E, k = a.k;
-    float zmax = -FLT_MAX;
-#pragma unroll
-    for (int j = 0; j < EJ; ++j)
-        if (lane + 32 * j < E) zmax = fmaxf(zmax, z[j]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
-    float ex[EJ], graw[EJ];
-    uint64_t key[EJ];
-    float esum = 0.f;
-#pragma unroll
-    for (int j = 0; j < EJ; ++j) {
-        const int e = lane + 32 * j;
-        ex[j] = 0.f;
-        graw[j] = 0.f;
-        key[j] = 0;  // below every real key
-        if (e < E) {
-            ex[j] = expf(z[j] - zmax);
-            esum += ex[j];
-            if (a.router == kSigmoid) {
-                const float sg = 1.0f / (1.0f + expf(-z[j]));
-                key[j] = rank_key(sg + (a.b_sel ? a.b_sel[e] : 0.f), e);
-                graw[j] = sg;
-            } else {
-                key[j] = rank_key(z[j], e);
-                graw[j] = ex[j];
-            }
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) esum += __shfl_xor_sync(0xffffffffu, esum, o);
-    const float inv_esum = 1.0f / esum;
-
-    uint32_t taken = 0;
-    int my_id = -1;
-    float my_gate = 0.f;
-#pragma unroll 1
-    for (int r = 0; r < k; ++r) {
-        uint64_t best = 0;
-        float bg = 0.f;
-        int bj = 0;
-#pragma unroll
-        for (int j = 0; j < EJ; ++j) {
-            if (!((taken >> j) & 1u) && key[j] > best) {
-                best = key[j];
-                bg = graw[j];
-                bj = j;
-            }
-        }
-        uint64_t win = best;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const uint64_t other = __shfl_xor_sync(0xffffffffu, win, o);
-            win = other > win ? other : win;
-        }
-        const int e = 0xFFFF - static_cast<int>(win & 0xFFFFu);
-        const int owner = e & 31;
-        if (lane == owner) taken |= 1u << bj;  // the owner's best is the winner
-        const float g = __shfl_sync(0xffffffffu, bg, owner);
-        if (lane == r) {
-            my_id = e;
-            my_gate = g;
-        }
-    }
-    // sum of the k chosen gates, in a fixed butterfly order
-    float gs = lane < k ? my_gate : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
-    if (write && a.lse && lane == 0) a.lse[n] = zmax + logf(esum);
-    if (write && lane < k) {
-        float wr;
-        if (a.router == kSoftmaxTopk) wr = a.norm_topk ? my_gate / gs : my_gate * inv_esum;
-        else if (a.router == kTopkSoftmax) wr = my_gate / gs;
-        else wr = a.norm_topk ? my_gate / gs : my_gate;
-        a.ids[n * k + lane] = my_id;
-        a.w[n * k + lane] = wr * a.scaling;
-    }
-#pragma unroll
-    for (int j = 0; j < EJ; ++j) {
-        const int e = lane + 32 * j;
-        z[j] = e < E ? ex[j] * inv_esum : 0.f;
-        if (write && a.probs && e < E) a.probs[n * E + e] = z[j];
-    }
-    *sel_id = my_id;
-    return zmax + logf(esum);
-}
-
 // Sums v[e] over the 32 lanes of a warp for all EB (8, 16 or 32) values at
 // once, in a fixed order: at each step the lanes with bit o set keep the upper
 // half of their values and add their partner's copy of it, the others the
