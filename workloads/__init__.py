@@ -130,7 +130,7 @@ def make_x(wl: Workload) -> torch.Tensor:
     """Token activations [N, d] in the workload's dtype (on the CPU)."""
     g = _gen(wl.seed * 7 + 1)
     x = torch.randn((wl.N, wl.d_model), generator=g, dtype=torch.float32) * wl.x_std
-    if wl.x_dist == "layernorm":
+    if wl.x_dist == "layernorm" and wl.N > 0:  # an empty batch has no rows to normalise
         mu = x.mean(dim=1, keepdim=True)
         var = x.var(dim=1, unbiased=False, keepdim=True)
         x = (x - mu) / torch.sqrt(var + 1e-5)
