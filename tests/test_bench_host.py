@@ -65,3 +65,20 @@ def test_traffic_entry_without_sources_is_ignored(tmp_path, monkeypatch):
     root = _root(tmp_path, monkeypatch)
     (root / "profiles" / "traffic.json").write_text(json.dumps({"gemm1:mixtral": {"bytes_per_launch": 1}}))
     assert bench.traffic_for("gemm1", "mixtral") is None
+
+
+def test_gpus_flag_relaunches_as_ranks_reference_arm():
+    """`--gpus 2` outside torchrun runs the script again as two ranks; the
+    reference arm needs no GPU, and rank 0 alone prints its one line."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "LOCAL_RANK", "WORLD_SIZE")}
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--impl", "reference",
+                          "--steps", "1", "--warmup", "0", "--workload", "tiny_fp32"],
+                         capture_output=True, text=True, timeout=240, env=env, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [json.loads(x) for x in out.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
+    assert lines[0]["cpu_baseline"]["kind"] == "oracle" and lines[0]["value"] > 0
