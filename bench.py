@@ -117,6 +117,23 @@ def weights_bytes(wl) -> int:
     return wl.E * wl.mats * wl.d_model * wl.d_ff * es
 
 
+def gemm1_bytes(wl, experts_used: int) -> int:
+    """Algorithmic DRAM bytes of GEMM1: the first-layer weights of every
+    expert that has rows (W1, and W3 for SwiGLU) read once, x_sorted read,
+    h written."""
+    es = 4 if wl.dtype == "f32" else 2
+    rows = wl.N * wl.k
+    mats1 = 2 if wl.act == "swiglu" else 1
+    return experts_used * mats1 * wl.d_model * wl.d_ff * es + rows * wl.d_model * es + rows * wl.d_ff * es
+
+
+def gemm1_bound(flops: float, nbytes: float, tflops_peak: float, hbm_gbs: float) -> str:
+    """'hbm' when the kernel's arithmetic intensity is below the ridge point
+    of the two peaks (it cannot keep the tensor cores fed from HBM), else
+    'tensor'."""
+    return "hbm" if flops / max(nbytes, 1.0) < tflops_peak * 1e12 / (hbm_gbs * 1e9) else "tensor"
+
+
 def traffic_for(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -556,6 +573,7 @@ def run_native(args, wl):
         local_ms = sum(start[i].elapsed_time(end[i]) for i in range(args.steps))
     gemm1_ms = sum(ev.elapsed_ms()["gemm1"] for ev in stage_ev) / args.steps
     total_ms = max_over_ranks(local_ms, world, dev)
+    experts_used = int((out["counts"] > 0).sum())  # experts whose weights GEMM1 reads
 
     # stage breakdown: every boundary recorded, untimed steps after the run
     n_stage = min(args.steps, 20)
@@ -621,18 +639,28 @@ def run_native(args, wl):
         kern = ("simt_gemm_kernel<GELU>" if fp32 else
                 ("ffn_gemm_pair_kernel" if wl.N * wl.k / wl.E > 192 else "ffn_gemm_single_kernel") +
                 ("<SwiGLU>" if wl.act == "swiglu" else "<GELU>")) + " (GEMM1)"
+        roofline_line = {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"{peak_src} {peak_name} (timed region {total_ms:.0f} ms)",
+                         "frac_of_burst_peak": achieved / burst,
+                         "frac_of_sustained_peak": achieved / sustained,
+                         "traffic": traffic_for("gemm1", wl.name), "flops_per_launch": gemm1_flops}
+        g1_bytes = gemm1_bytes(wl, experts_used)
+        if gemm1_bound(gemm1_flops, g1_bytes, burst, peaks["hbm_gbs"]) == "hbm":
+            # weight streaming (few rows per expert): the kernel is held
+            # against the copy bandwidth, its tensor throughput kept beside
+            gbs = g1_bytes / gemm1_s / 1e9
+            roofline_line.update({"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                  "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
+                                  "bytes_per_launch": g1_bytes, "tensor_tflops": achieved,
+                                  "frac_of_burst_peak": achieved / burst})
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
             "config": dict(describe(wl), l2=("inputs larger than L2 (expert weights %.2f GB)" % (weights_bytes(wl) / 1e9))
                            if big_inputs else "L2 flushed between steps (256 MiB write), per-step events"),
-            "roofline": {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak,
-                         "peak_source": f"{peak_src} {peak_name} (timed region {total_ms:.0f} ms)",
-                         "frac_of_burst_peak": achieved / burst,
-                         "frac_of_sustained_peak": achieved / sustained,
-                         "traffic": traffic_for("gemm1", wl.name), "flops_per_launch": gemm1_flops},
+            "roofline": roofline_line,
             "expert_ffn": {"tflops": ffn_tflops,
                            "frac_of_measured_sustained": ffn_tflops / sustained,
                            "frac_of_measured_burst": ffn_tflops / burst,

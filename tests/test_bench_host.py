@@ -82,3 +82,16 @@ def test_gpus_flag_relaunches_as_ranks_reference_arm():
     assert len(lines) == 1
     assert lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
     assert lines[0]["cpu_baseline"]["kind"] == "oracle" and lines[0]["value"] > 0
+
+
+def test_gemm1_bound_by_arithmetic_intensity():
+    import workloads as W
+    peaks = bench.FALLBACK_PEAKS
+    for name, bound in (("mixtral", "tensor"), ("qwen3_skew", "tensor"), ("gpt2_moe", "tensor"),
+                        ("deepseek_v3", "hbm")):
+        wl = W.WORKLOADS[name]
+        flops = 2 * (2 if wl.act == "swiglu" else 1) * wl.d_model * wl.d_ff * wl.N * wl.k
+        assert bench.gemm1_bound(flops, bench.gemm1_bytes(wl, wl.E), peaks["bf16_tflops"], peaks["hbm_gbs"]) == bound
+    wl = W.WORKLOADS["deepseek_v3"]
+    # weights of the used experts once, x_sorted in, h out
+    assert bench.gemm1_bytes(wl, 256) == 256 * 2 * 7168 * 2048 * 2 + 4096 * 8 * (7168 + 2048) * 2
