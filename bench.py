@@ -162,7 +162,7 @@ def sources_hash(sources):
 
 class ClockSampler:
     """SM clocks and clock-event (throttle) reasons of one GPU, polled through
-    NVML from a background thread every `interval_ms` (default 2 ms, so that
+    NVML from a background thread every `interval_ms` (default 1 ms, so that
     even a timed region of a few tens of milliseconds holds ten or more
     samples); `mark(t0, t1)` keeps the samples of the timed region.  Falls
     back to `nvidia-smi -lms` when NVML is unavailable.  Reads only."""
@@ -173,7 +173,7 @@ class ClockSampler:
     REASONS = (("hw_slowdown", 0x88), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
                ("sw_power_cap", 0x4))
 
-    def __init__(self, cuda_index: int, interval_ms: float = 2.0):
+    def __init__(self, cuda_index: int, interval_ms: float = 1.0):
         self.cuda_index = cuda_index
         self.interval_ms = interval_ms
         self.samples = []      # (time.monotonic(), sm_mhz, reasons bitmask)
