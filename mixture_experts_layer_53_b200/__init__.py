@@ -462,19 +462,32 @@ def moe_forward(cfg: MoeConfig, x: torch.Tensor, W_g: torch.Tensor, W1: torch.Te
 class HostPipeline:
     """moe_forward over batches that live in pinned host memory.
 
-    Each call of ``step(x_host, y_host)`` uploads one batch, runs the layer and
-    downloads y (and the Switch loss).  Uploads and downloads run on two copy
-    streams of their own, double-buffered, so batch i+1's upload and batch
-    i-1's download overlap batch i's forward on the compute stream.
-    ``finish()`` waits for the last download.  Only torch copies and CUDA
-    events are added around the library call; the layer is ``moe_forward``.
+    Each call of ``step(x_host, y_host, aux_host)`` hands over one batch: its
+    upload, the layer and the download of y (and the Switch loss) run on the
+    device while later calls proceed.  Uploads and downloads use two copy
+    streams of their own and two device buffers of each kind, so one batch's
+    upload and another's download overlap a third batch's forward.
+
+    ``graphs=True`` (the default) software-pipelines the calls: call i
+    enqueues the upload of batch i, the forward of batch i-1 and the download
+    of batch i-2 as the three branches of one CUDA graph, replayed with a
+    single launch (one graph per parity and set of host buffers, captured on
+    first use; the first two calls run eagerly).  Batch i's outputs are on the
+    host once call i+2 has completed on the device, or after ``flush()``.
+    ``graphs=False`` enqueues each batch's upload, forward and download in its
+    own call.  ``flush()`` enqueues the work still owed (without waiting);
+    ``finish()`` flushes and waits for the last download.  A host buffer must
+    stay untouched until its copy has run.  Only torch copies, CUDA events
+    and graph launches are added around the library call; the layer is
+    ``moe_forward``.
     """
 
     def __init__(self, cfg: MoeConfig, weights: Dict[str, Optional[torch.Tensor]], gamma: float = 0.0,
-                 device=None):
+                 device=None, graphs: bool = True):
         self.cfg = cfg
         self.w = weights
         self.gamma = gamma
+        self.graphs = graphs
         dev = torch.device(device or "cuda")
         self.compute = torch.cuda.current_stream(dev)
         self.upload = torch.cuda.Stream(dev)
@@ -486,30 +499,103 @@ class HostPipeline:
         self.computed = [torch.cuda.Event() for _ in range(2)]
         self.downloaded = [torch.cuda.Event() for _ in range(2)]
         self.i = 0
+        self._owed = []      # (batch, y_host, aux_host) uploaded, not yet downloaded, oldest first
+        self._cache = {}     # graph key -> CUDAGraph
 
-    def step(self, x_host: torch.Tensor, y_host: torch.Tensor, aux_host: Optional[torch.Tensor] = None):
-        b = self.i & 1
-        with torch.cuda.stream(self.upload):
-            # x buffer b was last read by the forward of step i-2
-            self.upload.wait_event(self.computed[b])
-            self.x[b].copy_(x_host, non_blocking=True)
-            self.uploaded[b].record(self.upload)
-        self.compute.wait_event(self.uploaded[b])
-        self.compute.wait_event(self.downloaded[b])  # outputs of step i-2 are on the host
+    def _forward(self, b: int, stream):
         w = self.w
         moe_forward(self.cfg, self.x[b], w["W_g"], w["W1"], w["W2"], W3=w.get("W3"), b1=w.get("b1"),
                     b2=w.get("b2"), b_e=w.get("b_e"), gamma=self.gamma, ws=self.ws, out=self.out[b],
-                    stream=self.compute, shared=w.get("shared"))
+                    stream=stream, shared=w.get("shared"))
+
+    def _upload(self, b: int, x_host: torch.Tensor):
+        with torch.cuda.stream(self.upload):
+            self.upload.wait_event(self.computed[b])  # x buffer b was last read by the forward two batches ago
+            self.x[b].copy_(x_host, non_blocking=True)
+            self.uploaded[b].record(self.upload)
+
+    def _run(self, b: int):
+        self.compute.wait_event(self.uploaded[b])
+        self.compute.wait_event(self.downloaded[b])  # outputs two batches ago are on the host
+        self._forward(b, self.compute)
         self.computed[b].record(self.compute)
+
+    def _download(self, b: int, y_host: torch.Tensor, aux_host: Optional[torch.Tensor]):
         with torch.cuda.stream(self.download):
             self.download.wait_event(self.computed[b])
             y_host.copy_(self.out[b]["y"], non_blocking=True)
             if aux_host is not None:
                 aux_host.copy_(self.out[b]["aux"], non_blocking=True)
             self.downloaded[b].record(self.download)
+
+    def _graph(self, p: int, x_host, y_host, aux_host):
+        """Upload into x[p], forward of x[1-p], download of out[p], as one graph."""
+        key = (p, x_host.data_ptr(), y_host.data_ptr(), aux_host.data_ptr() if aux_host is not None else 0)
+        g = self._cache.get(key)
+        if g is None:
+            torch.cuda.synchronize()  # no earlier work pending on the streams the capture joins
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="thread_local"):
+                cap = torch.cuda.current_stream()
+                fork = torch.cuda.Event()
+                fork.record(cap)
+                self.upload.wait_event(fork)
+                with torch.cuda.stream(self.upload):
+                    self.x[p].copy_(x_host, non_blocking=True)
+                self.download.wait_event(fork)
+                with torch.cuda.stream(self.download):
+                    y_host.copy_(self.out[p]["y"], non_blocking=True)
+                    if aux_host is not None:
+                        aux_host.copy_(self.out[p]["aux"], non_blocking=True)
+                self._forward(1 - p, cap)
+                cap.wait_stream(self.upload)
+                cap.wait_stream(self.download)
+            self._cache[key] = g
+        return g
+
+    def step(self, x_host: torch.Tensor, y_host: torch.Tensor, aux_host: Optional[torch.Tensor] = None):
+        b = self.i & 1
+        if not self.graphs:
+            self._upload(b, x_host)
+            self._run(b)
+            self._download(b, y_host, aux_host)
+            self.i += 1
+            return
+        self._owed.append((b, y_host, aux_host))
+        if self.i < 2:  # filling the pipeline: upload (and the first forward) eagerly
+            self._upload(b, x_host)
+            if self.i == 1:
+                self._run(0)
+            self.i += 1
+            return
+        # steady state: batch i up, batch i-1 through the layer, batch i-2 down
+        _, y_old, aux_old = self._owed.pop(0)
+        self.compute.wait_stream(self.upload)
+        self.compute.wait_stream(self.download)
+        self._graph(b, x_host, y_old, aux_old).replay()
+        self.computed[1 - b].record(self.compute)
         self.i += 1
 
+    def flush(self):
+        """Enqueues the forward and the downloads still owed (does not wait)."""
+        if not self.graphs or not self._owed:
+            return
+        if self.i >= 2:
+            # the graph launches ran on the compute stream: later copies follow them
+            self.upload.wait_stream(self.compute)
+            self.download.wait_stream(self.compute)
+            self.uploaded[(self.i - 1) & 1].record(self.compute)
+            self.downloaded[0].record(self.compute)
+            self.downloaded[1].record(self.compute)
+        last = self._owed[-1][0]
+        self._run(last)  # the last uploaded batch
+        for b, y_host, aux_host in self._owed:
+            self._download(b, y_host, aux_host)
+        self._owed = []
+        self.i = 0  # the next call starts a new pipeline
+
     def finish(self):
+        self.flush()
         for e in self.downloaded:
             e.synchronize()
 

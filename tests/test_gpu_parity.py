@@ -310,9 +310,11 @@ def test_collapsed_routing_single_expert_gets_everything():
     check_forward(wl, inp, gpu)
 
 
-def test_host_pipeline_matches_forward():
-    """Batches in pinned host memory through the overlapped copy pipeline give
-    the same y and loss as moe_forward on device tensors, batch by batch."""
+@pytest.mark.parametrize("graphs", [True, False])
+def test_host_pipeline_matches_forward(graphs):
+    """Batches in pinned host memory through the overlapped copy pipeline
+    (graph-pipelined or eager) give the same y and loss as moe_forward on
+    device tensors, batch by batch."""
     wl = SMALL["mixtral_small"]
     inp = W.make_inputs(wl, DEV)
     cfg = config_of(wl)
@@ -320,11 +322,18 @@ def test_host_pipeline_matches_forward():
     xs = [W.make_x(wl.scaled(seed=wl.seed + i)).pin_memory() for i in range(4)]
     ys = [torch.empty((wl.N, wl.d_model), dtype=torch.bfloat16).pin_memory() for _ in range(4)]
     auxs = [torch.empty(1, dtype=torch.float32).pin_memory() for _ in range(4)]
-    pipe = M.HostPipeline(cfg, weights, device=DEV)
-    for i in range(4):
+    pipe = M.HostPipeline(cfg, weights, device=DEV, graphs=graphs)
+    n = 6  # graph-pipelined: two eager calls, then both parities' graphs
+    xs = xs + [W.make_x(wl.scaled(seed=wl.seed + i)).pin_memory() for i in range(4, n)]
+    ys = ys + [torch.empty((wl.N, wl.d_model), dtype=torch.bfloat16).pin_memory() for _ in range(4, n)]
+    auxs = auxs + [torch.empty(1, dtype=torch.float32).pin_memory() for _ in range(4, n)]
+    for i in range(n):
         pipe.step(xs[i], ys[i], auxs[i])
     pipe.finish()
-    for i in range(4):
+    for i in range(3):  # a second pipeline on the same object, fewer batches than its depth
+        pipe.step(xs[i], ys[i], auxs[i])
+    pipe.finish()
+    for i in range(n):
         ref = M.moe_forward(cfg, xs[i].to(DEV), inp["W_g"], inp["W1"], inp["W2"], W3=inp["W3"])
         torch.cuda.synchronize()
         assert torch.equal(ys[i], ref["y"].cpu()), i
