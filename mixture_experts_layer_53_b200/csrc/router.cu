@@ -170,6 +170,17 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a)
 // logits; the gates' sum is formed round by round in choice order.  The
 // chunk's histogram uses integer shared-memory atomics (order-free); its
 // sum of p is taken per expert in token order.
+//
+// Before that, a shorter exact path is tried.  Let T be the k-th largest of
+// the G lanes' largest keys.  Those k lanes hold k keys at or above T, so
+// each of the token's k choices is at or above T: the choices are the k
+// largest of the keys >= T, about ten of them for random logits at E = 128
+// or 256.  When they fit one per lane (at most G of them, and k <= G), they
+// are gathered through shared memory and one bitonic sort across the group
+// ranks them; lane r then holds the r-th choice.  A warp in which any token
+// has more candidates (ties, or k > G) takes the rounds above.  Both paths
+// choose the same experts in the same order and form the gates' sum in the
+// same order, so their outputs are bitwise equal.
 template <int N> __device__ __forceinline__ void bitonic_sort_desc(uint64_t (&v)[N])
 {
 #pragma unroll
@@ -188,6 +199,21 @@ template <int N> __device__ __forceinline__ void bitonic_sort_desc(uint64_t (&v)
             }
 }
 
+// Sorts one 64-bit key per lane descending across each group of G lanes
+// (lane q of the group ends with the q-th largest), q = lane % G.
+template <int G> __device__ __forceinline__ uint64_t group_sort_desc(uint64_t v, int q)
+{
+#pragma unroll
+    for (int blk = 2; blk <= G; blk <<= 1)
+#pragma unroll
+        for (int j = blk >> 1; j > 0; j >>= 1) {
+            const uint64_t o = __shfl_xor_sync(0xffffffffu, v, j);
+            const bool keep_max = ((q & blk) == 0) == ((q & j) == 0);
+            v = keep_max ? (o > v ? o : v) : (o < v ? o : v);
+        }
+    return v;
+}
+
 template <int EJ, int G>
 __global__ void __launch_bounds__(kRT * G) select_kernel(SelectKernelArgs a)
 {
@@ -198,6 +224,8 @@ __global__ void __launch_bounds__(kRT * G) select_kernel(SelectKernelArgs a)
     float *pt = smem;                                          // [32][E+1] z, then p
     int *hist_s = reinterpret_cast<int *>(pt + kRT * ZS);      // [E]
     float *zl = reinterpret_cast<float *>(hist_s + kMaxE);     // [32] lse^2
+    uint64_t *cand = reinterpret_cast<uint64_t *>(               // [32][G] candidate keys (8-byte aligned)
+        reinterpret_cast<uintptr_t>(zl + kRT + 1) & ~static_cast<uintptr_t>(7));
     const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kRT;
     const int ntok = static_cast<int>(min64(kRT, a.N - tok0));
     const int lane = threadIdx.x & 31, q = lane & (G - 1);
@@ -259,14 +287,50 @@ __global__ void __launch_bounds__(kRT * G) select_kernel(SelectKernelArgs a)
             zrow[e] = z[j];
         }
     }
-    bitonic_sort_desc(key);
-    __syncwarp();
     auto raw_gate = [&](float zr) {
         return a.router == kSigmoid ? 1.0f / (1.0f + expf(-zr)) : expf(zr - zmax);
     };
-    // k rounds: the group's largest remaining key
     int my_id = -1, my_id2 = -1;  // lane q < k (and q + G < k): the q-th (q + G-th) choice
     float my_z = 0.f, my_z2 = 0.f, gs = 0.f;
+    // the candidates: keys at or above T, the k-th largest lane maximum
+    uint64_t lane_max = 0ull;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) lane_max = key[j] > lane_max ? key[j] : lane_max;
+    const uint64_t T = __shfl_sync(0xffffffffu, group_sort_desc<G>(lane_max, q), k <= G ? k - 1 : 0, G);
+    int cnt = 0;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) cnt += (key[j] != 0ull && key[j] >= T) ? 1 : 0;
+    int before = cnt;  // inclusive prefix of cnt over the group's lanes
+#pragma unroll
+    for (int o = 1; o < G; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, before, o, G);
+        if (q >= o) before += u;
+    }
+    const int C = __shfl_sync(0xffffffffu, before, G - 1, G);
+    before -= cnt;
+    const bool fits = k <= G && T != 0ull && C <= G;
+    __syncwarp();  // the group's logits are in shared memory
+    if (__all_sync(0xffffffffu, fits)) {
+        // this lane's candidates to slots before .. before + cnt - 1 of its
+        // token's G slots (C <= G of them in all)
+        uint64_t *slots = cand + t * G;
+#pragma unroll
+        for (int j = 0; j < EJ; ++j)
+            if (key[j] != 0ull && key[j] >= T) slots[before++] = key[j];
+        __syncwarp();
+        const uint64_t mine = group_sort_desc<G>(q < C ? slots[q] : 0ull, q);
+        // lane r < k: the r-th choice (every one of them a real key: C >= k)
+        const int e = 0xFFFF - static_cast<int>(mine & 0xFFFFu);
+        const float ez = q < k ? zrow[e] : 0.f;
+        const float g = raw_gate(ez);
+        for (int r = 0; r < k; ++r) gs += __shfl_sync(0xffffffffu, g, r, G);
+        if (q < k) {
+            my_id = e;
+            my_z = ez;
+        }
+    } else {
+    bitonic_sort_desc(key);
+    // k rounds: the group's largest remaining key
 #pragma unroll 1
     for (int r = 0; r < k; ++r) {
         uint64_t best = key[0];
@@ -291,6 +355,7 @@ __global__ void __launch_bounds__(kRT * G) select_kernel(SelectKernelArgs a)
             my_id2 = e;
             my_z2 = ez;
         }
+    }
     }
     // gates: raw gate of each choice over their sum (in choice order), then
     // this lane's one or two outputs
@@ -367,13 +432,17 @@ cudaError_t launch_select(const SelectKernelArgs &a, cudaStream_t s)
     // logits rows of ld >= E columns, a multiple of 4 (columns E .. ld-1 are
     // read as whole float4s and ignored)
     if (a.ld % 4 != 0 || a.ld < a.E || a.E > kMaxE) return cudaErrorInvalidValue;
-    const size_t smem = sizeof(float) * (kRT * (a.E + 1) + kRT) + sizeof(int) * kMaxE;
+    // logits / p rows, histogram, z-loss terms, then (8-byte aligned, at
+    // most 4 bytes of padding) G candidate keys per token
+    auto smem = [&](int G) {
+        return sizeof(float) * (kRT * (a.E + 1) + kRT) + sizeof(int) * kMaxE + 8 + sizeof(uint64_t) * kRT * G;
+    };
     // experts per lane x lanes per token: 8 x 8, 8 x 16 or 8 x 32 (eight keys
     // per lane keep the registers low enough for 32 warps per SM)
     const dim3 g(static_cast<unsigned>(grid));
-    if (a.E <= 64) return launch_k(select_kernel<8, 8>, g, dim3(kRT * 8), smem, s, a);
-    if (a.E <= 128) return launch_k(select_kernel<8, 16>, g, dim3(kRT * 16), smem, s, a);
-    return launch_k(select_kernel<8, 32>, g, dim3(kRT * 32), smem, s, a);
+    if (a.E <= 64) return launch_k(select_kernel<8, 8>, g, dim3(kRT * 8), smem(8), s, a);
+    if (a.E <= 128) return launch_k(select_kernel<8, 16>, g, dim3(kRT * 16), smem(16), s, a);
+    return launch_k(select_kernel<8, 32>, g, dim3(kRT * 32), smem(32), s, a);
 }
 
 cudaError_t launch_router(int dtype, const RouterArgs &a, cudaStream_t s)

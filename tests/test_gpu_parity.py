@@ -269,6 +269,44 @@ def test_aux_loss_entry_point_and_bias_rule():
     assert int(status[0]) == 0
 
 
+@pytest.mark.parametrize("E,k,router,group", [(128, 8, "softmax_topk", 1), (128, 8, "softmax_topk", 2),
+                                                (128, 8, "topk_softmax", 16), (256, 8, "sigmoid", 2),
+                                                (256, 8, "sigmoid", 32), (64, 4, "softmax_topk", 2),
+                                                (64, 8, "softmax_topk", 1)])
+def test_route_exact_ties_large_E(E, k, router, group):
+    """Exact ties through the E > 32 selection, both of its paths.
+
+    Experts come in groups of `group` with identical W_g rows, a constant c_g
+    per group (distinct, exact in bf16), and x is positive: tied experts get
+    bitwise-equal logits, groups are far apart, and the course module's rule
+    (ties to the lowest id, sec. 2.1) fixes the choice: groups by c_g
+    descending, ids ascending inside a group, the same for every token.
+    Groups of 1-2 leave about ten candidates per token (the short path);
+    groups of 16-32 leave more than a lane group holds (the k-round path).
+    """
+    N, d = 96, 64
+    wl = W.Workload("ties", N=N, d_model=d, d_ff=64, E=E, k=k, act="swiglu", router=router, dtype="bf16",
+                    seed=31 + E + group)
+    inp = W.make_inputs(wl, DEV)
+    g = torch.Generator().manual_seed(7 + group)
+    ngroups = E // group
+    c = (torch.randperm(ngroups, generator=g).to(torch.float32) + 1.0) / (2.0 * ngroups)  # 1/2n .. 1/2, exact
+    inp["W_g"] = c.repeat_interleave(group)[:, None].expand(E, d).contiguous().to(DEV, torch.bfloat16)
+    inp["x"] = (inp["x"].float().abs() * 0.05 + 0.01).to(torch.bfloat16)  # z = c_g * sum(x) in (0, 3)
+    if inp["b_e"] is not None:
+        inp["b_e"] = torch.zeros_like(inp["b_e"])
+    cg = c.repeat_interleave(group).numpy()
+    want = np.array(sorted(range(E), key=lambda e: (-cg[e], e))[:k], dtype=np.int32)
+    cfg = config_of(wl)
+    ids, w, _ = M.moe_route(cfg, inp["x"], inp["W_g"], b_e=inp["b_e"], want_probs=True)
+    torch.cuda.synchronize()
+    ids = ids.cpu().numpy()
+    assert np.array_equal(ids, np.tile(want, (N, 1)))
+    r = oracle_routing(wl, inp)
+    assert np.array_equal(r["ids"], ids)
+    assert np.max(np.abs(w.cpu().numpy() - r["w"])) <= 2e-5
+
+
 def test_balanced_router_gives_loss_k():
     """Circulant router: every expert in exactly k top-k sets, so L = k."""
     E, k = 8, 2
