@@ -470,9 +470,10 @@ class HostPipeline:
 
     ``graphs=True`` (the default) software-pipelines the calls: call i
     enqueues the upload of batch i, the forward of batch i-1 and the download
-    of batch i-2 as the three branches of one CUDA graph, replayed with a
-    single launch (one graph per parity and set of host buffers, captured on
-    first use; the first two calls run eagerly).  Batch i's outputs are on the
+    of batch i-2 as three branches of one piece of work (the first two calls
+    fill the pipeline).  A parity and set of host buffers met a second time
+    gets a CUDA graph of that work, replayed with one launch (at most
+    ``MAX_GRAPHS`` graphs); other calls enqueue the same work directly.  Batch i's outputs are on the
     host once call i+2 has completed on the device, or after ``flush()``.
     ``graphs=False`` enqueues each batch's upload, forward and download in its
     own call.  ``flush()`` enqueues the work still owed (without waiting);
@@ -501,6 +502,7 @@ class HostPipeline:
         self.i = 0
         self._owed = []      # (batch, y_host, aux_host) uploaded, not yet downloaded, oldest first
         self._cache = {}     # graph key -> CUDAGraph
+        self._seen = set()   # graph keys met once
 
     def _forward(self, b: int, stream):
         w = self.w
@@ -528,30 +530,48 @@ class HostPipeline:
                 aux_host.copy_(self.out[b]["aux"], non_blocking=True)
             self.downloaded[b].record(self.download)
 
-    def _graph(self, p: int, x_host, y_host, aux_host):
-        """Upload into x[p], forward of x[1-p], download of out[p], as one graph."""
+    def _steady(self, p: int, x_host, y_host, aux_host, cap):
+        """Upload into x[p], forward of x[1-p], download of out[p]: two
+        branches forked from stream `cap`, which runs the forward and joins
+        them (captured into a graph, or enqueued as it stands)."""
+        fork = torch.cuda.Event()
+        fork.record(cap)
+        self.upload.wait_event(fork)
+        with torch.cuda.stream(self.upload):
+            self.x[p].copy_(x_host, non_blocking=True)
+        self.download.wait_event(fork)
+        with torch.cuda.stream(self.download):
+            y_host.copy_(self.out[p]["y"], non_blocking=True)
+            if aux_host is not None:
+                aux_host.copy_(self.out[p]["aux"], non_blocking=True)
+        self._forward(1 - p, cap)
+        cap.wait_stream(self.upload)
+        cap.wait_stream(self.download)
+
+    # graphs kept at most, and buffer sets remembered while waiting for a second use
+    MAX_GRAPHS = 8
+    MAX_SEEN = 256
+
+    def _steady_step(self, p: int, x_host, y_host, aux_host):
+        """The steady-state call: a graph for a parity and set of host buffers
+        met before (captured on its second use, up to MAX_GRAPHS of them), so
+        that buffers a caller reuses cost one launch; otherwise the same work
+        enqueued directly, so that fresh buffers on every call cost no capture."""
         key = (p, x_host.data_ptr(), y_host.data_ptr(), aux_host.data_ptr() if aux_host is not None else 0)
         g = self._cache.get(key)
-        if g is None:
+        if g is None and key in self._seen and len(self._cache) < self.MAX_GRAPHS:
             torch.cuda.synchronize()  # no earlier work pending on the streams the capture joins
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, capture_error_mode="thread_local"):
-                cap = torch.cuda.current_stream()
-                fork = torch.cuda.Event()
-                fork.record(cap)
-                self.upload.wait_event(fork)
-                with torch.cuda.stream(self.upload):
-                    self.x[p].copy_(x_host, non_blocking=True)
-                self.download.wait_event(fork)
-                with torch.cuda.stream(self.download):
-                    y_host.copy_(self.out[p]["y"], non_blocking=True)
-                    if aux_host is not None:
-                        aux_host.copy_(self.out[p]["aux"], non_blocking=True)
-                self._forward(1 - p, cap)
-                cap.wait_stream(self.upload)
-                cap.wait_stream(self.download)
+                self._steady(p, x_host, y_host, aux_host, torch.cuda.current_stream())
             self._cache[key] = g
-        return g
+        if g is not None:
+            g.replay()
+            return
+        if len(self._seen) >= self.MAX_SEEN:
+            self._seen.clear()
+        self._seen.add(key)
+        self._steady(p, x_host, y_host, aux_host, self.compute)
 
     def step(self, x_host: torch.Tensor, y_host: torch.Tensor, aux_host: Optional[torch.Tensor] = None):
         b = self.i & 1
@@ -572,7 +592,7 @@ class HostPipeline:
         _, y_old, aux_old = self._owed.pop(0)
         self.compute.wait_stream(self.upload)
         self.compute.wait_stream(self.download)
-        self._graph(b, x_host, y_old, aux_old).replay()
+        self._steady_step(b, x_host, y_old, aux_old)
         self.computed[1 - b].record(self.compute)
         self.i += 1
 

@@ -361,7 +361,7 @@ def test_host_pipeline_matches_forward(graphs):
     ys = [torch.empty((wl.N, wl.d_model), dtype=torch.bfloat16).pin_memory() for _ in range(4)]
     auxs = [torch.empty(1, dtype=torch.float32).pin_memory() for _ in range(4)]
     pipe = M.HostPipeline(cfg, weights, device=DEV, graphs=graphs)
-    n = 6  # graph-pipelined: two eager calls, then both parities' graphs
+    n = 6  # fresh buffers on every call: the pipeline's work is enqueued directly
     xs = xs + [W.make_x(wl.scaled(seed=wl.seed + i)).pin_memory() for i in range(4, n)]
     ys = ys + [torch.empty((wl.N, wl.d_model), dtype=torch.bfloat16).pin_memory() for _ in range(4, n)]
     auxs = auxs + [torch.empty(1, dtype=torch.float32).pin_memory() for _ in range(4, n)]
@@ -376,3 +376,19 @@ def test_host_pipeline_matches_forward(graphs):
         torch.cuda.synchronize()
         assert torch.equal(ys[i], ref["y"].cpu()), i
         assert torch.equal(auxs[i], ref["aux"].cpu()), i
+    # two buffer sets used in turn: each parity's work is enqueued directly on
+    # its first use, captured on its second and replayed after that
+    for j in (4, 5):  # no copy is in flight after finish()
+        ys[j].zero_()
+        auxs[j].zero_()
+    for i in range(8):
+        j = 4 + (i & 1)
+        pipe.step(xs[j], ys[j], auxs[j])
+    pipe.finish()
+    if graphs:
+        assert len(pipe._cache) >= 2
+    for j in (4, 5):
+        ref = M.moe_forward(cfg, xs[j].to(DEV), inp["W_g"], inp["W1"], inp["W2"], W3=inp["W3"])
+        torch.cuda.synchronize()
+        assert torch.equal(ys[j], ref["y"].cpu()), j
+        assert torch.equal(auxs[j], ref["aux"].cpu()), j
