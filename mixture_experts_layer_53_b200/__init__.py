@@ -459,6 +459,35 @@ def moe_forward(cfg: MoeConfig, x: torch.Tensor, W_g: torch.Tensor, W1: torch.Te
     return out
 
 
+class GraphPolicy:
+    """Which steady-state calls of HostPipeline replay a CUDA graph.
+
+    ``decide(key)`` returns "replay" for a key that has a graph, "capture"
+    for a key met once before while fewer than ``max_graphs`` graphs exist
+    (the caller then stores it with ``stored(key, graph)``), and "direct"
+    otherwise; a "direct" key is remembered for its next call, at most
+    ``max_seen`` of them (the memory is cleared when full)."""
+
+    def __init__(self, max_graphs: int = 8, max_seen: int = 256):
+        self.max_graphs = max_graphs
+        self.max_seen = max_seen
+        self.graphs = {}
+        self.seen = set()
+
+    def decide(self, key) -> str:
+        if key in self.graphs:
+            return "replay"
+        if key in self.seen and len(self.graphs) < self.max_graphs:
+            return "capture"
+        if len(self.seen) >= self.max_seen:
+            self.seen.clear()
+        self.seen.add(key)
+        return "direct"
+
+    def stored(self, key, graph) -> None:
+        self.graphs[key] = graph
+
+
 class HostPipeline:
     """moe_forward over batches that live in pinned host memory.
 
@@ -473,7 +502,8 @@ class HostPipeline:
     of batch i-2 as three branches of one piece of work (the first two calls
     fill the pipeline).  A parity and set of host buffers met a second time
     gets a CUDA graph of that work, replayed with one launch (at most
-    ``MAX_GRAPHS`` graphs); other calls enqueue the same work directly.  Batch i's outputs are on the
+    ``GraphPolicy.max_graphs`` graphs); other calls enqueue the same work
+    directly.  Batch i's outputs are on the
     host once call i+2 has completed on the device, or after ``flush()``.
     ``graphs=False`` enqueues each batch's upload, forward and download in its
     own call.  ``flush()`` enqueues the work still owed (without waiting);
@@ -501,8 +531,7 @@ class HostPipeline:
         self.downloaded = [torch.cuda.Event() for _ in range(2)]
         self.i = 0
         self._owed = []      # (batch, y_host, aux_host) uploaded, not yet downloaded, oldest first
-        self._cache = {}     # graph key -> CUDAGraph
-        self._seen = set()   # graph keys met once
+        self.policy = GraphPolicy()  # which calls replay a graph
 
     def _forward(self, b: int, stream):
         w = self.w
@@ -548,29 +577,22 @@ class HostPipeline:
         cap.wait_stream(self.upload)
         cap.wait_stream(self.download)
 
-    # graphs kept at most, and buffer sets remembered while waiting for a second use
-    MAX_GRAPHS = 8
-    MAX_SEEN = 256
-
     def _steady_step(self, p: int, x_host, y_host, aux_host):
         """The steady-state call: a graph for a parity and set of host buffers
-        met before (captured on its second use, up to MAX_GRAPHS of them), so
-        that buffers a caller reuses cost one launch; otherwise the same work
-        enqueued directly, so that fresh buffers on every call cost no capture."""
+        met before (captured on its second use; GraphPolicy), so that buffers
+        a caller reuses cost one launch; otherwise the same work enqueued
+        directly, so that fresh buffers on every call cost no capture."""
         key = (p, x_host.data_ptr(), y_host.data_ptr(), aux_host.data_ptr() if aux_host is not None else 0)
-        g = self._cache.get(key)
-        if g is None and key in self._seen and len(self._cache) < self.MAX_GRAPHS:
+        how = self.policy.decide(key)
+        if how == "capture":
             torch.cuda.synchronize()  # no earlier work pending on the streams the capture joins
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, capture_error_mode="thread_local"):
                 self._steady(p, x_host, y_host, aux_host, torch.cuda.current_stream())
-            self._cache[key] = g
-        if g is not None:
-            g.replay()
+            self.policy.stored(key, g)
+        if how != "direct":
+            self.policy.graphs[key].replay()
             return
-        if len(self._seen) >= self.MAX_SEEN:
-            self._seen.clear()
-        self._seen.add(key)
         self._steady(p, x_host, y_host, aux_host, self.compute)
 
     def step(self, x_host: torch.Tensor, y_host: torch.Tensor, aux_host: Optional[torch.Tensor] = None):
